@@ -1,0 +1,107 @@
+"""Seeded synthetic inputs for the fused LoRA-adapted linear layer.
+
+This module is shared by the oracle (``oracle/``), the tests and ``bench.py``.
+It draws random tensors and encodes them as bfloat16 bit patterns; it holds
+none of the layer's arithmetic (no products, no activation, no gradient).
+
+Workloads (sizes are the Llama-3-8B projection shapes; no weights or datasets
+are used, every tensor is drawn here):
+
+* X  ~ N(0, 1)            tokens x d_in
+* W  ~ N(0, 1/d_in)       d_out x d_in   (frozen base weight)
+* A  ~ U(-1/sqrt(d_in), +1/sqrt(d_in))   r x d_in      (maps d_in -> r)
+* B  ~ N(0, 0.02^2)       d_out x r                    (maps r -> d_out)
+* dY ~ N(0, 1)            tokens x d_out (upstream gradient)
+
+Each tensor has its own stream: numpy's PCG64 seeded with (seed, tensor id).
+Values are drawn in float64, rounded to float32 (round-to-nearest-even) and
+then to bfloat16 (round-to-nearest-even); both sides of every comparison read
+the same bf16 bits, so this double rounding only defines the inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# Tensor ids for the per-tensor random streams.
+_TENSOR_IDS = {
+    "X": 1, "W": 2, "A": 3, "B": 4, "dY": 5,
+    "W_up": 6, "A_up": 7, "B_up": 8,
+}
+
+ACTS = ("identity", "silu", "swiglu")
+
+# The workloads.  ``act`` names the activation applied after the add;
+# ``swiglu`` pairs a gate projection with an up projection.
+CONFIGS = {
+    "tiny": dict(M=64, d_in=256, d_out=256, r=8, alpha=16.0, act="identity"),
+    "q_proj": dict(M=16384, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity"),
+    "v_proj": dict(M=16384, d_in=4096, d_out=1024, r=64, alpha=16.0, act="identity"),
+    "mlp_gate_up": dict(M=8192, d_in=4096, d_out=14336, r=64, alpha=16.0, act="swiglu"),
+    "mlp_down": dict(M=8192, d_in=14336, d_out=4096, r=64, alpha=16.0, act="identity"),
+    "small_m": dict(M=16, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity"),
+    "small_m_ragged": dict(M=1000, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity"),
+}
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Encode float64 values as bfloat16 bit patterns (uint16).
+
+    float64 -> float32 by numpy's RNE cast, then float32 -> bf16 by RNE on the
+    upper 16 bits.  Inputs here are finite and far from overflow.
+    """
+    f = np.ascontiguousarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Decode bf16 bit patterns to float32 (exact)."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _rng(seed: int, name: str) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _TENSOR_IDS[name]])))
+
+
+def draw(name: str, shape, seed: int, d_in: int) -> np.ndarray:
+    """Draw one tensor of the recipe above as bf16 bits."""
+    g = _rng(seed, name)
+    base = name.replace("_up", "")
+    if base in ("X", "dY"):
+        v = g.standard_normal(shape)
+    elif base == "W":
+        v = g.standard_normal(shape) * (1.0 / np.sqrt(d_in))
+    elif base == "A":
+        lim = 1.0 / np.sqrt(d_in)
+        v = g.uniform(-lim, lim, size=shape)
+    elif base == "B":
+        v = g.standard_normal(shape) * 0.02
+    else:  # pragma: no cover
+        raise KeyError(name)
+    return f64_to_bf16_bits(v)
+
+
+def make_inputs(M: int, d_in: int, d_out: int, r: int, act: str = "identity",
+                seed: int = 0, with_grad: bool = True) -> dict:
+    """All inputs of one fwd(+bwd) call as bf16 bit arrays (uint16, row-major)."""
+    out = {
+        "X": draw("X", (M, d_in), seed, d_in),
+        "W": draw("W", (d_out, d_in), seed, d_in),
+        "A": draw("A", (r, d_in), seed, d_in),
+        "B": draw("B", (d_out, r), seed, d_in),
+    }
+    if act == "swiglu":
+        out["W_up"] = draw("W_up", (d_out, d_in), seed, d_in)
+        out["A_up"] = draw("A_up", (r, d_in), seed, d_in)
+        out["B_up"] = draw("B_up", (d_out, r), seed, d_in)
+    if with_grad:
+        out["dY"] = draw("dY", (M, d_out), seed, d_in)
+    return out
+
+
+def config_inputs(name: str, seed: int = 0, with_grad: bool = True, M: int | None = None) -> dict:
+    """Inputs for a named workload; ``M`` overrides the token count."""
+    c = CONFIGS[name]
+    return make_inputs(M if M is not None else c["M"], c["d_in"], c["d_out"], c["r"],
+                       c["act"], seed=seed, with_grad=with_grad)
