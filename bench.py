@@ -1,0 +1,354 @@
+"""Benchmark of the fused LoRA-adapted linear layer, forward + backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config q_proj]
+
+One step = one forward (lora_linear_fwd) and one backward (lora_linear_bwd)
+over one batch of synthetic bf16 inputs of the workload (default: the
+Llama-3-8B q_proj shape, M = 16384 tokens, 4096 -> 4096, r = 8, alpha = 16).
+Algorithmic work per step: 4 M d_in d_out + 6 M r (d_in + d_out) FLOPs.
+
+Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
+the stream the library launches on; the L2 cache is flushed (a 512 MiB write)
+before every timed step, outside the events; a barrier + synchronize brackets
+the timed region and the time is the max over ranks.  N > 1 runs N independent
+replicas (one process per GPU, launched by torch.distributed.run): the layer
+has no exchange step, so there is no collective on the data path.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
+on the host cores instead (a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import seeded_inputs  # noqa: E402
+
+METRIC = "LoRA-linear fwd+bwd TFLOP/s (M=16384, 4096², r=8) & % of B200 roofline"
+UNIT = "TFLOP/s"
+
+
+def step_flops(M, d_in, d_out, r):
+    return 4.0 * M * d_in * d_out + 6.0 * M * r * (d_in + d_out)
+
+
+def fwd_flops(M, d_in, d_out, r):
+    return 2.0 * M * d_in * d_out + 2.0 * M * r * (d_in + d_out)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        busy = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(busy)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def oracle_sample_run(cfg, rows, inp_f64):
+    import oracle
+    g = inp_f64
+    X = g["X"][:rows]
+    dY = g["dY"][:rows]
+    t0 = time.perf_counter()
+    oracle.lora_backward(dY, X, g["W"], g["A"], g["B"], cfg["alpha"] / cfg["r"], cfg["act"],
+                         g.get("W_up"), g.get("A_up"), g.get("B_up"))
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
+    """Time the oracle on growing row samples until ~budget_s of CPU work."""
+    import oracle
+    M, d_in, d_out, r = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"]
+    rows_cap = max_rows or M
+    inp = seeded_inputs.make_inputs(min(M, rows_cap), d_in, d_out, r, cfg["act"], seed=0)
+    g = {k: oracle.bf16_to_f64(v) for k, v in inp.items()}
+    rows = 16
+    spent = 0.0
+    best = None
+    while True:
+        dt = oracle_sample_run(cfg, rows, g)
+        spent += dt
+        best = (rows, dt)
+        if dt > budget_s / 3 or rows >= min(M, rows_cap) or spent > budget_s:
+            break
+        rows = min(rows * 4, min(M, rows_cap))
+    rows, dt = best
+    val = step_flops(rows, d_in, d_out, r) / dt / 1e12
+    return {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle fwd+bwd on the first {rows} of {M} tokens "
+                      f"({d_in}->{d_out}, r={r}); {dt:.2f} s; FLOPs scaled by the same formula"}
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    import oracle
+    inp = seeded_inputs.make_inputs(min(cfg["M"], 4096), cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"], seed=0)
+    g = {k: oracle.bf16_to_f64(v) for k, v in inp.items()}
+    # rows per step: sized so the whole warm-up + timed run stays within a few minutes
+    rows = 64
+    while rows < 4096:
+        dt = oracle_sample_run(cfg, rows, g)
+        if dt * (steps + warm) > 60.0 or dt > 2.0:
+            break
+        rows *= 2
+    for _ in range(warm):
+        oracle_sample_run(cfg, rows, g)
+    tot = 0.0
+    for _ in range(steps):
+        tot += oracle_sample_run(cfg, rows, g)
+    val = step_flops(rows, cfg["d_in"], cfg["d_out"], cfg["r"]) * steps / tot / 1e12
+    sample = (f"fp64 numpy oracle fwd+bwd on {rows} of {cfg['M']} tokens per step "
+              f"({cfg['d_in']}->{cfg['d_out']}, r={cfg['r']})")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": tot / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.config, "M": cfg["M"], "d_in": cfg["d_in"], "d_out": cfg["d_out"],
+                       "r": cfg["r"], "alpha": cfg["alpha"], "act": cfg["act"], "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="q_proj", choices=sorted(seeded_inputs.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = dict(seeded_inputs.CONFIGS[args.config])
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, cfg, world, rank)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import lora_linear_fine_b200 as L
+
+    M, d_in, d_out, r, act = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]
+    s = cfg["alpha"] / r
+    inp = seeded_inputs.make_inputs(M, d_in, d_out, r, act, seed=rank)
+    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in inp.items()}
+    t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    desc = L.make_desc(M, d_in, d_out, r, s, act)
+    np_ = 2 if act == "swiglu" else 1
+    ws = L.Workspace(max(L.lora_linear_workspace_size(desc, 0), L.lora_linear_workspace_size(desc, 1)))
+    Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((np_, M, r), dtype=torch.float32, device="cuda")
+    Z = torch.empty((np_, M, d_out), dtype=torch.float32, device="cuda") if act != "identity" else None
+    dX = torch.empty((M, d_in), dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty((np_, r, d_in), dtype=torch.float32, device="cuda")
+    dB = torch.empty((np_, d_out, r), dtype=torch.float32, device="cuda")
+    p = lambda x: None if x is None else x.data_ptr()  # noqa: E731
+
+    def fwd():
+        st = L.lora_linear_fwd(desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
+                               p(t.get("A_up")), p(t.get("B_up")), p(Y), p(T), p(Z), ws.buf.data_ptr(),
+                               ws.nbytes, sh)
+        assert st == 0, L.status_string(st)
+
+    def bwd():
+        st = L.lora_linear_bwd(desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
+                               p(t.get("A_up")), p(t.get("B_up")), p(T), p(Z), p(dX), p(dA[0]), p(dB[0]),
+                               p(dA[1]) if np_ == 2 else None, p(dB[1]) if np_ == 2 else None,
+                               ws.buf.data_ptr(), ws.nbytes, sh)
+        assert st == 0, L.status_string(st)
+
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+
+    launches0 = L.lora_linear_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        fwd()
+        e1.record(stream)
+        bwd()
+        e2.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    launches = L.lora_linear_launch_count() - launches0
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    tot_ms = sum(step_ms)
+    if dist is not None:
+        tt = torch.tensor([tot_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        tot_ms = float(tt.item())
+    F = step_flops(M, d_in, d_out, r)
+    value = F * args.steps * world / (tot_ms * 1e-3) / 1e12
+
+    # e2e: the same step through the C ABI from pinned HOST buffers, copies included
+    out_host = {"Y": torch.empty_like(Y, device="cpu").pin_memory(),
+                "dX": torch.empty_like(dX, device="cpu").pin_memory(),
+                "dA": torch.empty_like(dA, device="cpu").pin_memory(),
+                "dB": torch.empty_like(dB, device="cpu").pin_memory()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ee0.record(stream)
+    for _ in range(args.e2e_steps):
+        for k, v in host.items():
+            t[k].copy_(v, non_blocking=True)
+        fwd()
+        bwd()
+        out_host["Y"].copy_(Y, non_blocking=True)
+        out_host["dX"].copy_(dX, non_blocking=True)
+        out_host["dA"].copy_(dA, non_blocking=True)
+        out_host["dB"].copy_(dB, non_blocking=True)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ee0.elapsed_time(ee1)
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e = F * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    peaks = read_peaks()
+    # dominant kernel: the forward GEMM (one lora_gemm_kernel launch plus a B^T
+    # copy of r x d_out elements inside the same events)
+    fwd_avg_s = statistics.mean(fwd_ms) * 1e-3
+    ach = fwd_flops(M, d_in, d_out, r) / fwd_avg_s / 1e12
+    roof = {"kernel": "lora_gemm_kernel (forward)", "bound": "tensor", "achieved": round(ach, 2),
+            "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+            "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
+            "peak_kind": f"bf16 sustained, {peaks['source']}", "traffic": None,
+            "step_frac": round(value / world / peaks["bf16_tflops_sustained"], 4)}
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(tot_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.config, "M": M, "d_in": d_in, "d_out": d_out, "r": r,
+                       "alpha": cfg["alpha"], "act": act, "parallelism": f"replicas x{world}",
+                       "l2": "flushed before each timed step (512 MiB write)"},
+            "roofline": roof, "gpu_launches": int(launches),
+            "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h)},
+            "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * lora_linear.h — C ABI of the B200 (sm_100a) fused LoRA-adapted linear layer.
+ *
+ * The operation (forward):
+ *     T = X A^T                       rank-r intermediate, M x r
+ *     Z = X W^T + s T B^T             M x d_out
+ *     Y = act(Z)
+ * follows "Liger-Kernel内核级优化：GPU利用率飙升至90%以上", section
+ * "为什么传统微调会“卡脖子”？" (y = Wx + B(Ax) and its four-call PyTorch form
+ * ax = linear(x, A); bax = linear(ax, B); wx = linear(x, W); y = wx + bax),
+ * with the LoRA branch scaled by s = alpha / r, and section
+ * "内核融合：把“碎片化”变成“流水线”" (activation fused after the add: SiLU).
+ * SwiGLU pairs a gate and an up projection, each a LoRA linear with its own
+ * W, A, B: Y = SiLU(Z_gate) * Z_up ("Swift-All一文详解：如何用Liger-Kernel提升
+ * 训练效率", 2.2 (2) "SwiGLU 激活函数融合").
+ *
+ * The backward is the chain rule of that forward (the pages say only that it
+ * is fused, with recompute: "系统架构与工作流程"):
+ *     dZ = dY * act'(Z)               (identity: dZ = dY)
+ *     U  = dZ B                       M x r
+ *     dX = dZ W + s U A               M x d_in
+ *     dA = s U^T X                    r x d_in
+ *     dB = s dZ^T T                   d_out x r
+ * W is frozen: there is no dW.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers marked "device" must point to memory of the current CUDA device;
+ *   all of them are caller-owned.  The library allocates nothing and keeps no
+ *   state between calls other than a per-device cache of the SM count.
+ * - Matrices are dense, row-major, with no padding between rows.
+ *   bf16 tensors are IEEE bfloat16 bit patterns (2 bytes per element).
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and never synchronises, except
+ *   lora_linear_device_status which reads the status word back.
+ * - Alignment: every tensor pointer is 16-byte aligned; d_in % 8 == 0,
+ *   d_out % 8 == 0; r % 8 == 0 with 0 <= r <= 64.  Violations return
+ *   LORA_ERR_ALIGNMENT (pointers, strides) or LORA_ERR_UNSUPPORTED (r) before
+ *   anything is launched.
+ * - r == 0 is a plain linear layer: A, B (and the _up twins) may be NULL and
+ *   T_save is ignored.
+ * - M may be 0 (nothing is launched; dA/dB are zero-filled in the backward).
+ * - Outputs are overwritten, never accumulated into.
+ * - Results: Y and dX are bf16 (round to nearest even of fp32 accumulators);
+ *   T_save, Z_save, dA, dB are fp32.
+ * - The device must be sm_100 (B200).  Anything else returns LORA_ERR_ARCH.
+ *   There is no CPU or fallback path.
+ * - The workspace holds a 32-bit device status word at offset 0.  Kernels OR
+ *   error bits into it (a bounded wait that gave up, a failed device-side
+ *   check); they never clear it.  Zero it once with lora_linear_workspace_init
+ *   before the first call; read it with lora_linear_device_status.
+ */
+#ifndef LORA_LINEAR_H
+#define LORA_LINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Activation applied after the add (see the header comment). */
+typedef enum lora_act_t {
+    LORA_ACT_IDENTITY = 0,
+    LORA_ACT_SILU = 1,
+    LORA_ACT_SWIGLU = 2
+} lora_act_t;
+
+typedef enum lora_status_t {
+    LORA_OK = 0,
+    LORA_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, bad act */
+    LORA_ERR_ALIGNMENT = 2,     /* pointer not 16-byte aligned, d_in/d_out not multiples of 8 */
+    LORA_ERR_UNSUPPORTED = 3,   /* r outside {0, 8, 16, ..., 64} or r not a multiple of 8 */
+    LORA_ERR_ARCH = 4,          /* current device is not sm_100 */
+    LORA_ERR_WORKSPACE = 5,     /* workspace NULL or smaller than lora_linear_workspace_size */
+    LORA_ERR_CUDA = 6,          /* a CUDA runtime/driver call or a launch failed */
+    LORA_ERR_DEVICE_STATUS = 7  /* the device status word is non-zero */
+} lora_status_t;
+
+/* Problem description.  M tokens; X is M x d_in; W is d_out x d_in;
+ * A is r x d_in; B is d_out x r; s = alpha / r; act is a lora_act_t. */
+typedef struct lora_linear_desc {
+    int64_t M;
+    int64_t d_in;
+    int64_t d_out;
+    int64_t r;
+    float s;
+    int32_t act;
+} lora_linear_desc;
+
+/* Bytes of device workspace lora_linear_fwd (for_backward == 0) or
+ * lora_linear_bwd (for_backward != 0) needs for `desc`.  Returns 0 for an
+ * invalid desc.  The size is a function of the desc only. */
+size_t lora_linear_workspace_size(const lora_linear_desc* desc, int for_backward);
+
+/* Zero the status word of a workspace (asynchronous, on `stream`). */
+lora_status_t lora_linear_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, copy the workspace status word to *out_status and
+ * return LORA_OK if it is zero, LORA_ERR_DEVICE_STATUS otherwise.  Bits:
+ *   0x1  a bounded wait on an mbarrier gave up (the kernel stopped its work)
+ *   0x2  a device-side argument check failed
+ * Intended for tests and debugging. */
+lora_status_t lora_linear_device_status(const void* workspace, void* stream, uint32_t* out_status);
+
+/* Forward.  Device pointers:
+ *   X [M x d_in] bf16, W [d_out x d_in] bf16, A [r x d_in] bf16, B [d_out x r] bf16.
+ *   W_up, A_up, B_up: the up projection's weights for LORA_ACT_SWIGLU, else NULL.
+ *   Y [M x d_out] bf16 (output).
+ *   T_save: NULL, or fp32 output [M x r] (SwiGLU: gate's [M x r] then up's [M x r])
+ *           holding T = X A^T for the backward.
+ *   Z_save: NULL, or fp32 output [M x d_out] (SwiGLU: Z_gate then Z_up, each
+ *           [M x d_out]) holding the pre-activation; ignored for identity.
+ *   workspace: device, >= lora_linear_workspace_size(desc, 0) bytes. */
+lora_status_t lora_linear_fwd(const lora_linear_desc* desc,
+                              const void* X, const void* W, const void* A, const void* B,
+                              const void* W_up, const void* A_up, const void* B_up,
+                              void* Y, float* T_save, float* Z_save,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward.  Device pointers:
+ *   dY [M x d_out] bf16; X, W, A, B (and the _up twins for SwiGLU) as in the forward.
+ *   T_save: the forward's T_save, or NULL to recompute T = X A^T.
+ *   Z_save: the forward's Z_save (required when act != identity), else NULL.
+ *   dX [M x d_in] bf16 (output).
+ *   dA [r x d_in] fp32, dB [d_out x r] fp32 (outputs; NULL when r == 0).
+ *   dA_up, dB_up: the up projection's adapter gradients for SwiGLU, else NULL.
+ *   workspace: device, >= lora_linear_workspace_size(desc, 1) bytes. */
+lora_status_t lora_linear_bwd(const lora_linear_desc* desc,
+                              const void* dY, const void* X, const void* W,
+                              const void* A, const void* B,
+                              const void* W_up, const void* A_up, const void* B_up,
+                              const float* T_save, const float* Z_save,
+                              void* dX, float* dA, float* dB, float* dA_up, float* dB_up,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static string for a status code (never NULL). */
+const char* lora_status_string(lora_status_t status);
+
+/* Library ABI version (incremented on any signature change). */
+int lora_linear_abi_version(void);
+
+/* Number of CUDA kernels this library has launched in the calling process
+ * (all devices, all threads).  For accounting in benchmarks and tests. */
+uint64_t lora_linear_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_LINEAR_H */

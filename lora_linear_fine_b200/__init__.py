@@ -1,0 +1,244 @@
+"""Python binding of the B200 fused LoRA-adapted linear layer (C ABI in
+``include/lora_linear.h``).
+
+The functions named like the C entry points (``lora_linear_fwd`` ...) take raw
+device pointers (ints) and return the C status code; they only marshal
+arguments.  ``forward`` / ``backward`` / ``LoRALinearFunction`` wrap them for
+torch tensors (torch provides device memory and the stream).  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback: if the
+library cannot be loaded, the first call raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblora_linear.so")
+
+ACT_IDENTITY, ACT_SILU, ACT_SWIGLU = 0, 1, 2
+ACT_CODES = {"identity": ACT_IDENTITY, "silu": ACT_SILU, "swiglu": ACT_SWIGLU}
+
+STATUS_NAMES = {
+    0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_ALIGNMENT", 3: "LORA_ERR_UNSUPPORTED",
+    4: "LORA_ERR_ARCH", 5: "LORA_ERR_WORKSPACE", 6: "LORA_ERR_CUDA", 7: "LORA_ERR_DEVICE_STATUS",
+}
+
+# Every symbol include/lora_linear.h declares.
+EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_linear_device_status",
+            "lora_linear_fwd", "lora_linear_bwd", "lora_status_string", "lora_linear_abi_version",
+            "lora_linear_launch_count")
+
+
+class LoraLinearDesc(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("d_in", ctypes.c_int64), ("d_out", ctypes.c_int64),
+                ("r", ctypes.c_int64), ("s", ctypes.c_float), ("act", ctypes.c_int32)]
+
+
+class LoraError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m lora_linear_fine_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, i32, u32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)
+    dp = ctypes.POINTER(LoraLinearDesc)
+    lib.lora_linear_workspace_size.argtypes = [dp, i32]
+    lib.lora_linear_workspace_size.restype = sz
+    lib.lora_linear_workspace_init.argtypes = [vp, sz, vp]
+    lib.lora_linear_workspace_init.restype = i32
+    lib.lora_linear_device_status.argtypes = [vp, vp, u32p]
+    lib.lora_linear_device_status.restype = i32
+    lib.lora_linear_fwd.argtypes = [dp] + [vp] * 10 + [vp, sz, vp]
+    lib.lora_linear_fwd.restype = i32
+    lib.lora_linear_bwd.argtypes = [dp] + [vp] * 15 + [vp, sz, vp]
+    lib.lora_linear_bwd.restype = i32
+    lib.lora_status_string.argtypes = [i32]
+    lib.lora_status_string.restype = ctypes.c_char_p
+    lib.lora_linear_abi_version.argtypes = []
+    lib.lora_linear_abi_version.restype = i32
+    lib.lora_linear_launch_count.argtypes = []
+    lib.lora_linear_launch_count.restype = ctypes.c_uint64
+    return lib
+
+
+class _LazyLib:
+    """Loads the shared library on first use (so the build script can import
+    this package before the library exists); a missing library raises."""
+
+    _h = None
+
+    def __getattr__(self, name):
+        if _LazyLib._h is None:
+            _LazyLib._h = _load()
+        return getattr(_LazyLib._h, name)
+
+
+_lib = _LazyLib()
+
+
+# ---------------------------------------------------------------------------
+# 1:1 wrappers of the C entry points (pointers are ints or None)
+# ---------------------------------------------------------------------------
+def make_desc(M, d_in, d_out, r, s, act) -> LoraLinearDesc:
+    if isinstance(act, str):
+        act = ACT_CODES[act]
+    return LoraLinearDesc(int(M), int(d_in), int(d_out), int(r), float(s), int(act))
+
+
+def lora_linear_workspace_size(desc: LoraLinearDesc, for_backward: int) -> int:
+    return int(_lib.lora_linear_workspace_size(ctypes.byref(desc), int(for_backward)))
+
+
+def lora_linear_workspace_init(workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_workspace_init(workspace, workspace_bytes, stream))
+
+
+def lora_linear_device_status(workspace, stream):
+    out = ctypes.c_uint32(0)
+    st = int(_lib.lora_linear_device_status(workspace, stream, ctypes.byref(out)))
+    return st, int(out.value)
+
+
+def lora_linear_fwd(desc, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, workspace, workspace_bytes,
+                    stream) -> int:
+    return int(_lib.lora_linear_fwd(ctypes.byref(desc), X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save,
+                                    workspace, workspace_bytes, stream))
+
+
+def lora_linear_bwd(desc, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up,
+                    workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_bwd(ctypes.byref(desc), dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save,
+                                    dX, dA, dB, dA_up, dB_up, workspace, workspace_bytes, stream))
+
+
+def status_string(status: int) -> str:
+    s = _lib.lora_status_string(int(status))
+    return s.decode() if s else "?"
+
+
+def lora_linear_abi_version() -> int:
+    return int(_lib.lora_linear_abi_version())
+
+
+def lora_linear_launch_count() -> int:
+    return int(_lib.lora_linear_launch_count())
+
+
+# ---------------------------------------------------------------------------
+# torch-tensor convenience layer (device memory + stream only)
+# ---------------------------------------------------------------------------
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise LoraError(st, what)
+
+
+class Workspace:
+    """A device workspace (torch uint8 tensor) whose status word is zeroed once."""
+
+    def __init__(self, nbytes: int, device=None, stream=None):
+        import torch
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+        _check(lora_linear_workspace_init(self.buf.data_ptr(), self.nbytes, _stream_handle(stream)),
+               "lora_linear_workspace_init")
+
+    def ensure(self, nbytes: int, stream=None):
+        if nbytes > self.nbytes:
+            self.__init__(nbytes, self.buf.device, stream)
+        return self
+
+    def status(self, stream=None):
+        st, word = lora_linear_device_status(self.buf.data_ptr(), _stream_handle(stream))
+        return word
+
+
+def forward(X, W, A, B, s, act="identity", W_up=None, A_up=None, B_up=None, save=True, workspace=None,
+            stream=None):
+    """Y (and the saved T, Z for the backward) for bf16 tensors on the current device."""
+    import torch
+    M, d_in = X.shape
+    d_out = W.shape[0]
+    r = 0 if A is None else A.shape[0]
+    act_code = ACT_CODES[act] if isinstance(act, str) else act
+    desc = make_desc(M, d_in, d_out, r, s, act_code)
+    np_ = 2 if act_code == ACT_SWIGLU else 1
+    Y = torch.empty((M, d_out), dtype=torch.bfloat16, device=X.device)
+    T = torch.empty((np_, M, r), dtype=torch.float32, device=X.device) if (save and r > 0) else None
+    Z = (torch.empty((np_, M, d_out), dtype=torch.float32, device=X.device)
+         if (save and act_code != ACT_IDENTITY) else None)
+    need = lora_linear_workspace_size(desc, 0)
+    ws = (workspace or Workspace(need, X.device, stream)).ensure(need, stream)
+    _check(lora_linear_fwd(desc, _ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(W_up), _ptr(A_up), _ptr(B_up),
+                           _ptr(Y), _ptr(T), _ptr(Z), ws.buf.data_ptr(), ws.nbytes, _stream_handle(stream)),
+           "lora_linear_fwd")
+    return Y, T, Z
+
+
+def backward(dY, X, W, A, B, s, act="identity", W_up=None, A_up=None, B_up=None, T_save=None, Z_save=None,
+             workspace=None, stream=None):
+    """dX, dA, dB (and dA_up, dB_up for swiglu)."""
+    import torch
+    M, d_in = X.shape
+    d_out = W.shape[0]
+    r = 0 if A is None else A.shape[0]
+    act_code = ACT_CODES[act] if isinstance(act, str) else act
+    desc = make_desc(M, d_in, d_out, r, s, act_code)
+    dX = torch.empty((M, d_in), dtype=torch.bfloat16, device=X.device)
+    dA = torch.empty((r, d_in), dtype=torch.float32, device=X.device) if r > 0 else None
+    dB = torch.empty((d_out, r), dtype=torch.float32, device=X.device) if r > 0 else None
+    sw = act_code == ACT_SWIGLU
+    dA_up = torch.empty_like(dA) if (sw and r > 0) else None
+    dB_up = torch.empty_like(dB) if (sw and r > 0) else None
+    need = lora_linear_workspace_size(desc, 1)
+    ws = (workspace or Workspace(need, X.device, stream)).ensure(need, stream)
+    _check(lora_linear_bwd(desc, _ptr(dY), _ptr(X), _ptr(W), _ptr(A), _ptr(B), _ptr(W_up), _ptr(A_up),
+                           _ptr(B_up), _ptr(T_save), _ptr(Z_save), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(dA_up),
+                           _ptr(dB_up), ws.buf.data_ptr(), ws.nbytes, _stream_handle(stream)),
+           "lora_linear_bwd")
+    return dX, dA, dB, dA_up, dB_up
+
+
+def _make_autograd():
+    import torch
+
+    class LoRALinearFunction(torch.autograd.Function):
+        """y = act(x W^T + s (x A^T) B^T) with W frozen; grads for x, A, B.
+
+        A and B are bf16 parameters; their gradients come back from the kernels
+        in fp32 and are cast to the parameter dtype by autograd's contract."""
+
+        @staticmethod
+        def forward(ctx, X, W, A, B, s, act):
+            Y, T, Z = forward(X, W, A, B, s, act)
+            ctx.save_for_backward(X, W, A, B, T, Z)
+            ctx.s, ctx.act = s, act
+            return Y
+
+        @staticmethod
+        def backward(ctx, dY):
+            X, W, A, B, T, Z = ctx.saved_tensors
+            dX, dA, dB, _, _ = backward(dY.contiguous(), X, W, A, B, ctx.s, ctx.act, T_save=T, Z_save=Z)
+            return dX, None, dA.to(A.dtype), dB.to(B.dtype), None, None
+
+    return LoRALinearFunction
+
+
+try:  # torch is optional for the 1:1 C wrappers
+    LoRALinearFunction = _make_autograd()
+except Exception:  # pragma: no cover
+    LoRALinearFunction = None

@@ -1,0 +1,278 @@
+// lora_rank.cuh — kernels for the rank-r side of the backward.
+//
+// rank_gemm_kernel: a split-K tcgen05 kernel for products whose result has
+//   only r (<= 64) columns and whose reduction runs over tokens or features:
+//     dA^T = X^T (s U)           [d_in  x r],  K = tokens   (X read MN-major)
+//     dB   = dZ^T (s T)          [d_out x r],  K = tokens   (dZ read MN-major)
+//     U_lo = dZ_lo B, T = X A^T  [M x r],      K = features (K-major)
+//   The fp32-grade operands (s U, s T) are split into bf16 hi + lo parts and
+//   summed as two MMAs into one fp32 accumulator, so the adapter gradients keep
+//   fp32-grade precision although the tensor cores take bf16.
+//   One CTA = one 128-row tile x one K range; it writes an fp32 partial that
+//   reduce_partials_kernel sums in a fixed order (deterministic, no atomics).
+// The elementwise kernels: B -> B^T, rank matrices -> transposed hi/lo bf16,
+// the activation backward dZ = dY * act'(Z) as hi/lo bf16.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace lora {
+
+constexpr int kRankThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+
+struct RankGemmParams {
+  CUtensorMap tm_a[2];
+  CUtensorMap tm_b[2];
+  int rows;          // rows of the result (M side of the MMA)
+  int K;             // reduction length
+  int m_tiles;
+  int kb_per_split;
+  float* partial;    // [splits][m_tiles*128][RP] fp32
+  uint32_t* status;
+};
+
+// Pair table: which A and B operand each accumulated product uses.
+//   kPairs == 1: A0 B0          kPairs == 2: A0 B0 + A0 B1
+//   kPairs == 3: A0 B0 + A0 B1 + A1 B0
+template <int kPairs> __device__ __forceinline__ int pair_a(int p) { return (kPairs == 3 && p == 2) ? 1 : 0; }
+template <int kPairs> __device__ __forceinline__ int pair_b(int p) { return (p == 1) ? 1 : 0; }
+
+template <bool kAMN, int kRP, int kPairs>
+struct RankCfg {
+  static constexpr int kNA = (kPairs == 3) ? 2 : 1;
+  static constexpr int kNB = (kPairs >= 2) ? 2 : 1;
+  static constexpr int kABytes = 128 * 64 * 2;
+  static constexpr int kBBytes = kRP * 128;
+  static constexpr int kStageBytes = kNA * kABytes + kNB * kBBytes;
+  static constexpr int kStages0 = (kSmemLimitBytes - 2048) / kStageBytes;
+  static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 2048;
+  static constexpr uint32_t kTmemCols = kRP < 32 ? 32 : kRP;
+};
+
+template <bool kAMN, int kRP, int kPairs>
+__global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid_constant__ RankGemmParams p) {
+  using C = RankCfg<kAMN, kRP, kPairs>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 2);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  AbortCtl ctl{abort_flag, p.status};
+  const int mt = blockIdx.x % p.m_tiles;
+  const int sp = blockIdx.x / p.m_tiles;
+  const int nkb_all = (p.K + 63) / 64;
+  const int kb0 = sp * p.kb_per_split;
+  int kb1 = kb0 + p.kb_per_split;
+  if (kb1 > nkb_all) kb1 = nkb_all;
+  const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && nkb > 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      RingPos rp;
+      for (int i = 0; i < nkb; ++i) {
+        if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
+        uint8_t* st = smem + rp.stage * C::kStageBytes;
+        uint64_t* fb = &full[rp.stage];
+        mbar_arrive_expect_tx(fb, C::kStageBytes);
+        const int k0 = (kb0 + i) * 64;
+        const int m0 = mt * 128;
+#pragma unroll
+        for (int a = 0; a < C::kNA; ++a) {
+          uint8_t* sa = st + a * C::kABytes;
+          if constexpr (kAMN) {
+            tma_load_2d_hint(sa, &p.tm_a[a], fb, m0, k0, pol);
+            tma_load_2d_hint(sa + 8192, &p.tm_a[a], fb, m0 + 64, k0, pol);
+          } else {
+            tma_load_2d_hint(sa, &p.tm_a[a], fb, k0, m0, pol);
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < C::kNB; ++b)
+          tma_load_2d(st + C::kNA * C::kABytes + b * C::kBBytes, &p.tm_b[b], fb, k0, 0);
+        rp.next(S);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nkb > 0) {
+      constexpr uint32_t kId = idesc_bf16(128, kRP, kAMN, false);
+      RingPos rp;
+      bool ok = true;
+      for (int i = 0; i < nkb; ++i) {
+        if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + rp.stage * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+          for (int pp = 0; pp < kPairs; ++pp) {
+            const uint32_t sa = st + pair_a<kPairs>(pp) * C::kABytes;
+            const uint32_t sb = st + C::kNA * C::kABytes + pair_b<kPairs>(pp) * C::kBBytes;
+            const uint64_t da = kAMN ? sdesc_sw128(sa + kk * 2048, 8192, 1024) : sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t db = sdesc_sw128(sb + kk * 32, 16, 1024);
+            mma_bf16(tbase, da, db, kId, (i == 0 && kk == 0 && pp == 0) ? 0u : 1u);
+          }
+        }
+        mma_commit(&empty[rp.stage]);
+        rp.next(S);
+      }
+      if (ok) mma_commit(acc_full);
+      // Teardown: every MMA issued here retires before TMEM is freed.
+      mma_commit(mma_done);
+      volatile uint32_t zero = 0u;
+      AbortCtl quiet{&zero, nullptr};
+      mbar_wait(mma_done, 0, quiet);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    float* dst = p.partial + (static_cast<size_t>(sp) * p.m_tiles * 128 + static_cast<size_t>(mt) * 128 + row) * kRP;
+    if (nkb == 0) {
+#pragma unroll
+      for (int c = 0; c < kRP; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else if (mbar_wait(acc_full, 0, ctl)) {
+      tc_fence_after();
+      __syncwarp();
+      const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+      for (int c0 = 0; c0 < kRP; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tl + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; c += 4)
+          *reinterpret_cast<float4*>(dst + c0 + c) = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                                                 __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::kTmemCols);
+  }
+}
+
+// dst = sum over splits of partial[sp][row][c] (+ add[row][c]); fixed order.
+// transpose == 0: dst[row * r + c];  transpose == 1: dst[c * rows + row].
+__global__ void reduce_partials_kernel(const float* __restrict__ partial, int splits, int rows_pad, int RP,
+                                       int rows, int r, const float* __restrict__ add, float* __restrict__ dst,
+                                       int transpose) {
+  const long long n = static_cast<long long>(rows) * r;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    int row, c;
+    if (transpose) { c = static_cast<int>(i / rows); row = static_cast<int>(i % rows); }
+    else { row = static_cast<int>(i / r); c = static_cast<int>(i % r); }
+    float acc = add ? add[static_cast<size_t>(row) * r + c] : 0.0f;
+    for (int sp = 0; sp < splits; ++sp) acc += partial[(static_cast<size_t>(sp) * rows_pad + row) * RP + c];
+    dst[i] = acc;
+  }
+}
+
+// src fp32 [M x r] -> hi, lo bf16 [r x ld] with v = scale * src, hi = bf16(v),
+// lo = bf16(v - hi).  Columns M..ld-1 are left untouched (never read).
+__global__ void rank_split_t_kernel(const float* __restrict__ src, int M, int r, float scale,
+                                    __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo, int ld) {
+  const long long n = static_cast<long long>(M) * r;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i / M);
+    const int m = static_cast<int>(i % M);
+    const float v = scale * src[static_cast<size_t>(m) * r + c];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[static_cast<size_t>(c) * ld + m] = h;
+    lo[static_cast<size_t>(c) * ld + m] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// B [d_out x r] -> B^T [r x d_out] (bf16, exact).
+__global__ void transpose_b_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r,
+                                   __nv_bfloat16* __restrict__ Bt) {
+  const long long n = static_cast<long long>(d_out) * r;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i / d_out);
+    const int j = static_cast<int>(i % d_out);
+    Bt[i] = B[static_cast<size_t>(j) * r + c];
+  }
+}
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+// Activation backward, 8 elements per thread-iteration (16-byte vectors).
+//   SiLU:   dZ = dY * s(z) (1 + z (1 - s(z)))
+//   SwiGLU: dZ_gate = dY * u * SiLU'(g),  dZ_up = dY * SiLU(g)
+// Each dZ is emitted as bf16 hi + bf16 lo (lo = bf16(dZ - hi)).
+template <bool kSwiglu>
+__global__ void act_bwd_kernel(const __nv_bfloat16* __restrict__ dY, const float* __restrict__ Z,
+                               const float* __restrict__ Zup, long long n, __nv_bfloat16* __restrict__ g_hi,
+                               __nv_bfloat16* __restrict__ g_lo, __nv_bfloat16* __restrict__ u_hi,
+                               __nv_bfloat16* __restrict__ u_lo) {
+  const long long nv = n / 8;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 dyv = reinterpret_cast<const uint4*>(dY)[i];
+    const __nv_bfloat16* dyb = reinterpret_cast<const __nv_bfloat16*>(&dyv);
+    const float4 z0 = reinterpret_cast<const float4*>(Z)[2 * i];
+    const float4 z1 = reinterpret_cast<const float4*>(Z)[2 * i + 1];
+    const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+    float uu[8];
+    if constexpr (kSwiglu) {
+      const float4 u0 = reinterpret_cast<const float4*>(Zup)[2 * i];
+      const float4 u1 = reinterpret_cast<const float4*>(Zup)[2 * i + 1];
+      uu[0] = u0.x; uu[1] = u0.y; uu[2] = u0.z; uu[3] = u0.w;
+      uu[4] = u1.x; uu[5] = u1.y; uu[6] = u1.z; uu[7] = u1.w;
+    }
+    __align__(16) __nv_bfloat16 gh[8], gl[8], uh[8], ul[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float dy = __bfloat162float(dyb[e]);
+      const float z = zz[e];
+      const float sg = sigmoidf_(z);
+      const float dsilu = sg * (1.0f + z * (1.0f - sg));
+      float dg;
+      if constexpr (kSwiglu) {
+        dg = dy * uu[e] * dsilu;
+        const float du = dy * (z * sg);
+        uh[e] = __float2bfloat16_rn(du);
+        ul[e] = __float2bfloat16_rn(du - __bfloat162float(uh[e]));
+      } else {
+        dg = dy * dsilu;
+      }
+      gh[e] = __float2bfloat16_rn(dg);
+      gl[e] = __float2bfloat16_rn(dg - __bfloat162float(gh[e]));
+    }
+    reinterpret_cast<uint4*>(g_hi)[i] = *reinterpret_cast<uint4*>(gh);
+    reinterpret_cast<uint4*>(g_lo)[i] = *reinterpret_cast<uint4*>(gl);
+    if constexpr (kSwiglu) {
+      reinterpret_cast<uint4*>(u_hi)[i] = *reinterpret_cast<uint4*>(uh);
+      reinterpret_cast<uint4*>(u_lo)[i] = *reinterpret_cast<uint4*>(ul);
+    }
+  }
+}
+
+}  // namespace lora

@@ -1,0 +1,91 @@
+"""The C-ABI library: it loads, exports every symbol include/lora_linear.h
+declares, and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_linear.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lora_linear_fine_b200 import build
+    build.build(quiet=True)
+    import lora_linear_fine_b200 as L
+    return L
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lora_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected(lib):
+    assert set(declared_functions()) == set(lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(so, name), name
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.lora_linear_abi_version() == 1
+    for code in range(8):
+        assert lib.status_string(code)
+    assert lib.status_string(99) == "unknown status"
+
+
+def test_workspace_size(lib):
+    d = lib.make_desc(64, 256, 256, 8, 2.0, "identity")
+    assert lib.lora_linear_workspace_size(d, 0) > 0
+    assert lib.lora_linear_workspace_size(d, 1) >= lib.lora_linear_workspace_size(d, 0)
+    # SwiGLU backward needs the hi/lo dZ buffers: 4 * M * d_out * 2 bytes at least
+    d2 = lib.make_desc(64, 256, 256, 8, 2.0, "swiglu")
+    assert lib.lora_linear_workspace_size(d2, 1) >= 4 * 64 * 256 * 2
+    for bad in [lib.make_desc(64, 256, 256, 12, 2.0, 0), lib.make_desc(64, 250, 256, 8, 2.0, 0),
+                lib.make_desc(-1, 256, 256, 8, 2.0, 0), lib.make_desc(64, 256, 256, 8, 2.0, 7),
+                lib.make_desc(64, 256, 256, 72, 2.0, 0)]:
+        assert lib.lora_linear_workspace_size(bad, 0) == 0
+        assert lib.lora_linear_workspace_size(bad, 1) == 0
+
+
+def _fwd(lib, desc, X=16, W=16, A=16, B=16, Y=16, ws=16, ws_bytes=1 << 20, **kw):
+    return lib.lora_linear_fwd(desc, X, W, A, B, kw.get("W_up"), kw.get("A_up"), kw.get("B_up"), Y,
+                               kw.get("T"), kw.get("Z"), ws, ws_bytes, None)
+
+
+def test_fwd_rejects_bad_arguments_without_launching(lib):
+    ok = lib.make_desc(64, 256, 256, 8, 2.0, "identity")
+    assert _fwd(lib, ok, X=None) == 1                 # INVALID_ARG
+    assert _fwd(lib, ok, A=None) == 1                 # r > 0 needs A, B
+    assert _fwd(lib, ok, X=24) == 2                   # not 16-byte aligned
+    assert _fwd(lib, lib.make_desc(64, 252, 256, 8, 2.0, 0)) == 2   # d_in % 8
+    assert _fwd(lib, lib.make_desc(64, 256, 256, 12, 2.0, 0)) == 3  # r % 8
+    assert _fwd(lib, lib.make_desc(64, 256, 256, 8, 2.0, 5)) == 1   # act
+    sw = lib.make_desc(64, 256, 256, 8, 2.0, "swiglu")
+    assert _fwd(lib, sw) == 1                         # swiglu needs the up projection
+
+
+def test_bwd_rejects_bad_arguments_without_launching(lib):
+    d = lib.make_desc(64, 256, 256, 8, 2.0, "silu")
+    # act != identity needs Z_save
+    st = lib.lora_linear_bwd(d, 16, 16, 16, 16, 16, None, None, None, 16, None, 16, 16, 16, None, None,
+                             16, 1 << 20, None)
+    assert st == 1
+    st = lib.lora_linear_bwd(d, 16, 16, 16, 16, 16, None, None, None, 16, 16, 16, 16, None, None, None,
+                             16, 1 << 20, None)
+    assert st == 1                                    # dB missing
+
+
+def test_no_gpu_means_cuda_error_not_crash(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    ok = lib.make_desc(64, 256, 256, 8, 2.0, "identity")
+    assert _fwd(lib, ok) == 6                         # LORA_ERR_CUDA: no device
