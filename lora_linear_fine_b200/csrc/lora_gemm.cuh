@@ -33,7 +33,10 @@ constexpr int kBN = 256;
 constexpr int kBK = 64;
 constexpr int kGemmThreads = 320;
 
-enum EpiKind : int { kEpiIdentity = 0, kEpiSilu = 1, kEpiSwiglu = 2, kEpiGrad = 3 };
+// kEpiGrad: backward dX with bf16 operands (dZ = dY exactly).
+// kEpiGradF16: backward dX with fp16 dZ and fp16 W / B^T (activation backward:
+//   dZ is fp32-valued and bf16 would round it too coarsely for dX).
+enum EpiKind : int { kEpiIdentity = 0, kEpiSilu = 1, kEpiSwiglu = 2, kEpiGrad = 3, kEpiGradF16 = 4 };
 
 struct GemmParams {
   CUtensorMap tm_a[2];    // M-side operand   fwd: X        bwd: dZ (per pair)
@@ -46,18 +49,22 @@ struct GemmParams {
   int r;                  // adapter rank (columns saved to rank_save)
   float s;                // LoRA scale
   __nv_bfloat16* out;     // [M x N] bf16
-  float* rank_save;       // [npair][M x r] fp32 or null
+  float* rank_save;       // [npair][M x r] fp32 or null (rank columns computed in the K-loop)
+  const float* rank_in;   // [npair][M x r] fp32: rank columns computed beforehand (kRankGlobal)
   float* z_save;          // [npair][M x N] fp32 or null (forward SiLU / SwiGLU)
   uint32_t* status;       // device status word or null
   int m_tiles, n_tiles, num_tiles, group_m;
 };
 
-template <bool kBwd, int kRP, int kNPair, int kEpi>
+// kRankGlobal == false: the rank columns T = X A^T (U = dZ B) ride the K-loop as
+//   extra MMA columns (X read from HBM once; costs RP/256 extra tensor work).
+// kRankGlobal == true: T (U) was computed by a rank pass; the epilogue loads it.
+template <bool kBwd, int kRP, int kNPair, int kEpi, bool kRankGlobal>
 struct GemmCfg {
   static constexpr bool kSwigluFwd = (!kBwd) && (kEpi == kEpiSwiglu);
   static constexpr int kOutCols = kSwigluFwd ? 128 : 256;           // output columns per tile
   static constexpr int kKPairs = kBwd ? kNPair : 1;                 // pairs walked along K
-  static constexpr int kRankRows = kSwigluFwd ? 2 * kRP : kRP;      // rank rows in one stage
+  static constexpr int kRankRows = kRankGlobal ? 0 : (kSwigluFwd ? 2 * kRP : kRP);  // rank rows per stage
   static constexpr int kUpCols = kSwigluFwd ? 128 : 256;            // N of one up-projection MMA
   static constexpr int kABytes = kBM * kBK * 2;                     // 16 KB
   static constexpr int kWBytes = kBN * kBK * 2;                     // 32 KB
@@ -68,7 +75,7 @@ struct GemmCfg {
   static constexpr int kStages0 = (kSmemLimitBytes - 1024 - kBarBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 6 ? 6 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;
-  static constexpr int kRankCols = kNPair * kRP;
+  static constexpr int kRankCols = kRankGlobal ? 0 : kNPair * kRP;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1 KB alignment");
   static_assert(kRP % 16 == 0 && kRP <= 64, "rank padding");
@@ -88,9 +95,10 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mt,
   nt = idx / gm;
 }
 
-template <bool kBwd, int kRP, int kNPair, int kEpi>
+template <bool kBwd, int kRP, int kNPair, int kEpi, bool kRankGlobal>
 __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<kBwd, kRP, kNPair, kEpi>;
+  using C = GemmCfg<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
+  constexpr bool kRankLoop = (kRP > 0) && !kRankGlobal;
   constexpr int S = C::kStages;
 
   extern __shared__ uint8_t smem_raw[];
@@ -124,7 +132,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid
   if (warp == 0 && lane == 0) {
     for (int j = 0; j < (C::kSwigluFwd ? 1 : kNPair); ++j) tma_prefetch_desc(&p.tm_a[j]);
     for (int j = 0; j < kNPair; ++j) tma_prefetch_desc(&p.tm_w[j]);
-    if (kRP > 0) for (int j = 0; j < kNPair; ++j) { tma_prefetch_desc(&p.tm_r[j]); tma_prefetch_desc(&p.tm_up[j]); }
+    if (kRankLoop) for (int j = 0; j < kNPair; ++j) tma_prefetch_desc(&p.tm_r[j]);
+    if (kRP > 0) for (int j = 0; j < kNPair; ++j) tma_prefetch_desc(&p.tm_up[j]);
   }
   if (warp == 1) { tmem_alloc(tmem_slot, C::kTmemCols); tmem_relinquish(); }
   tc_fence_before();
@@ -162,14 +171,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid
               } else {
                 tma_load_2d_hint(sw, &p.tm_w[0], fb, k0, n0, pol_keep);
               }
-              if constexpr (kRP > 0) {
+              if constexpr (kRankLoop) {
                 tma_load_2d_hint(sr, &p.tm_r[0], fb, k0, 0, pol_keep);
                 if constexpr (C::kSwigluFwd) tma_load_2d_hint(sr + kRP * 128, &p.tm_r[1], fb, k0, 0, pol_keep);
               }
             } else {
 #pragma unroll
               for (int b = 0; b < 4; ++b) tma_load_2d_hint(sw + b * 8192, &p.tm_w[j], fb, n0 + 64 * b, k0, pol_keep);
-              if constexpr (kRP > 0) tma_load_2d_hint(sr, &p.tm_r[j], fb, k0, 0, pol_keep);
+              if constexpr (kRankLoop) tma_load_2d_hint(sr, &p.tm_r[j], fb, k0, 0, pol_keep);
             }
             ++issued;
             rp.next(S);
@@ -205,8 +214,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdMain = idesc_bf16(128, 256, false, kBwd);
-      constexpr uint32_t kIdRank = idesc_bf16(128, C::kSwigluFwd ? 2 * (kRP > 0 ? kRP : 8) : (kRP > 0 ? kRP : 16), false, false);
+      constexpr bool kF16 = (kEpi == kEpiGradF16);
+      constexpr uint32_t kIdMain = idesc_mma(128, 256, false, kBwd, kF16);
+      constexpr uint32_t kIdRank =
+          idesc_mma(128, C::kSwigluFwd ? 2 * (kRP > 0 ? kRP : 8) : (kRP > 0 ? kRP : 16), false, false, kF16);
       constexpr uint32_t kIdUp = idesc_bf16(128, C::kUpCols, false, true);
       RingPos rp;
       uint32_t acc_phase = 0;
@@ -228,7 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid
               const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
               const uint64_t dw = kBwd ? sdesc_sw128(sw + kk * 2048, 8192, 1024) : sdesc_sw128(sw + kk * 32, 16, 1024);
               mma_bf16(tbase, da, dw, kIdMain, (first_main && kk == 0) ? 0u : 1u);
-              if constexpr (kRP > 0) {
+              if constexpr (kRankLoop) {
                 const uint64_t dr = sdesc_sw128(sr + kk * 32, 16, 1024);
                 mma_bf16(trank, da, dr, kIdRank, (kb == 0 && kk == 0) ? 0u : 1u);
               }
@@ -240,6 +251,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid
         }
         if (!ok) break;
         if constexpr (kRP > 0) {
+          // K-loop done: the epilogue may now use this tile's up-projection
+          // slots (waiting on them earlier could alias an older phase).
           mma_commit(acc_full);
           for (int j = 0; j < kNPair && ok; ++j) {
             if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
@@ -286,23 +299,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) lora_gemm_kernel(const __grid
       // Skip the ring positions of the K-loop.
       for (int i = 0; i < nkb_total; ++i) rp.next(S);
       if constexpr (kRP > 0) {
+        float rk[kRP];
+        if constexpr (!kRankLoop) {
+          // Rank values computed by the rank pass: fetch them while the K-loop runs.
+          if (h < kNPair) {
+            const float* src = p.rank_in + (static_cast<size_t>(h) * p.M + row) * p.r;
+#pragma unroll
+            for (int c = 0; c < kRP; c += 4) {
+              float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (row_ok && c < p.r) v4 = *reinterpret_cast<const float4*>(src + c);
+              rk[c] = v4.x; rk[c + 1] = v4.y; rk[c + 2] = v4.z; rk[c + 3] = v4.w;
+            }
+          }
+        }
+        // The up-projection slots of this tile are only safe to wait on once the
+        // K-loop is done: before that a slot's barrier may be two phases behind,
+        // where a parity wait would return early.
         if (!mbar_wait(acc_full, acc_phase, ctl)) break;
         tc_fence_after();
         bool ok = true;
         RingPos up = rp;
         for (int j = 0; j < kNPair; ++j) {
           if (j == h) {
-            __syncwarp();   // tcgen05.ld is .sync.aligned: converge the warp first
-            float rk[kRP];
+            if constexpr (kRankLoop) {
+              __syncwarp();   // tcgen05.ld is .sync.aligned: converge the warp first
 #pragma unroll
-            for (int c0 = 0; c0 < kRP; c0 += 16) {
-              uint32_t v[16];
-              tmem_ld16(tlane + 256 + j * kRP + c0, v);
-              tmem_wait_ld();
+              for (int c0 = 0; c0 < kRP; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tlane + 256 + j * kRP + c0, v);
+                tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 16; ++c) rk[c0 + c] = __uint_as_float(v[c]);
+                for (int c = 0; c < 16; ++c) rk[c0 + c] = __uint_as_float(v[c]);
+              }
             }
-            if (p.rank_save != nullptr && nt == 0 && row_ok) {
+            if (kRankLoop && p.rank_save != nullptr && nt == 0 && row_ok) {
               float* dst = p.rank_save + (static_cast<size_t>(j) * p.M + row) * p.r;
 #pragma unroll
               for (int c = 0; c < kRP; c += 4)

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "lora_gemm.cuh"
+#include "lora_gemm2.cuh"
 #include "lora_rank.cuh"
 #include "lora_small_m.cuh"
 
@@ -84,12 +85,13 @@ lora_status_t device_info(DevInfo* out) {
 // 2D bf16 tensor map with 128-byte swizzle: `inner` contiguous elements per
 // row, `outer` rows `row_elems` elements apart; box = box_inner x box_outer.
 bool make_tm(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_elems,
-             uint32_t box_inner, uint32_t box_outer) {
+             uint32_t box_inner, uint32_t box_outer, bool f16 = false) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_elems * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+  const CUtensorMapDataType dt = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUresult r = g_encode(tm, dt, 2, const_cast<void*>(ptr), dims, strides, box,
                               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) LORA_LOG("cuTensorMapEncodeTiled failed (%d): inner=%llu outer=%llu box=%ux%u", (int)r,
@@ -117,6 +119,24 @@ lora_status_t check_desc(const lora_linear_desc* d) {
   return LORA_OK;
 }
 
+// Workspace layouts (offsets in bytes, each 256-aligned, status word at 0).
+struct Plan {
+  // shapes
+  int np = 1;          // projections: 2 for SwiGLU (gate, up)
+  int RP = 0;          // r padded to the MMA granule (0, 16, 32, 64)
+  bool act_f16 = false;  // backward with an activation: fp16 dZ operands
+  bool rank_loop = false;  // rank columns inside the GEMM K-loop
+  int64_t M8 = 8;
+  // split-K widths of the rank passes
+  int splits_t = 1, splits_u = 1, splits_a = 1, splits_b = 1;
+  // regions
+  size_t bt[2] = {}, t_ws[2] = {}, part_t = 0;                 // forward + backward
+  size_t u_ws = 0, tt_hi[2] = {}, tt_lo[2] = {}, ut_hi[2] = {}, ut_lo[2] = {};
+  size_t dz_hi[2] = {}, dz_lo[2] = {}, w16[2] = {};
+  size_t part_u = 0, part_a = 0, part_b = 0;
+  size_t total = 0;
+};
+
 // Split-K width for a rank-r product with `tiles` row tiles and `nkb` 64-wide K blocks.
 int rank_splits(int64_t tiles, int64_t nkb) {
   int64_t s = kTargetCtas / (tiles > 0 ? tiles : 1);
@@ -126,62 +146,64 @@ int rank_splits(int64_t tiles, int64_t nkb) {
   return static_cast<int>(s);
 }
 
-// Workspace layout of the backward (offsets in bytes, each 256-aligned).
-struct BwdLayout {
-  size_t bt[2], tw[2], tt_hi[2], tt_lo[2], uw, ut_hi[2], ut_lo[2], dz_hi[2], dz_lo[2];
-  size_t part_a, part_b, part_u;
-  int splits_a, splits_b, splits_u, splits_t;
-  size_t total;
-};
-
-size_t fwd_workspace(const lora_linear_desc* d) {
-  const int np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
-  size_t off = kStatusBytes;
-  if (d->r > 0) off += np * align_up(static_cast<size_t>(d->r) * d->d_out * 2, 256);
-  return off;
-}
-
-BwdLayout bwd_layout(const lora_linear_desc* d) {
-  BwdLayout L{};
-  const int np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
-  const int RP = rank_pad(d->r);
-  const int64_t M8 = align_up(static_cast<size_t>(d->M > 0 ? d->M : 1), 8);
+Plan make_plan(const lora_linear_desc* d, bool backward) {
+  Plan P;
+  P.np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
+  P.RP = rank_pad(d->r);
+  P.act_f16 = backward && d->act != LORA_ACT_IDENTITY;
+  // The K-loop rank columns cost RP/256 of the tile's tensor work: worth it
+  // for RP = 16 (X or dY read once); a separate rank pass is cheaper above.
+  P.rank_loop = d->r > 0 && P.RP == 16 && !P.act_f16 && d->act != LORA_ACT_SWIGLU;
+  P.M8 = static_cast<int64_t>(align_up(static_cast<size_t>(d->M > 0 ? d->M : 1), 8));
+  const int64_t M = d->M, r = d->r;
+  const int64_t tiles_m = ceil_div(M > 0 ? M : 1, 128);
   size_t off = kStatusBytes;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += align_up(bytes, 256);
     return o;
   };
-  // U of all pairs is one [npair][M x r] block: the dX kernel writes it that way.
-  if (d->r > 0) L.uw = take(static_cast<size_t>(np) * d->M * d->r * 4);
-  for (int j = 0; j < np; ++j) {
-    if (d->r > 0) {
-      L.bt[j] = take(static_cast<size_t>(d->r) * d->d_out * 2);
-      L.tw[j] = take(static_cast<size_t>(d->M) * d->r * 4);
-      L.tt_hi[j] = take(static_cast<size_t>(d->r) * M8 * 2);
-      L.tt_lo[j] = take(static_cast<size_t>(d->r) * M8 * 2);
-      L.ut_hi[j] = take(static_cast<size_t>(d->r) * M8 * 2);
-      L.ut_lo[j] = take(static_cast<size_t>(d->r) * M8 * 2);
-    }
-    if (d->act != LORA_ACT_IDENTITY) {
-      L.dz_hi[j] = take(static_cast<size_t>(d->M) * d->d_out * 2);
-      L.dz_lo[j] = take(static_cast<size_t>(d->M) * d->d_out * 2);
+  if (r > 0) {
+    for (int j = 0; j < P.np; ++j) P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
+    P.splits_t = rank_splits(tiles_m, ceil_div(d->d_in, 64));
+    const bool need_t = backward || !P.rank_loop;
+    if (need_t) {
+      // T of all projections is one [np][M x r] block (the GEMM reads it that way).
+      P.t_ws[0] = take(static_cast<size_t>(P.np) * M * r * 4);
+      P.t_ws[1] = P.t_ws[0] + static_cast<size_t>(M) * r * 4;
+      P.part_t = take(static_cast<size_t>(P.splits_t) * tiles_m * 128 * P.RP * 4);
     }
   }
-  if (d->r > 0) {
-    const int64_t tiles_a = ceil_div(d->d_in, 128), tiles_b = ceil_div(d->d_out, 128), tiles_u = ceil_div(d->M, 128);
-    const int64_t nkb_tok = ceil_div(d->M, 64);
-    L.splits_a = rank_splits(tiles_a, nkb_tok);
-    L.splits_b = rank_splits(tiles_b, nkb_tok);
-    L.splits_u = rank_splits(tiles_u, ceil_div(d->d_out, 64));
-    L.splits_t = rank_splits(tiles_u, ceil_div(d->d_in, 64));
-    const int su = L.splits_u > L.splits_t ? L.splits_u : L.splits_t;
-    L.part_a = take(static_cast<size_t>(L.splits_a) * tiles_a * 128 * RP * 4);
-    L.part_b = take(static_cast<size_t>(L.splits_b) * tiles_b * 128 * RP * 4);
-    L.part_u = take(static_cast<size_t>(su) * (tiles_u > 0 ? tiles_u : 1) * 128 * RP * 4);
+  if (!backward) {
+    P.total = off;
+    return P;
   }
-  L.total = off;
-  return L;
+  if (P.act_f16) {
+    for (int j = 0; j < P.np; ++j) {
+      P.dz_hi[j] = take(static_cast<size_t>(M) * d->d_out * 2);
+      P.dz_lo[j] = take(static_cast<size_t>(M) * d->d_out * 2);
+      P.w16[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
+    }
+  }
+  if (r > 0) {
+    P.u_ws = take(static_cast<size_t>(P.np) * M * r * 4);
+    for (int j = 0; j < P.np; ++j) {
+      P.tt_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
+      P.tt_lo[j] = take(static_cast<size_t>(r) * P.M8 * 2);
+      P.ut_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
+      P.ut_lo[j] = take(static_cast<size_t>(r) * P.M8 * 2);
+    }
+    const int64_t tiles_a = ceil_div(d->d_in, 128), tiles_b = ceil_div(d->d_out, 128);
+    const int64_t nkb_tok = ceil_div(M > 0 ? M : 1, 64);
+    P.splits_u = rank_splits(tiles_m, ceil_div(d->d_out, 64));
+    P.splits_a = rank_splits(tiles_a, nkb_tok);
+    P.splits_b = rank_splits(tiles_b, nkb_tok);
+    P.part_u = take(static_cast<size_t>(P.splits_u) * tiles_m * 128 * P.RP * 4);
+    P.part_a = take(static_cast<size_t>(P.splits_a) * tiles_a * 128 * P.RP * 4);
+    P.part_b = take(static_cast<size_t>(P.splits_b) * tiles_b * 128 * P.RP * 4);
+  }
+  P.total = off;
+  return P;
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -203,51 +225,122 @@ lora_status_t check_launch(const char* what) {
   return LORA_OK;
 }
 
+#define LORA_TRY(...)                           \
+  do {                                          \
+    const lora_status_t _s = (__VA_ARGS__);     \
+    if (_s != LORA_OK) return _s;               \
+  } while (0)
+
 // ---------------------------------------------------------------------------
 // kernel launchers
 // ---------------------------------------------------------------------------
-template <bool kBwd, int kRP, int kNPair, int kEpi>
+template <bool kBwd, int kRP, int kNPair, int kEpi, bool kRankGlobal>
 lora_status_t launch_gemm(const GemmParams& p, int sms, cudaStream_t st) {
-  using C = GemmCfg<kBwd, kRP, kNPair, kEpi>;
-  auto k = lora_gemm_kernel<kBwd, kRP, kNPair, kEpi>;
+  using C = GemmCfg<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
+  auto k = lora_gemm_kernel<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return cuda_error("cudaFuncSetAttribute(gemm)");
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  LORA_LOG("gemm bwd=%d RP=%d npair=%d epi=%d tiles=%d grid=%d smem=%d stages=%d", (int)kBwd, kRP, kNPair, kEpi,
-           p.num_tiles, grid, C::kSmemBytes, C::kStages);
+  LORA_LOG("gemm bwd=%d RP=%d npair=%d epi=%d global=%d tiles=%d grid=%d smem=%d stages=%d", (int)kBwd, kRP,
+           kNPair, kEpi, (int)kRankGlobal, p.num_tiles, grid, C::kSmemBytes, C::kStages);
   k<<<grid, kGemmThreads, C::kSmemBytes, st>>>(p);
   return check_launch("lora_gemm_kernel");
 }
 
+// CTA-pair variant (tcgen05 cta_group::2, 256 x 256 tiles): launched as
+// clusters of two CTAs.  p.m_tiles counts 256-row tiles.
+template <bool kBwd, int kRP, int kNPair, int kEpi, bool kRankGlobal>
+lora_status_t launch_gemm2(const GemmParams& p, int sms, cudaStream_t st) {
+  using C = Gemm2Cfg<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
+  auto k = lora_gemm2_kernel<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return cuda_error("cudaFuncSetAttribute(gemm2)");
+  const int clusters = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LORA_LOG("gemm2 bwd=%d RP=%d npair=%d epi=%d global=%d tiles=%d clusters=%d smem=%d stages=%d", (int)kBwd, kRP,
+           kNPair, kEpi, (int)kRankGlobal, p.num_tiles, clusters, C::kSmemBytes, C::kStages);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, p);
+  if (e != cudaSuccess) {
+    LORA_LOG("gemm2 launch: %s", cudaGetErrorString(e));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return LORA_ERR_CUDA;
+  }
+  return check_launch("lora_gemm2_kernel");
+}
+
+bool pair_kernel_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("LORA_LINEAR_PAIR");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+// Instantiated variants: r = 0; RP = 16 with the rank columns in the K-loop;
+// RP in {16, 32, 64} with the rank columns from a rank pass.  `pair` selects
+// the CTA-pair kernel (p already tiled for it).
 template <bool kBwd, int kNPair, int kEpi>
-lora_status_t launch_gemm_rp(int RP, const GemmParams& p, int sms, cudaStream_t st) {
+lora_status_t launch_gemm_variant(int RP, bool rank_loop, bool pair, const GemmParams& p, int sms, cudaStream_t st) {
+  if (pair) {
+    if (RP == 0) return launch_gemm2<kBwd, 0, kNPair, kEpi, true>(p, sms, st);
+    if (rank_loop) {
+      if constexpr (kNPair == 1 && kEpi != kEpiSwiglu && kEpi != kEpiGradF16) {
+        if (RP == 16) return launch_gemm2<kBwd, 16, kNPair, kEpi, false>(p, sms, st);
+      }
+      return LORA_ERR_UNSUPPORTED;
+    }
+    switch (RP) {
+      case 16: return launch_gemm2<kBwd, 16, kNPair, kEpi, true>(p, sms, st);
+      case 32: return launch_gemm2<kBwd, 32, kNPair, kEpi, true>(p, sms, st);
+      case 64: return launch_gemm2<kBwd, 64, kNPair, kEpi, true>(p, sms, st);
+      default: return LORA_ERR_UNSUPPORTED;
+    }
+  }
+  if (RP == 0) return launch_gemm<kBwd, 0, kNPair, kEpi, true>(p, sms, st);
+  if (rank_loop) {
+    if constexpr (kNPair == 1 && kEpi != kEpiSwiglu && kEpi != kEpiGradF16) {
+      if (RP == 16) return launch_gemm<kBwd, 16, kNPair, kEpi, false>(p, sms, st);
+    }
+    return LORA_ERR_UNSUPPORTED;
+  }
   switch (RP) {
-    case 0: return launch_gemm<kBwd, 0, kNPair, kEpi>(p, sms, st);
-    case 16: return launch_gemm<kBwd, 16, kNPair, kEpi>(p, sms, st);
-    case 32: return launch_gemm<kBwd, 32, kNPair, kEpi>(p, sms, st);
-    case 64: return launch_gemm<kBwd, 64, kNPair, kEpi>(p, sms, st);
+    case 16: return launch_gemm<kBwd, 16, kNPair, kEpi, true>(p, sms, st);
+    case 32: return launch_gemm<kBwd, 32, kNPair, kEpi, true>(p, sms, st);
+    case 64: return launch_gemm<kBwd, 64, kNPair, kEpi, true>(p, sms, st);
     default: return LORA_ERR_UNSUPPORTED;
   }
 }
 
-template <bool kAMN, int kRP, int kPairs>
+template <bool kAMN, int kRP, int kNA, int kNB, bool kF16>
 lora_status_t launch_rank(const RankGemmParams& p, int splits, cudaStream_t st) {
-  using C = RankCfg<kAMN, kRP, kPairs>;
-  auto k = rank_gemm_kernel<kAMN, kRP, kPairs>;
+  using C = RankCfg<kAMN, kRP, kNA, kNB, kF16>;
+  auto k = rank_gemm_kernel<kAMN, kRP, kNA, kNB, kF16>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return cuda_error("cudaFuncSetAttribute(rank)");
-  LORA_LOG("rank mn=%d RP=%d pairs=%d rows=%d K=%d tiles=%d splits=%d", (int)kAMN, kRP, kPairs, p.rows, p.K,
-           p.m_tiles, splits);
+  LORA_LOG("rank mn=%d RP=%d na=%d nb=%d f16=%d pairs=%d rows=%d K=%d tiles=%d splits=%d", (int)kAMN, kRP, kNA,
+           kNB, (int)kF16, p.npairs, p.rows, p.K, p.m_tiles, splits);
   k<<<p.m_tiles * splits, kRankThreads, C::kSmemBytes, st>>>(p);
   return check_launch("rank_gemm_kernel");
 }
 
-template <bool kAMN, int kPairs>
+template <bool kAMN, int kNA, int kNB, bool kF16>
 lora_status_t launch_rank_rp(int RP, const RankGemmParams& p, int splits, cudaStream_t st) {
   switch (RP) {
-    case 16: return launch_rank<kAMN, 16, kPairs>(p, splits, st);
-    case 32: return launch_rank<kAMN, 32, kPairs>(p, splits, st);
-    case 64: return launch_rank<kAMN, 64, kPairs>(p, splits, st);
+    case 16: return launch_rank<kAMN, 16, kNA, kNB, kF16>(p, splits, st);
+    case 32: return launch_rank<kAMN, 32, kNA, kNB, kF16>(p, splits, st);
+    case 64: return launch_rank<kAMN, 64, kNA, kNB, kF16>(p, splits, st);
     default: return LORA_ERR_UNSUPPORTED;
   }
 }
@@ -259,10 +352,15 @@ int grid_for(long long n, int per_block, int sms) {
   return static_cast<int>(g);
 }
 
-lora_status_t transpose_b(const void* B, int64_t d_out, int64_t r, void* Bt, int sms, cudaStream_t st) {
+lora_status_t transpose_b(const void* B, int64_t d_out, int64_t r, void* Bt, bool f16, uint32_t* status, int sms,
+                          cudaStream_t st) {
   const long long n = d_out * r;
-  transpose_b_kernel<<<grid_for(n, 256, sms), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(B), (int)d_out,
-                                                           (int)r, static_cast<__nv_bfloat16*>(Bt));
+  if (f16)
+    transpose_b_kernel<__half><<<grid_for(n, 256, sms), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(B), (int)d_out, (int)r, static_cast<__half*>(Bt), status);
+  else
+    transpose_b_kernel<__nv_bfloat16><<<grid_for(n, 256, sms), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(B), (int)d_out, (int)r, static_cast<__nv_bfloat16*>(Bt), status);
   return check_launch("transpose_b_kernel");
 }
 
@@ -275,19 +373,85 @@ lora_status_t reduce_partials(const float* part, int splits, int rows, int RP, i
   return check_launch("reduce_partials_kernel");
 }
 
-lora_status_t rank_split_t(const float* src, int M, int r, float scale, void* hi, void* lo, int ld, int sms,
-                           cudaStream_t st) {
+lora_status_t rank_split_t(const float* src, int M, int r, float scale, void* hi, void* lo, int ld, bool f16,
+                           uint32_t* status, int sms, cudaStream_t st) {
   const long long n = static_cast<long long>(M) * r;
-  rank_split_t_kernel<<<grid_for(n, 256, sms), 256, 0, st>>>(src, M, r, scale, static_cast<__nv_bfloat16*>(hi),
-                                                             static_cast<__nv_bfloat16*>(lo), ld);
+  if (f16)
+    rank_split_t_kernel<__half><<<grid_for(n, 256, sms), 256, 0, st>>>(
+        src, M, r, scale, static_cast<__half*>(hi), static_cast<__half*>(lo), ld, status);
+  else
+    rank_split_t_kernel<__nv_bfloat16><<<grid_for(n, 256, sms), 256, 0, st>>>(
+        src, M, r, scale, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo), ld, status);
   return check_launch("rank_split_t_kernel");
 }
 
-#define LORA_TRY(...)                    \
-  do {                                   \
-    const lora_status_t _s = (__VA_ARGS__); \
-    if (_s != LORA_OK) return _s;        \
-  } while (0)
+// rows x r result of sum_q A[pa[q]] * B[pb[q]] reduced over K = 64-blocks split
+// `splits` ways, written (after a fixed-order reduction) to dst.
+struct RankJob {
+  bool a_mn = false;   // A read MN-major (result rows are the A tensor's columns)
+  bool f16 = false;
+  const void* a[2] = {nullptr, nullptr};
+  int64_t a_inner = 0, a_outer = 0, a_ld = 0;     // A tensors share one shape
+  const void* b[2] = {nullptr, nullptr};
+  int64_t b_inner = 0, b_ld = 0;                  // B tensors: r rows x b_inner
+  int na = 1, nb = 1, npairs = 1;
+  int pa[4] = {0, 0, 0, 0}, pb[4] = {0, 0, 0, 0};
+  int rows = 0, K = 0;
+  float* partial = nullptr;
+  int splits = 1;
+  const float* add = nullptr;
+  float* dst = nullptr;
+  int transpose = 0;
+};
+
+lora_status_t run_rank(const RankJob& J, int RP, int r, uint32_t* status, int sms, cudaStream_t st) {
+  RankGemmParams q;
+  std::memset(&q, 0, sizeof(q));
+  bool ok = true;
+  for (int i = 0; i < J.na; ++i)
+    ok = ok && make_tm(&q.tm_a[i], J.a[i], J.a_inner, J.a_outer, J.a_ld, 64, J.a_mn ? 64 : 128, J.f16);
+  for (int i = 0; i < J.nb; ++i) ok = ok && make_tm(&q.tm_b[i], J.b[i], J.b_inner, r, J.b_ld, 64, RP, J.f16);
+  if (!ok) return LORA_ERR_CUDA;
+  q.rows = J.rows;
+  q.K = J.K;
+  q.m_tiles = static_cast<int>(ceil_div(J.rows, 128));
+  q.kb_per_split = static_cast<int>(ceil_div(ceil_div(J.K, 64), J.splits));
+  q.npairs = J.npairs;
+  for (int i = 0; i < 4; ++i) { q.pa[i] = J.pa[i]; q.pb[i] = J.pb[i]; }
+  q.partial = J.partial;
+  q.status = status;
+  lora_status_t s;
+  if (J.a_mn) {
+    if (J.na == 1 && J.nb == 2 && !J.f16) s = launch_rank_rp<true, 1, 2, false>(RP, q, J.splits, st);
+    else if (J.na == 2 && J.nb == 2 && J.f16) s = launch_rank_rp<true, 2, 2, true>(RP, q, J.splits, st);
+    else s = LORA_ERR_UNSUPPORTED;
+  } else {
+    if (J.na == 1 && J.nb == 1 && !J.f16) s = launch_rank_rp<false, 1, 1, false>(RP, q, J.splits, st);
+    else if (J.na == 2 && J.nb == 1 && J.f16) s = launch_rank_rp<false, 2, 1, true>(RP, q, J.splits, st);
+    else s = LORA_ERR_UNSUPPORTED;
+  }
+  LORA_TRY(s);
+  return reduce_partials(J.partial, J.splits, J.rows, RP, r, J.add, J.dst, J.transpose, sms, st);
+}
+
+// T_j = X A_j^T (fp32 [M x r]) by a rank pass.
+lora_status_t compute_T(const lora_linear_desc* d, const Plan& P, const void* X, const void* Aj, float* dst,
+                        uint8_t* ws, uint32_t* status, int sms, cudaStream_t st) {
+  RankJob J;
+  J.a[0] = X;
+  J.a_inner = d->d_in;
+  J.a_outer = d->M;
+  J.a_ld = d->d_in;
+  J.b[0] = Aj;
+  J.b_inner = d->d_in;
+  J.b_ld = d->d_in;
+  J.rows = static_cast<int>(d->M);
+  J.K = static_cast<int>(d->d_in);
+  J.partial = reinterpret_cast<float*>(ws + P.part_t);
+  J.splits = P.splits_t;
+  J.dst = dst;
+  return run_rank(J, P.RP, static_cast<int>(d->r), status, sms, st);
+}
 
 lora_status_t common_checks(const lora_linear_desc* d, void* ws, size_t ws_bytes, size_t need, DevInfo* dev) {
   LORA_TRY(check_desc(d));
@@ -324,7 +488,7 @@ const char* lora_status_string(lora_status_t s) {
 
 size_t lora_linear_workspace_size(const lora_linear_desc* desc, int for_backward) {
   if (check_desc(desc) != LORA_OK) return 0;
-  return for_backward ? bwd_layout(desc).total : fwd_workspace(desc);
+  return make_plan(desc, for_backward != 0).total;
 }
 
 lora_status_t lora_linear_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
@@ -350,67 +514,101 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
                               float* Z_save, void* workspace, size_t workspace_bytes, void* stream) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
-  const int np = swiglu ? 2 : 1;
   if (X == nullptr || W == nullptr || Y == nullptr) return LORA_ERR_INVALID_ARG;
   if (d->r > 0 && (A == nullptr || B == nullptr)) return LORA_ERR_INVALID_ARG;
   if (swiglu && (W_up == nullptr || (d->r > 0 && (A_up == nullptr || B_up == nullptr)))) return LORA_ERR_INVALID_ARG;
   const void* ptrs[] = {X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
+  const Plan P = make_plan(d, false);
   DevInfo dev;
-  LORA_TRY(common_checks(d, workspace, workspace_bytes, fwd_workspace(d), &dev));
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
   if (d->M == 0) return LORA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  const int RP = rank_pad(d->r);
+  const int np = P.np, RP = P.RP;
+  const int64_t M = d->M, r = d->r;
 
-  if (d->M <= kSmallMMax && d->r > 0 && !swiglu) {
-    // Memory-bound small-token path: W streamed once, no B^T copy needed.
-    return small_m_forward(d, X, W, A, B, Y, T_save, Z_save, status, dev.sms, st);
+  if (M <= kSmallMMax && r > 0 && !swiglu) {
+    // Few tokens: bound by reading W once; split K over a thread-block cluster.
+    SmallMParams q;
+    std::memset(&q, 0, sizeof(q));
+    bool ok = make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128) &&
+              make_tm(&q.tm_x, X, d->d_in, M, d->d_in, 64, 128) && make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, RP);
+    if (!ok) return LORA_ERR_CUDA;
+    const int slices = static_cast<int>(ceil_div(d->d_out, 128));
+    const int nkb = static_cast<int>(ceil_div(d->d_in, 64));
+    int S = 1;
+    while (S < 8 && slices * S * 2 <= kTargetCtas && S * 2 <= nkb) S *= 2;
+    q.B = static_cast<const __nv_bfloat16*>(B);
+    q.Y = static_cast<__nv_bfloat16*>(Y);
+    q.T_save = T_save;
+    q.Z_save = d->act == LORA_ACT_SILU ? Z_save : nullptr;
+    q.status = status;
+    q.M = static_cast<int>(M);
+    q.d_in = static_cast<int>(d->d_in);
+    q.d_out = static_cast<int>(d->d_out);
+    q.r = static_cast<int>(r);
+    q.s = d->s;
+    q.act = d->act;
+    q.splits = S;
+    q.kb_per_split = (nkb + S - 1) / S;
+    const int nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    LORA_LOG("small_m M=%d nt=%d RP=%d slices=%d splits=%d", (int)M, nt, RP, slices, S);
+    const cudaError_t e = launch_small_m(q, nt, RP, slices, st);
+    if (e != cudaSuccess) {
+      LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      return LORA_ERR_CUDA;
+    }
+    return check_launch("small_m_kernel");
   }
 
   const void* Wp[2] = {W, W_up};
   const void* Ap[2] = {A, A_up};
   const void* Bp[2] = {B, B_up};
-  void* Bt[2] = {nullptr, nullptr};
-  if (d->r > 0) {
-    size_t off = kStatusBytes;
-    for (int j = 0; j < np; ++j) {
-      Bt[j] = ws + off;
-      off += align_up(static_cast<size_t>(d->r) * d->d_out * 2, 256);
-      LORA_TRY(transpose_b(Bp[j], d->d_out, d->r, Bt[j], dev.sms, st));
+  float* T[2] = {nullptr, nullptr};
+  if (r > 0) {
+    for (int j = 0; j < np; ++j) LORA_TRY(transpose_b(Bp[j], d->d_out, r, ws + P.bt[j], false, status, dev.sms, st));
+    if (!P.rank_loop) {
+      for (int j = 0; j < np; ++j) {
+        T[j] = T_save ? T_save + static_cast<size_t>(j) * M * r : reinterpret_cast<float*>(ws + P.t_ws[j]);
+        LORA_TRY(compute_T(d, P, X, Ap[j], T[j], ws, status, dev.sms, st));
+      }
     }
   }
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int outc = swiglu ? 128 : 256;
-  bool ok = make_tm(&p.tm_a[0], X, d->d_in, d->M, d->d_in, 64, 128);
+  const bool pair = pair_kernel_enabled() && M > 128;
+  bool ok = make_tm(&p.tm_a[0], X, d->d_in, M, d->d_in, 64, 128);
   for (int j = 0; j < np; ++j) {
-    ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, swiglu ? 128 : 256);
-    if (d->r > 0) {
-      ok = ok && make_tm(&p.tm_r[j], Ap[j], d->d_in, d->r, d->d_in, 64, RP);
-      ok = ok && make_tm(&p.tm_up[j], Bt[j], d->d_out, d->r, d->d_out, 64, RP);
+    ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, (swiglu || pair) ? 128 : 256);
+    if (r > 0) {
+      if (P.rank_loop) ok = ok && make_tm(&p.tm_r[j], Ap[j], d->d_in, r, d->d_in, 64, pair ? RP / 2 : RP);
+      ok = ok && make_tm(&p.tm_up[j], ws + P.bt[j], d->d_out, r, d->d_out, 64, RP);
     }
   }
   if (!ok) return LORA_ERR_CUDA;
-  p.M = static_cast<int>(d->M);
+  p.M = static_cast<int>(M);
   p.N = static_cast<int>(d->d_out);
   p.K = static_cast<int>(d->d_in);
-  p.r = static_cast<int>(d->r);
+  p.r = static_cast<int>(r);
   p.s = d->s;
   p.out = static_cast<__nv_bfloat16*>(Y);
-  p.rank_save = d->r > 0 ? T_save : nullptr;
+  p.rank_save = (r > 0 && P.rank_loop) ? T_save : nullptr;
+  p.rank_in = T[0];   // [np][M x r]: T_save's layout, or the workspace block
   p.z_save = d->act != LORA_ACT_IDENTITY ? Z_save : nullptr;
   p.status = status;
-  p.m_tiles = static_cast<int>(ceil_div(d->M, kBM));
+  p.m_tiles = static_cast<int>(ceil_div(M, pair ? 2 * kBM : kBM));
   p.n_tiles = static_cast<int>(ceil_div(d->d_out, outc));
   p.num_tiles = p.m_tiles * p.n_tiles;
-  p.group_m = 8;
+  p.group_m = pair ? 4 : 8;
   switch (d->act) {
-    case LORA_ACT_IDENTITY: return launch_gemm_rp<false, 1, kEpiIdentity>(RP, p, dev.sms, st);
-    case LORA_ACT_SILU: return launch_gemm_rp<false, 1, kEpiSilu>(RP, p, dev.sms, st);
-    default: return launch_gemm_rp<false, 2, kEpiSwiglu>(RP, p, dev.sms, st);
+    case LORA_ACT_IDENTITY: return launch_gemm_variant<false, 1, kEpiIdentity>(RP, P.rank_loop, pair, p, dev.sms, st);
+    case LORA_ACT_SILU: return launch_gemm_variant<false, 1, kEpiSilu>(RP, P.rank_loop, pair, p, dev.sms, st);
+    default: return launch_gemm_variant<false, 2, kEpiSwiglu>(RP, P.rank_loop, pair, p, dev.sms, st);
   }
 }
 
@@ -420,7 +618,6 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
                               float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
-  const int np = swiglu ? 2 : 1;
   if (dY == nullptr || X == nullptr || W == nullptr || dX == nullptr) return LORA_ERR_INVALID_ARG;
   if (d->r > 0 && (A == nullptr || B == nullptr || dA == nullptr || dB == nullptr)) return LORA_ERR_INVALID_ARG;
   if (swiglu && (W_up == nullptr || (d->r > 0 && (A_up == nullptr || B_up == nullptr || dA_up == nullptr ||
@@ -430,10 +627,11 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   const void* ptrs[] = {dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
-  const BwdLayout L = bwd_layout(d);
+  const Plan P = make_plan(d, true);
   DevInfo dev;
-  LORA_TRY(common_checks(d, workspace, workspace_bytes, L.total, &dev));
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int np = P.np, RP = P.RP;
   float* dAp[2] = {dA, dA_up};
   float* dBp[2] = {dB, dB_up};
   if (d->M == 0) {
@@ -446,70 +644,94 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  const int RP = rank_pad(d->r);
   const int M = static_cast<int>(d->M);
   const int r = static_cast<int>(d->r);
-  const int M8 = static_cast<int>(align_up(static_cast<size_t>(M), 8));
+  const int M8 = static_cast<int>(P.M8);
+  const bool f16 = P.act_f16;
   const void* Wp[2] = {W, W_up};
   const void* Ap[2] = {A, A_up};
   const void* Bp[2] = {B, B_up};
   auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
 
-  // 1. activation backward: dZ = dY * act'(Z) as hi + lo bf16
+  // 1. dZ operands.  identity: dZ = dY (bf16, exact).  Otherwise dZ = dY * act'(Z)
+  //    as fp16 hi + lo, and fp16 copies of W for the dX product.
   const void* dZ[2] = {dY, nullptr};
-  if (d->act != LORA_ACT_IDENTITY) {
+  const void* dZlo[2] = {nullptr, nullptr};
+  const void* Wmain[2] = {W, W_up};
+  if (f16) {
     const long long n = static_cast<long long>(M) * d->d_out;
     const int grid = grid_for(n / 8, 256, dev.sms);
-    if (swiglu) {
+    if (swiglu)
       act_bwd_kernel<true><<<grid, 256, 0, st>>>(
           static_cast<const __nv_bfloat16*>(dY), Z_save, Z_save + static_cast<size_t>(M) * d->d_out, n,
-          static_cast<__nv_bfloat16*>(at(L.dz_hi[0])), static_cast<__nv_bfloat16*>(at(L.dz_lo[0])),
-          static_cast<__nv_bfloat16*>(at(L.dz_hi[1])), static_cast<__nv_bfloat16*>(at(L.dz_lo[1])));
-    } else {
+          static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])),
+          static_cast<__half*>(at(P.dz_hi[1])), static_cast<__half*>(at(P.dz_lo[1])), status);
+    else
       act_bwd_kernel<false><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dY), Z_save, nullptr, n,
-                                                  static_cast<__nv_bfloat16*>(at(L.dz_hi[0])),
-                                                  static_cast<__nv_bfloat16*>(at(L.dz_lo[0])), nullptr, nullptr);
-    }
+                                                  static_cast<__half*>(at(P.dz_hi[0])),
+                                                  static_cast<__half*>(at(P.dz_lo[0])), nullptr, nullptr, status);
     LORA_TRY(check_launch("act_bwd_kernel"));
-    for (int j = 0; j < np; ++j) dZ[j] = at(L.dz_hi[j]);
+    const long long nw = static_cast<long long>(d->d_out) * d->d_in;
+    for (int j = 0; j < np; ++j) {
+      dZ[j] = at(P.dz_hi[j]);
+      dZlo[j] = at(P.dz_lo[j]);
+      convert_f16_kernel<<<grid_for(nw / 8, 256, dev.sms), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<__half*>(at(P.w16[j])), nw, status);
+      LORA_TRY(check_launch("convert_f16_kernel"));
+      Wmain[j] = at(P.w16[j]);
+    }
   }
 
-  // 2. B^T and T (saved or recomputed) as s*T split into hi + lo, transposed
+  // 2. B^T (in the dZ operand type); T (saved or recomputed) as s*T hi + lo, transposed.
+  float* U = r > 0 ? static_cast<float*>(at(P.u_ws)) : nullptr;   // [np][M x r]
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
-      LORA_TRY(transpose_b(Bp[j], d->d_out, r, at(L.bt[j]), dev.sms, st));
+      LORA_TRY(transpose_b(Bp[j], d->d_out, r, at(P.bt[j]), f16, status, dev.sms, st));
       const float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r : nullptr;
       if (Tj == nullptr) {
-        RankGemmParams q;
-        std::memset(&q, 0, sizeof(q));
-        bool ok = make_tm(&q.tm_a[0], X, d->d_in, M, d->d_in, 64, 128) &&
-                  make_tm(&q.tm_b[0], Ap[j], d->d_in, r, d->d_in, 64, RP);
-        if (!ok) return LORA_ERR_CUDA;
-        q.rows = M;
-        q.K = static_cast<int>(d->d_in);
-        q.m_tiles = static_cast<int>(ceil_div(M, 128));
-        q.kb_per_split = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), L.splits_t));
-        q.partial = static_cast<float*>(at(L.part_u));
-        q.status = status;
-        LORA_TRY(launch_rank_rp<false, 1>(RP, q, L.splits_t, st));
-        LORA_TRY(reduce_partials(q.partial, L.splits_t, M, RP, r, nullptr, static_cast<float*>(at(L.tw[j])), 0,
-                                 dev.sms, st));
-        Tj = static_cast<const float*>(at(L.tw[j]));
+        LORA_TRY(compute_T(d, P, X, Ap[j], static_cast<float*>(at(P.t_ws[j])), ws, status, dev.sms, st));
+        Tj = static_cast<const float*>(at(P.t_ws[j]));
       }
-      LORA_TRY(rank_split_t(Tj, M, r, d->s, at(L.tt_hi[j]), at(L.tt_lo[j]), M8, dev.sms, st));
+      LORA_TRY(rank_split_t(Tj, M, r, d->s, at(P.tt_hi[j]), at(P.tt_lo[j]), M8, f16, status, dev.sms, st));
+    }
+    // 3. U = dZ B by a rank pass unless it rides the dX K-loop.
+    if (!P.rank_loop) {
+      for (int j = 0; j < np; ++j) {
+        RankJob J;
+        J.f16 = f16;
+        J.a[0] = dZ[j];
+        J.a[1] = dZlo[j];
+        J.na = f16 ? 2 : 1;
+        J.npairs = f16 ? 2 : 1;
+        J.pa[1] = 1;   // dZ_lo B
+        J.a_inner = d->d_out;
+        J.a_outer = M;
+        J.a_ld = d->d_out;
+        J.b[0] = at(P.bt[j]);
+        J.b_inner = d->d_out;
+        J.b_ld = d->d_out;
+        J.rows = M;
+        J.K = static_cast<int>(d->d_out);
+        J.partial = static_cast<float*>(at(P.part_u));
+        J.splits = P.splits_u;
+        J.dst = U + static_cast<size_t>(j) * M * r;
+        LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
+      }
     }
   }
 
-  // 3. dX = dZ W + s U A with U = dZ B (U saved for dA)
+  // 4. dX = dZ W + s U A
   {
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
+    const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
     for (int j = 0; j < np; ++j) {
-      ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128);
-      ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, 64);
+      ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
+      ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_in, d->d_out, d->d_in, 64, 64, f16);
       if (r > 0) {
-        ok = ok && make_tm(&p.tm_r[j], at(L.bt[j]), d->d_out, r, d->d_out, 64, RP);
+        if (P.rank_loop)
+          ok = ok && make_tm(&p.tm_r[j], at(P.bt[j]), d->d_out, r, d->d_out, 64, pair ? RP / 2 : RP, f16);
         ok = ok && make_tm(&p.tm_up[j], Ap[j], d->d_in, r, d->d_in, 64, RP);
       }
     }
@@ -520,76 +742,76 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     p.r = r;
     p.s = d->s;
     p.out = static_cast<__nv_bfloat16*>(dX);
-    p.rank_save = r > 0 ? static_cast<float*>(at(L.uw)) : nullptr;
-    p.z_save = nullptr;
+    p.rank_save = (r > 0 && P.rank_loop) ? U : nullptr;
+    p.rank_in = (r > 0 && !P.rank_loop) ? U : nullptr;
     p.status = status;
-    p.m_tiles = static_cast<int>(ceil_div(M, kBM));
+    p.m_tiles = static_cast<int>(ceil_div(M, pair ? 2 * kBM : kBM));
     p.n_tiles = static_cast<int>(ceil_div(d->d_in, 256));
     p.num_tiles = p.m_tiles * p.n_tiles;
-    p.group_m = 8;
-    if (swiglu) LORA_TRY((launch_gemm_rp<true, 2, kEpiGrad>(RP, p, dev.sms, st)));
-    else LORA_TRY((launch_gemm_rp<true, 1, kEpiGrad>(RP, p, dev.sms, st)));
+    p.group_m = pair ? 4 : 8;
+    if (f16) {
+      if (np == 2) LORA_TRY((launch_gemm_variant<true, 2, kEpiGradF16>(RP, P.rank_loop, pair, p, dev.sms, st)));
+      else LORA_TRY((launch_gemm_variant<true, 1, kEpiGradF16>(RP, P.rank_loop, pair, p, dev.sms, st)));
+    } else {
+      LORA_TRY((launch_gemm_variant<true, 1, kEpiGrad>(RP, P.rank_loop, pair, p, dev.sms, st)));
+    }
   }
   if (r == 0) return LORA_OK;
 
   for (int j = 0; j < np; ++j) {
-    // U for pair j lives right after pair j-1's (the kernel saves [npair][M x r]).
-    float* Uj = static_cast<float*>(at(L.uw)) + static_cast<size_t>(j) * M * r;
-    // 4. act != identity: add the dZ_lo B part of U
-    if (d->act != LORA_ACT_IDENTITY) {
-      RankGemmParams q;
-      std::memset(&q, 0, sizeof(q));
-      bool ok = make_tm(&q.tm_a[0], at(L.dz_lo[j]), d->d_out, M, d->d_out, 64, 128) &&
-                make_tm(&q.tm_b[0], at(L.bt[j]), d->d_out, r, d->d_out, 64, RP);
-      if (!ok) return LORA_ERR_CUDA;
-      q.rows = M;
-      q.K = static_cast<int>(d->d_out);
-      q.m_tiles = static_cast<int>(ceil_div(M, 128));
-      q.kb_per_split = static_cast<int>(ceil_div(ceil_div(d->d_out, 64), L.splits_u));
-      q.partial = static_cast<float*>(at(L.part_u));
-      q.status = status;
-      LORA_TRY(launch_rank_rp<false, 1>(RP, q, L.splits_u, st));
-      LORA_TRY(reduce_partials(q.partial, L.splits_u, M, RP, r, Uj, Uj, 0, dev.sms, st));
-    }
-    // 5. s U as hi + lo, transposed
-    LORA_TRY(rank_split_t(Uj, M, r, d->s, at(L.ut_hi[j]), at(L.ut_lo[j]), M8, dev.sms, st));
+    float* Uj = U + static_cast<size_t>(j) * M * r;
+    // 5. s U as bf16 hi + lo, transposed
+    LORA_TRY(rank_split_t(Uj, M, r, d->s, at(P.ut_hi[j]), at(P.ut_lo[j]), M8, false, status, dev.sms, st));
     // 6. dA^T = X^T (s U)
     {
-      RankGemmParams q;
-      std::memset(&q, 0, sizeof(q));
-      bool ok = make_tm(&q.tm_a[0], X, d->d_in, M, d->d_in, 64, 64) &&
-                make_tm(&q.tm_b[0], at(L.ut_hi[j]), M, r, M8, 64, RP) &&
-                make_tm(&q.tm_b[1], at(L.ut_lo[j]), M, r, M8, 64, RP);
-      if (!ok) return LORA_ERR_CUDA;
-      q.rows = static_cast<int>(d->d_in);
-      q.K = M;
-      q.m_tiles = static_cast<int>(ceil_div(d->d_in, 128));
-      q.kb_per_split = static_cast<int>(ceil_div(ceil_div(M, 64), L.splits_a));
-      q.partial = static_cast<float*>(at(L.part_a));
-      q.status = status;
-      LORA_TRY(launch_rank_rp<true, 2>(RP, q, L.splits_a, st));
-      LORA_TRY(reduce_partials(q.partial, L.splits_a, static_cast<int>(d->d_in), RP, r, nullptr, dAp[j], 1, dev.sms,
-                               st));
+      RankJob J;
+      J.a_mn = true;
+      J.a[0] = X;
+      J.a_inner = d->d_in;
+      J.a_outer = M;
+      J.a_ld = d->d_in;
+      J.b[0] = at(P.ut_hi[j]);
+      J.b[1] = at(P.ut_lo[j]);
+      J.nb = 2;
+      J.b_inner = M;
+      J.b_ld = M8;
+      J.npairs = 2;
+      J.pb[1] = 1;
+      J.rows = static_cast<int>(d->d_in);
+      J.K = M;
+      J.partial = static_cast<float*>(at(P.part_a));
+      J.splits = P.splits_a;
+      J.dst = dAp[j];
+      J.transpose = 1;
+      LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
     }
     // 7. dB = dZ^T (s T)
     {
-      RankGemmParams q;
-      std::memset(&q, 0, sizeof(q));
-      bool ok = make_tm(&q.tm_a[0], dZ[j], d->d_out, M, d->d_out, 64, 64) &&
-                make_tm(&q.tm_b[0], at(L.tt_hi[j]), M, r, M8, 64, RP) &&
-                make_tm(&q.tm_b[1], at(L.tt_lo[j]), M, r, M8, 64, RP);
-      if (d->act != LORA_ACT_IDENTITY) ok = ok && make_tm(&q.tm_a[1], at(L.dz_lo[j]), d->d_out, M, d->d_out, 64, 64);
-      if (!ok) return LORA_ERR_CUDA;
-      q.rows = static_cast<int>(d->d_out);
-      q.K = M;
-      q.m_tiles = static_cast<int>(ceil_div(d->d_out, 128));
-      q.kb_per_split = static_cast<int>(ceil_div(ceil_div(M, 64), L.splits_b));
-      q.partial = static_cast<float*>(at(L.part_b));
-      q.status = status;
-      if (d->act == LORA_ACT_IDENTITY) LORA_TRY((launch_rank_rp<true, 2>(RP, q, L.splits_b, st)));
-      else LORA_TRY((launch_rank_rp<true, 3>(RP, q, L.splits_b, st)));
-      LORA_TRY(reduce_partials(q.partial, L.splits_b, static_cast<int>(d->d_out), RP, r, nullptr, dBp[j], 0,
-                               dev.sms, st));
+      RankJob J;
+      J.a_mn = true;
+      J.f16 = f16;
+      J.a[0] = dZ[j];
+      J.a[1] = dZlo[j];
+      J.na = f16 ? 2 : 1;
+      J.a_inner = d->d_out;
+      J.a_outer = M;
+      J.a_ld = d->d_out;
+      J.b[0] = at(P.tt_hi[j]);
+      J.b[1] = at(P.tt_lo[j]);
+      J.nb = 2;
+      J.b_inner = M;
+      J.b_ld = M8;
+      // dZ_hi (T_hi + T_lo) [+ dZ_lo T_hi]
+      J.npairs = f16 ? 3 : 2;
+      J.pb[1] = 1;
+      J.pa[2] = 1;
+      J.pb[2] = 0;
+      J.rows = static_cast<int>(d->d_out);
+      J.K = M;
+      J.partial = static_cast<float*>(at(P.part_b));
+      J.splits = P.splits_b;
+      J.dst = dBp[j];
+      LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
     }
   }
   return LORA_OK;

@@ -14,6 +14,8 @@
 // the activation backward dZ = dY * act'(Z) as hi/lo bf16.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace lora {
@@ -27,20 +29,17 @@ struct RankGemmParams {
   int K;             // reduction length
   int m_tiles;
   int kb_per_split;
+  int npairs;        // products accumulated: sum over q < npairs of A[pa[q]] * B[pb[q]]
+  int pa[4], pb[4];
   float* partial;    // [splits][m_tiles*128][RP] fp32
   uint32_t* status;
 };
 
-// Pair table: which A and B operand each accumulated product uses.
-//   kPairs == 1: A0 B0          kPairs == 2: A0 B0 + A0 B1
-//   kPairs == 3: A0 B0 + A0 B1 + A1 B0
-template <int kPairs> __device__ __forceinline__ int pair_a(int p) { return (kPairs == 3 && p == 2) ? 1 : 0; }
-template <int kPairs> __device__ __forceinline__ int pair_b(int p) { return (p == 1) ? 1 : 0; }
-
-template <bool kAMN, int kRP, int kPairs>
+// kNA / kNB: number of distinct A / B operand tiles per stage (1 or 2).
+template <bool kAMN, int kRP, int NA, int NB, bool kF16>
 struct RankCfg {
-  static constexpr int kNA = (kPairs == 3) ? 2 : 1;
-  static constexpr int kNB = (kPairs >= 2) ? 2 : 1;
+  static constexpr int kNA = NA;
+  static constexpr int kNB = NB;
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBBytes = kRP * 128;
   static constexpr int kStageBytes = kNA * kABytes + kNB * kBBytes;
@@ -50,9 +49,9 @@ struct RankCfg {
   static constexpr uint32_t kTmemCols = kRP < 32 ? 32 : kRP;
 };
 
-template <bool kAMN, int kRP, int kPairs>
+template <bool kAMN, int kRP, int kNA, int kNB, bool kF16>
 __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid_constant__ RankGemmParams p) {
-  using C = RankCfg<kAMN, kRP, kPairs>;
+  using C = RankCfg<kAMN, kRP, kNA, kNB, kF16>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -117,7 +116,7 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
     }
   } else if (warp == 1) {
     if (lane == 0 && nkb > 0) {
-      constexpr uint32_t kId = idesc_bf16(128, kRP, kAMN, false);
+      constexpr uint32_t kId = idesc_mma(128, kRP, kAMN, false, kF16);
       RingPos rp;
       bool ok = true;
       for (int i = 0; i < nkb; ++i) {
@@ -126,10 +125,9 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
         const uint32_t st = smem_u32(smem + rp.stage * C::kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-          for (int pp = 0; pp < kPairs; ++pp) {
-            const uint32_t sa = st + pair_a<kPairs>(pp) * C::kABytes;
-            const uint32_t sb = st + C::kNA * C::kABytes + pair_b<kPairs>(pp) * C::kBBytes;
+          for (int pp = 0; pp < p.npairs; ++pp) {
+            const uint32_t sa = st + p.pa[pp] * C::kABytes;
+            const uint32_t sb = st + C::kNA * C::kABytes + p.pb[pp] * C::kBBytes;
             const uint64_t da = kAMN ? sdesc_sw128(sa + kk * 2048, 8192, 1024) : sdesc_sw128(sa + kk * 32, 16, 1024);
             const uint64_t db = sdesc_sw128(sb + kk * 32, 16, 1024);
             mma_bf16(tbase, da, db, kId, (i == 0 && kk == 0 && pp == 0) ? 0u : 1u);
@@ -193,32 +191,73 @@ __global__ void reduce_partials_kernel(const float* __restrict__ partial, int sp
   }
 }
 
-// src fp32 [M x r] -> hi, lo bf16 [r x ld] with v = scale * src, hi = bf16(v),
-// lo = bf16(v - hi).  Columns M..ld-1 are left untouched (never read).
-__global__ void rank_split_t_kernel(const float* __restrict__ src, int M, int r, float scale,
-                                    __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo, int ld) {
+// Rounding of an fp32 value to the 16-bit operand type T (bf16 or fp16).
+template <typename T> __device__ __forceinline__ T to16(float v);
+template <> __device__ __forceinline__ __nv_bfloat16 to16<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ __half to16<__half>(float v) { return __float2half_rn(v); }
+__device__ __forceinline__ float from16(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float from16(__half v) { return __half2float(v); }
+constexpr float kF16Max = 65504.0f;
+
+// src fp32 [M x r] -> hi, lo [r x ld] (bf16 or fp16) with v = scale * src,
+// hi = round(v), lo = round(v - hi).  Columns M..ld-1 are never read.
+template <typename T>
+__global__ void rank_split_t_kernel(const float* __restrict__ src, int M, int r, float scale, T* __restrict__ hi,
+                                    T* __restrict__ lo, int ld, uint32_t* status) {
   const long long n = static_cast<long long>(M) * r;
+  bool bad = false;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(i / M);
     const int m = static_cast<int>(i % M);
     const float v = scale * src[static_cast<size_t>(m) * r + c];
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const T h = to16<T>(v);
     hi[static_cast<size_t>(c) * ld + m] = h;
-    lo[static_cast<size_t>(c) * ld + m] = __float2bfloat16_rn(v - __bfloat162float(h));
+    lo[static_cast<size_t>(c) * ld + m] = to16<T>(v - from16(h));
+    if (sizeof(T) == 2 && !std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
   }
+  if (bad && status) atomicOr(status, kStatusF16Range);
 }
 
-// B [d_out x r] -> B^T [r x d_out] (bf16, exact).
-__global__ void transpose_b_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r,
-                                   __nv_bfloat16* __restrict__ Bt) {
+// B [d_out x r] (bf16) -> B^T [r x d_out] in T (exact for bf16; for fp16 exact
+// inside fp16's normal range, values beyond it flag the status word).
+template <typename T>
+__global__ void transpose_b_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r, T* __restrict__ Bt,
+                                   uint32_t* status) {
   const long long n = static_cast<long long>(d_out) * r;
+  bool bad = false;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(i / d_out);
     const int j = static_cast<int>(i % d_out);
-    Bt[i] = B[static_cast<size_t>(j) * r + c];
+    const float v = __bfloat162float(B[static_cast<size_t>(j) * r + c]);
+    Bt[i] = to16<T>(v);
+    if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
   }
+  if (bad && status) atomicOr(status, kStatusF16Range);
+}
+
+// bf16 -> fp16 copy of a weight matrix, 8 elements per step.  bf16's 8-bit
+// significand fits fp16's 11 bits, so values inside fp16's normal range
+// convert exactly; |w| > 65504 flags the status word.
+__global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, long long n,
+                                   uint32_t* status) {
+  const long long nv = n / 8;
+  bool bad = false;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+    __align__(16) __half h[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float f = __bfloat162float(b[e]);
+      h[e] = __float2half_rn(f);
+      if (!(fabsf(f) <= kF16Max)) bad = true;
+    }
+    reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(h);
+  }
+  if (bad && status) atomicOr(status, kStatusF16Range);
 }
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
@@ -226,12 +265,15 @@ __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf
 // Activation backward, 8 elements per thread-iteration (16-byte vectors).
 //   SiLU:   dZ = dY * s(z) (1 + z (1 - s(z)))
 //   SwiGLU: dZ_gate = dY * u * SiLU'(g),  dZ_up = dY * SiLU(g)
-// Each dZ is emitted as bf16 hi + bf16 lo (lo = bf16(dZ - hi)).
+// Each dZ is emitted as fp16 hi + fp16 lo (lo = fp16(dZ - hi)): fp16's 11-bit
+// significand keeps dX's rounding error well inside the tolerance, and hi + lo
+// carries about 22 bits for U and dB.
 template <bool kSwiglu>
 __global__ void act_bwd_kernel(const __nv_bfloat16* __restrict__ dY, const float* __restrict__ Z,
-                               const float* __restrict__ Zup, long long n, __nv_bfloat16* __restrict__ g_hi,
-                               __nv_bfloat16* __restrict__ g_lo, __nv_bfloat16* __restrict__ u_hi,
-                               __nv_bfloat16* __restrict__ u_lo) {
+                               const float* __restrict__ Zup, long long n, __half* __restrict__ g_hi,
+                               __half* __restrict__ g_lo, __half* __restrict__ u_hi, __half* __restrict__ u_lo,
+                               uint32_t* status) {
+  bool bad = false;
   const long long nv = n / 8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -247,7 +289,7 @@ __global__ void act_bwd_kernel(const __nv_bfloat16* __restrict__ dY, const float
       uu[0] = u0.x; uu[1] = u0.y; uu[2] = u0.z; uu[3] = u0.w;
       uu[4] = u1.x; uu[5] = u1.y; uu[6] = u1.z; uu[7] = u1.w;
     }
-    __align__(16) __nv_bfloat16 gh[8], gl[8], uh[8], ul[8];
+    __align__(16) __half gh[8], gl[8], uh[8], ul[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float dy = __bfloat162float(dyb[e]);
@@ -258,13 +300,15 @@ __global__ void act_bwd_kernel(const __nv_bfloat16* __restrict__ dY, const float
       if constexpr (kSwiglu) {
         dg = dy * uu[e] * dsilu;
         const float du = dy * (z * sg);
-        uh[e] = __float2bfloat16_rn(du);
-        ul[e] = __float2bfloat16_rn(du - __bfloat162float(uh[e]));
+        uh[e] = __float2half_rn(du);
+        ul[e] = __float2half_rn(du - __half2float(uh[e]));
+        if (!(fabsf(du) <= kF16Max)) bad = true;
       } else {
         dg = dy * dsilu;
       }
-      gh[e] = __float2bfloat16_rn(dg);
-      gl[e] = __float2bfloat16_rn(dg - __bfloat162float(gh[e]));
+      gh[e] = __float2half_rn(dg);
+      gl[e] = __float2half_rn(dg - __half2float(gh[e]));
+      if (!(fabsf(dg) <= kF16Max)) bad = true;
     }
     reinterpret_cast<uint4*>(g_hi)[i] = *reinterpret_cast<uint4*>(gh);
     reinterpret_cast<uint4*>(g_lo)[i] = *reinterpret_cast<uint4*>(gl);
@@ -273,6 +317,7 @@ __global__ void act_bwd_kernel(const __nv_bfloat16* __restrict__ dY, const float
       reinterpret_cast<uint4*>(u_lo)[i] = *reinterpret_cast<uint4*>(ul);
     }
   }
+  if (bad && status) atomicOr(status, kStatusF16Range);
 }
 
 }  // namespace lora

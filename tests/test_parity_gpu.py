@@ -22,6 +22,11 @@ CASES = [
     (256, 512, 520, 64, 16.0, "swiglu"),
     (1, 256, 256, 8, 16.0, "identity"),         # single token
     (17, 264, 1032, 24, 16.0, "identity"),      # r not a power of two
+    # few tokens: the cluster split-K forward (W streamed once)
+    (5, 256, 264, 8, 16.0, "identity"),
+    (33, 512, 1032, 16, 16.0, "silu"),
+    (64, 768, 520, 64, 16.0, "identity"),
+    (16, 1024, 384, 32, 16.0, "identity"),
 ]
 
 
