@@ -12,8 +12,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "lora_gemm.cuh"
-#include "lora_gemm2.cuh"
+#include "lora_mma.cuh"
 #include "lora_rank.cuh"
 #include "lora_small_m.cuh"
 
@@ -125,12 +124,12 @@ struct Plan {
   int np = 1;          // projections: 2 for SwiGLU (gate, up)
   int RP = 0;          // r padded to the MMA granule (0, 16, 32, 64)
   bool act_f16 = false;  // backward with an activation: fp16 dZ operands
-  bool rank_loop = false;  // rank columns inside the GEMM K-loop
   int64_t M8 = 8;
   // split-K widths of the rank passes
   int splits_t = 1, splits_u = 1, splits_a = 1, splits_b = 1;
   // regions
   size_t bt[2] = {}, t_ws[2] = {}, part_t = 0;                 // forward + backward
+  size_t s16[2] = {};                                          // bf16 s*T (fwd) / s*U (bwd) [M x r]
   size_t u_ws = 0, tt_hi[2] = {}, tt_lo[2] = {}, ut_hi[2] = {}, ut_lo[2] = {};
   size_t dz_hi[2] = {}, dz_lo[2] = {}, w16[2] = {};
   size_t part_u = 0, part_a = 0, part_b = 0;
@@ -151,9 +150,9 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
   P.np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
   P.RP = rank_pad(d->r);
   P.act_f16 = backward && d->act != LORA_ACT_IDENTITY;
-  // The K-loop rank columns cost RP/256 of the tile's tensor work: worth it
-  // for RP = 16 (X or dY read once); a separate rank pass is cheaper above.
-  P.rank_loop = d->r > 0 && P.RP == 16 && !P.act_f16 && d->act != LORA_ACT_SWIGLU;
+  // The LoRA branch rides the GEMM's K-loop as extra K-blocks fed by a rank
+  // pass (T = X A^T, U = dZ B computed once per token): no rank columns in
+  // tensor memory, which then holds two accumulator buffers.
   P.M8 = static_cast<int64_t>(align_up(static_cast<size_t>(d->M > 0 ? d->M : 1), 8));
   const int64_t M = d->M, r = d->r;
   const int64_t tiles_m = ceil_div(M > 0 ? M : 1, 128);
@@ -164,9 +163,11 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     return o;
   };
   if (r > 0) {
-    for (int j = 0; j < P.np; ++j) P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
+    if (backward)
+      for (int j = 0; j < P.np; ++j) P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
+    for (int j = 0; j < P.np; ++j) P.s16[j] = take(static_cast<size_t>(M) * r * 2);
     P.splits_t = rank_splits(tiles_m, ceil_div(d->d_in, 64));
-    const bool need_t = backward || !P.rank_loop;
+    const bool need_t = true;
     if (need_t) {
       // T of all projections is one [np][M x r] block (the GEMM reads it that way).
       P.t_ws[0] = take(static_cast<size_t>(P.np) * M * r * 4);
@@ -234,95 +235,6 @@ lora_status_t check_launch(const char* what) {
 // ---------------------------------------------------------------------------
 // kernel launchers
 // ---------------------------------------------------------------------------
-template <bool kBwd, int kRP, int kNPair, int kEpi, bool kRankGlobal>
-lora_status_t launch_gemm(const GemmParams& p, int sms, cudaStream_t st) {
-  using C = GemmCfg<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
-  auto k = lora_gemm_kernel<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-    return cuda_error("cudaFuncSetAttribute(gemm)");
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  LORA_LOG("gemm bwd=%d RP=%d npair=%d epi=%d global=%d tiles=%d grid=%d smem=%d stages=%d", (int)kBwd, kRP,
-           kNPair, kEpi, (int)kRankGlobal, p.num_tiles, grid, C::kSmemBytes, C::kStages);
-  k<<<grid, kGemmThreads, C::kSmemBytes, st>>>(p);
-  return check_launch("lora_gemm_kernel");
-}
-
-// CTA-pair variant (tcgen05 cta_group::2, 256 x 256 tiles): launched as
-// clusters of two CTAs.  p.m_tiles counts 256-row tiles.
-template <bool kBwd, int kRP, int kNPair, int kEpi, bool kRankGlobal>
-lora_status_t launch_gemm2(const GemmParams& p, int sms, cudaStream_t st) {
-  using C = Gemm2Cfg<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
-  auto k = lora_gemm2_kernel<kBwd, kRP, kNPair, kEpi, kRankGlobal>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-    return cuda_error("cudaFuncSetAttribute(gemm2)");
-  const int clusters = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  LORA_LOG("gemm2 bwd=%d RP=%d npair=%d epi=%d global=%d tiles=%d clusters=%d smem=%d stages=%d", (int)kBwd, kRP,
-           kNPair, kEpi, (int)kRankGlobal, p.num_tiles, clusters, C::kSmemBytes, C::kStages);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, p);
-  if (e != cudaSuccess) {
-    LORA_LOG("gemm2 launch: %s", cudaGetErrorString(e));
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return LORA_ERR_CUDA;
-  }
-  return check_launch("lora_gemm2_kernel");
-}
-
-bool pair_kernel_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = std::getenv("LORA_LINEAR_PAIR");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
-}
-
-// Instantiated variants: r = 0; RP = 16 with the rank columns in the K-loop;
-// RP in {16, 32, 64} with the rank columns from a rank pass.  `pair` selects
-// the CTA-pair kernel (p already tiled for it).
-template <bool kBwd, int kNPair, int kEpi>
-lora_status_t launch_gemm_variant(int RP, bool rank_loop, bool pair, const GemmParams& p, int sms, cudaStream_t st) {
-  if (pair) {
-    if (RP == 0) return launch_gemm2<kBwd, 0, kNPair, kEpi, true>(p, sms, st);
-    if (rank_loop) {
-      if constexpr (kNPair == 1 && kEpi != kEpiSwiglu && kEpi != kEpiGradF16) {
-        if (RP == 16) return launch_gemm2<kBwd, 16, kNPair, kEpi, false>(p, sms, st);
-      }
-      return LORA_ERR_UNSUPPORTED;
-    }
-    switch (RP) {
-      case 16: return launch_gemm2<kBwd, 16, kNPair, kEpi, true>(p, sms, st);
-      case 32: return launch_gemm2<kBwd, 32, kNPair, kEpi, true>(p, sms, st);
-      case 64: return launch_gemm2<kBwd, 64, kNPair, kEpi, true>(p, sms, st);
-      default: return LORA_ERR_UNSUPPORTED;
-    }
-  }
-  if (RP == 0) return launch_gemm<kBwd, 0, kNPair, kEpi, true>(p, sms, st);
-  if (rank_loop) {
-    if constexpr (kNPair == 1 && kEpi != kEpiSwiglu && kEpi != kEpiGradF16) {
-      if (RP == 16) return launch_gemm<kBwd, 16, kNPair, kEpi, false>(p, sms, st);
-    }
-    return LORA_ERR_UNSUPPORTED;
-  }
-  switch (RP) {
-    case 16: return launch_gemm<kBwd, 16, kNPair, kEpi, true>(p, sms, st);
-    case 32: return launch_gemm<kBwd, 32, kNPair, kEpi, true>(p, sms, st);
-    case 64: return launch_gemm<kBwd, 64, kNPair, kEpi, true>(p, sms, st);
-    default: return LORA_ERR_UNSUPPORTED;
-  }
-}
-
 template <bool kAMN, int kRP, int kNA, int kNB, bool kF16>
 lora_status_t launch_rank(const RankGemmParams& p, int splits, cudaStream_t st) {
   using C = RankCfg<kAMN, kRP, kNA, kNB, kF16>;
@@ -365,11 +277,12 @@ lora_status_t transpose_b(const void* B, int64_t d_out, int64_t r, void* Bt, boo
 }
 
 lora_status_t reduce_partials(const float* part, int splits, int rows, int RP, int r, const float* add, float* dst,
-                              int transpose, int sms, cudaStream_t st) {
+                              int transpose, int sms, cudaStream_t st, void* dst16 = nullptr, float scale16 = 1.0f) {
   const long long n = static_cast<long long>(rows) * r;
   const int rows_pad = static_cast<int>(ceil_div(rows, 128) * 128);
   reduce_partials_kernel<<<grid_for(n, 256, sms), 256, 0, st>>>(part, splits, rows_pad, RP, rows, r, add, dst,
-                                                               transpose);
+                                                               transpose, static_cast<__nv_bfloat16*>(dst16),
+                                                               scale16);
   return check_launch("reduce_partials_kernel");
 }
 
@@ -402,6 +315,8 @@ struct RankJob {
   const float* add = nullptr;
   float* dst = nullptr;
   int transpose = 0;
+  void* dst16 = nullptr;     // optional bf16 copy of scale16 * dst
+  float scale16 = 1.0f;
 };
 
 lora_status_t run_rank(const RankJob& J, int RP, int r, uint32_t* status, int sms, cudaStream_t st) {
@@ -431,12 +346,13 @@ lora_status_t run_rank(const RankJob& J, int RP, int r, uint32_t* status, int sm
     else s = LORA_ERR_UNSUPPORTED;
   }
   LORA_TRY(s);
-  return reduce_partials(J.partial, J.splits, J.rows, RP, r, J.add, J.dst, J.transpose, sms, st);
+  return reduce_partials(J.partial, J.splits, J.rows, RP, r, J.add, J.dst, J.transpose, sms, st, J.dst16,
+                         J.scale16);
 }
 
-// T_j = X A_j^T (fp32 [M x r]) by a rank pass.
+// T_j = X A_j^T (fp32 [M x r]) by a rank pass; optionally also bf16(s T_j).
 lora_status_t compute_T(const lora_linear_desc* d, const Plan& P, const void* X, const void* Aj, float* dst,
-                        uint8_t* ws, uint32_t* status, int sms, cudaStream_t st) {
+                        uint8_t* ws, uint32_t* status, int sms, cudaStream_t st, void* dst16 = nullptr) {
   RankJob J;
   J.a[0] = X;
   J.a_inner = d->d_in;
@@ -450,7 +366,57 @@ lora_status_t compute_T(const lora_linear_desc* d, const Plan& P, const void* X,
   J.partial = reinterpret_cast<float*>(ws + P.part_t);
   J.splits = P.splits_t;
   J.dst = dst;
+  J.dst16 = dst16;
+  J.scale16 = d->s;
   return run_rank(J, P.RP, static_cast<int>(d->r), status, sms, st);
+}
+
+// ---------------------------------------------------------------------------
+// the LoRA GEMM (lora_mma_kernel): launch as single CTAs or CTA pairs
+// ---------------------------------------------------------------------------
+bool pair_kernel_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("LORA_LINEAR_PAIR");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+template <bool kPair, bool kBwd, int kNPair, int kEpi>
+lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
+  using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
+  auto k = lora_mma_kernel<kPair, kBwd, kNPair, kEpi>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return cuda_error("cudaFuncSetAttribute(mma)");
+  const int max_units = kPair ? sms / 2 : sms;
+  const int units = p.num_tiles < max_units ? p.num_tiles : max_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * C::kCtas), 1, 1);
+  cfg.blockDim = dim3(kMmaThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C::kCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kPair ? 1 : 0;
+  LORA_LOG("mma pair=%d bwd=%d npair=%d epi=%d tiles=%d units=%d smem=%d stages=%d lora_ksteps=%d", (int)kPair,
+           (int)kBwd, kNPair, kEpi, p.num_tiles, units, C::kSmemBytes, C::kStages, p.lora_ksteps);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, p);
+  if (e != cudaSuccess) {
+    LORA_LOG("mma launch: %s", cudaGetErrorString(e));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return LORA_ERR_CUDA;
+  }
+  return check_launch("lora_mma_kernel");
+}
+
+template <bool kBwd, int kNPair, int kEpi>
+lora_status_t launch_mma_any(bool pair, const MmaParams& p, int sms, cudaStream_t st) {
+  return pair ? launch_mma<true, kBwd, kNPair, kEpi>(p, sms, st) : launch_mma<false, kBwd, kNPair, kEpi>(p, sms, st);
 }
 
 lora_status_t common_checks(const lora_linear_desc* d, void* ws, size_t ws_bytes, size_t need, DevInfo* dev) {
@@ -568,47 +534,44 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   const void* Wp[2] = {W, W_up};
   const void* Ap[2] = {A, A_up};
   const void* Bp[2] = {B, B_up};
-  float* T[2] = {nullptr, nullptr};
+  // 1. T_j = X A_j^T (fp32, saved for the backward) and bf16(s T_j) for the LoRA K-block
   if (r > 0) {
-    for (int j = 0; j < np; ++j) LORA_TRY(transpose_b(Bp[j], d->d_out, r, ws + P.bt[j], false, status, dev.sms, st));
-    if (!P.rank_loop) {
-      for (int j = 0; j < np; ++j) {
-        T[j] = T_save ? T_save + static_cast<size_t>(j) * M * r : reinterpret_cast<float*>(ws + P.t_ws[j]);
-        LORA_TRY(compute_T(d, P, X, Ap[j], T[j], ws, status, dev.sms, st));
-      }
+    for (int j = 0; j < np; ++j) {
+      float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r
+                         : reinterpret_cast<float*>(ws + P.t_ws[0]) + static_cast<size_t>(j) * M * r;
+      LORA_TRY(compute_T(d, P, X, Ap[j], Tj, ws, status, dev.sms, st, ws + P.s16[j]));
     }
   }
-  GemmParams p;
+  // 2. Z = [X | sT] [W | B]^T, activation, bf16 Y
+  MmaParams p;
   std::memset(&p, 0, sizeof(p));
-  const int outc = swiglu ? 128 : 256;
   const bool pair = pair_kernel_enabled() && M > 128;
+  const int outc = swiglu ? 128 : 256;
+  const int brows = swiglu ? (pair ? 64 : 128) : (pair ? 128 : 256);   // N-side rows per CTA box
   bool ok = make_tm(&p.tm_a[0], X, d->d_in, M, d->d_in, 64, 128);
   for (int j = 0; j < np; ++j) {
     ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, (swiglu || pair) ? 128 : 256);
     if (r > 0) {
-      if (P.rank_loop) ok = ok && make_tm(&p.tm_r[j], Ap[j], d->d_in, r, d->d_in, 64, pair ? RP / 2 : RP);
-      ok = ok && make_tm(&p.tm_up[j], ws + P.bt[j], d->d_out, r, d->d_out, 64, RP);
+      ok = ok && make_tm(&p.tm_la[j], ws + P.s16[j], r, M, r, 64, 128);
+      ok = ok && make_tm(&p.tm_lb[j], Bp[j], r, d->d_out, r, 64, brows);
     }
   }
   if (!ok) return LORA_ERR_CUDA;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(d->d_out);
   p.K = static_cast<int>(d->d_in);
-  p.r = static_cast<int>(r);
-  p.s = d->s;
+  p.lora_ksteps = static_cast<int>((r + 15) / 16);
   p.out = static_cast<__nv_bfloat16*>(Y);
-  p.rank_save = (r > 0 && P.rank_loop) ? T_save : nullptr;
-  p.rank_in = T[0];   // [np][M x r]: T_save's layout, or the workspace block
   p.z_save = d->act != LORA_ACT_IDENTITY ? Z_save : nullptr;
   p.status = status;
-  p.m_tiles = static_cast<int>(ceil_div(M, pair ? 2 * kBM : kBM));
+  p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
   p.n_tiles = static_cast<int>(ceil_div(d->d_out, outc));
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.group_m = pair ? 4 : 8;
   switch (d->act) {
-    case LORA_ACT_IDENTITY: return launch_gemm_variant<false, 1, kEpiIdentity>(RP, P.rank_loop, pair, p, dev.sms, st);
-    case LORA_ACT_SILU: return launch_gemm_variant<false, 1, kEpiSilu>(RP, P.rank_loop, pair, p, dev.sms, st);
-    default: return launch_gemm_variant<false, 2, kEpiSwiglu>(RP, P.rank_loop, pair, p, dev.sms, st);
+    case LORA_ACT_IDENTITY: return launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st);
+    case LORA_ACT_SILU: return launch_mma_any<false, 1, kMEpiSilu>(pair, p, dev.sms, st);
+    default: return launch_mma_any<false, 2, kMEpiSwiglu>(pair, p, dev.sms, st);
   }
 }
 
@@ -694,8 +657,8 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
       }
       LORA_TRY(rank_split_t(Tj, M, r, d->s, at(P.tt_hi[j]), at(P.tt_lo[j]), M8, f16, status, dev.sms, st));
     }
-    // 3. U = dZ B by a rank pass unless it rides the dX K-loop.
-    if (!P.rank_loop) {
+    // 3. U = dZ B by a rank pass (fp32, and bf16 s U for the LoRA K-block of dX)
+    {
       for (int j = 0; j < np; ++j) {
         RankJob J;
         J.f16 = f16;
@@ -715,14 +678,16 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
         J.partial = static_cast<float*>(at(P.part_u));
         J.splits = P.splits_u;
         J.dst = U + static_cast<size_t>(j) * M * r;
+        J.dst16 = at(P.s16[j]);
+        J.scale16 = d->s;
         LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
       }
     }
   }
 
-  // 4. dX = dZ W + s U A
+  // 4. dX = [dZ | sU] [W ; A]
   {
-    GemmParams p;
+    MmaParams p;
     std::memset(&p, 0, sizeof(p));
     const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
@@ -730,30 +695,27 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
       ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
       ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_in, d->d_out, d->d_in, 64, 64, f16);
       if (r > 0) {
-        if (P.rank_loop)
-          ok = ok && make_tm(&p.tm_r[j], at(P.bt[j]), d->d_out, r, d->d_out, 64, pair ? RP / 2 : RP, f16);
-        ok = ok && make_tm(&p.tm_up[j], Ap[j], d->d_in, r, d->d_in, 64, RP);
+        ok = ok && make_tm(&p.tm_la[j], at(P.s16[j]), r, M, r, 64, 128);
+        ok = ok && make_tm(&p.tm_lb[j], Ap[j], d->d_in, r, d->d_in, 64, 64);
       }
     }
     if (!ok) return LORA_ERR_CUDA;
     p.M = M;
     p.N = static_cast<int>(d->d_in);
     p.K = static_cast<int>(d->d_out);
-    p.r = r;
-    p.s = d->s;
+    p.lora_ksteps = (r + 15) / 16;
     p.out = static_cast<__nv_bfloat16*>(dX);
-    p.rank_save = (r > 0 && P.rank_loop) ? U : nullptr;
-    p.rank_in = (r > 0 && !P.rank_loop) ? U : nullptr;
+    p.z_save = nullptr;
     p.status = status;
-    p.m_tiles = static_cast<int>(ceil_div(M, pair ? 2 * kBM : kBM));
+    p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
     p.n_tiles = static_cast<int>(ceil_div(d->d_in, 256));
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.group_m = pair ? 4 : 8;
     if (f16) {
-      if (np == 2) LORA_TRY((launch_gemm_variant<true, 2, kEpiGradF16>(RP, P.rank_loop, pair, p, dev.sms, st)));
-      else LORA_TRY((launch_gemm_variant<true, 1, kEpiGradF16>(RP, P.rank_loop, pair, p, dev.sms, st)));
+      if (np == 2) LORA_TRY((launch_mma_any<true, 2, kMEpiGradF16>(pair, p, dev.sms, st)));
+      else LORA_TRY((launch_mma_any<true, 1, kMEpiGradF16>(pair, p, dev.sms, st)));
     } else {
-      LORA_TRY((launch_gemm_variant<true, 1, kEpiGrad>(RP, P.rank_loop, pair, p, dev.sms, st)));
+      LORA_TRY((launch_mma_any<true, 1, kMEpiGrad>(pair, p, dev.sms, st)));
     }
   }
   if (r == 0) return LORA_OK;

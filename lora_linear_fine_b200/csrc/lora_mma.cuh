@@ -1,0 +1,401 @@
+// lora_mma.cuh — the fused LoRA-adapted linear layer as one tcgen05 GEMM whose
+// K-loop carries the LoRA branch as extra K-blocks:
+//
+//   forward   Z  = X W^T + s T B^T  = [ X | sT ] [ W | B ]^T      (T = X A^T)
+//   backward  dX = dZ W  + s U A    = [ dZ | sU ] [ W ; A ]       (U = dZ B)
+//
+// T (U) comes from the rank pass (lora_rank.cuh), which also writes s*T as bf16
+// [M x r]; the GEMM's last K-block(s) per tile multiply that tile of s*T (K = r,
+// zero-filled by TMA up to the 64-wide block) with the matching rows of B (A).
+// The up-projection thus runs on the tensor cores inside the same accumulator,
+// with no hand-off between the epilogue and the MMA issuer, which leaves the
+// tensor memory free for a double-buffered accumulator: 2 x 256 fp32 columns.
+// The epilogue of tile i (drain, activation, bf16 store) overlaps the K-loop of
+// tile i + 1.
+//
+// kPair = false: one CTA per 128 x 256 tile (tcgen05 cta_group::1).
+// kPair = true : a cluster of two CTAs per 256 x 256 tile (cta_group::2): CTA c
+//   holds rows [128c, 128c + 128) of the M-side operand and half of the N-side
+//   operand; the leader (c = 0) issues the MMAs; each CTA's tensor memory holds
+//   its own 128 accumulator rows.  The TMA transactions of both CTAs complete on
+//   the leader's `full` barrier; the leader's commits arrive on both CTAs'
+//   barriers; both CTAs' epilogues arrive on the leader's `acc_empty` barriers.
+//
+// SwiGLU forward: the N-side operand of a tile is 128 gate rows + 128 up rows
+// of the same outputs (paired kernel: gate in CTA 0, up in CTA 1); the LoRA
+// blocks are two N = 128 products, one per projection.  SwiGLU backward: the
+// K-loop runs through both projections (dZ_gate W_gate + dZ_up W_up + LoRA).
+//
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..9 epilogue (two warps per 32-lane TMEM quadrant).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace lora {
+
+constexpr int kMmaThreads = 320;
+
+// kEpi values
+enum MmaEpi : int { kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4 };
+
+struct MmaParams {
+  CUtensorMap tm_a[2];    // M-side operand per pair      fwd: X            bwd: dZ_j
+  CUtensorMap tm_w[2];    // N-side operand per pair      fwd: W_j (K-major) bwd: W_j (MN-major)
+  CUtensorMap tm_la[2];   // LoRA block, M side           s*T_j / s*U_j   bf16 [M x r]
+  CUtensorMap tm_lb[2];   // LoRA block, N side           fwd: B_j [d_out x r]   bwd: A_j [r x d_in]
+  int M, N, K;            // output rows / columns (per projection for SwiGLU fwd) / reduction per pair
+  int lora_ksteps;        // 16-wide K steps of the LoRA block: ceil(r / 16); 0 = no LoRA block
+  __nv_bfloat16* out;     // [M x N]
+  float* z_save;          // [npair][M x N] fp32 or null (SiLU / SwiGLU forward)
+  uint32_t* status;
+  int m_tiles, n_tiles, num_tiles, group_m;
+};
+
+template <bool kPair, bool kBwd, int kNPair, int kEpi>
+struct MmaCfg {
+  static constexpr bool kSwigluFwd = (!kBwd) && (kEpi == kMEpiSwiglu);
+  static constexpr int kCtas = kPair ? 2 : 1;
+  static constexpr int kTileM = 128 * kCtas;                 // rows per (pair) tile
+  static constexpr int kOutCols = kSwigluFwd ? 128 : 256;    // output columns per tile
+  static constexpr int kKPairs = kBwd ? kNPair : 1;          // projections walked along K
+  static constexpr int kLoraBlocks = kNPair;                 // LoRA K-blocks per tile
+  static constexpr int kABytes = 128 * 64 * 2;               // 16 KB
+  static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
+  static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages0 = (kSmemLimitBytes - 2048) / kStageBytes;
+  static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 2048;
+  static constexpr uint32_t kTmemCols = 512;                 // 2 accumulator buffers
+  static_assert(kStages >= 3, "ring too shallow");
+};
+
+__device__ __forceinline__ void mma_tile_coords(int t, const MmaParams& p, int& mt, int& nt) {
+  const int per_group = p.group_m * p.n_tiles;
+  const int g = t / per_group;
+  const int first_m = g * p.group_m;
+  const int rem = p.m_tiles - first_m;
+  const int gm = rem < p.group_m ? rem : p.group_m;
+  const int idx = t - g * per_group;
+  mt = first_m + idx % gm;
+  nt = idx / gm;
+}
+
+template <bool kPair>
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const AbortCtl& ctl) {
+  if constexpr (kPair) return mbar_wait_cluster(bar, parity, ctl);
+  else return mbar_wait(bar, parity, ctl);
+}
+
+template <bool kPair, bool kBwd, int kNPair, int kEpi>
+__global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_constant__ MmaParams p) {
+  using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
+  constexpr int S = C::kStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* full = bars;                  // [S]
+  uint64_t* empty = bars + S;             // [S]
+  uint64_t* acc_full = bars + 2 * S;      // [2] accumulator buffer b complete
+  uint64_t* acc_empty = acc_full + 2;     // [2] accumulator buffer b drained
+  uint64_t* mma_done = acc_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t crank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = crank == 0;
+  const int unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;        // scheduling unit (CTA or pair)
+  const int nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
+  AbortCtl ctl{abort_flag, p.status};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 256 * C::kCtas); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int j = 0; j < (C::kSwigluFwd ? 1 : kNPair); ++j) tma_prefetch_desc(&p.tm_a[j]);
+    for (int j = 0; j < kNPair; ++j) tma_prefetch_desc(&p.tm_w[j]);
+    if (p.lora_ksteps > 0)
+      for (int j = 0; j < kNPair; ++j) { tma_prefetch_desc(&p.tm_la[j]); tma_prefetch_desc(&p.tm_lb[j]); }
+  }
+  if (warp == 1) {
+    if constexpr (kPair) { tmem_alloc_pair(tmem_slot, C::kTmemCols); tmem_relinquish_pair(); }
+    else { tmem_alloc(tmem_slot, C::kTmemCols); tmem_relinquish(); }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (kPair) cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int nkb = (p.K + 63) / 64;
+  const int nlora = p.lora_ksteps > 0 ? C::kLoraBlocks : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = l2_policy_evict_first();
+      const uint64_t pol_keep = l2_policy_evict_last();
+      RingPos rp;
+      uint32_t issued = 0;
+      bool ok = true;
+      // One TMA box into this CTA's shared memory; completion on the stage's
+      // `full` barrier (the leader's for a pair).
+      auto load = [&](void* dst, const CUtensorMap* tm, uint32_t stage, int x, int y, uint64_t pol) {
+        if constexpr (kPair) tma_load_2d_pair(dst, tm, mapa_shared(smem_u32(&full[stage]), 0), x, y, pol);
+        else tma_load_2d_hint(dst, tm, &full[stage], x, y, pol);
+      };
+      // Bytes one stage brings into ALL CTAs of the unit: main and backward
+      // LoRA blocks fill both areas; a forward SwiGLU LoRA block fills the A
+      // area and 128 rows of N-side operand (64 per CTA of a pair).
+      constexpr uint32_t kTxFull = C::kCtas * C::kStageBytes;
+      constexpr uint32_t kTxSwigluLora = C::kCtas * C::kABytes + 128 * 64 * 2;
+      for (int t = unit; t < p.num_tiles && ok; t += nunits) {
+        int mt, nt;
+        mma_tile_coords(t, p, mt, nt);
+        const int m0 = mt * C::kTileM + 128 * static_cast<int>(crank);
+        const int n0 = nt * C::kOutCols;
+        const int nblocks = C::kKPairs * nkb + nlora;
+        for (int blk = 0; blk < nblocks; ++blk) {
+          if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* sa = smem + rp.stage * C::kStageBytes;
+          uint8_t* sb = sa + C::kABytes;
+          const uint32_t fb = rp.stage;
+          const bool lora_blk = blk >= C::kKPairs * nkb;
+          if (leader)
+            mbar_arrive_expect_tx(&full[rp.stage], (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull);
+          if (!lora_blk) {
+            // main block: projection j, K-block kb
+            const int j = blk / nkb;
+            const int k0 = (blk - j * nkb) * 64;
+            load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
+            if constexpr (!kBwd) {
+              if constexpr (C::kSwigluFwd) {
+                if constexpr (kPair) load(sb, &p.tm_w[crank], fb, k0, n0, pol_keep);
+                else {
+                  load(sb, &p.tm_w[0], fb, k0, n0, pol_keep);
+                  load(sb + C::kBBytes / 2, &p.tm_w[1], fb, k0, n0, pol_keep);
+                }
+              } else {
+                load(sb, &p.tm_w[0], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+              }
+            } else {
+#pragma unroll
+              for (int b = 0; b < C::kBRows / 64; ++b)
+                load(sb + b * 8192, &p.tm_w[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, k0, pol_keep);
+            }
+          } else {
+            // LoRA block of projection j: s*T_j (s*U_j) rows and B_j (A_j) rows, K = r zero-padded to 64
+            const int j = blk - C::kKPairs * nkb;
+            load(sa, &p.tm_la[j], fb, 0, m0, pol_keep);
+            if constexpr (!kBwd) {
+              if constexpr (C::kSwigluFwd) {
+                // N = 128 outputs of projection j: 128 rows (single) or 64 per CTA (pair)
+                load(sb, &p.tm_lb[j], fb, 0, n0 + 64 * static_cast<int>(crank), pol_keep);
+              } else {
+                load(sb, &p.tm_lb[0], fb, 0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+              }
+            } else {
+#pragma unroll
+              for (int b = 0; b < C::kBRows / 64; ++b)
+                load(sb + b * 8192, &p.tm_lb[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, 0, pol_keep);
+            }
+          }
+          ++issued;
+          rp.next(S);
+        }
+      }
+      if (!ok && leader) {
+        RingPos q = rp;
+        volatile uint32_t zero = 0u;
+        AbortCtl quiet{&zero, nullptr};
+        for (uint32_t i = 0; i < (issued < (uint32_t)S ? issued : (uint32_t)S); ++i) {
+          if (q.stage == 0) { q.stage = S - 1; q.phase ^= 1u; } else { --q.stage; }
+          wait_bar<kPair>(&full[q.stage], q.phase, quiet);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {
+      constexpr bool kF16 = (kEpi == kMEpiGradF16);
+      constexpr int kM = C::kTileM;
+      constexpr uint32_t kIdMain = idesc_mma(kM, 256, false, kBwd, kF16);
+      // LoRA block: bf16 s*T/s*U against bf16 B/A (A side K-major; B side K-major fwd, MN-major bwd)
+      constexpr uint32_t kIdLora = idesc_mma(kM, C::kSwigluFwd ? 128 : 256, false, kBwd, false);
+      constexpr uint16_t kBoth = 0x3;
+      auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (kPair) mma_bf16_pair(d, a, b, id, acc);
+        else mma_bf16(d, a, b, id, acc);
+      };
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (kPair) mma_commit_pair(bar, kBoth);
+        else mma_commit(bar);
+      };
+      RingPos rp;
+      uint32_t it = 0;
+      for (int t = unit; t < p.num_tiles; t += nunits, ++it) {
+        const uint32_t buf = it & 1u;
+        const uint32_t use = it >> 1;        // how many times this buffer was used before
+        if (!wait_bar<kPair>(&acc_empty[buf], (use & 1u) ^ 1u, ctl)) break;
+        tc_fence_after();
+        const uint32_t dacc = tbase + buf * 256;
+        const int nblocks = C::kKPairs * nkb + nlora;
+        bool ok = true;
+        for (int blk = 0; blk < nblocks; ++blk) {
+          if (!wait_bar<kPair>(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + rp.stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+          if (blk < C::kKPairs * nkb) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t db = kBwd ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
+              mma(dacc, da, db, kIdMain, (blk == 0 && kk == 0) ? 0u : 1u);
+            }
+          } else {
+            const int j = blk - C::kKPairs * nkb;
+            const uint32_t dcol = C::kSwigluFwd ? static_cast<uint32_t>(128 * j) : 0u;
+            for (int kk = 0; kk < p.lora_ksteps; ++kk) {
+              const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t db = kBwd ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
+              mma(dacc + dcol, da, db, kIdLora, 1u);
+            }
+          }
+          commit(&empty[rp.stage]);
+          rp.next(S);
+        }
+        if (!ok) break;
+        commit(&acc_full[buf]);
+      }
+      if constexpr (kPair) mma_commit_pair(mma_done, 0x1);
+      else mma_commit(mma_done);
+      volatile uint32_t zero = 0u;
+      AbortCtl quiet{&zero, nullptr};
+      wait_bar<kPair>(mma_done, 0, quiet);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                 // 0..7
+    const int q = warp & 3;                  // TMEM lane quadrant
+    const int h = ew >> 2;                   // column half
+    const int row_in_tile = q * 32 + lane;
+    uint32_t acc_empty_addr[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+      acc_empty_addr[b] = kPair ? mapa_shared(smem_u32(&acc_empty[b]), 0) : smem_u32(&acc_empty[b]);
+    uint32_t it = 0;
+    for (int t = unit; t < p.num_tiles; t += nunits, ++it) {
+      int mt, nt;
+      mma_tile_coords(t, p, mt, nt);
+      const uint32_t buf = it & 1u;
+      const uint32_t use = it >> 1;
+      const int row = mt * C::kTileM + 128 * static_cast<int>(crank) + row_in_tile;
+      const bool row_ok = row < p.M;
+      if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
+      tc_fence_after();
+      __syncwarp();   // tcgen05.ld is .sync.aligned
+      const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t v[128];
+      if constexpr (C::kSwigluFwd) {
+        tmem_ld32(tl + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tl + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld32(tl + 128 + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+        tmem_ld32(tl + 128 + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tl + h * 128 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      if constexpr (kPair) mbar_arrive_cluster(acc_empty_addr[buf]);
+      else mbar_arrive(&acc_empty[buf]);
+      if (!row_ok) continue;
+
+      if constexpr (C::kSwigluFwd) {
+        const int col0 = nt * 128 + h * 64;
+        const size_t base = static_cast<size_t>(row) * p.N + col0;
+        if (p.z_save != nullptr) {
+          float* zg = p.z_save + base;
+          float* zu = p.z_save + static_cast<size_t>(p.M) * p.N + base;
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            if (col0 + c < p.N) {
+              *reinterpret_cast<float4*>(zg + c) = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                                               __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+              *reinterpret_cast<float4*>(zu + c) =
+                  make_float4(__uint_as_float(v[64 + c]), __uint_as_float(v[65 + c]), __uint_as_float(v[66 + c]),
+                              __uint_as_float(v[67 + c]));
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          float hv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float g = __uint_as_float(v[c + e]);
+            const float u = __uint_as_float(v[64 + c + e]);
+            hv[e] = g / (1.0f + expf(-g)) * u;
+          }
+          if (col0 + c < p.N) {
+            uint4 pk;
+            pk.x = pack_bf16x2(hv[0], hv[1]);
+            pk.y = pack_bf16x2(hv[2], hv[3]);
+            pk.z = pack_bf16x2(hv[4], hv[5]);
+            pk.w = pack_bf16x2(hv[6], hv[7]);
+            *reinterpret_cast<uint4*>(p.out + base + c) = pk;
+          }
+        }
+      } else {
+        const int col0 = nt * 256 + h * 128;
+        const size_t base = static_cast<size_t>(row) * p.N + col0;
+        if constexpr (kEpi == kMEpiSilu) {
+          if (p.z_save != nullptr) {
+#pragma unroll
+            for (int c = 0; c < 128; c += 4)
+              if (col0 + c < p.N)
+                *reinterpret_cast<float4*>(p.z_save + base + c) =
+                    make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
+                                __uint_as_float(v[c + 3]));
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) {
+          float yv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float z = __uint_as_float(v[c + e]);
+            yv[e] = (kEpi == kMEpiSilu) ? z / (1.0f + expf(-z)) : z;
+          }
+          if (col0 + c < p.N) {
+            uint4 pk;
+            pk.x = pack_bf16x2(yv[0], yv[1]);
+            pk.y = pack_bf16x2(yv[2], yv[3]);
+            pk.z = pack_bf16x2(yv[4], yv[5]);
+            pk.w = pack_bf16x2(yv[6], yv[7]);
+            *reinterpret_cast<uint4*>(p.out + base + c) = pk;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (kPair) cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    if constexpr (kPair) tmem_dealloc_pair(tbase, C::kTmemCols);
+    else tmem_dealloc(tbase, C::kTmemCols);
+  }
+}
+
+}  // namespace lora

@@ -176,9 +176,10 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
 
 // dst = sum over splits of partial[sp][row][c] (+ add[row][c]); fixed order.
 // transpose == 0: dst[row * r + c];  transpose == 1: dst[c * rows + row].
+// dst16 (optional, transpose == 0 only): bf16(scale16 * dst) in the same layout.
 __global__ void reduce_partials_kernel(const float* __restrict__ partial, int splits, int rows_pad, int RP,
                                        int rows, int r, const float* __restrict__ add, float* __restrict__ dst,
-                                       int transpose) {
+                                       int transpose, __nv_bfloat16* __restrict__ dst16, float scale16) {
   const long long n = static_cast<long long>(rows) * r;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -188,6 +189,7 @@ __global__ void reduce_partials_kernel(const float* __restrict__ partial, int sp
     float acc = add ? add[static_cast<size_t>(row) * r + c] : 0.0f;
     for (int sp = 0; sp < splits; ++sp) acc += partial[(static_cast<size_t>(sp) * rows_pad + row) * RP + c];
     dst[i] = acc;
+    if (dst16 != nullptr) dst16[i] = __float2bfloat16_rn(scale16 * acc);
   }
 }
 
