@@ -145,6 +145,33 @@ int lora_linear_abi_version(void);
  * (all devices, all threads).  For accounting in benchmarks and tests. */
 uint64_t lora_linear_launch_count(void);
 
+/* Forward without a workspace argument, for callers that cannot allocate
+ * device memory: for example a plug-in inside a host application that owns
+ * every device allocation through its own pool and forbids direct cudaMalloc,
+ * or a latency-critical caller that must not pay for cudaMalloc's implicit
+ * synchronisation.  The pages describe no such variant; it has no counterpart
+ * there.
+ *
+ * Same arguments, results and errors as lora_linear_fwd, minus the workspace:
+ * the scratch memory lives in a file-scope device array of
+ * LORA_LINEAR_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU loading this
+ * library holds until the process exits.  Nothing is allocated by this call.
+ * - A problem whose forward workspace (lora_linear_workspace_size(desc, 0))
+ *   exceeds that size is rejected with LORA_ERR_UNSUPPORTED before anything
+ *   runs.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Every call, on every stream, shares the one array and leaves its contents
+ *   behind; each call clears the part that must start at zero (its status
+ *   word).  Calls that overlap on the GPU (e.g. on two streams at once) race
+ *   on it: serialise them. */
+#define LORA_LINEAR_NOALLOC_SCRATCH_BYTES (16u << 20)
+lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* desc,
+                                      const void* X, const void* W, const void* A, const void* B,
+                                      const void* W_up, const void* A_up, const void* B_up,
+                                      void* Y, float* T_save, float* Z_save, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

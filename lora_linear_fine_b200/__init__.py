@@ -27,7 +27,7 @@ STATUS_NAMES = {
 # Every symbol include/lora_linear.h declares.
 EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_linear_device_status",
             "lora_linear_fwd", "lora_linear_bwd", "lora_status_string", "lora_linear_abi_version",
-            "lora_linear_launch_count")
+            "lora_linear_launch_count", "lora_linear_fwd_noalloc")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -63,6 +63,8 @@ def _load():
     lib.lora_linear_abi_version.restype = i32
     lib.lora_linear_launch_count.argtypes = []
     lib.lora_linear_launch_count.restype = ctypes.c_uint64
+    lib.lora_linear_fwd_noalloc.argtypes = [dp] + [vp] * 10 + [vp]
+    lib.lora_linear_fwd_noalloc.restype = i32
     return lib
 
 
@@ -114,6 +116,16 @@ def lora_linear_bwd(desc, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, 
                     workspace, workspace_bytes, stream) -> int:
     return int(_lib.lora_linear_bwd(ctypes.byref(desc), dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save,
                                     dX, dA, dB, dA_up, dB_up, workspace, workspace_bytes, stream))
+
+
+def lora_linear_fwd_noalloc(desc, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, stream) -> int:
+    """The forward for callers that cannot allocate device memory: its scratch
+    is a fixed 16 MiB device array inside the library (see the C header)."""
+    return int(_lib.lora_linear_fwd_noalloc(ctypes.byref(desc), X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save,
+                                            stream))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def status_string(status: int) -> str:

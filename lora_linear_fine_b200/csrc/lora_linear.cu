@@ -779,4 +779,58 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   return LORA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Forward for callers that cannot allocate device memory: the workspace is a
+// file-scope device array (every device that loads this library holds it until
+// exit).  Its device address is looked up once per device, on that device's
+// first call, with the device current.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LORA_LINEAR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+lora_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cuda_error("cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      LORA_LOG("cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
+      return LORA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LORA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, const void* W, const void* A,
+                                      const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
+                                      float* T_save, float* Z_save, void* stream) {
+  LORA_TRY(check_desc(d));
+  const size_t need = make_plan(d, false).total;
+  if (need > LORA_LINEAR_NOALLOC_SCRATCH_BYTES) {
+    LORA_LOG("fwd_noalloc: needs %zu bytes of scratch, the static array holds %u", need,
+             LORA_LINEAR_NOALLOC_SCRATCH_BYTES);
+    return LORA_ERR_UNSUPPORTED;
+  }
+  void* ws = nullptr;
+  LORA_TRY(noalloc_scratch(&ws));
+  // The status word must start at zero; everything else the forward writes
+  // before it reads.
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return cuda_error("cudaMemsetAsync(scratch status)");
+  return lora_linear_fwd(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, ws, LORA_LINEAR_NOALLOC_SCRATCH_BYTES,
+                         stream);
+}
+
 }  // extern "C"
