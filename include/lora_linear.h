@@ -145,6 +145,19 @@ int lora_linear_abi_version(void);
  * (all devices, all threads).  For accounting in benchmarks and tests. */
 uint64_t lora_linear_launch_count(void);
 
+/* Benchmark instrumentation.  lora_linear_timing_enable(1) makes every later
+ * lora_linear_fwd / lora_linear_bwd call record a CUDA event pair around its
+ * main GEMM launch (the tcgen05 kernel that computes Y or dX) on the call's
+ * stream.  lora_linear_timing_read waits for those events, returns the summed
+ * milliseconds and launch counts of the forward and backward GEMMs recorded
+ * since the previous read, and resets them.  enable(0) stops recording.  The
+ * event objects are created by enable(1) (up to 1024 pairs per direction);
+ * further launches beyond that are not timed.  Not meant for concurrent calls
+ * from several host threads. */
+lora_status_t lora_linear_timing_enable(int enable);
+lora_status_t lora_linear_timing_read(double* fwd_ms, uint64_t* fwd_launches, double* bwd_ms,
+                                      uint64_t* bwd_launches);
+
 /* Forward without a workspace argument, for callers that cannot allocate
  * device memory: for example a plug-in inside a host application that owns
  * every device allocation through its own pool and forbids direct cudaMalloc,

@@ -27,7 +27,8 @@ STATUS_NAMES = {
 # Every symbol include/lora_linear.h declares.
 EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_linear_device_status",
             "lora_linear_fwd", "lora_linear_bwd", "lora_status_string", "lora_linear_abi_version",
-            "lora_linear_launch_count", "lora_linear_fwd_noalloc")
+            "lora_linear_launch_count", "lora_linear_fwd_noalloc", "lora_linear_timing_enable",
+            "lora_linear_timing_read")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -65,6 +66,11 @@ def _load():
     lib.lora_linear_launch_count.restype = ctypes.c_uint64
     lib.lora_linear_fwd_noalloc.argtypes = [dp] + [vp] * 10 + [vp]
     lib.lora_linear_fwd_noalloc.restype = i32
+    lib.lora_linear_timing_enable.argtypes = [i32]
+    lib.lora_linear_timing_enable.restype = i32
+    dblp, u64p = ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)
+    lib.lora_linear_timing_read.argtypes = [dblp, u64p, dblp, u64p]
+    lib.lora_linear_timing_read.restype = i32
     return lib
 
 
@@ -126,6 +132,18 @@ def lora_linear_fwd_noalloc(desc, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_sav
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def lora_linear_timing_enable(enable: int) -> int:
+    return int(_lib.lora_linear_timing_enable(int(enable)))
+
+
+def lora_linear_timing_read():
+    """(status, fwd_gemm_ms, fwd_launches, bwd_gemm_ms, bwd_launches) since the last read."""
+    fm, bm = ctypes.c_double(0), ctypes.c_double(0)
+    fl, bl = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    st = int(_lib.lora_linear_timing_read(ctypes.byref(fm), ctypes.byref(fl), ctypes.byref(bm), ctypes.byref(bl)))
+    return st, fm.value, int(fl.value), bm.value, int(bl.value)
 
 
 def status_string(status: int) -> str:

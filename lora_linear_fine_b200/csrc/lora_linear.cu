@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <atomic>
+#include <vector>
 #include <mutex>
 
 #include "lora_mma.cuh"
@@ -120,19 +121,20 @@ lora_status_t check_desc(const lora_linear_desc* d) {
 
 // Workspace layouts (offsets in bytes, each 256-aligned, status word at 0).
 struct Plan {
-  // shapes
-  int np = 1;          // projections: 2 for SwiGLU (gate, up)
-  int RP = 0;          // r padded to the MMA granule (0, 16, 32, 64)
-  bool act_f16 = false;  // backward with an activation: fp16 dZ operands
+  int np = 1;              // projections: 2 for SwiGLU (gate, up)
+  int RP = 0;              // r padded to the MMA granule (0, 16, 32, 64)
+  bool act_f16 = false;    // backward with an activation: fp16 dZ operands
   int64_t M8 = 8;
-  // split-K widths of the rank passes
+  // split-K widths of the rank passes (1 = results written directly)
   int splits_t = 1, splits_u = 1, splits_a = 1, splits_b = 1;
   // regions
-  size_t bt[2] = {}, t_ws[2] = {}, part_t = 0;                 // forward + backward
-  size_t s16[2] = {};                                          // bf16 s*T (fwd) / s*U (bwd) [M x r]
-  size_t u_ws = 0, tt_hi[2] = {}, tt_lo[2] = {}, ut_hi[2] = {}, ut_lo[2] = {};
-  size_t dz_hi[2] = {}, dz_lo[2] = {}, w16[2] = {};
-  size_t part_u = 0, part_a = 0, part_b = 0;
+  size_t s16[2] = {};                        // bf16 s*T (fwd) / s*U (bwd) [M x r]: LoRA K-block operand
+  size_t t_ws = 0;                           // fp32 T [np][M x r] when the caller saves none (fwd)
+  size_t bt[2] = {};                         // B^T [r x d_out] (bwd)
+  size_t tt_hi[2] = {}, tt_lo[2] = {};       // (s*T)^T hi / lo [r x M8] (bwd, dB)
+  size_t ut_hi[2] = {}, ut_lo[2] = {};       // (s*U)^T hi / lo [r x M8] (bwd, dA)
+  size_t dz_hi[2] = {}, dz_lo[2] = {}, w16[2] = {};   // activation backward: fp16 operands
+  size_t part_t = 0, part_u = 0, part_a = 0, part_b = 0;   // split-K partials
   size_t total = 0;
 };
 
@@ -150,9 +152,6 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
   P.np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
   P.RP = rank_pad(d->r);
   P.act_f16 = backward && d->act != LORA_ACT_IDENTITY;
-  // The LoRA branch rides the GEMM's K-loop as extra K-blocks fed by a rank
-  // pass (T = X A^T, U = dZ B computed once per token): no rank columns in
-  // tensor memory, which then holds two accumulator buffers.
   P.M8 = static_cast<int64_t>(align_up(static_cast<size_t>(d->M > 0 ? d->M : 1), 8));
   const int64_t M = d->M, r = d->r;
   const int64_t tiles_m = ceil_div(M > 0 ? M : 1, 128);
@@ -162,18 +161,17 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     off += align_up(bytes, 256);
     return o;
   };
+  auto partials = [&](int splits, int64_t tiles) -> size_t {
+    return splits > 1 ? take(static_cast<size_t>(splits) * tiles * 128 * P.RP * 4) : 0;
+  };
   if (r > 0) {
-    if (backward)
-      for (int j = 0; j < P.np; ++j) P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
+    // The LoRA branch rides the GEMM's K-loop as extra K-blocks fed by a rank
+    // pass (T = X A^T, U = dZ B computed once per token): no rank columns in
+    // tensor memory, which then holds two accumulator buffers.
     for (int j = 0; j < P.np; ++j) P.s16[j] = take(static_cast<size_t>(M) * r * 2);
     P.splits_t = rank_splits(tiles_m, ceil_div(d->d_in, 64));
-    const bool need_t = true;
-    if (need_t) {
-      // T of all projections is one [np][M x r] block (the GEMM reads it that way).
-      P.t_ws[0] = take(static_cast<size_t>(P.np) * M * r * 4);
-      P.t_ws[1] = P.t_ws[0] + static_cast<size_t>(M) * r * 4;
-      P.part_t = take(static_cast<size_t>(P.splits_t) * tiles_m * 128 * P.RP * 4);
-    }
+    P.part_t = partials(P.splits_t, tiles_m);
+    if (!backward) P.t_ws = take(static_cast<size_t>(P.np) * M * r * 4);
   }
   if (!backward) {
     P.total = off;
@@ -187,8 +185,8 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     }
   }
   if (r > 0) {
-    P.u_ws = take(static_cast<size_t>(P.np) * M * r * 4);
     for (int j = 0; j < P.np; ++j) {
+      P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
       P.tt_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
       P.tt_lo[j] = take(static_cast<size_t>(r) * P.M8 * 2);
       P.ut_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
@@ -199,9 +197,9 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     P.splits_u = rank_splits(tiles_m, ceil_div(d->d_out, 64));
     P.splits_a = rank_splits(tiles_a, nkb_tok);
     P.splits_b = rank_splits(tiles_b, nkb_tok);
-    P.part_u = take(static_cast<size_t>(P.splits_u) * tiles_m * 128 * P.RP * 4);
-    P.part_a = take(static_cast<size_t>(P.splits_a) * tiles_a * 128 * P.RP * 4);
-    P.part_b = take(static_cast<size_t>(P.splits_b) * tiles_b * 128 * P.RP * 4);
+    P.part_u = partials(P.splits_u, tiles_m);
+    P.part_a = partials(P.splits_a, tiles_a);
+    P.part_b = partials(P.splits_b, tiles_b);
   }
   P.total = off;
   return P;
@@ -224,6 +222,28 @@ lora_status_t check_launch(const char* what) {
     return LORA_ERR_CUDA;
   }
   return LORA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// benchmark instrumentation: CUDA events around the main GEMM launches
+// ---------------------------------------------------------------------------
+struct TimingState {
+  bool enabled = false;
+  std::vector<cudaEvent_t> ev[2];      // [direction] 2 events per launch
+  size_t used[2] = {0, 0};
+};
+TimingState g_timing;
+constexpr size_t kTimingPairs = 1024;
+
+void timing_begin(int dir, cudaStream_t st) {
+  if (!g_timing.enabled || g_timing.used[dir] >= kTimingPairs) return;
+  cudaEventRecord(g_timing.ev[dir][2 * g_timing.used[dir]], st);
+}
+
+void timing_end(int dir, cudaStream_t st) {
+  if (!g_timing.enabled || g_timing.used[dir] >= kTimingPairs) return;
+  cudaEventRecord(g_timing.ev[dir][2 * g_timing.used[dir] + 1], st);
+  ++g_timing.used[dir];
 }
 
 #define LORA_TRY(...)                           \
@@ -264,45 +284,12 @@ int grid_for(long long n, int per_block, int sms) {
   return static_cast<int>(g);
 }
 
-lora_status_t transpose_b(const void* B, int64_t d_out, int64_t r, void* Bt, bool f16, uint32_t* status, int sms,
-                          cudaStream_t st) {
-  const long long n = d_out * r;
-  if (f16)
-    transpose_b_kernel<__half><<<grid_for(n, 256, sms), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(B), (int)d_out, (int)r, static_cast<__half*>(Bt), status);
-  else
-    transpose_b_kernel<__nv_bfloat16><<<grid_for(n, 256, sms), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(B), (int)d_out, (int)r, static_cast<__nv_bfloat16*>(Bt), status);
-  return check_launch("transpose_b_kernel");
-}
-
-lora_status_t reduce_partials(const float* part, int splits, int rows, int RP, int r, const float* add, float* dst,
-                              int transpose, int sms, cudaStream_t st, void* dst16 = nullptr, float scale16 = 1.0f) {
-  const long long n = static_cast<long long>(rows) * r;
-  const int rows_pad = static_cast<int>(ceil_div(rows, 128) * 128);
-  reduce_partials_kernel<<<grid_for(n, 256, sms), 256, 0, st>>>(part, splits, rows_pad, RP, rows, r, add, dst,
-                                                               transpose, static_cast<__nv_bfloat16*>(dst16),
-                                                               scale16);
-  return check_launch("reduce_partials_kernel");
-}
-
-lora_status_t rank_split_t(const float* src, int M, int r, float scale, void* hi, void* lo, int ld, bool f16,
-                           uint32_t* status, int sms, cudaStream_t st) {
-  const long long n = static_cast<long long>(M) * r;
-  if (f16)
-    rank_split_t_kernel<__half><<<grid_for(n, 256, sms), 256, 0, st>>>(
-        src, M, r, scale, static_cast<__half*>(hi), static_cast<__half*>(lo), ld, status);
-  else
-    rank_split_t_kernel<__nv_bfloat16><<<grid_for(n, 256, sms), 256, 0, st>>>(
-        src, M, r, scale, static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo), ld, status);
-  return check_launch("rank_split_t_kernel");
-}
-
-// rows x r result of sum_q A[pa[q]] * B[pb[q]] reduced over K = 64-blocks split
-// `splits` ways, written (after a fixed-order reduction) to dst.
+// A rows x r rank product sum_q A[pa[q]] * B[pb[q]] over K (64-wide blocks
+// split `splits` ways).  splits == 1: the kernel writes `out` directly;
+// otherwise it writes fp32 partials to `partial` and reduce_rank finishes.
 struct RankJob {
   bool a_mn = false;   // A read MN-major (result rows are the A tensor's columns)
-  bool f16 = false;
+  bool f16 = false;    // A and B operands are fp16 (else bf16)
   const void* a[2] = {nullptr, nullptr};
   int64_t a_inner = 0, a_outer = 0, a_ld = 0;     // A tensors share one shape
   const void* b[2] = {nullptr, nullptr};
@@ -312,14 +299,19 @@ struct RankJob {
   int rows = 0, K = 0;
   float* partial = nullptr;
   int splits = 1;
-  const float* add = nullptr;
-  float* dst = nullptr;
-  int transpose = 0;
-  void* dst16 = nullptr;     // optional bf16 copy of scale16 * dst
-  float scale16 = 1.0f;
+  RankOut out = {};
 };
 
-lora_status_t run_rank(const RankJob& J, int RP, int r, uint32_t* status, int sms, cudaStream_t st) {
+RankOut rank_out(int rows, int r) {
+  RankOut o;
+  std::memset(&o, 0, sizeof(o));
+  o.rows = rows;
+  o.r = r;
+  o.scale = 1.0f;
+  return o;
+}
+
+lora_status_t run_rank_gemm(const RankJob& J, int RP, int r, uint32_t* status, cudaStream_t st) {
   RankGemmParams q;
   std::memset(&q, 0, sizeof(q));
   bool ok = true;
@@ -333,26 +325,49 @@ lora_status_t run_rank(const RankJob& J, int RP, int r, uint32_t* status, int sm
   q.kb_per_split = static_cast<int>(ceil_div(ceil_div(J.K, 64), J.splits));
   q.npairs = J.npairs;
   for (int i = 0; i < 4; ++i) { q.pa[i] = J.pa[i]; q.pb[i] = J.pb[i]; }
-  q.partial = J.partial;
+  q.partial = J.splits > 1 ? J.partial : nullptr;
+  q.out = J.out;
   q.status = status;
-  lora_status_t s;
   if (J.a_mn) {
-    if (J.na == 1 && J.nb == 2 && !J.f16) s = launch_rank_rp<true, 1, 2, false>(RP, q, J.splits, st);
-    else if (J.na == 2 && J.nb == 2 && J.f16) s = launch_rank_rp<true, 2, 2, true>(RP, q, J.splits, st);
-    else s = LORA_ERR_UNSUPPORTED;
+    if (J.na == 1 && J.nb == 2 && !J.f16) return launch_rank_rp<true, 1, 2, false>(RP, q, J.splits, st);
+    if (J.na == 2 && J.nb == 2 && J.f16) return launch_rank_rp<true, 2, 2, true>(RP, q, J.splits, st);
   } else {
-    if (J.na == 1 && J.nb == 1 && !J.f16) s = launch_rank_rp<false, 1, 1, false>(RP, q, J.splits, st);
-    else if (J.na == 2 && J.nb == 1 && J.f16) s = launch_rank_rp<false, 2, 1, true>(RP, q, J.splits, st);
-    else s = LORA_ERR_UNSUPPORTED;
+    if (J.na == 1 && J.nb == 1 && !J.f16) return launch_rank_rp<false, 1, 1, false>(RP, q, J.splits, st);
+    if (J.na == 2 && J.nb == 1 && J.f16) return launch_rank_rp<false, 2, 1, true>(RP, q, J.splits, st);
   }
-  LORA_TRY(s);
-  return reduce_partials(J.partial, J.splits, J.rows, RP, r, J.add, J.dst, J.transpose, sms, st, J.dst16,
-                         J.scale16);
+  return LORA_ERR_UNSUPPORTED;
 }
 
-// T_j = X A_j^T (fp32 [M x r]) by a rank pass; optionally also bf16(s T_j).
-lora_status_t compute_T(const lora_linear_desc* d, const Plan& P, const void* X, const void* Aj, float* dst,
-                        uint8_t* ws, uint32_t* status, int sms, cudaStream_t st, void* dst16 = nullptr) {
+RankReduceJob reduce_job(const RankJob& J, int RP) {
+  RankReduceJob R;
+  R.partial = J.partial;
+  R.splits = J.splits;
+  R.rows_pad = static_cast<int>(ceil_div(J.rows, 128) * 128);
+  R.RP = RP;
+  R.out = J.out;
+  return R;
+}
+
+// Finish the jobs that were split (at most two, one launch).
+lora_status_t finish_rank(const RankJob* j0, const RankJob* j1, int RP, cudaStream_t st) {
+  const RankJob* js[2] = {j0, j1};
+  RankReduceJob R[2];
+  int n = 0, rows = 0;
+  for (const RankJob* J : js) {
+    if (J == nullptr || J->splits <= 1) continue;
+    R[n++] = reduce_job(*J, RP);
+    rows = J->rows > rows ? J->rows : rows;
+  }
+  if (n == 0) return LORA_OK;
+  if (n == 1) R[1] = R[0];
+  const dim3 grid(static_cast<unsigned>(ceil_div(rows, 128)), static_cast<unsigned>(n), 1);
+  reduce_rank_kernel<<<grid, 128, 0, st>>>(R[0], R[1]);
+  return check_launch("reduce_rank_kernel");
+}
+
+// T_j = X A_j^T written to `out` (split K finished in place).
+lora_status_t rank_T(const lora_linear_desc* d, const Plan& P, const void* X, const void* Aj, const RankOut& out,
+                     uint8_t* ws, uint32_t* status, cudaStream_t st) {
   RankJob J;
   J.a[0] = X;
   J.a_inner = d->d_in;
@@ -365,10 +380,9 @@ lora_status_t compute_T(const lora_linear_desc* d, const Plan& P, const void* X,
   J.K = static_cast<int>(d->d_in);
   J.partial = reinterpret_cast<float*>(ws + P.part_t);
   J.splits = P.splits_t;
-  J.dst = dst;
-  J.dst16 = dst16;
-  J.scale16 = d->s;
-  return run_rank(J, P.RP, static_cast<int>(d->r), status, sms, st);
+  J.out = out;
+  LORA_TRY(run_rank_gemm(J, P.RP, static_cast<int>(d->r), status, st));
+  return finish_rank(&J, nullptr, P.RP, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -437,6 +451,41 @@ extern "C" {
 int lora_linear_abi_version(void) { return kAbiVersion; }
 
 uint64_t lora_linear_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+lora_status_t lora_linear_timing_enable(int enable) {
+  if (enable) {
+    for (int dir = 0; dir < 2; ++dir) {
+      while (g_timing.ev[dir].size() < 2 * kTimingPairs) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return cuda_error("cudaEventCreate");
+        g_timing.ev[dir].push_back(e);
+      }
+      g_timing.used[dir] = 0;
+    }
+  }
+  g_timing.enabled = enable != 0;
+  return LORA_OK;
+}
+
+lora_status_t lora_linear_timing_read(double* fwd_ms, uint64_t* fwd_launches, double* bwd_ms,
+                                      uint64_t* bwd_launches) {
+  double ms[2] = {0.0, 0.0};
+  for (int dir = 0; dir < 2; ++dir) {
+    for (size_t i = 0; i < g_timing.used[dir]; ++i) {
+      float t = 0.0f;
+      if (cudaEventSynchronize(g_timing.ev[dir][2 * i + 1]) != cudaSuccess ||
+          cudaEventElapsedTime(&t, g_timing.ev[dir][2 * i], g_timing.ev[dir][2 * i + 1]) != cudaSuccess)
+        return cuda_error("cudaEventElapsedTime");
+      ms[dir] += t;
+    }
+  }
+  if (fwd_ms) *fwd_ms = ms[0];
+  if (bwd_ms) *bwd_ms = ms[1];
+  if (fwd_launches) *fwd_launches = g_timing.used[0];
+  if (bwd_launches) *bwd_launches = g_timing.used[1];
+  g_timing.used[0] = g_timing.used[1] = 0;
+  return LORA_OK;
+}
 
 const char* lora_status_string(lora_status_t s) {
   switch (s) {
@@ -537,9 +586,12 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   // 1. T_j = X A_j^T (fp32, saved for the backward) and bf16(s T_j) for the LoRA K-block
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
-      float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r
-                         : reinterpret_cast<float*>(ws + P.t_ws[0]) + static_cast<size_t>(j) * M * r;
-      LORA_TRY(compute_T(d, P, X, Ap[j], Tj, ws, status, dev.sms, st, ws + P.s16[j]));
+      RankOut o = rank_out(static_cast<int>(M), static_cast<int>(r));
+      o.f32 = T_save ? T_save + static_cast<size_t>(j) * M * r
+                     : reinterpret_cast<float*>(ws + P.t_ws) + static_cast<size_t>(j) * M * r;
+      o.s16 = reinterpret_cast<__nv_bfloat16*>(ws + P.s16[j]);
+      o.scale = d->s;
+      LORA_TRY(rank_T(d, P, X, Ap[j], o, ws, status, st));
     }
   }
   // 2. Z = [X | sT] [W | B]^T, activation, bf16 Y
@@ -568,11 +620,15 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   p.n_tiles = static_cast<int>(ceil_div(d->d_out, outc));
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.group_m = pair ? 4 : 8;
+  timing_begin(0, st);
+  lora_status_t rs;
   switch (d->act) {
-    case LORA_ACT_IDENTITY: return launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st);
-    case LORA_ACT_SILU: return launch_mma_any<false, 1, kMEpiSilu>(pair, p, dev.sms, st);
-    default: return launch_mma_any<false, 2, kMEpiSwiglu>(pair, p, dev.sms, st);
+    case LORA_ACT_IDENTITY: rs = launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st); break;
+    case LORA_ACT_SILU: rs = launch_mma_any<false, 1, kMEpiSilu>(pair, p, dev.sms, st); break;
+    default: rs = launch_mma_any<false, 2, kMEpiSwiglu>(pair, p, dev.sms, st); break;
   }
+  timing_end(0, st);
+  return rs;
 }
 
 lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const void* X, const void* W, const void* A,
@@ -645,43 +701,60 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     }
   }
 
-  // 2. B^T (in the dZ operand type); T (saved or recomputed) as s*T hi + lo, transposed.
-  float* U = r > 0 ? static_cast<float*>(at(P.u_ws)) : nullptr;   // [np][M x r]
+  // 2. B^T and (s T)^T hi/lo (from the saved T, or a rank pass recomputing T),
+  //    in the dZ operand type.
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
-      LORA_TRY(transpose_b(Bp[j], d->d_out, r, at(P.bt[j]), f16, status, dev.sms, st));
       const float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r : nullptr;
+      const long long n = static_cast<long long>(d->d_out) * r + (Tj ? static_cast<long long>(M) * r : 0);
+      if (f16)
+        bwd_prep_kernel<__half><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
+            static_cast<__half*>(at(P.bt[j])), Tj, M, d->s, static_cast<__half*>(at(P.tt_hi[j])),
+            static_cast<__half*>(at(P.tt_lo[j])), M8, status);
+      else
+        bwd_prep_kernel<__nv_bfloat16><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
+            static_cast<__nv_bfloat16*>(at(P.bt[j])), Tj, M, d->s, static_cast<__nv_bfloat16*>(at(P.tt_hi[j])),
+            static_cast<__nv_bfloat16*>(at(P.tt_lo[j])), M8, status);
+      LORA_TRY(check_launch("bwd_prep_kernel"));
       if (Tj == nullptr) {
-        LORA_TRY(compute_T(d, P, X, Ap[j], static_cast<float*>(at(P.t_ws[j])), ws, status, dev.sms, st));
-        Tj = static_cast<const float*>(at(P.t_ws[j]));
+        RankOut o = rank_out(M, r);
+        o.hi = at(P.tt_hi[j]);
+        o.lo = at(P.tt_lo[j]);
+        o.ld = M8;
+        o.hilo_f16 = f16 ? 1 : 0;
+        o.scale = d->s;
+        LORA_TRY(rank_T(d, P, X, Ap[j], o, ws, status, st));
       }
-      LORA_TRY(rank_split_t(Tj, M, r, d->s, at(P.tt_hi[j]), at(P.tt_lo[j]), M8, f16, status, dev.sms, st));
     }
-    // 3. U = dZ B by a rank pass (fp32, and bf16 s U for the LoRA K-block of dX)
-    {
-      for (int j = 0; j < np; ++j) {
-        RankJob J;
-        J.f16 = f16;
-        J.a[0] = dZ[j];
-        J.a[1] = dZlo[j];
-        J.na = f16 ? 2 : 1;
-        J.npairs = f16 ? 2 : 1;
-        J.pa[1] = 1;   // dZ_lo B
-        J.a_inner = d->d_out;
-        J.a_outer = M;
-        J.a_ld = d->d_out;
-        J.b[0] = at(P.bt[j]);
-        J.b_inner = d->d_out;
-        J.b_ld = d->d_out;
-        J.rows = M;
-        J.K = static_cast<int>(d->d_out);
-        J.partial = static_cast<float*>(at(P.part_u));
-        J.splits = P.splits_u;
-        J.dst = U + static_cast<size_t>(j) * M * r;
-        J.dst16 = at(P.s16[j]);
-        J.scale16 = d->s;
-        LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
-      }
+    // 3. U = dZ B by a rank pass: bf16 s U (LoRA K-block of dX) and (s U)^T hi/lo (dA)
+    for (int j = 0; j < np; ++j) {
+      RankJob J;
+      J.f16 = f16;
+      J.a[0] = dZ[j];
+      J.a[1] = dZlo[j];
+      J.na = f16 ? 2 : 1;
+      J.npairs = f16 ? 2 : 1;
+      J.pa[1] = 1;   // dZ_lo B
+      J.a_inner = d->d_out;
+      J.a_outer = M;
+      J.a_ld = d->d_out;
+      J.b[0] = at(P.bt[j]);
+      J.b_inner = d->d_out;
+      J.b_ld = d->d_out;
+      J.rows = M;
+      J.K = static_cast<int>(d->d_out);
+      J.partial = static_cast<float*>(at(P.part_u));
+      J.splits = P.splits_u;
+      J.out = rank_out(M, r);
+      J.out.s16 = static_cast<__nv_bfloat16*>(at(P.s16[j]));
+      J.out.hi = at(P.ut_hi[j]);
+      J.out.lo = at(P.ut_lo[j]);
+      J.out.ld = M8;
+      J.out.scale = d->s;
+      LORA_TRY(run_rank_gemm(J, RP, r, status, st));
+      LORA_TRY(finish_rank(&J, nullptr, RP, st));
     }
   }
 
@@ -711,70 +784,70 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     p.n_tiles = static_cast<int>(ceil_div(d->d_in, 256));
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.group_m = pair ? 4 : 8;
+    timing_begin(1, st);
+    lora_status_t rs;
     if (f16) {
-      if (np == 2) LORA_TRY((launch_mma_any<true, 2, kMEpiGradF16>(pair, p, dev.sms, st)));
-      else LORA_TRY((launch_mma_any<true, 1, kMEpiGradF16>(pair, p, dev.sms, st)));
+      if (np == 2) rs = launch_mma_any<true, 2, kMEpiGradF16>(pair, p, dev.sms, st);
+      else rs = launch_mma_any<true, 1, kMEpiGradF16>(pair, p, dev.sms, st);
     } else {
-      LORA_TRY((launch_mma_any<true, 1, kMEpiGrad>(pair, p, dev.sms, st)));
+      rs = launch_mma_any<true, 1, kMEpiGrad>(pair, p, dev.sms, st);
     }
+    timing_end(1, st);
+    LORA_TRY(rs);
   }
   if (r == 0) return LORA_OK;
 
+  // 5. dA^T = X^T (s U) and dB = dZ^T (s T), hi/lo operands, split over tokens
   for (int j = 0; j < np; ++j) {
-    float* Uj = U + static_cast<size_t>(j) * M * r;
-    // 5. s U as bf16 hi + lo, transposed
-    LORA_TRY(rank_split_t(Uj, M, r, d->s, at(P.ut_hi[j]), at(P.ut_lo[j]), M8, false, status, dev.sms, st));
-    // 6. dA^T = X^T (s U)
-    {
-      RankJob J;
-      J.a_mn = true;
-      J.a[0] = X;
-      J.a_inner = d->d_in;
-      J.a_outer = M;
-      J.a_ld = d->d_in;
-      J.b[0] = at(P.ut_hi[j]);
-      J.b[1] = at(P.ut_lo[j]);
-      J.nb = 2;
-      J.b_inner = M;
-      J.b_ld = M8;
-      J.npairs = 2;
-      J.pb[1] = 1;
-      J.rows = static_cast<int>(d->d_in);
-      J.K = M;
-      J.partial = static_cast<float*>(at(P.part_a));
-      J.splits = P.splits_a;
-      J.dst = dAp[j];
-      J.transpose = 1;
-      LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
-    }
-    // 7. dB = dZ^T (s T)
-    {
-      RankJob J;
-      J.a_mn = true;
-      J.f16 = f16;
-      J.a[0] = dZ[j];
-      J.a[1] = dZlo[j];
-      J.na = f16 ? 2 : 1;
-      J.a_inner = d->d_out;
-      J.a_outer = M;
-      J.a_ld = d->d_out;
-      J.b[0] = at(P.tt_hi[j]);
-      J.b[1] = at(P.tt_lo[j]);
-      J.nb = 2;
-      J.b_inner = M;
-      J.b_ld = M8;
-      // dZ_hi (T_hi + T_lo) [+ dZ_lo T_hi]
-      J.npairs = f16 ? 3 : 2;
-      J.pb[1] = 1;
-      J.pa[2] = 1;
-      J.pb[2] = 0;
-      J.rows = static_cast<int>(d->d_out);
-      J.K = M;
-      J.partial = static_cast<float*>(at(P.part_b));
-      J.splits = P.splits_b;
-      J.dst = dBp[j];
-      LORA_TRY(run_rank(J, RP, r, status, dev.sms, st));
-    }
+    RankJob Ja;
+    Ja.a_mn = true;
+    Ja.a[0] = X;
+    Ja.a_inner = d->d_in;
+    Ja.a_outer = M;
+    Ja.a_ld = d->d_in;
+    Ja.b[0] = at(P.ut_hi[j]);
+    Ja.b[1] = at(P.ut_lo[j]);
+    Ja.nb = 2;
+    Ja.b_inner = M;
+    Ja.b_ld = M8;
+    Ja.npairs = 2;
+    Ja.pb[1] = 1;
+    Ja.rows = static_cast<int>(d->d_in);
+    Ja.K = M;
+    Ja.partial = static_cast<float*>(at(P.part_a));
+    Ja.splits = P.splits_a;
+    Ja.out = rank_out(static_cast<int>(d->d_in), r);
+    Ja.out.f32 = dAp[j];
+    Ja.out.transpose_f32 = 1;
+    LORA_TRY(run_rank_gemm(Ja, RP, r, status, st));
+
+    RankJob Jb;
+    Jb.a_mn = true;
+    Jb.f16 = f16;
+    Jb.a[0] = dZ[j];
+    Jb.a[1] = dZlo[j];
+    Jb.na = f16 ? 2 : 1;
+    Jb.a_inner = d->d_out;
+    Jb.a_outer = M;
+    Jb.a_ld = d->d_out;
+    Jb.b[0] = at(P.tt_hi[j]);
+    Jb.b[1] = at(P.tt_lo[j]);
+    Jb.nb = 2;
+    Jb.b_inner = M;
+    Jb.b_ld = M8;
+    // dZ_hi (T_hi + T_lo) [+ dZ_lo T_hi]
+    Jb.npairs = f16 ? 3 : 2;
+    Jb.pb[1] = 1;
+    Jb.pa[2] = 1;
+    Jb.pb[2] = 0;
+    Jb.rows = static_cast<int>(d->d_out);
+    Jb.K = M;
+    Jb.partial = static_cast<float*>(at(P.part_b));
+    Jb.splits = P.splits_b;
+    Jb.out = rank_out(static_cast<int>(d->d_out), r);
+    Jb.out.f32 = dBp[j];
+    LORA_TRY(run_rank_gemm(Jb, RP, r, status, st));
+    LORA_TRY(finish_rank(&Ja, &Jb, RP, st));
   }
   return LORA_OK;
 }

@@ -10,8 +10,9 @@
 //   fp32-grade precision although the tensor cores take bf16.
 //   One CTA = one 128-row tile x one K range; it writes an fp32 partial that
 //   reduce_partials_kernel sums in a fixed order (deterministic, no atomics).
-// The elementwise kernels: B -> B^T, rank matrices -> transposed hi/lo bf16,
-// the activation backward dZ = dY * act'(Z) as hi/lo bf16.
+// Also: the fixed-order reduction of split-K partials, the backward's
+// preparation (B^T, transposed hi/lo s*T), the fp16 weight copy and the
+// activation backward dZ = dY * act'(Z) as fp16 hi/lo.
 #pragma once
 
 #include <type_traits>
@@ -22,6 +23,60 @@ namespace lora {
 
 constexpr int kRankThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 
+// Where a finished rows x r rank result goes (any subset of the outputs):
+//   f32  fp32, row-major [rows x r] (transpose_f32: [r x rows])
+//   s16  bf16(scale * v), row-major [rows x r] (the LoRA K-block operand)
+//   hi/lo  scale * v split into a 16-bit hi part and the rounded remainder,
+//          transposed [r x ld] (bf16, or fp16 when hilo_f16)
+struct RankOut {
+  float* f32;
+  int transpose_f32;
+  __nv_bfloat16* s16;
+  void* hi;
+  void* lo;
+  int ld;
+  int hilo_f16;
+  float scale;
+  int rows, r;
+};
+
+__device__ __forceinline__ void emit_rank_row(const float* v, int row, const RankOut& o) {
+  if (o.f32 != nullptr) {
+    if (o.transpose_f32) {
+      for (int c = 0; c < o.r; ++c) o.f32[static_cast<size_t>(c) * o.rows + row] = v[c];
+    } else {
+      float* d = o.f32 + static_cast<size_t>(row) * o.r;
+      for (int c = 0; c < o.r; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+    }
+  }
+  if (o.s16 != nullptr) {
+    __nv_bfloat16* d = o.s16 + static_cast<size_t>(row) * o.r;
+    for (int c = 0; c < o.r; c += 8) {
+      uint4 pk;
+      pk.x = pack_bf16x2(o.scale * v[c + 0], o.scale * v[c + 1]);
+      pk.y = pack_bf16x2(o.scale * v[c + 2], o.scale * v[c + 3]);
+      pk.z = pack_bf16x2(o.scale * v[c + 4], o.scale * v[c + 5]);
+      pk.w = pack_bf16x2(o.scale * v[c + 6], o.scale * v[c + 7]);
+      *reinterpret_cast<uint4*>(d + c) = pk;
+    }
+  }
+  if (o.hi != nullptr) {
+    for (int c = 0; c < o.r; ++c) {
+      const float x = o.scale * v[c];
+      const size_t i = static_cast<size_t>(c) * o.ld + row;
+      if (o.hilo_f16) {
+        const __half h = __float2half_rn(x);
+        static_cast<__half*>(o.hi)[i] = h;
+        static_cast<__half*>(o.lo)[i] = __float2half_rn(x - __half2float(h));
+      } else {
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        static_cast<__nv_bfloat16*>(o.hi)[i] = h;
+        static_cast<__nv_bfloat16*>(o.lo)[i] = __float2bfloat16_rn(x - __bfloat162float(h));
+      }
+    }
+  }
+}
+
 struct RankGemmParams {
   CUtensorMap tm_a[2];
   CUtensorMap tm_b[2];
@@ -31,7 +86,8 @@ struct RankGemmParams {
   int kb_per_split;
   int npairs;        // products accumulated: sum over q < npairs of A[pa[q]] * B[pb[q]]
   int pa[4], pb[4];
-  float* partial;    // [splits][m_tiles*128][RP] fp32
+  float* partial;    // [splits][m_tiles*128][RP] fp32; null when K is not split: results go to `out`
+  RankOut out;
   uint32_t* status;
 };
 
@@ -146,11 +202,12 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   } else {
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    float* dst = p.partial + (static_cast<size_t>(sp) * p.m_tiles * 128 + static_cast<size_t>(mt) * 128 + row) * kRP;
-    if (nkb == 0) {
+    float acc[kRP];
 #pragma unroll
-      for (int c = 0; c < kRP; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else if (mbar_wait(acc_full, 0, ctl)) {
+    for (int c = 0; c < kRP; ++c) acc[c] = 0.0f;
+    bool have = nkb == 0;
+    if (nkb > 0 && mbar_wait(acc_full, 0, ctl)) {
+      have = true;
       tc_fence_after();
       __syncwarp();
       const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
@@ -160,9 +217,17 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
         tmem_ld16(tl + c0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; c += 4)
-          *reinterpret_cast<float4*>(dst + c0 + c) = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                                                 __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+        for (int c = 0; c < 16; ++c) acc[c0 + c] = __uint_as_float(v[c]);
+      }
+    }
+    if (have) {
+      if (p.partial != nullptr) {
+        float* dst = p.partial + (static_cast<size_t>(sp) * p.m_tiles * 128 + static_cast<size_t>(mt) * 128 + row) * kRP;
+#pragma unroll
+        for (int c = 0; c < kRP; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+      } else {
+        const int grow = mt * 128 + row;
+        if (grow < p.rows) emit_rank_row(acc, grow, p.out);
       }
     }
   }
@@ -174,23 +239,28 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   }
 }
 
-// dst = sum over splits of partial[sp][row][c] (+ add[row][c]); fixed order.
-// transpose == 0: dst[row * r + c];  transpose == 1: dst[c * rows + row].
-// dst16 (optional, transpose == 0 only): bf16(scale16 * dst) in the same layout.
-__global__ void reduce_partials_kernel(const float* __restrict__ partial, int splits, int rows_pad, int RP,
-                                       int rows, int r, const float* __restrict__ add, float* __restrict__ dst,
-                                       int transpose, __nv_bfloat16* __restrict__ dst16, float scale16) {
-  const long long n = static_cast<long long>(rows) * r;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    int row, c;
-    if (transpose) { c = static_cast<int>(i / rows); row = static_cast<int>(i % rows); }
-    else { row = static_cast<int>(i / r); c = static_cast<int>(i % r); }
-    float acc = add ? add[static_cast<size_t>(row) * r + c] : 0.0f;
-    for (int sp = 0; sp < splits; ++sp) acc += partial[(static_cast<size_t>(sp) * rows_pad + row) * RP + c];
-    dst[i] = acc;
-    if (dst16 != nullptr) dst16[i] = __float2bfloat16_rn(scale16 * acc);
+// Fixed-order sum of split-K partials, one thread per result row, for up to
+// two independent jobs in one launch (blockIdx.y selects the job).
+struct RankReduceJob {
+  const float* partial;   // [splits][rows_pad][RP]
+  int splits, rows_pad, RP;
+  RankOut out;
+};
+
+__global__ void reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
+  const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= J.out.rows) return;
+  float acc[64];
+  for (int c = 0; c < J.out.r; ++c) acc[c] = 0.0f;
+  for (int sp = 0; sp < J.splits; ++sp) {
+    const float* src = J.partial + (static_cast<size_t>(sp) * J.rows_pad + row) * J.RP;
+    for (int c = 0; c < J.out.r; c += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src + c);
+      acc[c] += v.x; acc[c + 1] += v.y; acc[c + 2] += v.z; acc[c + 3] += v.w;
+    }
   }
+  emit_rank_row(acc, row, J.out);
 }
 
 // Rounding of an fp32 value to the 16-bit operand type T (bf16 or fp16).
@@ -201,40 +271,33 @@ __device__ __forceinline__ float from16(__nv_bfloat16 v) { return __bfloat162flo
 __device__ __forceinline__ float from16(__half v) { return __half2float(v); }
 constexpr float kF16Max = 65504.0f;
 
-// src fp32 [M x r] -> hi, lo [r x ld] (bf16 or fp16) with v = scale * src,
-// hi = round(v), lo = round(v - hi).  Columns M..ld-1 are never read.
+// Backward preparation in one launch: B^T ([r x d_out], bf16 or fp16) and the
+// transposed hi/lo split of s*T ([r x ld]) from the forward's fp32 T.
 template <typename T>
-__global__ void rank_split_t_kernel(const float* __restrict__ src, int M, int r, float scale, T* __restrict__ hi,
-                                    T* __restrict__ lo, int ld, uint32_t* status) {
-  const long long n = static_cast<long long>(M) * r;
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r, T* __restrict__ Bt,
+                                const float* __restrict__ Tsave, int M, float s, T* __restrict__ t_hi,
+                                T* __restrict__ t_lo, int ld, uint32_t* status) {
+  const long long nb = static_cast<long long>(d_out) * r;
+  const long long nt = Tsave != nullptr ? static_cast<long long>(M) * r : 0;
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nb + nt;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(i / M);
-    const int m = static_cast<int>(i % M);
-    const float v = scale * src[static_cast<size_t>(m) * r + c];
-    const T h = to16<T>(v);
-    hi[static_cast<size_t>(c) * ld + m] = h;
-    lo[static_cast<size_t>(c) * ld + m] = to16<T>(v - from16(h));
-    if (sizeof(T) == 2 && !std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
-  }
-  if (bad && status) atomicOr(status, kStatusF16Range);
-}
-
-// B [d_out x r] (bf16) -> B^T [r x d_out] in T (exact for bf16; for fp16 exact
-// inside fp16's normal range, values beyond it flag the status word).
-template <typename T>
-__global__ void transpose_b_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r, T* __restrict__ Bt,
-                                   uint32_t* status) {
-  const long long n = static_cast<long long>(d_out) * r;
-  bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(i / d_out);
-    const int j = static_cast<int>(i % d_out);
-    const float v = __bfloat162float(B[static_cast<size_t>(j) * r + c]);
-    Bt[i] = to16<T>(v);
-    if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
+    if (i < nb) {
+      const int c = static_cast<int>(i / d_out);
+      const int jd = static_cast<int>(i % d_out);
+      const float v = __bfloat162float(B[static_cast<size_t>(jd) * r + c]);
+      Bt[i] = to16<T>(v);
+      if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
+    } else {
+      const long long k = i - nb;
+      const int c = static_cast<int>(k / M);
+      const int m = static_cast<int>(k % M);
+      const float v = s * Tsave[static_cast<size_t>(m) * r + c];
+      const T h = to16<T>(v);
+      t_hi[static_cast<size_t>(c) * ld + m] = h;
+      t_lo[static_cast<size_t>(c) * ld + m] = to16<T>(v - from16(h));
+      if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
+    }
   }
   if (bad && status) atomicOr(status, kStatusF16Range);
 }
