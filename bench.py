@@ -196,6 +196,25 @@ def run_reference(args, cfg, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# multi-rank helpers (replicas: one process per GPU, no collective on the data
+# path; ranks only meet for the timing barrier and the max over ranks)
+# ---------------------------------------------------------------------------
+def max_over_ranks(x, dist, device):
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step, steps, world, max_ms):
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return units_per_step * steps * world / (max_ms * 1e-3)
+
+
 def committed_traffic(workload):
     """DRAM bytes per launch of the forward GEMM from a committed ncu summary,
     valid only while the kernel source is unchanged (else None)."""
@@ -352,12 +371,9 @@ def main():
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
     tot_ms = sum(step_ms)
-    if dist is not None:
-        tt = torch.tensor([tot_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        tot_ms = float(tt.item())
+    tot_ms = max_over_ranks(tot_ms, dist, "cuda")
     F = step_flops(M, d_in, d_out, r, act)
-    value = F * args.steps * world / (tot_ms * 1e-3) / 1e12
+    value = job_throughput(F, args.steps, world, tot_ms) / 1e12
 
     # e2e: the same step through the C ABI from pinned HOST buffers, copies included
     out_host = {"Y": torch.empty_like(Y, device="cpu").pin_memory(),
@@ -383,11 +399,8 @@ def main():
     ee1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ee0.elapsed_time(ee1)
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e = F * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
+    e2e = job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12
 
     peaks = read_peaks()
     # Dominant kernels: the forward and backward GEMMs (lora_mma_kernel), each

@@ -315,14 +315,15 @@ lora_status_t run_rank_gemm(const RankJob& J, int RP, int r, uint32_t* status, c
   RankGemmParams q;
   std::memset(&q, 0, sizeof(q));
   bool ok = true;
+  const int ks = J.na == 1 ? 2 : 1;   // 64-wide K blocks per stage (RankCfg::kKS)
   for (int i = 0; i < J.na; ++i)
-    ok = ok && make_tm(&q.tm_a[i], J.a[i], J.a_inner, J.a_outer, J.a_ld, 64, J.a_mn ? 64 : 128, J.f16);
+    ok = ok && make_tm(&q.tm_a[i], J.a[i], J.a_inner, J.a_outer, J.a_ld, 64, J.a_mn ? 64 * ks : 128, J.f16);
   for (int i = 0; i < J.nb; ++i) ok = ok && make_tm(&q.tm_b[i], J.b[i], J.b_inner, r, J.b_ld, 64, RP, J.f16);
   if (!ok) return LORA_ERR_CUDA;
   q.rows = J.rows;
   q.K = J.K;
   q.m_tiles = static_cast<int>(ceil_div(J.rows, 128));
-  q.kb_per_split = static_cast<int>(ceil_div(ceil_div(J.K, 64), J.splits));
+  q.kb_per_split = static_cast<int>(ceil_div(ceil_div(J.K, 64 * ks), J.splits));
   q.npairs = J.npairs;
   for (int i = 0; i < 4; ++i) { q.pa[i] = J.pa[i]; q.pb[i] = J.pb[i]; }
   q.partial = J.splits > 1 ? J.partial : nullptr;
@@ -352,16 +353,22 @@ RankReduceJob reduce_job(const RankJob& J, int RP) {
 lora_status_t finish_rank(const RankJob* j0, const RankJob* j1, int RP, cudaStream_t st) {
   const RankJob* js[2] = {j0, j1};
   RankReduceJob R[2];
-  int n = 0, rows = 0;
+  int n = 0;
   for (const RankJob* J : js) {
     if (J == nullptr || J->splits <= 1) continue;
     R[n++] = reduce_job(*J, RP);
-    rows = J->rows > rows ? J->rows : rows;
   }
   if (n == 0) return LORA_OK;
   if (n == 1) R[1] = R[0];
-  const dim3 grid(static_cast<unsigned>(ceil_div(rows, 128)), static_cast<unsigned>(n), 1);
-  reduce_rank_kernel<<<grid, 128, 0, st>>>(R[0], R[1]);
+  long long elems = 0;
+  for (int i = 0; i < n; ++i) {
+    const long long e = static_cast<long long>(R[i].out.rows) * R[i].out.r;
+    elems = e > elems ? e : elems;
+  }
+  long long gx = (elems + 255) / 256;
+  if (gx > 1184) gx = 1184;
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(n), 1);
+  reduce_rank_kernel<<<grid, 256, 0, st>>>(R[0], R[1]);
   return check_launch("reduce_rank_kernel");
 }
 
@@ -426,6 +433,19 @@ lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
     return LORA_ERR_CUDA;
   }
   return check_launch("lora_mma_kernel");
+}
+
+// Raster choice for the GEMM: keep in L2 whichever operand fits.  m_bytes /
+// n_bytes: total bytes of the M-side / N-side operands streamed by the K-loop.
+void set_raster(MmaParams& p, bool pair, double m_bytes, double n_bytes) {
+  constexpr double kL2Resident = 64.0 * 1024 * 1024;   // comfortably inside the 126 MB L2
+  if (m_bytes <= kL2Resident && n_bytes > m_bytes) {
+    p.group_along_n = 1;   // sweep all M tiles per group of N tiles: the N side streams once
+    p.group = 1;
+  } else {
+    p.group_along_n = 0;   // sweep all N tiles per group of M tiles: the N side stays in L2
+    p.group = pair ? 4 : 8;
+  }
 }
 
 template <bool kBwd, int kNPair, int kEpi>
@@ -619,7 +639,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
   p.n_tiles = static_cast<int>(ceil_div(d->d_out, outc));
   p.num_tiles = p.m_tiles * p.n_tiles;
-  p.group_m = pair ? 4 : 8;
+  set_raster(p, pair, 2.0 * M * d->d_in, 2.0 * np * d->d_out * d->d_in);
   timing_begin(0, st);
   lora_status_t rs;
   switch (d->act) {
@@ -783,7 +803,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
     p.n_tiles = static_cast<int>(ceil_div(d->d_in, 256));
     p.num_tiles = p.m_tiles * p.n_tiles;
-    p.group_m = pair ? 4 : 8;
+    set_raster(p, pair, 2.0 * np * M * d->d_out, 2.0 * np * d->d_out * d->d_in);
     timing_begin(1, st);
     lora_status_t rs;
     if (f16) {

@@ -92,12 +92,19 @@ struct RankGemmParams {
 };
 
 // kNA / kNB: number of distinct A / B operand tiles per stage (1 or 2).
+// One pipeline stage covers kKS consecutive 64-wide K blocks: per A operand
+// kKS K-major boxes of 128 rows x 64 (or two MN-major boxes of 64 x 64*kKS),
+// per B operand kKS boxes of RP rows x 64.  Larger TMA boxes and several
+// boxes per stage keep more DRAM traffic in flight per request (measured:
+// 8 KB boxes stream at about half the rate of 32-64 KB stages).
 template <bool kAMN, int kRP, int NA, int NB, bool kF16>
 struct RankCfg {
   static constexpr int kNA = NA;
   static constexpr int kNB = NB;
-  static constexpr int kABytes = 128 * 64 * 2;
-  static constexpr int kBBytes = kRP * 128;
+  static constexpr int kKS = NA == 1 ? 2 : 1;             // 64-wide K blocks per stage
+  static constexpr int kABytes = 128 * 64 * 2 * kKS;      // one A operand per stage
+  static constexpr int kBBox = kRP * 128;                 // one B box (64 K)
+  static constexpr int kBBytes = kBBox * kKS;             // one B operand per stage
   static constexpr int kStageBytes = kNA * kABytes + kNB * kBBytes;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
@@ -124,7 +131,8 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   AbortCtl ctl{abort_flag, p.status};
   const int mt = blockIdx.x % p.m_tiles;
   const int sp = blockIdx.x / p.m_tiles;
-  const int nkb_all = (p.K + 63) / 64;
+  constexpr int KS = C::kKS;
+  const int nkb_all = (p.K + 64 * KS - 1) / (64 * KS);     // stages over the whole K
   const int kb0 = sp * p.kb_per_split;
   int kb1 = kb0 + p.kb_per_split;
   if (kb1 > nkb_all) kb1 = nkb_all;
@@ -152,21 +160,25 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
         uint8_t* st = smem + rp.stage * C::kStageBytes;
         uint64_t* fb = &full[rp.stage];
         mbar_arrive_expect_tx(fb, C::kStageBytes);
-        const int k0 = (kb0 + i) * 64;
+        const int k0 = (kb0 + i) * 64 * KS;
         const int m0 = mt * 128;
 #pragma unroll
         for (int a = 0; a < C::kNA; ++a) {
           uint8_t* sa = st + a * C::kABytes;
           if constexpr (kAMN) {
+            // two boxes of 64 rows-of-the-result x 64*KS K (tokens)
             tma_load_2d_hint(sa, &p.tm_a[a], fb, m0, k0, pol);
-            tma_load_2d_hint(sa + 8192, &p.tm_a[a], fb, m0 + 64, k0, pol);
+            tma_load_2d_hint(sa + C::kABytes / 2, &p.tm_a[a], fb, m0 + 64, k0, pol);
           } else {
-            tma_load_2d_hint(sa, &p.tm_a[a], fb, k0, m0, pol);
+#pragma unroll
+            for (int kb = 0; kb < KS; ++kb) tma_load_2d_hint(sa + kb * 16384, &p.tm_a[a], fb, k0 + 64 * kb, m0, pol);
           }
         }
 #pragma unroll
         for (int b = 0; b < C::kNB; ++b)
-          tma_load_2d(st + C::kNA * C::kABytes + b * C::kBBytes, &p.tm_b[b], fb, k0, 0);
+#pragma unroll
+          for (int kb = 0; kb < KS; ++kb)
+            tma_load_2d(st + C::kNA * C::kABytes + b * C::kBBytes + kb * C::kBBox, &p.tm_b[b], fb, k0 + 64 * kb, 0);
         rp.next(S);
       }
     }
@@ -180,12 +192,13 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
         tc_fence_after();
         const uint32_t st = smem_u32(smem + rp.stage * C::kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < 4 * KS; ++kk) {
           for (int pp = 0; pp < p.npairs; ++pp) {
             const uint32_t sa = st + p.pa[pp] * C::kABytes;
-            const uint32_t sb = st + C::kNA * C::kABytes + p.pb[pp] * C::kBBytes;
-            const uint64_t da = kAMN ? sdesc_sw128(sa + kk * 2048, 8192, 1024) : sdesc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t db = sdesc_sw128(sb + kk * 32, 16, 1024);
+            const uint32_t sb = st + C::kNA * C::kABytes + p.pb[pp] * C::kBBytes + (kk >> 2) * C::kBBox;
+            const uint64_t da = kAMN ? sdesc_sw128(sa + kk * 2048, C::kABytes / 2, 1024)
+                                     : sdesc_sw128(sa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t db = sdesc_sw128(sb + (kk & 3) * 32, 16, 1024);
             mma_bf16(tbase, da, db, kId, (i == 0 && kk == 0 && pp == 0) ? 0u : 1u);
           }
         }
@@ -247,20 +260,40 @@ struct RankReduceJob {
   RankOut out;
 };
 
-__global__ void reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
-  const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
-  const int row = blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= J.out.rows) return;
-  float acc[64];
-  for (int c = 0; c < J.out.r; ++c) acc[c] = 0.0f;
-  for (int sp = 0; sp < J.splits; ++sp) {
-    const float* src = J.partial + (static_cast<size_t>(sp) * J.rows_pad + row) * J.RP;
-    for (int c = 0; c < J.out.r; c += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src + c);
-      acc[c] += v.x; acc[c + 1] += v.y; acc[c + 2] += v.z; acc[c + 3] += v.w;
+// One element of a finished rank result (same outputs as emit_rank_row).
+__device__ __forceinline__ void emit_rank_elem(float v, int row, int c, const RankOut& o) {
+  if (o.f32 != nullptr) {
+    if (o.transpose_f32) o.f32[static_cast<size_t>(c) * o.rows + row] = v;
+    else o.f32[static_cast<size_t>(row) * o.r + c] = v;
+  }
+  if (o.s16 != nullptr) o.s16[static_cast<size_t>(row) * o.r + c] = __float2bfloat16_rn(o.scale * v);
+  if (o.hi != nullptr) {
+    const float x = o.scale * v;
+    const size_t i = static_cast<size_t>(c) * o.ld + row;
+    if (o.hilo_f16) {
+      const __half h = __float2half_rn(x);
+      static_cast<__half*>(o.hi)[i] = h;
+      static_cast<__half*>(o.lo)[i] = __float2half_rn(x - __half2float(h));
+    } else {
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
+      static_cast<__nv_bfloat16*>(o.hi)[i] = h;
+      static_cast<__nv_bfloat16*>(o.lo)[i] = __float2bfloat16_rn(x - __bfloat162float(h));
     }
   }
-  emit_rank_row(acc, row, J.out);
+}
+
+// One thread per (row, column) element; grid-stride; splits summed in order.
+__global__ void reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
+  const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
+  const long long n = static_cast<long long>(J.out.rows) * J.out.r;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(i / J.out.r);
+    const int c = static_cast<int>(i % J.out.r);
+    float acc = 0.0f;
+    for (int sp = 0; sp < J.splits; ++sp) acc += J.partial[(static_cast<size_t>(sp) * J.rows_pad + row) * J.RP + c];
+    emit_rank_elem(acc, row, c, J.out);
+  }
 }
 
 // Rounding of an fp32 value to the 16-bit operand type T (bf16 or fp16).
