@@ -49,7 +49,10 @@ struct MmaParams {
   __nv_bfloat16* out;     // [M x N]
   float* z_save;          // [npair][M x N] fp32 or null (SiLU / SwiGLU forward)
   uint32_t* status;
-  int m_tiles, n_tiles, num_tiles, group_m;
+  int m_tiles, n_tiles, num_tiles;
+  int group;              // raster group width (tiles)
+  int group_along_n;      // 0: groups of `group` M tiles sweep all N tiles (the N-side operand stays in L2)
+                          // 1: groups of `group` N tiles sweep all M tiles (the M-side operand stays in L2)
 };
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
@@ -71,15 +74,28 @@ struct MmaCfg {
   static_assert(kStages >= 3, "ring too shallow");
 };
 
+// Tile t of the raster.  Consecutive tiles (processed at the same time by
+// neighbouring CTAs) share their N-side operand (group_along_n = 0: M fastest
+// inside a group of `group` M tiles) or their M-side operand (group_along_n = 1:
+// M fastest inside a group of `group` N tiles, so the whole M-side operand is
+// swept per group and stays in L2 while the N-side operand streams once).
 __device__ __forceinline__ void mma_tile_coords(int t, const MmaParams& p, int& mt, int& nt) {
-  const int per_group = p.group_m * p.n_tiles;
-  const int g = t / per_group;
-  const int first_m = g * p.group_m;
-  const int rem = p.m_tiles - first_m;
-  const int gm = rem < p.group_m ? rem : p.group_m;
-  const int idx = t - g * per_group;
-  mt = first_m + idx % gm;
-  nt = idx / gm;
+  if (p.group_along_n) {
+    const int per_group = p.group * p.m_tiles;
+    const int g = t / per_group;
+    const int idx = t - g * per_group;
+    mt = idx % p.m_tiles;
+    nt = g * p.group + idx / p.m_tiles;
+  } else {
+    const int per_group = p.group * p.n_tiles;
+    const int g = t / per_group;
+    const int first_m = g * p.group;
+    const int rem = p.m_tiles - first_m;
+    const int gm = rem < p.group ? rem : p.group;
+    const int idx = t - g * per_group;
+    mt = first_m + idx % gm;
+    nt = idx / gm;
+  }
 }
 
 template <bool kPair>
@@ -287,6 +303,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
     const int q = warp & 3;                  // TMEM lane quadrant
     const int h = ew >> 2;                   // column half
     const int row_in_tile = q * 32 + lane;
+    const uint64_t pol_out = l2_policy_evict_first();
     uint32_t acc_empty_addr[2];
 #pragma unroll
     for (int b = 0; b < 2; ++b)
@@ -328,11 +345,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
             if (col0 + c < p.N) {
-              *reinterpret_cast<float4*>(zg + c) = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                                               __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-              *reinterpret_cast<float4*>(zu + c) =
-                  make_float4(__uint_as_float(v[64 + c]), __uint_as_float(v[65 + c]), __uint_as_float(v[66 + c]),
-                              __uint_as_float(v[67 + c]));
+              st_global_v4_hint(zg + c, make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]), pol_out);
+              st_global_v4_hint(zu + c, make_uint4(v[64 + c], v[65 + c], v[66 + c], v[67 + c]), pol_out);
             }
           }
         }
@@ -351,7 +365,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             pk.y = pack_bf16x2(hv[2], hv[3]);
             pk.z = pack_bf16x2(hv[4], hv[5]);
             pk.w = pack_bf16x2(hv[6], hv[7]);
-            *reinterpret_cast<uint4*>(p.out + base + c) = pk;
+            st_global_v4_hint(p.out + base + c, pk, pol_out);
           }
         }
       } else {
@@ -362,9 +376,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 #pragma unroll
             for (int c = 0; c < 128; c += 4)
               if (col0 + c < p.N)
-                *reinterpret_cast<float4*>(p.z_save + base + c) =
-                    make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
-                                __uint_as_float(v[c + 3]));
+                st_global_v4_hint(p.z_save + base + c, make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]), pol_out);
           }
         }
 #pragma unroll
@@ -381,7 +393,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             pk.y = pack_bf16x2(yv[2], yv[3]);
             pk.z = pack_bf16x2(yv[4], yv[5]);
             pk.w = pack_bf16x2(yv[6], yv[7]);
-            *reinterpret_cast<uint4*>(p.out + base + c) = pk;
+            st_global_v4_hint(p.out + base + c, pk, pol_out);
           }
         }
       }
