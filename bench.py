@@ -281,9 +281,18 @@ def main():
     ap.add_argument("--config", default="q_proj", choices=sorted(seeded_inputs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--shape", default=None,
+                    help="M,d_in,d_out,r,act: this shape instead of --config (profiling, with --calls)")
+    ap.add_argument("--calls", type=int, default=0,
+                    help="run this many untimed forward(+backward) calls, print nothing else, exit (for profilers)")
+    ap.add_argument("--fwd-only", action="store_true", help="with --calls: forward calls only")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = dict(seeded_inputs.CONFIGS[args.config])
+    if args.shape:
+        f = args.shape.split(",")
+        cfg = dict(M=int(f[0]), d_in=int(f[1]), d_out=int(f[2]), r=int(f[3]), alpha=16.0, act=f[4])
+        args.config = "shape " + args.shape
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -305,7 +314,7 @@ def main():
     import lora_linear_fine_b200 as L
 
     M, d_in, d_out, r, act = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]
-    s = cfg["alpha"] / r
+    s = cfg["alpha"] / r if r else 0.0
     inp = seeded_inputs.make_inputs(M, d_in, d_out, r, act, seed=rank)
     host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in inp.items()}
     t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
@@ -335,6 +344,14 @@ def main():
                                ws.buf.data_ptr(), ws.nbytes, sh)
         assert st == 0, L.status_string(st)
 
+    if args.calls > 0:
+        for _ in range(args.calls):
+            fwd()
+            if not args.fwd_only:
+                bwd()
+        torch.cuda.synchronize()
+        print("ok", flush=True)
+        return
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     if args.config.startswith("small_m"):
         run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist)

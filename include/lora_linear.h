@@ -49,6 +49,8 @@
  *   error bits into it (a bounded wait that gave up, a failed device-side
  *   check); they never clear it.  Zero it once with lora_linear_workspace_init
  *   before the first call; read it with lora_linear_device_status.
+ * - Calls that share a workspace must not overlap in time (issue them on one
+ *   stream): they use the same scratch regions and counters.
  */
 #ifndef LORA_LINEAR_H
 #define LORA_LINEAR_H
@@ -91,10 +93,16 @@ typedef struct lora_linear_desc {
 
 /* Bytes of device workspace lora_linear_fwd (for_backward == 0) or
  * lora_linear_bwd (for_backward != 0) needs for `desc`.  Returns 0 for an
- * invalid desc.  The size is a function of the desc only. */
+ * invalid desc.  The size is a function of the desc only, and the backward
+ * size is never below the forward size, so one workspace sized for the
+ * backward serves both calls (one after the other, on one stream). */
 size_t lora_linear_workspace_size(const lora_linear_desc* desc, int for_backward);
 
-/* Zero the status word of a workspace (asynchronous, on `stream`). */
+/* Zero the header of a workspace (asynchronous, on `stream`): the status word
+ * and the arrival counters the few-token forward keeps there.  Both are zero
+ * at rest; call this once after allocating the workspace, and again after any
+ * call that left a non-zero status (an aborted call can leave counters set).
+ * workspace_bytes must be at least the header (4352 bytes). */
 lora_status_t lora_linear_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, copy the workspace status word to *out_status and
@@ -134,6 +142,20 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* desc,
                               const float* T_save, const float* Z_save,
                               void* dX, float* dA, float* dB, float* dA_up, float* dB_up,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Failure-detection self-test.  The pages have no counterpart: it checks this
+ * library's own give-up path.  Launches one CTA on `stream` whose thread waits
+ * on an mbarrier that nothing arrives on, through the same bounded-wait
+ * routine every kernel here uses, with a limit of 2^limit_log2 SM cycles
+ * instead of the usual 2^34.  The wait gives up, ORs 0x1 into the workspace
+ * status word and the kernel returns: no trap, the context stays usable.
+ * Read the outcome with lora_linear_device_status; clear it with
+ * lora_linear_workspace_init.
+ *   workspace: device, >= 4352 bytes (the header), 16-byte aligned, else
+ *              LORA_ERR_WORKSPACE.
+ *   limit_log2: 10..30, else LORA_ERR_INVALID_ARG. */
+lora_status_t lora_linear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_log2,
+                                                void* stream);
 
 /* Static string for a status code (never NULL). */
 const char* lora_status_string(lora_status_t status);

@@ -28,7 +28,7 @@ STATUS_NAMES = {
 EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_linear_device_status",
             "lora_linear_fwd", "lora_linear_bwd", "lora_status_string", "lora_linear_abi_version",
             "lora_linear_launch_count", "lora_linear_fwd_noalloc", "lora_linear_timing_enable",
-            "lora_linear_timing_read")
+            "lora_linear_timing_read", "lora_linear_selftest_wait_timeout")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -71,6 +71,8 @@ def _load():
     dblp, u64p = ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)
     lib.lora_linear_timing_read.argtypes = [dblp, u64p, dblp, u64p]
     lib.lora_linear_timing_read.restype = i32
+    lib.lora_linear_selftest_wait_timeout.argtypes = [vp, sz, i32, vp]
+    lib.lora_linear_selftest_wait_timeout.restype = i32
     return lib
 
 
@@ -104,6 +106,10 @@ def lora_linear_workspace_size(desc: LoraLinearDesc, for_backward: int) -> int:
 
 def lora_linear_workspace_init(workspace, workspace_bytes, stream) -> int:
     return int(_lib.lora_linear_workspace_init(workspace, workspace_bytes, stream))
+
+
+def lora_linear_selftest_wait_timeout(workspace, workspace_bytes, limit_log2, stream) -> int:
+    return int(_lib.lora_linear_selftest_wait_timeout(workspace, workspace_bytes, int(limit_log2), stream))
 
 
 def lora_linear_device_status(workspace, stream):

@@ -15,6 +15,7 @@
 
 #include "lora_mma.cuh"
 #include "lora_rank.cuh"
+#include "lora_rank2d.cuh"
 #include "lora_small_m.cuh"
 
 namespace {
@@ -24,6 +25,10 @@ using namespace lora;
 constexpr int kAbiVersion = 1;
 constexpr int kTargetCtas = 148;   // SM count of a B200; sets split-K widths
 constexpr size_t kStatusBytes = 256;
+// Workspace header, zero at rest: the status block, then the arrival counters
+// of the few-token forward (one per 128-row slice of [A ; W], plus two).
+constexpr size_t kCounterWords = 1024;
+constexpr size_t kHeaderBytes = kStatusBytes + kCounterWords * 4;
 
 // ---------------------------------------------------------------------------
 // debug logging (LORA_LINEAR_DEBUG=1)
@@ -133,10 +138,28 @@ struct Plan {
   size_t bt[2] = {};                         // B^T [r x d_out] (bwd)
   size_t tt_hi[2] = {}, tt_lo[2] = {};       // (s*T)^T hi / lo [r x M8] (bwd, dB)
   size_t ut_hi[2] = {}, ut_lo[2] = {};       // (s*U)^T hi / lo [r x M8] (bwd, dA)
-  size_t dz_hi[2] = {}, dz_lo[2] = {}, w16[2] = {};   // activation backward: fp16 operands
+  size_t dz_hi[2] = {}, dz_lo[2] = {};     // activation backward: fp16 dZ operands
+  size_t wt[2] = {};                        // W^T [d_in x d_out] (bf16, fp16 with an activation): dX's K-major operand
+  size_t at_[2] = {};                       // A^T [d_in x r] bf16: the dX LoRA block's K-major operand
   size_t part_t = 0, part_u = 0, part_a = 0, part_b = 0;   // split-K partials
+  // backward rank passes on rank2d_kernel: U and dB from one read of dZ
+  // (identity, r <= 32), dA over X
+  bool dual = false;
+  Rank2dSplit sp_dual, sp_a;
+  // few-token forward
+  bool small_m = false;
+  int sm_nt = 16;                            // tokens padded to the MMA N granule
+  SmallMSplit sm;
+  size_t sm_t_buf = 0, sm_d_part = 0;
   size_t total = 0;
 };
+
+// The few-token forward applies to identity / SiLU with an adapter and at most
+// kSmallMMax tokens, while its slice counters fit the workspace header.
+bool small_m_applies(const lora_linear_desc* d) {
+  return d->M > 0 && d->M <= kSmallMMax && d->r > 0 && d->act != LORA_ACT_SWIGLU &&
+         static_cast<size_t>(1 + ceil_div(d->d_out, 128)) + 2 <= kCounterWords;
+}
 
 // Split-K width for a rank-r product with `tiles` row tiles and `nkb` 64-wide K blocks.
 int rank_splits(int64_t tiles, int64_t nkb) {
@@ -155,7 +178,7 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
   P.M8 = static_cast<int64_t>(align_up(static_cast<size_t>(d->M > 0 ? d->M : 1), 8));
   const int64_t M = d->M, r = d->r;
   const int64_t tiles_m = ceil_div(M > 0 ? M : 1, 128);
-  size_t off = kStatusBytes;
+  size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += align_up(bytes, 256);
@@ -174,18 +197,26 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     if (!backward) P.t_ws = take(static_cast<size_t>(P.np) * M * r * 4);
   }
   if (!backward) {
+    if (small_m_applies(d)) {
+      P.small_m = true;
+      P.sm_nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+      P.sm = small_m_split(d->d_in, d->d_out, kTargetCtas);
+      P.sm_t_buf = take(static_cast<size_t>(M) * r * 4);
+      P.sm_d_part = take(static_cast<size_t>(P.sm.slices) * P.sm.max_seg * 128 * P.sm_nt * 4);
+    }
     P.total = off;
     return P;
   }
-  if (P.act_f16) {
-    for (int j = 0; j < P.np; ++j) {
+  for (int j = 0; j < P.np; ++j) {
+    P.wt[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
+    if (P.act_f16) {
       P.dz_hi[j] = take(static_cast<size_t>(M) * d->d_out * 2);
       P.dz_lo[j] = take(static_cast<size_t>(M) * d->d_out * 2);
-      P.w16[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
     }
   }
   if (r > 0) {
     for (int j = 0; j < P.np; ++j) {
+      P.at_[j] = take(static_cast<size_t>(d->d_in) * r * 2);
       P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
       P.tt_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
       P.tt_lo[j] = take(static_cast<size_t>(r) * P.M8 * 2);
@@ -194,12 +225,20 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     }
     const int64_t tiles_a = ceil_div(d->d_in, 128), tiles_b = ceil_div(d->d_out, 128);
     const int64_t nkb_tok = ceil_div(M > 0 ? M : 1, 64);
-    P.splits_u = rank_splits(tiles_m, ceil_div(d->d_out, 64));
-    P.splits_a = rank_splits(tiles_a, nkb_tok);
-    P.splits_b = rank_splits(tiles_b, nkb_tok);
-    P.part_u = partials(P.splits_u, tiles_m);
-    P.part_a = partials(P.splits_a, tiles_a);
-    P.part_b = partials(P.splits_b, tiles_b);
+    P.dual = d->act == LORA_ACT_IDENTITY && P.RP <= 32;
+    if (P.dual) {
+      P.sp_dual = rank2d_split(static_cast<int>(tiles_m), static_cast<int>(tiles_b), P.RP, true, true,
+                               rank2d_max_rb(P.RP), kTargetCtas);
+      if (P.sp_dual.fs > 1) P.part_u = take(static_cast<size_t>(P.sp_dual.fs) * tiles_m * 128 * P.RP * 4);
+      if (P.sp_dual.ts > 1) P.part_b = take(static_cast<size_t>(P.sp_dual.ts) * tiles_b * 128 * P.RP * 4);
+    } else {
+      P.splits_u = rank_splits(tiles_m, ceil_div(d->d_out, 64));
+      P.splits_b = rank_splits(tiles_b, nkb_tok);
+      P.part_u = partials(P.splits_u, tiles_m);
+      P.part_b = partials(P.splits_b, tiles_b);
+    }
+    P.sp_a = rank2d_split(static_cast<int>(tiles_m), static_cast<int>(tiles_a), P.RP, false, true, 0, kTargetCtas);
+    if (P.sp_a.ts > 1) P.part_a = take(static_cast<size_t>(P.sp_a.ts) * tiles_a * 128 * P.RP * 4);
   }
   P.total = off;
   return P;
@@ -349,6 +388,22 @@ RankReduceJob reduce_job(const RankJob& J, int RP) {
   return R;
 }
 
+// Fixed-order reduction of up to two split results in one launch.
+lora_status_t launch_reduce(RankReduceJob* R, int n, cudaStream_t st) {
+  if (n == 0) return LORA_OK;
+  if (n == 1) R[1] = R[0];
+  long long blocks = 0;
+  for (int i = 0; i < n; ++i) {
+    const long long b = (R[i].out.rows + kReduceRows - 1) / kReduceRows;
+    blocks = b > blocks ? b : blocks;
+  }
+  long long gx = blocks;
+  if (gx > 1184) gx = 1184;
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(n), 1);
+  reduce_rank_kernel<<<grid, 256, 0, st>>>(R[0], R[1]);
+  return check_launch("reduce_rank_kernel");
+}
+
 // Finish the jobs that were split (at most two, one launch).
 lora_status_t finish_rank(const RankJob* j0, const RankJob* j1, int RP, cudaStream_t st) {
   const RankJob* js[2] = {j0, j1};
@@ -358,18 +413,83 @@ lora_status_t finish_rank(const RankJob* j0, const RankJob* j1, int RP, cudaStre
     if (J == nullptr || J->splits <= 1) continue;
     R[n++] = reduce_job(*J, RP);
   }
-  if (n == 0) return LORA_OK;
-  if (n == 1) R[1] = R[0];
-  long long elems = 0;
-  for (int i = 0; i < n; ++i) {
-    const long long e = static_cast<long long>(R[i].out.rows) * R[i].out.r;
-    elems = e > elems ? e : elems;
+  return launch_reduce(R, n, st);
+}
+
+// One rank2d_kernel pass over Z [mtok x F] (bf16): the row product Z RB
+// (rb = RB^T [r x F], or null) and/or the col product Z^T (CB_hi + CB_lo)
+// (cb = [r x mtok] parts with row stride ld_cb), then the fixed-order
+// reduction of whichever result was split.
+template <int kRP, bool kRow, bool kCol>
+lora_status_t launch_rank2d_t(const Rank2dParams& p, int grid, cudaStream_t st) {
+  using C = Rank2dCfg<kRP, kRow, kCol>;
+  auto k = rank2d_kernel<kRP, kRow, kCol>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return cuda_error("cudaFuncSetAttribute(rank2d)");
+  LORA_LOG("rank2d RP=%d row=%d col=%d grid=%d a=%d b=%d fs=%d stages=%d", kRP, (int)kRow, (int)kCol, grid,
+           p.a_tiles, p.b_blocks, p.fs, C::kStages);
+  k<<<grid, kRank2dThreads, C::kSmemBytes, st>>>(p);
+  return check_launch("rank2d_kernel");
+}
+
+template <bool kRow, bool kCol>
+lora_status_t launch_rank2d_rp(int RP, const Rank2dParams& p, int grid, cudaStream_t st) {
+  switch (RP) {
+    case 16: return launch_rank2d_t<16, kRow, kCol>(p, grid, st);
+    case 32: return launch_rank2d_t<32, kRow, kCol>(p, grid, st);
+    case 64: return launch_rank2d_t<64, kRow, kCol>(p, grid, st);
+    default: return LORA_ERR_UNSUPPORTED;
   }
-  long long gx = (elems + 255) / 256;
-  if (gx > 1184) gx = 1184;
-  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(n), 1);
-  reduce_rank_kernel<<<grid, 256, 0, st>>>(R[0], R[1]);
-  return check_launch("reduce_rank_kernel");
+}
+
+lora_status_t run_rank2d(const void* Z, int64_t F, int64_t mtok, int r, int RP, const void* rb, const void* cb_hi,
+                         const void* cb_lo, int64_t ld_cb, const Rank2dSplit& sp, float* row_partial,
+                         float* col_partial, const RankOut& row_out, const RankOut& col_out, uint32_t* status,
+                         cudaStream_t st) {
+  const bool row = rb != nullptr, col = cb_hi != nullptr;
+  Rank2dParams p;
+  std::memset(&p, 0, sizeof(p));
+  bool ok = make_tm(&p.tm_z, Z, F, mtok, F, 64, 128);
+  if (row) ok = ok && make_tm(&p.tm_rb, rb, F, r, F, 64, RP);
+  if (col) ok = ok && make_tm(&p.tm_cb[0], cb_hi, mtok, r, ld_cb, 64, RP) && make_tm(&p.tm_cb[1], cb_lo, mtok, r, ld_cb, 64, RP);
+  if (!ok) return LORA_ERR_CUDA;
+  p.mtok = static_cast<int>(mtok);
+  p.F = static_cast<int>(F);
+  p.m_tiles = static_cast<int>(ceil_div(mtok, 128));
+  p.f_blocks = static_cast<int>(ceil_div(F, 128));
+  p.a_tiles = sp.a;
+  p.b_blocks = sp.b;
+  p.fs = sp.fs;
+  p.row_partial = sp.fs > 1 ? row_partial : nullptr;
+  p.col_partial = sp.ts > 1 ? col_partial : nullptr;
+  p.row_out = row_out;
+  p.col_out = col_out;
+  p.status = status;
+  const int grid = sp.ts * sp.fs;
+  lora_status_t rs;
+  if (row && col) rs = launch_rank2d_rp<true, true>(RP, p, grid, st);
+  else if (col) rs = launch_rank2d_rp<false, true>(RP, p, grid, st);
+  else return LORA_ERR_UNSUPPORTED;
+  LORA_TRY(rs);
+  RankReduceJob R[2];
+  int n = 0;
+  if (row && sp.fs > 1) {
+    R[n].partial = row_partial;
+    R[n].splits = sp.fs;
+    R[n].rows_pad = p.m_tiles * 128;
+    R[n].RP = RP;
+    R[n].out = row_out;
+    ++n;
+  }
+  if (col && sp.ts > 1) {
+    R[n].partial = col_partial;
+    R[n].splits = sp.ts;
+    R[n].rows_pad = p.f_blocks * 128;
+    R[n].RP = RP;
+    R[n].out = col_out;
+    ++n;
+  }
+  return launch_reduce(R, n, st);
 }
 
 // T_j = X A_j^T written to `out` (split K finished in place).
@@ -453,6 +573,24 @@ lora_status_t launch_mma_any(bool pair, const MmaParams& p, int sms, cudaStream_
   return pair ? launch_mma<true, kBwd, kNPair, kEpi>(p, sms, st) : launch_mma<false, kBwd, kNPair, kEpi>(p, sms, st);
 }
 
+// Failure-detection self-test: one thread waits, through the library's
+// bounded mbarrier wait, for a phase that nothing completes.  The wait gives
+// up after `limit` cycles and ORs kStatusWaitTimeout into the status word.
+__global__ void selftest_wait_kernel(uint32_t* status, long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    AbortCtl ctl{&flag, status};
+    mbar_wait(&bar, 0u, ctl, limit);
+  }
+}
+
 lora_status_t common_checks(const lora_linear_desc* d, void* ws, size_t ws_bytes, size_t need, DevInfo* dev) {
   LORA_TRY(check_desc(d));
   LORA_TRY(device_info(dev));
@@ -507,6 +645,18 @@ lora_status_t lora_linear_timing_read(double* fwd_ms, uint64_t* fwd_launches, do
   return LORA_OK;
 }
 
+lora_status_t lora_linear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_log2,
+                                                void* stream) {
+  if (workspace == nullptr || workspace_bytes < kHeaderBytes || !aligned16(workspace)) return LORA_ERR_WORKSPACE;
+  if (limit_log2 < 10 || limit_log2 > 30) return LORA_ERR_INVALID_ARG;
+  DevInfo dev;
+  LORA_TRY(device_info(&dev));
+  if (dev.major != 10 || dev.minor != 0) return LORA_ERR_ARCH;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(workspace),
+                                                                        1ll << limit_log2);
+  return check_launch("selftest_wait_kernel");
+}
+
 const char* lora_status_string(lora_status_t s) {
   switch (s) {
     case LORA_OK: return "ok";
@@ -523,12 +673,15 @@ const char* lora_status_string(lora_status_t s) {
 
 size_t lora_linear_workspace_size(const lora_linear_desc* desc, int for_backward) {
   if (check_desc(desc) != LORA_OK) return 0;
-  return make_plan(desc, for_backward != 0).total;
+  const size_t fwd = make_plan(desc, false).total;
+  if (for_backward == 0) return fwd;
+  const size_t bwd = make_plan(desc, true).total;
+  return bwd > fwd ? bwd : fwd;     // one workspace sized for the backward serves both
 }
 
 lora_status_t lora_linear_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
-  if (workspace == nullptr || workspace_bytes < kStatusBytes) return LORA_ERR_WORKSPACE;
-  if (cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (workspace == nullptr || workspace_bytes < kHeaderBytes) return LORA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return cuda_error("cudaMemsetAsync");
   return LORA_OK;
 }
@@ -563,23 +716,25 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const int np = P.np, RP = P.RP;
+  (void)RP;
   const int64_t M = d->M, r = d->r;
 
-  if (M <= kSmallMMax && r > 0 && !swiglu) {
-    // Few tokens: bound by reading W once; split K over a thread-block cluster.
+  if (P.small_m && dev.sms >= kTargetCtas) {
+    // Few tokens: bound by reading W once; stream-K over all SMs.
+    const int nt = P.sm_nt;
     SmallMParams q;
     std::memset(&q, 0, sizeof(q));
-    bool ok = make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128) &&
-              make_tm(&q.tm_x, X, d->d_in, M, d->d_in, 64, 128) && make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, RP);
-    if (!ok) return LORA_ERR_CUDA;
-    const int slices = static_cast<int>(ceil_div(d->d_out, 128));
-    const int nkb = static_cast<int>(ceil_div(d->d_in, 64));
-    int S = 1;
-    while (S < 8 && slices * S * 2 <= kTargetCtas && S * 2 <= nkb) S *= 2;
+    if (!make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128) ||
+        !make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, 128) ||
+        !make_tm(&q.tm_x, X, d->d_in, M, d->d_in, 64, static_cast<uint32_t>(nt)))
+      return LORA_ERR_CUDA;
     q.B = static_cast<const __nv_bfloat16*>(B);
     q.Y = static_cast<__nv_bfloat16*>(Y);
     q.T_save = T_save;
     q.Z_save = d->act == LORA_ACT_SILU ? Z_save : nullptr;
+    q.t_buf = reinterpret_cast<float*>(ws + P.sm_t_buf);
+    q.d_part = reinterpret_cast<float*>(ws + P.sm_d_part);
+    q.counters = reinterpret_cast<uint32_t*>(ws + kStatusBytes);
     q.status = status;
     q.M = static_cast<int>(M);
     q.d_in = static_cast<int>(d->d_in);
@@ -587,11 +742,14 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     q.r = static_cast<int>(r);
     q.s = d->s;
     q.act = d->act;
-    q.splits = S;
-    q.kb_per_split = (nkb + S - 1) / S;
-    const int nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-    LORA_LOG("small_m M=%d nt=%d RP=%d slices=%d splits=%d", (int)M, nt, RP, slices, S);
-    const cudaError_t e = launch_small_m(q, nt, RP, slices, st);
+    q.slices = P.sm.slices;
+    q.nkc = P.sm.nkc;
+    q.run = P.sm.run;
+    q.max_seg = P.sm.max_seg;
+    const int grid = P.sm.n_w;
+    LORA_LOG("small_m M=%d nt=%d slices=%d nkc=%d run=%d grid=%d max_seg=%d", (int)M, nt, q.slices, q.nkc, q.run,
+             grid, q.max_seg);
+    const cudaError_t e = launch_small_m(q, nt, grid, st);
     if (e != cudaSuccess) {
       LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
       g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -671,6 +829,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int np = P.np, RP = P.RP;
+  (void)RP;
   float* dAp[2] = {dA, dA_up};
   float* dBp[2] = {dB, dB_up};
   if (d->M == 0) {
@@ -693,10 +852,24 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
 
   // 1. dZ operands.  identity: dZ = dY (bf16, exact).  Otherwise dZ = dY * act'(Z)
-  //    as fp16 hi + lo, and fp16 copies of W for the dX product.
+  //    as fp16 hi + lo.  W^T for the dX product, in the dZ operand type.
   const void* dZ[2] = {dY, nullptr};
   const void* dZlo[2] = {nullptr, nullptr};
-  const void* Wmain[2] = {W, W_up};
+  {
+    const long long tiles = ceil_div(d->d_out, 64) * ceil_div(d->d_in, 64);
+    const int grid = static_cast<int>(tiles < static_cast<long long>(dev.sms) * 8 ? tiles : dev.sms * 8);
+    for (int j = 0; j < np; ++j) {
+      if (f16)
+        transpose_w_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Wp[j]),
+                                                         static_cast<int>(d->d_out), static_cast<int>(d->d_in),
+                                                         static_cast<__half*>(at(P.wt[j])), status);
+      else
+        transpose_w_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Wp[j]),
+                                                                static_cast<int>(d->d_out), static_cast<int>(d->d_in),
+                                                                static_cast<__nv_bfloat16*>(at(P.wt[j])), status);
+      LORA_TRY(check_launch("transpose_w_kernel"));
+    }
+  }
   if (f16) {
     const long long n = static_cast<long long>(M) * d->d_out;
     const int grid = grid_for(n / 8, 256, dev.sms);
@@ -710,33 +883,30 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
                                                   static_cast<__half*>(at(P.dz_hi[0])),
                                                   static_cast<__half*>(at(P.dz_lo[0])), nullptr, nullptr, status);
     LORA_TRY(check_launch("act_bwd_kernel"));
-    const long long nw = static_cast<long long>(d->d_out) * d->d_in;
     for (int j = 0; j < np; ++j) {
       dZ[j] = at(P.dz_hi[j]);
       dZlo[j] = at(P.dz_lo[j]);
-      convert_f16_kernel<<<grid_for(nw / 8, 256, dev.sms), 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<__half*>(at(P.w16[j])), nw, status);
-      LORA_TRY(check_launch("convert_f16_kernel"));
-      Wmain[j] = at(P.w16[j]);
     }
   }
 
-  // 2. B^T and (s T)^T hi/lo (from the saved T, or a rank pass recomputing T),
-  //    in the dZ operand type.
+  // 2. B^T, A^T and (s T)^T hi/lo (from the saved T, or a rank pass recomputing
+  //    T); B^T and (s T)^T in the dZ operand type.
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
       const float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r : nullptr;
-      const long long n = static_cast<long long>(d->d_out) * r + (Tj ? static_cast<long long>(M) * r : 0);
+      const long long n = static_cast<long long>(d->d_out + d->d_in) * r + (Tj ? static_cast<long long>(M) * r : 0);
+      const __nv_bfloat16* Aj = static_cast<const __nv_bfloat16*>(Ap[j]);
+      __nv_bfloat16* Atj = static_cast<__nv_bfloat16*>(at(P.at_[j]));
       if (f16)
         bwd_prep_kernel<__half><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
-            static_cast<__half*>(at(P.bt[j])), Tj, M, d->s, static_cast<__half*>(at(P.tt_hi[j])),
-            static_cast<__half*>(at(P.tt_lo[j])), M8, status);
+            static_cast<__half*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
+            static_cast<__half*>(at(P.tt_hi[j])), static_cast<__half*>(at(P.tt_lo[j])), M8, status);
       else
         bwd_prep_kernel<__nv_bfloat16><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
-            static_cast<__nv_bfloat16*>(at(P.bt[j])), Tj, M, d->s, static_cast<__nv_bfloat16*>(at(P.tt_hi[j])),
-            static_cast<__nv_bfloat16*>(at(P.tt_lo[j])), M8, status);
+            static_cast<__nv_bfloat16*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
+            static_cast<__nv_bfloat16*>(at(P.tt_hi[j])), static_cast<__nv_bfloat16*>(at(P.tt_lo[j])), M8, status);
       LORA_TRY(check_launch("bwd_prep_kernel"));
       if (Tj == nullptr) {
         RankOut o = rank_out(M, r);
@@ -748,8 +918,21 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
         LORA_TRY(rank_T(d, P, X, Ap[j], o, ws, status, st));
       }
     }
-    // 3. U = dZ B by a rank pass: bf16 s U (LoRA K-block of dX) and (s U)^T hi/lo (dA)
-    for (int j = 0; j < np; ++j) {
+    // 3. U = dZ B by a rank pass: bf16 s U (LoRA K-block of dX) and (s U)^T hi/lo (dA).
+    //    Identity with r <= 32: the same pass over dZ = dY also gives dB = dZ^T (sT).
+    if (P.dual) {
+      RankOut uo = rank_out(M, r);
+      uo.s16 = static_cast<__nv_bfloat16*>(at(P.s16[0]));
+      uo.hi = at(P.ut_hi[0]);
+      uo.lo = at(P.ut_lo[0]);
+      uo.ld = M8;
+      uo.scale = d->s;
+      RankOut bo = rank_out(static_cast<int>(d->d_out), r);
+      bo.f32 = dBp[0];
+      LORA_TRY(run_rank2d(dZ[0], d->d_out, M, r, RP, at(P.bt[0]), at(P.tt_hi[0]), at(P.tt_lo[0]), M8, P.sp_dual,
+                          static_cast<float*>(at(P.part_u)), static_cast<float*>(at(P.part_b)), uo, bo, status, st));
+    }
+    for (int j = 0; j < np && !P.dual; ++j) {
       RankJob J;
       J.f16 = f16;
       J.a[0] = dZ[j];
@@ -784,12 +967,13 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     std::memset(&p, 0, sizeof(p));
     const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
+    const uint32_t brows = pair ? 128 : 256;   // N-side rows per CTA box
     for (int j = 0; j < np; ++j) {
       ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
-      ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_in, d->d_out, d->d_in, 64, 64, f16);
+      ok = ok && make_tm(&p.tm_w[j], at(P.wt[j]), d->d_out, d->d_in, d->d_out, 64, brows, f16);
       if (r > 0) {
         ok = ok && make_tm(&p.tm_la[j], at(P.s16[j]), r, M, r, 64, 128);
-        ok = ok && make_tm(&p.tm_lb[j], Ap[j], d->d_in, r, d->d_in, 64, 64);
+        ok = ok && make_tm(&p.tm_lb[j], at(P.at_[j]), r, d->d_in, r, 64, brows);
       }
     }
     if (!ok) return LORA_ERR_CUDA;
@@ -817,30 +1001,15 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   }
   if (r == 0) return LORA_OK;
 
-  // 5. dA^T = X^T (s U) and dB = dZ^T (s T), hi/lo operands, split over tokens
+  // 5. dA^T = X^T (s U) (hi/lo operand) in one pass over X; without the fused
+  //    pass above, dB = dZ^T (s T) too, hi/lo operands, split over tokens
   for (int j = 0; j < np; ++j) {
-    RankJob Ja;
-    Ja.a_mn = true;
-    Ja.a[0] = X;
-    Ja.a_inner = d->d_in;
-    Ja.a_outer = M;
-    Ja.a_ld = d->d_in;
-    Ja.b[0] = at(P.ut_hi[j]);
-    Ja.b[1] = at(P.ut_lo[j]);
-    Ja.nb = 2;
-    Ja.b_inner = M;
-    Ja.b_ld = M8;
-    Ja.npairs = 2;
-    Ja.pb[1] = 1;
-    Ja.rows = static_cast<int>(d->d_in);
-    Ja.K = M;
-    Ja.partial = static_cast<float*>(at(P.part_a));
-    Ja.splits = P.splits_a;
-    Ja.out = rank_out(static_cast<int>(d->d_in), r);
-    Ja.out.f32 = dAp[j];
-    Ja.out.transpose_f32 = 1;
-    LORA_TRY(run_rank_gemm(Ja, RP, r, status, st));
-
+    RankOut ao = rank_out(static_cast<int>(d->d_in), r);
+    ao.f32 = dAp[j];
+    ao.transpose_f32 = 1;
+    LORA_TRY(run_rank2d(X, d->d_in, M, r, RP, nullptr, at(P.ut_hi[j]), at(P.ut_lo[j]), M8, P.sp_a, nullptr,
+                        static_cast<float*>(at(P.part_a)), rank_out(M, r), ao, status, st));
+    if (P.dual) continue;
     RankJob Jb;
     Jb.a_mn = true;
     Jb.f16 = f16;
@@ -867,7 +1036,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     Jb.out = rank_out(static_cast<int>(d->d_out), r);
     Jb.out.f32 = dBp[j];
     LORA_TRY(run_rank_gemm(Jb, RP, r, status, st));
-    LORA_TRY(finish_rank(&Ja, &Jb, RP, st));
+    LORA_TRY(finish_rank(&Jb, nullptr, RP, st));
   }
   return LORA_OK;
 }
@@ -918,9 +1087,9 @@ lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, 
   }
   void* ws = nullptr;
   LORA_TRY(noalloc_scratch(&ws));
-  // The status word must start at zero; everything else the forward writes
-  // before it reads.
-  if (cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // The header (status word, slice counters) must start at zero; everything
+  // else the forward writes before it reads.
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return cuda_error("cudaMemsetAsync(scratch status)");
   return lora_linear_fwd(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, ws, LORA_LINEAR_NOALLOC_SCRATCH_BYTES,
                          stream);

@@ -252,47 +252,81 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   }
 }
 
-// Fixed-order sum of split-K partials, one thread per result row, for up to
-// two independent jobs in one launch (blockIdx.y selects the job).
+// Fixed-order sum of split-K partials for up to two independent jobs in one
+// launch.
 struct RankReduceJob {
   const float* partial;   // [splits][rows_pad][RP]
   int splits, rows_pad, RP;
   RankOut out;
 };
 
-// One element of a finished rank result (same outputs as emit_rank_row).
-__device__ __forceinline__ void emit_rank_elem(float v, int row, int c, const RankOut& o) {
-  if (o.f32 != nullptr) {
-    if (o.transpose_f32) o.f32[static_cast<size_t>(c) * o.rows + row] = v;
-    else o.f32[static_cast<size_t>(row) * o.r + c] = v;
-  }
-  if (o.s16 != nullptr) o.s16[static_cast<size_t>(row) * o.r + c] = __float2bfloat16_rn(o.scale * v);
-  if (o.hi != nullptr) {
-    const float x = o.scale * v;
-    const size_t i = static_cast<size_t>(c) * o.ld + row;
-    if (o.hilo_f16) {
-      const __half h = __float2half_rn(x);
-      static_cast<__half*>(o.hi)[i] = h;
-      static_cast<__half*>(o.lo)[i] = __float2half_rn(x - __half2float(h));
-    } else {
-      const __nv_bfloat16 h = __float2bfloat16_rn(x);
-      static_cast<__nv_bfloat16*>(o.hi)[i] = h;
-      static_cast<__nv_bfloat16*>(o.lo)[i] = __float2bfloat16_rn(x - __bfloat162float(h));
-    }
-  }
-}
+// Blocks of 64 result rows (grid-stride over row blocks; blockIdx.y selects
+// the job).  Splits are summed in order into a shared-memory tile with the
+// column fastest (the partials' layout), then row-major outputs are written
+// column-fastest and transposed outputs row-fastest, so every global access
+// is coalesced.
+constexpr int kReduceRows = 64;
 
-// One thread per (row, column) element; grid-stride; splits summed in order.
-__global__ void reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
+__global__ void __launch_bounds__(256) reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
   const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
-  const long long n = static_cast<long long>(J.out.rows) * J.out.r;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int row = static_cast<int>(i / J.out.r);
-    const int c = static_cast<int>(i % J.out.r);
-    float acc = 0.0f;
-    for (int sp = 0; sp < J.splits; ++sp) acc += J.partial[(static_cast<size_t>(sp) * J.rows_pad + row) * J.RP + c];
-    emit_rank_elem(acc, row, c, J.out);
+  __shared__ float tile[kReduceRows][65];
+  const int r = J.out.r;
+  const RankOut& o = J.out;
+  const int nblk = (J.out.rows + kReduceRows - 1) / kReduceRows;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+    const int row0 = blk * kReduceRows;
+    const int nrows = J.out.rows - row0 < kReduceRows ? J.out.rows - row0 : kReduceRows;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nrows * r; i += blockDim.x) {
+      const int rr = i / r, c = i - rr * r;
+      // loads in batches of 8 (independent, in flight together), sums in split order
+      const float* src = J.partial + static_cast<size_t>(row0 + rr) * J.RP + c;
+      const size_t stride = static_cast<size_t>(J.rows_pad) * J.RP;
+      float acc = 0.0f;
+      int sp = 0;
+      for (; sp + 8 <= J.splits; sp += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = src[(sp + u) * stride];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc += v[u];
+      }
+      for (; sp < J.splits; ++sp) acc += src[sp * stride];
+      tile[rr][c] = acc;
+    }
+    __syncthreads();
+    // row-major outputs: column fastest
+    if ((o.f32 != nullptr && !o.transpose_f32) || o.s16 != nullptr) {
+      for (int i = threadIdx.x; i < nrows * r; i += blockDim.x) {
+        const int rr = i / r, c = i - rr * r;
+        const float v = tile[rr][c];
+        const size_t idx = static_cast<size_t>(row0 + rr) * r + c;
+        if (o.f32 != nullptr && !o.transpose_f32) o.f32[idx] = v;
+        if (o.s16 != nullptr) o.s16[idx] = __float2bfloat16_rn(o.scale * v);
+      }
+    }
+    // transposed outputs: row fastest
+    if ((o.f32 != nullptr && o.transpose_f32) || o.hi != nullptr) {
+      for (int i = threadIdx.x; i < nrows * r; i += blockDim.x) {
+        const int c = i / nrows, rr = i - c * nrows;
+        const float v = tile[rr][c];
+        const int row = row0 + rr;
+        if (o.f32 != nullptr && o.transpose_f32) o.f32[static_cast<size_t>(c) * o.rows + row] = v;
+        if (o.hi != nullptr) {
+          const float x = o.scale * v;
+          const size_t k = static_cast<size_t>(c) * o.ld + row;
+          if (o.hilo_f16) {
+            const __half h = __float2half_rn(x);
+            static_cast<__half*>(o.hi)[k] = h;
+            static_cast<__half*>(o.lo)[k] = __float2half_rn(x - __half2float(h));
+          } else {
+            const __nv_bfloat16 h = __float2bfloat16_rn(x);
+            static_cast<__nv_bfloat16*>(o.hi)[k] = h;
+            static_cast<__nv_bfloat16*>(o.lo)[k] = __float2bfloat16_rn(x - __bfloat162float(h));
+          }
+        }
+      }
+    }
   }
 }
 
@@ -304,25 +338,33 @@ __device__ __forceinline__ float from16(__nv_bfloat16 v) { return __bfloat162flo
 __device__ __forceinline__ float from16(__half v) { return __half2float(v); }
 constexpr float kF16Max = 65504.0f;
 
-// Backward preparation in one launch: B^T ([r x d_out], bf16 or fp16) and the
+// Backward preparation in one launch: B^T ([r x d_out], bf16 or fp16), A^T
+// ([d_in x r], bf16: the K-major N-side operand of the dX LoRA block) and the
 // transposed hi/lo split of s*T ([r x ld]) from the forward's fp32 T.
 template <typename T>
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r, T* __restrict__ Bt,
+                                const __nv_bfloat16* __restrict__ A, int d_in, __nv_bfloat16* __restrict__ At,
                                 const float* __restrict__ Tsave, int M, float s, T* __restrict__ t_hi,
                                 T* __restrict__ t_lo, int ld, uint32_t* status) {
   const long long nb = static_cast<long long>(d_out) * r;
+  const long long na = static_cast<long long>(d_in) * r;
   const long long nt = Tsave != nullptr ? static_cast<long long>(M) * r : 0;
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nb + nt;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nb + na + nt;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    if (i < nb) {
+    if (i >= nb && i < nb + na) {
+      const long long k = i - nb;                 // At[k] = A[c][di], k = di * r + c
+      const int di = static_cast<int>(k / r);
+      const int c = static_cast<int>(k % r);
+      At[k] = A[static_cast<size_t>(c) * d_in + di];
+    } else if (i < nb) {
       const int c = static_cast<int>(i / d_out);
       const int jd = static_cast<int>(i % d_out);
       const float v = __bfloat162float(B[static_cast<size_t>(jd) * r + c]);
       Bt[i] = to16<T>(v);
       if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
     } else {
-      const long long k = i - nb;
+      const long long k = i - nb - na;
       const int c = static_cast<int>(k / M);
       const int m = static_cast<int>(k % M);
       const float v = s * Tsave[static_cast<size_t>(m) * r + c];
@@ -335,25 +377,72 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, 
   if (bad && status) atomicOr(status, kStatusF16Range);
 }
 
-// bf16 -> fp16 copy of a weight matrix, 8 elements per step.  bf16's 8-bit
-// significand fits fp16's 11 bits, so values inside fp16's normal range
-// convert exactly; |w| > 65504 flags the status word.
-__global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, long long n,
-                                   uint32_t* status) {
-  const long long nv = n / 8;
+// W [rows x cols] bf16 -> Wt [cols x rows] in T (bf16, or fp16: exact for
+// |w| <= 65504, else the status bit), so that the dX product reads W K-major.
+// 64 x 64 tiles through shared memory: each thread loads the same 8 columns of
+// two adjacent rows and packs them pairwise into 32-bit words
+// tile[column][row pair], which makes both the shared-memory writes and the
+// row-contiguous reads conflict-free and every global access 16 bytes.
+// rows and cols are multiples of 8.
+template <typename T>
+__global__ void __launch_bounds__(256) transpose_w_kernel(const __nv_bfloat16* __restrict__ W, int rows, int cols,
+                                                          T* __restrict__ Wt, uint32_t* status) {
+  __shared__ uint32_t tile[64][33];
+  const int tiles_c = (cols + 63) / 64;
+  const long long ntiles = static_cast<long long>((rows + 63) / 64) * tiles_c;
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
-    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
-    __align__(16) __half h[8];
+  for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int r0 = static_cast<int>(t / tiles_c) * 64;
+    const int c0 = static_cast<int>(t % tiles_c) * 64;
+    __syncthreads();
+    {
+      const int pr = threadIdx.x & 31;          // row pair
+      const int cv = (threadIdx.x >> 5) * 8;    // 8 columns
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
+      const int ra = r0 + 2 * pr;
+      if (c0 + cv < cols) {
+        if (ra < rows) a = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(ra) * cols + c0 + cv);
+        if (ra + 1 < rows) b = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(ra + 1) * cols + c0 + cv);
+      }
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float f = __bfloat162float(b[e]);
-      h[e] = __float2half_rn(f);
-      if (!(fabsf(f) <= kF16Max)) bad = true;
+      for (int e = 0; e < 4; ++e) {
+        // columns cv + 2e (low halves) and cv + 2e + 1 (high halves)
+        tile[cv + 2 * e][pr] = (av[e] & 0xffffu) | (bv[e] << 16);
+        tile[cv + 2 * e + 1][pr] = (av[e] >> 16) | (bv[e] & 0xffff0000u);
+      }
     }
-    reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(h);
+    __syncthreads();
+    {
+      const int qv = threadIdx.x & 7;           // 8 output elements: input rows r0 + 8 qv ...
+      const int cc0 = threadIdx.x >> 3;         // output rows (input columns) cc0, cc0 + 32
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cc = cc0 + 32 * h;
+        if (c0 + cc < cols && r0 + 8 * qv < rows) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) w[k] = tile[cc][4 * qv + k];
+          uint4 o;
+          if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+            o = make_uint4(w[0], w[1], w[2], w[3]);
+          } else {
+            uint32_t hv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float lo = __uint_as_float(w[k] << 16);
+              const float hi = __uint_as_float(w[k] & 0xffff0000u);
+              if (!(fabsf(lo) <= kF16Max) || !(fabsf(hi) <= kF16Max)) bad = true;
+              const __half2 h2 = __floats2half2_rn(lo, hi);
+              hv[k] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            o = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          }
+          *reinterpret_cast<uint4*>(Wt + static_cast<size_t>(c0 + cc) * rows + r0 + 8 * qv) = o;
+        }
+      }
+    }
   }
   if (bad && status) atomicOr(status, kStatusF16Range);
 }

@@ -74,13 +74,14 @@ struct AbortCtl {
 // Wait for the phase with parity `parity` of `bar` to complete.  Returns false
 // if the CTA is aborting or the wait exceeded kWaitLimitCycles (then the status
 // word and the CTA abort flag are set).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const AbortCtl& ctl) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const AbortCtl& ctl,
+                                          long long limit_cycles = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*ctl.flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit_cycles) {
       if (ctl.status) atomicOr(ctl.status, kStatusWaitTimeout);
       *ctl.flag = 1u;
       return false;
@@ -142,6 +143,28 @@ __device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t p
   asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy)
                : "memory");
+}
+
+// Named barrier `id` over `n` threads that also ANDs a predicate: every
+// participant gets the same answer, so a group can leave a loop together
+// when any of its bounded waits gave up.
+template <int id, int n>
+__device__ __forceinline__ bool bar_sync_and(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "n"(id), "n"(n)
+      : "memory");
+  return r != 0u;
+}
+
+template <int id, int n>
+__device__ __forceinline__ void bar_sync_named() {
+  asm volatile("barrier.cta.sync %0, %1;" ::"n"(id), "n"(n) : "memory");
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy

@@ -89,3 +89,10 @@ def test_no_gpu_means_cuda_error_not_crash(lib):
         pytest.skip("a GPU is present")
     ok = lib.make_desc(64, 256, 256, 8, 2.0, "identity")
     assert _fwd(lib, ok) == 6                         # LORA_ERR_CUDA: no device
+
+
+def test_selftest_rejects_bad_arguments_without_launching(lib):
+    assert lib.lora_linear_selftest_wait_timeout(None, 1 << 20, 16, None) == 5   # WORKSPACE
+    assert lib.lora_linear_selftest_wait_timeout(16, 64, 16, None) == 5          # below the header
+    assert lib.lora_linear_selftest_wait_timeout(16, 1 << 20, 5, None) == 1      # INVALID_ARG
+    assert lib.lora_linear_selftest_wait_timeout(16, 1 << 20, 31, None) == 1
