@@ -24,6 +24,7 @@ using namespace lora;
 
 constexpr int kAbiVersion = 1;
 constexpr int kTargetCtas = 148;   // SM count of a B200; sets split-K widths
+constexpr int64_t kKMajorMinTokens = 12288;   // dX from a W^T copy at and above this many tokens
 constexpr size_t kStatusBytes = 256;
 // Workspace header, zero at rest: the status block, then the arrival counters
 // of the few-token forward (one per 128-row slice of [A ; W], plus two).
@@ -33,14 +34,15 @@ constexpr size_t kHeaderBytes = kStatusBytes + kCounterWords * 4;
 // ---------------------------------------------------------------------------
 // debug logging (LORA_LINEAR_DEBUG=1)
 // ---------------------------------------------------------------------------
-bool debug_on() {
+int debug_level() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("LORA_LINEAR_DEBUG");
-    v = (e && e[0] && e[0] != '0') ? 1 : 0;
+    v = (e && e[0] >= '1' && e[0] <= '9') ? e[0] - '0' : 0;
   }
-  return v == 1;
+  return v;
 }
+bool debug_on() { return debug_level() >= 1; }
 #define LORA_LOG(...)                                  \
   do {                                                 \
     if (debug_on()) {                                  \
@@ -139,8 +141,11 @@ struct Plan {
   size_t tt_hi[2] = {}, tt_lo[2] = {};       // (s*T)^T hi / lo [r x M8] (bwd, dB)
   size_t ut_hi[2] = {}, ut_lo[2] = {};       // (s*U)^T hi / lo [r x M8] (bwd, dA)
   size_t dz_hi[2] = {}, dz_lo[2] = {};     // activation backward: fp16 dZ operands
-  size_t wt[2] = {};                        // W^T [d_in x d_out] (bf16, fp16 with an activation): dX's K-major operand
-  size_t at_[2] = {};                       // A^T [d_in x r] bf16: the dX LoRA block's K-major operand
+  // dX's N-side operands: K-major copies W^T [d_in x d_out], A^T [d_in x r]
+  // (kmajor), or W read in place MN-major (an fp16 copy with an activation)
+  bool kmajor = false;
+  size_t wt[2] = {};
+  size_t at_[2] = {};
   size_t part_t = 0, part_u = 0, part_a = 0, part_b = 0;   // split-K partials
   // backward rank passes on rank2d_kernel: U and dB from one read of dZ
   // (identity, r <= 32), dA over X
@@ -207,8 +212,11 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     P.total = off;
     return P;
   }
+  // The W^T copy pays for itself when the dX GEMM is long against one pass
+  // over W: many tokens (measured: M = 16384 gains, M = 8192 does not).
+  P.kmajor = d->act == LORA_ACT_IDENTITY && M >= kKMajorMinTokens;
   for (int j = 0; j < P.np; ++j) {
-    P.wt[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
+    if (P.kmajor || P.act_f16) P.wt[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
     if (P.act_f16) {
       P.dz_hi[j] = take(static_cast<size_t>(M) * d->d_out * 2);
       P.dz_lo[j] = take(static_cast<size_t>(M) * d->d_out * 2);
@@ -216,7 +224,7 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
   }
   if (r > 0) {
     for (int j = 0; j < P.np; ++j) {
-      P.at_[j] = take(static_cast<size_t>(d->d_in) * r * 2);
+      if (P.kmajor) P.at_[j] = take(static_cast<size_t>(d->d_in) * r * 2);
       P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
       P.tt_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
       P.tt_lo[j] = take(static_cast<size_t>(r) * P.M8 * 2);
@@ -225,7 +233,7 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     }
     const int64_t tiles_a = ceil_div(d->d_in, 128), tiles_b = ceil_div(d->d_out, 128);
     const int64_t nkb_tok = ceil_div(M > 0 ? M : 1, 64);
-    P.dual = d->act == LORA_ACT_IDENTITY && P.RP <= 32;
+    P.dual = d->act == LORA_ACT_IDENTITY;
     if (P.dual) {
       P.sp_dual = rank2d_split(static_cast<int>(tiles_m), static_cast<int>(tiles_b), P.RP, true, true,
                                rank2d_max_rb(P.RP), kTargetCtas);
@@ -749,13 +757,46 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     const int grid = P.sm.n_w;
     LORA_LOG("small_m M=%d nt=%d slices=%d nkc=%d run=%d grid=%d max_seg=%d", (int)M, nt, q.slices, q.nkc, q.run,
              grid, q.max_seg);
+    // LORA_LINEAR_DEBUG=2: per-CTA phase stamps, printed after the launch
+    // (synchronises the stream; for debugging only).
+    static unsigned long long* trace = nullptr;
+    if (debug_level() >= 2 && trace == nullptr &&
+        cudaMalloc(&trace, sizeof(unsigned long long) * 1024 * kSmTracePoints) != cudaSuccess)
+      trace = nullptr;
+    if (debug_level() >= 2 && trace != nullptr && grid <= 1024) {
+      q.trace = trace;
+      cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTracePoints, st);
+    }
     const cudaError_t e = launch_small_m(q, nt, grid, st);
     if (e != cudaSuccess) {
       LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
       g_launches.fetch_add(1, std::memory_order_relaxed);
       return LORA_ERR_CUDA;
     }
-    return check_launch("small_m_kernel");
+    const lora_status_t ls = check_launch("small_m_kernel");
+    if (q.trace != nullptr && cudaStreamSynchronize(st) == cudaSuccess) {
+      std::vector<unsigned long long> h(static_cast<size_t>(grid) * kSmTracePoints);
+      cudaMemcpy(h.data(), trace, h.size() * sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+      unsigned long long t0 = ~0ull;
+      for (int b = 0; b < grid; ++b) t0 = h[b * kSmTracePoints] && h[b * kSmTracePoints] < t0 ? h[b * kSmTracePoints] : t0;
+      static const char* names[kSmTracePoints] = {"entry", "first_issue", "first_data", "last_mma", "published",
+                                                  "combined", "exit"};
+      for (int k = 0; k < kSmTracePoints; ++k) {
+        double mn = 1e30, mx = 0, sum = 0;
+        int n = 0;
+        for (int b = 0; b < grid; ++b) {
+          const unsigned long long v = h[b * kSmTracePoints + k];
+          if (v == 0) continue;
+          const double us = (v - t0) * 1e-3;
+          mn = us < mn ? us : mn;
+          mx = us > mx ? us : mx;
+          sum += us;
+          ++n;
+        }
+        if (n) LORA_LOG("small_m trace %-12s n=%3d min %7.2f mean %7.2f max %7.2f us", names[k], n, mn, sum / n, mx);
+      }
+    }
+    return ls;
   }
 
   const void* Wp[2] = {W, W_up};
@@ -852,22 +893,20 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
 
   // 1. dZ operands.  identity: dZ = dY (bf16, exact).  Otherwise dZ = dY * act'(Z)
-  //    as fp16 hi + lo.  W^T for the dX product, in the dZ operand type.
+  //    as fp16 hi + lo.  W for the dX product: a K-major copy W^T (kmajor), or
+  //    read in place (an fp16 copy with an activation).
   const void* dZ[2] = {dY, nullptr};
   const void* dZlo[2] = {nullptr, nullptr};
-  {
+  const void* Wmain[2] = {W, W_up};
+  if (P.kmajor) {
     const long long tiles = ceil_div(d->d_out, 64) * ceil_div(d->d_in, 64);
     const int grid = static_cast<int>(tiles < static_cast<long long>(dev.sms) * 8 ? tiles : dev.sms * 8);
     for (int j = 0; j < np; ++j) {
-      if (f16)
-        transpose_w_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Wp[j]),
-                                                         static_cast<int>(d->d_out), static_cast<int>(d->d_in),
-                                                         static_cast<__half*>(at(P.wt[j])), status);
-      else
-        transpose_w_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Wp[j]),
-                                                                static_cast<int>(d->d_out), static_cast<int>(d->d_in),
-                                                                static_cast<__nv_bfloat16*>(at(P.wt[j])), status);
+      transpose_w_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Wp[j]),
+                                                              static_cast<int>(d->d_out), static_cast<int>(d->d_in),
+                                                              static_cast<__nv_bfloat16*>(at(P.wt[j])), status);
       LORA_TRY(check_launch("transpose_w_kernel"));
+      Wmain[j] = at(P.wt[j]);
     }
   }
   if (f16) {
@@ -883,9 +922,14 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
                                                   static_cast<__half*>(at(P.dz_hi[0])),
                                                   static_cast<__half*>(at(P.dz_lo[0])), nullptr, nullptr, status);
     LORA_TRY(check_launch("act_bwd_kernel"));
+    const long long nw = static_cast<long long>(d->d_out) * d->d_in;
     for (int j = 0; j < np; ++j) {
       dZ[j] = at(P.dz_hi[j]);
       dZlo[j] = at(P.dz_lo[j]);
+      convert_f16_kernel<<<grid_for(nw / 8, 256, dev.sms), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<__half*>(at(P.wt[j])), nw, status);
+      LORA_TRY(check_launch("convert_f16_kernel"));
+      Wmain[j] = at(P.wt[j]);
     }
   }
 
@@ -894,9 +938,9 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
       const float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r : nullptr;
-      const long long n = static_cast<long long>(d->d_out + d->d_in) * r + (Tj ? static_cast<long long>(M) * r : 0);
+      const long long n = d->d_out + (P.kmajor ? d->d_in : 0) + (Tj ? M : 0);   // one thread per row
       const __nv_bfloat16* Aj = static_cast<const __nv_bfloat16*>(Ap[j]);
-      __nv_bfloat16* Atj = static_cast<__nv_bfloat16*>(at(P.at_[j]));
+      __nv_bfloat16* Atj = P.kmajor ? static_cast<__nv_bfloat16*>(at(P.at_[j])) : nullptr;
       if (f16)
         bwd_prep_kernel<__half><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
@@ -967,15 +1011,21 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     std::memset(&p, 0, sizeof(p));
     const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
-    const uint32_t brows = pair ? 128 : 256;   // N-side rows per CTA box
+    const uint32_t brows = pair ? 128 : 256;   // N-side rows per CTA box (K-major)
     for (int j = 0; j < np; ++j) {
       ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
-      ok = ok && make_tm(&p.tm_w[j], at(P.wt[j]), d->d_out, d->d_in, d->d_out, 64, brows, f16);
+      if (P.kmajor) {
+        ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_out, d->d_in, d->d_out, 64, brows, f16);
+      } else {
+        ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_in, d->d_out, d->d_in, 64, 64, f16);
+      }
       if (r > 0) {
         ok = ok && make_tm(&p.tm_la[j], at(P.s16[j]), r, M, r, 64, 128);
-        ok = ok && make_tm(&p.tm_lb[j], at(P.at_[j]), r, d->d_in, r, 64, brows);
+        if (P.kmajor) ok = ok && make_tm(&p.tm_lb[j], at(P.at_[j]), r, d->d_in, r, 64, brows);
+        else ok = ok && make_tm(&p.tm_lb[j], Ap[j], d->d_in, r, d->d_in, 64, 64);
       }
     }
+    p.b_mn = P.kmajor ? 0 : 1;
     if (!ok) return LORA_ERR_CUDA;
     p.M = M;
     p.N = static_cast<int>(d->d_in);

@@ -10,9 +10,10 @@
 // The up-projection thus runs on the tensor cores inside the same accumulator,
 // with no hand-off between the epilogue and the MMA issuer, which leaves the
 // tensor memory free for a double-buffered accumulator: 2 x 256 fp32 columns.
-// Every operand is K-major: the backward multiplies by transposed copies of W
-// and A that it writes first (W^T costs one read and one write of W, and the
-// tensor pipe then runs as in the forward; read MN-major it idled ~10 % more).
+// The backward reads W and A either in place as MN-major operands (b_mn = 1),
+// or as K-major copies W^T and A^T that it writes first (b_mn = 0): the copy
+// costs one read and one write of W, and the tensor pipe then runs as in the
+// forward, where the MN-major read left it idle ~10 % more often on q_proj.
 // The epilogue of tile i (drain, activation, bf16 store) overlaps the K-loop of
 // tile i + 1.
 //
@@ -44,9 +45,9 @@ enum MmaEpi : int { kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad
 
 struct MmaParams {
   CUtensorMap tm_a[2];    // M-side operand per pair      fwd: X            bwd: dZ_j
-  CUtensorMap tm_w[2];    // N-side operand per pair      fwd: W_j          bwd: W_j^T (K-major copy)
+  CUtensorMap tm_w[2];    // N-side operand per pair      fwd: W_j          bwd: W_j (b_mn) or W_j^T
   CUtensorMap tm_la[2];   // LoRA block, M side           s*T_j / s*U_j   bf16 [M x r]
-  CUtensorMap tm_lb[2];   // LoRA block, N side           fwd: B_j [d_out x r]   bwd: A_j^T [d_in x r]
+  CUtensorMap tm_lb[2];   // LoRA block, N side           fwd: B_j [d_out x r]   bwd: A_j (b_mn) or A_j^T
   int M, N, K;            // output rows / columns (per projection for SwiGLU fwd) / reduction per pair
   int lora_ksteps;        // 16-wide K steps of the LoRA block: ceil(r / 16); 0 = no LoRA block
   __nv_bfloat16* out;     // [M x N]
@@ -56,6 +57,7 @@ struct MmaParams {
   int group;              // raster group width (tiles)
   int group_along_n;      // 0: groups of `group` M tiles sweep all N tiles (the N-side operand stays in L2)
                           // 1: groups of `group` N tiles sweep all M tiles (the M-side operand stays in L2)
+  int b_mn;               // backward: N-side operands read MN-major (W [K x N], A [r x N]) instead of K-major copies
 };
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
@@ -204,6 +206,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               } else {
                 load(sb, &p.tm_w[0], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
               }
+            } else if (p.b_mn) {
+#pragma unroll
+              for (int b = 0; b < C::kBRows / 64; ++b)
+                load(sb + b * 8192, &p.tm_w[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, k0, pol_keep);
             } else {
               // W^T (K-major copy of W made by the backward): rows = outputs of dX
               load(sb, &p.tm_w[j], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
@@ -219,6 +225,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               } else {
                 load(sb, &p.tm_lb[0], fb, 0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
               }
+            } else if (p.b_mn) {
+#pragma unroll
+              for (int b = 0; b < C::kBRows / 64; ++b)
+                load(sb + b * 8192, &p.tm_lb[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, 0, pol_keep);
             } else {
               load(sb, &p.tm_lb[j], fb, 0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);   // A^T rows
             }
@@ -242,9 +252,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
     if (lane == 0 && leader) {
       constexpr bool kF16 = (kEpi == kMEpiGradF16);
       constexpr int kM = C::kTileM;
-      constexpr uint32_t kIdMain = idesc_mma(kM, 256, false, false, kF16);
-      // LoRA block: bf16 s*T/s*U against bf16 B (fwd) / A^T (bwd); every operand K-major
-      constexpr uint32_t kIdLora = idesc_mma(kM, C::kSwigluFwd ? 128 : 256, false, false, false);
+      // N-side operand MN-major only in a backward that reads W and A in place
+      const bool bmn = kBwd && p.b_mn != 0;
+      const uint32_t kIdMain = bmn ? idesc_mma(kM, 256, false, true, kF16) : idesc_mma(kM, 256, false, false, kF16);
+      // LoRA block: bf16 s*T/s*U against bf16 B (fwd) / A or A^T (bwd)
+      const uint32_t kIdLora = bmn ? idesc_mma(kM, 256, false, true, false)
+                                   : idesc_mma(kM, C::kSwigluFwd ? 128 : 256, false, false, false);
       constexpr uint16_t kBoth = 0x3;
       auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
         if constexpr (kPair) mma_bf16_pair(d, a, b, id, acc);
@@ -273,7 +286,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t db = sdesc_sw128(sb + kk * 32, 16, 1024);
+              const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
               mma(dacc, da, db, kIdMain, (blk == 0 && kk == 0) ? 0u : 1u);
             }
           } else {
@@ -281,7 +294,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             const uint32_t dcol = C::kSwigluFwd ? static_cast<uint32_t>(128 * j) : 0u;
             for (int kk = 0; kk < p.lora_ksteps; ++kk) {
               const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t db = sdesc_sw128(sb + kk * 32, 16, 1024);
+              const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
               mma(dacc + dcol, da, db, kIdLora, 1u);
             }
           }

@@ -260,39 +260,55 @@ struct RankReduceJob {
   RankOut out;
 };
 
-// Blocks of 64 result rows (grid-stride over row blocks; blockIdx.y selects
-// the job).  Splits are summed in order into a shared-memory tile with the
-// column fastest (the partials' layout), then row-major outputs are written
-// column-fastest and transposed outputs row-fastest, so every global access
-// is coalesced.
-constexpr int kReduceRows = 64;
+// Blocks of kReduceRows result rows (grid-stride over row blocks; blockIdx.y
+// selects the job).  Splits are summed in order into a shared-memory tile with
+// the column fastest (the partials' layout), each thread keeping up to
+// 2 elements x 8 splits of loads in flight; then row-major outputs are written
+// column-fastest and transposed outputs row-fastest, so every global access is
+// coalesced.
+constexpr int kReduceRows = 32;
 
-__global__ void __launch_bounds__(256) reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
+__global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
   const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
   __shared__ float tile[kReduceRows][65];
   const int r = J.out.r;
   const RankOut& o = J.out;
   const int nblk = (J.out.rows + kReduceRows - 1) / kReduceRows;
+  const size_t stride = static_cast<size_t>(J.rows_pad) * J.RP;   // between splits
+  constexpr int kEPT = 2;
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
     const int row0 = blk * kReduceRows;
     const int nrows = J.out.rows - row0 < kReduceRows ? J.out.rows - row0 : kReduceRows;
+    const int E = nrows * r;
     __syncthreads();
-    for (int i = threadIdx.x; i < nrows * r; i += blockDim.x) {
-      const int rr = i / r, c = i - rr * r;
-      // loads in batches of 8 (independent, in flight together), sums in split order
-      const float* src = J.partial + static_cast<size_t>(row0 + rr) * J.RP + c;
-      const size_t stride = static_cast<size_t>(J.rows_pad) * J.RP;
-      float acc = 0.0f;
-      int sp = 0;
-      for (; sp + 8 <= J.splits; sp += 8) {
-        float v[8];
+    for (int base = 0; base < E; base += 256 * kEPT) {
+      float acc[kEPT];
+      const float* src[kEPT];
+      bool in[kEPT];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = src[(sp + u) * stride];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc += v[u];
+      for (int e = 0; e < kEPT; ++e) {
+        const int i = base + static_cast<int>(threadIdx.x) + 256 * e;
+        in[e] = i < E;
+        const int rr = in[e] ? i / r : 0, c = in[e] ? i - rr * r : 0;
+        src[e] = J.partial + static_cast<size_t>(row0 + rr) * J.RP + c;
+        acc[e] = 0.0f;
       }
-      for (; sp < J.splits; ++sp) acc += src[sp * stride];
-      tile[rr][c] = acc;
+      for (int sp0 = 0; sp0 < J.splits; sp0 += 8) {
+        float v[kEPT][8];
+#pragma unroll
+        for (int e = 0; e < kEPT; ++e)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[e][u] = (in[e] && sp0 + u < J.splits) ? src[e][(sp0 + u) * stride] : 0.0f;
+#pragma unroll
+        for (int e = 0; e < kEPT; ++e)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[e] += v[e][u];      // split order; + 0 past the last split
+      }
+#pragma unroll
+      for (int e = 0; e < kEPT; ++e) {
+        const int i = base + static_cast<int>(threadIdx.x) + 256 * e;
+        if (in[e]) tile[i / r][i % r] = acc[e];
+      }
     }
     __syncthreads();
     // row-major outputs: column fastest
@@ -338,41 +354,81 @@ __device__ __forceinline__ float from16(__nv_bfloat16 v) { return __bfloat162flo
 __device__ __forceinline__ float from16(__half v) { return __half2float(v); }
 constexpr float kF16Max = 65504.0f;
 
-// Backward preparation in one launch: B^T ([r x d_out], bf16 or fp16), A^T
-// ([d_in x r], bf16: the K-major N-side operand of the dX LoRA block) and the
-// transposed hi/lo split of s*T ([r x ld]) from the forward's fp32 T.
+// Backward preparation in one launch, one thread per row of the small
+// operands (so that each thread moves whole 16-byte rows and every warp access
+// is coalesced): B^T ([r x d_out], bf16 or fp16), A^T ([d_in x r], bf16, the
+// K-major N-side operand of the dX LoRA block; skipped when At is null) and
+// the transposed hi/lo split of s*T ([r x ld]) from the forward's fp32 T
+// (skipped when Tsave is null).  r is a multiple of 8.
 template <typename T>
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r, T* __restrict__ Bt,
                                 const __nv_bfloat16* __restrict__ A, int d_in, __nv_bfloat16* __restrict__ At,
                                 const float* __restrict__ Tsave, int M, float s, T* __restrict__ t_hi,
                                 T* __restrict__ t_lo, int ld, uint32_t* status) {
-  const long long nb = static_cast<long long>(d_out) * r;
-  const long long na = static_cast<long long>(d_in) * r;
-  const long long nt = Tsave != nullptr ? static_cast<long long>(M) * r : 0;
+  const long long nb = d_out;
+  const long long na = At != nullptr ? d_in : 0;
+  const long long nt = Tsave != nullptr ? M : 0;
   bool bad = false;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nb + na + nt;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    if (i >= nb && i < nb + na) {
-      const long long k = i - nb;                 // At[k] = A[c][di], k = di * r + c
-      const int di = static_cast<int>(k / r);
-      const int c = static_cast<int>(k % r);
-      At[k] = A[static_cast<size_t>(c) * d_in + di];
-    } else if (i < nb) {
-      const int c = static_cast<int>(i / d_out);
-      const int jd = static_cast<int>(i % d_out);
-      const float v = __bfloat162float(B[static_cast<size_t>(jd) * r + c]);
-      Bt[i] = to16<T>(v);
-      if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
+    if (i < nb) {
+      const int jd = static_cast<int>(i);
+      for (int c0 = 0; c0 < r; c0 += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(B + static_cast<size_t>(jd) * r + c0);
+        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float f = __bfloat162float(b[e]);
+          Bt[static_cast<size_t>(c0 + e) * d_out + jd] = to16<T>(f);
+          if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(f) <= kF16Max)) bad = true;
+        }
+      }
+    } else if (i < nb + na) {
+      const int di = static_cast<int>(i - nb);
+      for (int c0 = 0; c0 < r; c0 += 8) {
+        __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = A[static_cast<size_t>(c0 + e) * d_in + di];
+        *reinterpret_cast<uint4*>(At + static_cast<size_t>(di) * r + c0) = *reinterpret_cast<const uint4*>(o);
+      }
     } else {
-      const long long k = i - nb - na;
-      const int c = static_cast<int>(k / M);
-      const int m = static_cast<int>(k % M);
-      const float v = s * Tsave[static_cast<size_t>(m) * r + c];
-      const T h = to16<T>(v);
-      t_hi[static_cast<size_t>(c) * ld + m] = h;
-      t_lo[static_cast<size_t>(c) * ld + m] = to16<T>(v - from16(h));
-      if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
+      const int m = static_cast<int>(i - nb - na);
+      for (int c0 = 0; c0 < r; c0 += 4) {
+        const float4 tv = *reinterpret_cast<const float4*>(Tsave + static_cast<size_t>(m) * r + c0);
+        const float t4[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v = s * t4[e];
+          const T h = to16<T>(v);
+          t_hi[static_cast<size_t>(c0 + e) * ld + m] = h;
+          t_lo[static_cast<size_t>(c0 + e) * ld + m] = to16<T>(v - from16(h));
+          if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
+        }
+      }
     }
+  }
+  if (bad && status) atomicOr(status, kStatusF16Range);
+}
+
+// bf16 -> fp16 copy of a weight matrix, 8 elements per step.  bf16's 8-bit
+// significand fits fp16's 11 bits, so values inside fp16's normal range
+// convert exactly; |w| > 65504 flags the status word.
+__global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, long long n,
+                                   uint32_t* status) {
+  const long long nv = n / 8;
+  bool bad = false;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+    __align__(16) __half h[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float f = __bfloat162float(b[e]);
+      h[e] = __float2half_rn(f);
+      if (!(fabsf(f) <= kF16Max)) bad = true;
+    }
+    reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(h);
   }
   if (bad && status) atomicOr(status, kStatusF16Range);
 }

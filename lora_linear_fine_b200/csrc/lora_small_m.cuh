@@ -54,7 +54,21 @@ struct SmallMParams {
   int slices, nkc;           // 128-row slices of [A ; W] (1 + ceil(d_out / 128)); 128-wide K chunks
   int run;                   // units per CTA
   int max_seg;               // partial slots per slice
+  unsigned long long* trace; // null, or [grid][kSmTracePoints] globaltimer stamps (debugging)
 };
+
+// Trace points of one CTA (LORA_LINEAR_DEBUG=2 prints them per launch).
+enum SmTrace : int {
+  kTrEntry = 0, kTrFirstIssue, kTrFirstData, kTrLastMma, kTrPublished, kTrCombined, kTrExit, kSmTracePoints
+};
+
+__device__ __forceinline__ void sm_trace(const SmallMParams& p, int point) {
+  if (p.trace != nullptr) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + point] = t;
+  }
+}
 
 template <int kNT>
 struct SmallMCfg {
@@ -115,6 +129,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  if (threadIdx.x == 0) sm_trace(p, kTrEntry);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -135,6 +150,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         }
         tma_load_2d_hint(st + 2 * C::kWBox, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
         tma_load_2d_hint(st + 2 * C::kWBox + C::kXBox, &p.tm_x, &full[rp.stage], k0 + 64, 0, pol_x);
+        if (u == u0) sm_trace(p, kTrFirstIssue);
         rp.next(S);
       }
     }
@@ -154,6 +170,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         }
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
         tc_fence_after();
+        if (u == u0) sm_trace(p, kTrFirstData);
         const uint32_t sw = smem_u32(smem + rp.stage * C::kStageBytes);
         const uint32_t sx = sw + 2 * C::kWBox;
 #pragma unroll
@@ -176,6 +193,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       volatile uint32_t zero = 0u;
       AbortCtl quiet{&zero, nullptr};
       mbar_wait(mma_done, 0, quiet);
+      sm_trace(p, kTrLastMma);
     }
   } else {
     // ------------------------------------------------------------ epilogue warps (128 threads)
@@ -220,6 +238,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         *last_flag = arrived == static_cast<uint32_t>(w_last - w_first + 1) ? 1 : 0;
       }
       bar_sync_named<1, 128>();
+      if (et == 0) sm_trace(p, kTrPublished);
       if (*last_flag == 0) continue;
       __threadfence();
       // ---- combine: the slice's partials in slot order
@@ -300,6 +319,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         }
       }
       if (et == 0) {
+        sm_trace(p, kTrCombined);
         p.counters[slice] = 0u;        // back to zero for the next call
         const uint32_t done = atomicAdd(slices_done, 1u) + 1u;
         if (done == static_cast<uint32_t>(p.slices)) {
@@ -313,6 +333,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) sm_trace(p, kTrExit);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, C::kTmemCols);
