@@ -155,7 +155,7 @@ struct Plan {
   bool small_m = false;
   int sm_nt = 16;                            // tokens padded to the MMA N granule
   SmallMSplit sm;
-  size_t sm_t_buf = 0, sm_d_part = 0;
+  size_t sm_t_buf = 0, sm_d_part0 = 0, sm_d_part = 0;
   size_t total = 0;
 };
 
@@ -163,7 +163,7 @@ struct Plan {
 // kSmallMMax tokens, while its slice counters fit the workspace header.
 bool small_m_applies(const lora_linear_desc* d) {
   return d->M > 0 && d->M <= kSmallMMax && d->r > 0 && d->act != LORA_ACT_SWIGLU &&
-         static_cast<size_t>(1 + ceil_div(d->d_out, 128)) + 2 <= kCounterWords;
+         static_cast<size_t>(3 + ceil_div(d->d_out, 128)) <= kCounterWords;
 }
 
 // Split-K width for a rank-r product with `tiles` row tiles and `nkb` 64-wide K blocks.
@@ -207,7 +207,8 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
       P.sm_nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
       P.sm = small_m_split(d->d_in, d->d_out, kTargetCtas);
       P.sm_t_buf = take(static_cast<size_t>(M) * r * 4);
-      P.sm_d_part = take(static_cast<size_t>(P.sm.slices) * P.sm.max_seg * 128 * P.sm_nt * 4);
+      P.sm_d_part0 = take(static_cast<size_t>(P.sm.nseg0) * 128 * P.sm_nt * 4);
+      P.sm_d_part = take(static_cast<size_t>(P.sm.wslices) * P.sm.max_seg * 128 * P.sm_nt * 4);
     }
     P.total = off;
     return P;
@@ -271,6 +272,47 @@ lora_status_t check_launch(const char* what) {
   return LORA_OK;
 }
 
+// Kernel launch with programmatic stream serialization: the kernel may start
+// while its predecessor in the stream finishes (hiding launch latency and the
+// prologue); every kernel of this library waits for its predecessor with
+// griddepcontrol.wait before touching global memory.  LORA_LINEAR_PDL=0 turns
+// the attribute off.  cluster2: launch as clusters of two CTAs.
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("LORA_LINEAR_PDL");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool cluster2,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster2) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 2;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // benchmark instrumentation: CUDA events around the main GEMM launches
 // ---------------------------------------------------------------------------
@@ -310,7 +352,7 @@ lora_status_t launch_rank(const RankGemmParams& p, int splits, cudaStream_t st) 
     return cuda_error("cudaFuncSetAttribute(rank)");
   LORA_LOG("rank mn=%d RP=%d na=%d nb=%d f16=%d pairs=%d rows=%d K=%d tiles=%d splits=%d", (int)kAMN, kRP, kNA,
            kNB, (int)kF16, p.npairs, p.rows, p.K, p.m_tiles, splits);
-  k<<<p.m_tiles * splits, kRankThreads, C::kSmemBytes, st>>>(p);
+  launch_k(k, dim3(p.m_tiles * splits), dim3(kRankThreads), C::kSmemBytes, st, false, p);
   return check_launch("rank_gemm_kernel");
 }
 
@@ -408,7 +450,7 @@ lora_status_t launch_reduce(RankReduceJob* R, int n, cudaStream_t st) {
   long long gx = blocks;
   if (gx > 1184) gx = 1184;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(n), 1);
-  reduce_rank_kernel<<<grid, 256, 0, st>>>(R[0], R[1]);
+  launch_k(reduce_rank_kernel, grid, dim3(256), 0, st, false, R[0], R[1]);
   return check_launch("reduce_rank_kernel");
 }
 
@@ -436,7 +478,7 @@ lora_status_t launch_rank2d_t(const Rank2dParams& p, int grid, cudaStream_t st) 
     return cuda_error("cudaFuncSetAttribute(rank2d)");
   LORA_LOG("rank2d RP=%d row=%d col=%d grid=%d a=%d b=%d fs=%d stages=%d", kRP, (int)kRow, (int)kCol, grid,
            p.a_tiles, p.b_blocks, p.fs, C::kStages);
-  k<<<grid, kRank2dThreads, C::kSmemBytes, st>>>(p);
+  launch_k(k, dim3(grid), dim3(kRank2dThreads), C::kSmemBytes, st, false, p);
   return check_launch("rank2d_kernel");
 }
 
@@ -540,21 +582,10 @@ lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
     return cuda_error("cudaFuncSetAttribute(mma)");
   const int max_units = kPair ? sms / 2 : sms;
   const int units = p.num_tiles < max_units ? p.num_tiles : max_units;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(units * C::kCtas), 1, 1);
-  cfg.blockDim = dim3(kMmaThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C::kCtas;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = kPair ? 1 : 0;
   LORA_LOG("mma pair=%d bwd=%d npair=%d epi=%d tiles=%d units=%d smem=%d stages=%d lora_ksteps=%d", (int)kPair,
            (int)kBwd, kNPair, kEpi, p.num_tiles, units, C::kSmemBytes, C::kStages, p.lora_ksteps);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, p);
+  const cudaError_t e = launch_k(k, dim3(static_cast<unsigned>(units * C::kCtas)), dim3(kMmaThreads), C::kSmemBytes,
+                                 st, kPair, p);
   if (e != cudaSuccess) {
     LORA_LOG("mma launch: %s", cudaGetErrorString(e));
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -741,6 +772,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     q.T_save = T_save;
     q.Z_save = d->act == LORA_ACT_SILU ? Z_save : nullptr;
     q.t_buf = reinterpret_cast<float*>(ws + P.sm_t_buf);
+    q.d_part0 = reinterpret_cast<float*>(ws + P.sm_d_part0);
     q.d_part = reinterpret_cast<float*>(ws + P.sm_d_part);
     q.counters = reinterpret_cast<uint32_t*>(ws + kStatusBytes);
     q.status = status;
@@ -750,13 +782,15 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     q.r = static_cast<int>(r);
     q.s = d->s;
     q.act = d->act;
-    q.slices = P.sm.slices;
+    q.wslices = P.sm.wslices;
     q.nkc = P.sm.nkc;
     q.run = P.sm.run;
+    q.grid = P.sm.grid;
+    q.nseg0 = P.sm.nseg0;
     q.max_seg = P.sm.max_seg;
-    const int grid = P.sm.n_w;
-    LORA_LOG("small_m M=%d nt=%d slices=%d nkc=%d run=%d grid=%d max_seg=%d", (int)M, nt, q.slices, q.nkc, q.run,
-             grid, q.max_seg);
+    const int grid = q.grid;
+    LORA_LOG("small_m M=%d nt=%d wslices=%d nkc=%d run=%d grid=%d nseg0=%d max_seg=%d", (int)M, nt, q.wslices, q.nkc,
+             q.run, grid, q.nseg0, q.max_seg);
     // LORA_LINEAR_DEBUG=2: per-CTA phase stamps, printed after the launch
     // (synchronises the stream; for debugging only).
     static unsigned long long* trace = nullptr;
@@ -767,7 +801,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
       q.trace = trace;
       cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTracePoints, st);
     }
-    const cudaError_t e = launch_small_m(q, nt, grid, st);
+    const cudaError_t e = launch_small_m(q, nt, st);
     if (e != cudaSuccess) {
       LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
       g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -902,9 +936,9 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     const long long tiles = ceil_div(d->d_out, 64) * ceil_div(d->d_in, 64);
     const int grid = static_cast<int>(tiles < static_cast<long long>(dev.sms) * 8 ? tiles : dev.sms * 8);
     for (int j = 0; j < np; ++j) {
-      transpose_w_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(Wp[j]),
-                                                              static_cast<int>(d->d_out), static_cast<int>(d->d_in),
-                                                              static_cast<__nv_bfloat16*>(at(P.wt[j])), status);
+      launch_k(transpose_w_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, false,
+               static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<int>(d->d_out), static_cast<int>(d->d_in),
+               static_cast<__nv_bfloat16*>(at(P.wt[j])), status);
       LORA_TRY(check_launch("transpose_w_kernel"));
       Wmain[j] = at(P.wt[j]);
     }
@@ -913,21 +947,23 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     const long long n = static_cast<long long>(M) * d->d_out;
     const int grid = grid_for(n / 8, 256, dev.sms);
     if (swiglu)
-      act_bwd_kernel<true><<<grid, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(dY), Z_save, Z_save + static_cast<size_t>(M) * d->d_out, n,
-          static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])),
-          static_cast<__half*>(at(P.dz_hi[1])), static_cast<__half*>(at(P.dz_lo[1])), status);
+      launch_k(act_bwd_kernel<true>, dim3(grid), dim3(256), 0, st, false, static_cast<const __nv_bfloat16*>(dY),
+               static_cast<const float*>(Z_save), static_cast<const float*>(Z_save + static_cast<size_t>(M) * d->d_out),
+               static_cast<long long>(n), static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])),
+               static_cast<__half*>(at(P.dz_hi[1])), static_cast<__half*>(at(P.dz_lo[1])), status);
     else
-      act_bwd_kernel<false><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dY), Z_save, nullptr, n,
-                                                  static_cast<__half*>(at(P.dz_hi[0])),
-                                                  static_cast<__half*>(at(P.dz_lo[0])), nullptr, nullptr, status);
+      launch_k(act_bwd_kernel<false>, dim3(grid), dim3(256), 0, st, false, static_cast<const __nv_bfloat16*>(dY),
+               static_cast<const float*>(Z_save), static_cast<const float*>(nullptr), static_cast<long long>(n),
+               static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])),
+               static_cast<__half*>(nullptr), static_cast<__half*>(nullptr), status);
     LORA_TRY(check_launch("act_bwd_kernel"));
     const long long nw = static_cast<long long>(d->d_out) * d->d_in;
     for (int j = 0; j < np; ++j) {
       dZ[j] = at(P.dz_hi[j]);
       dZlo[j] = at(P.dz_lo[j]);
-      convert_f16_kernel<<<grid_for(nw / 8, 256, dev.sms), 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<__half*>(at(P.wt[j])), nw, status);
+      launch_k(convert_f16_kernel, dim3(grid_for(nw / 8, 256, dev.sms)), dim3(256), 0, st, false,
+               static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<__half*>(at(P.wt[j])), static_cast<long long>(nw),
+               status);
       LORA_TRY(check_launch("convert_f16_kernel"));
       Wmain[j] = at(P.wt[j]);
     }
@@ -942,15 +978,16 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
       const __nv_bfloat16* Aj = static_cast<const __nv_bfloat16*>(Ap[j]);
       __nv_bfloat16* Atj = P.kmajor ? static_cast<__nv_bfloat16*>(at(P.at_[j])) : nullptr;
       if (f16)
-        bwd_prep_kernel<__half><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
-            static_cast<__half*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
-            static_cast<__half*>(at(P.tt_hi[j])), static_cast<__half*>(at(P.tt_lo[j])), M8, status);
+        launch_k(bwd_prep_kernel<__half>, dim3(grid_for(n, 256, dev.sms)), dim3(256), 0, st, false,
+                 static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
+                 static_cast<__half*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
+                 static_cast<__half*>(at(P.tt_hi[j])), static_cast<__half*>(at(P.tt_lo[j])), M8, status);
       else
-        bwd_prep_kernel<__nv_bfloat16><<<grid_for(n, 256, dev.sms), 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
-            static_cast<__nv_bfloat16*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
-            static_cast<__nv_bfloat16*>(at(P.tt_hi[j])), static_cast<__nv_bfloat16*>(at(P.tt_lo[j])), M8, status);
+        launch_k(bwd_prep_kernel<__nv_bfloat16>, dim3(grid_for(n, 256, dev.sms)), dim3(256), 0, st, false,
+                 static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
+                 static_cast<__nv_bfloat16*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
+                 static_cast<__nv_bfloat16*>(at(P.tt_hi[j])), static_cast<__nv_bfloat16*>(at(P.tt_lo[j])), M8,
+                 status);
       LORA_TRY(check_launch("bwd_prep_kernel"));
       if (Tj == nullptr) {
         RankOut o = rank_out(M, r);

@@ -72,9 +72,13 @@ struct MmaCfg {
   static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
   static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages0 = (kSmemLimitBytes - 2048) / kStageBytes;
+  // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
+  // shared memory (4 KB per warp) so that global stores are row-contiguous.
+  static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu;
+  static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : 0;
+  static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 2048;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kEpiStageBytes + 2048;
   static constexpr uint32_t kTmemCols = 512;                 // 2 accumulator buffers
   static_assert(kStages >= 3, "ring too shallow");
 };
@@ -116,7 +120,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint8_t* epi_stage = smem + S * C::kStageBytes;          // [8 warps][4 KB] (kStaged)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kEpiStageBytes);
   uint64_t* full = bars;                  // [S]
   uint64_t* empty = bars + S;             // [S]
   uint64_t* acc_full = bars + 2 * S;      // [2] accumulator buffer b complete
@@ -155,6 +160,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   if constexpr (kPair) cluster_sync_all();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  grid_dep_wait();
   const int nkb = (p.K + 63) / 64;
   const int nlora = p.lora_ksteps > 0 ? C::kLoraBlocks : 0;
 
@@ -347,67 +353,85 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       tc_fence_before();
       if constexpr (kPair) mbar_arrive_cluster(acc_empty_addr[buf]);
       else mbar_arrive(&acc_empty[buf]);
-      if (!row_ok) continue;
-
-      if constexpr (C::kSwigluFwd) {
-        const int col0 = nt * 128 + h * 64;
-        const size_t base = static_cast<size_t>(row) * p.N + col0;
-        if (p.z_save != nullptr) {
-          float* zg = p.z_save + base;
-          float* zu = p.z_save + static_cast<size_t>(p.M) * p.N + base;
+      if constexpr (C::kStaged) {
+        // Stage 32 rows x 8 uint4 (this lane's row) through shared memory,
+        // then store them row-contiguous: 8 lanes cover 128 bytes of a row.
+        const int row0 = row - lane;                 // first row of this warp's 32
+        uint4* stg = reinterpret_cast<uint4*>(epi_stage + ew * 4096);
+        auto flush = [&](const uint4 (&mine)[8], auto&& store) {
 #pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            if (col0 + c < p.N) {
-              st_global_v4_hint(zg + c, make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]), pol_out);
-              st_global_v4_hint(zu + c, make_uint4(v[64 + c], v[65 + c], v[66 + c], v[67 + c]), pol_out);
+          for (int j = 0; j < 8; ++j) stg[lane * 8 + (j ^ (lane & 7))] = mine[j];
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3), j = lane & 7;
+            if (row0 + rr < p.M) store(row0 + rr, j, stg[rr * 8 + (j ^ (rr & 7))]);
+          }
+          __syncwarp();
+        };
+        const int ncol = C::kSwigluFwd ? 64 : 128;         // columns of this thread
+        const int col0 = C::kSwigluFwd ? nt * 128 + h * 64 : nt * 256 + h * 128;
+        if (p.z_save != nullptr) {
+          // fp32 Z: 32 columns per flush (gate then up for SwiGLU)
+#pragma unroll
+          for (int part = 0; part < (C::kSwigluFwd ? 2 : 1); ++part) {
+            float* zdst = p.z_save + static_cast<size_t>(part) * p.M * p.N;
+#pragma unroll
+            for (int cb = 0; cb < ncol; cb += 32) {
+              uint4 mine[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int c = part * 64 + cb + 4 * j;
+                mine[j] = make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+              }
+              flush(mine, [&](int grow, int j, uint4 val) {
+                const int col = col0 + cb + 4 * j;
+                if (col < p.N) st_global_v4_hint(zdst + static_cast<size_t>(grow) * p.N + col, val, pol_out);
+              });
             }
           }
         }
+        // bf16 Y: 64 columns per flush
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          float hv[8];
+        for (int cb = 0; cb < ncol; cb += 64) {
+          uint4 mine[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float g = __uint_as_float(v[c + e]);
-            const float u = __uint_as_float(v[64 + c + e]);
-            hv[e] = g / (1.0f + expf(-g)) * u;
+          for (int j = 0; j < 8; ++j) {
+            float yv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c = cb + 8 * j + e;
+              if constexpr (C::kSwigluFwd) {
+                const float g = __uint_as_float(v[c]);
+                const float u = __uint_as_float(v[64 + c]);
+                yv[e] = g / (1.0f + expf(-g)) * u;
+              } else {
+                const float z = __uint_as_float(v[c]);
+                yv[e] = z / (1.0f + expf(-z));
+              }
+            }
+            mine[j].x = pack_bf16x2(yv[0], yv[1]);
+            mine[j].y = pack_bf16x2(yv[2], yv[3]);
+            mine[j].z = pack_bf16x2(yv[4], yv[5]);
+            mine[j].w = pack_bf16x2(yv[6], yv[7]);
           }
-          if (col0 + c < p.N) {
-            uint4 pk;
-            pk.x = pack_bf16x2(hv[0], hv[1]);
-            pk.y = pack_bf16x2(hv[2], hv[3]);
-            pk.z = pack_bf16x2(hv[4], hv[5]);
-            pk.w = pack_bf16x2(hv[6], hv[7]);
-            st_global_v4_hint(p.out + base + c, pk, pol_out);
-          }
+          flush(mine, [&](int grow, int j, uint4 val) {
+            const int col = col0 + cb + 8 * j;
+            if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
+          });
         }
       } else {
+        if (!row_ok) continue;
         const int col0 = nt * 256 + h * 128;
         const size_t base = static_cast<size_t>(row) * p.N + col0;
-        if constexpr (kEpi == kMEpiSilu) {
-          if (p.z_save != nullptr) {
-#pragma unroll
-            for (int c = 0; c < 128; c += 4)
-              if (col0 + c < p.N)
-                st_global_v4_hint(p.z_save + base + c, make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]), pol_out);
-          }
-        }
 #pragma unroll
         for (int c = 0; c < 128; c += 8) {
-          float yv[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float z = __uint_as_float(v[c + e]);
-            yv[e] = (kEpi == kMEpiSilu) ? z / (1.0f + expf(-z)) : z;
-          }
-          if (col0 + c < p.N) {
-            uint4 pk;
-            pk.x = pack_bf16x2(yv[0], yv[1]);
-            pk.y = pack_bf16x2(yv[2], yv[3]);
-            pk.z = pack_bf16x2(yv[4], yv[5]);
-            pk.w = pack_bf16x2(yv[6], yv[7]);
-            st_global_v4_hint(p.out + base + c, pk, pol_out);
-          }
+          uint4 pk;
+          pk.x = pack_bf16x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+          pk.y = pack_bf16x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+          pk.z = pack_bf16x2(__uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+          pk.w = pack_bf16x2(__uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
+          if (col0 + c < p.N) st_global_v4_hint(p.out + base + c, pk, pol_out);
         }
       }
     }

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  grid_dep_wait();
 
   if (warp == 0) {
     if (lane == 0 && nkb > 0) {
@@ -269,6 +270,7 @@ struct RankReduceJob {
 constexpr int kReduceRows = 32;
 
 __global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
+  grid_dep_wait();
   const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
   __shared__ float tile[kReduceRows][65];
   const int r = J.out.r;
@@ -365,6 +367,7 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, 
                                 const __nv_bfloat16* __restrict__ A, int d_in, __nv_bfloat16* __restrict__ At,
                                 const float* __restrict__ Tsave, int M, float s, T* __restrict__ t_hi,
                                 T* __restrict__ t_lo, int ld, uint32_t* status) {
+  grid_dep_wait();
   const long long nb = d_out;
   const long long na = At != nullptr ? d_in : 0;
   const long long nt = Tsave != nullptr ? M : 0;
@@ -415,6 +418,7 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, 
 // convert exactly; |w| > 65504 flags the status word.
 __global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, long long n,
                                    uint32_t* status) {
+  grid_dep_wait();
   const long long nv = n / 8;
   bool bad = false;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;
@@ -444,6 +448,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) transpose_w_kernel(const __nv_bfloat16* __restrict__ W, int rows, int cols,
                                                           T* __restrict__ Wt, uint32_t* status) {
   __shared__ uint32_t tile[64][33];
+  grid_dep_wait();
   const int tiles_c = (cols + 63) / 64;
   const long long ntiles = static_cast<long long>((rows + 63) / 64) * tiles_c;
   bool bad = false;
@@ -516,6 +521,7 @@ __global__ void act_bwd_kernel(const __nv_bfloat16* __restrict__ dY, const float
                                const float* __restrict__ Zup, long long n, __half* __restrict__ g_hi,
                                __half* __restrict__ g_lo, __half* __restrict__ u_hi, __half* __restrict__ u_lo,
                                uint32_t* status) {
+  grid_dep_wait();
   bool bad = false;
   const long long nv = n / 8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nv;

@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  grid_dep_wait();
 
   if (warp == 0) {
     if (lane == 0) {

@@ -2,28 +2,31 @@
 // layer is bound by reading W once from HBM (2 M d_in d_out FLOP on about
 // 2 d_in d_out bytes), so the kernel is laid out for bandwidth.
 //
-// The rows of A are treated as one more 128-row slice in front of W's slices:
-// streaming [A ; W] against X gives [T^T ; Z_main^T] in one pass, so T = X A^T
-// costs no separate kernel, no extra CTAs and no dependent round trips while
-// the memory system is busy with W.  Slice 0 (A, r rows, zero-filled to 128 by
-// the TMA box) has almost no DRAM traffic and finishes first.
+// The rows of A are streamed like one more 128-row slice of weights ("slice
+// 0", in front of W's slices 1..): [A ; W] against X gives [T^T ; Z_main^T] in
+// one pass, so T = X A^T needs no kernel of its own.  Slice 0's K chunks are
+// spread one per CTA as the first unit of CTAs 0, 1, ... (A has r rows, so a
+// chunk costs almost no DRAM traffic): T is complete about one unit into the
+// pass, long before any slice of W.
 //
-// One cooperative grid of at most one CTA per SM, stream-K over units of
-// (128-row slice x 128-wide K chunk), slice-major, cut into equal contiguous
-// runs (one per CTA).  Per unit one TMA stage brings two 64-wide boxes of the
-// slice and the matching X boxes (M tokens, zero-filled to kNT rows); the MMA
-// warp accumulates [128 rows x kNT tokens] in tensor memory (swap-AB: the
-// weight rows are the M-side operand), double-buffered across segments.  When
-// a CTA's part of a slice ends, its fp32 partial goes to global memory and the
-// CTA bumps the slice's arrival counter; the CTA that arrives last (it learns
-// so from the counter, without waiting) sums the slice's partials in slot
-// order and finishes the slice:
-//   slice 0:  T (and T_save) from rows < r, then a release of the T-ready flag;
-//   slice s:  after a bounded wait for T-ready (set long before, in practice),
-//             Z = partial sum + s T B^T, activation, Y.
-// The cooperative launch guarantees that every CTA is resident, so the wait
-// for the slice-0 CTAs always ends.  The counters live in the workspace header
-// and are zero at rest: the calls that use them put them back to zero.
+// One cooperative grid of at most one CTA per SM.  W's units (128-row slice x
+// 128-wide K chunk, slice-major) are cut into equal contiguous runs, one per
+// CTA.  Per unit one TMA stage brings two 64-wide boxes of the slice and the
+// matching X boxes (M tokens, zero-filled to kNT rows); the MMA warp
+// accumulates [128 rows x kNT tokens] in tensor memory (swap-AB: the weight
+// rows are the M-side operand), double-buffered across segments.  When a
+// CTA's part of a slice ends, its fp32 partial goes to global memory and the
+// CTA bumps the slice's arrival counter; the CTA whose arrival completes the
+// slice (it learns so from the counter value) finishes it:
+//   slice 0: sums the partials in slot order, writes T (and T_save) from
+//     rows < r, and releases the T-ready flag;
+//   a slice of W: sums the partials in slot order (deterministic), adds
+//     s T B^T, applies the activation and stores Y.  It needs T: T is ready
+//     about one unit into the pass, so the bounded wait for the flag is
+//     normally already over; the cooperative launch makes every CTA resident,
+//     so the wait always ends.
+// The counters live in the workspace header and are zero at rest: the last
+// finisher of a call puts them back to zero.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -44,16 +47,19 @@ struct SmallMParams {
   __nv_bfloat16* Y;          // [M x d_out]
   float* T_save;             // [M x r] or null
   float* Z_save;             // [M x d_out] or null (SiLU)
-  float* t_buf;              // [M x r] T, written by slice 0's combiner
-  float* d_part;             // [slices][max_seg][128 x kNT] partials ([A ; W] slices)
-  uint32_t* counters;        // [slices] arrivals, then t_ready, slices_done (zero at rest)
+  float* t_buf;              // [M x r] T, written by slice 0's finisher
+  float* d_part0;            // [nseg0][128 x kNT] slice-0 partials
+  float* d_part;             // [wslices][max_seg][128 x kNT] partials of W's slices
+  uint32_t* counters;        // [1 + wslices] arrivals, then T-ready, finished slices (zero at rest)
   uint32_t* status;
   int M, d_in, d_out, r;
   float s;
   int act;
-  int slices, nkc;           // 128-row slices of [A ; W] (1 + ceil(d_out / 128)); 128-wide K chunks
-  int run;                   // units per CTA
-  int max_seg;               // partial slots per slice
+  int wslices, nkc;          // 128-row slices of W; 128-wide K chunks
+  int run;                   // W units per CTA
+  int grid;                  // CTAs
+  int nseg0;                 // CTAs holding slice-0 chunks: min(nkc, grid)
+  int max_seg;               // partial slots per slice of W
   unsigned long long* trace; // null, or [grid][kSmTracePoints] globaltimer stamps (debugging)
 };
 
@@ -65,7 +71,7 @@ enum SmTrace : int {
 __device__ __forceinline__ void sm_trace(const SmallMParams& p, int point) {
   if (p.trace != nullptr) {
     unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) : : "memory");
     p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + point] = t;
   }
 }
@@ -84,10 +90,178 @@ struct SmallMCfg {
   static_assert(kStages >= 3, "ring too shallow");
 };
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+// The units of CTA w, in order: its slice-0 chunks w, w + grid, ... (< nkc),
+// then its run of W units.
+struct SmUnits {
+  int na;    // slice-0 chunks
+  int uw0;   // first W unit
+  int n;     // units in all
+  __device__ __forceinline__ SmUnits(const SmallMParams& p, int w) {
+    na = w < p.nkc ? (p.nkc - 1 - w) / p.grid + 1 : 0;
+    const int total_w = p.wslices * p.nkc;
+    uw0 = w * p.run;
+    const int uw1 = uw0 + p.run < total_w ? uw0 + p.run : total_w;
+    n = na + (uw1 > uw0 ? uw1 - uw0 : 0);
+  }
+  // slice (0 = A, s >= 1 = W rows [128 (s - 1), +128)) and K chunk of unit i
+  __device__ __forceinline__ void at(const SmallMParams& p, int w, int i, int& slice, int& kc) const {
+    if (i < na) {
+      slice = 0;
+      kc = w + i * p.grid;
+    } else {
+      const int u = uw0 + (i - na);
+      slice = 1 + u / p.nkc;
+      kc = u - (slice - 1) * p.nkc;
+    }
+  }
+};
+
+__device__ __forceinline__ int small_m_first_cta(const SmallMParams& p, int slice) {
+  return ((slice - 1) * p.nkc) / p.run;
+}
+__device__ __forceinline__ int small_m_nseg(const SmallMParams& p, int slice) {
+  if (slice == 0) return p.nseg0;
+  return ((slice - 1) * p.nkc + p.nkc - 1) / p.run - small_m_first_cta(p, slice) + 1;
+}
+// Arrivals that finish a slice: one per CTA holding part of it.
+__device__ __forceinline__ uint32_t small_m_target(const SmallMParams& p, int slice) {
+  return static_cast<uint32_t>(small_m_nseg(p, slice));
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* a) {
   uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
   return v;
+}
+
+// A slice is finished: count it; the last finisher of the call resets the
+// shared words (every finisher of W has passed its wait for T by then).
+__device__ __forceinline__ void small_m_slice_done(const SmallMParams& p, int slice) {
+  uint32_t* t_ready = p.counters + 1 + p.wslices;
+  uint32_t* done = t_ready + 1;
+  p.counters[slice] = 0u;
+  if (atomicAdd(done, 1u) + 1u == static_cast<uint32_t>(1 + p.wslices)) {
+    *done = 0u;
+    *t_ready = 0u;
+  }
+}
+__device__ __forceinline__ float* small_m_slot(const SmallMParams& p, int slice, int slot, int lrow, int nt) {
+  if (slice == 0) return p.d_part0 + (static_cast<size_t>(slot) * 128 + lrow) * nt;
+  return p.d_part + ((static_cast<size_t>(slice - 1) * p.max_seg + slot) * 128 + lrow) * nt;
+}
+
+// Sum of a slice's partials for row lrow, in slot order.
+template <int kNT>
+__device__ __forceinline__ void small_m_sum_partials(const SmallMParams& p, int slice, int lrow, float (&z)[kNT]) {
+  const int nseg = small_m_nseg(p, slice);
+#pragma unroll
+  for (int m = 0; m < kNT; ++m) z[m] = 0.0f;
+  constexpr int kSegUnroll = kNT <= 16 ? 4 : (kNT <= 32 ? 2 : 1);   // partial loads in flight
+#pragma unroll kSegUnroll
+  for (int sg = 0; sg < nseg; ++sg) {
+    const float4* src = reinterpret_cast<const float4*>(small_m_slot(p, slice, sg, lrow, kNT));
+#pragma unroll
+    for (int m4 = 0; m4 < kNT / 4; ++m4) {
+      const float4 v = __ldcg(src + m4);
+      z[4 * m4] += v.x;
+      z[4 * m4 + 1] += v.y;
+      z[4 * m4 + 2] += v.z;
+      z[4 * m4 + 3] += v.w;
+    }
+  }
+}
+
+// Finish slice 0 (all 128 epilogue threads): T[m][c] = sum over the slice-0
+// partials, in slot order, of row c (< r), column m (< M).  One element per
+// thread at a time with 16 partial loads in flight.
+template <int kNT>
+__device__ __forceinline__ void small_m_finish_t(const SmallMParams& p, int et) {
+  const int ne = p.r * p.M;
+  const size_t stride = static_cast<size_t>(128) * kNT;     // between slots
+  for (int e = et; e < ne; e += 128) {
+    const int row = e / p.M, m = e - row * p.M;
+    const float* src = p.d_part0 + static_cast<size_t>(row) * kNT + m;
+    float acc = 0.0f;
+    for (int s0 = 0; s0 < p.nseg0; s0 += 16) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = s0 + u < p.nseg0 ? __ldcg(src + (s0 + u) * stride) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) acc += v[u];                // slot order; + 0 past the last slot
+    }
+    __stcg(p.t_buf + static_cast<size_t>(m) * p.r + row, acc);
+    if (p.T_save != nullptr) p.T_save[static_cast<size_t>(m) * p.r + row] = acc;
+  }
+}
+
+// Finish a slice of W (all 128 epilogue threads): Z = partial sum + s T B^T,
+// activation, Y (and Z_save).  T, this thread's row of B and the partials are
+// all requested before the first use.
+template <int kNT>
+__device__ __forceinline__ void small_m_finish_slice(const SmallMParams& p, int slice, int et, int lrow, float* Ts) {
+  const int n = (slice - 1) * 128 + lrow;
+  if (et == 0) {
+    const uint32_t* t_ready = p.counters + 1 + p.wslices;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(t_ready) == 0u) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicOr(p.status, kStatusWaitTimeout);
+        break;
+      }
+    }
+  }
+  bar_sync_named<1, 128>();
+  __threadfence();
+#pragma unroll
+  for (int k = 0; k < kNT / 2; ++k) {
+    const int i = et + 128 * k;
+    const int m = i >> 6, c = i & 63;
+    Ts[i] = (m < p.M && c < p.r) ? __ldcg(p.t_buf + m * p.r + c) : 0.0f;
+  }
+  // B row prefetched in registers only while they are plentiful (kNT = 16)
+  constexpr int kBq = kNT <= 16 ? 8 : 1;
+  uint4 bq[kBq];
+#pragma unroll
+  for (int c8 = 0; c8 < kBq; ++c8)
+    bq[c8] = (c8 * 8 < p.r && n < p.d_out)
+                 ? __ldg(reinterpret_cast<const uint4*>(p.B + static_cast<size_t>(n) * p.r + c8 * 8))
+                 : make_uint4(0u, 0u, 0u, 0u);
+  float z[kNT];
+  small_m_sum_partials<kNT>(p, slice, lrow, z);
+  bar_sync_named<1, 128>();                 // T in shared memory
+  if (n < p.d_out) {
+#pragma unroll(kBq)
+    for (int c8 = 0; c8 < 8; ++c8) {
+      if (c8 * 8 < p.r) {
+        uint4 bv;
+        if constexpr (kBq == 8) bv = bq[c8];
+        else bv = __ldg(reinterpret_cast<const uint4*>(p.B + static_cast<size_t>(n) * p.r + c8 * 8));
+        const __nv_bfloat16* b8 = reinterpret_cast<const __nv_bfloat16*>(&bv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float b = p.s * __bfloat162float(b8[e]);
+#pragma unroll
+          for (int m = 0; m < kNT; ++m) z[m] = fmaf(b, Ts[m * 64 + c8 * 8 + e], z[m]);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < kNT; ++m) {
+      if (m < p.M) {
+        float y = z[m];
+        if (p.act == LORA_ACT_SILU) {
+          if (p.Z_save != nullptr) p.Z_save[static_cast<size_t>(m) * p.d_out + n] = y;
+          y = y / (1.0f + expf(-y));
+        }
+        p.Y[static_cast<size_t>(m) * p.d_out + n] = __float2bfloat16_rn(y);
+      }
+    }
+  }
+  bar_sync_named<1, 128>();                 // Ts is reused by the next finish
+  if (et == 0) {
+    sm_trace(p, kTrCombined);
+    small_m_slice_done(p, slice);
+  }
 }
 
 template <int kNT>
@@ -105,18 +279,13 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(seg_full + 5);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  float* Ts = reinterpret_cast<float*>(smem + S * C::kStageBytes + 1024);   // T [kNT x 64]
-
-  uint32_t* t_ready = p.counters + p.slices;
-  uint32_t* slices_done = p.counters + p.slices + 1;
+  float* Ts = reinterpret_cast<float*>(smem + S * C::kStageBytes + 1024);                // T [kNT x 64]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   AbortCtl ctl{abort_flag, p.status};
   const int w = blockIdx.x;
-  const int units = p.slices * p.nkc;
-  const int u0 = w * p.run;
-  const int u1 = u0 + p.run < units ? u0 + p.run : units;
+  const SmUnits units(p, w);
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&seg_full[b], 1); mbar_init(&seg_empty[b], 128); }
@@ -129,17 +298,19 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  grid_dep_wait();
   if (threadIdx.x == 0) sm_trace(p, kTrEntry);
 
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t pol_x = l2_policy_evict_last();     // X is re-read by every CTA
       RingPos rp;
-      for (int u = u0; u < u1; ++u) {
+      for (int i = 0; i < units.n; ++i) {
         if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
-        const int slice = u / p.nkc;
-        const int k0 = (u - slice * p.nkc) * 128;
+        int slice, kc;
+        units.at(p, w, i, slice, kc);
+        const int k0 = kc * 128;
         mbar_arrive_expect_tx(&full[rp.stage], C::kStageBytes);
         if (slice == 0) {
           tma_load_2d(st, &p.tm_a, &full[rp.stage], k0, 0);
@@ -150,7 +321,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         }
         tma_load_2d_hint(st + 2 * C::kWBox, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
         tma_load_2d_hint(st + 2 * C::kWBox + C::kXBox, &p.tm_x, &full[rp.stage], k0 + 64, 0, pol_x);
-        if (u == u0) sm_trace(p, kTrFirstIssue);
+        if (i == 0) sm_trace(p, kTrFirstIssue);
         rp.next(S);
       }
     }
@@ -160,8 +331,9 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       RingPos rp;
       int seg = 0;
       bool first = true;
-      for (int u = u0; u < u1; ++u) {
-        const int slice = u / p.nkc;
+      for (int i = 0; i < units.n; ++i) {
+        int slice, kc;
+        units.at(p, w, i, slice, kc);
         const uint32_t buf = seg & 1;
         if (first) {
           // a new segment: its accumulator buffer must have been read out
@@ -170,7 +342,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         }
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
         tc_fence_after();
-        if (u == u0) sm_trace(p, kTrFirstData);
+        if (i == 0) sm_trace(p, kTrFirstData);
         const uint32_t sw = smem_u32(smem + rp.stage * C::kStageBytes);
         const uint32_t sx = sw + 2 * C::kWBox;
 #pragma unroll
@@ -182,7 +354,9 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         mma_commit(&empty[rp.stage]);
         rp.next(S);
         first = false;
-        if (u + 1 == u1 || (u + 1) / p.nkc != slice) {
+        int next_slice = -1, next_kc = 0;
+        if (i + 1 < units.n) units.at(p, w, i + 1, next_slice, next_kc);
+        if (next_slice != slice) {
           mma_commit(&seg_full[buf]);
           ++seg;
           first = true;
@@ -201,19 +375,24 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int lrow = q * 32 + lane;         // row within the slice
     int seg = 0;
-    int u = u0;
-    bool have_t = false;                    // T staged in shared memory
-    while (u < u1) {
-      const int slice = u / p.nkc;
-      const int ue = (slice + 1) * p.nkc < u1 ? (slice + 1) * p.nkc : u1;
+    int i = 0;
+    while (i < units.n) {
+      int slice, kc;
+      units.at(p, w, i, slice, kc);
+      // the segment runs while the slice stays the same
+      int ie = i + 1;
+      while (ie < units.n) {
+        int s2, k2;
+        units.at(p, w, ie, s2, k2);
+        if (s2 != slice) break;
+        ++ie;
+      }
       const uint32_t buf = seg & 1;
       const bool got = mbar_wait(&seg_full[buf], (seg >> 1) & 1, ctl);
       if (!bar_sync_and<1, 128>(got)) break;        // all epilogue threads leave together
       tc_fence_after();
-      // CTAs w_first..w_last share this slice; this CTA's partial goes to slot w - w_first
-      const int w_first = (slice * p.nkc) / p.run;
-      const int w_last = (slice * p.nkc + p.nkc - 1) / p.run;
-      float* dst = p.d_part + ((static_cast<size_t>(slice) * p.max_seg + (w - w_first)) * 128 + lrow) * kNT;
+      const int slot = slice == 0 ? w : w - small_m_first_cta(p, slice);
+      float* dst = small_m_slot(p, slice, slot, lrow, kNT);
       const uint32_t tl = tbase + buf * kNT + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
       for (int c0 = 0; c0 < kNT; c0 += 16) {
@@ -229,105 +408,29 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&seg_empty[buf]);
       ++seg;
-      u = ue;
-      // publish the partial; the CTA that completes the slice combines it
+      i = ie;
+      // publish the partial; the arrival that completes the slice finishes it
       __threadfence();
       bar_sync_named<1, 128>();
       if (et == 0) {
         const uint32_t arrived = atomicAdd(&p.counters[slice], 1u) + 1u;
-        *last_flag = arrived == static_cast<uint32_t>(w_last - w_first + 1) ? 1 : 0;
+        *last_flag = arrived == small_m_target(p, slice) ? 1 : 0;
       }
       bar_sync_named<1, 128>();
       if (et == 0) sm_trace(p, kTrPublished);
       if (*last_flag == 0) continue;
       __threadfence();
-      // ---- combine: the slice's partials in slot order
-      const int nseg = w_last - w_first + 1;
-      float z[kNT];
-#pragma unroll
-      for (int m = 0; m < kNT; ++m) z[m] = 0.0f;
-      constexpr int kSegUnroll = kNT <= 16 ? 4 : (kNT <= 32 ? 2 : 1);   // partial loads in flight
-#pragma unroll kSegUnroll
-      for (int sg = 0; sg < nseg; ++sg) {
-        const float4* src =
-            reinterpret_cast<const float4*>(p.d_part + ((static_cast<size_t>(slice) * p.max_seg + sg) * 128 + lrow) * kNT);
-#pragma unroll
-        for (int m4 = 0; m4 < kNT / 4; ++m4) {
-          const float4 v = __ldcg(src + m4);
-          z[4 * m4] += v.x;
-          z[4 * m4 + 1] += v.y;
-          z[4 * m4 + 2] += v.z;
-          z[4 * m4 + 3] += v.w;
-        }
+      if (slice != 0) {
+        small_m_finish_slice<kNT>(p, slice, et, lrow, Ts);
+        continue;
       }
-      if (slice == 0) {
-        // rows < r hold T^T: T[m][lrow] for the M real tokens
-        if (lrow < p.r) {
-#pragma unroll
-          for (int m = 0; m < kNT; ++m) {
-            if (m < p.M) {
-              __stcg(p.t_buf + static_cast<size_t>(m) * p.r + lrow, z[m]);
-              if (p.T_save != nullptr) p.T_save[static_cast<size_t>(m) * p.r + lrow] = z[m];
-            }
-          }
-        }
-        __threadfence();
-        bar_sync_named<1, 128>();
-        if (et == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(t_ready), "r"(1u) : "memory");
-      } else {
-        if (!have_t) {
-          // T-ready was released by slice 0's combiner, normally long ago
-          if (et == 0) {
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(t_ready) == 0u) {
-              if (clock64() - t0 > kWaitLimitCycles) {
-                atomicOr(p.status, kStatusWaitTimeout);
-                break;
-              }
-            }
-          }
-          bar_sync_named<1, 128>();
-          __threadfence();
-#pragma unroll
-          for (int k = 0; k < kNT / 2; ++k) {
-            const int i = et + 128 * k;
-            const int m = i >> 6, c = i & 63;
-            Ts[i] = (m < p.M && c < p.r) ? __ldcg(p.t_buf + m * p.r + c) : 0.0f;
-          }
-          bar_sync_named<1, 128>();
-          have_t = true;
-        }
-        const int n = (slice - 1) * 128 + lrow;
-        if (n < p.d_out) {
-#pragma unroll 8
-          for (int c = 0; c < p.r; ++c) {
-            const float b = p.s * __bfloat162float(p.B[static_cast<size_t>(n) * p.r + c]);
-#pragma unroll
-            for (int m = 0; m < kNT; ++m) z[m] = fmaf(b, Ts[m * 64 + c], z[m]);
-          }
-#pragma unroll
-          for (int m = 0; m < kNT; ++m) {
-            if (m < p.M) {
-              float y = z[m];
-              if (p.act == LORA_ACT_SILU) {
-                if (p.Z_save != nullptr) p.Z_save[static_cast<size_t>(m) * p.d_out + n] = y;
-                y = y / (1.0f + expf(-y));
-              }
-              p.Y[static_cast<size_t>(m) * p.d_out + n] = __float2bfloat16_rn(y);
-            }
-          }
-        }
-      }
+      // ---- slice 0: T = X A^T from rows < r, then the T-ready flag
+      small_m_finish_t<kNT>(p, et);
+      __threadfence();
+      bar_sync_named<1, 128>();
       if (et == 0) {
-        sm_trace(p, kTrCombined);
-        p.counters[slice] = 0u;        // back to zero for the next call
-        const uint32_t done = atomicAdd(slices_done, 1u) + 1u;
-        if (done == static_cast<uint32_t>(p.slices)) {
-          // every slice is finished: slice 0 has released T and every other
-          // combiner has passed its wait for it
-          *slices_done = 0u;
-          *t_ready = 0u;
-        }
+        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.counters + 1 + p.wslices), "r"(1u) : "memory");
+        small_m_slice_done(p, 0);
       }
     }
   }
@@ -341,48 +444,49 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
 }
 
 template <int kNT>
-cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_small_m_kernel(const SmallMParams& p, cudaStream_t st) {
   using C = SmallMCfg<kNT>;
   auto k = small_m_kernel<kNT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
   cfg.blockDim = dim3(kSmThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs co-resident: a combiner may wait for slice 0
+  attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs resident: a finisher may wait for T
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k, p);
 }
 
-// Work split for a grid of at most `grid` CTAs: slices of [A ; W], units of
-// 128 K columns, equal contiguous runs.
+// Work split for at most `grid` CTAs: W's units in equal contiguous runs,
+// slice 0's K chunks one per CTA.
 struct SmallMSplit {
-  int slices = 0, nkc = 0, run = 0, n_w = 0, max_seg = 0;
+  int wslices = 0, nkc = 0, run = 0, grid = 0, nseg0 = 0, max_seg = 0;
 };
 
 inline SmallMSplit small_m_split(int64_t d_in, int64_t d_out, int grid) {
   SmallMSplit s;
-  s.slices = 1 + static_cast<int>((d_out + 127) / 128);
+  s.wslices = static_cast<int>((d_out + 127) / 128);
   s.nkc = static_cast<int>((d_in + 127) / 128);
-  const int units = s.slices * s.nkc;
+  const int units = s.wslices * s.nkc;
   s.run = (units + grid - 1) / grid;
-  s.n_w = (units + s.run - 1) / s.run;
-  for (int sl = 0; sl < s.slices; ++sl) {
+  s.grid = (units + s.run - 1) / s.run;
+  s.nseg0 = s.nkc < s.grid ? s.nkc : s.grid;
+  for (int sl = 0; sl < s.wslices; ++sl) {
     const int seg = (sl * s.nkc + s.nkc - 1) / s.run - (sl * s.nkc) / s.run + 1;
     if (seg > s.max_seg) s.max_seg = seg;
   }
   return s;
 }
 
-inline cudaError_t launch_small_m(const SmallMParams& p, int nt, int grid, cudaStream_t st) {
-  if (nt == 16) return launch_small_m_kernel<16>(p, grid, st);
-  if (nt == 32) return launch_small_m_kernel<32>(p, grid, st);
-  return launch_small_m_kernel<64>(p, grid, st);
+inline cudaError_t launch_small_m(const SmallMParams& p, int nt, cudaStream_t st) {
+  if (nt == 16) return launch_small_m_kernel<16>(p, st);
+  if (nt == 32) return launch_small_m_kernel<32>(p, st);
+  return launch_small_m_kernel<64>(p, st);
 }
 
 }  // namespace lora

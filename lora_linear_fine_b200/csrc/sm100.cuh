@@ -167,6 +167,14 @@ __device__ __forceinline__ void bar_sync_named() {
   asm volatile("barrier.cta.sync %0, %1;" ::"n"(id), "n"(n) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while its predecessor in the stream is finishing;
+// grid_dep_wait() blocks the calling thread until the predecessor grid has
+// completed and its memory operations are visible (without the attribute it
+// returns at once).  Every kernel here calls it from every thread after its
+// prologue (barriers, tensor memory) and before its first global access.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tensor core operand reads, TMA stores).
 __device__ __forceinline__ void fence_proxy_async_smem() {
