@@ -120,7 +120,13 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
  *           holding T = X A^T for the backward.
  *   Z_save: NULL, or fp32 output [M x d_out] (SwiGLU: Z_gate then Z_up, each
  *           [M x d_out]) holding the pre-activation; ignored for identity.
- *   workspace: device, >= lora_linear_workspace_size(desc, 0) bytes. */
+ *   workspace: device, >= lora_linear_workspace_size(desc, 0) bytes.
+ * Launches: kernels are stream-ordered and may start while the preceding
+ * kernel in the stream drains (programmatic dependent launch; each waits for
+ * its predecessor before touching memory).  With 1..64 tokens, identity or
+ * SiLU and r > 0 the forward is one cooperative launch of at most one CTA per
+ * SM (it fails with LORA_ERR_CUDA where the device cannot make the whole grid
+ * resident, e.g. under a partitioned device). */
 lora_status_t lora_linear_fwd(const lora_linear_desc* desc,
                               const void* X, const void* W, const void* A, const void* B,
                               const void* W_up, const void* A_up, const void* B_up,
