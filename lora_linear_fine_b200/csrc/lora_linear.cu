@@ -441,12 +441,17 @@ RankReduceJob reduce_job(const RankJob& J, int RP) {
 // Fixed-order reduction of up to two split results in one launch.
 lora_status_t launch_reduce(RankReduceJob* R, int n, cudaStream_t st) {
   if (n == 0) return LORA_OK;
-  if (n == 1) R[1] = R[0];
   long long blocks = 0;
   for (int i = 0; i < n; ++i) {
-    const long long b = (R[i].out.rows + kReduceRows - 1) / kReduceRows;
+    // rows per block: all kReduceRows while there are many rows, fewer (a
+    // power of two) so that a short result still spreads over >= 256 blocks
+    int rpb = kReduceRows;
+    while (rpb > 1 && (R[i].out.rows + rpb - 1) / rpb < 256) rpb >>= 1;
+    R[i].rpb = rpb;
+    const long long b = (R[i].out.rows + rpb - 1) / rpb;
     blocks = b > blocks ? b : blocks;
   }
+  if (n == 1) R[1] = R[0];
   long long gx = blocks;
   if (gx > 1184) gx = 1184;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(n), 1);

@@ -258,10 +258,11 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
 struct RankReduceJob {
   const float* partial;   // [splits][rows_pad][RP]
   int splits, rows_pad, RP;
+  int rpb;                // result rows per block (1..kReduceRows): fewer rows, more blocks, for few rows
   RankOut out;
 };
 
-// Blocks of kReduceRows result rows (grid-stride over row blocks; blockIdx.y
+// Blocks of rpb (<= kReduceRows) result rows (grid-stride over row blocks; blockIdx.y
 // selects the job).  Splits are summed in order into a shared-memory tile with
 // the column fastest (the partials' layout), each thread keeping up to
 // 2 elements x 8 splits of loads in flight; then row-major outputs are written
@@ -275,12 +276,13 @@ __global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, R
   __shared__ float tile[kReduceRows][65];
   const int r = J.out.r;
   const RankOut& o = J.out;
-  const int nblk = (J.out.rows + kReduceRows - 1) / kReduceRows;
+  const int rpb = J.rpb;
+  const int nblk = (J.out.rows + rpb - 1) / rpb;
   const size_t stride = static_cast<size_t>(J.rows_pad) * J.RP;   // between splits
   constexpr int kEPT = 2;
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
-    const int row0 = blk * kReduceRows;
-    const int nrows = J.out.rows - row0 < kReduceRows ? J.out.rows - row0 : kReduceRows;
+    const int row0 = blk * rpb;
+    const int nrows = J.out.rows - row0 < rpb ? J.out.rows - row0 : rpb;
     const int E = nrows * r;
     __syncthreads();
     for (int base = 0; base < E; base += 256 * kEPT) {
