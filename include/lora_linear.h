@@ -50,7 +50,7 @@
  *   check); they never clear it.  Zero it once with lora_linear_workspace_init
  *   before the first call; read it with lora_linear_device_status.
  * - Calls that share a workspace must not overlap in time (issue them on one
- *   stream): they use the same scratch regions and counters.
+ *   stream): they use the same scratch regions.
  */
 #ifndef LORA_LINEAR_H
 #define LORA_LINEAR_H
@@ -98,11 +98,10 @@ typedef struct lora_linear_desc {
  * backward serves both calls (one after the other, on one stream). */
 size_t lora_linear_workspace_size(const lora_linear_desc* desc, int for_backward);
 
-/* Zero the header of a workspace (asynchronous, on `stream`): the status word
- * and the arrival counters the few-token forward keeps there.  Both are zero
- * at rest; call this once after allocating the workspace, and again after any
- * call that left a non-zero status (an aborted call can leave counters set).
- * workspace_bytes must be at least the header (4352 bytes). */
+/* Zero the header of a workspace (asynchronous, on `stream`): the status
+ * block, whose word 0 is the status word.  Call this once after allocating
+ * the workspace, and again after any call that left a non-zero status.
+ * workspace_bytes must be at least the header (256 bytes). */
 lora_status_t lora_linear_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, copy the workspace status word to *out_status and
@@ -124,9 +123,9 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
  * Launches: kernels are stream-ordered and may start while the preceding
  * kernel in the stream drains (programmatic dependent launch; each waits for
  * its predecessor before touching memory).  With 1..64 tokens, identity or
- * SiLU and r > 0 the forward is one cooperative launch of at most one CTA per
- * SM (it fails with LORA_ERR_CUDA where the device cannot make the whole grid
- * resident, e.g. under a partitioned device). */
+ * SiLU and r > 0 the forward is one launch of thread-block clusters (one
+ * cluster of 1..16 CTAs per 128 output features; the cluster size is the
+ * largest the device reports it can keep resident for every slice at once). */
 lora_status_t lora_linear_fwd(const lora_linear_desc* desc,
                               const void* X, const void* W, const void* A, const void* B,
                               const void* W_up, const void* A_up, const void* B_up,
@@ -157,7 +156,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* desc,
  * status word and the kernel returns: no trap, the context stays usable.
  * Read the outcome with lora_linear_device_status; clear it with
  * lora_linear_workspace_init.
- *   workspace: device, >= 4352 bytes (the header), 16-byte aligned, else
+ *   workspace: device, >= 256 bytes (the header), 16-byte aligned, else
  *              LORA_ERR_WORKSPACE.
  *   limit_log2: 10..30, else LORA_ERR_INVALID_ARG. */
 lora_status_t lora_linear_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int limit_log2,

@@ -25,11 +25,8 @@ using namespace lora;
 constexpr int kAbiVersion = 1;
 constexpr int kTargetCtas = 148;   // SM count of a B200; sets split-K widths
 constexpr int64_t kKMajorMinTokens = 12288;   // dX from a W^T copy at and above this many tokens
-constexpr size_t kStatusBytes = 256;
-// Workspace header, zero at rest: the status block, then the arrival counters
-// of the few-token forward (one per 128-row slice of [A ; W], plus two).
-constexpr size_t kCounterWords = 1024;
-constexpr size_t kHeaderBytes = kStatusBytes + kCounterWords * 4;
+// Workspace header, zero at rest: the status block (word 0 is the status word).
+constexpr size_t kHeaderBytes = 256;
 
 // ---------------------------------------------------------------------------
 // debug logging (LORA_LINEAR_DEBUG=1)
@@ -154,16 +151,13 @@ struct Plan {
   // few-token forward
   bool small_m = false;
   int sm_nt = 16;                            // tokens padded to the MMA N granule
-  SmallMSplit sm;
-  size_t sm_t_buf = 0, sm_d_part0 = 0, sm_d_part = 0;
   size_t total = 0;
 };
 
 // The few-token forward applies to identity / SiLU with an adapter and at most
-// kSmallMMax tokens, while its slice counters fit the workspace header.
+// kSmallMMax tokens.
 bool small_m_applies(const lora_linear_desc* d) {
-  return d->M > 0 && d->M <= kSmallMMax && d->r > 0 && d->act != LORA_ACT_SWIGLU &&
-         static_cast<size_t>(3 + ceil_div(d->d_out, 128)) <= kCounterWords;
+  return d->M > 0 && d->M <= kSmallMMax && d->r > 0 && d->act != LORA_ACT_SWIGLU;
 }
 
 // Split-K width for a rank-r product with `tiles` row tiles and `nkb` 64-wide K blocks.
@@ -192,6 +186,13 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
   auto partials = [&](int splits, int64_t tiles) -> size_t {
     return splits > 1 ? take(static_cast<size_t>(splits) * tiles * 128 * P.RP * 4) : 0;
   };
+  if (!backward && small_m_applies(d)) {
+    // The few-token forward keeps everything on chip: no workspace regions.
+    P.small_m = true;
+    P.sm_nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    P.total = off;
+    return P;
+  }
   if (r > 0) {
     // The LoRA branch rides the GEMM's K-loop as extra K-blocks fed by a rank
     // pass (T = X A^T, U = dZ B computed once per token): no rank columns in
@@ -202,14 +203,6 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     if (!backward) P.t_ws = take(static_cast<size_t>(P.np) * M * r * 4);
   }
   if (!backward) {
-    if (small_m_applies(d)) {
-      P.small_m = true;
-      P.sm_nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-      P.sm = small_m_split(d->d_in, d->d_out, kTargetCtas);
-      P.sm_t_buf = take(static_cast<size_t>(M) * r * 4);
-      P.sm_d_part0 = take(static_cast<size_t>(P.sm.nseg0) * 128 * P.sm_nt * 4);
-      P.sm_d_part = take(static_cast<size_t>(P.sm.wslices) * P.sm.max_seg * 128 * P.sm_nt * 4);
-    }
     P.total = off;
     return P;
   }
@@ -763,8 +756,8 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   (void)RP;
   const int64_t M = d->M, r = d->r;
 
-  if (P.small_m && dev.sms >= kTargetCtas) {
-    // Few tokens: bound by reading W once; stream-K over all SMs.
+  if (P.small_m) {
+    // Few tokens: bound by reading W once; one cluster per 128-row slice of W.
     const int nt = P.sm_nt;
     SmallMParams q;
     std::memset(&q, 0, sizeof(q));
@@ -776,10 +769,6 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     q.Y = static_cast<__nv_bfloat16*>(Y);
     q.T_save = T_save;
     q.Z_save = d->act == LORA_ACT_SILU ? Z_save : nullptr;
-    q.t_buf = reinterpret_cast<float*>(ws + P.sm_t_buf);
-    q.d_part0 = reinterpret_cast<float*>(ws + P.sm_d_part0);
-    q.d_part = reinterpret_cast<float*>(ws + P.sm_d_part);
-    q.counters = reinterpret_cast<uint32_t*>(ws + kStatusBytes);
     q.status = status;
     q.M = static_cast<int>(M);
     q.d_in = static_cast<int>(d->d_in);
@@ -787,15 +776,12 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     q.r = static_cast<int>(r);
     q.s = d->s;
     q.act = d->act;
-    q.wslices = P.sm.wslices;
-    q.nkc = P.sm.nkc;
-    q.run = P.sm.run;
-    q.grid = P.sm.grid;
-    q.nseg0 = P.sm.nseg0;
-    q.max_seg = P.sm.max_seg;
-    const int grid = q.grid;
-    LORA_LOG("small_m M=%d nt=%d wslices=%d nkc=%d run=%d grid=%d nseg0=%d max_seg=%d", (int)M, nt, q.wslices, q.nkc,
-             q.run, grid, q.nseg0, q.max_seg);
+    const int slices = static_cast<int>(ceil_div(d->d_out, 128));
+    q.splits = small_m_splits(nt, d->d_in, d->d_out);
+    q.kb_per = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), q.splits));
+    const int grid = slices * q.splits;
+    LORA_LOG("small_m M=%d nt=%d slices=%d splits=%d kb_per=%d grid=%d", (int)M, nt, slices, q.splits, q.kb_per,
+             grid);
     // LORA_LINEAR_DEBUG=2: per-CTA phase stamps, printed after the launch
     // (synchronises the stream; for debugging only).
     static unsigned long long* trace = nullptr;
@@ -806,7 +792,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
       q.trace = trace;
       cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTracePoints, st);
     }
-    const cudaError_t e = launch_small_m(q, nt, st);
+    const cudaError_t e = launch_small_m(q, nt, slices, pdl_enabled(), st);
     if (e != cudaSuccess) {
       LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
       g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -1179,7 +1165,7 @@ lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, 
   }
   void* ws = nullptr;
   LORA_TRY(noalloc_scratch(&ws));
-  // The header (status word, slice counters) must start at zero; everything
+  // The header (status word) must start at zero; everything
   // else the forward writes before it reads.
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return cuda_error("cudaMemsetAsync(scratch status)");
