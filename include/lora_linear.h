@@ -34,12 +34,14 @@
  *   default stream) and never synchronises, except
  *   lora_linear_device_status which reads the status word back.
  * - Alignment: every tensor pointer is 16-byte aligned; d_in % 8 == 0,
- *   d_out % 8 == 0; r % 8 == 0 with 0 <= r <= 64.  Violations return
+ *   d_out % 8 == 0; r % 8 == 0 with 0 <= r <= 128.  Violations return
  *   LORA_ERR_ALIGNMENT (pointers, strides) or LORA_ERR_UNSUPPORTED (r) before
  *   anything is launched.
  * - r == 0 is a plain linear layer: A, B (and the _up twins) may be NULL and
  *   T_save is ignored.
- * - M may be 0 (nothing is launched; dA/dB are zero-filled in the backward).
+ * - M may be 0: the per-token tensors (X, Y, T_save, Z_save, dY, dX) are
+ *   empty and may be NULL; the forward launches nothing and the backward
+ *   zero-fills dA and dB.
  * - Outputs are overwritten, never accumulated into.
  * - Results: Y and dX are bf16 (round to nearest even of fp32 accumulators);
  *   T_save, Z_save, dA, dB are fp32.

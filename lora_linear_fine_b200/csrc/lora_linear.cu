@@ -110,7 +110,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int rank_pad(int64_t r) { return r == 0 ? 0 : (r <= 16 ? 16 : (r <= 32 ? 32 : 64)); }
+int rank_pad(int64_t r) { return r == 0 ? 0 : (r <= 16 ? 16 : (r <= 32 ? 32 : (r <= 64 ? 64 : 128))); }
 
 lora_status_t check_desc(const lora_linear_desc* d) {
   if (d == nullptr) return LORA_ERR_INVALID_ARG;
@@ -119,14 +119,14 @@ lora_status_t check_desc(const lora_linear_desc* d) {
   if (d->M > (int64_t(1) << 31) - 1 || d->d_in > (int64_t(1) << 30) || d->d_out > (int64_t(1) << 30))
     return LORA_ERR_UNSUPPORTED;
   if (d->d_in % 8 != 0 || d->d_out % 8 != 0) return LORA_ERR_ALIGNMENT;
-  if (d->r % 8 != 0 || d->r > 64) return LORA_ERR_UNSUPPORTED;
+  if (d->r % 8 != 0 || d->r > 128) return LORA_ERR_UNSUPPORTED;
   return LORA_OK;
 }
 
 // Workspace layouts (offsets in bytes, each 256-aligned, status word at 0).
 struct Plan {
   int np = 1;              // projections: 2 for SwiGLU (gate, up)
-  int RP = 0;              // r padded to the MMA granule (0, 16, 32, 64)
+  int RP = 0;              // r padded to the MMA granule (0, 16, 32, 64, 128)
   bool act_f16 = false;    // backward with an activation: fp16 dZ operands
   int64_t M8 = 8;
   // split-K widths of the rank passes (1 = results written directly)
@@ -154,10 +154,10 @@ struct Plan {
   size_t total = 0;
 };
 
-// The few-token forward applies to identity / SiLU with an adapter and at most
-// kSmallMMax tokens.
+// The few-token forward applies to identity / SiLU with an adapter of rank at
+// most 64 and at most kSmallMMax tokens.
 bool small_m_applies(const lora_linear_desc* d) {
-  return d->M > 0 && d->M <= kSmallMMax && d->r > 0 && d->act != LORA_ACT_SWIGLU;
+  return d->M > 0 && d->M <= kSmallMMax && d->r > 0 && d->r <= 64 && d->act != LORA_ACT_SWIGLU;
 }
 
 // Split-K width for a rank-r product with `tiles` row tiles and `nkb` 64-wide K blocks.
@@ -227,7 +227,10 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
     }
     const int64_t tiles_a = ceil_div(d->d_in, 128), tiles_b = ceil_div(d->d_out, 128);
     const int64_t nkb_tok = ceil_div(M > 0 ? M : 1, 64);
-    P.dual = d->act == LORA_ACT_IDENTITY;
+    // U and dB from one read of dY: identity, and r <= 64 (at r = 128 the
+    // two accumulators and both B operands leave too little tensor and
+    // shared memory)
+    P.dual = d->act == LORA_ACT_IDENTITY && P.RP <= 64;
     if (P.dual) {
       P.sp_dual = rank2d_split(static_cast<int>(tiles_m), static_cast<int>(tiles_b), P.RP, true, true,
                                rank2d_max_rb(P.RP), kTargetCtas);
@@ -355,6 +358,7 @@ lora_status_t launch_rank_rp(int RP, const RankGemmParams& p, int splits, cudaSt
     case 16: return launch_rank<kAMN, 16, kNA, kNB, kF16>(p, splits, st);
     case 32: return launch_rank<kAMN, 32, kNA, kNB, kF16>(p, splits, st);
     case 64: return launch_rank<kAMN, 64, kNA, kNB, kF16>(p, splits, st);
+    case 128: return launch_rank<kAMN, 128, kNA, kNB, kF16>(p, splits, st);
     default: return LORA_ERR_UNSUPPORTED;
   }
 }
@@ -397,7 +401,7 @@ lora_status_t run_rank_gemm(const RankJob& J, int RP, int r, uint32_t* status, c
   RankGemmParams q;
   std::memset(&q, 0, sizeof(q));
   bool ok = true;
-  const int ks = J.na == 1 ? 2 : 1;   // 64-wide K blocks per stage (RankCfg::kKS)
+  const int ks = rank_ks(J.na, RP);   // 64-wide K blocks per stage (RankCfg::kKS)
   for (int i = 0; i < J.na; ++i)
     ok = ok && make_tm(&q.tm_a[i], J.a[i], J.a_inner, J.a_outer, J.a_ld, 64, J.a_mn ? 64 * ks : 128, J.f16);
   for (int i = 0; i < J.nb; ++i) ok = ok && make_tm(&q.tm_b[i], J.b[i], J.b_inner, r, J.b_ld, 64, RP, J.f16);
@@ -486,6 +490,9 @@ lora_status_t launch_rank2d_rp(int RP, const Rank2dParams& p, int grid, cudaStre
     case 16: return launch_rank2d_t<16, kRow, kCol>(p, grid, st);
     case 32: return launch_rank2d_t<32, kRow, kCol>(p, grid, st);
     case 64: return launch_rank2d_t<64, kRow, kCol>(p, grid, st);
+    case 128:
+      if constexpr (!kRow) return launch_rank2d_t<128, kRow, kCol>(p, grid, st);   // col product only
+      else return LORA_ERR_UNSUPPORTED;
     default: return LORA_ERR_UNSUPPORTED;
   }
 }
@@ -739,7 +746,8 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
                               float* Z_save, void* workspace, size_t workspace_bytes, void* stream) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
-  if (X == nullptr || W == nullptr || Y == nullptr) return LORA_ERR_INVALID_ARG;
+  // with M == 0 the per-token tensors are empty and may be NULL
+  if (W == nullptr || (d->M > 0 && (X == nullptr || Y == nullptr))) return LORA_ERR_INVALID_ARG;
   if (d->r > 0 && (A == nullptr || B == nullptr)) return LORA_ERR_INVALID_ARG;
   if (swiglu && (W_up == nullptr || (d->r > 0 && (A_up == nullptr || B_up == nullptr)))) return LORA_ERR_INVALID_ARG;
   const void* ptrs[] = {X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save};
@@ -762,7 +770,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     SmallMParams q;
     std::memset(&q, 0, sizeof(q));
     if (!make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128) ||
-        !make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, 128) ||
+        !make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, static_cast<uint32_t>(align_up(static_cast<size_t>(r), 16))) ||
         !make_tm(&q.tm_x, X, d->d_in, M, d->d_in, 64, static_cast<uint32_t>(nt)))
       return LORA_ERR_CUDA;
     q.B = static_cast<const __nv_bfloat16*>(B);
@@ -776,6 +784,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
     q.r = static_cast<int>(r);
     q.s = d->s;
     q.act = d->act;
+    q.a_rows = static_cast<int>(align_up(static_cast<size_t>(r), 16));
     const int slices = static_cast<int>(ceil_div(d->d_out, 128));
     q.splits = small_m_splits(nt, d->d_in, d->d_out);
     q.kb_per = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), q.splits));
@@ -805,7 +814,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
       unsigned long long t0 = ~0ull;
       for (int b = 0; b < grid; ++b) t0 = h[b * kSmTracePoints] && h[b * kSmTracePoints] < t0 ? h[b * kSmTracePoints] : t0;
       static const char* names[kSmTracePoints] = {"entry", "first_issue", "first_data", "last_mma", "published",
-                                                  "combined", "exit"};
+                                                  "synced", "t_summed", "combined", "exit"};
       for (int k = 0; k < kSmTracePoints; ++k) {
         double mn = 1e30, mx = 0, sum = 0;
         int n = 0;
@@ -881,12 +890,13 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
                               float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
-  if (dY == nullptr || X == nullptr || W == nullptr || dX == nullptr) return LORA_ERR_INVALID_ARG;
+  // with M == 0 the per-token tensors are empty and may be NULL
+  if (W == nullptr || (d->M > 0 && (dY == nullptr || X == nullptr || dX == nullptr))) return LORA_ERR_INVALID_ARG;
   if (d->r > 0 && (A == nullptr || B == nullptr || dA == nullptr || dB == nullptr)) return LORA_ERR_INVALID_ARG;
   if (swiglu && (W_up == nullptr || (d->r > 0 && (A_up == nullptr || B_up == nullptr || dA_up == nullptr ||
                                                   dB_up == nullptr))))
     return LORA_ERR_INVALID_ARG;
-  if (d->act != LORA_ACT_IDENTITY && Z_save == nullptr) return LORA_ERR_INVALID_ARG;
+  if (d->act != LORA_ACT_IDENTITY && d->M > 0 && Z_save == nullptr) return LORA_ERR_INVALID_ARG;
   const void* ptrs[] = {dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;

@@ -5,8 +5,9 @@
 //   backward  dX = dZ W  + s U A    = [ dZ | sU ] [ W ; A ]       (U = dZ B)
 //
 // T (U) comes from the rank pass (lora_rank.cuh), which also writes s*T as bf16
-// [M x r]; the GEMM's last K-block(s) per tile multiply that tile of s*T (K = r,
-// zero-filled by TMA up to the 64-wide block) with the matching rows of B (A).
+// [M x r]; the GEMM's last K-blocks per tile (one per 64 of r and projection)
+// multiply that tile of s*T (K = r, zero-filled by TMA up to a whole 64-wide
+// block) with the matching rows of B (A).
 // The up-projection thus runs on the tensor cores inside the same accumulator,
 // with no hand-off between the epilogue and the MMA issuer, which leaves the
 // tensor memory free for a double-buffered accumulator: 2 x 256 fp32 columns.
@@ -49,7 +50,7 @@ struct MmaParams {
   CUtensorMap tm_la[2];   // LoRA block, M side           s*T_j / s*U_j   bf16 [M x r]
   CUtensorMap tm_lb[2];   // LoRA block, N side           fwd: B_j [d_out x r]   bwd: A_j (b_mn) or A_j^T
   int M, N, K;            // output rows / columns (per projection for SwiGLU fwd) / reduction per pair
-  int lora_ksteps;        // 16-wide K steps of the LoRA block: ceil(r / 16); 0 = no LoRA block
+  int lora_ksteps;        // 16-wide K steps of a projection's LoRA blocks: ceil(r / 16) <= 8; 0 = none
   __nv_bfloat16* out;     // [M x N]
   float* z_save;          // [npair][M x N] fp32 or null (SiLU / SwiGLU forward)
   uint32_t* status;
@@ -67,7 +68,7 @@ struct MmaCfg {
   static constexpr int kTileM = 128 * kCtas;                 // rows per (pair) tile
   static constexpr int kOutCols = kSwigluFwd ? 128 : 256;    // output columns per tile
   static constexpr int kKPairs = kBwd ? kNPair : 1;          // projections walked along K
-  static constexpr int kLoraBlocks = kNPair;                 // LoRA K-blocks per tile
+  static constexpr int kLoraProj = kNPair;                   // projections with a LoRA branch per tile
   static constexpr int kABytes = 128 * 64 * 2;               // 16 KB
   static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
   static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
@@ -162,7 +163,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   const uint32_t tbase = *tmem_slot;
   grid_dep_wait();
   const int nkb = (p.K + 63) / 64;
-  const int nlora = p.lora_ksteps > 0 ? C::kLoraBlocks : 0;
+  const int lkb = (p.lora_ksteps + 3) / 4;                   // 64-wide LoRA K-blocks per projection
+  const int nlora = C::kLoraProj * lkb;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -221,22 +223,25 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               load(sb, &p.tm_w[j], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
             }
           } else {
-            // LoRA block of projection j: s*T_j (s*U_j) rows and B_j (A_j) rows, K = r zero-padded to 64
-            const int j = blk - C::kKPairs * nkb;
-            load(sa, &p.tm_la[j], fb, 0, m0, pol_keep);
+            // LoRA block of projection j: s*T_j (s*U_j) rows and B_j (A_j) rows,
+            // K = r columns [kx, kx + 64) of the rank, zero-filled past r
+            const int lb = blk - C::kKPairs * nkb;
+            const int j = lb / lkb;
+            const int kx = (lb - j * lkb) * 64;
+            load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
             if constexpr (!kBwd) {
               if constexpr (C::kSwigluFwd) {
                 // N = 128 outputs of projection j: 128 rows (single) or 64 per CTA (pair)
-                load(sb, &p.tm_lb[j], fb, 0, n0 + 64 * static_cast<int>(crank), pol_keep);
+                load(sb, &p.tm_lb[j], fb, kx, n0 + 64 * static_cast<int>(crank), pol_keep);
               } else {
-                load(sb, &p.tm_lb[0], fb, 0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+                load(sb, &p.tm_lb[0], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
               }
             } else if (p.b_mn) {
 #pragma unroll
               for (int b = 0; b < C::kBRows / 64; ++b)
-                load(sb + b * 8192, &p.tm_lb[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, 0, pol_keep);
+                load(sb + b * 8192, &p.tm_lb[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, kx, pol_keep);
             } else {
-              load(sb, &p.tm_lb[j], fb, 0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);   // A^T rows
+              load(sb, &p.tm_lb[j], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);   // A^T rows
             }
           }
           ++issued;
@@ -296,9 +301,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               mma(dacc, da, db, kIdMain, (blk == 0 && kk == 0) ? 0u : 1u);
             }
           } else {
-            const int j = blk - C::kKPairs * nkb;
+            const int lb = blk - C::kKPairs * nkb;
+            const int j = lb / lkb;
+            const int steps = p.lora_ksteps - 4 * (lb - j * lkb);     // this block's 16-wide steps
             const uint32_t dcol = C::kSwigluFwd ? static_cast<uint32_t>(128 * j) : 0u;
-            for (int kk = 0; kk < p.lora_ksteps; ++kk) {
+            for (int kk = 0; kk < (steps < 4 ? steps : 4); ++kk) {
               const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
               const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
               mma(dacc + dcol, da, db, kIdLora, 1u);
@@ -339,23 +346,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
       const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
-      uint32_t v[128];
-      if constexpr (C::kSwigluFwd) {
-        tmem_ld32(tl + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tl + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_ld32(tl + 128 + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
-        tmem_ld32(tl + 128 + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tl + h * 128 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      if constexpr (kPair) mbar_arrive_cluster(acc_empty_addr[buf]);
-      else mbar_arrive(&acc_empty[buf]);
+      auto release_acc = [&]() {
+        tc_fence_before();
+        if constexpr (kPair) mbar_arrive_cluster(acc_empty_addr[buf]);
+        else mbar_arrive(&acc_empty[buf]);
+      };
       if constexpr (C::kStaged) {
-        // Stage 32 rows x 8 uint4 (this lane's row) through shared memory,
-        // then store them row-contiguous: 8 lanes cover 128 bytes of a row.
+        // Two halves of this thread's columns (SiLU: 64 + 64 of its 128;
+        // SwiGLU: 32 + 32 gate columns with their up columns), so that only 64
+        // accumulator values are live at a time.  Rows go out through shared
+        // memory, 32 rows x 8 uint4 per flush, then row-contiguous: 8 lanes
+        // cover 128 bytes of a row.
         const int row0 = row - lane;                 // first row of this warp's 32
         uint4* stg = reinterpret_cast<uint4*>(epi_stage + ew * 4096);
         auto flush = [&](const uint4 (&mine)[8], auto&& store) {
@@ -369,58 +370,95 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           }
           __syncwarp();
         };
-        const int ncol = C::kSwigluFwd ? 64 : 128;         // columns of this thread
         const int col0 = C::kSwigluFwd ? nt * 128 + h * 64 : nt * 256 + h * 128;
-        if (p.z_save != nullptr) {
-          // fp32 Z: 32 columns per flush (gate then up for SwiGLU)
+        uint32_t ylo[16];                            // SwiGLU: packed bf16 Y of the first half
 #pragma unroll
-          for (int part = 0; part < (C::kSwigluFwd ? 2 : 1); ++part) {
-            float* zdst = p.z_save + static_cast<size_t>(part) * p.M * p.N;
+        for (int hv = 0; hv < 2; ++hv) {
+          uint32_t v[64];
+          if constexpr (C::kSwigluFwd) {
+            tmem_ld32(tl + h * 64 + 32 * hv, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));          // gate
+            tmem_ld32(tl + 128 + h * 64 + 32 * hv, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));   // up
+          } else {
+            tmem_ld32(tl + h * 128 + 64 * hv, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld32(tl + h * 128 + 64 * hv + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          }
+          tmem_wait_ld();
+          if (hv == 1) release_acc();
+          if (p.z_save != nullptr) {
+            // fp32 Z, 32 columns per flush: SwiGLU gate then up; SiLU two column runs
 #pragma unroll
-            for (int cb = 0; cb < ncol; cb += 32) {
+            for (int part = 0; part < 2; ++part) {
+              float* zdst = p.z_save + (C::kSwigluFwd ? static_cast<size_t>(part) * p.M * p.N : 0);
+              const int zc0 = C::kSwigluFwd ? col0 + 32 * hv : col0 + 64 * hv + 32 * part;
               uint4 mine[8];
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const int c = part * 64 + cb + 4 * j;
+                const int c = part * 32 + 4 * j;
                 mine[j] = make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]);
               }
               flush(mine, [&](int grow, int j, uint4 val) {
-                const int col = col0 + cb + 4 * j;
+                const int col = zc0 + 4 * j;
                 if (col < p.N) st_global_v4_hint(zdst + static_cast<size_t>(grow) * p.N + col, val, pol_out);
               });
             }
           }
-        }
-        // bf16 Y: 64 columns per flush
+          if constexpr (C::kSwigluFwd) {
+            // bf16 Y = SiLU(gate) * up: 32 columns per half, one 64-column flush
+            uint32_t y[16];
 #pragma unroll
-        for (int cb = 0; cb < ncol; cb += 64) {
-          uint4 mine[8];
+            for (int e = 0; e < 16; ++e) {
+              float yy[2];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float yv[8];
+              for (int k = 0; k < 2; ++k) {
+                const float g = __uint_as_float(v[2 * e + k]);
+                const float u = __uint_as_float(v[32 + 2 * e + k]);
+                yy[k] = g / (1.0f + expf(-g)) * u;
+              }
+              y[e] = pack_bf16x2(yy[0], yy[1]);
+            }
+            if (hv == 0) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int c = cb + 8 * j + e;
-              if constexpr (C::kSwigluFwd) {
-                const float g = __uint_as_float(v[c]);
-                const float u = __uint_as_float(v[64 + c]);
-                yv[e] = g / (1.0f + expf(-g)) * u;
-              } else {
-                const float z = __uint_as_float(v[c]);
+              for (int e = 0; e < 16; ++e) ylo[e] = y[e];
+            } else {
+              uint4 mine[8];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                mine[j] = make_uint4(ylo[4 * j], ylo[4 * j + 1], ylo[4 * j + 2], ylo[4 * j + 3]);
+                mine[4 + j] = make_uint4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+              }
+              flush(mine, [&](int grow, int j, uint4 val) {
+                const int col = col0 + 8 * j;
+                if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
+              });
+            }
+          } else {
+            // bf16 Y = SiLU(z): 64 columns per half, one flush
+            uint4 mine[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float yv[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float z = __uint_as_float(v[8 * j + e]);
                 yv[e] = z / (1.0f + expf(-z));
               }
+              mine[j].x = pack_bf16x2(yv[0], yv[1]);
+              mine[j].y = pack_bf16x2(yv[2], yv[3]);
+              mine[j].z = pack_bf16x2(yv[4], yv[5]);
+              mine[j].w = pack_bf16x2(yv[6], yv[7]);
             }
-            mine[j].x = pack_bf16x2(yv[0], yv[1]);
-            mine[j].y = pack_bf16x2(yv[2], yv[3]);
-            mine[j].z = pack_bf16x2(yv[4], yv[5]);
-            mine[j].w = pack_bf16x2(yv[6], yv[7]);
+            flush(mine, [&](int grow, int j, uint4 val) {
+              const int col = col0 + 64 * hv + 8 * j;
+              if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
+            });
           }
-          flush(mine, [&](int grow, int j, uint4 val) {
-            const int col = col0 + cb + 8 * j;
-            if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
-          });
         }
       } else {
+        uint32_t v[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tl + h * 128 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+        tmem_wait_ld();
+        release_acc();
         if (!row_ok) continue;
         const int col0 = nt * 256 + h * 128;
         const size_t base = static_cast<size_t>(row) * p.N + col0;

@@ -1,7 +1,7 @@
 // lora_rank.cuh — kernels for the rank-r side of the backward.
 //
 // rank_gemm_kernel: a split-K tcgen05 kernel for products whose result has
-//   only r (<= 64) columns and whose reduction runs over tokens or features:
+//   only r (<= 128) columns and whose reduction runs over tokens or features:
 //     dA^T = X^T (s U)           [d_in  x r],  K = tokens   (X read MN-major)
 //     dB   = dZ^T (s T)          [d_out x r],  K = tokens   (dZ read MN-major)
 //     U_lo = dZ_lo B, T = X A^T  [M x r],      K = features (K-major)
@@ -97,11 +97,16 @@ struct RankGemmParams {
 // per B operand kKS boxes of RP rows x 64.  Larger TMA boxes and several
 // boxes per stage keep more DRAM traffic in flight per request (measured:
 // 8 KB boxes stream at about half the rate of 32-64 KB stages).
+// 64-wide K blocks per pipeline stage of rank_gemm_kernel: two for a single A
+// operand of rank <= 64, else one (so that a stage stays within a quarter of
+// shared memory).  The host sizes its TMA boxes and K splits with the same rule.
+constexpr int rank_ks(int na, int rp) { return (na == 1 && rp <= 64) ? 2 : 1; }
+
 template <bool kAMN, int kRP, int NA, int NB, bool kF16>
 struct RankCfg {
   static constexpr int kNA = NA;
   static constexpr int kNB = NB;
-  static constexpr int kKS = NA == 1 ? 2 : 1;             // 64-wide K blocks per stage
+  static constexpr int kKS = rank_ks(NA, kRP);             // 64-wide K blocks per stage
   static constexpr int kABytes = 128 * 64 * 2 * kKS;      // one A operand per stage
   static constexpr int kBBox = kRP * 128;                 // one B box (64 K)
   static constexpr int kBBytes = kBBox * kKS;             // one B operand per stage
@@ -269,11 +274,12 @@ struct RankReduceJob {
 // column-fastest and transposed outputs row-fastest, so every global access is
 // coalesced.
 constexpr int kReduceRows = 32;
+constexpr int kMaxRank = 128;
 
 __global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, RankReduceJob j1) {
   grid_dep_wait();
   const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
-  __shared__ float tile[kReduceRows][65];
+  __shared__ float tile[kReduceRows][kMaxRank + 1];
   const int r = J.out.r;
   const RankOut& o = J.out;
   const int rpb = J.rpb;

@@ -7,7 +7,9 @@
 // CTA per SM); the CTAs of a cluster split the K dimension.  Per 64-wide K
 // block one TMA stage brings
 //   W tile [128 rows x 64]                    -> Z^T partial  D_Z [128 x kNT] += W  X^T
-//   A tile [128 rows x 64], rows >= r zero    -> T^T partial  D_T [128 x kNT] += A  X^T
+//   A tile [a_rows x 64] into a 128-row slot  -> T^T partial  D_T [128 x kNT] += A  X^T
+//     (a_rows = r rounded up to 16, rows >= r zero; the slot's other rows hold
+//     stale data, so rows >= a_rows of D_T are garbage and never read)
 //   X tile [kNT tokens x 64], rows >= M zero
 // (swap-AB: the weight rows are the M side of the MMA, the tokens are N).
 // Every cluster covers all of K, so each computes the full T for itself: no
@@ -31,7 +33,7 @@ constexpr int kSmMaxCluster = 16;
 
 struct SmallMParams {
   CUtensorMap tm_w;          // W [d_out x d_in], box 64 x 128
-  CUtensorMap tm_a;          // A [r x d_in],     box 64 x 128 (rows >= r zero-filled)
+  CUtensorMap tm_a;          // A [r x d_in],     box 64 x a_rows (rows >= r zero-filled)
   CUtensorMap tm_x;          // X [M x d_in],     box 64 x kNT (rows >= M zero-filled)
   const __nv_bfloat16* B;    // [d_out x r]
   __nv_bfloat16* Y;          // [M x d_out]
@@ -43,12 +45,14 @@ struct SmallMParams {
   int act;
   int splits;                // CTAs per cluster (K splits)
   int kb_per;                // 64-wide K blocks per CTA
+  int a_rows;                // rows of A loaded per K block: r rounded up to 16
   unsigned long long* trace; // null, or [grid][kSmTracePoints] globaltimer stamps (debugging)
 };
 
 // Trace points of one CTA (LORA_LINEAR_DEBUG=2 prints them per launch).
 enum SmTrace : int {
-  kTrEntry = 0, kTrFirstIssue, kTrFirstData, kTrLastMma, kTrPublished, kTrCombined, kTrExit, kSmTracePoints
+  kTrEntry = 0, kTrFirstIssue, kTrFirstData, kTrLastMma, kTrPublished, kTrSynced, kTrTSummed, kTrCombined, kTrExit,
+  kSmTracePoints
 };
 
 __device__ __forceinline__ void sm_trace(const SmallMParams& p, int point) {
@@ -59,26 +63,43 @@ __device__ __forceinline__ void sm_trace(const SmallMParams& p, int point) {
   }
 }
 
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
   return v;
+}
+
+// Sum of the float4 at shared offset `saddr` over the cluster's first
+// `splits` CTAs, in rank order.  All loads are issued before the first add.
+__device__ __forceinline__ float4 cluster_sum4(uint32_t saddr, int splits) {
+  float4 v[kSmMaxCluster];
+#pragma unroll
+  for (int qq = 0; qq < kSmMaxCluster; ++qq)
+    if (qq < splits) v[qq] = ld_dsmem_f32x4(mapa_shared(saddr, static_cast<uint32_t>(qq)));
+  float4 t = v[0];
+#pragma unroll
+  for (int qq = 1; qq < kSmMaxCluster; ++qq)
+    if (qq < splits) { t.x += v[qq].x; t.y += v[qq].y; t.z += v[qq].z; t.w += v[qq].w; }
+  return t;
 }
 
 template <int kNT>
 struct SmallMCfg {
   static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64
-  static constexpr int kABox = 128 * 64 * 2;            // A tile: 128 rows (r real) x 64
+  static constexpr int kABox = 128 * 64 * 2;            // A slot: 128 rows, the first a_rows loaded
   static constexpr int kXBox = kNT * 64 * 2;            // X tile: kNT rows x 64
   static constexpr int kStageBytes = kWBox + kABox + kXBox;
-  static constexpr int kLd = kNT + 1;                   // parked row stride (floats): conflict-free columns
+  static constexpr int kLd = kNT + 4;                   // parked row stride (floats): 16-byte rows, conflict-free float4 stores
   static constexpr int kBsBytes = 128 * 65 * 4;         // B rows of this CTA's features, fp32, stride r + 1
   static constexpr int kTailBytes = 1024 + kBsBytes + 1024;   // barriers, B rows, alignment slack
   static constexpr int kStages0 = (kSmemLimitBytes - kTailBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
   static constexpr uint32_t kTmemCols = (2 * kNT) <= 32 ? 32 : ((2 * kNT) <= 64 ? 64 : 128);
-  // after the K loop the ring holds: Dp [128][kLd], Tp [128][kLd], Tf [kNT][64]
+  // after the K loop the ring holds: Dp [128][kLd], Tp [128][kLd], Tf [64][kNT]
   static constexpr int kParkBytes = 2 * 128 * kLd * 4 + kNT * 64 * 4;
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kStages >= 3, "ring too shallow");
@@ -101,7 +122,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   float* Bs = reinterpret_cast<float*>(smem + S * C::kStageBytes + 1024);   // [F][r + 1]
   float* Dp = reinterpret_cast<float*>(smem);                               // [128][kLd]  Z^T partial
   float* Tp = Dp + 128 * C::kLd;                                            // [128][kLd]  T^T partial
-  float* Tf = Tp + 128 * C::kLd;                                            // [kNT][64]   summed T
+  float* Tf = Tp + 128 * C::kLd;                                            // [64][kNT]   summed T, tokens contiguous
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -127,6 +148,11 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&p.tm_w);
+    tma_prefetch_desc(&p.tm_a);
+    tma_prefetch_desc(&p.tm_x);
+  }
   grid_dep_wait();
   if (threadIdx.x == 0) sm_trace(p, kTrEntry);
 
@@ -138,7 +164,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
         const int k0 = (kb0 + i) * 64;
-        mbar_arrive_expect_tx(&full[rp.stage], C::kStageBytes);
+        mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kWBox + C::kXBox + p.a_rows * 128));
         tma_load_2d(st, &p.tm_w, &full[rp.stage], k0, slice * 128);
         tma_load_2d_hint(st + C::kWBox, &p.tm_a, &full[rp.stage], k0, 0, pol_x);
         tma_load_2d_hint(st + C::kWBox + C::kABox, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
@@ -183,7 +209,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
     const int et = threadIdx.x - 64;
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int lrow = q * 32 + lane;
-    // this CTA's rows of B, as fp32 with a padded stride (loaded during the K loop)
+    // this CTA's F rows of B, as fp32 with a padded stride, loaded during the K loop
     for (int i = et; i < F * p.r; i += 128) {
       const int fl = i / p.r, c = i - fl * p.r;
       const int n = slice * 128 + f0 + fl;
@@ -191,28 +217,47 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
     }
     bool got = true;
     if (nk > 0) got = mbar_wait(acc_full, 0, ctl);
-    if (bar_sync_and<1, 128>(got)) {
+    const bool ok = bar_sync_and<1, 128>(got);
+    // only the first r rows of the T partial are real (warp-uniform test)
+    const bool t_rows = q * 32 < p.r;
+    float4* drow = reinterpret_cast<float4*>(Dp + lrow * C::kLd);
+    float4* trow = reinterpret_cast<float4*>(Tp + lrow * C::kLd);
+    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
+    if (ok && t_rows) {
       if (nk > 0) {
         tc_fence_after();
-        const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
         for (int c0 = 0; c0 < kNT; c0 += 16) {
-          uint32_t v[16], t[16];
-          tmem_ld16(tl + c0, v);
+          uint32_t t[16];
           tmem_ld16(tl + kNT + c0, t);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            Dp[lrow * C::kLd + c0 + c] = __uint_as_float(v[c]);
-            Tp[lrow * C::kLd + c0 + c] = __uint_as_float(t[c]);
-          }
+          for (int c = 0; c < 16; c += 4)
+            trow[(c0 + c) / 4] = make_float4(__uint_as_float(t[c]), __uint_as_float(t[c + 1]),
+                                             __uint_as_float(t[c + 2]), __uint_as_float(t[c + 3]));
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < kNT; ++c) {
-          Dp[lrow * C::kLd + c] = 0.0f;
-          Tp[lrow * C::kLd + c] = 0.0f;
+        for (int c = 0; c < kNT / 4; ++c) trow[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+    }
+    if (ok) {
+      // Z partial of feature row lrow
+      if (nk > 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < kNT; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tl + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            drow[(c0 + c) / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                             __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
         }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kNT / 4; ++c) drow[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       }
     }
     if (et == 0) sm_trace(p, kTrPublished);
@@ -224,43 +269,71 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
 
   if (warp >= 2 && *abort_flag == 0u) {
     const int et = threadIdx.x - 64;
+    if (et == 0) sm_trace(p, kTrSynced);
     const uint32_t dp_addr = smem_u32(Dp), tp_addr = smem_u32(Tp);
-    // T[m][c] = sum over the cluster's ranks (in order) of T^T[c][m]
-    for (int i = et; i < p.M * p.r; i += 128) {
-      const int c = i / p.M, m = i - c * p.M;
-      const uint32_t off = static_cast<uint32_t>((c * C::kLd + m) * 4);
-      float v[kSmMaxCluster];
+    const int M4 = (p.M + 3) >> 2;          // token quads (rows >= M hold zeros)
+    const int nz = F * M4;                  // Z items: (feature, token quad)
+    // Issue the peers' loads of this thread's first Z item now, so that their
+    // latency overlaps the T sum below; they are summed after it.
+    float4 zv[kSmMaxCluster];
+    if (et < nz) {
+      const int fl = et / M4, m0 = (et - fl * M4) * 4;
+      const uint32_t a = dp_addr + static_cast<uint32_t>(((f0 + fl) * C::kLd + m0) * 4);
 #pragma unroll
       for (int qq = 0; qq < kSmMaxCluster; ++qq)
-        v[qq] = qq < p.splits ? ld_dsmem_f32(mapa_shared(tp_addr + off, qq)) : 0.0f;
-      float t = 0.0f;
+        if (qq < p.splits) zv[qq] = ld_dsmem_f32x4(mapa_shared(a, static_cast<uint32_t>(qq)));
+    }
+    // T[m][c] = sum over the cluster's ranks (in order) of T^T[c][m], 4 tokens at a time
+    for (int i = et; i < p.r * M4; i += 128) {
+      const int c = i / M4, m0 = (i - c * M4) * 4;
+      const float4 t = cluster_sum4(tp_addr + static_cast<uint32_t>((c * C::kLd + m0) * 4), p.splits);
+      reinterpret_cast<float4*>(Tf)[(c * kNT + m0) / 4] = t;
+      if (slice == 0 && rank == 0 && p.T_save != nullptr) {
+        const float tv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-      for (int qq = 0; qq < kSmMaxCluster; ++qq) t += v[qq];
-      Tf[m * 64 + c] = t;
-      if (slice == 0 && rank == 0 && p.T_save != nullptr) p.T_save[static_cast<size_t>(m) * p.r + c] = t;
+        for (int j = 0; j < 4; ++j)
+          if (m0 + j < p.M) p.T_save[static_cast<size_t>(m0 + j) * p.r + c] = tv[j];
+      }
     }
     bar_sync_named<1, 128>();
-    // this CTA's features [f0, f0 + F) of the slice, every token
-    for (int i = et; i < F * p.M; i += 128) {
-      const int m = i / F, fl = i - m * F;          // consecutive threads: consecutive features
+    if (et == 0) sm_trace(p, kTrTSummed);
+    // this CTA's features [f0, f0 + F) of the slice, 4 tokens per item
+    for (int i = et; i < nz; i += 128) {
+      const int fl = i / M4, m0 = (i - fl * M4) * 4;   // consecutive threads: consecutive quads of a row
       const int n = slice * 128 + f0 + fl;
-      const uint32_t off = static_cast<uint32_t>(((f0 + fl) * C::kLd + m) * 4);
-      float v[kSmMaxCluster];
+      float4 zs;
+      if (i == et) {
+        zs = zv[0];
 #pragma unroll
-      for (int qq = 0; qq < kSmMaxCluster; ++qq)
-        v[qq] = qq < p.splits ? ld_dsmem_f32(mapa_shared(dp_addr + off, qq)) : 0.0f;
-      float z = 0.0f;
-#pragma unroll
-      for (int qq = 0; qq < kSmMaxCluster; ++qq) z += v[qq];
-      float lora = 0.0f;
-      for (int c = 0; c < p.r; ++c) lora = fmaf(Bs[fl * (p.r + 1) + c], Tf[m * 64 + c], lora);
-      z = fmaf(p.s, lora, z);
+        for (int qq = 1; qq < kSmMaxCluster; ++qq)
+          if (qq < p.splits) { zs.x += zv[qq].x; zs.y += zv[qq].y; zs.z += zv[qq].z; zs.w += zv[qq].w; }
+      } else {
+        zs = cluster_sum4(dp_addr + static_cast<uint32_t>(((f0 + fl) * C::kLd + m0) * 4), p.splits);
+      }
+      float z[4] = {zs.x, zs.y, zs.z, zs.w};
+      float lora[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const float* brow = Bs + fl * (p.r + 1);
+      const float4* tcol = reinterpret_cast<const float4*>(Tf) + m0 / 4;
+      for (int c = 0; c < p.r; ++c) {
+        const float b = brow[c];
+        const float4 t = tcol[c * (kNT / 4)];
+        lora[0] = fmaf(b, t.x, lora[0]);
+        lora[1] = fmaf(b, t.y, lora[1]);
+        lora[2] = fmaf(b, t.z, lora[2]);
+        lora[3] = fmaf(b, t.w, lora[3]);
+      }
       if (n < p.d_out) {
-        if (p.act == LORA_ACT_SILU) {
-          if (p.Z_save != nullptr) p.Z_save[static_cast<size_t>(m) * p.d_out + n] = z;
-          z = z / (1.0f + expf(-z));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = m0 + j;
+          if (m >= p.M) break;
+          float v = fmaf(p.s, lora[j], z[j]);
+          if (p.act == LORA_ACT_SILU) {
+            if (p.Z_save != nullptr) p.Z_save[static_cast<size_t>(m) * p.d_out + n] = v;
+            v = v / (1.0f + expf(-v));
+          }
+          p.Y[static_cast<size_t>(m) * p.d_out + n] = __float2bfloat16_rn(v);
         }
-        p.Y[static_cast<size_t>(m) * p.d_out + n] = __float2bfloat16_rn(z);
       }
     }
     if (et == 0) sm_trace(p, kTrCombined);

@@ -22,6 +22,12 @@ CASES = [
     (256, 512, 520, 64, 16.0, "swiglu"),
     (1, 256, 256, 8, 16.0, "identity"),         # single token
     (17, 264, 1032, 24, 16.0, "identity"),      # r not a power of two
+    # ranks above 64: two 64-wide LoRA K-blocks per projection
+    (256, 512, 520, 128, 16.0, "identity"),
+    (300, 640, 264, 72, 16.0, "identity"),
+    (200, 384, 264, 96, 16.0, "silu"),
+    (136, 256, 392, 128, 16.0, "swiglu"),
+    (16, 512, 264, 128, 16.0, "identity"),      # few tokens, rank 128: the tiled path
     # few tokens: the cluster split-K forward (W streamed once)
     (5, 256, 264, 8, 16.0, "identity"),
     (33, 512, 1032, 16, 16.0, "silu"),
@@ -75,3 +81,27 @@ def test_device_status_clean_after_calls():
     L.backward(t["dY"], t["X"], t["W"], t["A"], t["B"], 2.0, "identity", T_save=T, workspace=ws)
     torch.cuda.synchronize()
     assert ws.status() == 0
+
+
+def test_empty_batch():
+    """M = 0: the forward is a no-op that accepts NULL token tensors; the
+    backward's adapter gradients are sums over no tokens, so exactly zero."""
+    import lora_linear_fine_b200 as L
+    import torch
+    d_in, d_out, r = 256, 264, 16
+    inp = seeded_inputs.make_inputs(8, d_in, d_out, r, "silu", seed=5)
+    t = {k: G.dev(v) for k, v in inp.items()}
+    for act in ("identity", "silu"):
+        desc = L.make_desc(0, d_in, d_out, r, 1.0, act)
+        ws = L.Workspace(L.lora_linear_workspace_size(desc, 1))
+        sh = torch.cuda.current_stream().cuda_stream
+        p = lambda x: x.data_ptr()
+        assert L.lora_linear_fwd(desc, None, p(t["W"]), p(t["A"]), p(t["B"]), None, None, None, None, None, None,
+                                 ws.buf.data_ptr(), ws.nbytes, sh) == 0
+        dA = torch.full((r, d_in), float("nan"), device="cuda")
+        dB = torch.full((d_out, r), float("nan"), device="cuda")
+        assert L.lora_linear_bwd(desc, None, None, p(t["W"]), p(t["A"]), p(t["B"]), None, None, None, None, None,
+                                 None, p(dA), p(dB), None, None, ws.buf.data_ptr(), ws.nbytes, sh) == 0
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
+        assert ws.status() == 0
