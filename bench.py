@@ -215,14 +215,14 @@ def job_throughput(units_per_step, steps, world, max_ms):
     return units_per_step * steps * world / (max_ms * 1e-3)
 
 
-def committed_traffic(workload):
-    """DRAM bytes per launch of the forward GEMM from a committed ncu summary,
-    valid only while the kernel source is unchanged (else None)."""
+def committed_traffic(workload, record="gemm_traffic.json", source="lora_mma.cuh"):
+    """DRAM bytes per launch of a kernel from a committed ncu summary, valid
+    only while the kernel source is unchanged (else None)."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "gemm_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", record)) as f:
             rec = json.load(f)
-        src = open(os.path.join(ROOT, "lora_linear_fine_b200", "csrc", "lora_mma.cuh"), "rb").read()
+        src = open(os.path.join(ROOT, "lora_linear_fine_b200", "csrc", source), "rb").read()
         if rec.get("kernel_sha256") != hashlib.sha256(src).hexdigest():
             return None
         return rec.get("per_launch_bytes", {}).get(workload)
@@ -262,7 +262,9 @@ def run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist):
                        "l2": "flushed before each timed step (512 MiB write)"},
             "roofline": {"kernel": "small_m_kernel" if M <= 64 else "lora_gemm_kernel (forward)", "bound": "hbm",
                          "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                         "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "traffic": committed_traffic(args.config, "small_m_traffic.json", "lora_small_m.cuh")
+                         if M <= 64 else None,
                          "bytes_per_launch": byts},
             "gpu_launches": int(launches)}
     if rank == 0:
