@@ -249,7 +249,10 @@ def run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist):
     ms = [a.elapsed_time(b) for a, b in ev]
     med = statistics.median(ms)
     F = fwd_flops(M, d_in, d_out, r)
-    byts = 2.0 * (M * d_in + d_out * d_in + r * d_in + d_out * r + M * d_out) + 4.0 * M * r
+    w4 = cfg.get("weight") == "w4"
+    # the base weight: bf16, or 4-bit codes plus one bf16 scale per row and 64 features
+    w_bytes = (d_out * d_in / 2.0 + 2.0 * d_out * (d_in // 64)) if w4 else 2.0 * d_out * d_in
+    byts = w_bytes + 2.0 * (M * d_in + r * d_in + d_out * r + M * d_out) + 4.0 * M * r
     peaks = read_peaks()
     gbs = byts / (med * 1e-3) / 1e9
     line = {"metric": "LoRA-linear forward (few tokens), HBM roofline", "value": round(F / (med * 1e-3) / 1e12, 3),
@@ -258,7 +261,7 @@ def run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": args.config, "M": M, "d_in": d_in, "d_out": d_out, "r": r,
-                       "alpha": cfg["alpha"], "act": cfg["act"],
+                       "alpha": cfg["alpha"], "act": cfg["act"], "weight": "w4g64" if w4 else "bf16",
                        "l2": "flushed before each timed step (512 MiB write)"},
             "roofline": {"kernel": "small_m_kernel" if M <= 64 else "lora_gemm_kernel (forward)", "bound": "hbm",
                          "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -318,13 +321,30 @@ def main():
     M, d_in, d_out, r, act = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]
     s = cfg["alpha"] / r if r else 0.0
     inp = seeded_inputs.make_inputs(M, d_in, d_out, r, act, seed=rank)
+    w4 = cfg.get("weight") == "w4"
+    if w4:   # the 4-bit base weight replaces W (forward-only few-token workload)
+        inp.pop("W")
+        Wq, Ws = seeded_inputs.draw_w4("W", d_out, d_in, rank)
     host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in inp.items()}
     t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+    if w4:
+        t["Wq"] = torch.from_numpy(Wq).cuda()
+        t["Ws"] = torch.from_numpy(Ws.view(np.int16)).view(torch.bfloat16).cuda()
+    p_drop = cfg.get("dropout")
+    if p_drop is not None:   # dropout on the adapter input: one mask per projection, an input like X
+        for name in ("mask", "mask_up") if act == "swiglu" else ("mask",):
+            host[name] = torch.from_numpy(seeded_inputs.draw_mask(name, M, d_in, p_drop, rank)).pin_memory()
+            t[name] = host[name].to("cuda", non_blocking=True)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
     desc = L.make_desc(M, d_in, d_out, r, s, act)
     np_ = 2 if act == "swiglu" else 1
-    ws = L.Workspace(max(L.lora_linear_workspace_size(desc, 0), L.lora_linear_workspace_size(desc, 1)))
+    if w4:
+        ws = L.Workspace(L.lora_linear_workspace_size_w4(desc, 0))
+    elif p_drop is not None:
+        ws = L.Workspace(L.lora_linear_workspace_size_dropout(desc, 1))
+    else:
+        ws = L.Workspace(max(L.lora_linear_workspace_size(desc, 0), L.lora_linear_workspace_size(desc, 1)))
     Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
     T = torch.empty((np_, M, r), dtype=torch.float32, device="cuda")
     Z = torch.empty((np_, M, d_out), dtype=torch.float32, device="cuda") if act != "identity" else None
@@ -334,12 +354,28 @@ def main():
     p = lambda x: None if x is None else x.data_ptr()  # noqa: E731
 
     def fwd():
-        st = L.lora_linear_fwd(desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
-                               p(t.get("A_up")), p(t.get("B_up")), p(Y), p(T), p(Z), ws.buf.data_ptr(),
-                               ws.nbytes, sh)
+        if w4:
+            st = L.lora_linear_fwd_w4(desc, p(t["X"]), p(t["Wq"]), p(t["Ws"]), p(t["A"]), p(t["B"]), None, None,
+                                      None, None, p(Y), p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
+        elif p_drop is not None:
+            st = L.lora_linear_fwd_dropout(desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
+                                           p(t.get("A_up")), p(t.get("B_up")), p(t["mask"]), p(t.get("mask_up")),
+                                           p_drop, p(Y), p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
+        else:
+            st = L.lora_linear_fwd(desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
+                                   p(t.get("A_up")), p(t.get("B_up")), p(Y), p(T), p(Z), ws.buf.data_ptr(),
+                                   ws.nbytes, sh)
         assert st == 0, L.status_string(st)
 
     def bwd():
+        if p_drop is not None:
+            st = L.lora_linear_bwd_dropout(desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]),
+                                           p(t.get("W_up")), p(t.get("A_up")), p(t.get("B_up")), p(t["mask"]),
+                                           p(t.get("mask_up")), p_drop, p(T), p(Z), p(dX), p(dA[0]), p(dB[0]),
+                                           p(dA[1]) if np_ == 2 else None, p(dB[1]) if np_ == 2 else None,
+                                           ws.buf.data_ptr(), ws.nbytes, sh)
+            assert st == 0, L.status_string(st)
+            return
         st = L.lora_linear_bwd(desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
                                p(t.get("A_up")), p(t.get("B_up")), p(T), p(Z), p(dX), p(dA[0]), p(dB[0]),
                                p(dA[1]) if np_ == 2 else None, p(dB[1]) if np_ == 2 else None,
@@ -448,7 +484,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.config, "M": M, "d_in": d_in, "d_out": d_out, "r": r,
                        "alpha": cfg["alpha"], "act": act, "parallelism": f"replicas x{world}",
-                       "l2": "flushed before each timed step (512 MiB write)"},
+                       "l2": "flushed before each timed step (512 MiB write)",
+                       **({"dropout": p_drop} if p_drop is not None else {})},
             "roofline": roof, "gpu_launches": int(launches),
             "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},

@@ -214,6 +214,95 @@ lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* desc,
                                       const void* W_up, const void* A_up, const void* B_up,
                                       void* Y, float* T_save, float* Z_save, void* stream);
 
+/* ------------------------------------------------------------------------
+ * 4-bit frozen base weight ("w4g64").  The pages name QLoRA fine-tuning, whose
+ * frozen weight is stored at 4 bits, among the settings the fused kernels
+ * serve ("Liger-Kernel内核级优化：GPU利用率飙升至90%以上", opening section;
+ * "Swift-All一文详解：如何用Liger-Kernel提升训练效率", section 2.3, table), but
+ * they give no storage format.  This library's format:
+ *   Wq [d_out x d_in/2] uint8: the codes q[n][k] in 0..15, two per byte, byte
+ *      j of row n holding q[n][2j] in its low nibble and q[n][2j+1] in its
+ *      high nibble;
+ *   Ws [d_in/64 x d_out] bf16 (group-major): Ws[g][n] scales
+ *      W[n][64g .. 64g+63];
+ *   W[n][k] = bf16(Ws[k/64][n] * (q[n][k] - 8)), rounded to nearest even (the
+ *      product is exact in fp32).
+ * The layer is the bf16 layer above on that W.  d_in must be a multiple of 64
+ * (LORA_ERR_ALIGNMENT otherwise); Wq, Ws (and Wq_up, Ws_up for SwiGLU) are
+ * required, device-resident, 16-byte aligned and only read.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes for lora_linear_fwd_w4 (for_backward = 0) or
+ * lora_linear_bwd_w4 (1): the bf16 workspace plus, except for the few-token
+ * forward, room to expand the weight(s) to bf16 (d_out * d_in * 2 bytes per
+ * projection).  0 for an invalid desc or d_in % 64 != 0. */
+size_t lora_linear_workspace_size_w4(const lora_linear_desc* desc, int for_backward);
+
+/* Expand a 4-bit weight to bf16: W [d_out x d_in] bf16 (device, written).
+ * Asynchronous on `stream`.  d_in % 64 == 0 and d_out % 8 == 0, pointers
+ * 16-byte aligned (LORA_ERR_ALIGNMENT), d_out, d_in > 0 (LORA_ERR_INVALID_ARG). */
+lora_status_t lora_linear_dequant_w4(const void* Wq, const void* Ws, int64_t d_out, int64_t d_in, void* W,
+                                     void* stream);
+
+/* Forward with 4-bit base weight(s).  Arguments as lora_linear_fwd, with
+ * (Wq, Ws) in place of W and (Wq_up, Ws_up) in place of W_up.  With 1..64
+ * tokens, identity or SiLU and 0 < r <= 64 the codes are streamed once and
+ * expanded inside the few-token kernel (one launch); otherwise the weight(s)
+ * are expanded into the workspace and the bf16 path runs on them.
+ * workspace: >= lora_linear_workspace_size_w4(desc, 0) bytes. */
+lora_status_t lora_linear_fwd_w4(const lora_linear_desc* desc, const void* X, const void* Wq, const void* Ws,
+                                 const void* A, const void* B, const void* Wq_up, const void* Ws_up,
+                                 const void* A_up, const void* B_up, void* Y, float* T_save, float* Z_save,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward with 4-bit base weight(s) (frozen: no gradient for them).
+ * Arguments as lora_linear_bwd with (Wq, Ws), (Wq_up, Ws_up) in place of W,
+ * W_up; the weight(s) are expanded into the workspace, then the bf16 backward
+ * runs.  workspace: >= lora_linear_workspace_size_w4(desc, 1) bytes. */
+lora_status_t lora_linear_bwd_w4(const lora_linear_desc* desc, const void* dY, const void* X, const void* Wq,
+                                 const void* Ws, const void* A, const void* B, const void* Wq_up, const void* Ws_up,
+                                 const void* A_up, const void* B_up, const float* T_save, const float* Z_save,
+                                 void* dX, float* dA, float* dB, float* dA_up, float* dB_up, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dropout on the adapter branch's input.  The pages' LoRA configurations set
+ * a LoRA dropout (lora_dropout = 0.05 in "Swift-All一文详解：如何用Liger-Kernel
+ * 提升训练效率", section 3's training configuration; 0.1 in the usage example
+ * of "企业官网建设流程全解析") without saying where it applies; the reading
+ * taken is the usual one: only the adapter sees the dropped input,
+ *   X_d = X * mask / (1 - p_drop),   T = X_d A^T,   Z = X W^T + s T B^T,
+ * and the backward is its chain rule (dX = dZ W + mask * (s U A) / (1 - p),
+ * dA = s U^T X_d, dB = s dZ^T T).  The random draws are an input:
+ *   mask, mask_up: device, [M x d_in/8] bytes; bit j of byte b (least
+ *     significant first) keeps element 8b + j of that token's row of X.
+ *     mask_up (SwiGLU's up projection; its own draw) is required for SwiGLU,
+ *     NULL otherwise.  Both may be NULL when M == 0.  Only read.
+ *   p_drop: the drop probability, 0 <= p_drop < 1 (else LORA_ERR_INVALID_ARG).
+ * T_save holds (X * mask) A^T, without the 1/(1 - p_drop) factor; pass it
+ * back to lora_linear_bwd_dropout unchanged.  With r == 0 these calls are the
+ * plain ones.  The few-token kernel is not used (dropout is a training-time
+ * transform); the masked input is written to the workspace, and the LoRA term
+ * of dX is added after the dX GEMM (dx_dropout_kernel).
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes for lora_linear_fwd_dropout (0) / lora_linear_bwd_dropout
+ * (1): the layer's workspace plus the masked input(s), M * d_in * 2 bytes per
+ * projection.  0 for an invalid desc. */
+size_t lora_linear_workspace_size_dropout(const lora_linear_desc* desc, int for_backward);
+
+lora_status_t lora_linear_fwd_dropout(const lora_linear_desc* desc, const void* X, const void* W, const void* A,
+                                      const void* B, const void* W_up, const void* A_up, const void* B_up,
+                                      const void* mask, const void* mask_up, float p_drop, void* Y, float* T_save,
+                                      float* Z_save, void* workspace, size_t workspace_bytes, void* stream);
+
+lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* desc, const void* dY, const void* X, const void* W,
+                                      const void* A, const void* B, const void* W_up, const void* A_up,
+                                      const void* B_up, const void* mask, const void* mask_up, float p_drop,
+                                      const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
+                                      float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

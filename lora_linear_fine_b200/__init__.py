@@ -28,7 +28,9 @@ STATUS_NAMES = {
 EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_linear_device_status",
             "lora_linear_fwd", "lora_linear_bwd", "lora_status_string", "lora_linear_abi_version",
             "lora_linear_launch_count", "lora_linear_fwd_noalloc", "lora_linear_timing_enable",
-            "lora_linear_timing_read", "lora_linear_selftest_wait_timeout")
+            "lora_linear_timing_read", "lora_linear_selftest_wait_timeout",
+            "lora_linear_workspace_size_w4", "lora_linear_dequant_w4", "lora_linear_fwd_w4", "lora_linear_bwd_w4",
+            "lora_linear_workspace_size_dropout", "lora_linear_fwd_dropout", "lora_linear_bwd_dropout")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -73,6 +75,21 @@ def _load():
     lib.lora_linear_timing_read.restype = i32
     lib.lora_linear_selftest_wait_timeout.argtypes = [vp, sz, i32, vp]
     lib.lora_linear_selftest_wait_timeout.restype = i32
+    lib.lora_linear_workspace_size_w4.argtypes = [dp, i32]
+    lib.lora_linear_workspace_size_w4.restype = sz
+    lib.lora_linear_dequant_w4.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int64, vp, vp]
+    lib.lora_linear_dequant_w4.restype = i32
+    lib.lora_linear_fwd_w4.argtypes = [dp] + [vp] * 12 + [vp, sz, vp]
+    lib.lora_linear_fwd_w4.restype = i32
+    lib.lora_linear_bwd_w4.argtypes = [dp] + [vp] * 17 + [vp, sz, vp]
+    lib.lora_linear_bwd_w4.restype = i32
+    f32 = ctypes.c_float
+    lib.lora_linear_workspace_size_dropout.argtypes = [dp, i32]
+    lib.lora_linear_workspace_size_dropout.restype = sz
+    lib.lora_linear_fwd_dropout.argtypes = [dp] + [vp] * 9 + [f32] + [vp] * 3 + [vp, sz, vp]
+    lib.lora_linear_fwd_dropout.restype = i32
+    lib.lora_linear_bwd_dropout.argtypes = [dp] + [vp] * 10 + [f32] + [vp] * 7 + [vp, sz, vp]
+    lib.lora_linear_bwd_dropout.restype = i32
     return lib
 
 
@@ -138,6 +155,28 @@ def lora_linear_fwd_noalloc(desc, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_sav
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+# 4-bit frozen base weight ("w4g64": codes two per byte, low nibble first; one
+# bf16 scale per row and 64 input features, group-major; W = bf16(scale * (code - 8)))
+def lora_linear_workspace_size_w4(desc: LoraLinearDesc, for_backward: int) -> int:
+    return int(_lib.lora_linear_workspace_size_w4(ctypes.byref(desc), int(for_backward)))
+
+
+def lora_linear_dequant_w4(Wq, Ws, d_out, d_in, W, stream) -> int:
+    return int(_lib.lora_linear_dequant_w4(Wq, Ws, int(d_out), int(d_in), W, stream))
+
+
+def lora_linear_fwd_w4(desc, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, Y, T_save, Z_save, workspace,
+                       workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_fwd_w4(ctypes.byref(desc), X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, Y, T_save,
+                                       Z_save, workspace, workspace_bytes, stream))
+
+
+def lora_linear_bwd_w4(desc, dY, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up,
+                       dB_up, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_bwd_w4(ctypes.byref(desc), dY, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, T_save,
+                                       Z_save, dX, dA, dB, dA_up, dB_up, workspace, workspace_bytes, stream))
 
 
 def lora_linear_timing_enable(enable: int) -> int:
@@ -278,3 +317,21 @@ try:  # torch is optional for the 1:1 C wrappers
     LoRALinearFunction = _make_autograd()
 except Exception:  # pragma: no cover
     LoRALinearFunction = None
+
+
+# dropout on the adapter branch's input (mask: [M x d_in/8] bytes, bit j of byte b keeps element 8b + j)
+def lora_linear_workspace_size_dropout(desc: LoraLinearDesc, for_backward: int) -> int:
+    return int(_lib.lora_linear_workspace_size_dropout(ctypes.byref(desc), int(for_backward)))
+
+
+def lora_linear_fwd_dropout(desc, X, W, A, B, W_up, A_up, B_up, mask, mask_up, p_drop, Y, T_save, Z_save,
+                            workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_fwd_dropout(ctypes.byref(desc), X, W, A, B, W_up, A_up, B_up, mask, mask_up,
+                                            float(p_drop), Y, T_save, Z_save, workspace, workspace_bytes, stream))
+
+
+def lora_linear_bwd_dropout(desc, dY, X, W, A, B, W_up, A_up, B_up, mask, mask_up, p_drop, T_save, Z_save, dX, dA,
+                            dB, dA_up, dB_up, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_bwd_dropout(ctypes.byref(desc), dY, X, W, A, B, W_up, A_up, B_up, mask, mask_up,
+                                            float(p_drop), T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace,
+                                            workspace_bytes, stream))

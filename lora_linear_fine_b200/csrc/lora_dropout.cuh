@@ -1,0 +1,136 @@
+// lora_dropout.cuh — dropout on the input of the LoRA branch.
+//
+// With a {0,1} mask m (one bit per element of X, given by the caller) and
+// drop probability p, the adapter sees X_d = X * m / (1 - p) while the frozen
+// path sees X.  Writing X_m = X * m (exact in bf16: each element is kept or
+// zeroed) and s' = s / (1 - p), the layer is the plain one with the adapter
+// input X_m and the scale s':
+//   Z  = X W^T + s' (X_m A^T) B^T
+//   dA = s' U^T X_m,   dB = s' dZ^T (X_m A^T),   U = dZ B
+//   dX = dZ W + m * (s' U A)
+// so the rank passes run unchanged on X_m, and only the LoRA term of dX needs
+// the mask: the dX GEMM then runs without its LoRA K-block and
+// dx_dropout_kernel adds m * (s' U A) afterwards.
+//
+// Mask layout: [M x d_in/8] bytes, bit j of byte b (least significant first)
+// keeps element 8 b + j.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+
+namespace lora {
+
+// X_m = X * m, bf16 [M x d_in].  One thread per 8 elements (16 bytes of X, one
+// mask byte), grid-stride, coalesced.
+__global__ void __launch_bounds__(256) mask_x_kernel(const __nv_bfloat16* __restrict__ X,
+                                                     const uint8_t* __restrict__ mask, long long n8,
+                                                     __nv_bfloat16* __restrict__ Xm) {
+  grid_dep_wait();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(X)[i];
+    const uint32_t b = mask[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
+      const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
+      o[e] = w[e] & (lo | hi);
+    }
+    reinterpret_cast<uint4*>(Xm)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+struct DxDropoutJob {
+  const uint8_t* mask;          // [M x d_in/8]
+  const __nv_bfloat16* ut_hi;   // (s' U)^T hi [r x ld]
+  const __nv_bfloat16* ut_lo;   // (s' U)^T lo [r x ld]
+  const __nv_bfloat16* A;       // [r x d_in]
+};
+
+constexpr int kDxRows = 16, kDxCols = 128, kDxMaxRank = 128;
+
+// dX += sum_j m_j * ((s' U_j) A_j) for one or two projections, in place on the
+// bf16 dX.  A block takes a 16-row x 128-column tile: it stages the rows'
+// s'U (hi + lo, fp32) and the tile's columns of A (bf16) in shared memory,
+// then each thread adds to 8 consecutive outputs of one row (16-byte dX and
+// one mask byte per thread; rows are 256 contiguous bytes per 16 threads).
+__global__ void __launch_bounds__(256) dx_dropout_kernel(__nv_bfloat16* __restrict__ dX, int M, int d_in, int r,
+                                                         int ld, DxDropoutJob j0, DxDropoutJob j1, int np) {
+  grid_dep_wait();
+  __shared__ float sU[kDxRows][kDxMaxRank + 1];
+  __shared__ __align__(16) __nv_bfloat16 sA[kDxMaxRank][kDxCols];
+  const int t = threadIdx.x;
+  const int row = t >> 4, cg = t & 15;        // this thread: one row, columns 8 cg .. 8 cg + 7 of the tile
+  const int tiles_m = (M + kDxRows - 1) / kDxRows, tiles_n = d_in / kDxCols + (d_in % kDxCols ? 1 : 0);
+  for (long long tile = blockIdx.x; tile < static_cast<long long>(tiles_m) * tiles_n; tile += gridDim.x) {
+    const int m0 = static_cast<int>(tile / tiles_n) * kDxRows;
+    const int k0 = static_cast<int>(tile % tiles_n) * kDxCols;
+    const int m = m0 + row, k = k0 + 8 * cg;
+    const bool live = m < M && k < d_in;
+    float acc[8];
+    uint4 cur = make_uint4(0, 0, 0, 0);
+    if (live) cur = *reinterpret_cast<const uint4*>(dX + static_cast<size_t>(m) * d_in + k);
+    {
+      const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] = __uint_as_float(w[e] << 16);
+        acc[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+    for (int jj = 0; jj < np; ++jj) {
+      const DxDropoutJob& J = jj == 0 ? j0 : j1;
+      __syncthreads();   // the previous use of sU / sA is over
+      for (int i = t; i < kDxRows * r; i += 256) {
+        const int c = i / kDxRows, rr = i - c * kDxRows;
+        const int mm = m0 + rr;
+        float u = 0.0f;
+        if (mm < M) {
+          const size_t at = static_cast<size_t>(c) * ld + mm;
+          u = __bfloat162float(J.ut_hi[at]) + __bfloat162float(J.ut_lo[at]);
+        }
+        sU[rr][c] = u;
+      }
+      for (int i = t; i < r * (kDxCols / 8); i += 256) {
+        const int c = i / (kDxCols / 8), q = i - c * (kDxCols / 8);
+        const int kk = k0 + 8 * q;
+        uint4 a = make_uint4(0, 0, 0, 0);
+        if (kk < d_in) a = *reinterpret_cast<const uint4*>(J.A + static_cast<size_t>(c) * d_in + kk);
+        *reinterpret_cast<uint4*>(&sA[c][8 * q]) = a;
+      }
+      __syncthreads();
+      if (live) {
+        float add[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < r; ++c) {
+          const float u = sU[row][c];
+          const uint4 a = *reinterpret_cast<const uint4*>(&sA[c][8 * cg]);
+          const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            add[2 * e] = fmaf(u, __uint_as_float(w[e] << 16), add[2 * e]);
+            add[2 * e + 1] = fmaf(u, __uint_as_float(w[e] & 0xFFFF0000u), add[2 * e + 1]);
+          }
+        }
+        const uint32_t b = J.mask[static_cast<size_t>(m) * (d_in / 8) + k / 8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if ((b >> e) & 1u) acc[e] += add[e];
+      }
+    }
+    if (live) {
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(dX + static_cast<size_t>(m) * d_in + k) = o;
+    }
+  }
+}
+
+}  // namespace lora

@@ -17,6 +17,8 @@
 #include "lora_rank.cuh"
 #include "lora_rank2d.cuh"
 #include "lora_small_m.cuh"
+#include "lora_w4.cuh"
+#include "lora_dropout.cuh"
 
 namespace {
 
@@ -103,6 +105,22 @@ bool make_tm(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, u
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a plain row-major array without swizzle (the 4-bit weight's
+// codes and scales): inner x outer elements of elem_bytes, rows row_bytes apart.
+bool make_tm_plain(CUtensorMap* tm, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = g_encode(tm, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) LORA_LOG("cuTensorMapEncodeTiled (plain) failed (%d): inner=%llu outer=%llu box=%ux%u", (int)r,
+                                  (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // argument checks and sizes
 // ---------------------------------------------------------------------------
@@ -169,7 +187,7 @@ int rank_splits(int64_t tiles, int64_t nkb) {
   return static_cast<int>(s);
 }
 
-Plan make_plan(const lora_linear_desc* d, bool backward) {
+Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = true) {
   Plan P;
   P.np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
   P.RP = rank_pad(d->r);
@@ -186,7 +204,7 @@ Plan make_plan(const lora_linear_desc* d, bool backward) {
   auto partials = [&](int splits, int64_t tiles) -> size_t {
     return splits > 1 ? take(static_cast<size_t>(splits) * tiles * 128 * P.RP * 4) : 0;
   };
-  if (!backward && small_m_applies(d)) {
+  if (!backward && allow_small_m && small_m_applies(d)) {
     // The few-token forward keeps everything on chip: no workspace regions.
     P.small_m = true;
     P.sm_nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
@@ -643,6 +661,158 @@ lora_status_t common_checks(const lora_linear_desc* d, void* ws, size_t ws_bytes
   return LORA_OK;
 }
 
+// Few tokens: bound by reading W once; one cluster per 128-row slice of W.
+// W is bf16, or (Wq != null) the 4-bit codes Wq with scales Ws.
+lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, const void* W, const void* Wq,
+                              const void* Ws, const void* A, const void* B, void* Y, float* T_save, float* Z_save,
+                              uint32_t* status, cudaStream_t st) {
+  const int64_t M = d->M, r = d->r;
+  SmallMParams q;
+  std::memset(&q, 0, sizeof(q));
+  const bool w4 = Wq != nullptr;
+  bool ok = w4 ? make_tm_plain(&q.tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, d->d_in / 2, d->d_out, d->d_in / 2, 32,
+                               128) &&
+                     make_tm_plain(&q.tm_ws, Ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->d_out, d->d_in / kW4Group,
+                                   d->d_out * 2, 128, 1)
+               : make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128);
+  if (!ok ||
+      !make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, static_cast<uint32_t>(align_up(static_cast<size_t>(r), 16))) ||
+      !make_tm(&q.tm_x, X, d->d_in, M, d->d_in, 64, static_cast<uint32_t>(nt)))
+    return LORA_ERR_CUDA;
+  q.B = static_cast<const __nv_bfloat16*>(B);
+  q.Y = static_cast<__nv_bfloat16*>(Y);
+  q.T_save = T_save;
+  q.Z_save = d->act == LORA_ACT_SILU ? Z_save : nullptr;
+  q.status = status;
+  q.M = static_cast<int>(M);
+  q.d_in = static_cast<int>(d->d_in);
+  q.d_out = static_cast<int>(d->d_out);
+  q.r = static_cast<int>(r);
+  q.s = d->s;
+  q.act = d->act;
+  q.a_rows = static_cast<int>(align_up(static_cast<size_t>(r), 16));
+  const int slices = static_cast<int>(ceil_div(d->d_out, 128));
+  q.splits = small_m_splits(nt, w4, d->d_in, d->d_out);
+  q.kb_per = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), q.splits));
+  const int grid = slices * q.splits;
+  LORA_LOG("small_m M=%d nt=%d w4=%d slices=%d splits=%d kb_per=%d grid=%d", (int)M, nt, (int)w4, slices,
+           q.splits, q.kb_per, grid);
+  // LORA_LINEAR_DEBUG=2: per-CTA phase stamps, printed after the launch
+  // (synchronises the stream; for debugging only).
+  static unsigned long long* trace = nullptr;
+  if (debug_level() >= 2 && trace == nullptr &&
+      cudaMalloc(&trace, sizeof(unsigned long long) * 1024 * kSmTracePoints) != cudaSuccess)
+    trace = nullptr;
+  if (debug_level() >= 2 && trace != nullptr && grid <= 1024) {
+    q.trace = trace;
+    cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTracePoints, st);
+  }
+  const cudaError_t e = launch_small_m(q, nt, w4, slices, pdl_enabled(), st);
+  if (e != cudaSuccess) {
+    LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return LORA_ERR_CUDA;
+  }
+  const lora_status_t ls = check_launch("small_m_kernel");
+  if (q.trace != nullptr && cudaStreamSynchronize(st) == cudaSuccess) {
+    std::vector<unsigned long long> h(static_cast<size_t>(grid) * kSmTracePoints);
+    cudaMemcpy(h.data(), trace, h.size() * sizeof(unsigned long long), cudaMemcpyDeviceToHost);
+    unsigned long long t0 = ~0ull;
+    for (int b = 0; b < grid; ++b) t0 = h[b * kSmTracePoints] && h[b * kSmTracePoints] < t0 ? h[b * kSmTracePoints] : t0;
+    static const char* names[kSmTracePoints] = {"entry", "first_issue", "first_data", "last_mma", "published",
+                                                "synced", "t_summed", "combined", "exit"};
+    for (int k = 0; k < kSmTracePoints; ++k) {
+      double mn = 1e30, mx = 0, sum = 0;
+      int n = 0;
+      for (int b = 0; b < grid; ++b) {
+        const unsigned long long v = h[b * kSmTracePoints + k];
+        if (v == 0) continue;
+        const double us = (v - t0) * 1e-3;
+        mn = us < mn ? us : mn;
+        mx = us > mx ? us : mx;
+        sum += us;
+        ++n;
+      }
+      if (n) LORA_LOG("small_m trace %-12s n=%3d min %7.2f mean %7.2f max %7.2f us", names[k], n, mn, sum / n, mx);
+    }
+  }
+  return ls;
+}
+
+// 4-bit frozen base weight: shared checks and the expansion to bf16.
+// Checks shared by the 4-bit entry points: the codes and scales of W (and of
+// W_up for SwiGLU) are required and 16-byte aligned; d_in is a multiple of 64.
+lora_status_t check_w4(const lora_linear_desc* d, const void* Wq, const void* Ws, const void* Wq_up,
+                       const void* Ws_up) {
+  LORA_TRY(check_desc(d));
+  if (Wq == nullptr || Ws == nullptr) return LORA_ERR_INVALID_ARG;
+  if (d->act == LORA_ACT_SWIGLU && (Wq_up == nullptr || Ws_up == nullptr)) return LORA_ERR_INVALID_ARG;
+  if (d->d_in % kW4Group != 0) return LORA_ERR_ALIGNMENT;
+  const void* ptrs[] = {Wq, Ws, Wq_up, Ws_up};
+  for (const void* q : ptrs)
+    if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
+  return LORA_OK;
+}
+
+// Bytes of the bf16 weight(s) the tiled path expands into (after the regular
+// workspace), 0 for the few-token forward, which reads the codes directly.
+size_t w4_expand_bytes(const lora_linear_desc* d, bool backward) {
+  if (!backward && small_m_applies(d)) return 0;
+  const size_t np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
+  return np * static_cast<size_t>(d->d_out) * static_cast<size_t>(d->d_in) * 2;
+}
+
+lora_status_t dequant_w4(const void* Wq, const void* Ws, int64_t d_out, int64_t d_in, void* W, cudaStream_t st) {
+  DevInfo dev;
+  LORA_TRY(device_info(&dev));
+  const long long n = d_out * (d_in / 16);
+  launch_k(dequant_w4_kernel, dim3(grid_for(n, 256, dev.sms)), dim3(256), 0, st, false,
+           static_cast<const uint8_t*>(Wq), static_cast<const __nv_bfloat16*>(Ws), static_cast<long long>(d_out),
+           static_cast<int>(d_in), static_cast<__nv_bfloat16*>(W));
+  return check_launch("dequant_w4_kernel");
+}
+
+// Dropout on the adapter branch's input: checks, workspace, the masked inputs.
+lora_status_t check_dropout(const lora_linear_desc* d, const void* X, const void* mask, const void* mask_up,
+                            float p_drop) {
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return LORA_ERR_INVALID_ARG;
+  if (d->M > 0 && (X == nullptr || mask == nullptr || (d->act == LORA_ACT_SWIGLU && mask_up == nullptr)))
+    return LORA_ERR_INVALID_ARG;
+  if (X != nullptr && !aligned16(X)) return LORA_ERR_ALIGNMENT;
+  return LORA_OK;
+}
+
+// The workspace of the layer without the few-token path (dropout always runs tiled).
+size_t dropout_base_bytes(const lora_linear_desc* d, bool backward) {
+  const size_t fwd = make_plan(d, false, false).total;
+  if (!backward) return fwd;
+  const size_t bwd = make_plan(d, true).total;
+  return bwd > fwd ? bwd : fwd;
+}
+
+// The masked copies X * m_j of the adapter inputs, one per projection.
+size_t dropout_xm_bytes(const lora_linear_desc* d) {
+  const size_t np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
+  return np * align_up(static_cast<size_t>(d->M) * static_cast<size_t>(d->d_in) * 2, 256);
+}
+
+lora_status_t mask_inputs(const lora_linear_desc* d, const void* X, const void* mask, const void* mask_up,
+                          uint8_t* dst, const void* Xl[2], const DevInfo& dev, cudaStream_t st) {
+  const int np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
+  const long long n8 = d->M * d->d_in / 8;
+  const size_t stride = align_up(static_cast<size_t>(d->M) * static_cast<size_t>(d->d_in) * 2, 256);
+  for (int j = 0; j < 2; ++j) {
+    if (j >= np) { Xl[j] = Xl[0]; continue; }
+    uint8_t* xm = dst + j * stride;
+    launch_k(mask_x_kernel, dim3(grid_for(n8, 256, dev.sms)), dim3(256), 0, st, false,
+             static_cast<const __nv_bfloat16*>(X), static_cast<const uint8_t*>(j == 0 ? mask : mask_up), n8,
+             reinterpret_cast<__nv_bfloat16*>(xm));
+    LORA_TRY(check_launch("mask_x_kernel"));
+    Xl[j] = xm;
+  }
+  return LORA_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -741,9 +911,13 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
   return v == 0 ? LORA_OK : LORA_ERR_DEVICE_STATUS;
 }
 
-lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const void* W, const void* A, const void* B,
-                              const void* W_up, const void* A_up, const void* B_up, void* Y, float* T_save,
-                              float* Z_save, void* workspace, size_t workspace_bytes, void* stream) {
+// The forward.  Xl[j] is the input of projection j's adapter branch (X, or
+// the dropout-masked copy of X); allow_small_m = false keeps the tiled path
+// for few tokens.
+static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const void* W, const void* A,
+                              const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
+                              float* T_save, float* Z_save, void* workspace, size_t workspace_bytes, void* stream,
+                              const void* const Xl[2], bool allow_small_m) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
   // with M == 0 the per-token tensors are empty and may be NULL
@@ -753,7 +927,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   const void* ptrs[] = {X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
-  const Plan P = make_plan(d, false);
+  const Plan P = make_plan(d, false, allow_small_m);
   DevInfo dev;
   LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
   if (d->M == 0) return LORA_OK;
@@ -764,74 +938,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   (void)RP;
   const int64_t M = d->M, r = d->r;
 
-  if (P.small_m) {
-    // Few tokens: bound by reading W once; one cluster per 128-row slice of W.
-    const int nt = P.sm_nt;
-    SmallMParams q;
-    std::memset(&q, 0, sizeof(q));
-    if (!make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128) ||
-        !make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, static_cast<uint32_t>(align_up(static_cast<size_t>(r), 16))) ||
-        !make_tm(&q.tm_x, X, d->d_in, M, d->d_in, 64, static_cast<uint32_t>(nt)))
-      return LORA_ERR_CUDA;
-    q.B = static_cast<const __nv_bfloat16*>(B);
-    q.Y = static_cast<__nv_bfloat16*>(Y);
-    q.T_save = T_save;
-    q.Z_save = d->act == LORA_ACT_SILU ? Z_save : nullptr;
-    q.status = status;
-    q.M = static_cast<int>(M);
-    q.d_in = static_cast<int>(d->d_in);
-    q.d_out = static_cast<int>(d->d_out);
-    q.r = static_cast<int>(r);
-    q.s = d->s;
-    q.act = d->act;
-    q.a_rows = static_cast<int>(align_up(static_cast<size_t>(r), 16));
-    const int slices = static_cast<int>(ceil_div(d->d_out, 128));
-    q.splits = small_m_splits(nt, d->d_in, d->d_out);
-    q.kb_per = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), q.splits));
-    const int grid = slices * q.splits;
-    LORA_LOG("small_m M=%d nt=%d slices=%d splits=%d kb_per=%d grid=%d", (int)M, nt, slices, q.splits, q.kb_per,
-             grid);
-    // LORA_LINEAR_DEBUG=2: per-CTA phase stamps, printed after the launch
-    // (synchronises the stream; for debugging only).
-    static unsigned long long* trace = nullptr;
-    if (debug_level() >= 2 && trace == nullptr &&
-        cudaMalloc(&trace, sizeof(unsigned long long) * 1024 * kSmTracePoints) != cudaSuccess)
-      trace = nullptr;
-    if (debug_level() >= 2 && trace != nullptr && grid <= 1024) {
-      q.trace = trace;
-      cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTracePoints, st);
-    }
-    const cudaError_t e = launch_small_m(q, nt, slices, pdl_enabled(), st);
-    if (e != cudaSuccess) {
-      LORA_LOG("small_m launch: %s", cudaGetErrorString(e));
-      g_launches.fetch_add(1, std::memory_order_relaxed);
-      return LORA_ERR_CUDA;
-    }
-    const lora_status_t ls = check_launch("small_m_kernel");
-    if (q.trace != nullptr && cudaStreamSynchronize(st) == cudaSuccess) {
-      std::vector<unsigned long long> h(static_cast<size_t>(grid) * kSmTracePoints);
-      cudaMemcpy(h.data(), trace, h.size() * sizeof(unsigned long long), cudaMemcpyDeviceToHost);
-      unsigned long long t0 = ~0ull;
-      for (int b = 0; b < grid; ++b) t0 = h[b * kSmTracePoints] && h[b * kSmTracePoints] < t0 ? h[b * kSmTracePoints] : t0;
-      static const char* names[kSmTracePoints] = {"entry", "first_issue", "first_data", "last_mma", "published",
-                                                  "synced", "t_summed", "combined", "exit"};
-      for (int k = 0; k < kSmTracePoints; ++k) {
-        double mn = 1e30, mx = 0, sum = 0;
-        int n = 0;
-        for (int b = 0; b < grid; ++b) {
-          const unsigned long long v = h[b * kSmTracePoints + k];
-          if (v == 0) continue;
-          const double us = (v - t0) * 1e-3;
-          mn = us < mn ? us : mn;
-          mx = us > mx ? us : mx;
-          sum += us;
-          ++n;
-        }
-        if (n) LORA_LOG("small_m trace %-12s n=%3d min %7.2f mean %7.2f max %7.2f us", names[k], n, mn, sum / n, mx);
-      }
-    }
-    return ls;
-  }
+  if (P.small_m) return run_small_m_fwd(d, P.sm_nt, X, W, nullptr, nullptr, A, B, Y, T_save, Z_save, status, st);
 
   const void* Wp[2] = {W, W_up};
   const void* Ap[2] = {A, A_up};
@@ -844,7 +951,7 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
                      : reinterpret_cast<float*>(ws + P.t_ws) + static_cast<size_t>(j) * M * r;
       o.s16 = reinterpret_cast<__nv_bfloat16*>(ws + P.s16[j]);
       o.scale = d->s;
-      LORA_TRY(rank_T(d, P, X, Ap[j], o, ws, status, st));
+      LORA_TRY(rank_T(d, P, Xl[j], Ap[j], o, ws, status, st));
     }
   }
   // 2. Z = [X | sT] [W | B]^T, activation, bf16 Y
@@ -884,10 +991,21 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
   return rs;
 }
 
-lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const void* X, const void* W, const void* A,
+lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const void* W, const void* A, const void* B,
+                              const void* W_up, const void* A_up, const void* B_up, void* Y, float* T_save,
+                              float* Z_save, void* workspace, size_t workspace_bytes, void* stream) {
+  const void* Xl[2] = {X, X};
+  return fwd_core(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, workspace, workspace_bytes, stream, Xl, true);
+}
+
+// The backward.  Xl[j] is the input of projection j's adapter branch; with
+// dropout masks (masks[0] != null) the dX GEMM runs without its LoRA K-block
+// and dx_dropout_kernel adds the masked LoRA term afterwards.
+static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const void* X, const void* W, const void* A,
                               const void* B, const void* W_up, const void* A_up, const void* B_up,
                               const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
-                              float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream) {
+                              float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream,
+                              const void* const Xl[2], const uint8_t* const masks[2]) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
   // with M == 0 the per-token tensors are empty and may be NULL
@@ -997,7 +1115,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
         o.ld = M8;
         o.hilo_f16 = f16 ? 1 : 0;
         o.scale = d->s;
-        LORA_TRY(rank_T(d, P, X, Ap[j], o, ws, status, st));
+        LORA_TRY(rank_T(d, P, Xl[j], Ap[j], o, ws, status, st));
       }
     }
     // 3. U = dZ B by a rank pass: bf16 s U (LoRA K-block of dX) and (s U)^T hi/lo (dA).
@@ -1068,7 +1186,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     p.M = M;
     p.N = static_cast<int>(d->d_in);
     p.K = static_cast<int>(d->d_out);
-    p.lora_ksteps = (r + 15) / 16;
+    p.lora_ksteps = masks[0] != nullptr ? 0 : (r + 15) / 16;   // dropout: the LoRA term comes after
     p.out = static_cast<__nv_bfloat16*>(dX);
     p.z_save = nullptr;
     p.status = status;
@@ -1088,6 +1206,22 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     LORA_TRY(rs);
   }
   if (r == 0) return LORA_OK;
+  if (masks[0] != nullptr) {
+    // dX += sum_j mask_j * (s' U_j A_j), from the (s' U_j)^T hi/lo of the U pass
+    DxDropoutJob jb[2];
+    for (int j = 0; j < 2; ++j) {
+      const int jj = j < np ? j : 0;
+      jb[j].mask = masks[jj];
+      jb[j].ut_hi = static_cast<const __nv_bfloat16*>(at(P.ut_hi[jj]));
+      jb[j].ut_lo = static_cast<const __nv_bfloat16*>(at(P.ut_lo[jj]));
+      jb[j].A = static_cast<const __nv_bfloat16*>(Ap[jj]);
+    }
+    const long long tiles = ceil_div(M, kDxRows) * ceil_div(d->d_in, kDxCols);
+    const int grid = static_cast<int>(tiles < static_cast<long long>(dev.sms) * 8 ? tiles : dev.sms * 8);
+    launch_k(dx_dropout_kernel, dim3(grid), dim3(256), 0, st, false, static_cast<__nv_bfloat16*>(dX), M,
+             static_cast<int>(d->d_in), r, M8, jb[0], jb[1], np);
+    LORA_TRY(check_launch("dx_dropout_kernel"));
+  }
 
   // 5. dA^T = X^T (s U) (hi/lo operand) in one pass over X; without the fused
   //    pass above, dB = dZ^T (s T) too, hi/lo operands, split over tokens
@@ -1095,7 +1229,7 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
     RankOut ao = rank_out(static_cast<int>(d->d_in), r);
     ao.f32 = dAp[j];
     ao.transpose_f32 = 1;
-    LORA_TRY(run_rank2d(X, d->d_in, M, r, RP, nullptr, at(P.ut_hi[j]), at(P.ut_lo[j]), M8, P.sp_a, nullptr,
+    LORA_TRY(run_rank2d(Xl[j], d->d_in, M, r, RP, nullptr, at(P.ut_hi[j]), at(P.ut_lo[j]), M8, P.sp_a, nullptr,
                         static_cast<float*>(at(P.part_a)), rank_out(M, r), ao, status, st));
     if (P.dual) continue;
     RankJob Jb;
@@ -1163,6 +1297,16 @@ lora_status_t noalloc_scratch(void** out) {
 
 extern "C" {
 
+lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const void* X, const void* W, const void* A,
+                              const void* B, const void* W_up, const void* A_up, const void* B_up,
+                              const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
+                              float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream) {
+  const void* Xl[2] = {X, X};
+  const uint8_t* masks[2] = {nullptr, nullptr};
+  return bwd_core(d, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace,
+                  workspace_bytes, stream, Xl, masks);
+}
+
 lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, const void* W, const void* A,
                                       const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
                                       float* T_save, float* Z_save, void* stream) {
@@ -1181,6 +1325,137 @@ lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, 
     return cuda_error("cudaMemsetAsync(scratch status)");
   return lora_linear_fwd(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, ws, LORA_LINEAR_NOALLOC_SCRATCH_BYTES,
                          stream);
+}
+
+// ---------------------------------------------------------------------------
+// 4-bit frozen base weight ("w4g64", lora_w4.cuh)
+// ---------------------------------------------------------------------------
+
+size_t lora_linear_workspace_size_w4(const lora_linear_desc* desc, int for_backward) {
+  if (check_desc(desc) != LORA_OK || desc->d_in % kW4Group != 0) return 0;
+  const size_t base = align_up(lora_linear_workspace_size(desc, for_backward), 256);
+  return base + w4_expand_bytes(desc, for_backward != 0);
+}
+
+lora_status_t lora_linear_dequant_w4(const void* Wq, const void* Ws, int64_t d_out, int64_t d_in, void* W,
+                                     void* stream) {
+  if (Wq == nullptr || Ws == nullptr || W == nullptr || d_out <= 0 || d_in <= 0) return LORA_ERR_INVALID_ARG;
+  if (d_in % kW4Group != 0 || d_out % 8 != 0 || !aligned16(Wq) || !aligned16(Ws) || !aligned16(W))
+    return LORA_ERR_ALIGNMENT;
+  if (d_out > (int64_t(1) << 30) || d_in > (int64_t(1) << 30)) return LORA_ERR_UNSUPPORTED;
+  DevInfo dev;
+  LORA_TRY(device_info(&dev));
+  if (dev.major != 10 || dev.minor != 0) return LORA_ERR_ARCH;
+  return dequant_w4(Wq, Ws, d_out, d_in, W, static_cast<cudaStream_t>(stream));
+}
+
+lora_status_t lora_linear_fwd_w4(const lora_linear_desc* d, const void* X, const void* Wq, const void* Ws,
+                                 const void* A, const void* B, const void* Wq_up, const void* Ws_up, const void* A_up,
+                                 const void* B_up, void* Y, float* T_save, float* Z_save, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_w4(d, Wq, Ws, Wq_up, Ws_up));
+  const bool swiglu = d->act == LORA_ACT_SWIGLU;
+  if (d->M > 0 && (X == nullptr || Y == nullptr)) return LORA_ERR_INVALID_ARG;
+  if (d->r > 0 && (A == nullptr || B == nullptr)) return LORA_ERR_INVALID_ARG;
+  if (swiglu && d->r > 0 && (A_up == nullptr || B_up == nullptr)) return LORA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, A, B, A_up, B_up, Y, T_save, Z_save};
+  for (const void* q : ptrs)
+    if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
+  const size_t base = align_up(lora_linear_workspace_size(d, 0), 256);
+  DevInfo dev;
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, base + w4_expand_bytes(d, false), &dev));
+  if (d->M == 0) return LORA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (small_m_applies(d)) {
+    const Plan P = make_plan(d, false);
+    return run_small_m_fwd(d, P.sm_nt, X, nullptr, Wq, Ws, A, B, Y, T_save, Z_save, reinterpret_cast<uint32_t*>(ws),
+                           st);
+  }
+  // Many tokens: expand the weight(s) to bf16 once, then the bf16 layer.
+  uint8_t* Wd = ws + base;
+  uint8_t* Wd_up = swiglu ? Wd + static_cast<size_t>(d->d_out) * d->d_in * 2 : nullptr;
+  LORA_TRY(dequant_w4(Wq, Ws, d->d_out, d->d_in, Wd, st));
+  if (swiglu) LORA_TRY(dequant_w4(Wq_up, Ws_up, d->d_out, d->d_in, Wd_up, st));
+  return lora_linear_fwd(d, X, Wd, A, B, Wd_up, A_up, B_up, Y, T_save, Z_save, workspace, base, stream);
+}
+
+lora_status_t lora_linear_bwd_w4(const lora_linear_desc* d, const void* dY, const void* X, const void* Wq,
+                                 const void* Ws, const void* A, const void* B, const void* Wq_up, const void* Ws_up,
+                                 const void* A_up, const void* B_up, const float* T_save, const float* Z_save, void* dX,
+                                 float* dA, float* dB, float* dA_up, float* dB_up, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_w4(d, Wq, Ws, Wq_up, Ws_up));
+  const bool swiglu = d->act == LORA_ACT_SWIGLU;
+  const size_t base = align_up(lora_linear_workspace_size(d, 1), 256);
+  DevInfo dev;
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, base + w4_expand_bytes(d, true), &dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* Wd = ws + base;
+  uint8_t* Wd_up = swiglu ? Wd + static_cast<size_t>(d->d_out) * d->d_in * 2 : nullptr;
+  if (d->M > 0) {
+    LORA_TRY(dequant_w4(Wq, Ws, d->d_out, d->d_in, Wd, st));
+    if (swiglu) LORA_TRY(dequant_w4(Wq_up, Ws_up, d->d_out, d->d_in, Wd_up, st));
+  }
+  // the bf16 backward checks the remaining arguments (with M == 0 it only
+  // zero-fills dA and dB and never reads the expanded weight)
+  return lora_linear_bwd(d, dY, X, Wd, A, B, Wd_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace,
+                         base, stream);
+}
+
+// ---------------------------------------------------------------------------
+// dropout on the adapter branch's input (lora_dropout.cuh)
+// ---------------------------------------------------------------------------
+size_t lora_linear_workspace_size_dropout(const lora_linear_desc* desc, int for_backward) {
+  if (check_desc(desc) != LORA_OK) return 0;
+  return align_up(dropout_base_bytes(desc, for_backward != 0), 256) + dropout_xm_bytes(desc);
+}
+
+lora_status_t lora_linear_fwd_dropout(const lora_linear_desc* d, const void* X, const void* W, const void* A,
+                                      const void* B, const void* W_up, const void* A_up, const void* B_up,
+                                      const void* mask, const void* mask_up, float p_drop, void* Y, float* T_save,
+                                      float* Z_save, void* workspace, size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_desc(d));
+  if (d->r == 0)   // no adapter: nothing to drop
+    return lora_linear_fwd(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, workspace, workspace_bytes, stream);
+  LORA_TRY(check_dropout(d, X, mask, mask_up, p_drop));
+  lora_linear_desc d2 = *d;
+  d2.s = d->s / (1.0f - p_drop);
+  const size_t base = align_up(dropout_base_bytes(d, false), 256);
+  DevInfo dev;
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, base + dropout_xm_bytes(d), &dev));
+  if (d->M == 0) return LORA_OK;
+  const void* Xl[2];
+  LORA_TRY(mask_inputs(d, X, mask, mask_up, static_cast<uint8_t*>(workspace) + base, Xl, dev,
+                       static_cast<cudaStream_t>(stream)));
+  return fwd_core(&d2, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, workspace, base, stream, Xl, false);
+}
+
+lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* d, const void* dY, const void* X, const void* W,
+                                      const void* A, const void* B, const void* W_up, const void* A_up,
+                                      const void* B_up, const void* mask, const void* mask_up, float p_drop,
+                                      const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
+                                      float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  LORA_TRY(check_desc(d));
+  if (d->r == 0)
+    return lora_linear_bwd(d, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace,
+                           workspace_bytes, stream);
+  LORA_TRY(check_dropout(d, X, mask, mask_up, p_drop));
+  lora_linear_desc d2 = *d;
+  d2.s = d->s / (1.0f - p_drop);
+  const size_t base = align_up(dropout_base_bytes(d, true), 256);
+  DevInfo dev;
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, base + dropout_xm_bytes(d), &dev));
+  const void* Xl[2] = {X, X};
+  if (d->M > 0)
+    LORA_TRY(mask_inputs(d, X, mask, mask_up, static_cast<uint8_t*>(workspace) + base, Xl, dev,
+                         static_cast<cudaStream_t>(stream)));
+  const uint8_t* masks[2] = {static_cast<const uint8_t*>(mask),
+                             static_cast<const uint8_t*>(mask_up != nullptr ? mask_up : mask)};
+  return bwd_core(&d2, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace, base,
+                  stream, Xl, masks);
 }
 
 }  // extern "C"

@@ -23,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include "lora_linear.h"
+#include "lora_w4.cuh"
 #include "sm100.cuh"
 
 namespace lora {
@@ -32,7 +33,8 @@ constexpr int kSmThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epi
 constexpr int kSmMaxCluster = 16;
 
 struct SmallMParams {
-  CUtensorMap tm_w;          // W [d_out x d_in], box 64 x 128
+  CUtensorMap tm_w;          // W [d_out x d_in], box 64 x 128; 4-bit weight: Wq [d_out x d_in/2] bytes, box 32 x 128
+  CUtensorMap tm_ws;         // 4-bit weight only: scales [d_in/64 x d_out] bf16, box 128 x 1
   CUtensorMap tm_a;          // A [r x d_in],     box 64 x a_rows (rows >= r zero-filled)
   CUtensorMap tm_x;          // X [M x d_in],     box 64 x kNT (rows >= M zero-filled)
   const __nv_bfloat16* B;    // [d_out x r]
@@ -86,15 +88,24 @@ __device__ __forceinline__ float4 cluster_sum4(uint32_t saddr, int splits) {
   return t;
 }
 
-template <int kNT>
+template <int kNT, bool kW4>
 struct SmallMCfg {
-  static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64
-  static constexpr int kABox = 128 * 64 * 2;            // A slot: 128 rows, the first a_rows loaded
+  static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64 (4-bit weight: dequantised here)
+  // A slot: 64 rows (r <= 64 here), the first a_rows loaded.  The MMA reads a
+  // 128-row window from its start, which runs on into the bytes after it
+  // (the X, code and scale slots, the next stage, or for the last stage the
+  // B rows at the start of the tail): rows >= a_rows of D_T are garbage and
+  // never read, and the window stays inside this CTA's shared memory.
+  static constexpr int kABox = 64 * 64 * 2;
   static constexpr int kXBox = kNT * 64 * 2;            // X tile: kNT rows x 64
-  static constexpr int kStageBytes = kWBox + kABox + kXBox;
+  static constexpr int kQBox = kW4 ? 128 * 32 : 0;      // 4-bit weight: packed codes, 128 rows x 32 bytes
+  static constexpr int kSBox = kW4 ? 128 * 2 : 0;       // 4-bit weight: the 128 rows' scales of this K block
+  static constexpr int kQOff = kWBox + kABox + kXBox;
+  static constexpr int kSOff = kQOff + kQBox;
+  static constexpr int kStageBytes = (kSOff + kSBox + 1023) / 1024 * 1024;
   static constexpr int kLd = kNT + 4;                   // parked row stride (floats): 16-byte rows, conflict-free float4 stores
   static constexpr int kBsBytes = 128 * 65 * 4;         // B rows of this CTA's features, fp32, stride r + 1
-  static constexpr int kTailBytes = 1024 + kBsBytes + 1024;   // barriers, B rows, alignment slack
+  static constexpr int kTailBytes = kBsBytes + 1024 + 1024;   // B rows, barriers, alignment slack
   static constexpr int kStages0 = (kSmemLimitBytes - kTailBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
@@ -106,20 +117,25 @@ struct SmallMCfg {
   static_assert(kParkBytes <= kStages * kStageBytes, "parked partials must fit the ring");
 };
 
-template <int kNT>
+// kW4: the base weight arrives as 4-bit codes with one bf16 scale per row and
+// 64 input features; the epilogue warps, idle during the K loop, turn each
+// stage's codes into the bf16 W tile (value = bf16(scale * (code - 8)), laid
+// out as the SWIZZLE_128B tile TMA would have written) before the MMA reads it.
+template <int kNT, bool kW4>
 __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_constant__ SmallMParams p) {
-  using C = SmallMCfg<kNT>;
+  using C = SmallMCfg<kNT, kW4>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kBsBytes);
   uint64_t* full = bars;                 // [S]
   uint64_t* empty = bars + S;            // [S]
-  uint64_t* acc_full = bars + 2 * S;
+  uint64_t* dq_full = bars + 2 * S;      // [S] 4-bit weight: W tile dequantised (128 arrivals)
+  uint64_t* acc_full = bars + 3 * S;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  float* Bs = reinterpret_cast<float*>(smem + S * C::kStageBytes + 1024);   // [F][r + 1]
+  float* Bs = reinterpret_cast<float*>(smem + S * C::kStageBytes);          // [F][r + 1], first in the tail
   float* Dp = reinterpret_cast<float*>(smem);                               // [128][kLd]  Z^T partial
   float* Tp = Dp + 128 * C::kLd;                                            // [128][kLd]  T^T partial
   float* Tf = Tp + 128 * C::kLd;                                            // [64][kNT]   summed T, tokens contiguous
@@ -137,7 +153,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   const int f0 = rank * F;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); mbar_init(&dq_full[i], 128); }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -149,6 +165,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   if (threadIdx.x == 0) {
+    if constexpr (kW4) tma_prefetch_desc(&p.tm_ws);
     tma_prefetch_desc(&p.tm_w);
     tma_prefetch_desc(&p.tm_a);
     tma_prefetch_desc(&p.tm_x);
@@ -164,8 +181,14 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
         const int k0 = (kb0 + i) * 64;
-        mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kWBox + C::kXBox + p.a_rows * 128));
-        tma_load_2d(st, &p.tm_w, &full[rp.stage], k0, slice * 128);
+        if constexpr (kW4) {
+          mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kQBox + C::kSBox + C::kXBox + p.a_rows * 128));
+          tma_load_2d(st + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);    // codes: k0 / 2 bytes in
+          tma_load_2d(st + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb0 + i);   // scales of group kb0 + i
+        } else {
+          mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kWBox + C::kXBox + p.a_rows * 128));
+          tma_load_2d(st, &p.tm_w, &full[rp.stage], k0, slice * 128);
+        }
         tma_load_2d_hint(st + C::kWBox, &p.tm_a, &full[rp.stage], k0, 0, pol_x);
         tma_load_2d_hint(st + C::kWBox + C::kABox, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
         if (i == 0) sm_trace(p, kTrFirstIssue);
@@ -179,6 +202,9 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+        if constexpr (kW4) {
+          if (!mbar_wait(&dq_full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+        }
         tc_fence_after();
         if (i == 0) sm_trace(p, kTrFirstData);
         const uint32_t sw = smem_u32(smem + rp.stage * C::kStageBytes);
@@ -214,6 +240,27 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       const int fl = i / p.r, c = i - fl * p.r;
       const int n = slice * 128 + f0 + fl;
       Bs[fl * (p.r + 1) + c] = n < p.d_out ? __bfloat162float(p.B[static_cast<size_t>(n) * p.r + c]) : 0.0f;
+    }
+    if constexpr (kW4) {
+      // Dequantise each stage's W tile: thread lrow owns row lrow (32 bytes of
+      // codes, one scale) and writes its 128-byte row of the SWIZZLE_128B tile,
+      // 16-byte chunk c (features 8c .. 8c + 7) at position c ^ (lrow & 7).
+      RingPos rp;
+      for (int i = 0; i < nk; ++i) {
+        if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
+        uint8_t* st = smem + rp.stage * C::kStageBytes;
+        const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + lrow * 32);
+        const uint4 c0 = codes[0], c1 = codes[1];
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const __nv_bfloat162 sc2 =
+            __bfloat162bfloat162(reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff)[lrow]);
+        uint4* wrow = reinterpret_cast<uint4*>(st + lrow * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
+        fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
+        mbar_arrive(&dq_full[rp.stage]);
+        rp.next(S);
+      }
     }
     bool got = true;
     if (nk > 0) got = mbar_wait(acc_full, 0, ctl);
@@ -348,10 +395,10 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   }
 }
 
-template <int kNT>
+template <int kNT, bool kW4>
 cudaError_t launch_small_m_kernel(const SmallMParams& p, int slices, bool pdl, cudaStream_t st) {
-  using C = SmallMCfg<kNT>;
-  auto k = small_m_kernel<kNT>;
+  using C = SmallMCfg<kNT, kW4>;
+  auto k = small_m_kernel<kNT, kW4>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -376,10 +423,10 @@ cudaError_t launch_small_m_kernel(const SmallMParams& p, int slices, bool pdl, c
 // Cluster size: the largest power of two (<= 16, <= the K blocks) with which
 // all slices' clusters are resident at once (the device's answer for this
 // kernel, shared memory and cluster shape), so the launch is a single wave.
-template <int kNT>
+template <int kNT, bool kW4>
 int small_m_splits_t(int slices, int nkb) {
-  using C = SmallMCfg<kNT>;
-  auto k = small_m_kernel<kNT>;
+  using C = SmallMCfg<kNT, kW4>;
+  auto k = small_m_kernel<kNT, kW4>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
@@ -409,18 +456,28 @@ int small_m_splits_t(int slices, int nkb) {
   return best;
 }
 
-inline int small_m_splits(int nt, int64_t d_in, int64_t d_out) {
+inline int small_m_splits(int nt, bool w4, int64_t d_in, int64_t d_out) {
   const int slices = static_cast<int>((d_out + 127) / 128);
   const int nkb = static_cast<int>((d_in + 63) / 64);
-  if (nt == 16) return small_m_splits_t<16>(slices, nkb);
-  if (nt == 32) return small_m_splits_t<32>(slices, nkb);
-  return small_m_splits_t<64>(slices, nkb);
+  if (w4) {
+    if (nt == 16) return small_m_splits_t<16, true>(slices, nkb);
+    if (nt == 32) return small_m_splits_t<32, true>(slices, nkb);
+    return small_m_splits_t<64, true>(slices, nkb);
+  }
+  if (nt == 16) return small_m_splits_t<16, false>(slices, nkb);
+  if (nt == 32) return small_m_splits_t<32, false>(slices, nkb);
+  return small_m_splits_t<64, false>(slices, nkb);
 }
 
-inline cudaError_t launch_small_m(const SmallMParams& p, int nt, int slices, bool pdl, cudaStream_t st) {
-  if (nt == 16) return launch_small_m_kernel<16>(p, slices, pdl, st);
-  if (nt == 32) return launch_small_m_kernel<32>(p, slices, pdl, st);
-  return launch_small_m_kernel<64>(p, slices, pdl, st);
+inline cudaError_t launch_small_m(const SmallMParams& p, int nt, bool w4, int slices, bool pdl, cudaStream_t st) {
+  if (w4) {
+    if (nt == 16) return launch_small_m_kernel<16, true>(p, slices, pdl, st);
+    if (nt == 32) return launch_small_m_kernel<32, true>(p, slices, pdl, st);
+    return launch_small_m_kernel<64, true>(p, slices, pdl, st);
+  }
+  if (nt == 16) return launch_small_m_kernel<16, false>(p, slices, pdl, st);
+  if (nt == 32) return launch_small_m_kernel<32, false>(p, slices, pdl, st);
+  return launch_small_m_kernel<64, false>(p, slices, pdl, st);
 }
 
 }  // namespace lora

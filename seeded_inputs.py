@@ -12,6 +12,14 @@ are used, every tensor is drawn here):
 * A  ~ U(-1/sqrt(d_in), +1/sqrt(d_in))   r x d_in      (maps d_in -> r)
 * B  ~ N(0, 0.02^2)       d_out x r                    (maps r -> d_out)
 * dY ~ N(0, 1)            tokens x d_out (upstream gradient)
+* 4-bit base weight (the library's "w4g64" format): codes uniform in 0..15,
+  packed two per byte (Wq: uint8 d_out x d_in/2, drawn as uniform bytes), and
+  one scale per row and group of 64 input features (Ws: bf16 d_in/64 x d_out)
+  ~ U(0.5, 1.5) / (4.6 sqrt(d_in)), so that the weight has roughly the spread
+  of W above (the codes minus 8 have a standard deviation of about 4.6).
+* dropout masks on the adapter input: each element of X kept with probability
+  1 - p, packed eight per byte (bit j of byte b, least significant first, is
+  element 8 b + j): uint8 tokens x d_in/8.
 
 Each tensor has its own stream: numpy's PCG64 seeded with (seed, tensor id).
 Values are drawn in float64, rounded to float32 (round-to-nearest-even) and
@@ -26,6 +34,8 @@ import numpy as np
 _TENSOR_IDS = {
     "X": 1, "W": 2, "A": 3, "B": 4, "dY": 5,
     "W_up": 6, "A_up": 7, "B_up": 8,
+    "Wq": 9, "Ws": 10, "Wq_up": 11, "Ws_up": 12,
+    "mask": 13, "mask_up": 14,
 }
 
 ACTS = ("identity", "silu", "swiglu")
@@ -40,6 +50,10 @@ CONFIGS = {
     "mlp_down": dict(M=8192, d_in=14336, d_out=4096, r=64, alpha=16.0, act="identity"),
     "small_m": dict(M=16, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity"),
     "small_m_ragged": dict(M=1000, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity"),
+    # the few-token workload with the base weight in the 4-bit "w4g64" format
+    "small_m_w4": dict(M=16, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity", weight="w4"),
+    # q_proj with dropout p = 0.1 on the adapter input (the mask is drawn here)
+    "q_proj_dropout": dict(M=16384, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity", dropout=0.1),
 }
 
 
@@ -80,6 +94,23 @@ def draw(name: str, shape, seed: int, d_in: int) -> np.ndarray:
     else:  # pragma: no cover
         raise KeyError(name)
     return f64_to_bf16_bits(v)
+
+
+def draw_w4(name: str, d_out: int, d_in: int, seed: int):
+    """A 4-bit weight of the recipe above: (Wq uint8 [d_out x d_in/2], Ws bf16 bits [d_in/64 x d_out]).
+    ``name`` is "W" or "W_up"."""
+    suffix = name[1:]                       # "" or "_up"
+    gq = _rng(seed, "Wq" + suffix)
+    Wq = gq.integers(0, 256, size=(d_out, d_in // 2), dtype=np.uint8)
+    gs = _rng(seed, "Ws" + suffix)
+    Ws = f64_to_bf16_bits(gs.uniform(0.5, 1.5, size=(d_in // 64, d_out)) / (4.6 * np.sqrt(d_in)))
+    return Wq, Ws
+
+
+def draw_mask(name: str, M: int, d_in: int, p_drop: float, seed: int) -> np.ndarray:
+    """A packed dropout mask of the recipe above; ``name`` is "mask" or "mask_up"."""
+    keep = _rng(seed, name).random((M, d_in)) >= p_drop
+    return np.packbits(keep.astype(np.uint8), axis=1, bitorder="little")
 
 
 def make_inputs(M: int, d_in: int, d_out: int, r: int, act: str = "identity",

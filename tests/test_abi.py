@@ -28,6 +28,24 @@ def test_header_declares_expected(lib):
     assert set(declared_functions()) == set(lib.EXPORTED)
 
 
+def declared_arity():
+    """{function: number of parameters} from the header's prototypes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(lora_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_bindings_match_header_arity(lib):
+    """Every ctypes binding declares as many arguments as the C prototype."""
+    lib.lora_linear_abi_version()          # loads the library and its argtypes
+    handle = lib._LazyLib._h
+    for name, n in declared_arity().items():
+        assert len(getattr(handle, name).argtypes) == n, name
+
+
 def test_library_exports_every_declared_symbol(lib):
     so = ctypes.CDLL(lib.LIB_PATH)
     for name in declared_functions():
@@ -106,3 +124,31 @@ def test_selftest_rejects_bad_arguments_without_launching(lib):
     assert lib.lora_linear_selftest_wait_timeout(16, 64, 16, None) == 5          # below the header
     assert lib.lora_linear_selftest_wait_timeout(16, 1 << 20, 5, None) == 1      # INVALID_ARG
     assert lib.lora_linear_selftest_wait_timeout(16, 1 << 20, 31, None) == 1
+
+
+def test_dropout_and_w4_argument_checks(lib):
+    d = lib.make_desc(64, 256, 256, 8, 2.0, "identity")
+    assert lib.lora_linear_workspace_size_dropout(d, 1) >= lib.lora_linear_workspace_size_dropout(d, 0) > 0
+    # the masked input copy is part of the dropout workspace
+    assert lib.lora_linear_workspace_size_dropout(d, 0) >= lib.lora_linear_workspace_size(d, 0) + 64 * 256 * 2
+    fwd = lambda mask=16, p=0.1, **kw: lib.lora_linear_fwd_dropout(d, 16, 16, 16, 16, None, None, None, mask, None,
+                                                                   p, 16, None, None, 16, 1 << 30, None)
+    assert fwd(p=1.0) == 1                     # p_drop must be < 1
+    assert fwd(p=-0.1) == 1
+    assert fwd(mask=None) == 1                 # the mask is required with tokens and an adapter
+    sw = lib.make_desc(64, 256, 256, 8, 2.0, "swiglu")
+    assert lib.lora_linear_fwd_dropout(sw, 16, 16, 16, 16, 16, 16, 16, 16, None, 0.1, 16, None, None, 16, 1 << 30,
+                                       None) == 1   # SwiGLU needs its up projection's mask
+    # 4-bit weight: d_in must be a multiple of 64; the codes and scales are required
+    assert lib.lora_linear_workspace_size_w4(lib.make_desc(64, 264, 256, 8, 2.0, 0), 0) == 0
+    few = lib.make_desc(16, 256, 256, 8, 2.0, "identity")
+    many = lib.make_desc(4096, 256, 256, 8, 2.0, "identity")
+    assert lib.lora_linear_workspace_size_w4(few, 0) == 256      # the few-token forward reads the codes directly
+    assert lib.lora_linear_workspace_size_w4(many, 0) >= lib.lora_linear_workspace_size(many, 0) + 256 * 256 * 2
+    w4 = lambda desc, Wq=16, Ws=16: lib.lora_linear_fwd_w4(desc, 16, Wq, Ws, 16, 16, None, None, None, None, 16,
+                                                           None, None, 16, 1 << 30, None)
+    assert w4(lib.make_desc(64, 264, 256, 8, 2.0, 0)) == 2       # d_in % 64
+    assert w4(few, Wq=None) == 1
+    assert w4(few, Ws=24) == 2                                     # 16-byte alignment
+    assert lib.lora_linear_dequant_w4(16, 16, 256, 100, 16, None) == 2
+    assert lib.lora_linear_dequant_w4(None, 16, 256, 128, 16, None) == 1
