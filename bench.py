@@ -330,6 +330,10 @@ def main():
     if w4:
         t["Wq"] = torch.from_numpy(Wq).cuda()
         t["Ws"] = torch.from_numpy(Ws.view(np.int16)).view(torch.bfloat16).cuda()
+        # the frozen weight's codes in the few-token kernel's tiled layout (a load-time step)
+        t["Wt"] = torch.empty(L.lora_linear_w4_tiled_bytes(d_out, d_in), dtype=torch.uint8, device="cuda")
+        assert L.lora_linear_w4_tile(t["Wq"].data_ptr(), d_out, d_in, t["Wt"].data_ptr(),
+                                     torch.cuda.current_stream().cuda_stream) == 0
     p_drop = cfg.get("dropout")
     if p_drop is not None:   # dropout on the adapter input: one mask per projection, an input like X
         for name in ("mask", "mask_up") if act == "swiglu" else ("mask",):
@@ -354,7 +358,10 @@ def main():
     p = lambda x: None if x is None else x.data_ptr()  # noqa: E731
 
     def fwd():
-        if w4:
+        if w4 and M <= 64:
+            st = L.lora_linear_fwd_w4_tiled(desc, p(t["X"]), p(t["Wt"]), p(t["Ws"]), p(t["A"]), p(t["B"]), p(Y),
+                                            p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
+        elif w4:
             st = L.lora_linear_fwd_w4(desc, p(t["X"]), p(t["Wq"]), p(t["Ws"]), p(t["A"]), p(t["B"]), None, None,
                                       None, None, p(Y), p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
         elif p_drop is not None:

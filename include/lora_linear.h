@@ -265,6 +265,27 @@ lora_status_t lora_linear_bwd_w4(const lora_linear_desc* desc, const void* dY, c
                                  void* dX, float* dA, float* dB, float* dA_up, float* dB_up, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* Tiled code layout for the few-token forward: the codes of each 128-row x
+ * 64-feature tile are 4096 contiguous bytes (row i of the tile at byte 32 i,
+ * same nibble order), tiles ordered by 128-row slice, then by 64-feature
+ * block: tile (g, kb) at byte (g * d_in/64 + kb) * 4096; rows past d_out are
+ * zero.  A stage then loads one contiguous 4 KB block instead of 128
+ * 32-byte row pieces.  The base weight is frozen, so this is a load-time
+ * step.
+ * lora_linear_w4_tiled_bytes: size of the tiled codes (0 if d_in % 64 != 0
+ *   or a size is not positive).
+ * lora_linear_w4_tile: writes Wt (device, that size) from the row-major Wq;
+ *   asynchronous on `stream`; 16-byte aligned pointers.
+ * lora_linear_fwd_w4_tiled: the few-token forward (1..64 tokens, identity or
+ *   SiLU, 0 < r <= 64; else LORA_ERR_UNSUPPORTED; M == 0 is a no-op) on the
+ *   tiled codes Wt and the scales Ws; other arguments as lora_linear_fwd;
+ *   workspace >= lora_linear_workspace_size(desc, 0). */
+size_t lora_linear_w4_tiled_bytes(int64_t d_out, int64_t d_in);
+lora_status_t lora_linear_w4_tile(const void* Wq, int64_t d_out, int64_t d_in, void* Wt, void* stream);
+lora_status_t lora_linear_fwd_w4_tiled(const lora_linear_desc* desc, const void* X, const void* Wt, const void* Ws,
+                                       const void* A, const void* B, void* Y, float* T_save, float* Z_save,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Dropout on the adapter branch's input.  The pages' LoRA configurations set
  * a LoRA dropout (lora_dropout = 0.05 in "Swift-All一文详解：如何用Liger-Kernel

@@ -30,7 +30,8 @@ EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_li
             "lora_linear_launch_count", "lora_linear_fwd_noalloc", "lora_linear_timing_enable",
             "lora_linear_timing_read", "lora_linear_selftest_wait_timeout",
             "lora_linear_workspace_size_w4", "lora_linear_dequant_w4", "lora_linear_fwd_w4", "lora_linear_bwd_w4",
-            "lora_linear_workspace_size_dropout", "lora_linear_fwd_dropout", "lora_linear_bwd_dropout")
+            "lora_linear_workspace_size_dropout", "lora_linear_fwd_dropout", "lora_linear_bwd_dropout",
+            "lora_linear_w4_tiled_bytes", "lora_linear_w4_tile", "lora_linear_fwd_w4_tiled")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -83,6 +84,13 @@ def _load():
     lib.lora_linear_fwd_w4.restype = i32
     lib.lora_linear_bwd_w4.argtypes = [dp] + [vp] * 17 + [vp, sz, vp]
     lib.lora_linear_bwd_w4.restype = i32
+    i64 = ctypes.c_int64
+    lib.lora_linear_w4_tiled_bytes.argtypes = [i64, i64]
+    lib.lora_linear_w4_tiled_bytes.restype = sz
+    lib.lora_linear_w4_tile.argtypes = [vp, i64, i64, vp, vp]
+    lib.lora_linear_w4_tile.restype = i32
+    lib.lora_linear_fwd_w4_tiled.argtypes = [dp] + [vp] * 8 + [vp, sz, vp]
+    lib.lora_linear_fwd_w4_tiled.restype = i32
     f32 = ctypes.c_float
     lib.lora_linear_workspace_size_dropout.argtypes = [dp, i32]
     lib.lora_linear_workspace_size_dropout.restype = sz
@@ -171,6 +179,19 @@ def lora_linear_fwd_w4(desc, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, Y, T_sav
                        workspace_bytes, stream) -> int:
     return int(_lib.lora_linear_fwd_w4(ctypes.byref(desc), X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, Y, T_save,
                                        Z_save, workspace, workspace_bytes, stream))
+
+
+def lora_linear_w4_tiled_bytes(d_out, d_in) -> int:
+    return int(_lib.lora_linear_w4_tiled_bytes(int(d_out), int(d_in)))
+
+
+def lora_linear_w4_tile(Wq, d_out, d_in, Wt, stream) -> int:
+    return int(_lib.lora_linear_w4_tile(Wq, int(d_out), int(d_in), Wt, stream))
+
+
+def lora_linear_fwd_w4_tiled(desc, X, Wt, Ws, A, B, Y, T_save, Z_save, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_fwd_w4_tiled(ctypes.byref(desc), X, Wt, Ws, A, B, Y, T_save, Z_save, workspace,
+                                             workspace_bytes, stream))
 
 
 def lora_linear_bwd_w4(desc, dY, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up,

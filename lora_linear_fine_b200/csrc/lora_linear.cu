@@ -665,12 +665,15 @@ lora_status_t common_checks(const lora_linear_desc* d, void* ws, size_t ws_bytes
 // W is bf16, or (Wq != null) the 4-bit codes Wq with scales Ws.
 lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, const void* W, const void* Wq,
                               const void* Ws, const void* A, const void* B, void* Y, float* T_save, float* Z_save,
-                              uint32_t* status, cudaStream_t st) {
+                              uint32_t* status, cudaStream_t st, const void* Wt = nullptr) {
   const int64_t M = d->M, r = d->r;
   SmallMParams q;
   std::memset(&q, 0, sizeof(q));
-  const bool w4 = Wq != nullptr;
-  bool ok = w4 ? make_tm_plain(&q.tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, d->d_in / 2, d->d_out, d->d_in / 2, 32,
+  const bool w4 = Wq != nullptr || Wt != nullptr;
+  q.Wt = static_cast<const uint8_t*>(Wt);
+  bool ok = Wt != nullptr ? make_tm_plain(&q.tm_ws, Ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->d_out,
+                                          d->d_in / kW4Group, d->d_out * 2, 128, 1)
+          : w4 ? make_tm_plain(&q.tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, d->d_in / 2, d->d_out, d->d_in / 2, 32,
                                128) &&
                      make_tm_plain(&q.tm_ws, Ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->d_out, d->d_in / kW4Group,
                                    d->d_out * 2, 128, 1)
@@ -720,8 +723,16 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
     unsigned long long t0 = ~0ull;
     for (int b = 0; b < grid; ++b) t0 = h[b * kSmTracePoints] && h[b * kSmTracePoints] < t0 ? h[b * kSmTracePoints] : t0;
     static const char* names[kSmTracePoints] = {"entry", "first_issue", "first_data", "last_mma", "published",
-                                                "synced", "t_summed", "combined", "exit"};
+                                                "synced", "t_summed", "combined", "exit", "dq_wait", "dq_work"};
     for (int k = 0; k < kSmTracePoints; ++k) {
+      if (k == kTrDqWait || k == kTrDqWork) {   // durations, not stamps
+        double tot = 0;
+        int cnt = 0;
+        for (int b = 0; b < grid; ++b)
+          if (h[b * kSmTracePoints + k]) { tot += h[b * kSmTracePoints + k] * 1e-3; ++cnt; }
+        if (cnt) LORA_LOG("small_m trace %-12s n=%3d mean total %7.2f us", names[k], cnt, tot / cnt);
+        continue;
+      }
       double mn = 1e30, mx = 0, sum = 0;
       int n = 0;
       for (int b = 0; b < grid; ++b) {
@@ -1456,6 +1467,44 @@ lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* d, const void* dY,
                              static_cast<const uint8_t*>(mask_up != nullptr ? mask_up : mask)};
   return bwd_core(&d2, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace, base,
                   stream, Xl, masks);
+}
+
+// 4-bit weight, tiled code layout for the few-token forward (lora_w4.cuh)
+size_t lora_linear_w4_tiled_bytes(int64_t d_out, int64_t d_in) {
+  if (d_out <= 0 || d_in <= 0 || d_in % kW4Group != 0) return 0;
+  return static_cast<size_t>((d_out + 127) / 128) * static_cast<size_t>(d_in / kW4Group) * kW4TileBytes;
+}
+
+lora_status_t lora_linear_w4_tile(const void* Wq, int64_t d_out, int64_t d_in, void* Wt, void* stream) {
+  if (Wq == nullptr || Wt == nullptr || d_out <= 0 || d_in <= 0) return LORA_ERR_INVALID_ARG;
+  if (d_in % kW4Group != 0 || !aligned16(Wq) || !aligned16(Wt)) return LORA_ERR_ALIGNMENT;
+  if (d_out > (int64_t(1) << 30) || d_in > (int64_t(1) << 30)) return LORA_ERR_UNSUPPORTED;
+  DevInfo dev;
+  LORA_TRY(device_info(&dev));
+  if (dev.major != 10 || dev.minor != 0) return LORA_ERR_ARCH;
+  const long long n16 = static_cast<long long>(lora_linear_w4_tiled_bytes(d_out, d_in) / 16);
+  launch_k(tile_w4_kernel, dim3(grid_for(n16, 256, dev.sms)), dim3(256), 0, static_cast<cudaStream_t>(stream), false,
+           static_cast<const uint8_t*>(Wq), static_cast<long long>(d_out), static_cast<int>(d_in),
+           static_cast<uint8_t*>(Wt));
+  return check_launch("tile_w4_kernel");
+}
+
+lora_status_t lora_linear_fwd_w4_tiled(const lora_linear_desc* d, const void* X, const void* Wt, const void* Ws,
+                                       const void* A, const void* B, void* Y, float* T_save, float* Z_save,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_w4(d, Wt, Ws, nullptr, nullptr));
+  if (d->M != 0 && !small_m_applies(d)) return LORA_ERR_UNSUPPORTED;
+  if (d->M > 0 && (X == nullptr || Y == nullptr)) return LORA_ERR_INVALID_ARG;
+  if (A == nullptr || B == nullptr) return LORA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, A, B, Y, T_save, Z_save};
+  for (const void* q : ptrs)
+    if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
+  const Plan P = make_plan(d, false);
+  DevInfo dev;
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
+  if (d->M == 0) return LORA_OK;
+  return run_small_m_fwd(d, P.sm_nt, X, nullptr, nullptr, Ws, A, B, Y, T_save, Z_save,
+                         reinterpret_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream), Wt);
 }
 
 }  // extern "C"

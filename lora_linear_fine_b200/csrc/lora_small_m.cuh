@@ -35,6 +35,7 @@ constexpr int kSmMaxCluster = 16;
 struct SmallMParams {
   CUtensorMap tm_w;          // W [d_out x d_in], box 64 x 128; 4-bit weight: Wq [d_out x d_in/2] bytes, box 32 x 128
   CUtensorMap tm_ws;         // 4-bit weight only: scales [d_in/64 x d_out] bf16, box 128 x 1
+  const uint8_t* Wt;         // 4-bit weight: the codes in the tiled layout (lora_w4.cuh), or null (tm_w)
   CUtensorMap tm_a;          // A [r x d_in],     box 64 x a_rows (rows >= r zero-filled)
   CUtensorMap tm_x;          // X [M x d_in],     box 64 x kNT (rows >= M zero-filled)
   const __nv_bfloat16* B;    // [d_out x r]
@@ -54,8 +55,15 @@ struct SmallMParams {
 // Trace points of one CTA (LORA_LINEAR_DEBUG=2 prints them per launch).
 enum SmTrace : int {
   kTrEntry = 0, kTrFirstIssue, kTrFirstData, kTrLastMma, kTrPublished, kTrSynced, kTrTSummed, kTrCombined, kTrExit,
+  kTrDqWait, kTrDqWork,   // 4-bit weight: total ns the expanding warps waited for data / spent expanding
   kSmTracePoints
 };
+
+__device__ __forceinline__ unsigned long long sm_clock_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) : : "memory");
+  return t;
+}
 
 __device__ __forceinline__ void sm_trace(const SmallMParams& p, int point) {
   if (p.trace != nullptr) {
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   const uint32_t tbase = *tmem_slot;
   if (threadIdx.x == 0) {
     if constexpr (kW4) tma_prefetch_desc(&p.tm_ws);
-    tma_prefetch_desc(&p.tm_w);
+    if (!kW4 || p.Wt == nullptr) tma_prefetch_desc(&p.tm_w);
     tma_prefetch_desc(&p.tm_a);
     tma_prefetch_desc(&p.tm_x);
   }
@@ -183,7 +191,11 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         const int k0 = (kb0 + i) * 64;
         if constexpr (kW4) {
           mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kQBox + C::kSBox + C::kXBox + p.a_rows * 128));
-          tma_load_2d(st + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);    // codes: k0 / 2 bytes in
+          if (p.Wt != nullptr)      // one 4 KB tile of codes
+            bulk_load_1d(st + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kb0 + i) * kW4TileBytes,
+                         kW4TileBytes, &full[rp.stage]);
+          else
+            tma_load_2d(st + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);  // codes: k0 / 2 bytes in
           tma_load_2d(st + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb0 + i);   // scales of group kb0 + i
         } else {
           mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kWBox + C::kXBox + p.a_rows * 128));
@@ -246,8 +258,11 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       // codes, one scale) and writes its 128-byte row of the SWIZZLE_128B tile,
       // 16-byte chunk c (features 8c .. 8c + 7) at position c ^ (lrow & 7).
       RingPos rp;
+      const bool tr = p.trace != nullptr && et == 0;
+      unsigned long long t_wait = 0, t_work = 0, t0 = tr ? sm_clock_ns() : 0;
       for (int i = 0; i < nk; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
+        if (tr) { const unsigned long long t1 = sm_clock_ns(); t_wait += t1 - t0; t0 = t1; }
         uint8_t* st = smem + rp.stage * C::kStageBytes;
         const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + lrow * 32);
         const uint4 c0 = codes[0], c1 = codes[1];
@@ -259,7 +274,12 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
         fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
         mbar_arrive(&dq_full[rp.stage]);
+        if (tr) { const unsigned long long t1 = sm_clock_ns(); t_work += t1 - t0; t0 = t1; }
         rp.next(S);
+      }
+      if (tr) {
+        p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + kTrDqWait] = t_wait;
+        p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + kTrDqWork] = t_work;
       }
     }
     bool got = true;

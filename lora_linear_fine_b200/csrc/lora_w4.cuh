@@ -56,4 +56,32 @@ __global__ void __launch_bounds__(256) dequant_w4_kernel(const uint8_t* __restri
   }
 }
 
+// Tiled layout of the codes for the few-token kernel: the codes of each
+// 128-row x 64-feature tile are 4096 contiguous bytes (row i of the tile at
+// 32 i, the nibble order of the row-major format), tiles ordered by 128-row
+// slice, then by 64-feature block: tile (g, kb) starts at (g * d_in/64 + kb) *
+// 4096.  Rows past d_out (in the last slice) are zero.  One 4 KB bulk copy
+// then brings a stage's codes, instead of 128 separate 32-byte row pieces.
+constexpr int kW4TileBytes = 128 * 32;
+
+// One thread per 16 bytes of the tiled output, grid-stride.
+__global__ void __launch_bounds__(256) tile_w4_kernel(const uint8_t* __restrict__ Wq, long long d_out, int d_in,
+                                                      uint8_t* __restrict__ Wt) {
+  grid_dep_wait();
+  const int nkb = d_in / kW4Group;
+  const long long slices = (d_out + 127) / 128;
+  const long long n16 = slices * nkb * (kW4TileBytes / 16);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long tile = i / (kW4TileBytes / 16);
+    const int within = static_cast<int>(i - tile * (kW4TileBytes / 16));   // 16-byte piece: row within / 2, half within % 2
+    const long long g = tile / nkb;
+    const int kb = static_cast<int>(tile - g * nkb);
+    const long long n = g * 128 + within / 2;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (n < d_out) v = *reinterpret_cast<const uint4*>(Wq + n * (d_in / 2) + kb * 32 + (within & 1) * 16);
+    reinterpret_cast<uint4*>(Wt)[i] = v;
+  }
+}
+
 }  // namespace lora

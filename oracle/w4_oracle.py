@@ -62,6 +62,20 @@ def w4_dequant(Wq: np.ndarray, Ws_bits: np.ndarray) -> np.ndarray:
     return round_to_bf16(per_elem * (q - 8).astype(np.float64))
 
 
+def w4_tile(Wq: np.ndarray) -> np.ndarray:
+    """The tiled code layout of the few-token kernel: tiles of 128 rows x 64
+    features (4096 bytes each, row i of a tile at byte 32 i), ordered by
+    128-row slice then by 64-feature block; rows past d_out are zero.
+    Returns a flat uint8 array."""
+    b = np.asarray(Wq, dtype=np.uint8)
+    d_out, half = b.shape
+    slices, nkb = (d_out + 127) // 128, half // 32
+    padded = np.zeros((slices * 128, half), dtype=np.uint8)
+    padded[:d_out] = b
+    t = padded.reshape(slices, 128, nkb, 32).transpose(0, 2, 1, 3)   # [slice][kblock][row][32 bytes]
+    return np.ascontiguousarray(t).reshape(-1)
+
+
 def w4_forward(X, Wq, Ws_bits, A, B, s, act="identity", Wq_up=None, Ws_up_bits=None, A_up=None, B_up=None):
     """The LoRA forward with the dequantised base weight(s)."""
     W = w4_dequant(Wq, Ws_bits)

@@ -106,3 +106,48 @@ def test_fwd_w4_few_tokens(M, d_in, d_out, r, act):
 def test_fwd_bwd_w4(M, d_in, d_out, r, act):
     out, ref, _ = _run(M, d_in, d_out, r, act, seed=8, backward=True)
     G.assert_all_ok(G.compare_all(out, ref, act, r, backward=True))
+
+
+@pytest.mark.parametrize("d_out,d_in", [(264, 384), (4096, 4096)])
+def test_tile_bit_exact(d_out, d_in):
+    import lora_linear_fine_b200 as L
+    import torch
+    Wq, _ = seeded_inputs.draw_w4("W", d_out, d_in, 4)
+    Wq_d = _u8(Wq)
+    Wt = torch.empty(L.lora_linear_w4_tiled_bytes(d_out, d_in), dtype=torch.uint8, device="cuda")
+    assert L.lora_linear_w4_tile(Wq_d.data_ptr(), d_out, d_in, Wt.data_ptr(),
+                                 torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert np.array_equal(Wt.cpu().numpy(), w4_oracle.w4_tile(Wq))
+
+
+@pytest.mark.parametrize("M,d_in,d_out,r,act", [
+    (16, 4096, 4096, 8, "identity"),
+    (5, 512, 264, 16, "silu"),
+    (64, 768, 520, 64, "identity"),
+])
+def test_fwd_w4_tiled_few_tokens(M, d_in, d_out, r, act):
+    """The tiled-code forward: parity with the oracle, and bit-identical to the
+    row-major-code forward (same kernel, same arithmetic, only the loads differ)."""
+    import lora_linear_fine_b200 as L
+    import torch
+    out, ref, s = _run(M, d_in, d_out, r, act, seed=7, backward=False)
+    inp, w4 = _w4_inputs(M, d_in, d_out, r, act, 7)
+    t = {k: G.dev(v) for k, v in inp.items()}
+    Wq_d, Ws_d = _u8(w4["Wq"]), G.dev(w4["Ws"])
+    sh = torch.cuda.current_stream().cuda_stream
+    Wt = torch.empty(L.lora_linear_w4_tiled_bytes(d_out, d_in), dtype=torch.uint8, device="cuda")
+    assert L.lora_linear_w4_tile(Wq_d.data_ptr(), d_out, d_in, Wt.data_ptr(), sh) == 0
+    desc = L.make_desc(M, d_in, d_out, r, s, act)
+    ws = L.Workspace(L.lora_linear_workspace_size(desc, 0))
+    Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
+    T = torch.empty((1, M, r), dtype=torch.float32, device="cuda")
+    Z = torch.empty((1, M, d_out), dtype=torch.float32, device="cuda") if act != "identity" else None
+    st = L.lora_linear_fwd_w4_tiled(desc, t["X"].data_ptr(), Wt.data_ptr(), Ws_d.data_ptr(), t["A"].data_ptr(),
+                                    t["B"].data_ptr(), Y.data_ptr(), T.data_ptr(),
+                                    Z.data_ptr() if Z is not None else None, ws.buf.data_ptr(), ws.nbytes, sh)
+    assert st == 0, L.status_string(st)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    assert torch.equal(Y, out["Y"]) and torch.equal(T, out["T"])
+    G.assert_all_ok(G.compare_all({"Y": Y, "T": T, "Z": Z}, ref, act, r, backward=False))

@@ -15,9 +15,10 @@ def test_w4_pin(check):
     check(w4_oracle)
 
 
-def _namespace(dequant):
+def _namespace(dequant, tile=None):
     ns = types.SimpleNamespace()
     ns.w4_dequant = dequant
+    ns.w4_tile = tile or w4_oracle.w4_tile
 
     def fwd(X, Wq, Ws, A, B, s, act="identity", *rest):
         return oracle.lora_forward(X, dequant(Wq, Ws), A, B, s, act)
@@ -81,6 +82,28 @@ def m_group_32(Wq, Ws):
 
 MUTANTS = [m_swapped_nibbles, m_zero_point_7, m_scales_row_major, m_truncate_not_round, m_no_rounding,
            m_group_32]
+
+
+def t_kblock_major(Wq):
+    """Tiles ordered by 64-feature block first, then by slice."""
+    b = np.asarray(Wq, dtype=np.uint8)
+    d_out, half = b.shape
+    slices, nkb = (d_out + 127) // 128, half // 32
+    padded = np.zeros((slices * 128, half), dtype=np.uint8)
+    padded[:d_out] = b
+    return np.ascontiguousarray(padded.reshape(slices, 128, nkb, 32).transpose(2, 0, 1, 3)).reshape(-1)
+
+
+def t_rows_not_padded(Wq):
+    """The last slice's missing rows left out instead of zero-filled."""
+    return w4_oracle.w4_tile(Wq)[: np.asarray(Wq).size]
+
+
+@pytest.mark.parametrize("tile", [t_kblock_major, t_rows_not_padded], ids=lambda m: m.__name__)
+def test_w4_tile_planted_mistake_fails_a_pin(tile):
+    ns = _namespace(w4_oracle.w4_dequant, tile)
+    with pytest.raises(AssertionError):
+        w4_pins.check_w4_tile_brute_force(ns)
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda m: m.__name__)

@@ -12,7 +12,9 @@ scale * (code - 8)).  The facts used are therefore:
   inputs (bit fields by shifts, the bf16 rounding by integer arithmetic on the
   float32 bit pattern), independent of the oracle's vectorised numpy code;
 * with B = 0 the quantised layer is the plain product with the dequantised
-  weight, by scalar loops.
+  weight, by scalar loops;
+* the tiled code layout of the few-token kernel, element by element with
+  loops.
 
 Each ``check_*`` takes the module (or a copy with a planted mistake) and raises
 AssertionError when it disagrees with the fact.
@@ -114,9 +116,28 @@ def check_w4_zero_adapter_is_plain_product(w4):
             assert Y[m, n] == acc, (m, n, Y[m, n], acc)
 
 
+def check_w4_tile_brute_force(w4):
+    """The tiled code layout, element by element with loops: tile (g, kb), row
+    i, byte j holds byte kb*32 + j of weight row g*128 + i (zero past d_out)."""
+    rng = np.random.default_rng(14)
+    d_out, d_in = 130, 128
+    Wq = rng.integers(0, 256, size=(d_out, d_in // 2), dtype=np.uint8)
+    t = w4.w4_tile(Wq)
+    nkb, slices = d_in // 64, (d_out + 127) // 128
+    assert t.shape == (slices * nkb * 4096,)
+    for g in range(slices):
+        for kb in range(nkb):
+            for i in range(128):
+                for j in range(32):
+                    n = g * 128 + i
+                    want = int(Wq[n, kb * 32 + j]) if n < d_out else 0
+                    assert int(t[((g * nkb + kb) * 128 + i) * 32 + j]) == want, (g, kb, i, j)
+
+
 ALL_CHECKS = [
     check_w4_golden,
     check_w4_power_of_two_scales_are_exact,
     check_w4_brute_force_decoding,
     check_w4_zero_adapter_is_plain_product,
+    check_w4_tile_brute_force,
 ]
