@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 256 * C::kCtas); }
+    // acc_empty: one arrival per epilogue warp of every CTA of the unit
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 8 * C::kCtas); }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -346,10 +347,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
       const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
-      auto release_acc = [&]() {
+      auto release_acc = [&]() {   // every lane's tcgen05.ld has completed (tmem_wait_ld)
         tc_fence_before();
-        if constexpr (kPair) mbar_arrive_cluster(acc_empty_addr[buf]);
-        else mbar_arrive(&acc_empty[buf]);
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(acc_empty_addr[buf]);
+          else mbar_arrive(&acc_empty[buf]);
+        }
       };
       if constexpr (C::kStaged) {
         // Two halves of this thread's columns (SiLU: 64 + 64 of its 128;

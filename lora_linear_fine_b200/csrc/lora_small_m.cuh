@@ -96,6 +96,15 @@ __device__ __forceinline__ float4 cluster_sum4(uint32_t saddr, int splits) {
   return t;
 }
 
+// 16 fp32 columns of this warp's TMEM lanes.
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&out)[16]) {
+  uint32_t v[16];
+  tmem_ld16(taddr, v);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 16; ++c) out[c] = __uint_as_float(v[c]);
+}
+
 template <int kNT, bool kW4>
 struct SmallMCfg {
   static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64 (4-bit weight: dequantised here)
@@ -138,7 +147,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kBsBytes);
   uint64_t* full = bars;                 // [S]
   uint64_t* empty = bars + S;            // [S]
-  uint64_t* dq_full = bars + 2 * S;      // [S] 4-bit weight: W tile dequantised (128 arrivals)
+  uint64_t* dq_full = bars + 2 * S;      // [S] 4-bit weight: W tile expanded (one arrival per epilogue warp)
   uint64_t* acc_full = bars + 3 * S;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 2);
@@ -161,7 +170,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   const int f0 = rank * F;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); mbar_init(&dq_full[i], 128); }
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); mbar_init(&dq_full[i], 4); }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -184,19 +193,24 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t pol_x = l2_policy_evict_last();     // X and A are re-read by every cluster
+      // Every slice's CTA of the same rank reads the same A and X tiles; each
+      // slice starts its K loop at a different block (slice mod nk) so that
+      // those reads spread over the L2 instead of converging on one tile.
+      const int rot = nk > 0 ? slice % nk : 0;
       RingPos rp;
       for (int i = 0; i < nk; ++i) {
+        const int kb = kb0 + (i + rot) % nk;
         if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
-        const int k0 = (kb0 + i) * 64;
+        const int k0 = kb * 64;
         if constexpr (kW4) {
           mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kQBox + C::kSBox + C::kXBox + p.a_rows * 128));
           if (p.Wt != nullptr)      // one 4 KB tile of codes
-            bulk_load_1d(st + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kb0 + i) * kW4TileBytes,
+            bulk_load_1d(st + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kb) * kW4TileBytes,
                          kW4TileBytes, &full[rp.stage]);
           else
             tma_load_2d(st + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);  // codes: k0 / 2 bytes in
-          tma_load_2d(st + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb0 + i);   // scales of group kb0 + i
+          tma_load_2d(st + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb);   // scales of group kb
         } else {
           mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kWBox + C::kXBox + p.a_rows * 128));
           tma_load_2d(st, &p.tm_w, &full[rp.stage], k0, slice * 128);
@@ -273,7 +287,8 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
 #pragma unroll
         for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
         fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
-        mbar_arrive(&dq_full[rp.stage]);
+        __syncwarp();                 // the warp's rows are written; one arrival per warp
+        if (lane == 0) mbar_arrive(&dq_full[rp.stage]);
         if (tr) { const unsigned long long t1 = sm_clock_ns(); t_work += t1 - t0; t0 = t1; }
         rp.next(S);
       }
@@ -295,13 +310,10 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < kNT; c0 += 16) {
-          uint32_t t[16];
-          tmem_ld16(tl + kNT + c0, t);
-          tmem_wait_ld();
+          float t[16];
+          tmem_ld16f(tl + static_cast<uint32_t>(kNT + c0), t);
 #pragma unroll
-          for (int c = 0; c < 16; c += 4)
-            trow[(c0 + c) / 4] = make_float4(__uint_as_float(t[c]), __uint_as_float(t[c + 1]),
-                                             __uint_as_float(t[c + 2]), __uint_as_float(t[c + 3]));
+          for (int c = 0; c < 16; c += 4) trow[(c0 + c) / 4] = make_float4(t[c], t[c + 1], t[c + 2], t[c + 3]);
         }
       } else {
 #pragma unroll
@@ -314,13 +326,10 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < kNT; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(tl + c0, v);
-          tmem_wait_ld();
+          float v[16];
+          tmem_ld16f(tl + static_cast<uint32_t>(c0), v);
 #pragma unroll
-          for (int c = 0; c < 16; c += 4)
-            drow[(c0 + c) / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                             __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+          for (int c = 0; c < 16; c += 4) drow[(c0 + c) / 4] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
         }
       } else {
 #pragma unroll
