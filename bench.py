@@ -437,29 +437,59 @@ def main():
     F = step_flops(M, d_in, d_out, r, act)
     value = job_throughput(F, args.steps, world, tot_ms) / 1e12
 
-    # e2e: the same step through the C ABI from pinned HOST buffers, copies included
-    out_host = {"Y": torch.empty_like(Y, device="cpu").pin_memory(),
-                "dX": torch.empty_like(dX, device="cpu").pin_memory(),
-                "dA": torch.empty_like(dA, device="cpu").pin_memory(),
-                "dB": torch.empty_like(dB, device="cpu").pin_memory()}
+    # e2e: the same step through the C ABI from pinned HOST buffers, copies
+    # included: every step copies its inputs host -> device and its results
+    # device -> host.  Two buffer sets and one copy stream per direction let
+    # step i+1's input copy and step i-1's result copy run while step i
+    # computes (PCIe is full duplex), as a training loop feeding the layer
+    # would arrange them.
+    bufs = [dict(t=t, Y=Y, dX=dX, dA=dA, dB=dB),
+            dict(t={k: torch.empty_like(v) for k, v in t.items()}, Y=torch.empty_like(Y),
+                 dX=torch.empty_like(dX), dA=torch.empty_like(dA), dB=torch.empty_like(dB))]
+    for k in bufs[1]["t"]:
+        if k not in host:                 # inputs that are not copied per step (none in the bf16 path)
+            bufs[1]["t"][k].copy_(t[k])
+    out_host = [{k: torch.empty_like(bufs[0][k], device="cpu").pin_memory() for k in ("Y", "dX", "dA", "dB")}
+                for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host[0].values())
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
     ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     ee0.record(stream)
-    for _ in range(args.e2e_steps):
-        for k, v in host.items():
-            t[k].copy_(v, non_blocking=True)
+    s_in.wait_event(ee0)
+    s_out.wait_event(ee0)
+    for i in range(args.e2e_steps):
+        b = i % 2
+        cur = bufs[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(comp_done[b])        # step i-2 no longer reads these inputs
+            for k, v in host.items():
+                cur["t"][k].copy_(v, non_blocking=True)
+            in_ready[b].record(s_in)
+        stream.wait_event(in_ready[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])           # step i-2's results are on the host
+        t, Y, dX, dA, dB = cur["t"], cur["Y"], cur["dX"], cur["dA"], cur["dB"]
         fwd()
         bwd()
-        out_host["Y"].copy_(Y, non_blocking=True)
-        out_host["dX"].copy_(dX, non_blocking=True)
-        out_host["dA"].copy_(dA, non_blocking=True)
-        out_host["dB"].copy_(dB, non_blocking=True)
+        comp_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            for k in ("Y", "dX", "dA", "dB"):
+                out_host[b][k].copy_(cur[k], non_blocking=True)
+            out_done[b].record(s_out)
+    for b in range(min(2, args.e2e_steps)):
+        stream.wait_event(out_done[b])
     ee1.record(stream)
     torch.cuda.synchronize()
+    t, Y, dX, dA, dB = bufs[0]["t"], bufs[0]["Y"], bufs[0]["dX"], bufs[0]["dA"], bufs[0]["dB"]
     e2e_ms = ee0.elapsed_time(ee1)
     e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
     e2e = job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12

@@ -1,6 +1,7 @@
 """Parity of the CUDA path with the fp64 oracle on the same seeded bf16
 inputs (per element |err| <= 1e-2 + 1e-2 |ref| and normwise <= 5e-3 on every
 output tensor).  Sizes span several 128 x 256 tiles and ragged tails."""
+import numpy as np
 import pytest
 
 import seeded_inputs
@@ -105,3 +106,23 @@ def test_empty_batch():
         torch.cuda.synchronize()
         assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
         assert ws.status() == 0
+
+
+def test_zero_B_is_the_plain_layer_bit_for_bit():
+    """B = 0: the adapter block adds exact zeros to the same fp32 accumulator,
+    so Y is bit-identical to the r = 0 layer, and dA = s U^T X with U = 0 is
+    exactly zero."""
+    import lora_linear_fine_b200 as L
+    import torch
+    M, d_in, d_out, r = 256, 512, 264, 16
+    inp = seeded_inputs.make_inputs(M, d_in, d_out, r, "identity", seed=11)
+    inp["B"] = np.zeros_like(inp["B"])
+    t = {k: G.dev(v) for k, v in inp.items()}
+    Y1, T1, _ = L.forward(t["X"], t["W"], t["A"], t["B"], 2.0, "identity")
+    Y0, _, _ = L.forward(t["X"], t["W"], None, None, 0.0, "identity")
+    dX1, dA1, dB1, _, _ = L.backward(t["dY"], t["X"], t["W"], t["A"], t["B"], 2.0, "identity", T_save=T1)
+    dX0, _, _, _, _ = L.backward(t["dY"], t["X"], t["W"], None, None, 0.0, "identity")
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y0)
+    assert torch.equal(dX1, dX0)
+    assert torch.count_nonzero(dA1).item() == 0
