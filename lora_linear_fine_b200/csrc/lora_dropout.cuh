@@ -52,35 +52,56 @@ struct DxDropoutJob {
   const __nv_bfloat16* A;       // [r x d_in]
 };
 
-constexpr int kDxRows = 16, kDxCols = 128, kDxMaxRank = 128;
+constexpr int kDxRows = 64, kDxCols = 128, kDxRowsPerThread = kDxRows / 16;
+
+// Dynamic shared memory of dx_dropout_kernel for rank r: the rows' s'U
+// (fp32, stride r + 1) and the tile's columns of A (bf16).
+inline size_t dx_dropout_smem_bytes(int r) {
+  return (static_cast<size_t>(kDxRows) * (r + 1) * 4 + 15) / 16 * 16 + static_cast<size_t>(r) * kDxCols * 2;
+}
 
 // dX += sum_j m_j * ((s' U_j) A_j) for one or two projections, in place on the
-// bf16 dX.  A block takes a 16-row x 128-column tile: it stages the rows'
-// s'U (hi + lo, fp32) and the tile's columns of A (bf16) in shared memory,
-// then each thread adds to 8 consecutive outputs of one row (16-byte dX and
-// one mask byte per thread; rows are 256 contiguous bytes per 16 threads).
+// bf16 dX.  A block takes a 64-row x 128-column tile: it stages the rows'
+// s'U (hi + lo, fp32) and the tile's columns of A (bf16) in shared memory
+// sized for r.  Each thread owns 8 consecutive columns of 4 rows (16 apart):
+// its four 16-byte dX loads and mask bytes are issued before the staging
+// barrier, so each thread keeps four independent loads in flight (rows are
+// 256 contiguous bytes per 16 threads).
 __global__ void __launch_bounds__(256) dx_dropout_kernel(__nv_bfloat16* __restrict__ dX, int M, int d_in, int r,
                                                          int ld, DxDropoutJob j0, DxDropoutJob j1, int np) {
   grid_dep_wait();
-  __shared__ float sU[kDxRows][kDxMaxRank + 1];
-  __shared__ __align__(16) __nv_bfloat16 sA[kDxMaxRank][kDxCols];
+  extern __shared__ __align__(16) uint8_t dx_smem[];
+  float* sU = reinterpret_cast<float*>(dx_smem);                                   // [kDxRows][r + 1]
+  __nv_bfloat16* sA = reinterpret_cast<__nv_bfloat16*>(
+      dx_smem + (static_cast<size_t>(kDxRows) * (r + 1) * 4 + 15) / 16 * 16);        // [r][kDxCols]
   const int t = threadIdx.x;
-  const int row = t >> 4, cg = t & 15;        // this thread: one row, columns 8 cg .. 8 cg + 7 of the tile
+  const int rg = t >> 4, cg = t & 15;         // rows rg + 16 i, columns 8 cg .. 8 cg + 7 of the tile
   const int tiles_m = (M + kDxRows - 1) / kDxRows, tiles_n = d_in / kDxCols + (d_in % kDxCols ? 1 : 0);
   for (long long tile = blockIdx.x; tile < static_cast<long long>(tiles_m) * tiles_n; tile += gridDim.x) {
     const int m0 = static_cast<int>(tile / tiles_n) * kDxRows;
     const int k0 = static_cast<int>(tile % tiles_n) * kDxCols;
-    const int m = m0 + row, k = k0 + 8 * cg;
-    const bool live = m < M && k < d_in;
-    float acc[8];
-    uint4 cur = make_uint4(0, 0, 0, 0);
-    if (live) cur = *reinterpret_cast<const uint4*>(dX + static_cast<size_t>(m) * d_in + k);
-    {
-      const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w};
+    const int k = k0 + 8 * cg;
+    float acc[kDxRowsPerThread][8];
+    uint4 cur[kDxRowsPerThread];
+    uint32_t mb[kDxRowsPerThread][2];
+#pragma unroll
+    for (int i = 0; i < kDxRowsPerThread; ++i) {
+      const int m = m0 + rg + 16 * i;
+      cur[i] = make_uint4(0, 0, 0, 0);
+      mb[i][0] = mb[i][1] = 0u;
+      if (m < M && k < d_in) {
+        cur[i] = *reinterpret_cast<const uint4*>(dX + static_cast<size_t>(m) * d_in + k);
+        mb[i][0] = j0.mask[static_cast<size_t>(m) * (d_in / 8) + k / 8];
+        if (np > 1) mb[i][1] = j1.mask[static_cast<size_t>(m) * (d_in / 8) + k / 8];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kDxRowsPerThread; ++i) {
+      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        acc[2 * e] = __uint_as_float(w[e] << 16);
-        acc[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        acc[i][2 * e] = __uint_as_float(w[e] << 16);
+        acc[i][2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
       }
     }
     for (int jj = 0; jj < np; ++jj) {
@@ -94,41 +115,54 @@ __global__ void __launch_bounds__(256) dx_dropout_kernel(__nv_bfloat16* __restri
           const size_t at = static_cast<size_t>(c) * ld + mm;
           u = __bfloat162float(J.ut_hi[at]) + __bfloat162float(J.ut_lo[at]);
         }
-        sU[rr][c] = u;
+        sU[rr * (r + 1) + c] = u;
       }
       for (int i = t; i < r * (kDxCols / 8); i += 256) {
         const int c = i / (kDxCols / 8), q = i - c * (kDxCols / 8);
         const int kk = k0 + 8 * q;
         uint4 a = make_uint4(0, 0, 0, 0);
         if (kk < d_in) a = *reinterpret_cast<const uint4*>(J.A + static_cast<size_t>(c) * d_in + kk);
-        *reinterpret_cast<uint4*>(&sA[c][8 * q]) = a;
+        *reinterpret_cast<uint4*>(&sA[c * kDxCols + 8 * q]) = a;
       }
       __syncthreads();
-      if (live) {
-        float add[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int c = 0; c < r; ++c) {
-          const float u = sU[row][c];
-          const uint4 a = *reinterpret_cast<const uint4*>(&sA[c][8 * cg]);
-          const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+      float add[kDxRowsPerThread][8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            add[2 * e] = fmaf(u, __uint_as_float(w[e] << 16), add[2 * e]);
-            add[2 * e + 1] = fmaf(u, __uint_as_float(w[e] & 0xFFFF0000u), add[2 * e + 1]);
-          }
+      for (int i = 0; i < kDxRowsPerThread; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) add[i][e] = 0.0f;
+      for (int c = 0; c < r; ++c) {
+        const uint4 a = *reinterpret_cast<const uint4*>(&sA[c * kDxCols + 8 * cg]);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        float av[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          av[2 * e] = __uint_as_float(w[e] << 16);
+          av[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
         }
-        const uint32_t b = J.mask[static_cast<size_t>(m) * (d_in / 8) + k / 8];
+#pragma unroll
+        for (int i = 0; i < kDxRowsPerThread; ++i) {
+          const float u = sU[(rg + 16 * i) * (r + 1) + c];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) add[i][e] = fmaf(u, av[e], add[i][e]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kDxRowsPerThread; ++i)
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          if ((b >> e) & 1u) acc[e] += add[e];
-      }
+          if (((jj == 0 ? mb[i][0] : mb[i][1]) >> e) & 1u) acc[i][e] += add[i][e];
     }
-    if (live) {
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(dX + static_cast<size_t>(m) * d_in + k) = o;
+#pragma unroll
+    for (int i = 0; i < kDxRowsPerThread; ++i) {
+      const int m = m0 + rg + 16 * i;
+      if (m < M && k < d_in) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[i][0], acc[i][1]);
+        o.y = pack_bf16x2(acc[i][2], acc[i][3]);
+        o.z = pack_bf16x2(acc[i][4], acc[i][5]);
+        o.w = pack_bf16x2(acc[i][6], acc[i][7]);
+        *reinterpret_cast<uint4*>(dX + static_cast<size_t>(m) * d_in + k) = o;
+      }
     }
   }
 }

@@ -1229,7 +1229,12 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     }
     const long long tiles = ceil_div(M, kDxRows) * ceil_div(d->d_in, kDxCols);
     const int grid = static_cast<int>(tiles < static_cast<long long>(dev.sms) * 8 ? tiles : dev.sms * 8);
-    launch_k(dx_dropout_kernel, dim3(grid), dim3(256), 0, st, false, static_cast<__nv_bfloat16*>(dX), M,
+    const size_t smem = dx_dropout_smem_bytes(r);   // <= 65 KB at r = 128
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(dx_dropout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return cuda_error("cudaFuncSetAttribute(dx_dropout)");
+    launch_k(dx_dropout_kernel, dim3(grid), dim3(256), smem, st, false, static_cast<__nv_bfloat16*>(dX), M,
              static_cast<int>(d->d_in), r, M8, jb[0], jb[1], np);
     LORA_TRY(check_launch("dx_dropout_kernel"));
   }
