@@ -11,7 +11,9 @@
 #include <cstring>
 #include <atomic>
 #include <vector>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "lora_mma.cuh"
 #include "lora_rank.cuh"
@@ -695,7 +697,19 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
   q.act = d->act;
   q.a_rows = static_cast<int>(align_up(static_cast<size_t>(r), 16));
   const int slices = static_cast<int>(ceil_div(d->d_out, 128));
-  q.splits = small_m_splits(nt, w4, d->d_in, d->d_out);
+  {
+    // The cluster size depends only on the device and the shape: ask the
+    // occupancy API once per (device, nt, w4, d_in, d_out) and keep the answer.
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int, int64_t, int64_t>, int> cache;
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    const auto key = std::make_tuple(dev_id, nt, static_cast<int>(w4), d->d_in, d->d_out);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it == cache.end()) it = cache.emplace(key, small_m_splits(nt, w4, d->d_in, d->d_out)).first;
+    q.splits = it->second;
+  }
   q.kb_per = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), q.splits));
   const int grid = slices * q.splits;
   LORA_LOG("small_m M=%d nt=%d w4=%d slices=%d splits=%d kb_per=%d grid=%d", (int)M, nt, (int)w4, slices,

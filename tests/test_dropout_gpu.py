@@ -98,3 +98,37 @@ def test_dropout_all_kept_matches_plain_layer():
                                      None, 0.0, p(Y2), p(T2), None, ws.buf.data_ptr(), ws.nbytes, sh) == 0
     torch.cuda.synchronize()
     assert torch.equal(Y1, Y2) and torch.equal(T1, T2)
+
+
+def test_dropout_and_w4_empty_batch():
+    """M = 0 through the dropout and 4-bit entry points: no token tensors (NULL),
+    no launches but the zero-fill of the adapter gradients."""
+    import lora_linear_fine_b200 as L
+    import torch
+    d_in, d_out, r = 256, 264, 16
+    inp = seeded_inputs.make_inputs(8, d_in, d_out, r, "identity", seed=12)
+    t = {k: G.dev(v) for k, v in inp.items()}
+    Wq, Ws = seeded_inputs.draw_w4("W", d_out, d_in, 12)
+    Wq_d, Ws_d = torch.from_numpy(Wq).cuda(), G.dev(Ws)
+    sh = torch.cuda.current_stream().cuda_stream
+    desc = L.make_desc(0, d_in, d_out, r, 1.0, "identity")
+    p = lambda x: x.data_ptr()
+    ws = L.Workspace(max(L.lora_linear_workspace_size_dropout(desc, 1), L.lora_linear_workspace_size_w4(desc, 1)))
+    for call in ("dropout", "w4"):
+        dA = torch.full((r, d_in), float("nan"), device="cuda")
+        dB = torch.full((d_out, r), float("nan"), device="cuda")
+        if call == "dropout":
+            assert L.lora_linear_fwd_dropout(desc, None, p(t["W"]), p(t["A"]), p(t["B"]), None, None, None, None, None,
+                                             0.1, None, None, None, ws.buf.data_ptr(), ws.nbytes, sh) == 0
+            assert L.lora_linear_bwd_dropout(desc, None, None, p(t["W"]), p(t["A"]), p(t["B"]), None, None, None,
+                                             None, None, 0.1, None, None, None, p(dA), p(dB), None, None,
+                                             ws.buf.data_ptr(), ws.nbytes, sh) == 0
+        else:
+            assert L.lora_linear_fwd_w4(desc, None, p(Wq_d), p(Ws_d), p(t["A"]), p(t["B"]), None, None, None, None,
+                                        None, None, None, ws.buf.data_ptr(), ws.nbytes, sh) == 0
+            assert L.lora_linear_bwd_w4(desc, None, None, p(Wq_d), p(Ws_d), p(t["A"]), p(t["B"]), None, None, None,
+                                        None, None, None, None, p(dA), p(dB), None, None, ws.buf.data_ptr(),
+                                        ws.nbytes, sh) == 0
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0, call
+    assert ws.status() == 0
