@@ -52,19 +52,21 @@ def forward(X, W, A, B, s, act="identity"):
     return {"T": T, "Z": Z, "Y": Y}
 
 
-def backward(dY, X, W, A, B, s, act="identity", fwd=None, single_u_rounding=False):
+def backward(dY, X, W, A, B, s, act="identity", fwd=None, single_u_rounding=False, dz_type="f16"):
     """dX (bf16), dA, dB (fp32) as the backward kernels produce them.
 
     single_u_rounding=True replaces the hi/lo split of s*U by one bf16
-    rounding: the cheaper design that the split exists to avoid."""
+    rounding, and dz_type="bf16" stores dZ (with an activation) as bf16
+    instead of fp16: the cheaper designs that the kernels' choices avoid."""
     fwd = fwd or forward(X, W, A, B, s, act)
     if act == "identity":
         dZ_parts = [dY]                            # bf16 already
         Wop = W
     else:
         dZ = to_f32(dY * oracle.silu_grad(fwd["Z"]))
-        dZ_parts = list(hi_lo(dZ, to_f16))         # fp16 hi + lo
-        Wop = to_f16(W)                            # exact fp16 copy of the bf16 weight
+        rnd16 = to_f16 if dz_type == "f16" else to_bf16
+        dZ_parts = list(hi_lo(dZ, rnd16))          # fp16 (or bf16) hi + lo
+        Wop = to_f16(W) if dz_type == "f16" else W  # exact fp16 copy of the bf16 weight
     Bop = B if act == "identity" else to_f16(B)
     U = to_f32(sum(p @ Bop for p in dZ_parts))      # rank pass over dZ (both parts)
     sU16 = to_bf16(s * U)                          # dX's adapter K-block operand

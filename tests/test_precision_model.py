@@ -38,3 +38,19 @@ def test_single_bf16_rounding_of_U_breaks_dA():
     assert oracle.compare(good["dA"], ref["dA"])["ok"]
     res = oracle.compare(bad["dA"], ref["dA"])
     assert res["nfail"] > 0, res
+
+
+def test_bf16_dZ_breaks_dX_over_a_long_reduction():
+    """With an activation, dX = dZ W sums over d_out.  Over a long sum (here
+    d_out = 28672, the SwiGLU pair's K) one bf16 rounding of dZ leaves
+    per-element errors past the bound; the fp16 dZ the kernels use does not."""
+    Ml, d_in, d_out, r = 128, 256, 28672, 16
+    inp = seeded_inputs.make_inputs(Ml, d_in, d_out, r, "silu", seed=33)
+    g = {k: oracle.bf16_to_f64(v) for k, v in inp.items()}
+    ref = oracle.lora_backward(g["dY"], g["X"], g["W"], g["A"], g["B"], S, "silu")
+    fwd = PM.forward(g["X"], g["W"], g["A"], g["B"], S, "silu")
+    good = PM.backward(g["dY"], g["X"], g["W"], g["A"], g["B"], S, "silu", fwd=fwd)
+    bad = PM.backward(g["dY"], g["X"], g["W"], g["A"], g["B"], S, "silu", fwd=fwd, dz_type="bf16")
+    assert oracle.compare(good["dX"], ref["dX"])["ok"]
+    res = oracle.compare(bad["dX"], ref["dX"])
+    assert res["nfail"] > 0, res
