@@ -35,6 +35,7 @@ import numpy as np  # noqa: E402
 import seeded_inputs  # noqa: E402
 
 METRIC = "LoRA-linear fwd+bwd TFLOP/s (M=16384, 4096², r=8) & % of B200 roofline"
+METRIC_QKV = "LoRA attention-input block (RMSNorm + q/k/v + rotary) fwd+bwd TFLOP/s & % of B200 roofline"
 UNIT = "TFLOP/s"
 
 
@@ -114,9 +115,48 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
+def is_qkv(cfg):
+    return "d_kv" in cfg
+
+
+def cfg_step_flops(cfg, M):
+    """FLOPs of one step of a workload at M tokens: the attention-input block
+    counts its three projections (the norm and the rotation are O(M d) and not
+    counted)."""
+    if is_qkv(cfg):
+        return sum(step_flops(M, cfg["d_in"], n, cfg["r"]) for n in qkv_douts(cfg))
+    return step_flops(M, cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"])
+
+
+def qkv_douts(cfg):
+    return (cfg["d_out"], cfg["d_kv"], cfg["d_kv"])
+
+
+def qkv_inputs(cfg, M, seed):
+    """Host inputs of the attention-input block: bf16 bits (X, g, W_j, A_j, B_j,
+    dY_j for j = q, k, v), int32 positions (whole sequences), fp32 tables."""
+    d, r = cfg["d_in"], cfg["r"]
+    out = {"X": seeded_inputs.draw("X", (M, d), seed, d), "g": seeded_inputs.draw_norm_weight(d, seed)}
+    for j, d_out in enumerate(qkv_douts(cfg)):
+        inp = seeded_inputs.make_inputs(M, d, d_out, r, "identity", seed=seed * 10 + j)
+        for k in ("W", "A", "B", "dY"):
+            out[f"{k}{j}"] = inp[k]
+    out["pos"] = seeded_inputs.sequence_positions(M, cfg["seq_len"])
+    out["cos"], out["sin"] = seeded_inputs.rotary_tables(cfg["seq_len"], cfg["head_dim"])
+    return out
+
+
 def oracle_sample_run(cfg, rows, inp_f64):
     import oracle
     g = inp_f64
+    if is_qkv(cfg):
+        from oracle import norm_rope_oracle
+        projs = [{k: g[f"{k}{j}"] for k in ("W", "A", "B")} for j in range(3)]
+        t0 = time.perf_counter()
+        norm_rope_oracle.qkv_backward([g[f"dY{j}"][:rows] for j in range(3)], g["X"][:rows], g["g"],
+                                      float(np.float32(cfg["eps"])), projs, cfg["alpha"] / cfg["r"],
+                                      [True, True, False], g["pos"][:rows], g["cos"], g["sin"], cfg["head_dim"])
+        return time.perf_counter() - t0
     X = g["X"][:rows]
     dY = g["dY"][:rows]
     t0 = time.perf_counter()
@@ -138,9 +178,8 @@ def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
     """Time the oracle on growing row samples until ~budget_s of CPU work."""
     import oracle
     M, d_in, d_out, r = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"]
-    rows_cap = max_rows or M
-    inp = seeded_inputs.make_inputs(min(M, rows_cap), d_in, d_out, r, cfg["act"], seed=0)
-    g = {k: oracle.bf16_to_f64(v) for k, v in inp.items()}
+    rows_cap = max_rows or (4096 if is_qkv(cfg) else M)
+    g = oracle_inputs(cfg, min(M, rows_cap))
     rows = 16
     spent = 0.0
     best = None
@@ -157,20 +196,30 @@ def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
     while sum(times) < budget_s / 2 and len(times) < 20:
         times.append(oracle_sample_run(cfg, rows, g))
     dt = statistics.mean(times)
-    val = step_flops(rows, d_in, d_out, r, cfg["act"]) / dt / 1e12
+    val = cfg_step_flops(cfg, rows) / dt / 1e12
+    what = (f"the norm, q/k/v projections ({d_in}->{'/'.join(map(str, qkv_douts(cfg)))}) and rotation"
+            if is_qkv(cfg) else f"({d_in}->{d_out}, r={r})")
     return {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 numpy oracle fwd+bwd on the first {rows} of {M} tokens "
-                      f"({d_in}->{d_out}, r={r}); mean of {len(times)} runs of {dt:.2f} s; "
-                      f"FLOPs by the same formula"}
+                      f"{what}, r={r}; mean of {len(times)} runs of {dt:.2f} s; FLOPs by the same formula"}
+
+
+def oracle_inputs(cfg, M):
+    """The workload's inputs for the oracle (float64; positions and tables as given)."""
+    import oracle
+    if is_qkv(cfg):
+        raw = qkv_inputs(cfg, M, 0)
+        return {k: (v.astype(np.float64) if k in ("cos", "sin") else v if k == "pos" else oracle.bf16_to_f64(v))
+                for k, v in raw.items()}
+    inp = seeded_inputs.make_inputs(M, cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"], seed=0)
+    return {k: oracle.bf16_to_f64(v) for k, v in inp.items()}
 
 
 def run_reference(args, cfg, world, rank):
     if rank != 0:
         return
     steps, warm = args.steps, args.warmup
-    import oracle
-    inp = seeded_inputs.make_inputs(min(cfg["M"], 4096), cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"], seed=0)
-    g = {k: oracle.bf16_to_f64(v) for k, v in inp.items()}
+    g = oracle_inputs(cfg, min(cfg["M"], 4096))
     # rows per step: sized so the whole warm-up + timed run stays within a few minutes
     rows = 64
     while rows < 4096:
@@ -183,10 +232,11 @@ def run_reference(args, cfg, world, rank):
     tot = 0.0
     for _ in range(steps):
         tot += oracle_sample_run(cfg, rows, g)
-    val = step_flops(rows, cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]) * steps / tot / 1e12
-    sample = (f"fp64 numpy oracle fwd+bwd on {rows} of {cfg['M']} tokens per step "
-              f"({cfg['d_in']}->{cfg['d_out']}, r={cfg['r']})")
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": steps,
+    val = cfg_step_flops(cfg, rows) * steps / tot / 1e12
+    shape = (f"norm + {cfg['d_in']}->{'/'.join(map(str, qkv_douts(cfg)))} + rotary" if is_qkv(cfg)
+             else f"{cfg['d_in']}->{cfg['d_out']}")
+    sample = f"fp64 numpy oracle fwd+bwd on {rows} of {cfg['M']} tokens per step ({shape}, r={cfg['r']})"
+    line = {"impl": "reference", "metric": METRIC_QKV if is_qkv(cfg) else METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": steps,
             "warmup": warm, "ms_per_step": tot / steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.config, "M": cfg["M"], "d_in": cfg["d_in"], "d_out": cfg["d_out"],
@@ -277,6 +327,166 @@ def run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def run_qkv(args, cfg, L, world, rank, local, dist):
+    """The attention-input block: RMSNorm, the q, k, v projections (q and k
+    rotated in the GEMM epilogue), their backward, and the norm's backward over
+    the three input gradients; every step through the C ABI."""
+    import torch
+    M, d, r, hd, eps = cfg["M"], cfg["d_in"], cfg["r"], cfg["head_dim"], cfg["eps"]
+    douts = qkv_douts(cfg)
+    s = cfg["alpha"] / r
+    n_pos = cfg["seq_len"]
+    raw = qkv_inputs(cfg, M, rank)
+    host = {k: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+                else torch.from_numpy(v)).pin_memory() for k, v in raw.items()}
+    t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    p = lambda x: None if x is None else x.data_ptr()  # noqa: E731
+    descs = [L.make_desc(M, d, n, r, s, "identity") for n in douts]
+    ws = L.Workspace(max(max(L.lora_linear_workspace_size_rope(x, 1), L.lora_linear_workspace_size(x, 1))
+                         for x in descs))
+    bf, f32 = torch.bfloat16, torch.float32
+    Xn = torch.empty((M, d), dtype=bf, device="cuda")
+    rstd = torch.empty(M, dtype=f32, device="cuda")
+    o = {"Y": [torch.empty((M, n), dtype=bf, device="cuda") for n in douts],
+         "T": [torch.empty((M, r), dtype=f32, device="cuda") for _ in douts],
+         "dXn": [torch.empty((M, d), dtype=bf, device="cuda") for _ in douts],
+         "dA": [torch.empty((r, d), dtype=f32, device="cuda") for _ in douts],
+         "dB": [torch.empty((n, r), dtype=f32, device="cuda") for n in douts],
+         "dX": torch.empty((M, d), dtype=bf, device="cuda")}
+    rope = L.make_rope_desc(p(t["pos"]), p(t["cos"]), p(t["sin"]), n_pos, hd)
+    wsp = (ws.buf.data_ptr(), ws.nbytes, sh)
+
+    def fwd(norm_done=None):
+        assert L.lora_linear_rmsnorm_fwd(p(t["X"]), p(t["g"]), M, d, eps, p(Xn), p(rstd), sh) == 0
+        if norm_done is not None:
+            norm_done.record(stream)
+        for j in range(3):
+            w = (p(t[f"W{j}"]), p(t[f"A{j}"]), p(t[f"B{j}"]))
+            if j < 2:
+                st = L.lora_linear_fwd_rope(descs[j], rope, p(Xn), *w, p(o["Y"][j]), p(o["T"][j]), *wsp)
+            else:
+                st = L.lora_linear_fwd(descs[j], p(Xn), *w, None, None, None, p(o["Y"][j]), p(o["T"][j]), None, *wsp)
+            assert st == 0, L.status_string(st)
+
+    def bwd():
+        for j in range(3):
+            w = (p(t[f"W{j}"]), p(t[f"A{j}"]), p(t[f"B{j}"]))
+            g = (p(o["T"][j]), p(o["dXn"][j]), p(o["dA"][j]), p(o["dB"][j]))
+            if j < 2:
+                st = L.lora_linear_bwd_rope(descs[j], rope, p(t[f"dY{j}"]), p(Xn), *w, *g, *wsp)
+            else:
+                st = L.lora_linear_bwd(descs[j], p(t[f"dY{j}"]), p(Xn), *w, None, None, None, g[0], None, *g[1:],
+                                       None, None, *wsp)
+            assert st == 0, L.status_string(st)
+        assert L.lora_linear_rmsnorm_bwd(p(t["X"]), p(t["g"]), p(rstd), [x.data_ptr() for x in o["dXn"]], M, d,
+                                         p(o["dX"]), sh) == 0
+
+    if args.calls > 0:
+        for _ in range(args.calls):
+            fwd()
+            if not args.fwd_only:
+                bwd()
+        torch.cuda.synchronize()
+        print("ok", flush=True)
+        return
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    launches0 = L.lora_linear_launch_count()
+    L.lora_linear_timing_enable(1)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        fwd(norm_done=ev[i][1])
+        ev[i][2].record(stream)
+        bwd()
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    launches = L.lora_linear_launch_count() - launches0
+    _, gemm_fwd_ms, gemm_fwd_n, gemm_bwd_ms, gemm_bwd_n = L.lora_linear_timing_read()
+    L.lora_linear_timing_enable(0)
+    tot_ms = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in ev), dist, "cuda")
+    norm_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    F = cfg_step_flops(cfg, M)
+    value = job_throughput(F, args.steps, world, tot_ms) / 1e12
+
+    # e2e: every step copies its inputs from pinned host memory and its results
+    # (Y_q, Y_k, Y_v, dX, dA_j, dB_j) back, serialised with the compute
+    out_host = {k: torch.empty_like(v, device="cpu").pin_memory()
+                for k, v in [(f"Y{j}", o["Y"][j]) for j in range(3)] + [(f"dA{j}", o["dA"][j]) for j in range(3)]
+                + [(f"dB{j}", o["dB"][j]) for j in range(3)] + [("dX", o["dX"])]}
+    dev_out = {**{f"Y{j}": o["Y"][j] for j in range(3)}, **{f"dA{j}": o["dA"][j] for j in range(3)},
+               **{f"dB{j}": o["dB"][j] for j in range(3)}, "dX": o["dX"]}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ee0.record(stream)
+    for _ in range(args.e2e_steps):
+        for k, v in host.items():
+            t[k].copy_(v, non_blocking=True)
+        fwd()
+        bwd()
+        for k, v in dev_out.items():
+            out_host[k].copy_(v, non_blocking=True)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ee0.elapsed_time(ee1), dist, "cuda")
+    e2e = job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12
+
+    peaks = read_peaks()
+    f_fwd = sum(2.0 * M * d * n + 2.0 * M * r * n for n in douts)     # the three forward GEMMs per step
+    f_bwd = sum(2.0 * M * d * n + 2.0 * M * r * d for n in douts)     # the three dX GEMMs per step
+    ach_f = f_fwd * args.steps / (gemm_fwd_ms * 1e-3) / 1e12 if gemm_fwd_n else None
+    ach_b = f_bwd * args.steps / (gemm_bwd_ms * 1e-3) / 1e12 if gemm_bwd_n else None
+    pk = peaks["bf16_tflops"]
+    norm_bytes = 2.0 * M * d * 2 + 4.0 * M + 2.0 * d                # read X, write x_n, rstd, g
+    norm_gbs = norm_bytes / (norm_ms * 1e-3) / 1e9
+    roof = {"kernel": "lora_mma_kernel (forward GEMMs of q, k, v; q and k with the rotary epilogue)",
+            "bound": "tensor", "achieved": round(ach_f, 2) if ach_f else None, "peak": pk, "unit": "TFLOP/s",
+            "frac": round(ach_f / pk, 4) if ach_f else None,
+            "peak_kind": f"bf16 burst, {peaks['source']} (sustained {peaks['bf16_tflops_sustained']})",
+            "flop_per_step": f_fwd, "launches_per_step": 3, "traffic": None,
+            "backward_gemms": {"achieved": round(ach_b, 2) if ach_b else None,
+                               "frac": round(ach_b / pk, 4) if ach_b else None, "flop_per_step": f_bwd},
+            "rmsnorm_fwd": {"bound": "hbm", "achieved": round(norm_gbs, 1), "peak": peaks["hbm_gbs"],
+                            "unit": "GB/s", "frac": round(norm_gbs / peaks["hbm_gbs"], 4),
+                            "bytes_per_launch": norm_bytes, "ms_per_launch": round(norm_ms, 5)},
+            "step_frac": round(value / world / pk, 4)}
+    line = {"metric": METRIC_QKV, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.config, "M": M, "d_in": d, "d_out_q": douts[0], "d_out_kv": douts[1],
+                       "r": r, "alpha": cfg["alpha"], "head_dim": hd, "seq_len": n_pos, "eps": eps,
+                       "parallelism": f"replicas x{world}", "l2": "flushed before each timed step (512 MiB write)"},
+            "roofline": roof, "gpu_launches": int(launches),
+            "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h), "copies": "serialised with the compute"},
+            "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -318,6 +528,9 @@ def main():
 
     import lora_linear_fine_b200 as L
 
+    if is_qkv(cfg):
+        run_qkv(args, cfg, L, world, rank, local, dist)
+        return
     M, d_in, d_out, r, act = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]
     s = cfg["alpha"] / r if r else 0.0
     inp = seeded_inputs.make_inputs(M, d_in, d_out, r, act, seed=rank)

@@ -109,7 +109,10 @@ lora_status_t lora_linear_workspace_init(void* workspace, size_t workspace_bytes
 /* Synchronise `stream`, copy the workspace status word to *out_status and
  * return LORA_OK if it is zero, LORA_ERR_DEVICE_STATUS otherwise.  Bits:
  *   0x1  a bounded wait on an mbarrier gave up (the kernel stopped its work)
- *   0x2  a device-side argument check failed
+ *   0x2  a device-side argument check failed (e.g. a rotary position outside
+ *        its table)
+ *   0x4  a value converted to fp16 was outside fp16's finite range (backward
+ *        with an activation, or of a rotated projection)
  * Intended for tests and debugging. */
 lora_status_t lora_linear_device_status(const void* workspace, void* stream, uint32_t* out_status);
 
@@ -323,6 +326,88 @@ lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* desc, const void* 
                                       const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
                                       float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes,
                                       void* stream);
+
+/* ------------------------------------------------------------------------
+ * RMSNorm prologue and rotary-embedding epilogue of the attention-input
+ * (q, k, v) projections.  "Swift-All一文详解：如何用Liger-Kernel提升训练效率",
+ * 2.2 (1) "RMSNorm + Rotary Embedding + Attention QKV 融合", gives the
+ * sequence they fuse: normalise x, project it to q, k and v, rotate q and k.
+ * The sketch of that kernel in "企业官网建设流程全解析" (the page's extracted
+ * title), section "融合内核是如何工作的", fixes the norm (reciprocal square
+ * root of the mean square plus 1e-6, times the norm's weight) and takes the
+ * rotation's cosine and sine tables as arguments, indexed by the feature's
+ * offset within half a head.  Readings taken:
+ *   x_n = bf16(x * rstd * g),   rstd = 1 / sqrt(mean_j x_j^2 + eps)  per token,
+ *     rounded once (to nearest even) from the exact value; g is frozen;
+ *   q = rot(Z_q), k = rot(Z_k) with Z the identity LoRA linear of x_n; rot
+ *     turns feature i of each head of head_dim features with feature
+ *     i + head_dim/2 by the table angle at the token's position:
+ *       (a, b) -> (a cos - b sin, b cos + a sin);
+ *   the backward is the chain rule (the projections' input gradients add up
+ *     before the norm's backward).
+ * A block step is: lora_linear_rmsnorm_fwd; lora_linear_fwd_rope for q and k
+ * and lora_linear_fwd for v, all on x_n; then lora_linear_bwd_rope /
+ * lora_linear_bwd, whose dX outputs are the dx_n inputs of
+ * lora_linear_rmsnorm_bwd.
+ * ------------------------------------------------------------------------ */
+
+/* Rotary tables.  pos: device int32 [M], each token's position (0 <= pos <
+ * n_pos; a position outside sets status bit 0x2 and leaves that token
+ * unrotated), 4-byte aligned.  cos, sin: device fp32 [n_pos x head_dim/2],
+ * 16-byte aligned; row p holds the angle's cosine / sine for pair i of a head
+ * at position p.  head_dim: 64 or 128 (LORA_ERR_UNSUPPORTED otherwise), and a
+ * divisor of d_out (LORA_ERR_INVALID_ARG).  All caller-owned, only read.
+ * pos, cos, sin may be NULL when M == 0. */
+typedef struct lora_rope_desc {
+    const int32_t* pos;
+    const float* cos;
+    const float* sin;
+    int64_t n_pos;
+    int32_t head_dim;
+} lora_rope_desc;
+
+/* x_n = bf16(x * rstd * g) and rstd = 1 / sqrt(mean(x^2) + eps), per token.
+ * X [M x d] bf16, g [d] bf16 (device, read); Xn [M x d] bf16 and rstd [M] fp32
+ * (device, written; rstd is the backward's input).  The sum of squares, rstd
+ * and the product are taken in fp64, and x_n is their correctly rounded bf16
+ * value.  d % 8 == 0 and X, g, Xn 16-byte aligned, rstd 4-byte aligned
+ * (LORA_ERR_ALIGNMENT); eps >= 0 and finite, M >= 0, d > 0
+ * (LORA_ERR_INVALID_ARG).  M == 0 launches nothing.  Asynchronous on `stream`. */
+lora_status_t lora_linear_rmsnorm_fwd(const void* X, const void* g, int64_t M, int64_t d, float eps, void* Xn,
+                                      float* rstd, void* stream);
+
+/* dX [M x d] bf16 = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd,
+ * where dx_n is the sum (in fp32) of the n_grads bf16 gradients dXn[0..n-1]
+ * [M x d] (the dX outputs of the projections that read x_n).  dXn is a host
+ * array of n_grads device pointers, 1 <= n_grads <= 4.  rstd: the forward's
+ * output.  Alignment and errors as lora_linear_rmsnorm_fwd.  g gets no
+ * gradient (frozen). */
+lora_status_t lora_linear_rmsnorm_bwd(const void* X, const void* g, const float* rstd, const void* const* dXn,
+                                      int n_grads, int64_t M, int64_t d, void* dX, void* stream);
+
+/* Workspace bytes for lora_linear_fwd_rope (0) / lora_linear_bwd_rope (1); 0
+ * for an invalid desc or an activation other than identity. */
+size_t lora_linear_workspace_size_rope(const lora_linear_desc* desc, int for_backward);
+
+/* Forward of a rotated projection: Y = rot(X W^T + s (X A^T) B^T), bf16, the
+ * rotation applied to the fp32 accumulator in the GEMM's epilogue (one
+ * rounding).  desc->act must be LORA_ACT_IDENTITY (LORA_ERR_UNSUPPORTED).
+ * X is x_n.  Other arguments as lora_linear_fwd (no SwiGLU twins, no Z_save);
+ * T_save holds T = X A^T for the backward.  The few-token kernel is not used.
+ * workspace >= lora_linear_workspace_size_rope(desc, 0). */
+lora_status_t lora_linear_fwd_rope(const lora_linear_desc* desc, const lora_rope_desc* rope, const void* X,
+                                   const void* W, const void* A, const void* B, void* Y, float* T_save,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of a rotated projection: dZ = rot^T(dY) (emitted as fp16 hi + lo;
+ * a value outside fp16's range sets status bit 0x4), then the layer's
+ * backward on dZ: dX = dZ W + s U A, dA = s U^T X, dB = s dZ^T T, U = dZ B.
+ * Arguments as lora_linear_bwd without the SwiGLU twins and Z_save.
+ * workspace >= lora_linear_workspace_size_rope(desc, 1). */
+lora_status_t lora_linear_bwd_rope(const lora_linear_desc* desc, const lora_rope_desc* rope, const void* dY,
+                                   const void* X, const void* W, const void* A, const void* B, const float* T_save,
+                                   void* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 #ifdef __cplusplus
 }

@@ -31,12 +31,20 @@ EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_li
             "lora_linear_timing_read", "lora_linear_selftest_wait_timeout",
             "lora_linear_workspace_size_w4", "lora_linear_dequant_w4", "lora_linear_fwd_w4", "lora_linear_bwd_w4",
             "lora_linear_workspace_size_dropout", "lora_linear_fwd_dropout", "lora_linear_bwd_dropout",
-            "lora_linear_w4_tiled_bytes", "lora_linear_w4_tile", "lora_linear_fwd_w4_tiled")
+            "lora_linear_w4_tiled_bytes", "lora_linear_w4_tile", "lora_linear_fwd_w4_tiled",
+            "lora_linear_rmsnorm_fwd", "lora_linear_rmsnorm_bwd", "lora_linear_workspace_size_rope",
+            "lora_linear_fwd_rope", "lora_linear_bwd_rope")
 
 
 class LoraLinearDesc(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("d_in", ctypes.c_int64), ("d_out", ctypes.c_int64),
                 ("r", ctypes.c_int64), ("s", ctypes.c_float), ("act", ctypes.c_int32)]
+
+
+class LoraRopeDesc(ctypes.Structure):
+    """Rotary tables: pos (int32 [M]), cos / sin (fp32 [n_pos x head_dim/2]) device pointers."""
+    _fields_ = [("pos", ctypes.c_void_p), ("cos", ctypes.c_void_p), ("sin", ctypes.c_void_p),
+                ("n_pos", ctypes.c_int64), ("head_dim", ctypes.c_int32)]
 
 
 class LoraError(RuntimeError):
@@ -98,6 +106,17 @@ def _load():
     lib.lora_linear_fwd_dropout.restype = i32
     lib.lora_linear_bwd_dropout.argtypes = [dp] + [vp] * 10 + [f32] + [vp] * 7 + [vp, sz, vp]
     lib.lora_linear_bwd_dropout.restype = i32
+    rp = ctypes.POINTER(LoraRopeDesc)
+    lib.lora_linear_rmsnorm_fwd.argtypes = [vp, vp, i64, i64, f32, vp, vp, vp]
+    lib.lora_linear_rmsnorm_fwd.restype = i32
+    lib.lora_linear_rmsnorm_bwd.argtypes = [vp, vp, vp, ctypes.POINTER(vp), i32, i64, i64, vp, vp]
+    lib.lora_linear_rmsnorm_bwd.restype = i32
+    lib.lora_linear_workspace_size_rope.argtypes = [dp, i32]
+    lib.lora_linear_workspace_size_rope.restype = sz
+    lib.lora_linear_fwd_rope.argtypes = [dp, rp] + [vp] * 6 + [vp, sz, vp]
+    lib.lora_linear_fwd_rope.restype = i32
+    lib.lora_linear_bwd_rope.argtypes = [dp, rp] + [vp] * 9 + [vp, sz, vp]
+    lib.lora_linear_bwd_rope.restype = i32
     return lib
 
 
@@ -198,6 +217,36 @@ def lora_linear_bwd_w4(desc, dY, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, T_sa
                        dB_up, workspace, workspace_bytes, stream) -> int:
     return int(_lib.lora_linear_bwd_w4(ctypes.byref(desc), dY, X, Wq, Ws, A, B, Wq_up, Ws_up, A_up, B_up, T_save,
                                        Z_save, dX, dA, dB, dA_up, dB_up, workspace, workspace_bytes, stream))
+
+
+# RMSNorm prologue and rotary-embedding epilogue of the attention-input projections
+def make_rope_desc(pos, cos, sin, n_pos, head_dim) -> LoraRopeDesc:
+    return LoraRopeDesc(pos, cos, sin, int(n_pos), int(head_dim))
+
+
+def lora_linear_rmsnorm_fwd(X, g, M, d, eps, Xn, rstd, stream) -> int:
+    return int(_lib.lora_linear_rmsnorm_fwd(X, g, int(M), int(d), float(eps), Xn, rstd, stream))
+
+
+def lora_linear_rmsnorm_bwd(X, g, rstd, dXn, M, d, dX, stream) -> int:
+    """dXn: a sequence of device pointers (the projections' dX), summed."""
+    n = len(dXn)
+    arr = (ctypes.c_void_p * max(n, 1))(*dXn)
+    return int(_lib.lora_linear_rmsnorm_bwd(X, g, rstd, arr, n, int(M), int(d), dX, stream))
+
+
+def lora_linear_workspace_size_rope(desc: LoraLinearDesc, for_backward: int) -> int:
+    return int(_lib.lora_linear_workspace_size_rope(ctypes.byref(desc), int(for_backward)))
+
+
+def lora_linear_fwd_rope(desc, rope, X, W, A, B, Y, T_save, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_fwd_rope(ctypes.byref(desc), ctypes.byref(rope), X, W, A, B, Y, T_save, workspace,
+                                         workspace_bytes, stream))
+
+
+def lora_linear_bwd_rope(desc, rope, dY, X, W, A, B, T_save, dX, dA, dB, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_bwd_rope(ctypes.byref(desc), ctypes.byref(rope), dY, X, W, A, B, T_save, dX, dA,
+                                         dB, workspace, workspace_bytes, stream))
 
 
 def lora_linear_timing_enable(enable: int) -> int:

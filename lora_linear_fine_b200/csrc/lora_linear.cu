@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -21,6 +22,7 @@
 #include "lora_small_m.cuh"
 #include "lora_w4.cuh"
 #include "lora_dropout.cuh"
+#include "lora_norm_rope.cuh"
 
 namespace {
 
@@ -189,11 +191,14 @@ int rank_splits(int64_t tiles, int64_t nkb) {
   return static_cast<int>(s);
 }
 
-Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = true) {
+// grad_f16: the backward's dZ comes as fp16 hi + lo even without an activation
+// (the rotated projections: dZ = R^T dY), so it takes the activation's operand
+// path: fp16 W copy, no K-major W^T, no fused U + dB pass.
+Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = true, bool grad_f16 = false) {
   Plan P;
   P.np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
   P.RP = rank_pad(d->r);
-  P.act_f16 = backward && d->act != LORA_ACT_IDENTITY;
+  P.act_f16 = backward && (d->act != LORA_ACT_IDENTITY || grad_f16);
   P.M8 = static_cast<int64_t>(align_up(static_cast<size_t>(d->M > 0 ? d->M : 1), 8));
   const int64_t M = d->M, r = d->r;
   const int64_t tiles_m = ceil_div(M > 0 ? M : 1, 128);
@@ -228,7 +233,7 @@ Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = tr
   }
   // The W^T copy pays for itself when the dX GEMM is long against one pass
   // over W: many tokens (measured: M = 16384 gains, M = 8192 does not).
-  P.kmajor = d->act == LORA_ACT_IDENTITY && M >= kKMajorMinTokens;
+  P.kmajor = !P.act_f16 && M >= kKMajorMinTokens;
   for (int j = 0; j < P.np; ++j) {
     if (P.kmajor || P.act_f16) P.wt[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
     if (P.act_f16) {
@@ -250,7 +255,7 @@ Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = tr
     // U and dB from one read of dY: identity, and r <= 64 (at r = 128 the
     // two accumulators and both B operands leave too little tensor and
     // shared memory)
-    P.dual = d->act == LORA_ACT_IDENTITY && P.RP <= 64;
+    P.dual = !P.act_f16 && P.RP <= 64;
     if (P.dual) {
       P.sp_dual = rank2d_split(static_cast<int>(tiles_m), static_cast<int>(tiles_b), P.RP, true, true,
                                rank2d_max_rb(P.RP), kTargetCtas);
@@ -838,6 +843,37 @@ lora_status_t mask_inputs(const lora_linear_desc* d, const void* X, const void* 
   return LORA_OK;
 }
 
+// Rotary tables of the attention-input projections: checks shared by the
+// forward and the backward.
+lora_status_t check_rope(const lora_linear_desc* d, const lora_rope_desc* rd, RopeTables* out) {
+  if (rd == nullptr) return LORA_ERR_INVALID_ARG;
+  if (d->act != LORA_ACT_IDENTITY) return LORA_ERR_UNSUPPORTED;
+  if (rd->head_dim != 64 && rd->head_dim != 128) return LORA_ERR_UNSUPPORTED;
+  if (d->d_out % rd->head_dim != 0) return LORA_ERR_INVALID_ARG;
+  if (rd->n_pos < 1 || rd->n_pos > (int64_t(1) << 31)) return LORA_ERR_INVALID_ARG;
+  if (d->M > 0 && (rd->pos == nullptr || rd->cos == nullptr || rd->sin == nullptr)) return LORA_ERR_INVALID_ARG;
+  if ((rd->cos != nullptr && !aligned16(rd->cos)) || (rd->sin != nullptr && !aligned16(rd->sin)) ||
+      (reinterpret_cast<uintptr_t>(rd->pos) & 3u) != 0)
+    return LORA_ERR_ALIGNMENT;
+  out->pos = rd->pos;
+  out->cos = rd->cos;
+  out->sin = rd->sin;
+  out->n_pos = rd->n_pos;
+  out->half = rd->head_dim / 2;
+  return LORA_OK;
+}
+
+lora_status_t check_arch(DevInfo* dev) {
+  LORA_TRY(device_info(dev));
+  return (dev->major == 10 && dev->minor == 0) ? LORA_OK : LORA_ERR_ARCH;
+}
+
+int norm_grid(int64_t M, const DevInfo& dev) {
+  const int64_t blocks = ceil_div(M, kNormWarps);
+  const int64_t cap = static_cast<int64_t>(dev.sms) * 8;   // 8 CTAs of 8 warps fill an SM
+  return static_cast<int>(blocks < cap ? blocks : cap);
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -942,7 +978,7 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
 static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const void* W, const void* A,
                               const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
                               float* T_save, float* Z_save, void* workspace, size_t workspace_bytes, void* stream,
-                              const void* const Xl[2], bool allow_small_m) {
+                              const void* const Xl[2], bool allow_small_m, const RopeTables* rope = nullptr) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
   // with M == 0 the per-token tensors are empty and may be NULL
@@ -1007,6 +1043,12 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   set_raster(p, pair, 2.0 * M * d->d_in, 2.0 * np * d->d_out * d->d_in);
   timing_begin(0, st);
   lora_status_t rs;
+  if (rope != nullptr) {
+    p.rope = *rope;
+    rs = launch_mma_any<false, 1, kMEpiRope>(pair, p, dev.sms, st);
+    timing_end(0, st);
+    return rs;
+  }
   switch (d->act) {
     case LORA_ACT_IDENTITY: rs = launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st); break;
     case LORA_ACT_SILU: rs = launch_mma_any<false, 1, kMEpiSilu>(pair, p, dev.sms, st); break;
@@ -1030,7 +1072,8 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
                               const void* B, const void* W_up, const void* A_up, const void* B_up,
                               const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
                               float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream,
-                              const void* const Xl[2], const uint8_t* const masks[2]) {
+                              const void* const Xl[2], const uint8_t* const masks[2],
+                              const RopeTables* rope = nullptr) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
   // with M == 0 the per-token tensors are empty and may be NULL
@@ -1043,7 +1086,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
   const void* ptrs[] = {dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
-  const Plan P = make_plan(d, true);
+  const Plan P = make_plan(d, true, true, rope != nullptr);
   DevInfo dev;
   LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1090,7 +1133,11 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
   if (f16) {
     const long long n = static_cast<long long>(M) * d->d_out;
     const int grid = grid_for(n / 8, 256, dev.sms);
-    if (swiglu)
+    if (rope != nullptr)
+      launch_k(rope_bwd_kernel, dim3(grid_for(n / 16, 256, dev.sms)), dim3(256), 0, st, false,
+               static_cast<const __nv_bfloat16*>(dY), *rope, static_cast<long long>(M), static_cast<int>(d->d_out),
+               static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])), status);
+    else if (swiglu)
       launch_k(act_bwd_kernel<true>, dim3(grid), dim3(256), 0, st, false, static_cast<const __nv_bfloat16*>(dY),
                static_cast<const float*>(Z_save), static_cast<const float*>(Z_save + static_cast<size_t>(M) * d->d_out),
                static_cast<long long>(n), static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])),
@@ -1100,7 +1147,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
                static_cast<const float*>(Z_save), static_cast<const float*>(nullptr), static_cast<long long>(n),
                static_cast<__half*>(at(P.dz_hi[0])), static_cast<__half*>(at(P.dz_lo[0])),
                static_cast<__half*>(nullptr), static_cast<__half*>(nullptr), status);
-    LORA_TRY(check_launch("act_bwd_kernel"));
+    LORA_TRY(check_launch(rope != nullptr ? "rope_bwd_kernel" : "act_bwd_kernel"));
     const long long nw = static_cast<long long>(d->d_out) * d->d_in;
     for (int j = 0; j < np; ++j) {
       dZ[j] = at(P.dz_hi[j]);
@@ -1524,6 +1571,83 @@ lora_status_t lora_linear_fwd_w4_tiled(const lora_linear_desc* d, const void* X,
   if (d->M == 0) return LORA_OK;
   return run_small_m_fwd(d, P.sm_nt, X, nullptr, nullptr, Ws, A, B, Y, T_save, Z_save,
                          reinterpret_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream), Wt);
+}
+
+// RMSNorm prologue and rotary-embedding epilogue (lora_norm_rope.cuh)
+lora_status_t lora_linear_rmsnorm_fwd(const void* X, const void* g, int64_t M, int64_t d, float eps, void* Xn,
+                                      float* rstd, void* stream) {
+  if (M < 0 || d <= 0 || !std::isfinite(eps) || eps < 0.0f || g == nullptr) return LORA_ERR_INVALID_ARG;
+  if (M > 0 && (X == nullptr || Xn == nullptr || rstd == nullptr)) return LORA_ERR_INVALID_ARG;
+  if (d % 8 != 0 || !aligned16(g) || (X != nullptr && !aligned16(X)) || (Xn != nullptr && !aligned16(Xn)) ||
+      (reinterpret_cast<uintptr_t>(rstd) & 3u) != 0)
+    return LORA_ERR_ALIGNMENT;
+  if (d > (int64_t(1) << 24) || M > (int64_t(1) << 40)) return LORA_ERR_UNSUPPORTED;
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
+  if (M == 0) return LORA_OK;
+  launch_k(rmsnorm_fwd_kernel, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
+           false, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(g),
+           static_cast<long long>(M), static_cast<int>(d), static_cast<double>(eps), static_cast<__nv_bfloat16*>(Xn),
+           rstd);
+  return check_launch("rmsnorm_fwd_kernel");
+}
+
+lora_status_t lora_linear_rmsnorm_bwd(const void* X, const void* g, const float* rstd, const void* const* dXn,
+                                      int n_grads, int64_t M, int64_t d, void* dX, void* stream) {
+  if (M < 0 || d <= 0 || n_grads < 1 || n_grads > kNormMaxGrads || g == nullptr) return LORA_ERR_INVALID_ARG;
+  if (M > 0 && (X == nullptr || rstd == nullptr || dX == nullptr || dXn == nullptr)) return LORA_ERR_INVALID_ARG;
+  NormGrads gr{};
+  gr.n = n_grads;
+  if (M > 0) {
+    for (int j = 0; j < n_grads; ++j) {
+      if (dXn[j] == nullptr) return LORA_ERR_INVALID_ARG;
+      if (!aligned16(dXn[j])) return LORA_ERR_ALIGNMENT;
+      gr.p[j] = static_cast<const __nv_bfloat16*>(dXn[j]);
+    }
+  }
+  if (d % 8 != 0 || !aligned16(g) || (X != nullptr && !aligned16(X)) || (dX != nullptr && !aligned16(dX)) ||
+      (reinterpret_cast<uintptr_t>(rstd) & 3u) != 0)
+    return LORA_ERR_ALIGNMENT;
+  if (d > (int64_t(1) << 24) || M > (int64_t(1) << 40)) return LORA_ERR_UNSUPPORTED;
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
+  if (M == 0) return LORA_OK;
+  launch_k(rmsnorm_bwd_kernel, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
+           false, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(g), rstd, gr,
+           static_cast<long long>(M), static_cast<int>(d), static_cast<__nv_bfloat16*>(dX));
+  return check_launch("rmsnorm_bwd_kernel");
+}
+
+size_t lora_linear_workspace_size_rope(const lora_linear_desc* desc, int for_backward) {
+  if (check_desc(desc) != LORA_OK || desc->act != LORA_ACT_IDENTITY) return 0;
+  const size_t fwd = make_plan(desc, false, false).total;
+  if (!for_backward) return fwd;
+  const size_t bwd = make_plan(desc, true, true, true).total;
+  return bwd > fwd ? bwd : fwd;
+}
+
+lora_status_t lora_linear_fwd_rope(const lora_linear_desc* d, const lora_rope_desc* rope, const void* X,
+                                   const void* W, const void* A, const void* B, void* Y, float* T_save,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_desc(d));
+  RopeTables t;
+  LORA_TRY(check_rope(d, rope, &t));
+  const void* Xl[2] = {X, X};
+  return fwd_core(d, X, W, A, B, nullptr, nullptr, nullptr, Y, T_save, nullptr, workspace, workspace_bytes, stream,
+                  Xl, false, &t);
+}
+
+lora_status_t lora_linear_bwd_rope(const lora_linear_desc* d, const lora_rope_desc* rope, const void* dY,
+                                   const void* X, const void* W, const void* A, const void* B, const float* T_save,
+                                   void* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  LORA_TRY(check_desc(d));
+  RopeTables t;
+  LORA_TRY(check_rope(d, rope, &t));
+  const void* Xl[2] = {X, X};
+  const uint8_t* masks[2] = {nullptr, nullptr};
+  return bwd_core(d, dY, X, W, A, B, nullptr, nullptr, nullptr, T_save, nullptr, dX, dA, dB, nullptr, nullptr,
+                  workspace, workspace_bytes, stream, Xl, masks, &t);
 }
 
 }  // extern "C"

@@ -36,13 +36,16 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "lora_norm_rope.cuh"
 
 namespace lora {
 
 constexpr int kMmaThreads = 320;
 
 // kEpi values
-enum MmaEpi : int { kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4 };
+// kMEpiRope: identity, then the rotary embedding of each token's heads on the
+// fp32 accumulator (lora_norm_rope.cuh) before the bf16 store.
+enum MmaEpi : int { kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5 };
 
 struct MmaParams {
   CUtensorMap tm_a[2];    // M-side operand per pair      fwd: X            bwd: dZ_j
@@ -59,6 +62,7 @@ struct MmaParams {
   int group_along_n;      // 0: groups of `group` M tiles sweep all N tiles (the N-side operand stays in L2)
                           // 1: groups of `group` N tiles sweep all M tiles (the M-side operand stays in L2)
   int b_mn;               // backward: N-side operands read MN-major (W [K x N], A [r x N]) instead of K-major copies
+  RopeTables rope;        // kMEpiRope: positions and cos / sin tables (half = 32 or 64)
 };
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
@@ -455,6 +459,46 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               const int col = col0 + 64 * hv + 8 * j;
               if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
             });
+          }
+        }
+      } else if constexpr (kEpi == kMEpiRope) {
+        // Identity plus the rotary embedding.  This thread's 128 columns start
+        // at a multiple of 128, so they hold whole heads (half = 64: one head,
+        // pairs (c, c + 64); half = 32: two heads, pairs (c, c + 32) in each).
+        // Two passes, each loading 32 columns at c0 and 32 at c0 + half, so
+        // that a pass holds 32 whole pairs: u[e], u[e + 32].
+        const int half = p.rope.half;
+        const int pr = row_ok ? __ldg(p.rope.pos + row) : 0;
+        const bool turn = row_ok && pr >= 0 && pr < p.rope.n_pos;
+        if (row_ok && !turn && p.status) atomicOr(p.status, kStatusBadArgument);   // left unturned
+        const size_t trow = static_cast<size_t>(turn ? pr : 0) * half;
+        const int col0 = nt * 256 + h * 128;
+        const size_t base = static_cast<size_t>(row) * p.N + col0;
+#pragma unroll
+        for (int hv = 0; hv < 2; ++hv) {
+          const int c0 = half == 64 ? 32 * hv : 64 * hv;
+          uint32_t u[64];
+          __syncwarp();   // lanes past M skipped the stores of the previous pass; tcgen05.ld is .sync.aligned
+          tmem_ld32(tl + h * 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld32(tl + h * 128 + c0 + half, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_wait_ld();
+          if (hv == 1) release_acc();
+          if (!row_ok) continue;
+          const int toff = c0 % half;
+          if (turn) rope_rotate32(u, p.rope.cos + trow + toff, p.rope.sin + trow + toff);
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const int cc = c0 + part * half;
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              const uint32_t* w = &u[32 * part + j];
+              uint4 pk;
+              pk.x = pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+              pk.y = pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+              pk.z = pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5]));
+              pk.w = pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7]));
+              if (col0 + cc + j < p.N) st_global_v4_hint(p.out + base + cc + j, pk, pol_out);
+            }
           }
         }
       } else {

@@ -20,6 +20,13 @@ are used, every tensor is drawn here):
 * dropout masks on the adapter input: each element of X kept with probability
   1 - p, packed eight per byte (bit j of byte b, least significant first, is
   element 8 b + j): uint8 tokens x d_in/8.
+* attention-input block (RMSNorm, then the q, k, v projections, q and k
+  rotated): the norm's weight g ~ U(0.5, 1.5) (bf16, d_in); each projection j
+  has its own W, A, B, dY drawn as above from the seed (seed, j); token
+  positions int32, uniform in [0, n_pos) for the tests, or m mod seq_len (a
+  batch of whole sequences) for the benchmark; rotary tables float32
+  [n_pos x head_dim/2] holding the cosine and sine of p * 10000^(-2i/head_dim),
+  the RoFormer frequencies, as a model precomputes them.
 
 Each tensor has its own stream: numpy's PCG64 seeded with (seed, tensor id).
 Values are drawn in float64, rounded to float32 (round-to-nearest-even) and
@@ -36,6 +43,7 @@ _TENSOR_IDS = {
     "W_up": 6, "A_up": 7, "B_up": 8,
     "Wq": 9, "Ws": 10, "Wq_up": 11, "Ws_up": 12,
     "mask": 13, "mask_up": 14,
+    "g": 15, "pos": 16,
 }
 
 ACTS = ("identity", "silu", "swiglu")
@@ -54,6 +62,10 @@ CONFIGS = {
     "small_m_w4": dict(M=16, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity", weight="w4"),
     # q_proj with dropout p = 0.1 on the adapter input (the mask is drawn here)
     "q_proj_dropout": dict(M=16384, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity", dropout=0.1),
+    # RMSNorm -> q (4096), k (1024), v (1024) LoRA projections, q and k rotated
+    # (32 query and 8 key/value heads of 128); 4 sequences of 4096 tokens
+    "qkv_rmsnorm_rope": dict(M=16384, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity",
+                             d_kv=1024, head_dim=128, seq_len=4096, eps=1e-6),
 }
 
 
@@ -111,6 +123,28 @@ def draw_mask(name: str, M: int, d_in: int, p_drop: float, seed: int) -> np.ndar
     """A packed dropout mask of the recipe above; ``name`` is "mask" or "mask_up"."""
     keep = _rng(seed, name).random((M, d_in)) >= p_drop
     return np.packbits(keep.astype(np.uint8), axis=1, bitorder="little")
+
+
+def draw_norm_weight(d: int, seed: int) -> np.ndarray:
+    """The RMSNorm weight g [d] of the recipe above, as bf16 bits."""
+    return f64_to_bf16_bits(_rng(seed, "g").uniform(0.5, 1.5, size=d))
+
+
+def draw_positions(M: int, n_pos: int, seed: int) -> np.ndarray:
+    """Token positions uniform in [0, n_pos), int32 [M]."""
+    return _rng(seed, "pos").integers(0, n_pos, size=M).astype(np.int32)
+
+
+def sequence_positions(M: int, seq_len: int) -> np.ndarray:
+    """Positions of a batch of whole sequences: m mod seq_len, int32 [M]."""
+    return (np.arange(M, dtype=np.int64) % seq_len).astype(np.int32)
+
+
+def rotary_tables(n_pos: int, head_dim: int, base: float = 10000.0):
+    """(cos, sin) float32 [n_pos x head_dim/2] of the angles p * base^(-2i/head_dim)."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    ang = np.arange(n_pos, dtype=np.float64)[:, None] * base ** (-2.0 * i / head_dim)[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
 
 
 def make_inputs(M: int, d_in: int, d_out: int, r: int, act: str = "identity",

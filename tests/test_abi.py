@@ -152,3 +152,46 @@ def test_dropout_and_w4_argument_checks(lib):
     assert w4(few, Ws=24) == 2                                     # 16-byte alignment
     assert lib.lora_linear_dequant_w4(16, 16, 256, 100, 16, None) == 2
     assert lib.lora_linear_dequant_w4(None, 16, 256, 128, 16, None) == 1
+
+
+def test_norm_and_rope_argument_checks(lib):
+    """RMSNorm prologue and rotary epilogue: every bad argument is caught on the
+    host (these checks come before any device query)."""
+    # RMSNorm forward: d % 8, eps, required pointers, alignment
+    assert lib.lora_linear_rmsnorm_fwd(16, 16, 4, 100, 1e-6, 16, 16, None) == 2
+    assert lib.lora_linear_rmsnorm_fwd(16, 16, 4, 64, -1.0, 16, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_fwd(16, 16, 4, 64, float("nan"), 16, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_fwd(16, None, 4, 64, 1e-6, 16, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_fwd(None, 16, 4, 64, 1e-6, 16, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_fwd(24, 16, 4, 64, 1e-6, 16, 16, None) == 2
+    assert lib.lora_linear_rmsnorm_fwd(16, 16, 4, 64, 1e-6, 16, 18, None) == 2      # rstd 4-byte aligned
+    # RMSNorm backward: 1..4 gradients, each present and aligned
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [], 4, 64, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [16] * 5, 4, 64, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [16, None], 4, 64, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [16, 24], 4, 64, 16, None) == 2
+    # rotary projections: identity only, head_dim 64 / 128 dividing d_out, tables aligned
+    d = lib.make_desc(256, 512, 256, 8, 2.0, "identity")
+    f = lib.lora_linear_workspace_size_rope(d, 0)
+    b = lib.lora_linear_workspace_size_rope(d, 1)
+    assert b >= f > 0
+    assert b >= 2 * 256 * 256 * 2 + 256 * 512 * 2       # fp16 dZ hi + lo and the fp16 copy of W
+    assert lib.lora_linear_workspace_size_rope(lib.make_desc(256, 512, 256, 8, 2.0, "silu"), 0) == 0
+
+    def fwd(desc=d, pos=16, cos=16, sin=16, n_pos=32, head_dim=128):
+        rope = lib.make_rope_desc(pos, cos, sin, n_pos, head_dim)
+        return lib.lora_linear_fwd_rope(desc, rope, 16, 16, 16, 16, 16, None, 16, 1 << 30, None)
+
+    assert fwd(head_dim=96) == 3
+    assert fwd(head_dim=32) == 3
+    assert fwd(desc=lib.make_desc(256, 512, 192, 8, 2.0, "identity")) == 1   # 192 % 128
+    assert fwd(desc=lib.make_desc(256, 512, 256, 8, 2.0, "silu")) == 3
+    assert fwd(n_pos=0) == 1
+    assert fwd(pos=None) == 1
+    assert fwd(cos=24) == 2
+    assert fwd(pos=18) == 2
+    raw = lib._LazyLib._h
+    assert raw.lora_linear_fwd_rope(ctypes.byref(d), None, 16, 16, 16, 16, 16, None, 16, 1 << 30, None) == 1
+    rope = lib.make_rope_desc(16, 16, 16, 32, 64)
+    assert lib.lora_linear_bwd_rope(lib.make_desc(256, 512, 256, 8, 2.0, "swiglu"), rope, 16, 16, 16, 16, 16, None,
+                                    16, 16, 16, 16, 1 << 30, None) == 3
