@@ -351,7 +351,7 @@ def run_qkv(args, cfg, L, world, rank, local, dist):
     rstd = torch.empty(M, dtype=f32, device="cuda")
     o = {"Y": [torch.empty((M, n), dtype=bf, device="cuda") for n in douts],
          "T": [torch.empty((M, r), dtype=f32, device="cuda") for _ in douts],
-         "dXn": [torch.empty((M, d), dtype=bf, device="cuda") for _ in douts],
+         "dXn": torch.empty((M, d), dtype=f32, device="cuda"),     # fp32 sum of the three input gradients
          "dA": [torch.empty((r, d), dtype=f32, device="cuda") for _ in douts],
          "dB": [torch.empty((n, r), dtype=f32, device="cuda") for n in douts],
          "dX": torch.empty((M, d), dtype=bf, device="cuda")}
@@ -371,17 +371,13 @@ def run_qkv(args, cfg, L, world, rank, local, dist):
             assert st == 0, L.status_string(st)
 
     def bwd():
+        # q writes the fp32 dx_n, k and v add to it (v is not rotated)
         for j in range(3):
             w = (p(t[f"W{j}"]), p(t[f"A{j}"]), p(t[f"B{j}"]))
-            g = (p(o["T"][j]), p(o["dXn"][j]), p(o["dA"][j]), p(o["dB"][j]))
-            if j < 2:
-                st = L.lora_linear_bwd_rope(descs[j], rope, p(t[f"dY{j}"]), p(Xn), *w, *g, *wsp)
-            else:
-                st = L.lora_linear_bwd(descs[j], p(t[f"dY{j}"]), p(Xn), *w, None, None, None, g[0], None, *g[1:],
-                                       None, None, *wsp)
+            st = L.lora_linear_bwd_rope(descs[j], rope if j < 2 else None, p(t[f"dY{j}"]), p(Xn), *w, p(o["T"][j]),
+                                        p(o["dXn"]), 1 if j else 0, p(o["dA"][j]), p(o["dB"][j]), *wsp)
             assert st == 0, L.status_string(st)
-        assert L.lora_linear_rmsnorm_bwd(p(t["X"]), p(t["g"]), p(rstd), [x.data_ptr() for x in o["dXn"]], M, d,
-                                         p(o["dX"]), sh) == 0
+        assert L.lora_linear_rmsnorm_bwd(p(t["X"]), p(t["g"]), p(rstd), p(o["dXn"]), M, d, p(o["dX"]), sh) == 0
 
     if args.calls > 0:
         for _ in range(args.calls):

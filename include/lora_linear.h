@@ -346,9 +346,11 @@ lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* desc, const void* 
  *   the backward is the chain rule (the projections' input gradients add up
  *     before the norm's backward).
  * A block step is: lora_linear_rmsnorm_fwd; lora_linear_fwd_rope for q and k
- * and lora_linear_fwd for v, all on x_n; then lora_linear_bwd_rope /
- * lora_linear_bwd, whose dX outputs are the dx_n inputs of
- * lora_linear_rmsnorm_bwd.
+ * and lora_linear_fwd for v, all on x_n; then lora_linear_bwd_rope for q, k
+ * and v (rope NULL for v), the first writing and the others adding their
+ * input gradients into one fp32 dx_n; then lora_linear_rmsnorm_bwd on dx_n.
+ * dx_n is fp32 because three bf16 roundings before the sum would exceed the
+ * tolerance on the near-zero entries of dx.
  * ------------------------------------------------------------------------ */
 
 /* Rotary tables.  pos: device int32 [M], each token's position (0 <= pos <
@@ -376,14 +378,13 @@ typedef struct lora_rope_desc {
 lora_status_t lora_linear_rmsnorm_fwd(const void* X, const void* g, int64_t M, int64_t d, float eps, void* Xn,
                                       float* rstd, void* stream);
 
-/* dX [M x d] bf16 = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd,
- * where dx_n is the sum (in fp32) of the n_grads bf16 gradients dXn[0..n-1]
- * [M x d] (the dX outputs of the projections that read x_n).  dXn is a host
- * array of n_grads device pointers, 1 <= n_grads <= 4.  rstd: the forward's
- * output.  Alignment and errors as lora_linear_rmsnorm_fwd.  g gets no
- * gradient (frozen). */
-lora_status_t lora_linear_rmsnorm_bwd(const void* X, const void* g, const float* rstd, const void* const* dXn,
-                                      int n_grads, int64_t M, int64_t d, void* dX, void* stream);
+/* dX [M x d] bf16 = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd.
+ * dXn: device fp32 [M x d], the summed input gradients of the projections
+ * that read x_n (lora_linear_bwd_rope's output), 16-byte aligned.  rstd: the
+ * forward's output.  Alignment and errors as lora_linear_rmsnorm_fwd.  g gets
+ * no gradient (frozen). */
+lora_status_t lora_linear_rmsnorm_bwd(const void* X, const void* g, const float* rstd, const float* dXn, int64_t M,
+                                      int64_t d, void* dX, void* stream);
 
 /* Workspace bytes for lora_linear_fwd_rope (0) / lora_linear_bwd_rope (1); 0
  * for an invalid desc or an activation other than identity. */
@@ -399,15 +400,19 @@ lora_status_t lora_linear_fwd_rope(const lora_linear_desc* desc, const lora_rope
                                    const void* W, const void* A, const void* B, void* Y, float* T_save,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
-/* Backward of a rotated projection: dZ = rot^T(dY) (emitted as fp16 hi + lo;
- * a value outside fp16's range sets status bit 0x4), then the layer's
- * backward on dZ: dX = dZ W + s U A, dA = s U^T X, dB = s dZ^T T, U = dZ B.
- * Arguments as lora_linear_bwd without the SwiGLU twins and Z_save.
+/* Backward of a projection of the block.  rope != NULL (q, k): dZ =
+ * rot^T(dY), emitted as fp16 hi + lo (a value outside fp16's range sets status
+ * bit 0x4); rope == NULL (v): dZ = dY.  Then the layer's backward on dZ:
+ * dx = dZ W + s U A, dA = s U^T X, dB = s dZ^T T, U = dZ B.
+ * dXn: device fp32 [M x d_in], 16-byte aligned: accumulate == 0 writes dx
+ * into it, accumulate == 1 adds dx to it (other values: LORA_ERR_INVALID_ARG).
+ * Other arguments as lora_linear_bwd without the SwiGLU twins and Z_save;
+ * desc->act must be LORA_ACT_IDENTITY (LORA_ERR_UNSUPPORTED).
  * workspace >= lora_linear_workspace_size_rope(desc, 1). */
 lora_status_t lora_linear_bwd_rope(const lora_linear_desc* desc, const lora_rope_desc* rope, const void* dY,
                                    const void* X, const void* W, const void* A, const void* B, const float* T_save,
-                                   void* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
-                                   void* stream);
+                                   float* dXn, int accumulate, float* dA, float* dB, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

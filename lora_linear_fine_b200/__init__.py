@@ -109,13 +109,13 @@ def _load():
     rp = ctypes.POINTER(LoraRopeDesc)
     lib.lora_linear_rmsnorm_fwd.argtypes = [vp, vp, i64, i64, f32, vp, vp, vp]
     lib.lora_linear_rmsnorm_fwd.restype = i32
-    lib.lora_linear_rmsnorm_bwd.argtypes = [vp, vp, vp, ctypes.POINTER(vp), i32, i64, i64, vp, vp]
+    lib.lora_linear_rmsnorm_bwd.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp]
     lib.lora_linear_rmsnorm_bwd.restype = i32
     lib.lora_linear_workspace_size_rope.argtypes = [dp, i32]
     lib.lora_linear_workspace_size_rope.restype = sz
     lib.lora_linear_fwd_rope.argtypes = [dp, rp] + [vp] * 6 + [vp, sz, vp]
     lib.lora_linear_fwd_rope.restype = i32
-    lib.lora_linear_bwd_rope.argtypes = [dp, rp] + [vp] * 9 + [vp, sz, vp]
+    lib.lora_linear_bwd_rope.argtypes = [dp, rp] + [vp] * 7 + [i32, vp, vp] + [vp, sz, vp]
     lib.lora_linear_bwd_rope.restype = i32
     return lib
 
@@ -229,10 +229,8 @@ def lora_linear_rmsnorm_fwd(X, g, M, d, eps, Xn, rstd, stream) -> int:
 
 
 def lora_linear_rmsnorm_bwd(X, g, rstd, dXn, M, d, dX, stream) -> int:
-    """dXn: a sequence of device pointers (the projections' dX), summed."""
-    n = len(dXn)
-    arr = (ctypes.c_void_p * max(n, 1))(*dXn)
-    return int(_lib.lora_linear_rmsnorm_bwd(X, g, rstd, arr, n, int(M), int(d), dX, stream))
+    """dXn: the fp32 sum of the projections' input gradients."""
+    return int(_lib.lora_linear_rmsnorm_bwd(X, g, rstd, dXn, int(M), int(d), dX, stream))
 
 
 def lora_linear_workspace_size_rope(desc: LoraLinearDesc, for_backward: int) -> int:
@@ -244,9 +242,13 @@ def lora_linear_fwd_rope(desc, rope, X, W, A, B, Y, T_save, workspace, workspace
                                          workspace_bytes, stream))
 
 
-def lora_linear_bwd_rope(desc, rope, dY, X, W, A, B, T_save, dX, dA, dB, workspace, workspace_bytes, stream) -> int:
-    return int(_lib.lora_linear_bwd_rope(ctypes.byref(desc), ctypes.byref(rope), dY, X, W, A, B, T_save, dX, dA,
-                                         dB, workspace, workspace_bytes, stream))
+def lora_linear_bwd_rope(desc, rope, dY, X, W, A, B, T_save, dXn, accumulate, dA, dB, workspace, workspace_bytes,
+                         stream) -> int:
+    """rope None: the projection is not rotated (v).  dXn: fp32, written
+    (accumulate 0) or added to (accumulate 1)."""
+    return int(_lib.lora_linear_bwd_rope(ctypes.byref(desc), None if rope is None else ctypes.byref(rope), dY, X, W,
+                                         A, B, T_save, dXn, int(accumulate), dA, dB, workspace, workspace_bytes,
+                                         stream))
 
 
 def lora_linear_timing_enable(enable: int) -> int:

@@ -1073,17 +1073,19 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
                               const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
                               float* dA_up, float* dB_up, void* workspace, size_t workspace_bytes, void* stream,
                               const void* const Xl[2], const uint8_t* const masks[2],
-                              const RopeTables* rope = nullptr) {
+                              const RopeTables* rope = nullptr, float* dXf = nullptr, int dXf_acc = 0) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
-  // with M == 0 the per-token tensors are empty and may be NULL
-  if (W == nullptr || (d->M > 0 && (dY == nullptr || X == nullptr || dX == nullptr))) return LORA_ERR_INVALID_ARG;
+  // with M == 0 the per-token tensors are empty and may be NULL; dXf (fp32,
+  // written or added to) replaces the bf16 dX
+  if (W == nullptr || (d->M > 0 && (dY == nullptr || X == nullptr || (dX == nullptr && dXf == nullptr))))
+    return LORA_ERR_INVALID_ARG;
   if (d->r > 0 && (A == nullptr || B == nullptr || dA == nullptr || dB == nullptr)) return LORA_ERR_INVALID_ARG;
   if (swiglu && (W_up == nullptr || (d->r > 0 && (A_up == nullptr || B_up == nullptr || dA_up == nullptr ||
                                                   dB_up == nullptr))))
     return LORA_ERR_INVALID_ARG;
   if (d->act != LORA_ACT_IDENTITY && d->M > 0 && Z_save == nullptr) return LORA_ERR_INVALID_ARG;
-  const void* ptrs[] = {dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up};
+  const void* ptrs[] = {dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, dXf};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
   const Plan P = make_plan(d, true, true, rope != nullptr);
@@ -1260,6 +1262,8 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     p.K = static_cast<int>(d->d_out);
     p.lora_ksteps = masks[0] != nullptr ? 0 : (r + 15) / 16;   // dropout: the LoRA term comes after
     p.out = static_cast<__nv_bfloat16*>(dX);
+    p.out_f32 = dXf;
+    p.out_acc = dXf_acc;
     p.z_save = nullptr;
     p.status = status;
     p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
@@ -1592,28 +1596,19 @@ lora_status_t lora_linear_rmsnorm_fwd(const void* X, const void* g, int64_t M, i
   return check_launch("rmsnorm_fwd_kernel");
 }
 
-lora_status_t lora_linear_rmsnorm_bwd(const void* X, const void* g, const float* rstd, const void* const* dXn,
-                                      int n_grads, int64_t M, int64_t d, void* dX, void* stream) {
-  if (M < 0 || d <= 0 || n_grads < 1 || n_grads > kNormMaxGrads || g == nullptr) return LORA_ERR_INVALID_ARG;
+lora_status_t lora_linear_rmsnorm_bwd(const void* X, const void* g, const float* rstd, const float* dXn, int64_t M,
+                                      int64_t d, void* dX, void* stream) {
+  if (M < 0 || d <= 0 || g == nullptr) return LORA_ERR_INVALID_ARG;
   if (M > 0 && (X == nullptr || rstd == nullptr || dX == nullptr || dXn == nullptr)) return LORA_ERR_INVALID_ARG;
-  NormGrads gr{};
-  gr.n = n_grads;
-  if (M > 0) {
-    for (int j = 0; j < n_grads; ++j) {
-      if (dXn[j] == nullptr) return LORA_ERR_INVALID_ARG;
-      if (!aligned16(dXn[j])) return LORA_ERR_ALIGNMENT;
-      gr.p[j] = static_cast<const __nv_bfloat16*>(dXn[j]);
-    }
-  }
   if (d % 8 != 0 || !aligned16(g) || (X != nullptr && !aligned16(X)) || (dX != nullptr && !aligned16(dX)) ||
-      (reinterpret_cast<uintptr_t>(rstd) & 3u) != 0)
+      (dXn != nullptr && !aligned16(dXn)) || (reinterpret_cast<uintptr_t>(rstd) & 3u) != 0)
     return LORA_ERR_ALIGNMENT;
   if (d > (int64_t(1) << 24) || M > (int64_t(1) << 40)) return LORA_ERR_UNSUPPORTED;
   DevInfo dev;
   LORA_TRY(check_arch(&dev));
   if (M == 0) return LORA_OK;
   launch_k(rmsnorm_bwd_kernel, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
-           false, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(g), rstd, gr,
+           false, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(g), rstd, dXn,
            static_cast<long long>(M), static_cast<int>(d), static_cast<__nv_bfloat16*>(dX));
   return check_launch("rmsnorm_bwd_kernel");
 }
@@ -1622,7 +1617,9 @@ size_t lora_linear_workspace_size_rope(const lora_linear_desc* desc, int for_bac
   if (check_desc(desc) != LORA_OK || desc->act != LORA_ACT_IDENTITY) return 0;
   const size_t fwd = make_plan(desc, false, false).total;
   if (!for_backward) return fwd;
-  const size_t bwd = make_plan(desc, true, true, true).total;
+  const size_t rot = make_plan(desc, true, true, true).total;    // rotated: fp16 dZ operands
+  const size_t plain = make_plan(desc, true).total;              // not rotated (rope == NULL)
+  const size_t bwd = rot > plain ? rot : plain;
   return bwd > fwd ? bwd : fwd;
 }
 
@@ -1639,15 +1636,18 @@ lora_status_t lora_linear_fwd_rope(const lora_linear_desc* d, const lora_rope_de
 
 lora_status_t lora_linear_bwd_rope(const lora_linear_desc* d, const lora_rope_desc* rope, const void* dY,
                                    const void* X, const void* W, const void* A, const void* B, const float* T_save,
-                                   void* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
+                                   float* dXn, int accumulate, float* dA, float* dB, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
   LORA_TRY(check_desc(d));
+  if (d->act != LORA_ACT_IDENTITY) return LORA_ERR_UNSUPPORTED;
+  if (accumulate != 0 && accumulate != 1) return LORA_ERR_INVALID_ARG;
+  if (d->M > 0 && dXn == nullptr) return LORA_ERR_INVALID_ARG;
   RopeTables t;
-  LORA_TRY(check_rope(d, rope, &t));
+  if (rope != nullptr) LORA_TRY(check_rope(d, rope, &t));
   const void* Xl[2] = {X, X};
   const uint8_t* masks[2] = {nullptr, nullptr};
-  return bwd_core(d, dY, X, W, A, B, nullptr, nullptr, nullptr, T_save, nullptr, dX, dA, dB, nullptr, nullptr,
-                  workspace, workspace_bytes, stream, Xl, masks, &t);
+  return bwd_core(d, dY, X, W, A, B, nullptr, nullptr, nullptr, T_save, nullptr, nullptr, dA, dB, nullptr, nullptr,
+                  workspace, workspace_bytes, stream, Xl, masks, rope != nullptr ? &t : nullptr, dXn, accumulate);
 }
 
 }  // extern "C"

@@ -63,6 +63,8 @@ struct MmaParams {
                           // 1: groups of `group` N tiles sweep all M tiles (the M-side operand stays in L2)
   int b_mn;               // backward: N-side operands read MN-major (W [K x N], A [r x N]) instead of K-major copies
   RopeTables rope;        // kMEpiRope: positions and cos / sin tables (half = 32 or 64)
+  float* out_f32;         // backward: fp32 dX [M x N] instead of the bf16 `out` (null: bf16)
+  int out_acc;            // with out_f32: dX += the product (else dX = the product)
 };
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
@@ -510,6 +512,30 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         if (!row_ok) continue;
         const int col0 = nt * 256 + h * 128;
         const size_t base = static_cast<size_t>(row) * p.N + col0;
+        if constexpr (kBwd) {
+          if (p.out_f32 != nullptr) {
+            // fp32 dX, written or added to (several projections' input
+            // gradients summed in a fixed order, one launch after another)
+            float* dst = p.out_f32 + base;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+              if (col0 + c < p.N) {
+                float4 o = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
+                                       __uint_as_float(v[c + 3]));
+                if (p.out_acc) {
+                  const float4 a = *reinterpret_cast<const float4*>(dst + c);
+                  o.x += a.x;
+                  o.y += a.y;
+                  o.z += a.z;
+                  o.w += a.w;
+                }
+                st_global_v4_hint(dst + c, make_uint4(__float_as_uint(o.x), __float_as_uint(o.y),
+                                                      __float_as_uint(o.z), __float_as_uint(o.w)), pol_out);
+              }
+            }
+            continue;
+          }
+        }
 #pragma unroll
         for (int c = 0; c < 128; c += 8) {
           uint4 pk;

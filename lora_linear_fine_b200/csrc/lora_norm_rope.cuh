@@ -19,8 +19,9 @@
 //   values never leave the chip.
 // * rope_bwd_kernel turns dY back (dZ = R^T dY) and emits dZ as fp16 hi + lo,
 //   the operand form of the backward with an activation.
-// * rmsnorm_bwd_kernel sums the projections' dx_n and applies the norm's
-//   backward: dx = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd.
+// * The projections' dX GEMMs write and then add their input gradients into
+//   one fp32 dx_n; rmsnorm_bwd_kernel applies the norm's backward:
+//   dx = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,7 +33,6 @@
 namespace lora {
 
 constexpr int kNormWarps = 8;      // token rows per CTA: one warp per row
-constexpr int kNormMaxGrads = 4;   // projections whose dx_n the norm's backward sums
 constexpr float kRopeF16Max = 65504.0f;   // largest finite fp16
 
 // Nearest bf16 (ties to even) of a double, without double rounding:
@@ -99,31 +99,23 @@ __global__ void __launch_bounds__(32 * kNormWarps)
   }
 }
 
-struct NormGrads {
-  const __nv_bfloat16* p[kNormMaxGrads];   // dx_n of each projection, [M x d] bf16
-  int n;
-};
-
 // dX [M x d] bf16 = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd,
-// dx_n the fp32 sum of the n gradients.  One warp per row, fp32, two passes.
+// dx_n [M x d] fp32: the projections' input gradients summed in fp32 by their
+// dX GEMMs (three bf16 roundings before the sum would cost the bound on the
+// near-zero entries of dx).  One warp per row, fp32, two passes.
 __global__ void __launch_bounds__(32 * kNormWarps)
     rmsnorm_bwd_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ g,
-                       const float* __restrict__ rstd, NormGrads dxn, long long M, int d,
+                       const float* __restrict__ rstd, const float* __restrict__ dxn, long long M, int d,
                        __nv_bfloat16* __restrict__ dX) {
   grid_dep_wait();
   const int lane = threadIdx.x & 31;
   const int nv = d / 8;
   const uint4* gv = reinterpret_cast<const uint4*>(g);
   auto grad8 = [&](long long row, int c, float (&dy)[8]) {
-    unpack_bf16x8(reinterpret_cast<const uint4*>(dxn.p[0] + row * d)[c], dy);
-#pragma unroll
-    for (int j = 1; j < kNormMaxGrads; ++j) {   // constant indices: the pointers stay in registers
-      if (j >= dxn.n) break;
-      float t[8];
-      unpack_bf16x8(reinterpret_cast<const uint4*>(dxn.p[j] + row * d)[c], t);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dy[e] += t[e];
-    }
+    const float4* q = reinterpret_cast<const float4*>(dxn + row * d) + 2 * c;
+    const float4 a = q[0], b = q[1];
+    dy[0] = a.x; dy[1] = a.y; dy[2] = a.z; dy[3] = a.w;
+    dy[4] = b.x; dy[5] = b.y; dy[6] = b.z; dy[7] = b.w;
   };
   for (long long row = blockIdx.x * static_cast<long long>(kNormWarps) + (threadIdx.x >> 5); row < M;
        row += static_cast<long long>(gridDim.x) * kNormWarps) {

@@ -165,11 +165,10 @@ def test_norm_and_rope_argument_checks(lib):
     assert lib.lora_linear_rmsnorm_fwd(None, 16, 4, 64, 1e-6, 16, 16, None) == 1
     assert lib.lora_linear_rmsnorm_fwd(24, 16, 4, 64, 1e-6, 16, 16, None) == 2
     assert lib.lora_linear_rmsnorm_fwd(16, 16, 4, 64, 1e-6, 16, 18, None) == 2      # rstd 4-byte aligned
-    # RMSNorm backward: 1..4 gradients, each present and aligned
-    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [], 4, 64, 16, None) == 1
-    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [16] * 5, 4, 64, 16, None) == 1
-    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [16, None], 4, 64, 16, None) == 1
-    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, [16, 24], 4, 64, 16, None) == 2
+    # RMSNorm backward: the fp32 gradient sum is required and aligned
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, None, 4, 64, 16, None) == 1
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, 24, 4, 64, 16, None) == 2
+    assert lib.lora_linear_rmsnorm_bwd(16, 16, 16, 16, 4, 60, 16, None) == 2
     # rotary projections: identity only, head_dim 64 / 128 dividing d_out, tables aligned
     d = lib.make_desc(256, 512, 256, 8, 2.0, "identity")
     f = lib.lora_linear_workspace_size_rope(d, 0)
@@ -193,5 +192,11 @@ def test_norm_and_rope_argument_checks(lib):
     raw = lib._LazyLib._h
     assert raw.lora_linear_fwd_rope(ctypes.byref(d), None, 16, 16, 16, 16, 16, None, 16, 1 << 30, None) == 1
     rope = lib.make_rope_desc(16, 16, 16, 32, 64)
-    assert lib.lora_linear_bwd_rope(lib.make_desc(256, 512, 256, 8, 2.0, "swiglu"), rope, 16, 16, 16, 16, 16, None,
-                                    16, 16, 16, 16, 1 << 30, None) == 3
+    bwd = lambda desc=d, rope=rope, dXn=16, acc=0: lib.lora_linear_bwd_rope(desc, rope, 16, 16, 16, 16, 16, None, dXn,
+                                                                            acc, 16, 16, 16, 1 << 30, None)
+    assert bwd(desc=lib.make_desc(256, 512, 256, 8, 2.0, "swiglu")) == 3
+    assert bwd(desc=lib.make_desc(256, 512, 256, 8, 2.0, "silu"), rope=None) == 3   # identity only, rotated or not
+    assert bwd(acc=2) == 1
+    assert bwd(dXn=None) == 1
+    assert bwd(dXn=24) == 2
+    assert bwd(rope=lib.make_rope_desc(16, 16, 16, 32, 96)) == 3

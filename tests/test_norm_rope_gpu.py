@@ -58,6 +58,8 @@ def test_rmsnorm_forward_bit_exact(M, d, eps):
 
 @pytest.mark.parametrize("M,d,n", [(37, 264, 1), (300, 4096, 3), (129, 512, 2), (4, 8, 4)])
 def test_rmsnorm_backward(M, d, n):
+    """dx_n: the fp32 sum of n drawn gradients (as the projections' dX GEMMs
+    leave it)."""
     import lora_linear_fine_b200 as L
     import torch
     Xb, gb = _norm_inputs(M, d, 42, zero_row=False)
@@ -66,19 +68,20 @@ def test_rmsnorm_backward(M, d, n):
     Xn = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
     rstd = torch.empty(M, dtype=torch.float32, device="cuda")
     assert L.lora_linear_rmsnorm_fwd(X.data_ptr(), g.data_ptr(), M, d, eps, Xn.data_ptr(), rstd.data_ptr(), _sh()) == 0
-    grads = [S.draw("dY", (M, d), 50 + j, d) for j in range(n)]
-    gd = [G.dev(b) for b in grads]
+    dXn = sum(G.f64(S.draw("dY", (M, d), 50 + j, d)) for j in range(n)).astype(np.float32)
+    dXn_d = torch.from_numpy(dXn).cuda()
     dX = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
-    assert L.lora_linear_rmsnorm_bwd(X.data_ptr(), g.data_ptr(), rstd.data_ptr(), [t.data_ptr() for t in gd], M, d,
+    assert L.lora_linear_rmsnorm_bwd(X.data_ptr(), g.data_ptr(), rstd.data_ptr(), dXn_d.data_ptr(), M, d,
                                      dX.data_ptr(), _sh()) == 0
     torch.cuda.synchronize()
-    dXn = sum(G.f64(b) for b in grads)
+    dXn = dXn.astype(np.float64)
     ref = NR.rms_norm_backward(dXn, G.f64(Xb), G.f64(gb), float(np.float32(eps)))
     G.assert_all_ok({"dX": oracle.compare(G.host_f64(dX), ref)})
 
 
-def _rope_call(L, M, d_in, d_out, r, s, t, pos, cos, sin, n_pos, hd):
-    """One forward + backward of a rotated projection through the C ABI."""
+def _rope_call(L, M, d_in, d_out, r, s, t, pos, cos, sin, n_pos, hd, prefill=None):
+    """One forward + backward of a rotated projection through the C ABI.  The
+    input gradient is fp32; with ``prefill`` it is added to that tensor."""
     import torch
     p = lambda x: None if x is None else x.data_ptr()
     desc = L.make_desc(M, d_in, d_out, r, s, "identity")
@@ -89,11 +92,12 @@ def _rope_call(L, M, d_in, d_out, r, s, t, pos, cos, sin, n_pos, hd):
     st = L.lora_linear_fwd_rope(desc, rope, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(Y), p(T),
                                 ws.buf.data_ptr(), ws.nbytes, _sh())
     assert st == 0, L.status_string(st)
-    dX = torch.empty((M, d_in), dtype=torch.bfloat16, device="cuda")
+    dX = (torch.from_numpy(prefill).cuda() if prefill is not None
+          else torch.empty((M, d_in), dtype=torch.float32, device="cuda"))
     dA = torch.empty((r, d_in), dtype=torch.float32, device="cuda")
     dB = torch.empty((d_out, r), dtype=torch.float32, device="cuda")
     st = L.lora_linear_bwd_rope(desc, rope, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(T), p(dX),
-                                p(dA), p(dB), ws.buf.data_ptr(), ws.nbytes, _sh())
+                                0 if prefill is None else 1, p(dA), p(dB), ws.buf.data_ptr(), ws.nbytes, _sh())
     assert st == 0, L.status_string(st)
     torch.cuda.synchronize()
     return {"Y": Y, "T": T, "dX": dX, "dA": dA, "dB": dB}, ws
@@ -105,14 +109,14 @@ def _tables_dev(n_pos, hd):
     return cos, sin, torch.from_numpy(cos).cuda(), torch.from_numpy(sin).cuda()
 
 
-@pytest.mark.parametrize("M,d_in,d_out,r,hd", [
-    (200, 384, 256, 8, 128),     # CTA-pair GEMM, ragged last tile
-    (96, 512, 384, 16, 64),      # single-CTA GEMM, two heads per 128 columns
-    (260, 256, 640, 64, 128),    # the last N tile runs past d_out
-    (136, 512, 192, 128, 64),    # rank 128; d_out not a multiple of 128
-    (3, 256, 128, 8, 128),       # a few tokens still take the tiled GEMM
+@pytest.mark.parametrize("M,d_in,d_out,r,hd,acc", [
+    (200, 384, 256, 8, 128, False),     # CTA-pair GEMM, ragged last tile
+    (96, 512, 384, 16, 64, True),       # single-CTA GEMM, two heads per 128 columns; dx added to a prefilled dx_n
+    (260, 256, 640, 64, 128, False),    # the last N tile runs past d_out
+    (136, 512, 192, 128, 64, True),     # rank 128; d_out not a multiple of 128; added
+    (3, 256, 128, 8, 128, False),       # a few tokens still take the tiled GEMM
 ])
-def test_rotated_projection(M, d_in, d_out, r, hd):
+def test_rotated_projection(M, d_in, d_out, r, hd, acc):
     import lora_linear_fine_b200 as L
     import torch
     s = 16.0 / r
@@ -121,8 +125,10 @@ def test_rotated_projection(M, d_in, d_out, r, hd):
     pos = S.draw_positions(M, n_pos, 21)
     cos, sin, cos_d, sin_d = _tables_dev(n_pos, hd)
     t = {k: G.dev(v) for k, v in inp.items()}
-    out, ws = _rope_call(L, M, d_in, d_out, r, s, t, torch.from_numpy(pos).cuda(), cos_d, sin_d, n_pos, hd)
+    pre = (np.random.default_rng(5).standard_normal((M, d_in)).astype(np.float32) if acc else None)
+    out, ws = _rope_call(L, M, d_in, d_out, r, s, t, torch.from_numpy(pos).cuda(), cos_d, sin_d, n_pos, hd, pre)
     assert ws.status() == 0
+    dx = G.host_f64(out["dX"]) - (pre.astype(np.float64) if acc else 0.0)
     g = {k: G.f64(v) for k, v in inp.items()}
     c64, s64 = cos.astype(np.float64), sin.astype(np.float64)
     f = oracle.lora_forward(g["X"], g["W"], g["A"], g["B"], s)
@@ -130,7 +136,7 @@ def test_rotated_projection(M, d_in, d_out, r, hd):
     b = oracle.lora_linear_branch_backward(dZ, g["X"], g["W"], g["A"], g["B"], f["T"], s)
     G.assert_all_ok({"Y": oracle.compare(G.host_f64(out["Y"]), NR.apply_rotary(f["Z"], pos, c64, s64, hd)),
                      "T": oracle.compare(G.host_f64(out["T"]), f["T"]),
-                     "dX": oracle.compare(G.host_f64(out["dX"]), b["dX"]),
+                     "dX": oracle.compare(dx, b["dX"]),
                      "dA": oracle.compare(G.host_f64(out["dA"]), b["dA"]),
                      "dB": oracle.compare(G.host_f64(out["dB"]), b["dB"])})
 
@@ -176,6 +182,7 @@ def _qkv_run(L, M, d, douts, r, hd, eps, Xb, gb, proj_inp, pos, cos_d, sin_d, n_
     rstd = torch.empty(M, dtype=torch.float32, device="cuda")
     assert L.lora_linear_rmsnorm_fwd(p(X), p(g), M, d, eps, p(Xn), p(rstd), _sh()) == 0
     rope = L.make_rope_desc(p(pos), p(cos_d), p(sin_d), n_pos, hd)
+    dXn = torch.empty((M, d), dtype=torch.float32, device="cuda")
     outs = []
     for j, (d_out, inp) in enumerate(zip(douts, proj_inp)):
         t = {k: G.dev(v) for k, v in inp.items() if k != "X"}
@@ -183,24 +190,21 @@ def _qkv_run(L, M, d, douts, r, hd, eps, Xb, gb, proj_inp, pos, cos_d, sin_d, n_
         ws = L.Workspace(max(L.lora_linear_workspace_size_rope(desc, 1), L.lora_linear_workspace_size(desc, 1)))
         Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
         T = torch.empty((M, r), dtype=torch.float32, device="cuda")
-        dX = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
         dA = torch.empty((r, d), dtype=torch.float32, device="cuda")
         dB = torch.empty((d_out, r), dtype=torch.float32, device="cuda")
         args = (p(t["W"]), p(t["A"]), p(t["B"]))
         if j < 2:
             assert L.lora_linear_fwd_rope(desc, rope, p(Xn), *args, p(Y), p(T), ws.buf.data_ptr(), ws.nbytes,
                                           _sh()) == 0
-            assert L.lora_linear_bwd_rope(desc, rope, p(t["dY"]), p(Xn), *args, p(T), p(dX), p(dA), p(dB),
-                                          ws.buf.data_ptr(), ws.nbytes, _sh()) == 0
         else:
             assert L.lora_linear_fwd(desc, p(Xn), *args, None, None, None, p(Y), p(T), None, ws.buf.data_ptr(),
                                      ws.nbytes, _sh()) == 0
-            assert L.lora_linear_bwd(desc, p(t["dY"]), p(Xn), *args, None, None, None, p(T), None, p(dX), p(dA),
-                                     p(dB), None, None, ws.buf.data_ptr(), ws.nbytes, _sh()) == 0
-        outs.append({"Y": Y, "T": T, "dX": dX, "dA": dA, "dB": dB, "ws": ws, "t": t})
+        # q writes the fp32 dx_n, k and v add to it; v is not rotated
+        assert L.lora_linear_bwd_rope(desc, rope if j < 2 else None, p(t["dY"]), p(Xn), *args, p(T), p(dXn),
+                                      1 if j else 0, p(dA), p(dB), ws.buf.data_ptr(), ws.nbytes, _sh()) == 0
+        outs.append({"Y": Y, "T": T, "dA": dA, "dB": dB, "ws": ws, "t": t})
     dXall = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
-    assert L.lora_linear_rmsnorm_bwd(p(X), p(g), p(rstd), [o["dX"].data_ptr() for o in outs], M, d, p(dXall),
-                                     _sh()) == 0
+    assert L.lora_linear_rmsnorm_bwd(p(X), p(g), p(rstd), p(dXn), M, d, p(dXall), _sh()) == 0
     torch.cuda.synchronize()
     for o in outs:
         assert o["ws"].status() == 0

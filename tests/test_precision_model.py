@@ -54,3 +54,30 @@ def test_bf16_dZ_breaks_dX_over_a_long_reduction():
     assert oracle.compare(good["dX"], ref["dX"])["ok"]
     res = oracle.compare(bad["dX"], ref["dX"])
     assert res["nfail"] > 0, res
+
+
+def test_block_input_gradient_needs_fp32_sum():
+    """The attention-input block: the norm's backward reads the sum of the q,
+    k and v input gradients.  Stored as three bf16 tensors and then summed,
+    they put entries of dx past the per-element bound (the norm's backward
+    scales their roundings by rstd g); summed in fp32 (as the dX GEMMs do, one
+    writing and two adding), dx stays well inside it."""
+    import numpy as np
+    from oracle import norm_rope_oracle as NR
+    M, d, douts, r, hd, n_pos = 130, 256, (256, 256, 256), 16, 128, 512
+    X = oracle.bf16_to_f64(seeded_inputs.draw("X", (M, d), 23, d))
+    g = oracle.bf16_to_f64(seeded_inputs.draw_norm_weight(d, 23))
+    proj = [seeded_inputs.make_inputs(M, d, n, r, "identity", seed=230 + j) for j, n in enumerate(douts)]
+    projs = [{k: oracle.bf16_to_f64(p[k]) for k in ("W", "A", "B")} for p in proj]
+    dYs = [oracle.bf16_to_f64(p["dY"]) for p in proj]
+    pos = seeded_inputs.draw_positions(M, n_pos, 23)
+    cos, sin = (t.astype(np.float64) for t in seeded_inputs.rotary_tables(n_pos, hd))
+    s, eps = 16.0 / r, float(np.float32(1e-6))
+    ref = NR.qkv_backward(dYs, X, g, eps, projs, s, [True, True, False], pos, cos, sin, hd)
+    parts = [ref["dZ"][j] @ projs[j]["W"] + s * ((ref["dZ"][j] @ projs[j]["B"]) @ projs[j]["A"]) for j in range(3)]
+    as_bf16 = oracle.compare(PM.to_bf16(NR.rms_norm_backward(sum(PM.to_bf16(q) for q in parts), X, g, eps)),
+                             ref["dX"])
+    as_fp32 = oracle.compare(PM.to_bf16(NR.rms_norm_backward(PM.to_f32(sum(PM.to_f32(q) for q in parts)), X, g, eps)),
+                             ref["dX"])
+    assert not as_bf16["ok"] and as_bf16["worst_ratio"] > 1.0, as_bf16
+    assert as_fp32["ok"] and as_fp32["worst_ratio"] < 0.5, as_fp32
