@@ -198,7 +198,7 @@ def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
     dt = statistics.mean(times)
     val = cfg_step_flops(cfg, rows) / dt / 1e12
     what = (f"the norm, q/k/v projections ({d_in}->{'/'.join(map(str, qkv_douts(cfg)))}) and rotation"
-            if is_qkv(cfg) else f"({d_in}->{d_out}, r={r})")
+            if is_qkv(cfg) else f"({d_in}->{d_out})")
     return {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 numpy oracle fwd+bwd on the first {rows} of {M} tokens "
                       f"{what}, r={r}; mean of {len(times)} runs of {dt:.2f} s; FLOPs by the same formula"}
