@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -73,7 +74,8 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # scratch: the samples are summarised into the JSON line
+        self.path = os.path.join(tempfile.gettempdir(), f"lora_bench_clocks_rank{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
