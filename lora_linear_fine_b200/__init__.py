@@ -7,6 +7,21 @@ arguments.  ``forward`` / ``backward`` / ``LoRALinearFunction`` wrap them for
 torch tensors (torch provides device memory and the stream).  Every step of the
 computation runs in the library's CUDA kernels; there is no fallback: if the
 library cannot be loaded, the first call raises ImportError.
+
+The attention-input block (RMSNorm, then the q, k, v projections, q and k
+rotated) is a sequence of calls on one stream:
+
+    lora_linear_rmsnorm_fwd(X, g, M, d, eps, Xn, rstd, s)
+    lora_linear_fwd_rope(desc_q, rope, Xn, Wq, Aq, Bq, Yq, Tq, ws, n, s)   # q, rotated
+    lora_linear_fwd_rope(desc_k, rope, Xn, Wk, Ak, Bk, Yk, Tk, ws, n, s)   # k, rotated
+    lora_linear_fwd(desc_v, Xn, Wv, Av, Bv, None, None, None, Yv, Tv, None, ws, n, s)
+    lora_linear_bwd_rope(desc_q, rope, dYq, Xn, Wq, Aq, Bq, Tq, dXn, 0, dAq, dBq, ws, n, s)
+    lora_linear_bwd_rope(desc_k, rope, dYk, Xn, Wk, Ak, Bk, Tk, dXn, 1, dAk, dBk, ws, n, s)
+    lora_linear_bwd_rope(desc_v, None, dYv, Xn, Wv, Av, Bv, Tv, dXn, 1, dAv, dBv, ws, n, s)
+    lora_linear_rmsnorm_bwd(X, g, rstd, dXn, M, d, dX, s)
+
+with rope = make_rope_desc(pos, cos, sin, n_pos, head_dim) and dXn an fp32
+[M x d] buffer that the q call writes and the k and v calls add to.
 """
 from __future__ import annotations
 
