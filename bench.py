@@ -86,6 +86,15 @@ class ClockSampler:
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: wait (at most 2 s) for its first
+        # sample so that a short timed region is still sampled
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 2.0 and self.proc.poll() is None:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
