@@ -1,11 +1,17 @@
 """Shared helpers of the GPU parity tests: seeded inputs on the device, one
-call of the library, and the oracle on the same bf16 bits."""
+call of the library, and the oracle on the same bf16 bits.
+
+The layer's oracle here is the plain C statement (oracle/lora_oracle_c.c,
+scalar fp64 loops).  Full-size tests whose M-long sums need a whole-batch W
+product use the numpy statement (oracle/lora_oracle.py, matmul as the
+library primitive), which the same pins hold to the same facts."""
 from __future__ import annotations
 
 import numpy as np
 
 import oracle
 import seeded_inputs
+from oracle import lora_oracle_c
 
 
 def dev(bits):
@@ -41,9 +47,12 @@ def run_library(inp, M, d_in, d_out, r, s, act, backward=True, recompute_T=False
     return out
 
 
-def run_oracle(inp, s, act):
-    g = {k: f64(v) for k, v in inp.items()}
-    b = oracle.lora_backward(g["dY"], g["X"], g["W"], g["A"], g["B"], s, act,
+def run_oracle(inp, s, act, impl=None):
+    """The layer's forward and backward on the inputs' bf16 values (the plain
+    C oracle unless ``impl`` names another pinned statement)."""
+    o = impl or lora_oracle_c
+    g = {k: o.bf16_to_f64(v) for k, v in inp.items()}
+    b = o.lora_backward(g["dY"], g["X"], g["W"], g["A"], g["B"], s, act,
                              g.get("W_up"), g.get("A_up"), g.get("B_up"))
     return b
 

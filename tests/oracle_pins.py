@@ -62,6 +62,35 @@ def _bwd(o, p, s, act):
 
 
 # ---------------------------------------------------------------------------
+def check_bf16_decoding(o):
+    """bf16 bit patterns decode to the IEEE values they stand for: a bf16
+    number is the upper half of a binary32 (sign, 8 exponent bits, 7 fraction
+    bits).  Expected values are written from that definition, bit by bit."""
+    cases = [
+        (0x3F80, 1.0),                          # exponent 127, fraction 0
+        (0xC040, -3.0),                         # sign, exponent 128, fraction 1000000b
+        (0x4049, 3.140625),                     # exponent 128, fraction 1001001b: 2 (1 + 73/128)
+        (0x3E80, 0.25),
+        (0xBF81, -(1.0 + 2.0 ** -7)),           # the smallest step above 1, negated
+        (0x7F7F, (2.0 - 2.0 ** -7) * 2.0 ** 127),   # the largest finite bf16
+        (0x0080, 2.0 ** -126),                  # the smallest normal
+        (0x0001, 2.0 ** -133),                  # the smallest subnormal: 2^-126 * 2^-7
+        (0x007F, 127 * 2.0 ** -133),            # the largest subnormal
+        (0x8000, -0.0),
+        (0x0000, 0.0),
+        (0x7F80, math.inf),
+        (0xFF80, -math.inf),
+    ]
+    bits = np.array([[b for b, _ in cases]], dtype=np.uint16)
+    got = np.asarray(o.bf16_to_f64(bits))
+    assert got.shape == bits.shape and got.dtype == np.float64, (got.shape, got.dtype)
+    for (b, want), v in zip(cases, got[0]):
+        assert v == want, f"bf16 0x{b:04X}: got {v!r}, want {want!r}"
+        assert math.copysign(1.0, v) == math.copysign(1.0, want), f"bf16 0x{b:04X}: sign of {v!r}"
+    nan = np.asarray(o.bf16_to_f64(np.array([0x7FC0], dtype=np.uint16)))
+    assert np.isnan(nan[0]), nan
+
+
 def check_golden_examples(o):
     for ex in _golden()["examples"]:
         X, W, A, B, dY = (_arr(ex[k]) for k in ("X", "W", "A", "B", "dY"))
@@ -252,6 +281,7 @@ def check_row_sampling_matches_full(o):
 
 
 ALL_CHECKS = [
+    check_bf16_decoding,
     check_golden_examples,
     check_activation_closed_forms,
     check_swiglu_with_unit_up_is_silu,

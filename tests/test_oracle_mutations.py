@@ -131,7 +131,30 @@ def m_identity_uses_silu_grad(o):
     o.act_backward = ab
 
 
-MUTATIONS = [m_drop_scale, m_double_scale, m_scaled_T, m_act_before_add, m_sigmoid_sign,
+def m_bf16_shift15(o):
+    o.bf16_to_f64 = lambda bits: (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 15).view(
+        np.float32).astype(np.float64)
+
+
+def m_bf16_as_fp16(o):
+    o.bf16_to_f64 = lambda bits: np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def m_bf16_drops_sign(o):
+    orig = o.bf16_to_f64
+    o.bf16_to_f64 = lambda bits: np.abs(orig(bits))
+
+
+def m_bf16_flushes_subnormals(o):
+    orig = o.bf16_to_f64
+
+    def dec(bits):
+        v = orig(bits)
+        return np.where(np.abs(v) < 2.0 ** -126, 0.0 * v, v)
+    o.bf16_to_f64 = dec
+
+
+MUTATIONS = [m_bf16_shift15, m_bf16_as_fp16, m_bf16_drops_sign, m_bf16_flushes_subnormals, m_drop_scale, m_double_scale, m_scaled_T, m_act_before_add, m_sigmoid_sign,
              m_silu_grad_sign, m_swiglu_swapped, m_swiglu_up_grad, m_dx_missing_lora,
              m_dA_no_scale, m_dB_wrong_operand, m_dx_sign, m_U_transposed_B,
              m_identity_uses_silu_grad]
