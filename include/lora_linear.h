@@ -27,7 +27,12 @@
  * ---------------------------------------
  * - Pointers marked "device" must point to memory of the current CUDA device;
  *   all of them are caller-owned.  The library allocates nothing and keeps no
- *   state between calls other than a per-device cache of the SM count.
+ *   state between calls other than a per-device cache of the SM count (and,
+ *   for lora_linear_fwd_noalloc, of its static scratch array's address).  The
+ *   one exception is a debugging aid: with the environment variable
+ *   LORA_LINEAR_DEBUG=2 the few-token forward allocates an 8 MB device trace
+ *   buffer once (cudaMalloc) and prints per-CTA phase timestamps after each
+ *   launch.  Production callers leave LORA_LINEAR_DEBUG unset (or 0/1).
  * - Matrices are dense, row-major, with no padding between rows.
  *   bf16 tensors are IEEE bfloat16 bit patterns (2 bytes per element).
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -75,7 +80,8 @@ typedef enum lora_status_t {
     LORA_OK = 0,
     LORA_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, bad act */
     LORA_ERR_ALIGNMENT = 2,     /* pointer not 16-byte aligned, d_in/d_out not multiples of 8 */
-    LORA_ERR_UNSUPPORTED = 3,   /* r outside {0, 8, 16, ..., 64} or r not a multiple of 8 */
+    LORA_ERR_UNSUPPORTED = 3,   /* r not a multiple of 8 or above 128; a size or option an entry point
+                                   does not serve (stated with that entry point) */
     LORA_ERR_ARCH = 4,          /* current device is not sm_100 */
     LORA_ERR_WORKSPACE = 5,     /* workspace NULL or smaller than lora_linear_workspace_size */
     LORA_ERR_CUDA = 6,          /* a CUDA runtime/driver call or a launch failed */
@@ -209,13 +215,34 @@ lora_status_t lora_linear_timing_read(double* fwd_ms, uint64_t* fwd_launches, do
  *   before any stream capture.
  * - Every call, on every stream, shares the one array and leaves its contents
  *   behind; each call clears the part that must start at zero (its status
- *   word).  Calls that overlap on the GPU (e.g. on two streams at once) race
- *   on it: serialise them. */
+ *   word) and writes every other byte it reads before reading it.  Calls that
+ *   overlap on the GPU (e.g. on two streams at once) race on it: serialise
+ *   them.
+ * - Arguments are checked in lora_linear_fwd's order (desc, pointers,
+ *   alignment, device architecture, then the scratch size) before the array
+ *   is touched, so a rejected call queues nothing.
+ * - The cached address belongs to the device's primary context: do not use
+ *   this entry point across a cudaDeviceReset of that device.  Devices with
+ *   an ordinal of 64 or more are not served (LORA_ERR_UNSUPPORTED).
+ * - A kernel that gives up (a bounded wait that ran out) records it in the
+ *   array's status word, not in a return value: read it with
+ *   lora_linear_noalloc_status after the call and before the next one (the
+ *   next call clears it). */
 #define LORA_LINEAR_NOALLOC_SCRATCH_BYTES (16u << 20)
 lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* desc,
                                       const void* X, const void* W, const void* A, const void* B,
                                       const void* W_up, const void* A_up, const void* B_up,
                                       void* Y, float* T_save, float* Z_save, void* stream);
+
+/* The device status word of lora_linear_fwd_noalloc's scratch array on the
+ * current device (same bits as lora_linear_device_status).  Synchronises
+ * `stream`, copies the word to *out_status (host) and returns LORA_OK if it is
+ * zero, LORA_ERR_DEVICE_STATUS otherwise.  Call it on the stream of the
+ * no-alloc call whose outcome you want, after that call and before the next
+ * one.  Allocates nothing.  out_status NULL: LORA_ERR_INVALID_ARG; not sm_100:
+ * LORA_ERR_ARCH.  The pages have no counterpart: it reports this library's
+ * own failure detection. */
+lora_status_t lora_linear_noalloc_status(void* stream, uint32_t* out_status);
 
 /* ------------------------------------------------------------------------
  * 4-bit frozen base weight ("w4g64").  The pages name QLoRA fine-tuning, whose

@@ -42,7 +42,8 @@ STATUS_NAMES = {
 # Every symbol include/lora_linear.h declares.
 EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_linear_device_status",
             "lora_linear_fwd", "lora_linear_bwd", "lora_status_string", "lora_linear_abi_version",
-            "lora_linear_launch_count", "lora_linear_fwd_noalloc", "lora_linear_timing_enable",
+            "lora_linear_launch_count", "lora_linear_fwd_noalloc", "lora_linear_noalloc_status",
+            "lora_linear_timing_enable",
             "lora_linear_timing_read", "lora_linear_selftest_wait_timeout",
             "lora_linear_workspace_size_w4", "lora_linear_dequant_w4", "lora_linear_fwd_w4", "lora_linear_bwd_w4",
             "lora_linear_workspace_size_dropout", "lora_linear_fwd_dropout", "lora_linear_bwd_dropout",
@@ -92,6 +93,8 @@ def _load():
     lib.lora_linear_launch_count.restype = ctypes.c_uint64
     lib.lora_linear_fwd_noalloc.argtypes = [dp] + [vp] * 10 + [vp]
     lib.lora_linear_fwd_noalloc.restype = i32
+    lib.lora_linear_noalloc_status.argtypes = [vp, u32p]
+    lib.lora_linear_noalloc_status.restype = i32
     lib.lora_linear_timing_enable.argtypes = [i32]
     lib.lora_linear_timing_enable.restype = i32
     dblp, u64p = ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)
@@ -194,6 +197,14 @@ def lora_linear_fwd_noalloc(desc, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_sav
     is a fixed 16 MiB device array inside the library (see the C header)."""
     return int(_lib.lora_linear_fwd_noalloc(ctypes.byref(desc), X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save,
                                             stream))
+
+
+def lora_linear_noalloc_status(stream):
+    """(status code, status word) of the no-alloc forward's scratch array on the
+    current device; synchronises ``stream``."""
+    out = ctypes.c_uint32(0)
+    st = int(_lib.lora_linear_noalloc_status(stream, ctypes.byref(out)))
+    return st, int(out.value)
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

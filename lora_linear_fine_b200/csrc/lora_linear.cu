@@ -937,7 +937,7 @@ const char* lora_status_string(lora_status_t s) {
     case LORA_OK: return "ok";
     case LORA_ERR_INVALID_ARG: return "invalid argument";
     case LORA_ERR_ALIGNMENT: return "misaligned pointer or dimension (16-byte pointers, d_in/d_out multiples of 8)";
-    case LORA_ERR_UNSUPPORTED: return "unsupported shape (r must be 0 or a multiple of 8 up to 64)";
+    case LORA_ERR_UNSUPPORTED: return "unsupported shape or option (r must be 0 or a multiple of 8 up to 128)";
     case LORA_ERR_ARCH: return "current device is not sm_100 (B200)";
     case LORA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case LORA_ERR_CUDA: return "CUDA error";
@@ -975,10 +975,11 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
 // The forward.  Xl[j] is the input of projection j's adapter branch (X, or
 // the dropout-masked copy of X); allow_small_m = false keeps the tiled path
 // for few tokens.
-static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const void* W, const void* A,
-                              const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
-                              float* T_save, float* Z_save, void* workspace, size_t workspace_bytes, void* stream,
-                              const void* const Xl[2], bool allow_small_m, const RopeTables* rope = nullptr) {
+// Host-side argument checks of a forward (desc, required pointers,
+// alignment): everything that needs neither the device nor the workspace.
+static lora_status_t fwd_check_args(const lora_linear_desc* d, const void* X, const void* W, const void* A,
+                                    const void* B, const void* W_up, const void* A_up, const void* B_up,
+                                    const void* Y, const void* T_save, const void* Z_save) {
   LORA_TRY(check_desc(d));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
   // with M == 0 the per-token tensors are empty and may be NULL
@@ -988,6 +989,15 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   const void* ptrs[] = {X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save};
   for (const void* q : ptrs)
     if (q != nullptr && !aligned16(q)) return LORA_ERR_ALIGNMENT;
+  return LORA_OK;
+}
+
+static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const void* W, const void* A,
+                              const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
+                              float* T_save, float* Z_save, void* workspace, size_t workspace_bytes, void* stream,
+                              const void* const Xl[2], bool allow_small_m, const RopeTables* rope = nullptr) {
+  LORA_TRY(fwd_check_args(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save));
+  const bool swiglu = d->act == LORA_ACT_SWIGLU;
   const Plan P = make_plan(d, false, allow_small_m);
   DevInfo dev;
   LORA_TRY(common_checks(d, workspace, workspace_bytes, P.total, &dev));
@@ -1360,7 +1370,11 @@ void* g_noalloc_ptr[64] = {};
 
 lora_status_t noalloc_scratch(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cuda_error("cudaGetDevice");
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_error("cudaGetDevice");
+  if (dev < 0 || dev >= 64) {
+    LORA_LOG("fwd_noalloc: device ordinal %d is beyond the 64 devices whose scratch address is cached", dev);
+    return LORA_ERR_UNSUPPORTED;
+  }
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
   if (g_noalloc_ptr[dev] == nullptr) {
     void* p = nullptr;
@@ -1391,7 +1405,11 @@ lora_status_t lora_linear_bwd(const lora_linear_desc* d, const void* dY, const v
 lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, const void* W, const void* A,
                                       const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
                                       float* T_save, float* Z_save, void* stream) {
-  LORA_TRY(check_desc(d));
+  // the same argument and device checks as lora_linear_fwd, in the same
+  // order, before the scratch is touched
+  LORA_TRY(fwd_check_args(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save));
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
   const size_t need = make_plan(d, false).total;
   if (need > LORA_LINEAR_NOALLOC_SCRATCH_BYTES) {
     LORA_LOG("fwd_noalloc: needs %zu bytes of scratch, the static array holds %u", need,
@@ -1406,6 +1424,15 @@ lora_status_t lora_linear_fwd_noalloc(const lora_linear_desc* d, const void* X, 
     return cuda_error("cudaMemsetAsync(scratch status)");
   return lora_linear_fwd(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, ws, LORA_LINEAR_NOALLOC_SCRATCH_BYTES,
                          stream);
+}
+
+lora_status_t lora_linear_noalloc_status(void* stream, uint32_t* out_status) {
+  if (out_status == nullptr) return LORA_ERR_INVALID_ARG;
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
+  void* ws = nullptr;
+  LORA_TRY(noalloc_scratch(&ws));
+  return lora_linear_device_status(ws, stream, out_status);
 }
 
 // ---------------------------------------------------------------------------

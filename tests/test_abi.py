@@ -119,6 +119,20 @@ def test_no_gpu_means_cuda_error_not_crash(lib):
     assert _fwd(lib, ok) == 6                         # LORA_ERR_CUDA: no device
 
 
+def test_noalloc_rejects_bad_arguments_before_touching_the_scratch(lib):
+    """The no-alloc forward checks its arguments in lora_linear_fwd's order,
+    before any device query, symbol lookup or memset."""
+    ok = lib.make_desc(64, 256, 256, 8, 2.0, "identity")
+    na = lambda desc=ok, X=16, A=16, Y=16: lib.lora_linear_fwd_noalloc(desc, X, 16, A, 16, None, None, None, Y,
+                                                                       None, None, None)
+    assert na(X=None) == 1                       # INVALID_ARG: X required with M > 0
+    assert na(A=None) == 1
+    assert na(Y=24) == 2                         # ALIGNMENT
+    assert na(desc=lib.make_desc(64, 256, 256, 12, 2.0, 0)) == 3
+    raw = lib._LazyLib._h
+    assert raw.lora_linear_noalloc_status(None, None) == 1     # out_status NULL
+
+
 def test_selftest_rejects_bad_arguments_without_launching(lib):
     assert lib.lora_linear_selftest_wait_timeout(None, 1 << 20, 16, None) == 5   # WORKSPACE
     assert lib.lora_linear_selftest_wait_timeout(16, 64, 16, None) == 5          # below the header
