@@ -36,6 +36,8 @@ import numpy as np  # noqa: E402
 import seeded_inputs  # noqa: E402
 
 METRIC = "LoRA-linear fwd+bwd TFLOP/s (M=16384, 4096², r=8) & % of B200 roofline"
+METRIC_CE = "LoRA fine-tuning output projection + cross-entropy fwd+bwd TFLOP/s & % of B200 roofline"
+METRIC_SMALL_M = "LoRA-linear forward (few tokens) TFLOP/s & % of B200 HBM roofline"
 METRIC_QKV = "LoRA attention-input block (RMSNorm + q/k/v + rotary) fwd+bwd TFLOP/s & % of B200 roofline"
 UNIT = "TFLOP/s"
 
@@ -136,6 +138,8 @@ def cfg_step_flops(cfg, M):
     counted)."""
     if is_qkv(cfg):
         return sum(step_flops(M, cfg["d_in"], n, cfg["r"]) for n in qkv_douts(cfg))
+    if cfg["act"] == "ce":       # logits + dH of the output projection fused with the loss
+        return 4.0 * M * cfg["d_in"] * cfg["d_out"]
     return step_flops(M, cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"])
 
 
@@ -157,8 +161,10 @@ def qkv_inputs(cfg, M, seed):
     return out
 
 
-def oracle_sample_run(cfg, rows, inp_f64):
-    import oracle
+def oracle_sample_run(cfg, rows, inp_f64, fwd_only=False):
+    """Seconds the oracle takes for one sample of `rows` tokens of the
+    workload: the plain C fp64 oracle for the layer, the numpy block oracle
+    (norm, three projections, rotation) for the attention-input block."""
     g = inp_f64
     if is_qkv(cfg):
         from oracle import norm_rope_oracle
@@ -168,26 +174,44 @@ def oracle_sample_run(cfg, rows, inp_f64):
                                       float(np.float32(cfg["eps"])), projs, cfg["alpha"] / cfg["r"],
                                       [True, True, False], g["pos"][:rows], g["cos"], g["sin"], cfg["head_dim"])
         return time.perf_counter() - t0
+    if cfg["act"] == "ce":
+        from oracle import linear_ce_oracle
+        t0 = time.perf_counter()
+        linear_ce_oracle.linear_ce_backward(g["H"][:rows], g["W"], g["labels"][:rows])
+        return time.perf_counter() - t0
+    from oracle import lora_oracle_c
     X = g["X"][:rows]
-    dY = g["dY"][:rows]
+    s = cfg["alpha"] / cfg["r"]
     t0 = time.perf_counter()
-    oracle.lora_backward(dY, X, g["W"], g["A"], g["B"], cfg["alpha"] / cfg["r"], cfg["act"],
-                         g.get("W_up"), g.get("A_up"), g.get("B_up"))
+    if fwd_only:
+        lora_oracle_c.lora_forward(X, g["W"], g["A"], g["B"], s, cfg["act"], g.get("W_up"), g.get("A_up"),
+                                   g.get("B_up"))
+    else:
+        lora_oracle_c.lora_backward(g["dY"][:rows], X, g["W"], g["A"], g["B"], s, cfg["act"], g.get("W_up"),
+                                    g.get("A_up"), g.get("B_up"))
     return time.perf_counter() - t0
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else os.cpu_count()
-    except Exception:
-        return os.cpu_count()
+def oracle_cores(cfg):
+    """Threads the oracle runs on: the C oracle's POSIX threads, or numpy's BLAS pool."""
+    if is_qkv(cfg) or cfg["act"] == "ce":
+        try:
+            from threadpoolctl import threadpool_info
+            n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+            return max(n) if n else os.cpu_count()
+        except Exception:
+            return os.cpu_count()
+    from oracle import lora_oracle_c
+    return lora_oracle_c.threads()
 
 
-def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
+def oracle_kind(cfg):
+    return ("fp64 numpy oracle (matmul through the BLAS)" if is_qkv(cfg) or cfg["act"] == "ce"
+            else "plain C fp64 oracle (scalar loops, POSIX threads over output rows)")
+
+
+def cpu_baseline(cfg, budget_s=12.0, max_rows=None, fwd_only=False):
     """Time the oracle on growing row samples until ~budget_s of CPU work."""
-    import oracle
     M, d_in, d_out, r = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"]
     rows_cap = max_rows or (4096 if is_qkv(cfg) else M)
     g = oracle_inputs(cfg, min(M, rows_cap))
@@ -195,7 +219,7 @@ def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
     spent = 0.0
     best = None
     while True:
-        dt = oracle_sample_run(cfg, rows, g)
+        dt = oracle_sample_run(cfg, rows, g, fwd_only)
         spent += dt
         best = (rows, dt)
         if dt > budget_s / 3 or rows >= min(M, rows_cap) or spent > budget_s:
@@ -205,19 +229,24 @@ def cpu_baseline(cfg, budget_s=12.0, max_rows=None):
     # repeat the chosen sample until ~budget_s / 2 of work has been timed
     times = [dt]
     while sum(times) < budget_s / 2 and len(times) < 20:
-        times.append(oracle_sample_run(cfg, rows, g))
+        times.append(oracle_sample_run(cfg, rows, g, fwd_only))
     dt = statistics.mean(times)
-    val = cfg_step_flops(cfg, rows) / dt / 1e12
+    flops = fwd_flops(rows, d_in, d_out, r, cfg["act"]) if fwd_only else cfg_step_flops(cfg, rows)
+    val = flops / dt / 1e12
     what = (f"the norm, q/k/v projections ({d_in}->{'/'.join(map(str, qkv_douts(cfg)))}) and rotation"
-            if is_qkv(cfg) else f"({d_in}->{d_out})")
-    return {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle fwd+bwd on the first {rows} of {M} tokens "
-                      f"{what}, r={r}; mean of {len(times)} runs of {dt:.2f} s; FLOPs by the same formula"}
+            if is_qkv(cfg) else f"(output projection {d_in}->{d_out} + cross-entropy)" if cfg["act"] == "ce"
+            else f"({d_in}->{d_out}, {cfg['act']})")
+    return {"value": val, "unit": UNIT, "cores": oracle_cores(cfg), "kind": "oracle",
+            "sample": f"{oracle_kind(cfg)}, {'forward' if fwd_only else 'fwd+bwd'} on the first {rows} of {M} "
+                      f"tokens {what}, r={r}; mean of {len(times)} runs of {dt:.2f} s; FLOPs by the same formula"}
 
 
 def oracle_inputs(cfg, M):
     """The workload's inputs for the oracle (float64; positions and tables as given)."""
     import oracle
+    if cfg["act"] == "ce":
+        H, W, labels = seeded_inputs.draw_ce(M, cfg["d_in"], cfg["d_out"], 0)
+        return {"H": oracle.bf16_to_f64(H), "W": oracle.bf16_to_f64(W), "labels": labels}
     if is_qkv(cfg):
         raw = qkv_inputs(cfg, M, 0)
         return {k: (v.astype(np.float64) if k in ("cos", "sin") else v if k == "pos" else oracle.bf16_to_f64(v))
@@ -230,29 +259,37 @@ def run_reference(args, cfg, world, rank):
     if rank != 0:
         return
     steps, warm = args.steps, args.warmup
-    g = oracle_inputs(cfg, min(cfg["M"], 4096))
+    fwd_only = args.config.startswith("small_m")
+    g = oracle_inputs(cfg, min(cfg["M"], 256 if cfg["act"] == "ce" else 4096))
     # rows per step: sized so the whole warm-up + timed run stays within a few minutes
-    rows = 64
-    while rows < 4096:
-        dt = oracle_sample_run(cfg, rows, g)
+    rows = 16
+    cap = min(cfg["M"], 256 if cfg["act"] == "ce" else 4096)
+    while rows < cap:
+        dt = oracle_sample_run(cfg, rows, g, fwd_only)
         if dt * (steps + warm) > 60.0 or dt > 2.0:
             break
-        rows *= 2
+        rows = min(rows * 2, cap)
     for _ in range(warm):
-        oracle_sample_run(cfg, rows, g)
+        oracle_sample_run(cfg, rows, g, fwd_only)
     tot = 0.0
     for _ in range(steps):
-        tot += oracle_sample_run(cfg, rows, g)
-    val = cfg_step_flops(cfg, rows) * steps / tot / 1e12
+        tot += oracle_sample_run(cfg, rows, g, fwd_only)
+    flops = fwd_flops(rows, cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]) if fwd_only else cfg_step_flops(cfg, rows)
+    val = flops * steps / tot / 1e12
     shape = (f"norm + {cfg['d_in']}->{'/'.join(map(str, qkv_douts(cfg)))} + rotary" if is_qkv(cfg)
+             else f"output projection {cfg['d_in']}->{cfg['d_out']} + cross-entropy" if cfg["act"] == "ce"
              else f"{cfg['d_in']}->{cfg['d_out']}")
-    sample = f"fp64 numpy oracle fwd+bwd on {rows} of {cfg['M']} tokens per step ({shape}, r={cfg['r']})"
-    line = {"impl": "reference", "metric": METRIC_QKV if is_qkv(cfg) else METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": steps,
-            "warmup": warm, "ms_per_step": tot / steps * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+    sample = (f"{oracle_kind(cfg)}, {'forward' if fwd_only else 'fwd+bwd'} on {rows} of {cfg['M']} tokens per "
+              f"step ({shape}, r={cfg['r']})")
+    metric = (METRIC_QKV if is_qkv(cfg) else METRIC_CE if cfg["act"] == "ce"
+              else METRIC_SMALL_M if fwd_only else METRIC)
+    line = {"impl": "reference", "metric": metric, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": tot / steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.config, "M": cfg["M"], "d_in": cfg["d_in"], "d_out": cfg["d_out"],
                        "r": cfg["r"], "alpha": cfg["alpha"], "act": cfg["act"], "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle_cores(cfg), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -291,53 +328,390 @@ def committed_traffic(workload, record="gemm_traffic.json", source="lora_mma.cuh
         return None
 
 
-def run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist):
-    """Few tokens: forward only, bound by reading W once (HBM roofline)."""
+# ---------------------------------------------------------------------------
+# one LoRA-linear workload on the device
+# ---------------------------------------------------------------------------
+class Layer:
+    """Device inputs, outputs and workspace of one LoRA-linear workload, with
+    fwd() / bwd() closures that call the C ABI.  The input tensors live in
+    self.t and may be re-pointed (a chained MLP feeds one layer's output to the
+    next)."""
+
+    def __init__(self, L, cfg, seed, pin_host=False):
+        import torch
+        self.L, self.cfg = L, cfg
+        M, d_in, d_out, r, act = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]
+        self.M, self.d_in, self.d_out, self.r, self.act = M, d_in, d_out, r, act
+        self.s = cfg["alpha"] / r if r else 0.0
+        inp = seeded_inputs.make_inputs(M, d_in, d_out, r, act, seed=seed)
+        self.w4 = cfg.get("weight") == "w4"
+        if self.w4:   # the 4-bit base weight replaces W (forward-only few-token workload)
+            inp.pop("W")
+            Wq, Ws = seeded_inputs.draw_w4("W", d_out, d_in, seed)
+        host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) for k, v in inp.items()}
+        self.p_drop = cfg.get("dropout")
+        if self.p_drop is not None:   # dropout on the adapter input: one mask per projection, an input like X
+            for name in ("mask", "mask_up") if act == "swiglu" else ("mask",):
+                host[name] = torch.from_numpy(seeded_inputs.draw_mask(name, M, d_in, self.p_drop, seed))
+        if pin_host:
+            host = {k: v.pin_memory() for k, v in host.items()}
+        self.host = host
+        self.t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+        self.stream = torch.cuda.current_stream()
+        self.sh = self.stream.cuda_stream
+        if self.w4:
+            self.t["Wq"] = torch.from_numpy(Wq).cuda()
+            self.t["Ws"] = torch.from_numpy(Ws.view(np.int16)).view(torch.bfloat16).cuda()
+            # the frozen weight's codes in the few-token kernel's tiled layout (a load-time step)
+            self.t["Wt"] = torch.empty(L.lora_linear_w4_tiled_bytes(d_out, d_in), dtype=torch.uint8, device="cuda")
+            assert L.lora_linear_w4_tile(self.t["Wq"].data_ptr(), d_out, d_in, self.t["Wt"].data_ptr(), self.sh) == 0
+        self.desc = L.make_desc(M, d_in, d_out, r, self.s, act)
+        self.np = 2 if act == "swiglu" else 1
+        if self.w4:
+            nb = L.lora_linear_workspace_size_w4(self.desc, 0)
+        elif self.p_drop is not None:
+            nb = L.lora_linear_workspace_size_dropout(self.desc, 1)
+        else:
+            nb = max(L.lora_linear_workspace_size(self.desc, 0), L.lora_linear_workspace_size(self.desc, 1))
+        self.ws = L.Workspace(nb)
+        bf, f32 = torch.bfloat16, torch.float32
+        self.Y = torch.empty((M, d_out), dtype=bf, device="cuda")
+        self.T = torch.empty((self.np, M, r), dtype=f32, device="cuda")
+        self.Z = torch.empty((self.np, M, d_out), dtype=f32, device="cuda") if act != "identity" else None
+        self.dX = torch.empty((M, d_in), dtype=bf, device="cuda")
+        self.dA = torch.empty((self.np, r, d_in), dtype=f32, device="cuda")
+        self.dB = torch.empty((self.np, d_out, r), dtype=f32, device="cuda")
+
+    @staticmethod
+    def p(x):
+        return None if x is None else x.data_ptr()
+
+    def fwd(self):
+        L, t, p, sh = self.L, self.t, self.p, self.sh
+        ws = (self.ws.buf.data_ptr(), self.ws.nbytes, sh)
+        if self.w4 and self.M <= 64:
+            st = L.lora_linear_fwd_w4_tiled(self.desc, p(t["X"]), p(t["Wt"]), p(t["Ws"]), p(t["A"]), p(t["B"]),
+                                            p(self.Y), p(self.T), p(self.Z), *ws)
+        elif self.w4:
+            st = L.lora_linear_fwd_w4(self.desc, p(t["X"]), p(t["Wq"]), p(t["Ws"]), p(t["A"]), p(t["B"]), None,
+                                      None, None, None, p(self.Y), p(self.T), p(self.Z), *ws)
+        elif self.p_drop is not None:
+            st = L.lora_linear_fwd_dropout(self.desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
+                                           p(t.get("A_up")), p(t.get("B_up")), p(t["mask"]), p(t.get("mask_up")),
+                                           self.p_drop, p(self.Y), p(self.T), p(self.Z), *ws)
+        else:
+            st = L.lora_linear_fwd(self.desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
+                                   p(t.get("A_up")), p(t.get("B_up")), p(self.Y), p(self.T), p(self.Z), *ws)
+        assert st == 0, L.status_string(st)
+
+    def bwd(self):
+        L, t, p, sh = self.L, self.t, self.p, self.sh
+        ws = (self.ws.buf.data_ptr(), self.ws.nbytes, sh)
+        two = self.np == 2
+        grads = (p(self.dX), p(self.dA[0]), p(self.dB[0]), p(self.dA[1]) if two else None,
+                 p(self.dB[1]) if two else None)
+        if self.p_drop is not None:
+            st = L.lora_linear_bwd_dropout(self.desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]),
+                                           p(t.get("W_up")), p(t.get("A_up")), p(t.get("B_up")), p(t["mask"]),
+                                           p(t.get("mask_up")), self.p_drop, p(self.T), p(self.Z), *grads, *ws)
+        else:
+            st = L.lora_linear_bwd(self.desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]),
+                                   p(t.get("W_up")), p(t.get("A_up")), p(t.get("B_up")), p(self.T), p(self.Z),
+                                   *grads, *ws)
+        assert st == 0, L.status_string(st)
+
+    # algorithmic work
+    def step_flops(self):
+        return step_flops(self.M, self.d_in, self.d_out, self.r, self.act)
+
+    def fwd_gemm_flops(self):    # X W^T + (sT) B^T, per projection
+        return self.np * (2.0 * self.M * self.d_in * self.d_out + 2.0 * self.M * self.r * self.d_out)
+
+    def dx_gemm_flops(self):     # dZ W + (sU) A, per projection
+        return self.np * (2.0 * self.M * self.d_in * self.d_out + 2.0 * self.M * self.r * self.d_in)
+
+    def fwd_bytes(self):
+        """Algorithmic bytes of the forward: X, W (bf16, or 4-bit codes + scales), A, B
+        read once, Y written once, T (fp32) written once."""
+        d_in, d_out, M, r = self.d_in, self.d_out, self.M, self.r
+        w = (d_out * d_in / 2.0 + 2.0 * d_out * (d_in // 64)) if self.w4 else 2.0 * d_out * d_in
+        return self.np * (w + 2.0 * (r * d_in + d_out * r)) + 2.0 * (M * d_in + M * d_out) + 4.0 * self.np * M * r
+
+
+def time_steps(L, step, steps, warmup, flush, stream, local, dist=None, sample_clocks=True):
+    """Warm up, then time `steps` calls of step() with CUDA events on `stream`,
+    the L2 flushed (a 512 MiB write) before each, outside the events; the
+    library's own event pairs time its GEMM launches.  Returns per-step
+    milliseconds, the GEMM times, the launch count and the clock record."""
     import torch
-    M, d_in, d_out, r = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"]
-    for _ in range(args.warmup):
-        fwd()
+    for _ in range(warmup):
+        step()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     launches0 = L.lora_linear_launch_count()
-    for i in range(args.steps):
+    L.lora_linear_timing_enable(1)
+    L.lora_linear_timing_read()              # start from zero
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    clocks = ClockSampler(local) if sample_clocks else None
+    if clocks:
+        clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
-        fwd()
+        step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
     launches = L.lora_linear_launch_count() - launches0
-    ms = [a.elapsed_time(b) for a, b in ev]
-    med = statistics.median(ms)
-    F = fwd_flops(M, d_in, d_out, r)
-    w4 = cfg.get("weight") == "w4"
-    # the base weight: bf16, or 4-bit codes plus one bf16 scale per row and 64 features
-    w_bytes = (d_out * d_in / 2.0 + 2.0 * d_out * (d_in // 64)) if w4 else 2.0 * d_out * d_in
-    byts = w_bytes + 2.0 * (M * d_in + r * d_in + d_out * r + M * d_out) + 4.0 * M * r
-    peaks = read_peaks()
-    gbs = byts / (med * 1e-3) / 1e9
-    line = {"metric": "LoRA-linear forward (few tokens), HBM roofline", "value": round(F / (med * 1e-3) / 1e12, 3),
-            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(med, 5), "timing": "median of per-step CUDA events",
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": args.config, "M": M, "d_in": d_in, "d_out": d_out, "r": r,
-                       "alpha": cfg["alpha"], "act": cfg["act"], "weight": "w4g64" if w4 else "bf16",
-                       "l2": "flushed before each timed step (512 MiB write)"},
-            "roofline": {"kernel": "small_m_kernel" if M <= 64 else "lora_gemm_kernel (forward)", "bound": "hbm",
-                         "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "traffic": committed_traffic(args.config, "small_m_traffic.json", "lora_small_m.cuh")
-                         if M <= 64 else None,
-                         "bytes_per_launch": byts},
-            "gpu_launches": int(launches)}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    _, gf_ms, gf_n, gb_ms, gb_n = L.lora_linear_timing_read()
+    L.lora_linear_timing_enable(0)
+    return {"ms": [a.elapsed_time(b) for a, b in ev], "gemm_fwd_ms": gf_ms, "gemm_fwd_n": gf_n,
+            "gemm_bwd_ms": gb_ms, "gemm_bwd_n": gb_n, "launches": int(launches), "clocks": clk}
 
 
-# ---------------------------------------------------------------------------
-# our arm
-# ---------------------------------------------------------------------------
+def gemm_record(flop_per_step, ms_total, n_launch, launches_per_step, peak):
+    """Achieved TFLOP/s of the GEMM launches of one direction: their FLOPs over
+    their summed CUDA-event durations (the library times at most 1024 launches
+    per direction between reads, a whole number of steps)."""
+    if not n_launch:
+        return None
+    steps_timed = n_launch / launches_per_step
+    ach = flop_per_step * steps_timed / (ms_total * 1e-3) / 1e12
+    return {"achieved": round(ach, 2), "frac": round(ach / peak, 4), "flop_per_step": flop_per_step,
+            "launches_per_step": launches_per_step, "ms_per_launch": round(ms_total / n_launch, 5)}
+
+
+def steps_for(seconds, ms_guess, lo=10, hi=1000):
+    return int(max(lo, min(hi, seconds * 1e3 / max(ms_guess, 1e-3))))
+
+
+def measure_layer_workload(L, name, local, flush, seconds=0.5, peaks=None):
+    """A fwd+bwd workload timed on its own (the `workloads` entries)."""
+    import torch
+    cfg = dict(seeded_inputs.CONFIGS[name])
+    lay = Layer(L, cfg, seed=0)
+
+    def step():
+        lay.fwd()
+        lay.bwd()
+    probe = time_steps(L, step, 3, 3, flush, lay.stream, local, sample_clocks=False)
+    steps = steps_for(seconds, statistics.median(probe["ms"]))
+    r = time_steps(L, step, steps, 2, flush, lay.stream, local)
+    ms = statistics.median(r["ms"])
+    pk = peaks["bf16_tflops"]
+    F = lay.step_flops()
+    tf = F / (ms * 1e-3) / 1e12
+    out = {"M": cfg["M"], "d_in": cfg["d_in"], "d_out": cfg["d_out"], "r": cfg["r"], "act": cfg["act"],
+           "steps": steps, "ms_per_step": round(ms, 5), "timing": "median of per-step CUDA events, L2 flushed",
+           "value": round(tf, 2), "unit": UNIT,
+           "roofline": {"bound": "tensor", "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
+                        "flop_per_step": F},
+           "forward_gemm": gemm_record(lay.fwd_gemm_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 1, pk),
+           "dx_gemm": gemm_record(lay.dx_gemm_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"], 1, pk),
+           "gpu_launches_per_step": r["launches"] // steps, "clocks": r["clocks"]}
+    if name == "tiny":
+        out["roofline"]["bound"] = "latency (parity workload: 1.8e7 FLOP per step)"
+    del lay
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_mlp(L, local, flush, seconds=0.5, peaks=None):
+    """The Llama-3-8B MLP with LoRA r = 64 on gate, up and down, chained: the
+    gate/up layer (SwiGLU in its epilogue) feeds H to the down projection; the
+    down projection's input gradient is the gate/up layer's dY."""
+    import torch
+    gu = Layer(L, dict(seeded_inputs.CONFIGS["mlp_gate_up"]), seed=0)
+    dn = Layer(L, dict(seeded_inputs.CONFIGS["mlp_down"]), seed=1)
+    dn.t["X"] = gu.Y
+    gu.t["dY"] = dn.dX
+
+    def step():
+        gu.fwd()
+        dn.fwd()
+        dn.bwd()
+        gu.bwd()
+    probe = time_steps(L, step, 2, 2, flush, gu.stream, local, sample_clocks=False)
+    steps = steps_for(seconds, statistics.median(probe["ms"]), lo=10)
+    r = time_steps(L, step, steps, 2, flush, gu.stream, local)
+    ms = statistics.median(r["ms"])
+    pk = peaks["bf16_tflops"]
+    F = gu.step_flops() + dn.step_flops()
+    tf = F / (ms * 1e-3) / 1e12
+    out = {"M": gu.M, "d_model": gu.d_in, "d_ff": gu.d_out, "r": gu.r, "act": "swiglu (gate, up) -> down",
+           "steps": steps, "ms_per_step": round(ms, 5), "timing": "median of per-step CUDA events, L2 flushed",
+           "value": round(tf, 2), "unit": UNIT,
+           "roofline": {"bound": "tensor", "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
+                        "flop_per_step": F},
+           "forward_gemms": gemm_record(gu.fwd_gemm_flops() + dn.fwd_gemm_flops(), r["gemm_fwd_ms"],
+                                        r["gemm_fwd_n"], 2, pk),
+           "dx_gemms": gemm_record(gu.dx_gemm_flops() + dn.dx_gemm_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"],
+                                   2, pk),
+           "gpu_launches_per_step": r["launches"] // steps, "clocks": r["clocks"]}
+    del gu, dn
+    torch.cuda.empty_cache()
+    return out
+
+
+class CeWorkload:
+    """The output projection fused with the cross-entropy loss: H [M x d],
+    W [V x d] (bf16), int32 labels; one step = lora_linear_ce_fwd (loss, lse)
+    + lora_linear_ce_bwd (dH)."""
+
+    def __init__(self, L, cfg, seed, pin_host=False):
+        import torch
+        self.L = L
+        self.M, self.d, self.V = cfg["M"], cfg["d_in"], cfg["d_out"]
+        H, W, labels = seeded_inputs.draw_ce(self.M, self.d, self.V, seed)
+        host = {"H": torch.from_numpy(H.view(np.int16)).view(torch.bfloat16),
+                "W": torch.from_numpy(W.view(np.int16)).view(torch.bfloat16),
+                "labels": torch.from_numpy(labels)}
+        if pin_host:
+            host = {k: v.pin_memory() for k, v in host.items()}
+        self.host = host
+        self.t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+        self.stream = torch.cuda.current_stream()
+        self.sh = self.stream.cuda_stream
+        self.desc = L.make_ce_desc(self.M, self.d, self.V)
+        self.ws = L.Workspace(L.lora_linear_ce_workspace_size(self.desc, 1))
+        self.loss = torch.empty((), dtype=torch.float32, device="cuda")
+        self.lse = torch.empty(self.M, dtype=torch.float32, device="cuda")
+        self.dloss = torch.ones((), dtype=torch.float32, device="cuda")
+        self.dH = torch.empty((self.M, self.d), dtype=torch.bfloat16, device="cuda")
+
+    def fwd(self):
+        t = self.t
+        st = self.L.lora_linear_ce_fwd(self.desc, t["H"].data_ptr(), t["W"].data_ptr(), t["labels"].data_ptr(),
+                                       self.loss.data_ptr(), self.lse.data_ptr(), self.ws.buf.data_ptr(),
+                                       self.ws.nbytes, self.sh)
+        assert st == 0, self.L.status_string(st)
+
+    def bwd(self):
+        t = self.t
+        st = self.L.lora_linear_ce_bwd(self.desc, t["H"].data_ptr(), t["W"].data_ptr(), t["labels"].data_ptr(),
+                                       self.lse.data_ptr(), self.dloss.data_ptr(), self.dH.data_ptr(),
+                                       self.ws.buf.data_ptr(), self.ws.nbytes, self.sh)
+        assert st == 0, self.L.status_string(st)
+
+    def logit_flops(self):      # H W^T, once per forward and once more (recomputed) per backward
+        return 2.0 * self.M * self.V * self.d
+
+    def step_flops(self):       # the quantity: logits + dH = dz W (the recompute is not counted)
+        return 4.0 * self.M * self.V * self.d
+
+
+def measure_ce(L, cfg, local, flush, steps=None, warmup=3, peaks=None, dist=None, ce=None):
+    """Time the fused output projection + cross-entropy, forward + backward."""
+    ce = ce or CeWorkload(L, cfg, seed=0)
+
+    def step():
+        ce.fwd()
+        ce.bwd()
+    if steps is None:
+        probe = time_steps(L, step, 2, 2, flush, ce.stream, local, sample_clocks=False)
+        steps = steps_for(1.0, statistics.median(probe["ms"]), lo=5, hi=200)
+    r = time_steps(L, step, steps, warmup, flush, ce.stream, local, dist)
+    ms = statistics.median(r["ms"])
+    pk = peaks["bf16_tflops"]
+    F = ce.step_flops()
+    tf = F / (ms * 1e-3) / 1e12
+    # logits GEMMs (forward + recompute: timing direction 0), dH GEMM (direction 1)
+    logits = gemm_record(2 * ce.logit_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 2, pk)
+    dh = gemm_record(ce.logit_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"], 1, pk)
+    out = {"M": ce.M, "d": ce.d, "V": ce.V, "steps": steps, "ms_per_step": round(ms, 5),
+           "timing": "median of per-step CUDA events, L2 flushed",
+           "value": round(tf, 2), "unit": UNIT,
+           "roofline": {"bound": "tensor", "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
+                        "flop_per_step": F, "flop_executed_per_step": 1.5 * F,
+                        "frac_executed": round(1.5 * tf / pk, 4)},
+           "logit_gemms": logits, "dh_gemm": dh,
+           "gpu_launches_per_step": r["launches"] // steps, "clocks": r["clocks"]}
+    return out, ce, r
+
+
+def small_m_roofline(lay, ms, peaks):
+    """max(FLOPs / tensor peak, bytes / HBM bandwidth) against the measured time."""
+    F = lay.fwd_gemm_flops() + (2.0 * lay.M * lay.d_in * lay.r)
+    byts = lay.fwd_bytes()
+    t_tensor = F / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    bound = "hbm" if t_hbm >= t_tensor else "tensor"
+    gbs = byts / (ms * 1e-3) / 1e9
+    tf = F / (ms * 1e-3) / 1e12
+    if bound == "hbm":
+        return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_launch": byts, "flop_per_launch": F,
+                "tflops": round(tf, 3)}
+    return {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tf / peaks["bf16_tflops"], 4), "bytes_per_launch": byts, "flop_per_launch": F,
+            "hbm_gbs": round(gbs, 1), "roofline_us": round(max(t_tensor, t_hbm) * 1e6, 2)}
+
+
+def small_m_back_to_back(L, lay, peaks, copies=None, reps=20):
+    """Few-token forwards launched back to back over distinct copies of W (as
+    the layers of one decode step), no flush between them: each launch streams
+    its W from HBM (the copies together exceed twice the L2), and programmatic
+    dependent launch lets a launch start while its predecessor drains.  One
+    event pair around each chain of launches; returns the median per launch."""
+    import torch
+    if lay.w4 or "W" not in lay.t:
+        return None
+    wb = lay.t["W"].numel() * 2
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    n = copies or max(4, int(2 * l2 // wb) + 2)
+    Ws = [lay.t["W"].clone() for _ in range(n)]
+    orig = lay.t["W"]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    launches0 = L.lora_linear_launch_count()
+    for rep in range(reps + 2):
+        e0.record(lay.stream)
+        for w in Ws:
+            lay.t["W"] = w
+            lay.fwd()
+        e1.record(lay.stream)
+        torch.cuda.synchronize()
+        if rep >= 2:
+            ts.append(e0.elapsed_time(e1) / n)
+    lay.t["W"] = orig
+    launches = (L.lora_linear_launch_count() - launches0) // ((reps + 2) * n)
+    ms = statistics.median(ts)
+    roof = small_m_roofline(lay, ms, peaks)
+    del Ws
+    return {"ms_per_launch": round(ms, 5), "weight_copies": n, "chains": reps, "roofline": roof,
+            "launches_per_forward": launches,
+            "timing": "median over chains of (event pair around n back-to-back launches) / n"}
+
+
+def measure_small_m(L, name, local, flush, seconds=0.3, peaks=None, lay=None):
+    """A forward-only few-token workload: W read once (HBM roofline), or, for
+    the ragged M = 1000 run, the larger of the tensor and HBM times."""
+    import torch
+    cfg = dict(seeded_inputs.CONFIGS[name])
+    lay = lay or Layer(L, cfg, seed=0)
+    probe = time_steps(L, lay.fwd, 5, 3, flush, lay.stream, local, sample_clocks=False)
+    steps = steps_for(seconds, statistics.median(probe["ms"]) + 0.1, lo=50)
+    r = time_steps(L, lay.fwd, steps, 3, flush, lay.stream, local)
+    ms = statistics.median(r["ms"])
+    roof = small_m_roofline(lay, ms, peaks)
+    kernel = "small_m_kernel" if lay.M <= 64 else "rank_gemm_kernel (T) + lora_mma_kernel (forward GEMM)"
+    roof["kernel"] = kernel
+    if lay.M <= 64:
+        roof["traffic"] = committed_traffic(name, "small_m_traffic.json", "lora_small_m.cuh")
+    F = roof["flop_per_launch"]
+    out = {"M": lay.M, "d_in": lay.d_in, "d_out": lay.d_out, "r": lay.r, "act": lay.act,
+           "weight": "w4g64" if lay.w4 else "bf16", "steps": steps, "ms_per_step": round(ms, 5),
+           "timing": "median of per-launch CUDA events, L2 flushed before each (a single cold launch)",
+           "value": round(F / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "roofline": roof,
+           "gpu_launches_per_step": r["launches"] // steps, "clocks": r["clocks"],
+           "back_to_back": small_m_back_to_back(L, lay, peaks)}
+    return out, lay, r
+
+
 def run_qkv(args, cfg, L, world, rank, local, dist):
     """The attention-input block: RMSNorm, the q, k, v projections (q and k
     rotated in the GEMM epilogue), their backward, and the norm's backward over
@@ -494,6 +868,165 @@ def run_qkv(args, cfg, L, world, rank, local, dist):
         dist.destroy_process_group()
 
 
+def layer_e2e(lay, steps, dist, fwd_only=False):
+    """The same step through the C ABI from pinned HOST buffers, copies
+    included: every step copies its inputs host -> device and its results
+    device -> host.  Two buffer sets and one copy stream per direction let step
+    i+1's input copy and step i-1's result copy run while step i computes (PCIe
+    is full duplex), as a training loop feeding the layer would arrange them.
+    Returns (milliseconds for `steps` steps, h2d bytes, d2h bytes per step)."""
+    import copy
+    import torch
+    stream = lay.stream
+    outs = ("Y",) if fwd_only else ("Y", "dX", "dA", "dB")
+    host = {k: v if v.is_pinned() else v.pin_memory() for k, v in lay.host.items()
+            if not (fwd_only and k == "dY")}
+    second = copy.copy(lay)
+    second.t = dict(lay.t)
+    for k in host:
+        second.t[k] = torch.empty_like(lay.t[k])
+    for k in ("Y", "T", "Z", "dX", "dA", "dB"):
+        v = getattr(lay, k)
+        setattr(second, k, None if v is None else torch.empty_like(v))
+    bufs = [lay, second]
+    out_host = [{k: torch.empty_like(getattr(lay, k), device="cpu").pin_memory() for k in outs} for _ in range(2)]
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host[0].values())
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ee0.record(stream)
+    s_in.wait_event(ee0)
+    s_out.wait_event(ee0)
+    for i in range(steps):
+        b = i % 2
+        cur = bufs[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(comp_done[b])        # step i-2 no longer reads these inputs
+            for k, v in host.items():
+                cur.t[k].copy_(v, non_blocking=True)
+            in_ready[b].record(s_in)
+        stream.wait_event(in_ready[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])           # step i-2's results are on the host
+        cur.fwd()
+        if not fwd_only:
+            cur.bwd()
+        comp_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            for k in outs:
+                out_host[b][k].copy_(getattr(cur, k), non_blocking=True)
+            out_done[b].record(s_out)
+    for b in range(min(2, steps)):
+        stream.wait_event(out_done[b])
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    return ee0.elapsed_time(ee1), h2d, d2h
+
+
+def run_small_m_line(args, cfg, L, world, rank, local, dist, flush, peaks):
+    """Few tokens: forward only, bound by reading W once (HBM roofline); the
+    ragged M = 1000 run against the larger of its tensor and HBM times."""
+    lay = Layer(L, cfg, seed=rank, pin_host=True)
+    r = time_steps(L, lay.fwd, args.steps, args.warmup, flush, lay.stream, local, dist)
+    med = statistics.median(r["ms"])
+    tot_ms = max_over_ranks(sum(r["ms"]), dist, "cuda")
+    roof = small_m_roofline(lay, med, peaks)
+    roof["kernel"] = "small_m_kernel" if lay.M <= 64 else "rank_gemm_kernel (T) + lora_mma_kernel (forward GEMM)"
+    if lay.M <= 64:
+        roof["traffic"] = committed_traffic(args.config, "small_m_traffic.json", "lora_small_m.cuh")
+    F = roof["flop_per_launch"]
+    e2e_ms, h2d, d2h = layer_e2e(lay, args.e2e_steps, dist, fwd_only=True)
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
+    b2b = small_m_back_to_back(L, lay, peaks)
+    line = {"metric": METRIC_SMALL_M, "value": round(job_throughput(F, args.steps, world, tot_ms) / 1e12, 3),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_ms / args.steps, 5), "ms_median": round(med, 5),
+            "timing": "per-launch CUDA events, L2 flushed before each (value: total; frac: median launch)",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.config, "M": lay.M, "d_in": lay.d_in, "d_out": lay.d_out, "r": lay.r,
+                       "alpha": cfg["alpha"], "act": lay.act, "weight": "w4g64" if lay.w4 else "bf16",
+                       "parallelism": f"replicas x{world}", "l2": "flushed before each timed step (512 MiB write)"},
+            "roofline": roof, "gpu_launches": r["launches"],
+            "back_to_back": b2b,
+            "e2e": {"value": round(job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12, 3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "clocks": r["clocks"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, fwd_only=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_ce_line(args, cfg, L, world, rank, local, dist, flush, peaks):
+    """The output projection fused with the cross-entropy loss as the line's
+    workload (forward + backward per step)."""
+    import torch
+    ce = CeWorkload(L, cfg, seed=rank, pin_host=True)
+    ent, ce, r = measure_ce(L, cfg, local, flush, steps=args.steps, warmup=args.warmup, peaks=peaks, dist=dist,
+                            ce=ce)
+    tot_ms = max_over_ranks(sum(r["ms"]), dist, "cuda")
+    F = ce.step_flops()
+    value = job_throughput(F, args.steps, world, tot_ms) / 1e12
+    # e2e: per step, H, W and the labels from pinned host memory, the loss and
+    # dH back, serialised with the compute
+    outs = {"loss": ce.loss, "dH": ce.dH}
+    out_host = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in outs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in ce.host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ee0.record(ce.stream)
+    for _ in range(args.e2e_steps):
+        for k, v in ce.host.items():
+            ce.t[k].copy_(v, non_blocking=True)
+        ce.fwd()
+        ce.bwd()
+        for k, v in outs.items():
+            out_host[k].copy_(v, non_blocking=True)
+    ee1.record(ce.stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ee0.elapsed_time(ee1), dist, "cuda")
+    pk = peaks["bf16_tflops"]
+    lg, dh = ent["logit_gemms"], ent["dh_gemm"]
+    dom_is_dh = dh is not None and (lg is None or dh["ms_per_launch"] > lg["ms_per_launch"])
+    dom = dh if dom_is_dh else lg
+    roof = {"kernel": "lora_mma_kernel (dH = dz W, K = V)" if dom_is_dh
+            else "lora_mma_kernel (logits with the cross-entropy epilogue)",
+            "bound": "tensor", "achieved": dom["achieved"] if dom else None, "peak": pk, "unit": "TFLOP/s",
+            "frac": dom["frac"] if dom else None,
+            "peak_kind": f"bf16 burst, {peaks['source']} (sustained {peaks['bf16_tflops_sustained']})",
+            "ms_per_launch": dom["ms_per_launch"] if dom else None, "traffic": None,
+            "other_gemm": lg if dom_is_dh else dh, "step_frac": round(value / world / pk, 4),
+            "step_frac_executed": round(1.5 * value / world / pk, 4)}
+    line = {"metric": METRIC_CE,
+            "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_ms / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.config, "M": ce.M, "d": ce.d, "V": ce.V,
+                       "flops": "4 M V d per step (logits + dH; the backward's recompute of the logits, "
+                                "another 2 M V d, is not counted)",
+                       "parallelism": f"replicas x{world}", "l2": "flushed before each timed step (512 MiB write)"},
+            "roofline": roof, "gpu_launches": r["launches"],
+            "e2e": {"value": round(job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "copies": "serialised with the compute"},
+            "clocks": ent["clocks"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, max_rows=256)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,6 +1035,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="q_proj", choices=sorted(seeded_inputs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' entries of the default line")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--shape", default=None,
                     help="M,d_in,d_out,r,act: this shape instead of --config (profiling, with --calls)")
@@ -538,215 +1073,99 @@ def main():
     if is_qkv(cfg):
         run_qkv(args, cfg, L, world, rank, local, dist)
         return
-    M, d_in, d_out, r, act = cfg["M"], cfg["d_in"], cfg["d_out"], cfg["r"], cfg["act"]
-    s = cfg["alpha"] / r if r else 0.0
-    inp = seeded_inputs.make_inputs(M, d_in, d_out, r, act, seed=rank)
-    w4 = cfg.get("weight") == "w4"
-    if w4:   # the 4-bit base weight replaces W (forward-only few-token workload)
-        inp.pop("W")
-        Wq, Ws = seeded_inputs.draw_w4("W", d_out, d_in, rank)
-    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in inp.items()}
-    t = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
-    if w4:
-        t["Wq"] = torch.from_numpy(Wq).cuda()
-        t["Ws"] = torch.from_numpy(Ws.view(np.int16)).view(torch.bfloat16).cuda()
-        # the frozen weight's codes in the few-token kernel's tiled layout (a load-time step)
-        t["Wt"] = torch.empty(L.lora_linear_w4_tiled_bytes(d_out, d_in), dtype=torch.uint8, device="cuda")
-        assert L.lora_linear_w4_tile(t["Wq"].data_ptr(), d_out, d_in, t["Wt"].data_ptr(),
-                                     torch.cuda.current_stream().cuda_stream) == 0
-    p_drop = cfg.get("dropout")
-    if p_drop is not None:   # dropout on the adapter input: one mask per projection, an input like X
-        for name in ("mask", "mask_up") if act == "swiglu" else ("mask",):
-            host[name] = torch.from_numpy(seeded_inputs.draw_mask(name, M, d_in, p_drop, rank)).pin_memory()
-            t[name] = host[name].to("cuda", non_blocking=True)
-    stream = torch.cuda.current_stream()
-    sh = stream.cuda_stream
-    desc = L.make_desc(M, d_in, d_out, r, s, act)
-    np_ = 2 if act == "swiglu" else 1
-    if w4:
-        ws = L.Workspace(L.lora_linear_workspace_size_w4(desc, 0))
-    elif p_drop is not None:
-        ws = L.Workspace(L.lora_linear_workspace_size_dropout(desc, 1))
-    else:
-        ws = L.Workspace(max(L.lora_linear_workspace_size(desc, 0), L.lora_linear_workspace_size(desc, 1)))
-    Y = torch.empty((M, d_out), dtype=torch.bfloat16, device="cuda")
-    T = torch.empty((np_, M, r), dtype=torch.float32, device="cuda")
-    Z = torch.empty((np_, M, d_out), dtype=torch.float32, device="cuda") if act != "identity" else None
-    dX = torch.empty((M, d_in), dtype=torch.bfloat16, device="cuda")
-    dA = torch.empty((np_, r, d_in), dtype=torch.float32, device="cuda")
-    dB = torch.empty((np_, d_out, r), dtype=torch.float32, device="cuda")
-    p = lambda x: None if x is None else x.data_ptr()  # noqa: E731
-
-    def fwd():
-        if w4 and M <= 64:
-            st = L.lora_linear_fwd_w4_tiled(desc, p(t["X"]), p(t["Wt"]), p(t["Ws"]), p(t["A"]), p(t["B"]), p(Y),
-                                            p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
-        elif w4:
-            st = L.lora_linear_fwd_w4(desc, p(t["X"]), p(t["Wq"]), p(t["Ws"]), p(t["A"]), p(t["B"]), None, None,
-                                      None, None, p(Y), p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
-        elif p_drop is not None:
-            st = L.lora_linear_fwd_dropout(desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
-                                           p(t.get("A_up")), p(t.get("B_up")), p(t["mask"]), p(t.get("mask_up")),
-                                           p_drop, p(Y), p(T), p(Z), ws.buf.data_ptr(), ws.nbytes, sh)
-        else:
-            st = L.lora_linear_fwd(desc, p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
-                                   p(t.get("A_up")), p(t.get("B_up")), p(Y), p(T), p(Z), ws.buf.data_ptr(),
-                                   ws.nbytes, sh)
-        assert st == 0, L.status_string(st)
-
-    def bwd():
-        if p_drop is not None:
-            st = L.lora_linear_bwd_dropout(desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]),
-                                           p(t.get("W_up")), p(t.get("A_up")), p(t.get("B_up")), p(t["mask"]),
-                                           p(t.get("mask_up")), p_drop, p(T), p(Z), p(dX), p(dA[0]), p(dB[0]),
-                                           p(dA[1]) if np_ == 2 else None, p(dB[1]) if np_ == 2 else None,
-                                           ws.buf.data_ptr(), ws.nbytes, sh)
-            assert st == 0, L.status_string(st)
-            return
-        st = L.lora_linear_bwd(desc, p(t["dY"]), p(t["X"]), p(t["W"]), p(t["A"]), p(t["B"]), p(t.get("W_up")),
-                               p(t.get("A_up")), p(t.get("B_up")), p(T), p(Z), p(dX), p(dA[0]), p(dB[0]),
-                               p(dA[1]) if np_ == 2 else None, p(dB[1]) if np_ == 2 else None,
-                               ws.buf.data_ptr(), ws.nbytes, sh)
-        assert st == 0, L.status_string(st)
-
     if args.calls > 0:
+        lay = Layer(L, cfg, seed=rank)
         for _ in range(args.calls):
-            fwd()
+            lay.fwd()
             if not args.fwd_only:
-                bwd()
+                lay.bwd()
         torch.cuda.synchronize()
         print("ok", flush=True)
         return
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    if args.config.startswith("small_m"):
-        run_small_m(args, cfg, fwd, flush, stream, L, world, rank, dist)
+    peaks = read_peaks()
+    if cfg["act"] == "ce":
+        run_ce_line(args, cfg, L, world, rank, local, dist, flush, peaks)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
         return
-    for _ in range(args.warmup):
-        fwd()
-        bwd()
-    torch.cuda.synchronize()
+    if args.config.startswith("small_m"):
+        run_small_m_line(args, cfg, L, world, rank, local, dist, flush, peaks)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
-    launches0 = L.lora_linear_launch_count()
-    L.lora_linear_timing_enable(1)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        e0, e1, e2 = ev[i]
-        e0.record(stream)
-        fwd()
-        e1.record(stream)
-        bwd()
-        e2.record(stream)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    clk = clocks.stop()
-    launches = L.lora_linear_launch_count() - launches0
-    _, gemm_fwd_ms, gemm_fwd_n, gemm_bwd_ms, gemm_bwd_n = L.lora_linear_timing_read()
-    L.lora_linear_timing_enable(0)
-    step_ms = [a.elapsed_time(c) for a, _, c in ev]
-    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    tot_ms = sum(step_ms)
-    tot_ms = max_over_ranks(tot_ms, dist, "cuda")
-    F = step_flops(M, d_in, d_out, r, act)
+    lay = Layer(L, cfg, seed=rank, pin_host=True)
+
+    def step():
+        lay.fwd()
+        lay.bwd()
+    r = time_steps(L, step, args.steps, args.warmup, flush, lay.stream, local, dist)
+    tot_ms = max_over_ranks(sum(r["ms"]), dist, "cuda")
+    F = lay.step_flops()
     value = job_throughput(F, args.steps, world, tot_ms) / 1e12
-
-    # e2e: the same step through the C ABI from pinned HOST buffers, copies
-    # included: every step copies its inputs host -> device and its results
-    # device -> host.  Two buffer sets and one copy stream per direction let
-    # step i+1's input copy and step i-1's result copy run while step i
-    # computes (PCIe is full duplex), as a training loop feeding the layer
-    # would arrange them.
-    bufs = [dict(t=t, Y=Y, dX=dX, dA=dA, dB=dB),
-            dict(t={k: torch.empty_like(v) for k, v in t.items()}, Y=torch.empty_like(Y),
-                 dX=torch.empty_like(dX), dA=torch.empty_like(dA), dB=torch.empty_like(dB))]
-    for k in bufs[1]["t"]:
-        if k not in host:                 # inputs that are not copied per step (none in the bf16 path)
-            bufs[1]["t"][k].copy_(t[k])
-    out_host = [{k: torch.empty_like(bufs[0][k], device="cpu").pin_memory() for k in ("Y", "dX", "dA", "dB")}
-                for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = sum(v.numel() * v.element_size() for v in out_host[0].values())
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    in_ready = [torch.cuda.Event() for _ in range(2)]
-    comp_done = [torch.cuda.Event() for _ in range(2)]
-    out_done = [torch.cuda.Event() for _ in range(2)]
-    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ee0.record(stream)
-    s_in.wait_event(ee0)
-    s_out.wait_event(ee0)
-    for i in range(args.e2e_steps):
-        b = i % 2
-        cur = bufs[b]
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(comp_done[b])        # step i-2 no longer reads these inputs
-            for k, v in host.items():
-                cur["t"][k].copy_(v, non_blocking=True)
-            in_ready[b].record(s_in)
-        stream.wait_event(in_ready[b])
-        if i >= 2:
-            stream.wait_event(out_done[b])           # step i-2's results are on the host
-        t, Y, dX, dA, dB = cur["t"], cur["Y"], cur["dX"], cur["dA"], cur["dB"]
-        fwd()
-        bwd()
-        comp_done[b].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(comp_done[b])
-            for k in ("Y", "dX", "dA", "dB"):
-                out_host[b][k].copy_(cur[k], non_blocking=True)
-            out_done[b].record(s_out)
-    for b in range(min(2, args.e2e_steps)):
-        stream.wait_event(out_done[b])
-    ee1.record(stream)
-    torch.cuda.synchronize()
-    t, Y, dX, dA, dB = bufs[0]["t"], bufs[0]["Y"], bufs[0]["dX"], bufs[0]["dA"], bufs[0]["dB"]
-    e2e_ms = ee0.elapsed_time(ee1)
+    e2e_ms, h2d, d2h = layer_e2e(lay, args.e2e_steps, dist)
     e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
     e2e = job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12
 
-    peaks = read_peaks()
-    # Dominant kernels: the forward and backward GEMMs (lora_mma_kernel), each
-    # timed by the library's event pair around its launch on this stream.
-    np_ = 2 if act == "swiglu" else 1
-    f_fwd = np_ * (2.0 * M * d_in * d_out + 2.0 * M * r * d_out)       # X W^T + (sT) B^T
-    f_bwd = np_ * (2.0 * M * d_in * d_out + 2.0 * M * r * d_in)        # dZ W + (sU) A
-    ach_f = f_fwd / (gemm_fwd_ms / max(gemm_fwd_n, 1) * 1e-3) / 1e12 if gemm_fwd_n else None
-    ach_b = f_bwd / (gemm_bwd_ms / max(gemm_bwd_n, 1) * 1e-3) / 1e12 if gemm_bwd_n else None
+    # The dominant kernel: whichever of the two GEMM launches (lora_mma_kernel,
+    # forward or dX) took longer per launch, each timed by the library's event
+    # pair around its launch on this stream; the other is reported beside it.
     pk = peaks["bf16_tflops"]
+    gf = gemm_record(lay.fwd_gemm_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 1, pk)
+    gb = gemm_record(lay.dx_gemm_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"], 1, pk)
     traffic = committed_traffic(args.config)
-    roof = {"kernel": "lora_mma_kernel (forward GEMM)", "bound": "tensor",
-            "achieved": round(ach_f, 2) if ach_f else None, "peak": pk, "unit": "TFLOP/s",
-            "frac": round(ach_f / pk, 4) if ach_f else None,
+    dom_is_dx = gb is not None and (gf is None or gb["ms_per_launch"] > gf["ms_per_launch"])
+    dom, other = (gb, gf) if dom_is_dx else (gf, gb)
+    roof = {"kernel": "lora_mma_kernel (dX GEMM)" if dom_is_dx else "lora_mma_kernel (forward GEMM)",
+            "bound": "tensor", "achieved": dom["achieved"] if dom else None, "peak": pk, "unit": "TFLOP/s",
+            "frac": dom["frac"] if dom else None,
             "peak_kind": f"bf16 burst, {peaks['source']} (sustained {peaks['bf16_tflops_sustained']})",
-            "frac_of_sustained": round(ach_f / peaks["bf16_tflops_sustained"], 4) if ach_f else None,
-            "flop_per_launch": f_fwd, "ms_per_launch": round(gemm_fwd_ms / max(gemm_fwd_n, 1), 5),
-            "traffic": traffic,
-            "backward_gemm": {"achieved": round(ach_b, 2) if ach_b else None,
-                              "frac": round(ach_b / pk, 4) if ach_b else None, "flop_per_launch": f_bwd,
-                              "ms_per_launch": round(gemm_bwd_ms / max(gemm_bwd_n, 1), 5)},
+            "frac_of_sustained": round(dom["achieved"] / peaks["bf16_tflops_sustained"], 4) if dom else None,
+            "flop_per_launch": dom["flop_per_step"] if dom else None,
+            "ms_per_launch": dom["ms_per_launch"] if dom else None,
+            "traffic": (traffic or {}).get("dx" if dom_is_dx else "forward") if isinstance(traffic, dict) else None,
+            "other_gemm": dict(other or {}, kernel="lora_mma_kernel (forward GEMM)" if dom_is_dx
+                               else "lora_mma_kernel (dX GEMM)",
+                               traffic=(traffic or {}).get("forward" if dom_is_dx else "dx")
+                               if isinstance(traffic, dict) else None),
             "step_frac": round(value / world / pk, 4)}
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(tot_ms / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.config, "M": M, "d_in": d_in, "d_out": d_out, "r": r,
-                       "alpha": cfg["alpha"], "act": act, "parallelism": f"replicas x{world}",
+            "config": {"workload": args.config, "M": lay.M, "d_in": lay.d_in, "d_out": lay.d_out, "r": lay.r,
+                       "alpha": cfg["alpha"], "act": lay.act, "parallelism": f"replicas x{world}",
                        "l2": "flushed before each timed step (512 MiB write)",
-                       **({"dropout": p_drop} if p_drop is not None else {})},
-            "roofline": roof, "gpu_launches": int(launches),
+                       **({"dropout": lay.p_drop} if lay.p_drop is not None else {})},
+            "roofline": roof, "gpu_launches": r["launches"],
             "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
-            "clocks": clk}
+            "clocks": r["clocks"]}
+    if world == 1 and args.config == "q_proj" and not args.no_workloads:
+        # every other workload of the build, each timed on its own (N = 1)
+        del lay
+        torch.cuda.empty_cache()
+        wl = {}
+
+        def entry(name, fn):
+            # a workload that fails is reported as such; the others still run
+            try:
+                wl[name] = fn()
+            except Exception as e:  # noqa: BLE001
+                wl[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        for name in ("tiny", "v_proj"):
+            entry(name, lambda name=name: measure_layer_workload(L, name, local, flush, peaks=peaks))
+        entry("mlp", lambda: measure_mlp(L, local, flush, peaks=peaks))
+        for name in ("small_m", "small_m_ragged"):
+            entry(name, lambda name=name: measure_small_m(L, name, local, flush, peaks=peaks)[0])
+        entry("lm_head_ce",
+              lambda: measure_ce(L, dict(seeded_inputs.CONFIGS["lm_head_ce"]), local, flush, peaks=peaks)[0])
+        line["workloads"] = wl
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:

@@ -441,6 +441,61 @@ lora_status_t lora_linear_bwd_rope(const lora_linear_desc* desc, const lora_rope
                                    float* dXn, int accumulate, float* dA, float* dB, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Output projection fused with the cross-entropy loss.  "Swift-All一文详解：
+ * 如何用Liger-Kernel提升训练效率", 2.2 (3) "CrossEntropy Loss 与最后一层 Logits
+ * 计算融合": the loss is computed together with the last layer's logits, in a
+ * numerically stable way, and its gradient is taken straight from the
+ * previous layer's output without the full probability distribution.  The
+ * quantity is the usual language-model loss:
+ *     z_m  = h_m W^T                         logits of token m (V classes)
+ *     loss = (1/N) sum over valid m of (logsumexp(z_m) - z_m[y_m])
+ *     dh_m = d(loss) * (softmax(z_m) - onehot(y_m)) / N    (0 for ignored m)
+ * with N the number of valid tokens (0 <= y_m < V; y_m < 0 marks a token to
+ * ignore; with no valid token the loss and dh are 0).  W (V x d) is frozen:
+ * only dh is returned.  No bias.
+ * How it runs: the forward is one tcgen05 GEMM over 256-token x 256-entry
+ * tiles whose epilogue reduces each token's logits to a running (max, sum of
+ * exp) per 128-entry block and picks up z[y]; no logit reaches memory.  Two
+ * small kernels combine the blocks (log-sum-exp per token) and take the mean
+ * in a fixed order.  The backward recomputes the logits chunk by chunk of
+ * tokens, turns them into the bf16 gradient (softmax - onehot) * d(loss) / N
+ * in the epilogue, and multiplies that chunk by W (K = V) for dh.
+ * Conventions: H [M x d] bf16 and W [V x d] bf16 row-major, 16-byte aligned;
+ * d % 8 == 0 and V % 8 == 0 (LORA_ERR_ALIGNMENT); labels int32 [M], lse fp32
+ * [M], loss and dloss fp32 scalars, all device, 4-byte aligned.  A label >= V
+ * sets status bit 0x2 and that token is ignored.
+ * ------------------------------------------------------------------------ */
+typedef struct lora_ce_desc {
+    int64_t M;     /* tokens */
+    int64_t d;     /* hidden size (features of h) */
+    int64_t V;     /* vocabulary size (rows of W) */
+} lora_ce_desc;
+
+/* Bytes of device workspace lora_linear_ce_fwd (0) or lora_linear_ce_bwd (1)
+ * needs: the forward holds 8 bytes per token and 128-entry block of the
+ * vocabulary plus 8 bytes per token; the backward holds the gradient of the
+ * logits of one chunk of at most 8192 tokens (chunk * V * 2 bytes).  The
+ * backward size is never below the forward size.  0 for an invalid desc. */
+size_t lora_linear_ce_workspace_size(const lora_ce_desc* desc, int for_backward);
+
+/* Forward.  H, W (device, read); labels [M] (device, read); loss: device fp32
+ * scalar (written: the mean over valid tokens); lse: device fp32 [M] (written:
+ * each token's log-sum-exp, the backward's input).  M == 0 writes loss = 0 and
+ * needs no H, labels or lse.  workspace >= lora_linear_ce_workspace_size(desc,
+ * 0), 16-byte aligned (LORA_ERR_WORKSPACE); its header's status word as for
+ * the layer.  Asynchronous on `stream`. */
+lora_status_t lora_linear_ce_fwd(const lora_ce_desc* desc, const void* H, const void* W, const int32_t* labels,
+                                 float* loss, float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward: dH [M x d] bf16 (device, written) = d(loss) * dloss/dH with
+ * *dloss (a device fp32 scalar, e.g. autograd's incoming gradient) as the
+ * upstream factor.  lse: the forward's output.  Other arguments as the
+ * forward; workspace >= lora_linear_ce_workspace_size(desc, 1). */
+lora_status_t lora_linear_ce_bwd(const lora_ce_desc* desc, const void* H, const void* W, const int32_t* labels,
+                                 const float* lse, const float* dloss, void* dH, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -49,7 +49,8 @@ EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_li
             "lora_linear_workspace_size_dropout", "lora_linear_fwd_dropout", "lora_linear_bwd_dropout",
             "lora_linear_w4_tiled_bytes", "lora_linear_w4_tile", "lora_linear_fwd_w4_tiled",
             "lora_linear_rmsnorm_fwd", "lora_linear_rmsnorm_bwd", "lora_linear_workspace_size_rope",
-            "lora_linear_fwd_rope", "lora_linear_bwd_rope")
+            "lora_linear_fwd_rope", "lora_linear_bwd_rope", "lora_linear_ce_workspace_size",
+            "lora_linear_ce_fwd", "lora_linear_ce_bwd")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -61,6 +62,11 @@ class LoraRopeDesc(ctypes.Structure):
     """Rotary tables: pos (int32 [M]), cos / sin (fp32 [n_pos x head_dim/2]) device pointers."""
     _fields_ = [("pos", ctypes.c_void_p), ("cos", ctypes.c_void_p), ("sin", ctypes.c_void_p),
                 ("n_pos", ctypes.c_int64), ("head_dim", ctypes.c_int32)]
+
+
+class LoraCeDesc(ctypes.Structure):
+    """Output projection + cross-entropy: M tokens, hidden size d, vocabulary V."""
+    _fields_ = [("M", ctypes.c_int64), ("d", ctypes.c_int64), ("V", ctypes.c_int64)]
 
 
 class LoraError(RuntimeError):
@@ -135,6 +141,13 @@ def _load():
     lib.lora_linear_fwd_rope.restype = i32
     lib.lora_linear_bwd_rope.argtypes = [dp, rp] + [vp] * 7 + [i32, vp, vp] + [vp, sz, vp]
     lib.lora_linear_bwd_rope.restype = i32
+    cp = ctypes.POINTER(LoraCeDesc)
+    lib.lora_linear_ce_workspace_size.argtypes = [cp, i32]
+    lib.lora_linear_ce_workspace_size.restype = sz
+    lib.lora_linear_ce_fwd.argtypes = [cp] + [vp] * 5 + [vp, sz, vp]
+    lib.lora_linear_ce_fwd.restype = i32
+    lib.lora_linear_ce_bwd.argtypes = [cp] + [vp] * 6 + [vp, sz, vp]
+    lib.lora_linear_ce_bwd.restype = i32
     return lib
 
 
@@ -275,6 +288,56 @@ def lora_linear_bwd_rope(desc, rope, dY, X, W, A, B, T_save, dXn, accumulate, dA
     return int(_lib.lora_linear_bwd_rope(ctypes.byref(desc), None if rope is None else ctypes.byref(rope), dY, X, W,
                                          A, B, T_save, dXn, int(accumulate), dA, dB, workspace, workspace_bytes,
                                          stream))
+
+
+# Output projection fused with the cross-entropy loss.
+def make_ce_desc(M, d, V) -> LoraCeDesc:
+    return LoraCeDesc(int(M), int(d), int(V))
+
+
+def lora_linear_ce_workspace_size(desc, for_backward) -> int:
+    return int(_lib.lora_linear_ce_workspace_size(ctypes.byref(desc), int(for_backward)))
+
+
+def lora_linear_ce_fwd(desc, H, W, labels, loss, lse, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_ce_fwd(ctypes.byref(desc), H, W, labels, loss, lse, workspace, workspace_bytes,
+                                       stream))
+
+
+def lora_linear_ce_bwd(desc, H, W, labels, lse, dloss, dH, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_ce_bwd(ctypes.byref(desc), H, W, labels, lse, dloss, dH, workspace, workspace_bytes,
+                                       stream))
+
+
+def linear_cross_entropy(H, W, labels, workspace=None, stream=None):
+    """(loss, lse): the mean cross-entropy of the logits H W^T against int32
+    labels (below 0: ignored), for bf16 H [M x d] and W [V x d] on the current
+    device.  lse [M] fp32 is the backward's input."""
+    import torch
+    M, d = H.shape
+    V = W.shape[0]
+    desc = make_ce_desc(M, d, V)
+    ws = (workspace or Workspace(lora_linear_ce_workspace_size(desc, 0), H.device, stream)).ensure(
+        lora_linear_ce_workspace_size(desc, 0), stream)
+    loss = torch.empty((), dtype=torch.float32, device=H.device)
+    lse = torch.empty(M, dtype=torch.float32, device=H.device)
+    _check(lora_linear_ce_fwd(desc, _ptr(H), W.data_ptr(), _ptr(labels), loss.data_ptr(), _ptr(lse),
+                              ws.buf.data_ptr(), ws.nbytes, _stream_handle(stream)), "lora_linear_ce_fwd")
+    return loss, lse
+
+
+def linear_cross_entropy_backward(H, W, labels, lse, dloss, workspace=None, stream=None):
+    """dH (bf16 [M x d]) = dloss * d(loss)/dH; dloss a 0-d fp32 device tensor."""
+    import torch
+    M, d = H.shape
+    V = W.shape[0]
+    desc = make_ce_desc(M, d, V)
+    ws = (workspace or Workspace(lora_linear_ce_workspace_size(desc, 1), H.device, stream)).ensure(
+        lora_linear_ce_workspace_size(desc, 1), stream)
+    dH = torch.empty((M, d), dtype=torch.bfloat16, device=H.device)
+    _check(lora_linear_ce_bwd(desc, _ptr(H), W.data_ptr(), _ptr(labels), _ptr(lse), dloss.data_ptr(), _ptr(dH),
+                              ws.buf.data_ptr(), ws.nbytes, _stream_handle(stream)), "lora_linear_ce_bwd")
+    return dH
 
 
 def lora_linear_timing_enable(enable: int) -> int:

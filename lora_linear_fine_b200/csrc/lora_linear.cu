@@ -23,6 +23,7 @@
 #include "lora_w4.cuh"
 #include "lora_dropout.cuh"
 #include "lora_norm_rope.cuh"
+#include "lora_ce.cuh"
 
 namespace {
 
@@ -1616,7 +1617,12 @@ lora_status_t lora_linear_rmsnorm_fwd(const void* X, const void* g, int64_t M, i
   DevInfo dev;
   LORA_TRY(check_arch(&dev));
   if (M == 0) return LORA_OK;
-  launch_k(rmsnorm_fwd_kernel, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
+  // rows of up to 4096 features stay in registers between the two passes
+  const int64_t nv = d / 8;
+  auto kern = nv <= 32 * 4 ? rmsnorm_fwd_reg_kernel<4>
+            : nv <= 32 * 8 ? rmsnorm_fwd_reg_kernel<8>
+            : nv <= 32 * 16 ? rmsnorm_fwd_reg_kernel<16> : rmsnorm_fwd_kernel;
+  launch_k(kern, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
            false, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(g),
            static_cast<long long>(M), static_cast<int>(d), static_cast<double>(eps), static_cast<__nv_bfloat16*>(Xn),
            rstd);
@@ -1675,6 +1681,198 @@ lora_status_t lora_linear_bwd_rope(const lora_linear_desc* d, const lora_rope_de
   const uint8_t* masks[2] = {nullptr, nullptr};
   return bwd_core(d, dY, X, W, A, B, nullptr, nullptr, nullptr, T_save, nullptr, nullptr, dA, dB, nullptr, nullptr,
                   workspace, workspace_bytes, stream, Xl, masks, rope != nullptr ? &t : nullptr, dXn, accumulate);
+}
+
+
+// ---------------------------------------------------------------------------
+// Output projection fused with the cross-entropy loss (lora_ce.cuh and the
+// kMEpiCeFwd / kMEpiCeGrad epilogues of lora_mma.cuh)
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+// Tokens per backward chunk: the chunk's bf16 logit gradient [chunk x V] is
+// the only per-token buffer of the backward (2.1 GB at 8192 tokens and
+// V = 128256), and the dH GEMM of a chunk of 8192 tokens at d = 4096 has 512
+// CTA-pair tiles (7 waves of 74 pairs).
+constexpr int64_t kCeChunkTokens = 8192;
+
+struct CePlan {
+  int n_tiles = 0;        // 256-column vocabulary tiles
+  int64_t chunk = 0;      // tokens per backward chunk
+  size_t part = 0, zlab = 0, loss_tok = 0, scale = 0, dz = 0, total = 0;
+};
+
+lora_status_t check_ce_desc(const lora_ce_desc* d) {
+  if (d == nullptr) return LORA_ERR_INVALID_ARG;
+  if (d->M < 0 || d->d <= 0 || d->V <= 0) return LORA_ERR_INVALID_ARG;
+  if (d->M > (int64_t(1) << 31) - 1 || d->d > (int64_t(1) << 30) || d->V > (int64_t(1) << 30))
+    return LORA_ERR_UNSUPPORTED;
+  if (d->d % 8 != 0 || d->V % 8 != 0) return LORA_ERR_ALIGNMENT;
+  return LORA_OK;
+}
+
+CePlan ce_plan(const lora_ce_desc* d, bool backward) {
+  CePlan P;
+  const int64_t M = d->M > 0 ? d->M : 1;
+  P.n_tiles = static_cast<int>(ceil_div(d->V, 256));
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  if (!backward) {
+    P.part = take(static_cast<size_t>(2 * P.n_tiles) * M * sizeof(float2));
+    P.zlab = take(static_cast<size_t>(M) * 4);
+    P.loss_tok = take(static_cast<size_t>(M) * 4);
+  } else {
+    P.scale = take(4);
+    P.chunk = M < kCeChunkTokens ? M : kCeChunkTokens;
+    P.dz = take(static_cast<size_t>(P.chunk) * d->V * 2);
+  }
+  P.total = off;
+  return P;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// The logits GEMM of rows [0, M) of H against all of W: forward (kMEpiCeFwd)
+// or gradient recompute (kMEpiCeGrad).
+template <int kEpi>
+lora_status_t ce_logit_gemm(const void* H, const void* W, int64_t M, int64_t d, int64_t V, const CeParams& ce,
+                            void* dz, uint32_t* status, int sms, cudaStream_t st) {
+  MmaParams p;
+  std::memset(&p, 0, sizeof(p));
+  const bool pair = pair_kernel_enabled() && M > 128;
+  if (!make_tm(&p.tm_a[0], H, d, M, d, 64, 128) || !make_tm(&p.tm_w[0], W, d, V, d, 64, pair ? 128 : 256))
+    return LORA_ERR_CUDA;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(V);
+  p.K = static_cast<int>(d);
+  p.lora_ksteps = 0;
+  p.out = static_cast<__nv_bfloat16*>(dz);
+  p.status = status;
+  p.ce = ce;
+  p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
+  p.n_tiles = static_cast<int>(ceil_div(V, 256));
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  set_raster(p, pair, 2.0 * M * d, 2.0 * V * d);
+  timing_begin(0, st);
+  const lora_status_t rs = launch_mma_any<false, 1, kEpi>(pair, p, sms, st);
+  timing_end(0, st);
+  return rs;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lora_linear_ce_workspace_size(const lora_ce_desc* desc, int for_backward) {
+  if (check_ce_desc(desc) != LORA_OK) return 0;
+  const size_t fwd = ce_plan(desc, false).total;
+  if (for_backward == 0) return fwd;
+  const size_t bwd = ce_plan(desc, true).total;
+  return bwd > fwd ? bwd : fwd;
+}
+
+lora_status_t lora_linear_ce_fwd(const lora_ce_desc* d, const void* H, const void* W, const int32_t* labels,
+                                 float* loss, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_ce_desc(d));
+  if (W == nullptr || loss == nullptr || (d->M > 0 && (H == nullptr || labels == nullptr || lse == nullptr)))
+    return LORA_ERR_INVALID_ARG;
+  if ((H && !aligned16(H)) || !aligned16(W) || (labels && !aligned4(labels)) || !aligned4(loss) ||
+      (lse && !aligned4(lse)))
+    return LORA_ERR_ALIGNMENT;
+  const CePlan P = ce_plan(d, false);
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
+  if (workspace == nullptr || workspace_bytes < P.total || !aligned16(workspace)) return LORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->M == 0) {   // no token: the mean over no valid token is 0
+    if (cudaMemsetAsync(loss, 0, sizeof(float), st) != cudaSuccess) return cuda_error("cudaMemsetAsync(loss)");
+    return LORA_OK;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  CeParams ce{};
+  ce.labels = labels;
+  ce.part = reinterpret_cast<float2*>(ws + P.part);
+  ce.zlab = reinterpret_cast<float*>(ws + P.zlab);
+  // 1. logits tile by tile on the tensor cores; per token and 128-column block
+  //    the epilogue keeps (max, sum exp) and the label's logit
+  LORA_TRY(ce_logit_gemm<kMEpiCeFwd>(H, W, d->M, d->d, d->V, ce, nullptr, status, dev.sms, st));
+  // 2. lse and each token's loss; 3. the mean over valid tokens
+  const int M = static_cast<int>(d->M);
+  launch_k(ce_combine_kernel, dim3(grid_for(M, 256, dev.sms)), dim3(256), 0, st, false,
+           static_cast<const float2*>(ce.part), 2 * P.n_tiles, M, static_cast<int>(d->V), labels,
+           static_cast<const float*>(ce.zlab), lse, reinterpret_cast<float*>(ws + P.loss_tok), status);
+  LORA_TRY(check_launch("ce_combine_kernel"));
+  launch_k(ce_mean_kernel, dim3(1), dim3(kCeMeanThreads), 0, st, false,
+           static_cast<const float*>(reinterpret_cast<float*>(ws + P.loss_tok)), labels, M, static_cast<int>(d->V),
+           loss);
+  return check_launch("ce_mean_kernel");
+}
+
+lora_status_t lora_linear_ce_bwd(const lora_ce_desc* d, const void* H, const void* W, const int32_t* labels,
+                                 const float* lse, const float* dloss, void* dH, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_ce_desc(d));
+  if (W == nullptr || dloss == nullptr ||
+      (d->M > 0 && (H == nullptr || labels == nullptr || lse == nullptr || dH == nullptr)))
+    return LORA_ERR_INVALID_ARG;
+  if ((H && !aligned16(H)) || !aligned16(W) || (dH && !aligned16(dH)) || (labels && !aligned4(labels)) ||
+      (lse && !aligned4(lse)) || !aligned4(dloss))
+    return LORA_ERR_ALIGNMENT;
+  const CePlan P = ce_plan(d, true);
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
+  if (workspace == nullptr || workspace_bytes < P.total || !aligned16(workspace)) return LORA_ERR_WORKSPACE;
+  if (d->M == 0) return LORA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* scale = reinterpret_cast<float*>(ws + P.scale);
+  void* dz = ws + P.dz;
+  const int64_t M = d->M, dm = d->d, V = d->V;
+  // 1. scale = d(loss) / (number of valid tokens)
+  launch_k(ce_scale_kernel, dim3(1), dim3(kCeMeanThreads), 0, st, false, labels, static_cast<int>(M),
+           static_cast<int>(V), dloss, scale, status);
+  LORA_TRY(check_launch("ce_scale_kernel"));
+  for (int64_t m0 = 0; m0 < M; m0 += P.chunk) {
+    const int64_t C = (M - m0) < P.chunk ? (M - m0) : P.chunk;
+    const void* Hc = static_cast<const uint8_t*>(H) + static_cast<size_t>(m0) * dm * 2;
+    // 2. the chunk's logits again, turned into the gradient of the loss with
+    //    respect to them, bf16 [C x V]
+    CeParams ce{};
+    ce.labels = labels + m0;
+    ce.lse = lse + m0;
+    ce.scale = scale;
+    LORA_TRY(ce_logit_gemm<kMEpiCeGrad>(Hc, W, C, dm, V, ce, dz, status, dev.sms, st));
+    // 3. dH = dz W: K = V, W [V x d] read in place as the MN-major operand
+    MmaParams g;
+    std::memset(&g, 0, sizeof(g));
+    const bool pair = pair_kernel_enabled() && C > 128;
+    if (!make_tm(&g.tm_a[0], dz, V, C, V, 64, 128) || !make_tm(&g.tm_w[0], W, dm, V, dm, 64, 64))
+      return LORA_ERR_CUDA;
+    g.b_mn = 1;
+    g.M = static_cast<int>(C);
+    g.N = static_cast<int>(dm);
+    g.K = static_cast<int>(V);
+    g.lora_ksteps = 0;
+    g.out = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(dH) + static_cast<size_t>(m0) * dm * 2);
+    g.status = status;
+    g.m_tiles = static_cast<int>(ceil_div(C, pair ? 256 : 128));
+    g.n_tiles = static_cast<int>(ceil_div(dm, 256));
+    g.num_tiles = g.m_tiles * g.n_tiles;
+    set_raster(g, pair, 2.0 * C * V, 2.0 * V * dm);
+    timing_begin(1, st);
+    const lora_status_t rs = launch_mma_any<true, 1, kMEpiGrad>(pair, g, dev.sms, st);
+    timing_end(1, st);
+    LORA_TRY(rs);
+  }
+  return LORA_OK;
 }
 
 }  // extern "C"

@@ -45,7 +45,25 @@ constexpr int kMmaThreads = 320;
 // kEpi values
 // kMEpiRope: identity, then the rotary embedding of each token's heads on the
 // fp32 accumulator (lora_norm_rope.cuh) before the bf16 store.
-enum MmaEpi : int { kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5 };
+// kMEpiCeFwd: the output projection's logits z = H W^T of a 256 x 256 tile are
+// reduced in the epilogue to one (max, sum of exp(z - max)) pair per token and
+// 128-column block, and the label's logit is picked up; no logit is stored.
+// kMEpiCeGrad: the same logits recomputed and turned into the cross-entropy
+// gradient (exp(z - lse) - onehot(label)) * scale, stored as bf16.
+enum MmaEpi : int {
+  kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5,
+  kMEpiCeFwd = 6, kMEpiCeGrad = 7
+};
+
+// Output projection fused with the cross-entropy loss (rows = tokens of this
+// launch, columns = vocabulary entries).
+struct CeParams {
+  const int32_t* labels;  // [M] label per token; < 0 ignored (also >= N: flagged by the combine kernel)
+  float2* part;           // kMEpiCeFwd: [2 * n_tiles][M] (max, sum exp(z - max)) per 128-column block
+  float* zlab;            // kMEpiCeFwd: [M] z[label] (written by the block holding the label)
+  const float* lse;       // kMEpiCeGrad: [M] log-sum-exp of each token's logits
+  const float* scale;     // kMEpiCeGrad: device scalar, d(loss) / (number of valid tokens)
+};
 
 struct MmaParams {
   CUtensorMap tm_a[2];    // M-side operand per pair      fwd: X            bwd: dZ_j
@@ -65,6 +83,7 @@ struct MmaParams {
   RopeTables rope;        // kMEpiRope: positions and cos / sin tables (half = 32 or 64)
   float* out_f32;         // backward: fp32 dX [M x N] instead of the bf16 `out` (null: bf16)
   int out_acc;            // with out_f32: dX += the product (else dX = the product)
+  CeParams ce;            // kMEpiCeFwd / kMEpiCeGrad
 };
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
@@ -501,6 +520,73 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               pk.w = pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7]));
               if (col0 + cc + j < p.N) st_global_v4_hint(p.out + base + cc + j, pk, pol_out);
             }
+          }
+        }
+      } else if constexpr (kEpi == kMEpiCeFwd) {
+        // This thread's token row and 128 vocabulary columns [col0, col0 + 128):
+        // a running max and sum of exp(z - max) over four 32-column loads
+        // (columns past N count as -inf), and z[label] if the label is here.
+        const int col0 = nt * 256 + h * 128;
+        const int lab = row_ok ? __ldg(p.ce.labels + row) : -1;
+        float mx = -INFINITY, se = 0.0f, zl = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tl + h * 128 + 32 * c, v);
+          tmem_wait_ld();
+          if (c == 3) release_acc();
+          const int cb = col0 + 32 * c;
+          float cm = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float z = (cb + i < p.N) ? __uint_as_float(v[i]) : -INFINITY;
+            v[i] = __float_as_uint(z);
+            cm = fmaxf(cm, z);
+            if (cb + i == lab) zl = z;
+          }
+          if (cm == -INFINITY) continue;            // the whole chunk is past N
+          const float nm = fmaxf(mx, cm);
+          se *= __expf(mx - nm);                    // exp(-inf) = 0 on the first chunk
+#pragma unroll
+          for (int i = 0; i < 32; ++i) se += __expf(__uint_as_float(v[i]) - nm);
+          mx = nm;
+        }
+        if (row_ok) {
+          p.ce.part[static_cast<size_t>(nt * 2 + h) * p.M + row] = make_float2(mx, se);
+          if (lab >= col0 && lab < col0 + 128 && lab < p.N) p.ce.zlab[row] = zl;
+        }
+      } else if constexpr (kEpi == kMEpiCeGrad) {
+        // (exp(z - lse) - [column == label]) * scale for this thread's row and
+        // 128 columns, bf16, in four 32-column pieces; ignored tokens give 0.
+        const int col0 = nt * 256 + h * 128;
+        const int lab = row_ok ? __ldg(p.ce.labels + row) : -1;
+        const float lse = row_ok ? __ldg(p.ce.lse + row) : 0.0f;
+        const float sc = (row_ok && lab >= 0 && lab < p.N) ? __ldg(p.ce.scale) : 0.0f;
+        const size_t base = static_cast<size_t>(row) * p.N + col0;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tl + h * 128 + 32 * c, v);
+          tmem_wait_ld();
+          if (c == 3) release_acc();
+          if (!row_ok) continue;
+          const int cb = col0 + 32 * c;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            float g[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float pz = __expf(__uint_as_float(v[j + e]) - lse);
+              g[e] = (pz - (cb + j + e == lab ? 1.0f : 0.0f)) * sc;
+            }
+            uint4 pk;
+            pk.x = pack_bf16x2(g[0], g[1]);
+            pk.y = pack_bf16x2(g[2], g[3]);
+            pk.z = pack_bf16x2(g[4], g[5]);
+            pk.w = pack_bf16x2(g[6], g[7]);
+            if (cb + j < p.N) st_global_v4_hint(p.out + base + 32 * c + j, pk, pol_out);
           }
         }
       } else {

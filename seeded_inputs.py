@@ -20,6 +20,11 @@ are used, every tensor is drawn here):
 * dropout masks on the adapter input: each element of X kept with probability
   1 - p, packed eight per byte (bit j of byte b, least significant first, is
   element 8 b + j): uint8 tokens x d_in/8.
+* output projection + cross-entropy: hidden states H ~ N(0, 1) (tokens x d),
+  the frozen output projection W_out ~ N(0, 1/d) (V x d), so that the logits
+  H W_out^T are about N(0, 1); labels int32 uniform in [0, V), a given
+  fraction of them (5 % by default) replaced by -100 (tokens to ignore, as
+  padding would be).
 * attention-input block (RMSNorm, then the q, k, v projections, q and k
   rotated): the norm's weight g ~ U(0.5, 1.5) (bf16, d_in); each projection j
   has its own W, A, B, dY drawn as above from the seed (seed, j); token
@@ -44,6 +49,7 @@ _TENSOR_IDS = {
     "Wq": 9, "Ws": 10, "Wq_up": 11, "Ws_up": 12,
     "mask": 13, "mask_up": 14,
     "g": 15, "pos": 16,
+    "H": 17, "W_out": 18, "labels": 19, "ignore": 20,
 }
 
 ACTS = ("identity", "silu", "swiglu")
@@ -62,6 +68,9 @@ CONFIGS = {
     "small_m_w4": dict(M=16, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity", weight="w4"),
     # q_proj with dropout p = 0.1 on the adapter input (the mask is drawn here)
     "q_proj_dropout": dict(M=16384, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity", dropout=0.1),
+    # the Llama-3-8B output projection (vocabulary 128256) fused with the
+    # cross-entropy loss, 8192 tokens (M = tokens, d_in = hidden, d_out = V)
+    "lm_head_ce": dict(M=8192, d_in=4096, d_out=128256, r=0, alpha=0.0, act="ce"),
     # RMSNorm -> q (4096), k (1024), v (1024) LoRA projections, q and k rotated
     # (32 query and 8 key/value heads of 128); 4 sequences of 4096 tokens
     "qkv_rmsnorm_rope": dict(M=16384, d_in=4096, d_out=4096, r=8, alpha=16.0, act="identity",
@@ -117,6 +126,16 @@ def draw_w4(name: str, d_out: int, d_in: int, seed: int):
     gs = _rng(seed, "Ws" + suffix)
     Ws = f64_to_bf16_bits(gs.uniform(0.5, 1.5, size=(d_in // 64, d_out)) / (4.6 * np.sqrt(d_in)))
     return Wq, Ws
+
+
+def draw_ce(M: int, d: int, V: int, seed: int, ignore_frac: float = 0.05, h_scale: float = 1.0):
+    """Inputs of the output projection + cross-entropy: (H bf16 bits [M x d],
+    W_out bf16 bits [V x d], labels int32 [M]); ``h_scale`` widens the logits."""
+    H = f64_to_bf16_bits(_rng(seed, "H").standard_normal((M, d)) * h_scale)
+    W = f64_to_bf16_bits(_rng(seed, "W_out").standard_normal((V, d)) / np.sqrt(d))
+    labels = _rng(seed, "labels").integers(0, V, size=M).astype(np.int32)
+    labels[_rng(seed, "ignore").random(M) < ignore_frac] = -100
+    return H, W, labels
 
 
 def draw_mask(name: str, M: int, d_in: int, p_drop: float, seed: int) -> np.ndarray:

@@ -214,3 +214,31 @@ def test_norm_and_rope_argument_checks(lib):
     assert bwd(dXn=None) == 1
     assert bwd(dXn=24) == 2
     assert bwd(rope=lib.make_rope_desc(16, 16, 16, 32, 96)) == 3
+
+
+def test_cross_entropy_argument_checks(lib):
+    """Output projection + cross-entropy: sizes, required pointers and
+    alignment are checked on the host before any device query."""
+    d = lib.make_ce_desc(64, 256, 1000)
+    f = lib.lora_linear_ce_workspace_size(d, 0)
+    b = lib.lora_linear_ce_workspace_size(d, 1)
+    assert b >= f > 2 * 4 * 64 * 8                     # (max, sum) per token and 128-entry block
+    assert b >= 64 * 1000 * 2                          # the chunk's bf16 logit gradient
+    assert lib.lora_linear_ce_workspace_size(lib.make_ce_desc(64, 252, 1000), 0) == 0    # d % 8
+    assert lib.lora_linear_ce_workspace_size(lib.make_ce_desc(64, 256, 1001), 1) == 0    # V % 8
+    assert lib.lora_linear_ce_workspace_size(lib.make_ce_desc(-1, 256, 1000), 0) == 0
+    fwd = lambda desc=d, H=16, W=16, lab=16, loss=16, lse=16: lib.lora_linear_ce_fwd(desc, H, W, lab, loss, lse, 16,
+                                                                                   1 << 30, None)
+    assert fwd(desc=lib.make_ce_desc(64, 252, 1000)) == 2
+    assert fwd(desc=lib.make_ce_desc(64, 256, 1004)) == 2       # V % 8: ALIGNMENT
+    assert fwd(H=None) == 1
+    assert fwd(lab=None) == 1
+    assert fwd(loss=None) == 1
+    assert fwd(lse=None) == 1
+    assert fwd(H=24) == 2
+    assert fwd(lab=18) == 2
+    bwd = lambda H=16, lse=16, dl=16, dH=16: lib.lora_linear_ce_bwd(d, H, 16, 16, lse, dl, dH, 16, 1 << 30, None)
+    assert bwd(dl=None) == 1
+    assert bwd(dH=None) == 1
+    assert bwd(dH=24) == 2
+    assert bwd(lse=None) == 1
