@@ -605,16 +605,16 @@ bool pair_kernel_enabled() {
   return v == 1;
 }
 
-template <bool kPair, bool kBwd, int kNPair, int kEpi>
+template <bool kPair, bool kBwd, int kNPair, int kEpi, int kTN = 256>
 lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
-  using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
-  auto k = lora_mma_kernel<kPair, kBwd, kNPair, kEpi>;
+  using C = MmaCfg<kPair, kBwd, kNPair, kEpi, kTN>;
+  auto k = lora_mma_kernel<kPair, kBwd, kNPair, kEpi, kTN>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return cuda_error("cudaFuncSetAttribute(mma)");
   const int max_units = kPair ? sms / 2 : sms;
   const int units = p.num_tiles < max_units ? p.num_tiles : max_units;
-  LORA_LOG("mma pair=%d bwd=%d npair=%d epi=%d tiles=%d units=%d smem=%d stages=%d lora_ksteps=%d", (int)kPair,
-           (int)kBwd, kNPair, kEpi, p.num_tiles, units, C::kSmemBytes, C::kStages, p.lora_ksteps);
+  LORA_LOG("mma pair=%d bwd=%d npair=%d epi=%d tile_n=%d tiles=%d units=%d smem=%d stages=%d lora_ksteps=%d",
+           (int)kPair, (int)kBwd, kNPair, kEpi, kTN, p.num_tiles, units, C::kSmemBytes, C::kStages, p.lora_ksteps);
   const cudaError_t e = launch_k(k, dim3(static_cast<unsigned>(units * C::kCtas)), dim3(kMmaThreads), C::kSmemBytes,
                                  st, kPair, p);
   if (e != cudaSuccess) {
@@ -638,9 +638,24 @@ void set_raster(MmaParams& p, bool pair, double m_bytes, double n_bytes) {
   }
 }
 
-template <bool kBwd, int kNPair, int kEpi>
+template <bool kBwd, int kNPair, int kEpi, int kTN = 256>
 lora_status_t launch_mma_any(bool pair, const MmaParams& p, int sms, cudaStream_t st) {
-  return pair ? launch_mma<true, kBwd, kNPair, kEpi>(p, sms, st) : launch_mma<false, kBwd, kNPair, kEpi>(p, sms, st);
+  return pair ? launch_mma<true, kBwd, kNPair, kEpi, kTN>(p, sms, st)
+              : launch_mma<false, kBwd, kNPair, kEpi, kTN>(p, sms, st);
+}
+
+// Tile N of an identity GEMM (forward or bf16 dX): 128 when 128-wide tiles
+// fill the units' last wave clearly better than 256-wide ones (each unit runs
+// one tile at a time; the CTA pairs or CTAs are `units`).  A wave's
+// efficiency is tiles / (waves * units).
+int pick_tile_n(int64_t m_tiles, int64_t n_cols, int units) {
+  if (units < 1) return 256;
+  auto eff = [&](int tn) {
+    const int64_t tiles = m_tiles * ceil_div(n_cols, tn);
+    const int64_t waves = ceil_div(tiles, units);
+    return static_cast<double>(tiles) / static_cast<double>(waves * units);
+  };
+  return eff(128) > eff(256) + 0.05 ? 128 : 256;
 }
 
 // Failure-detection self-test: one thread waits, through the library's
@@ -1030,11 +1045,14 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   MmaParams p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = pair_kernel_enabled() && M > 128;
-  const int outc = swiglu ? 128 : 256;
-  const int brows = swiglu ? (pair ? 64 : 128) : (pair ? 128 : 256);   // N-side rows per CTA box
+  const int units = pair ? dev.sms / 2 : dev.sms;
+  const int tn = (d->act == LORA_ACT_IDENTITY && rope == nullptr)
+                     ? pick_tile_n(ceil_div(M, pair ? 256 : 128), d->d_out, units) : 256;
+  const int outc = swiglu ? 128 : tn;
+  const int brows = swiglu ? (pair ? 64 : 128) : (pair ? tn / 2 : tn);   // N-side rows per CTA box
   bool ok = make_tm(&p.tm_a[0], X, d->d_in, M, d->d_in, 64, 128);
   for (int j = 0; j < np; ++j) {
-    ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, (swiglu || pair) ? 128 : 256);
+    ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, swiglu ? 128 : brows);
     if (r > 0) {
       ok = ok && make_tm(&p.tm_la[j], ws + P.s16[j], r, M, r, 64, 128);
       ok = ok && make_tm(&p.tm_lb[j], Bp[j], r, d->d_out, r, 64, brows);
@@ -1061,7 +1079,10 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
     return rs;
   }
   switch (d->act) {
-    case LORA_ACT_IDENTITY: rs = launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st); break;
+    case LORA_ACT_IDENTITY:
+      rs = tn == 128 ? launch_mma_any<false, 1, kMEpiIdentity, 128>(pair, p, dev.sms, st)
+                     : launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st);
+      break;
     case LORA_ACT_SILU: rs = launch_mma_any<false, 1, kMEpiSilu>(pair, p, dev.sms, st); break;
     default: rs = launch_mma_any<false, 2, kMEpiSwiglu>(pair, p, dev.sms, st); break;
   }
@@ -1178,7 +1199,8 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
       const float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r : nullptr;
-      const long long n = d->d_out + (P.kmajor ? d->d_in : 0) + (Tj ? M : 0);   // one thread per row
+      // one thread per row and 8-column chunk
+      const long long n = (d->d_out + (P.kmajor ? d->d_in : 0) + (Tj ? M : 0)) * (r / 8);
       const __nv_bfloat16* Aj = static_cast<const __nv_bfloat16*>(Ap[j]);
       __nv_bfloat16* Atj = P.kmajor ? static_cast<__nv_bfloat16*>(at(P.at_[j])) : nullptr;
       if (f16)
@@ -1252,7 +1274,9 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     std::memset(&p, 0, sizeof(p));
     const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
-    const uint32_t brows = pair ? 128 : 256;   // N-side rows per CTA box (K-major)
+    const int units = pair ? dev.sms / 2 : dev.sms;
+    const int tn = f16 ? 256 : pick_tile_n(ceil_div(M, pair ? 256 : 128), d->d_in, units);
+    const uint32_t brows = static_cast<uint32_t>(pair ? tn / 2 : tn);   // N-side rows per CTA box (K-major)
     for (int j = 0; j < np; ++j) {
       ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
       if (P.kmajor) {
@@ -1278,7 +1302,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     p.z_save = nullptr;
     p.status = status;
     p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
-    p.n_tiles = static_cast<int>(ceil_div(d->d_in, 256));
+    p.n_tiles = static_cast<int>(ceil_div(d->d_in, tn));
     p.num_tiles = p.m_tiles * p.n_tiles;
     set_raster(p, pair, 2.0 * np * M * d->d_out, 2.0 * np * d->d_out * d->d_in);
     timing_begin(1, st);
@@ -1286,6 +1310,8 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     if (f16) {
       if (np == 2) rs = launch_mma_any<true, 2, kMEpiGradF16>(pair, p, dev.sms, st);
       else rs = launch_mma_any<true, 1, kMEpiGradF16>(pair, p, dev.sms, st);
+    } else if (tn == 128) {
+      rs = launch_mma_any<true, 1, kMEpiGrad, 128>(pair, p, dev.sms, st);
     } else {
       rs = launch_mma_any<true, 1, kMEpiGrad>(pair, p, dev.sms, st);
     }
@@ -1617,12 +1643,7 @@ lora_status_t lora_linear_rmsnorm_fwd(const void* X, const void* g, int64_t M, i
   DevInfo dev;
   LORA_TRY(check_arch(&dev));
   if (M == 0) return LORA_OK;
-  // rows of up to 4096 features stay in registers between the two passes
-  const int64_t nv = d / 8;
-  auto kern = nv <= 32 * 4 ? rmsnorm_fwd_reg_kernel<4>
-            : nv <= 32 * 8 ? rmsnorm_fwd_reg_kernel<8>
-            : nv <= 32 * 16 ? rmsnorm_fwd_reg_kernel<16> : rmsnorm_fwd_kernel;
-  launch_k(kern, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
+  launch_k(rmsnorm_fwd_kernel, dim3(norm_grid(M, dev)), dim3(32 * kNormWarps), 0, static_cast<cudaStream_t>(stream),
            false, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(g),
            static_cast<long long>(M), static_cast<int>(d), static_cast<double>(eps), static_cast<__nv_bfloat16*>(Xn),
            rstd);

@@ -86,17 +86,21 @@ struct MmaParams {
   CeParams ce;            // kMEpiCeFwd / kMEpiCeGrad
 };
 
-template <bool kPair, bool kBwd, int kNPair, int kEpi>
+// kTN: the tile's N (256, or 128 for the plain identity forward / dX when
+// 128-wide tiles fill the last wave of CTA pairs better).
+template <bool kPair, bool kBwd, int kNPair, int kEpi, int kTN = 256>
 struct MmaCfg {
+  static_assert(kTN == 256 || (kTN == 128 && (kEpi == kMEpiIdentity || kEpi == kMEpiGrad)),
+                "128-wide tiles serve the identity forward and the bf16 dX only");
   static constexpr bool kSwigluFwd = (!kBwd) && (kEpi == kMEpiSwiglu);
   static constexpr int kCtas = kPair ? 2 : 1;
   static constexpr int kTileM = 128 * kCtas;                 // rows per (pair) tile
-  static constexpr int kOutCols = kSwigluFwd ? 128 : 256;    // output columns per tile
+  static constexpr int kOutCols = kSwigluFwd ? 128 : kTN;    // output columns per tile
   static constexpr int kKPairs = kBwd ? kNPair : 1;          // projections walked along K
   static constexpr int kLoraProj = kNPair;                   // projections with a LoRA branch per tile
   static constexpr int kABytes = 128 * 64 * 2;               // 16 KB
-  static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
-  static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
+  static constexpr int kBRows = (kSwigluFwd ? 256 : kTN) / kCtas;   // N-side rows held per CTA
+  static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair) at N = 256
   static constexpr int kStageBytes = kABytes + kBBytes;
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
   // shared memory (4 KB per warp) so that global stores are row-contiguous.
@@ -105,7 +109,7 @@ struct MmaCfg {
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kEpiStageBytes + 2048;
-  static constexpr uint32_t kTmemCols = 512;                 // 2 accumulator buffers
+  static constexpr uint32_t kTmemCols = 2 * kTN;             // 2 accumulator buffers
   static_assert(kStages >= 3, "ring too shallow");
 };
 
@@ -139,9 +143,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
   else return mbar_wait(bar, parity, ctl);
 }
 
-template <bool kPair, bool kBwd, int kNPair, int kEpi>
+template <bool kPair, bool kBwd, int kNPair, int kEpi, int kTN = 256>
 __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_constant__ MmaParams p) {
-  using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
+  using C = MmaCfg<kPair, kBwd, kNPair, kEpi, kTN>;
   constexpr int S = C::kStages;
 
   extern __shared__ uint8_t smem_raw[];
@@ -291,10 +295,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       constexpr int kM = C::kTileM;
       // N-side operand MN-major only in a backward that reads W and A in place
       const bool bmn = kBwd && p.b_mn != 0;
-      const uint32_t kIdMain = bmn ? idesc_mma(kM, 256, false, true, kF16) : idesc_mma(kM, 256, false, false, kF16);
+      constexpr int kN = C::kSwigluFwd ? 256 : kTN;
+      const uint32_t kIdMain = bmn ? idesc_mma(kM, kN, false, true, kF16) : idesc_mma(kM, kN, false, false, kF16);
       // LoRA block: bf16 s*T/s*U against bf16 B (fwd) / A or A^T (bwd)
-      const uint32_t kIdLora = bmn ? idesc_mma(kM, 256, false, true, false)
-                                   : idesc_mma(kM, C::kSwigluFwd ? 128 : 256, false, false, false);
+      const uint32_t kIdLora = bmn ? idesc_mma(kM, kN, false, true, false)
+                                   : idesc_mma(kM, C::kSwigluFwd ? 128 : kN, false, false, false);
       constexpr uint16_t kBoth = 0x3;
       auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
         if constexpr (kPair) mma_bf16_pair(d, a, b, id, acc);
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         const uint32_t use = it >> 1;        // how many times this buffer was used before
         if (!wait_bar<kPair>(&acc_empty[buf], (use & 1u) ^ 1u, ctl)) break;
         tc_fence_after();
-        const uint32_t dacc = tbase + buf * 256;
+        const uint32_t dacc = tbase + buf * (C::kSwigluFwd ? 256 : kTN);
         const int nblocks = C::kKPairs * nkb + nlora;
         bool ok = true;
         for (int blk = 0; blk < nblocks; ++blk) {
@@ -371,7 +376,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
-      const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tl = tbase + buf * (C::kSwigluFwd ? 256 : kTN) + (static_cast<uint32_t>(q * 32) << 16);
       auto release_acc = [&]() {   // every lane's tcgen05.ld has completed (tmem_wait_ld)
         tc_fence_before();
         __syncwarp();
@@ -590,13 +595,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           }
         }
       } else {
-        uint32_t v[128];
+        constexpr int kHalf = kTN / 2;          // columns per epilogue thread
+        uint32_t v[kHalf];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tl + h * 128 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+        for (int c = 0; c < kHalf / 32; ++c)
+          tmem_ld32(tl + h * kHalf + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
         tmem_wait_ld();
         release_acc();
         if (!row_ok) continue;
-        const int col0 = nt * 256 + h * 128;
+        const int col0 = nt * kTN + h * kHalf;
         const size_t base = static_cast<size_t>(row) * p.N + col0;
         if constexpr (kBwd) {
           if (p.out_f32 != nullptr) {
@@ -604,7 +611,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             // gradients summed in a fixed order, one launch after another)
             float* dst = p.out_f32 + base;
 #pragma unroll
-            for (int c = 0; c < 128; c += 4) {
+            for (int c = 0; c < kHalf; c += 4) {
               if (col0 + c < p.N) {
                 float4 o = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
                                        __uint_as_float(v[c + 3]));
@@ -623,7 +630,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           }
         }
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
+        for (int c = 0; c < kHalf; c += 8) {
           uint4 pk;
           pk.x = pack_bf16x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
           pk.y = pack_bf16x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));

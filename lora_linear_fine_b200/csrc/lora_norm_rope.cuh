@@ -99,55 +99,6 @@ __global__ void __launch_bounds__(32 * kNormWarps)
   }
 }
 
-// The same for rows of at most 256 kV features: each lane issues all of its
-// row's kV 16-byte loads before the first use, keeps them in registers for
-// the second pass (no re-read of the row) and converts from there.  Same
-// arithmetic and rounding as rmsnorm_fwd_kernel, element by element.
-template <int kV>
-__global__ void __launch_bounds__(32 * kNormWarps)
-    rmsnorm_fwd_reg_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ g, long long M,
-                           int d, double eps, __nv_bfloat16* __restrict__ Xn, float* __restrict__ rstd) {
-  grid_dep_wait();
-  const int lane = threadIdx.x & 31;
-  const int nv = d / 8;
-  const uint4* gv = reinterpret_cast<const uint4*>(g);
-  for (long long row = blockIdx.x * static_cast<long long>(kNormWarps) + (threadIdx.x >> 5); row < M;
-       row += static_cast<long long>(gridDim.x) * kNormWarps) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + row * d);
-    uint4 v[kV];
-#pragma unroll
-    for (int j = 0; j < kV; ++j) {
-      const int c = lane + 32 * j;
-      v[j] = c < nv ? __ldcs(xr + c) : make_uint4(0u, 0u, 0u, 0u);   // streamed once: evict first
-    }
-    double ss = 0.0;
-#pragma unroll
-    for (int j = 0; j < kV; ++j) {
-      float f[8];
-      unpack_bf16x8(v[j], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fma(static_cast<double>(f[e]), static_cast<double>(f[e]), ss);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const double inv = 1.0 / sqrt(ss / static_cast<double>(d) + eps);
-    if (lane == 0) rstd[row] = static_cast<float>(inv);
-    uint4* yr = reinterpret_cast<uint4*>(Xn + row * d);
-#pragma unroll
-    for (int j = 0; j < kV; ++j) {
-      const int c = lane + 32 * j;
-      if (c >= nv) break;
-      float f[8], w[8];
-      unpack_bf16x8(v[j], f);
-      unpack_bf16x8(__ldg(gv + c), w);
-      __align__(16) __nv_bfloat16 o[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = bf16_from_f64((static_cast<double>(f[e]) * inv) * static_cast<double>(w[e]));
-      yr[c] = *reinterpret_cast<const uint4*>(o);
-    }
-  }
-}
-
 // dX [M x d] bf16 = rstd (g dx_n - x_hat mean(g dx_n x_hat)), x_hat = x rstd,
 // dx_n [M x d] fp32: the projections' input gradients summed in fp32 by their
 // dX GEMMs (three bf16 roundings before the sum would cost the bound on the

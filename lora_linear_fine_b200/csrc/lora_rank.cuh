@@ -365,8 +365,9 @@ __device__ __forceinline__ float from16(__half v) { return __half2float(v); }
 constexpr float kF16Max = 65504.0f;
 
 // Backward preparation in one launch, one thread per row of the small
-// operands (so that each thread moves whole 16-byte rows and every warp access
-// is coalesced): B^T ([r x d_out], bf16 or fp16), A^T ([d_in x r], bf16, the
+// operands and 8-column chunk (each thread moves one 16-byte piece of a row;
+// neighbouring threads take neighbouring rows, so the transposed writes are
+// coalesced): B^T ([r x d_out], bf16 or fp16), A^T ([d_in x r], bf16, the
 // K-major N-side operand of the dX LoRA block; skipped when At is null) and
 // the transposed hi/lo split of s*T ([r x ld]) from the forward's fp32 T
 // (skipped when Tsave is null).  r is a multiple of 8.
@@ -376,45 +377,45 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, 
                                 const float* __restrict__ Tsave, int M, float s, T* __restrict__ t_hi,
                                 T* __restrict__ t_lo, int ld, uint32_t* status) {
   grid_dep_wait();
+  // One thread per (row, 8-column chunk), rows fastest within a chunk so that
+  // the transposed stores of neighbouring threads are contiguous.
+  const long long nc = r / 8;
   const long long nb = d_out;
   const long long na = At != nullptr ? d_in : 0;
   const long long nt = Tsave != nullptr ? M : 0;
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nb + na + nt;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < (nb + na + nt) * nc;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    if (i < nb) {
-      const int jd = static_cast<int>(i);
-      for (int c0 = 0; c0 < r; c0 += 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(B + static_cast<size_t>(jd) * r + c0);
-        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+    if (i < nb * nc) {
+      const int jd = static_cast<int>(i % nb), c0 = static_cast<int>(i / nb) * 8;
+      const uint4 v = *reinterpret_cast<const uint4*>(B + static_cast<size_t>(jd) * r + c0);
+      const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float f = __bfloat162float(b[e]);
-          Bt[static_cast<size_t>(c0 + e) * d_out + jd] = to16<T>(f);
-          if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(f) <= kF16Max)) bad = true;
-        }
+      for (int e = 0; e < 8; ++e) {
+        const float f = __bfloat162float(b[e]);
+        Bt[static_cast<size_t>(c0 + e) * d_out + jd] = to16<T>(f);
+        if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(f) <= kF16Max)) bad = true;
       }
-    } else if (i < nb + na) {
-      const int di = static_cast<int>(i - nb);
-      for (int c0 = 0; c0 < r; c0 += 8) {
-        __align__(16) __nv_bfloat16 o[8];
+    } else if (i < (nb + na) * nc) {
+      const long long k = i - nb * nc;
+      const int di = static_cast<int>(k % na), c0 = static_cast<int>(k / na) * 8;
+      __align__(16) __nv_bfloat16 o[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = A[static_cast<size_t>(c0 + e) * d_in + di];
-        *reinterpret_cast<uint4*>(At + static_cast<size_t>(di) * r + c0) = *reinterpret_cast<const uint4*>(o);
-      }
+      for (int e = 0; e < 8; ++e) o[e] = A[static_cast<size_t>(c0 + e) * d_in + di];
+      *reinterpret_cast<uint4*>(At + static_cast<size_t>(di) * r + c0) = *reinterpret_cast<const uint4*>(o);
     } else {
-      const int m = static_cast<int>(i - nb - na);
-      for (int c0 = 0; c0 < r; c0 += 4) {
-        const float4 tv = *reinterpret_cast<const float4*>(Tsave + static_cast<size_t>(m) * r + c0);
-        const float t4[4] = {tv.x, tv.y, tv.z, tv.w};
+      const long long k = i - (nb + na) * nc;
+      const int m = static_cast<int>(k % nt), c0 = static_cast<int>(k / nt) * 8;
+      const float4* tp = reinterpret_cast<const float4*>(Tsave + static_cast<size_t>(m) * r + c0);
+      const float4 ta = tp[0], tb = tp[1];
+      const float t8[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float v = s * t4[e];
-          const T h = to16<T>(v);
-          t_hi[static_cast<size_t>(c0 + e) * ld + m] = h;
-          t_lo[static_cast<size_t>(c0 + e) * ld + m] = to16<T>(v - from16(h));
-          if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
-        }
+      for (int e = 0; e < 8; ++e) {
+        const float v = s * t8[e];
+        const T h = to16<T>(v);
+        t_hi[static_cast<size_t>(c0 + e) * ld + m] = h;
+        t_lo[static_cast<size_t>(c0 + e) * ld + m] = to16<T>(v - from16(h));
+        if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(v) <= kF16Max)) bad = true;
       }
     }
   }
