@@ -1039,7 +1039,8 @@ def main():
                     help="skip the other workloads' entries of the default line")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--shape", default=None,
-                    help="M,d_in,d_out,r,act: this shape instead of --config (profiling, with --calls)")
+                    help="M,d_in,d_out,r,act: this shape instead of --config (profiling, with --calls); "
+                         "act 'ce': the output projection + cross-entropy with d_in = hidden, d_out = V")
     ap.add_argument("--calls", type=int, default=0,
                     help="run this many untimed forward(+backward) calls, print nothing else, exit (for profilers)")
     ap.add_argument("--fwd-only", action="store_true", help="with --calls: forward calls only")
@@ -1048,7 +1049,8 @@ def main():
     cfg = dict(seeded_inputs.CONFIGS[args.config])
     if args.shape:
         f = args.shape.split(",")
-        cfg = dict(M=int(f[0]), d_in=int(f[1]), d_out=int(f[2]), r=int(f[3]), alpha=16.0, act=f[4])
+        cfg = dict(M=int(f[0]), d_in=int(f[1]), d_out=int(f[2]), r=int(f[3]), alpha=16.0 if int(f[3]) else 0.0,
+                   act=f[4])
         args.config = "shape " + args.shape
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -1074,7 +1076,7 @@ def main():
         run_qkv(args, cfg, L, world, rank, local, dist)
         return
     if args.calls > 0:
-        lay = Layer(L, cfg, seed=rank)
+        lay = CeWorkload(L, cfg, seed=rank) if cfg["act"] == "ce" else Layer(L, cfg, seed=rank)
         for _ in range(args.calls):
             lay.fwd()
             if not args.fwd_only:

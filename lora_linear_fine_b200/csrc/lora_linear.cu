@@ -412,6 +412,8 @@ struct RankJob {
   float* partial = nullptr;
   int splits = 1;
   RankOut out = {};
+  const uint8_t* mask = nullptr;   // dropout keep bits of the K-major A (X), [rows x mask_ld] bytes
+  int mask_ld = 0;
 };
 
 RankOut rank_out(int rows, int r) {
@@ -441,6 +443,8 @@ lora_status_t run_rank_gemm(const RankJob& J, int RP, int r, uint32_t* status, c
   q.partial = J.splits > 1 ? J.partial : nullptr;
   q.out = J.out;
   q.status = status;
+  q.mask = J.mask;
+  q.mask_ld = J.mask_ld;
   if (J.a_mn) {
     if (J.na == 1 && J.nb == 2 && !J.f16) return launch_rank_rp<true, 1, 2, false>(RP, q, J.splits, st);
     if (J.na == 2 && J.nb == 2 && J.f16) return launch_rank_rp<true, 2, 2, true>(RP, q, J.splits, st);
@@ -526,10 +530,13 @@ lora_status_t launch_rank2d_rp(int RP, const Rank2dParams& p, int grid, cudaStre
 lora_status_t run_rank2d(const void* Z, int64_t F, int64_t mtok, int r, int RP, const void* rb, const void* cb_hi,
                          const void* cb_lo, int64_t ld_cb, const Rank2dSplit& sp, float* row_partial,
                          float* col_partial, const RankOut& row_out, const RankOut& col_out, uint32_t* status,
-                         cudaStream_t st) {
+                         cudaStream_t st, const uint8_t* mask = nullptr) {
   const bool row = rb != nullptr, col = cb_hi != nullptr;
   Rank2dParams p;
   std::memset(&p, 0, sizeof(p));
+  if (mask != nullptr && row) return LORA_ERR_UNSUPPORTED;   // masking serves the col-only pass over X
+  p.mask = mask;
+  p.mask_ld = static_cast<int>(F / 8);
   bool ok = make_tm(&p.tm_z, Z, F, mtok, F, 64, 128);
   if (row) ok = ok && make_tm(&p.tm_rb, rb, F, r, F, 64, RP);
   if (col) ok = ok && make_tm(&p.tm_cb[0], cb_hi, mtok, r, ld_cb, 64, RP) && make_tm(&p.tm_cb[1], cb_lo, mtok, r, ld_cb, 64, RP);
@@ -574,10 +581,14 @@ lora_status_t run_rank2d(const void* Z, int64_t F, int64_t mtok, int r, int RP, 
 }
 
 // T_j = X A_j^T written to `out` (split K finished in place).
+// T_j = X A_j^T; with a dropout mask, T_j = (X * m) A_j^T with the mask applied
+// to X's tiles inside the pass.
 lora_status_t rank_T(const lora_linear_desc* d, const Plan& P, const void* X, const void* Aj, const RankOut& out,
-                     uint8_t* ws, uint32_t* status, cudaStream_t st) {
+                     uint8_t* ws, uint32_t* status, cudaStream_t st, const uint8_t* mask = nullptr) {
   RankJob J;
   J.a[0] = X;
+  J.mask = mask;
+  J.mask_ld = static_cast<int>(d->d_in / 8);
   J.a_inner = d->d_in;
   J.a_outer = d->M;
   J.a_ld = d->d_in;
@@ -605,16 +616,16 @@ bool pair_kernel_enabled() {
   return v == 1;
 }
 
-template <bool kPair, bool kBwd, int kNPair, int kEpi, int kTN = 256>
+template <bool kPair, bool kBwd, int kNPair, int kEpi>
 lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
-  using C = MmaCfg<kPair, kBwd, kNPair, kEpi, kTN>;
-  auto k = lora_mma_kernel<kPair, kBwd, kNPair, kEpi, kTN>;
+  using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
+  auto k = lora_mma_kernel<kPair, kBwd, kNPair, kEpi>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return cuda_error("cudaFuncSetAttribute(mma)");
   const int max_units = kPair ? sms / 2 : sms;
   const int units = p.num_tiles < max_units ? p.num_tiles : max_units;
-  LORA_LOG("mma pair=%d bwd=%d npair=%d epi=%d tile_n=%d tiles=%d units=%d smem=%d stages=%d lora_ksteps=%d",
-           (int)kPair, (int)kBwd, kNPair, kEpi, kTN, p.num_tiles, units, C::kSmemBytes, C::kStages, p.lora_ksteps);
+  LORA_LOG("mma pair=%d bwd=%d npair=%d epi=%d tiles=%d units=%d smem=%d stages=%d lora_ksteps=%d", (int)kPair,
+           (int)kBwd, kNPair, kEpi, p.num_tiles, units, C::kSmemBytes, C::kStages, p.lora_ksteps);
   const cudaError_t e = launch_k(k, dim3(static_cast<unsigned>(units * C::kCtas)), dim3(kMmaThreads), C::kSmemBytes,
                                  st, kPair, p);
   if (e != cudaSuccess) {
@@ -638,24 +649,9 @@ void set_raster(MmaParams& p, bool pair, double m_bytes, double n_bytes) {
   }
 }
 
-template <bool kBwd, int kNPair, int kEpi, int kTN = 256>
+template <bool kBwd, int kNPair, int kEpi>
 lora_status_t launch_mma_any(bool pair, const MmaParams& p, int sms, cudaStream_t st) {
-  return pair ? launch_mma<true, kBwd, kNPair, kEpi, kTN>(p, sms, st)
-              : launch_mma<false, kBwd, kNPair, kEpi, kTN>(p, sms, st);
-}
-
-// Tile N of an identity GEMM (forward or bf16 dX): 128 when 128-wide tiles
-// fill the units' last wave clearly better than 256-wide ones (each unit runs
-// one tile at a time; the CTA pairs or CTAs are `units`).  A wave's
-// efficiency is tiles / (waves * units).
-int pick_tile_n(int64_t m_tiles, int64_t n_cols, int units) {
-  if (units < 1) return 256;
-  auto eff = [&](int tn) {
-    const int64_t tiles = m_tiles * ceil_div(n_cols, tn);
-    const int64_t waves = ceil_div(tiles, units);
-    return static_cast<double>(tiles) / static_cast<double>(waves * units);
-  };
-  return eff(128) > eff(256) + 0.05 ? 128 : 256;
+  return pair ? launch_mma<true, kBwd, kNPair, kEpi>(p, sms, st) : launch_mma<false, kBwd, kNPair, kEpi>(p, sms, st);
 }
 
 // Failure-detection self-test: one thread waits, through the library's
@@ -725,10 +721,10 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
     static std::map<std::tuple<int, int, int, int64_t, int64_t>, int> cache;
     int dev_id = 0;
     cudaGetDevice(&dev_id);
-    const auto key = std::make_tuple(dev_id, nt, static_cast<int>(w4), d->d_in, d->d_out);
+    const auto key = std::make_tuple(dev_id, nt, static_cast<int>(w4) + 2 * small_m_ar(r), d->d_in, d->d_out);
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
-    if (it == cache.end()) it = cache.emplace(key, small_m_splits(nt, w4, d->d_in, d->d_out)).first;
+    if (it == cache.end()) it = cache.emplace(key, small_m_splits(nt, w4, r, d->d_in, d->d_out)).first;
     q.splits = it->second;
   }
   q.kb_per = static_cast<int>(ceil_div(ceil_div(d->d_in, 64), q.splits));
@@ -739,11 +735,11 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
   // (synchronises the stream; for debugging only).
   static unsigned long long* trace = nullptr;
   if (debug_level() >= 2 && trace == nullptr &&
-      cudaMalloc(&trace, sizeof(unsigned long long) * 1024 * kSmTracePoints) != cudaSuccess)
+      cudaMalloc(&trace, sizeof(unsigned long long) * 1024 * kSmTraceStride) != cudaSuccess)
     trace = nullptr;
   if (debug_level() >= 2 && trace != nullptr && grid <= 1024) {
     q.trace = trace;
-    cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTracePoints, st);
+    cudaMemsetAsync(trace, 0, sizeof(unsigned long long) * grid * kSmTraceStride, st);
   }
   const cudaError_t e = launch_small_m(q, nt, w4, slices, pdl_enabled(), st);
   if (e != cudaSuccess) {
@@ -753,25 +749,18 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
   }
   const lora_status_t ls = check_launch("small_m_kernel");
   if (q.trace != nullptr && cudaStreamSynchronize(st) == cudaSuccess) {
-    std::vector<unsigned long long> h(static_cast<size_t>(grid) * kSmTracePoints);
+    std::vector<unsigned long long> h(static_cast<size_t>(grid) * kSmTraceStride);
     cudaMemcpy(h.data(), trace, h.size() * sizeof(unsigned long long), cudaMemcpyDeviceToHost);
     unsigned long long t0 = ~0ull;
-    for (int b = 0; b < grid; ++b) t0 = h[b * kSmTracePoints] && h[b * kSmTracePoints] < t0 ? h[b * kSmTracePoints] : t0;
+    for (int b = 0; b < grid; ++b)
+      t0 = h[b * kSmTraceStride] && h[b * kSmTraceStride] < t0 ? h[b * kSmTraceStride] : t0;
     static const char* names[kSmTracePoints] = {"entry", "first_issue", "first_data", "last_mma", "published",
                                                 "synced", "t_summed", "combined", "exit", "dq_wait", "dq_work"};
-    for (int k = 0; k < kSmTracePoints; ++k) {
-      if (k == kTrDqWait || k == kTrDqWork) {   // durations, not stamps
-        double tot = 0;
-        int cnt = 0;
-        for (int b = 0; b < grid; ++b)
-          if (h[b * kSmTracePoints + k]) { tot += h[b * kSmTracePoints + k] * 1e-3; ++cnt; }
-        if (cnt) LORA_LOG("small_m trace %-12s n=%3d mean total %7.2f us", names[k], cnt, tot / cnt);
-        continue;
-      }
+    auto stats = [&](int k, const char* name) {
       double mn = 1e30, mx = 0, sum = 0;
       int n = 0;
       for (int b = 0; b < grid; ++b) {
-        const unsigned long long v = h[b * kSmTracePoints + k];
+        const unsigned long long v = h[b * kSmTraceStride + k];
         if (v == 0) continue;
         const double us = (v - t0) * 1e-3;
         mn = us < mn ? us : mn;
@@ -779,7 +768,25 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
         sum += us;
         ++n;
       }
-      if (n) LORA_LOG("small_m trace %-12s n=%3d min %7.2f mean %7.2f max %7.2f us", names[k], n, mn, sum / n, mx);
+      if (n) LORA_LOG("small_m trace %-12s n=%3d min %7.2f mean %7.2f max %7.2f us", name, n, mn, sum / n, mx);
+    };
+    for (int k = 0; k < kSmTracePoints; ++k) {
+      if (k == kTrDqWait || k == kTrDqWork) {   // durations, not stamps
+        double tot = 0;
+        int cnt = 0;
+        for (int b = 0; b < grid; ++b)
+          if (h[b * kSmTraceStride + k]) { tot += h[b * kSmTraceStride + k] * 1e-3; ++cnt; }
+        if (cnt) LORA_LOG("small_m trace %-12s n=%3d mean total %7.2f us", names[k], cnt, tot / cnt);
+        continue;
+      }
+      stats(k, names[k]);
+    }
+    char nm[32];
+    for (int i = 0; i < kSmTraceStages; ++i) {
+      std::snprintf(nm, sizeof nm, "issue[%d]", i);
+      stats(kSmTracePoints + i, nm);
+      std::snprintf(nm, sizeof nm, "full[%d]", i);
+      stats(kSmTracePoints + kSmTraceStages + i, nm);
     }
   }
   return ls;
@@ -1011,7 +1018,8 @@ static lora_status_t fwd_check_args(const lora_linear_desc* d, const void* X, co
 static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const void* W, const void* A,
                               const void* B, const void* W_up, const void* A_up, const void* B_up, void* Y,
                               float* T_save, float* Z_save, void* workspace, size_t workspace_bytes, void* stream,
-                              const void* const Xl[2], bool allow_small_m, const RopeTables* rope = nullptr) {
+                              const void* const Xl[2], bool allow_small_m, const RopeTables* rope = nullptr,
+                              const uint8_t* const fmasks[2] = nullptr) {
   LORA_TRY(fwd_check_args(d, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save));
   const bool swiglu = d->act == LORA_ACT_SWIGLU;
   const Plan P = make_plan(d, false, allow_small_m);
@@ -1038,18 +1046,15 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
                      : reinterpret_cast<float*>(ws + P.t_ws) + static_cast<size_t>(j) * M * r;
       o.s16 = reinterpret_cast<__nv_bfloat16*>(ws + P.s16[j]);
       o.scale = d->s;
-      LORA_TRY(rank_T(d, P, Xl[j], Ap[j], o, ws, status, st));
+      LORA_TRY(rank_T(d, P, Xl[j], Ap[j], o, ws, status, st, fmasks != nullptr ? fmasks[j] : nullptr));
     }
   }
   // 2. Z = [X | sT] [W | B]^T, activation, bf16 Y
   MmaParams p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = pair_kernel_enabled() && M > 128;
-  const int units = pair ? dev.sms / 2 : dev.sms;
-  const int tn = (d->act == LORA_ACT_IDENTITY && rope == nullptr)
-                     ? pick_tile_n(ceil_div(M, pair ? 256 : 128), d->d_out, units) : 256;
-  const int outc = swiglu ? 128 : tn;
-  const int brows = swiglu ? (pair ? 64 : 128) : (pair ? tn / 2 : tn);   // N-side rows per CTA box
+  const int outc = swiglu ? 128 : 256;
+  const int brows = swiglu ? (pair ? 64 : 128) : (pair ? 128 : 256);   // N-side rows per CTA box
   bool ok = make_tm(&p.tm_a[0], X, d->d_in, M, d->d_in, 64, 128);
   for (int j = 0; j < np; ++j) {
     ok = ok && make_tm(&p.tm_w[j], Wp[j], d->d_in, d->d_out, d->d_in, 64, swiglu ? 128 : brows);
@@ -1079,10 +1084,7 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
     return rs;
   }
   switch (d->act) {
-    case LORA_ACT_IDENTITY:
-      rs = tn == 128 ? launch_mma_any<false, 1, kMEpiIdentity, 128>(pair, p, dev.sms, st)
-                     : launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st);
-      break;
+    case LORA_ACT_IDENTITY: rs = launch_mma_any<false, 1, kMEpiIdentity>(pair, p, dev.sms, st); break;
     case LORA_ACT_SILU: rs = launch_mma_any<false, 1, kMEpiSilu>(pair, p, dev.sms, st); break;
     default: rs = launch_mma_any<false, 2, kMEpiSwiglu>(pair, p, dev.sms, st); break;
   }
@@ -1222,7 +1224,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
         o.ld = M8;
         o.hilo_f16 = f16 ? 1 : 0;
         o.scale = d->s;
-        LORA_TRY(rank_T(d, P, Xl[j], Ap[j], o, ws, status, st));
+        LORA_TRY(rank_T(d, P, Xl[j], Ap[j], o, ws, status, st, masks[j]));
       }
     }
     // 3. U = dZ B by a rank pass: bf16 s U (LoRA K-block of dX) and (s U)^T hi/lo (dA).
@@ -1274,9 +1276,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     std::memset(&p, 0, sizeof(p));
     const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
-    const int units = pair ? dev.sms / 2 : dev.sms;
-    const int tn = f16 ? 256 : pick_tile_n(ceil_div(M, pair ? 256 : 128), d->d_in, units);
-    const uint32_t brows = static_cast<uint32_t>(pair ? tn / 2 : tn);   // N-side rows per CTA box (K-major)
+    const uint32_t brows = pair ? 128 : 256;   // N-side rows per CTA box (K-major)
     for (int j = 0; j < np; ++j) {
       ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
       if (P.kmajor) {
@@ -1295,23 +1295,42 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     p.M = M;
     p.N = static_cast<int>(d->d_in);
     p.K = static_cast<int>(d->d_out);
-    p.lora_ksteps = masks[0] != nullptr ? 0 : (r + 15) / 16;   // dropout: the LoRA term comes after
+    p.lora_ksteps = masks[0] != nullptr ? 0 : (r + 15) / 16;   // dropout: the masked LoRA term is separate
+    // dropout, one projection, r <= 64: the masked LoRA term m * (s' U A) is
+    // added in the dX GEMM's epilogue; otherwise dx_dropout_kernel adds it
+    // after the GEMM
+    const bool drop_epi = masks[0] != nullptr && np == 1 && r > 0 && r <= kDropMaxRank && dXf == nullptr;
+    if (drop_epi) {
+      p.drop.mask = masks[0];
+      p.drop.ut_hi = static_cast<const __nv_bfloat16*>(at(P.ut_hi[0]));
+      p.drop.ut_lo = static_cast<const __nv_bfloat16*>(at(P.ut_lo[0]));
+      p.drop.A = static_cast<const __nv_bfloat16*>(Ap[0]);
+      p.drop.r = r;
+      p.drop.ld = M8;
+    }
     p.out = static_cast<__nv_bfloat16*>(dX);
     p.out_f32 = dXf;
     p.out_acc = dXf_acc;
     p.z_save = nullptr;
     p.status = status;
     p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
-    p.n_tiles = static_cast<int>(ceil_div(d->d_in, tn));
+    p.n_tiles = static_cast<int>(ceil_div(d->d_in, 256));
     p.num_tiles = p.m_tiles * p.n_tiles;
     set_raster(p, pair, 2.0 * np * M * d->d_out, 2.0 * np * d->d_out * d->d_in);
     timing_begin(1, st);
     lora_status_t rs;
-    if (f16) {
+    if (drop_epi) {
+      rs = f16 ? launch_mma_any<true, 1, kMEpiGradF16Drop>(pair, p, dev.sms, st)
+               : launch_mma_any<true, 1, kMEpiGradDrop>(pair, p, dev.sms, st);
+    } else if (dXf != nullptr) {
+      // fp32 dX (the attention-input block's summed input gradients): the
+      // staged epilogue
+      if (np != 1) return LORA_ERR_UNSUPPORTED;
+      rs = f16 ? launch_mma_any<true, 1, kMEpiGradF16F32>(pair, p, dev.sms, st)
+               : launch_mma_any<true, 1, kMEpiGradF32>(pair, p, dev.sms, st);
+    } else if (f16) {
       if (np == 2) rs = launch_mma_any<true, 2, kMEpiGradF16>(pair, p, dev.sms, st);
       else rs = launch_mma_any<true, 1, kMEpiGradF16>(pair, p, dev.sms, st);
-    } else if (tn == 128) {
-      rs = launch_mma_any<true, 1, kMEpiGrad, 128>(pair, p, dev.sms, st);
     } else {
       rs = launch_mma_any<true, 1, kMEpiGrad>(pair, p, dev.sms, st);
     }
@@ -1319,7 +1338,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     LORA_TRY(rs);
   }
   if (r == 0) return LORA_OK;
-  if (masks[0] != nullptr) {
+  if (masks[0] != nullptr && !(np == 1 && r <= kDropMaxRank && dXf == nullptr)) {
     // dX += sum_j mask_j * (s' U_j A_j), from the (s' U_j)^T hi/lo of the U pass
     DxDropoutJob jb[2];
     for (int j = 0; j < 2; ++j) {
@@ -1348,7 +1367,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     ao.f32 = dAp[j];
     ao.transpose_f32 = 1;
     LORA_TRY(run_rank2d(Xl[j], d->d_in, M, r, RP, nullptr, at(P.ut_hi[j]), at(P.ut_lo[j]), M8, P.sp_a, nullptr,
-                        static_cast<float*>(at(P.part_a)), rank_out(M, r), ao, status, st));
+                        static_cast<float*>(at(P.part_a)), rank_out(M, r), ao, status, st, masks[j]));
     if (P.dual) continue;
     RankJob Jb;
     Jb.a_mn = true;
@@ -1561,10 +1580,13 @@ lora_status_t lora_linear_fwd_dropout(const lora_linear_desc* d, const void* X, 
   DevInfo dev;
   LORA_TRY(common_checks(d, workspace, workspace_bytes, base + dropout_xm_bytes(d), &dev));
   if (d->M == 0) return LORA_OK;
-  const void* Xl[2];
-  LORA_TRY(mask_inputs(d, X, mask, mask_up, static_cast<uint8_t*>(workspace) + base, Xl, dev,
-                       static_cast<cudaStream_t>(stream)));
-  return fwd_core(&d2, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, workspace, base, stream, Xl, false);
+  // the T pass reads X and applies the mask to its tiles in shared memory:
+  // no masked copy of X in the forward
+  const void* Xl[2] = {X, X};
+  const uint8_t* fm[2] = {static_cast<const uint8_t*>(mask),
+                          static_cast<const uint8_t*>(d->act == LORA_ACT_SWIGLU ? mask_up : mask)};
+  return fwd_core(&d2, X, W, A, B, W_up, A_up, B_up, Y, T_save, Z_save, workspace, base, stream, Xl, false, nullptr,
+                  fm);
 }
 
 lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* d, const void* dY, const void* X, const void* W,
@@ -1583,10 +1605,9 @@ lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* d, const void* dY,
   const size_t base = align_up(dropout_base_bytes(d, true), 256);
   DevInfo dev;
   LORA_TRY(common_checks(d, workspace, workspace_bytes, base + dropout_xm_bytes(d), &dev));
+  // the rank passes read X and apply the mask to their tiles in shared
+  // memory; the dX GEMM adds the masked LoRA term in its epilogue
   const void* Xl[2] = {X, X};
-  if (d->M > 0)
-    LORA_TRY(mask_inputs(d, X, mask, mask_up, static_cast<uint8_t*>(workspace) + base, Xl, dev,
-                         static_cast<cudaStream_t>(stream)));
   const uint8_t* masks[2] = {static_cast<const uint8_t*>(mask),
                              static_cast<const uint8_t*>(mask_up != nullptr ? mask_up : mask)};
   return bwd_core(&d2, dY, X, W, A, B, W_up, A_up, B_up, T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace, base,

@@ -50,9 +50,27 @@ constexpr int kMmaThreads = 320;
 // 128-column block, and the label's logit is picked up; no logit is stored.
 // kMEpiCeGrad: the same logits recomputed and turned into the cross-entropy
 // gradient (exp(z - lse) - onehot(label)) * scale, stored as bf16.
+// kMEpiGradF32 / kMEpiGradF16F32: the dX GEMM (bf16 / fp16 operands) writing
+// or adding to an fp32 dX, staged through shared memory so that each global
+// access covers whole sectors of one row.
+// kMEpiGradDrop / kMEpiGradF16Drop: the dX GEMM (bf16 / fp16 operands, no
+// LoRA K-block) of a layer with dropout on the adapter input; the epilogue
+// adds the masked LoRA term m * (s' U A) on the CUDA cores before the one
+// bf16 rounding.
 enum MmaEpi : int {
   kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5,
-  kMEpiCeFwd = 6, kMEpiCeGrad = 7
+  kMEpiCeFwd = 6, kMEpiCeGrad = 7, kMEpiGradF32 = 8, kMEpiGradF16F32 = 9, kMEpiGradDrop = 10,
+  kMEpiGradF16Drop = 11
+};
+
+// Dropout on the adapter input, dX epilogue (kMEpiGradDrop / kMEpiGradF16Drop).
+constexpr int kDropMaxRank = 64;
+struct DropEpi {
+  const uint8_t* mask;            // [M x N/8] bits, least significant first
+  const __nv_bfloat16* ut_hi;     // (s' U)^T hi [r x ld]
+  const __nv_bfloat16* ut_lo;     // (s' U)^T lo [r x ld]
+  const __nv_bfloat16* A;         // [r x N]
+  int r, ld;                      // r <= kDropMaxRank
 };
 
 // Output projection fused with the cross-entropy loss (rows = tokens of this
@@ -84,32 +102,29 @@ struct MmaParams {
   float* out_f32;         // backward: fp32 dX [M x N] instead of the bf16 `out` (null: bf16)
   int out_acc;            // with out_f32: dX += the product (else dX = the product)
   CeParams ce;            // kMEpiCeFwd / kMEpiCeGrad
+  DropEpi drop;           // kMEpiGradDrop / kMEpiGradF16Drop
 };
 
-// kTN: the tile's N (256, or 128 for the plain identity forward / dX when
-// 128-wide tiles fill the last wave of CTA pairs better).
-template <bool kPair, bool kBwd, int kNPair, int kEpi, int kTN = 256>
+template <bool kPair, bool kBwd, int kNPair, int kEpi>
 struct MmaCfg {
-  static_assert(kTN == 256 || (kTN == 128 && (kEpi == kMEpiIdentity || kEpi == kMEpiGrad)),
-                "128-wide tiles serve the identity forward and the bf16 dX only");
   static constexpr bool kSwigluFwd = (!kBwd) && (kEpi == kMEpiSwiglu);
   static constexpr int kCtas = kPair ? 2 : 1;
   static constexpr int kTileM = 128 * kCtas;                 // rows per (pair) tile
-  static constexpr int kOutCols = kSwigluFwd ? 128 : kTN;    // output columns per tile
+  static constexpr int kOutCols = kSwigluFwd ? 128 : 256;    // output columns per tile
   static constexpr int kKPairs = kBwd ? kNPair : 1;          // projections walked along K
   static constexpr int kLoraProj = kNPair;                   // projections with a LoRA branch per tile
   static constexpr int kABytes = 128 * 64 * 2;               // 16 KB
-  static constexpr int kBRows = (kSwigluFwd ? 256 : kTN) / kCtas;   // N-side rows held per CTA
-  static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair) at N = 256
+  static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
+  static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
   static constexpr int kStageBytes = kABytes + kBBytes;
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
   // shared memory (4 KB per warp) so that global stores are row-contiguous.
-  static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu;
+  static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
   static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : 0;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kEpiStageBytes + 2048;
-  static constexpr uint32_t kTmemCols = 2 * kTN;             // 2 accumulator buffers
+  static constexpr uint32_t kTmemCols = 512;                 // 2 accumulator buffers
   static_assert(kStages >= 3, "ring too shallow");
 };
 
@@ -143,9 +158,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
   else return mbar_wait(bar, parity, ctl);
 }
 
-template <bool kPair, bool kBwd, int kNPair, int kEpi, int kTN = 256>
+template <bool kPair, bool kBwd, int kNPair, int kEpi>
 __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_constant__ MmaParams p) {
-  using C = MmaCfg<kPair, kBwd, kNPair, kEpi, kTN>;
+  using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
   constexpr int S = C::kStages;
 
   extern __shared__ uint8_t smem_raw[];
@@ -291,15 +306,14 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      constexpr bool kF16 = (kEpi == kMEpiGradF16);
+      constexpr bool kF16 = (kEpi == kMEpiGradF16 || kEpi == kMEpiGradF16F32 || kEpi == kMEpiGradF16Drop);
       constexpr int kM = C::kTileM;
       // N-side operand MN-major only in a backward that reads W and A in place
       const bool bmn = kBwd && p.b_mn != 0;
-      constexpr int kN = C::kSwigluFwd ? 256 : kTN;
-      const uint32_t kIdMain = bmn ? idesc_mma(kM, kN, false, true, kF16) : idesc_mma(kM, kN, false, false, kF16);
+      const uint32_t kIdMain = bmn ? idesc_mma(kM, 256, false, true, kF16) : idesc_mma(kM, 256, false, false, kF16);
       // LoRA block: bf16 s*T/s*U against bf16 B (fwd) / A or A^T (bwd)
-      const uint32_t kIdLora = bmn ? idesc_mma(kM, kN, false, true, false)
-                                   : idesc_mma(kM, C::kSwigluFwd ? 128 : kN, false, false, false);
+      const uint32_t kIdLora = bmn ? idesc_mma(kM, 256, false, true, false)
+                                   : idesc_mma(kM, C::kSwigluFwd ? 128 : 256, false, false, false);
       constexpr uint16_t kBoth = 0x3;
       auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
         if constexpr (kPair) mma_bf16_pair(d, a, b, id, acc);
@@ -316,7 +330,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         const uint32_t use = it >> 1;        // how many times this buffer was used before
         if (!wait_bar<kPair>(&acc_empty[buf], (use & 1u) ^ 1u, ctl)) break;
         tc_fence_after();
-        const uint32_t dacc = tbase + buf * (C::kSwigluFwd ? 256 : kTN);
+        const uint32_t dacc = tbase + buf * 256;
         const int nblocks = C::kKPairs * nkb + nlora;
         bool ok = true;
         for (int blk = 0; blk < nblocks; ++blk) {
@@ -376,7 +390,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
-      const uint32_t tl = tbase + buf * (C::kSwigluFwd ? 256 : kTN) + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
       auto release_acc = [&]() {   // every lane's tcgen05.ld has completed (tmem_wait_ld)
         tc_fence_before();
         __syncwarp();
@@ -385,7 +399,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           else mbar_arrive(&acc_empty[buf]);
         }
       };
-      if constexpr (C::kStaged) {
+      if constexpr (C::kSwigluFwd || kEpi == kMEpiSilu) {
         // Two halves of this thread's columns (SiLU: 64 + 64 of its 128;
         // SwiGLU: 32 + 32 gate columns with their up columns), so that only 64
         // accumulator values are live at a time.  Rows go out through shared
@@ -527,6 +541,117 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             }
           }
         }
+      } else if constexpr (kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32) {
+        // fp32 dX, written or added to (several projections' input gradients
+        // summed in a fixed order, one launch after another).  Each 32-column
+        // chunk of the warp's 32 rows goes through shared memory (4 KB per
+        // warp, 16-byte chunk j of row rr at j ^ (rr & 7)) and out row by
+        // row: 8 lanes cover 128 contiguous bytes of one row.
+        const int row0 = row - lane;                 // first row of this warp's 32
+        float4* stg = reinterpret_cast<float4*>(epi_stage + ew * 4096);
+        const int col0 = nt * 256 + h * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tl + h * 128 + 32 * c, v);
+          tmem_wait_ld();
+          if (c == 3) release_acc();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            stg[lane * 8 + (j ^ (lane & 7))] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                           __uint_as_float(v[4 * j + 2]),
+                                                           __uint_as_float(v[4 * j + 3]));
+          __syncwarp();
+          const int j = lane & 7;
+          const int col = col0 + 32 * c + 4 * j;
+          float4 a[8];
+          if (p.out_acc) {
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int grow = row0 + it * 4 + (lane >> 3);
+              a[it] = (grow < p.M && col < p.N)
+                          ? *reinterpret_cast<const float4*>(p.out_f32 + static_cast<size_t>(grow) * p.N + col)
+                          : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+          }
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3);
+            const int grow = row0 + rr;
+            if (grow < p.M && col < p.N) {
+              float4 o = stg[rr * 8 + (j ^ (rr & 7))];
+              if (p.out_acc) {
+                o.x += a[it].x;
+                o.y += a[it].y;
+                o.z += a[it].z;
+                o.w += a[it].w;
+              }
+              st_global_v4_hint(p.out_f32 + static_cast<size_t>(grow) * p.N + col,
+                                make_uint4(__float_as_uint(o.x), __float_as_uint(o.y), __float_as_uint(o.z),
+                                           __float_as_uint(o.w)),
+                                pol_out);
+            }
+          }
+        }
+      } else if constexpr (kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop) {
+        // dX = dZ W (the accumulator) + m * (s' U A): this thread's row of
+        // s'U (hi + lo, fp32) in registers, the tile's columns of A read as
+        // warp-wide broadcasts (every lane of a warp reads the same 16
+        // bytes), 16 columns at a time; one bf16 rounding at the end.
+        const int col0 = nt * 256 + h * 128;
+        const DropEpi& D = p.drop;
+        float u[kDropMaxRank];
+#pragma unroll
+        for (int c = 0; c < kDropMaxRank; ++c) {
+          u[c] = 0.0f;
+          if (c < D.r && row_ok) {
+            const size_t at = static_cast<size_t>(c) * D.ld + row;
+            u[c] = __bfloat162float(D.ut_hi[at]) + __bfloat162float(D.ut_lo[at]);
+          }
+        }
+        const size_t mrow = static_cast<size_t>(row) * (p.N / 8);
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t v[16];
+          __syncwarp();
+          tmem_ld16(tl + h * 128 + 16 * c16, v);
+          tmem_wait_ld();
+          if (c16 == 7) release_acc();
+          const int cb = col0 + 16 * c16;
+          if (!row_ok || cb >= p.N) continue;
+          float t[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) t[j] = 0.0f;
+          const bool two = cb + 8 < p.N;
+#pragma unroll
+          for (int c = 0; c < kDropMaxRank; ++c) {
+            if (c >= D.r) break;
+            const uint4* ap = reinterpret_cast<const uint4*>(D.A + static_cast<size_t>(c) * p.N + cb);
+            const uint4 a0 = __ldg(ap);
+            const uint4 a1 = two ? __ldg(ap + 1) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              t[2 * e] = fmaf(u[c], __uint_as_float(w[e] << 16), t[2 * e]);
+              t[2 * e + 1] = fmaf(u[c], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
+            }
+          }
+          const uint32_t mb = D.mask[mrow + cb / 8] | (two ? static_cast<uint32_t>(D.mask[mrow + cb / 8 + 1]) << 8 : 0u);
+          float z[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) z[j] = __uint_as_float(v[j]) + (((mb >> j) & 1u) ? t[j] : 0.0f);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            if (q == 1 && !two) break;
+            uint4 pk;
+            pk.x = pack_bf16x2(z[8 * q], z[8 * q + 1]);
+            pk.y = pack_bf16x2(z[8 * q + 2], z[8 * q + 3]);
+            pk.z = pack_bf16x2(z[8 * q + 4], z[8 * q + 5]);
+            pk.w = pack_bf16x2(z[8 * q + 6], z[8 * q + 7]);
+            st_global_v4_hint(p.out + static_cast<size_t>(row) * p.N + cb + 8 * q, pk, pol_out);
+          }
+        }
       } else if constexpr (kEpi == kMEpiCeFwd) {
         // This thread's token row and 128 vocabulary columns [col0, col0 + 128):
         // a running max and sum of exp(z - max) over four 32-column loads
@@ -595,42 +720,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           }
         }
       } else {
-        constexpr int kHalf = kTN / 2;          // columns per epilogue thread
-        uint32_t v[kHalf];
+        uint32_t v[128];
 #pragma unroll
-        for (int c = 0; c < kHalf / 32; ++c)
-          tmem_ld32(tl + h * kHalf + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+        for (int c = 0; c < 4; ++c) tmem_ld32(tl + h * 128 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
         tmem_wait_ld();
         release_acc();
         if (!row_ok) continue;
-        const int col0 = nt * kTN + h * kHalf;
+        const int col0 = nt * 256 + h * 128;
         const size_t base = static_cast<size_t>(row) * p.N + col0;
-        if constexpr (kBwd) {
-          if (p.out_f32 != nullptr) {
-            // fp32 dX, written or added to (several projections' input
-            // gradients summed in a fixed order, one launch after another)
-            float* dst = p.out_f32 + base;
 #pragma unroll
-            for (int c = 0; c < kHalf; c += 4) {
-              if (col0 + c < p.N) {
-                float4 o = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
-                                       __uint_as_float(v[c + 3]));
-                if (p.out_acc) {
-                  const float4 a = *reinterpret_cast<const float4*>(dst + c);
-                  o.x += a.x;
-                  o.y += a.y;
-                  o.z += a.z;
-                  o.w += a.w;
-                }
-                st_global_v4_hint(dst + c, make_uint4(__float_as_uint(o.x), __float_as_uint(o.y),
-                                                      __float_as_uint(o.z), __float_as_uint(o.w)), pol_out);
-              }
-            }
-            continue;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < kHalf; c += 8) {
+        for (int c = 0; c < 128; c += 8) {
           uint4 pk;
           pk.x = pack_bf16x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
           pk.y = pack_bf16x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));

@@ -80,6 +80,12 @@ __device__ __forceinline__ void emit_rank_row(const float* v, int row, const Ran
 struct RankGemmParams {
   CUtensorMap tm_a[2];
   CUtensorMap tm_b[2];
+  // Dropout on the adapter input (K-major A = X only): keep bits of X, [rows x
+  // mask_ld] bytes, bit j of byte b keeping element 8 b + j of a row; null for
+  // none.  The epilogue warps zero the dropped elements of each stage's X
+  // tiles in shared memory before the MMA warp reads them.
+  const uint8_t* mask;
+  int mask_ld;
   int rows;          // rows of the result (M side of the MMA)
   int K;             // reduction length
   int m_tiles;
@@ -128,12 +134,14 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   uint64_t* empty = bars + S;
   uint64_t* acc_full = bars + 2 * S;
   uint64_t* mma_done = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 2);
+  uint64_t* masked = acc_full + 2;     // [S] dropout: the stage's X tiles are masked (one arrival per epilogue warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(masked + S);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   AbortCtl ctl{abort_flag, p.status};
+  const bool masking = !kAMN && p.mask != nullptr;
   const int mt = blockIdx.x % p.m_tiles;
   const int sp = blockIdx.x / p.m_tiles;
   constexpr int KS = C::kKS;
@@ -144,7 +152,7 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); mbar_init(&masked[i], 4); }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -195,6 +203,7 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
       bool ok = true;
       for (int i = 0; i < nkb; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+        if (masking && !mbar_wait(&masked[rp.stage], rp.phase, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + rp.stage * C::kStageBytes);
 #pragma unroll
@@ -221,6 +230,46 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
   } else {
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    if (masking) {
+      // Dropout: zero the dropped elements of each stage's X tiles.  Thread
+      // `row` owns row `row` of every [128 x 64] SWIZZLE_128B box: 16-byte
+      // chunk c (features 8c .. 8c + 7) at position c ^ (row & 7), masked by
+      // byte c of the row's 8 mask bytes for that K block.
+      const int grow = mt * 128 + row;
+      const bool in_rows = grow < p.rows;
+      const uint8_t* mrow = p.mask + static_cast<size_t>(in_rows ? grow : 0) * p.mask_ld;
+      RingPos rp;
+      for (int i = 0; i < nkb; ++i) {
+        if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
+        uint8_t* st = smem + rp.stage * C::kStageBytes;
+        const int k0 = (kb0 + i) * 64 * KS;
+#pragma unroll
+        for (int kb = 0; kb < KS; ++kb) {
+          uint4* trow = reinterpret_cast<uint4*>(st + kb * 16384 + row * 128);
+          const int byte0 = (k0 + 64 * kb) / 8;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t b = (in_rows && byte0 + c < p.mask_ld) ? mrow[byte0 + c] : 0u;
+            if (b == 0xFFu) continue;
+            uint4& slot = trow[c ^ (row & 7)];
+            const uint4 v = slot;
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
+              const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
+              o[e] = w[e] & (lo | hi);
+            }
+            slot = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&masked[rp.stage]);
+        rp.next(S);
+      }
+    }
     float acc[kRP];
 #pragma unroll
     for (int c = 0; c < kRP; ++c) acc[c] = 0.0f;

@@ -46,6 +46,12 @@ struct Rank2dParams {
   float* col_partial;     // [ts][f_blocks*128][RP], or null (one token split: results to col_out)
   RankOut row_out, col_out;
   uint32_t* status;
+  // Dropout on the adapter input (col-only passes over X): keep bits [mtok x
+  // mask_ld] bytes, bit j of byte b keeping feature 8 b + j; null for none.
+  // The epilogue warps, idle until the end of a col-only pass, zero the
+  // dropped elements of each stage's tile before the MMA warp reads it.
+  const uint8_t* mask;
+  int mask_ld;
 };
 
 template <int kRP, bool kRow, bool kCol>
@@ -84,7 +90,8 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
   uint64_t* col_done = cb_empty + 2;
   uint64_t* mma_done = col_done + 1;
   uint64_t* row_done = mma_done + 1;                         // [kRank2dMaxRowTiles]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(row_done + kRank2dMaxRowTiles);
+  uint64_t* masked = row_done + kRank2dMaxRowTiles;          // [S] dropout: the stage's tile is masked
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(masked + S);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -97,6 +104,7 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
   const int fj0 = fsplit * p.b_blocks;
   const int fj1 = fj0 + p.b_blocks < p.f_blocks ? fj0 + p.b_blocks : p.f_blocks;
   const int na = ti1 - ti0, nb = fj1 - fj0;     // >= 1 by the host's choice of splits
+  const bool masking = kCol && !kRow && p.mask != nullptr;
   // tensor memory: row accumulators (RP columns each) first, then col accumulators (2 RP)
   const int row_cols = kRow ? na * kRP : 0;
   const uint32_t ncols_used = static_cast<uint32_t>(row_cols + (kCol ? nb * 2 * kRP : 0));
@@ -110,6 +118,7 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
     mbar_init(col_done, 1);
     mbar_init(mma_done, 1);
     for (int i = 0; i < kRank2dMaxRowTiles; ++i) mbar_init(&row_done[i], 1);
+    for (int i = 0; i < S; ++i) mbar_init(&masked[i], 4);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -173,6 +182,7 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
         const uint32_t acc_row = tbase + static_cast<uint32_t>(i * kRP);
         for (int j = 0; j < nb; ++j) {
           if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+          if (masking && !mbar_wait(&masked[rp.stage], rp.phase, ctl)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sz = smem_u32(smem + rp.stage * C::kStageBytes);
           if constexpr (kRow) {
@@ -237,6 +247,50 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
         }
       }
     }
+    if constexpr (kCol && !kRow) {
+      if (masking) {
+        // Thread lrow owns token row lrow of both boxes of every stage: 16-byte
+        // chunk c (features 8c .. 8c + 7 of the box) at position c ^ (lrow & 7),
+        // masked by byte c of the row's 8 mask bytes for that box.
+        RingPos rp;
+        bool ok = true;
+        for (int i = 0; i < na && ok; ++i) {
+          const int tok = (ti0 + i) * 128 + lrow;
+          const bool in_rows = tok < p.mtok;
+          const uint8_t* mrow = p.mask + static_cast<size_t>(in_rows ? tok : 0) * p.mask_ld;
+          for (int j = 0; j < nb; ++j) {
+            if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+            uint8_t* st = smem + rp.stage * C::kStageBytes;
+            const int f0 = (fj0 + j) * 128;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint4* trow = reinterpret_cast<uint4*>(st + h * C::kZBox + lrow * 128);
+              const int byte0 = (f0 + 64 * h) / 8;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint32_t b = (in_rows && byte0 + c < p.mask_ld) ? mrow[byte0 + c] : 0u;
+                if (b == 0xFFu) continue;
+                uint4& slot = trow[c ^ (lrow & 7)];
+                const uint4 v = slot;
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
+                  const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
+                  o[e] = w[e] & (lo | hi);
+                }
+                slot = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&masked[rp.stage]);
+            rp.next(S);
+          }
+        }
+      }
+    }
     if constexpr (kCol) {
       if (mbar_wait(col_done, 0, ctl)) {
         tc_fence_after();
@@ -282,10 +336,13 @@ struct Rank2dSplit {
 
 // Choose a x b rectangles: tensor memory ((a + 2b) RP columns, or the used
 // product's), the resident row B (b blocks), at most kRank2dMaxRowTiles row
-// tiles; among those, the least estimated time: the tile bytes of the most
-// loaded wave (imbalance included) + the partials written and read back,
-// with runs per token row shorter than 2 KB charged for their lower DRAM
-// efficiency.
+// tiles; among those, the least estimated time: the bytes a CTA of the most
+// loaded wave brings in (its Z tiles, with runs per token row shorter than
+// 2 KB charged for their lower DRAM efficiency; the col B operand once per
+// token tile; the resident row B once), times the CTAs of that wave, plus the
+// partials written and read back.  The col B operand (hi and lo, 512 RP bytes
+// per token tile) is as large as a Z tile at RP = 64, so a CTA that walks one
+// feature block per token tile spends half its loads on it.
 inline Rank2dSplit rank2d_split(int m_tiles, int f_blocks, int RP, bool row, bool col, int max_rb, int ctas) {
   Rank2dSplit best;
   double best_cost = 0.0;
@@ -311,9 +368,12 @@ inline Rank2dSplit rank2d_split(int m_tiles, int f_blocks, int RP, bool row, boo
     const long long n = static_cast<long long>(ts) * fs;
     const long long waves = (n + ctas - 1) / ctas;
     const double tile = 32768.0;
-    double cost = static_cast<double>(waves) * a * be * tile * static_cast<double>(n < ctas ? n : ctas);
+    const double width = static_cast<double>(waves) * static_cast<double>(n < ctas ? n : ctas);
+    double cost = width * a * be * tile;
     const double run = be * 256.0;
     if (run < 2048.0) cost *= 1.0 + 0.5 * (1.0 - run / 2048.0);
+    if (col) cost += width * a * 512.0 * RP;          // col B (hi + lo) per token tile
+    if (row) cost += width * be * 256.0 * RP;         // resident row B
     if (row && fs > 1) cost += 2.0 * fs * m_tiles * 128.0 * RP * 4.0;
     if (col && ts > 1) cost += 2.0 * ts * f_blocks * 128.0 * RP * 4.0;
     if (best.a == 0 || cost < best_cost) {

@@ -4,14 +4,21 @@
 // short tail after the stream.
 //
 // One thread-block cluster of S CTAs per 128-row slice of W (S = 1..16, one
-// CTA per SM); the CTAs of a cluster split the K dimension.  Per 64-wide K
-// block one TMA stage brings
-//   W tile [128 rows x 64]                    -> Z^T partial  D_Z [128 x kNT] += W  X^T
-//   A tile [a_rows x 64] into a 128-row slot  -> T^T partial  D_T [128 x kNT] += A  X^T
-//     (a_rows = r rounded up to 16, rows >= r zero; the slot's other rows hold
-//     stale data, so rows >= a_rows of D_T are garbage and never read)
+// CTA per SM); the CTAs of a cluster split the K dimension.  One TMA stage
+// brings kKPS 64-wide K blocks (two for a bf16 weight: 32 KB of W per stage
+// and per barrier round trip, which streams measurably faster than 16 KB
+// stages), each as
 //   X tile [kNT tokens x 64], rows >= M zero
-// (swap-AB: the weight rows are the M side of the MMA, the tokens are N).
+//   A tile [a_rows x 64], a_rows = r rounded up to 16, rows >= r zero
+//   W tile [128 rows x 64]
+// and two MMAs per 16-wide K step:
+//   Z^T partial  D_Z [128 x kNT]    += W X^T   (swap-AB: the weight rows are
+//                                              the M side, the tokens N)
+//   T partial    D_T [128 x a_rows] += X A^T   (M = a 128-row window from the
+//                                              X slot's start, which runs on
+//                                              into the A and W slots of the
+//                                              same block: rows >= kNT of D_T
+//                                              are garbage and never read)
 // Every cluster covers all of K, so each computes the full T for itself: no
 // CTA outside the cluster is ever needed.  After the K loop each CTA parks its
 // fp32 partials in its own shared memory; after a cluster barrier each CTA
@@ -49,7 +56,7 @@ struct SmallMParams {
   int splits;                // CTAs per cluster (K splits)
   int kb_per;                // 64-wide K blocks per CTA
   int a_rows;                // rows of A loaded per K block: r rounded up to 16
-  unsigned long long* trace; // null, or [grid][kSmTracePoints] globaltimer stamps (debugging)
+  unsigned long long* trace; // null, or [grid][kSmTraceStride] globaltimer stamps (debugging)
 };
 
 // Trace points of one CTA (LORA_LINEAR_DEBUG=2 prints them per launch).
@@ -58,6 +65,10 @@ enum SmTrace : int {
   kTrDqWait, kTrDqWork,   // 4-bit weight: total ns the expanding warps waited for data / spent expanding
   kSmTracePoints
 };
+// Per-stage stamps after the points above: when the producer issued stage i
+// and when the MMA warp saw it full (the first kSmTraceStages stages).
+constexpr int kSmTraceStages = 16;
+constexpr int kSmTraceStride = kSmTracePoints + 2 * kSmTraceStages;
 
 __device__ __forceinline__ unsigned long long sm_clock_ns() {
   unsigned long long t;
@@ -69,7 +80,7 @@ __device__ __forceinline__ void sm_trace(const SmallMParams& p, int point) {
   if (p.trace != nullptr) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t) : : "memory");
-    p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + point] = t;
+    p.trace[static_cast<size_t>(blockIdx.x) * kSmTraceStride + point] = t;
   }
 }
 
@@ -105,31 +116,35 @@ __device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&out)[16]) {
   for (int c = 0; c < 16; ++c) out[c] = __uint_as_float(v[c]);
 }
 
-template <int kNT, bool kW4>
+template <int kNT, bool kW4, int kAR>
 struct SmallMCfg {
-  static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64 (4-bit weight: dequantised here)
-  // A slot: 64 rows (r <= 64 here), the first a_rows loaded.  The MMA reads a
-  // 128-row window from its start, which runs on into the bytes after it
-  // (the X, code and scale slots, the next stage, or for the last stage the
-  // B rows at the start of the tail): rows >= a_rows of D_T are garbage and
-  // never read, and the window stays inside this CTA's shared memory.
-  static constexpr int kABox = 64 * 64 * 2;
+  static constexpr int kKPS = kW4 ? 1 : 2;              // 64-wide K blocks per stage
+  // per K block: [X slot | A slot | W tile | (4-bit) codes | scales]
   static constexpr int kXBox = kNT * 64 * 2;            // X tile: kNT rows x 64
+  static constexpr int kABox = kAR * 64 * 2;            // A slot: kAR >= a_rows rows x 64
+  static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64 (4-bit weight: expanded here)
   static constexpr int kQBox = kW4 ? 128 * 32 : 0;      // 4-bit weight: packed codes, 128 rows x 32 bytes
   static constexpr int kSBox = kW4 ? 128 * 2 : 0;       // 4-bit weight: the 128 rows' scales of this K block
-  static constexpr int kQOff = kWBox + kABox + kXBox;
+  static constexpr int kXOff = 0;
+  static constexpr int kAOff = kXBox;
+  static constexpr int kWOff = kXBox + kABox;
+  static constexpr int kQOff = kWOff + kWBox;
   static constexpr int kSOff = kQOff + kQBox;
-  static constexpr int kStageBytes = (kSOff + kSBox + 1023) / 1024 * 1024;
+  static constexpr int kBlockBytes = (kSOff + kSBox + 1023) / 1024 * 1024;
+  static constexpr int kStageBytes = kKPS * kBlockBytes;
   static constexpr int kLd = kNT + 4;                   // parked row stride (floats): 16-byte rows, conflict-free float4 stores
-  static constexpr int kBsBytes = 128 * 65 * 4;         // B rows of this CTA's features, fp32, stride r + 1
+  static constexpr int kBsBytes = 128 * 66 * 2;         // B rows of this CTA's features, bf16, stride r + 2
   static constexpr int kTailBytes = kBsBytes + 1024 + 1024;   // B rows, barriers, alignment slack
   static constexpr int kStages0 = (kSmemLimitBytes - kTailBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
-  static constexpr uint32_t kTmemCols = (2 * kNT) <= 32 ? 32 : ((2 * kNT) <= 64 ? 64 : 128);
+  static constexpr uint32_t kTmemCols = 128;            // D_Z: kNT columns, then D_T: kAR columns
   // after the K loop the ring holds: Dp [128][kLd], Tp [128][kLd], Tf [64][kNT]
   static constexpr int kParkBytes = 2 * 128 * kLd * 4 + kNT * 64 * 4;
-  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kXBox % 1024 == 0 && kABox % 1024 == 0 && kWBox % 1024 == 0, "swizzle atoms");
+  static_assert(kNT + kAR <= static_cast<int>(kTmemCols), "tensor memory");
+  // the T window (128 rows = 16 KB from the X slot) stays inside its block
+  static_assert(kXBox + kABox + kWBox >= 128 * 128, "T window");
   static_assert(kStages >= 3, "ring too shallow");
   static_assert(kParkBytes <= kStages * kStageBytes, "parked partials must fit the ring");
 };
@@ -138,9 +153,9 @@ struct SmallMCfg {
 // 64 input features; the epilogue warps, idle during the K loop, turn each
 // stage's codes into the bf16 W tile (value = bf16(scale * (code - 8)), laid
 // out as the SWIZZLE_128B tile TMA would have written) before the MMA reads it.
-template <int kNT, bool kW4>
+template <int kNT, bool kW4, int kAR>
 __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_constant__ SmallMParams p) {
-  using C = SmallMCfg<kNT, kW4>;
+  using C = SmallMCfg<kNT, kW4, kAR>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,7 +167,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  float* Bs = reinterpret_cast<float*>(smem + S * C::kStageBytes);          // [F][r + 1], first in the tail
+  __nv_bfloat16* Bs = reinterpret_cast<__nv_bfloat16*>(smem + S * C::kStageBytes);   // [F][r + 2], first in the tail
   float* Dp = reinterpret_cast<float*>(smem);                               // [128][kLd]  Z^T partial
   float* Tp = Dp + 128 * C::kLd;                                            // [128][kLd]  T^T partial
   float* Tf = Tp + 128 * C::kLd;                                            // [64][kNT]   summed T, tokens contiguous
@@ -198,52 +213,66 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       // those reads spread over the L2 instead of converging on one tile.
       const int rot = nk > 0 ? slice % nk : 0;
       RingPos rp;
-      for (int i = 0; i < nk; ++i) {
-        const int kb = kb0 + (i + rot) % nk;
+      const int ns = (nk + C::kKPS - 1) / C::kKPS;      // stages: kKPS K blocks each, the last possibly fewer
+      for (int i = 0; i < ns; ++i) {
         if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
-        const int k0 = kb * 64;
-        if constexpr (kW4) {
-          mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kQBox + C::kSBox + C::kXBox + p.a_rows * 128));
-          if (p.Wt != nullptr)      // one 4 KB tile of codes
-            bulk_load_1d(st + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kb) * kW4TileBytes,
-                         kW4TileBytes, &full[rp.stage]);
-          else
-            tma_load_2d(st + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);  // codes: k0 / 2 bytes in
-          tma_load_2d(st + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb);   // scales of group kb
-        } else {
-          mbar_arrive_expect_tx(&full[rp.stage], static_cast<uint32_t>(C::kWBox + C::kXBox + p.a_rows * 128));
-          tma_load_2d(st, &p.tm_w, &full[rp.stage], k0, slice * 128);
+        const int nb = (nk - i * C::kKPS) < C::kKPS ? (nk - i * C::kKPS) : C::kKPS;
+        constexpr uint32_t kWBytes = kW4 ? C::kQBox + C::kSBox : C::kWBox;
+        mbar_arrive_expect_tx(&full[rp.stage],
+                              static_cast<uint32_t>(nb * (kWBytes + C::kXBox + p.a_rows * 128)));
+        for (int j = 0; j < nb; ++j) {
+          const int kb = kb0 + (i * C::kKPS + j + rot) % nk;
+          const int k0 = kb * 64;
+          uint8_t* blk = st + j * C::kBlockBytes;
+          if constexpr (kW4) {
+            if (p.Wt != nullptr)      // one 4 KB tile of codes
+              bulk_load_1d(blk + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kb) * kW4TileBytes,
+                           kW4TileBytes, &full[rp.stage]);
+            else
+              tma_load_2d(blk + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);  // codes: k0 / 2 bytes in
+            tma_load_2d(blk + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb);    // scales of group kb
+          } else {
+            tma_load_2d(blk + C::kWOff, &p.tm_w, &full[rp.stage], k0, slice * 128);
+          }
+          tma_load_2d_hint(blk + C::kAOff, &p.tm_a, &full[rp.stage], k0, 0, pol_x);
+          tma_load_2d_hint(blk + C::kXOff, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
         }
-        tma_load_2d_hint(st + C::kWBox, &p.tm_a, &full[rp.stage], k0, 0, pol_x);
-        tma_load_2d_hint(st + C::kWBox + C::kABox, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
         if (i == 0) sm_trace(p, kTrFirstIssue);
+        if (i < kSmTraceStages) sm_trace(p, kSmTracePoints + i);
         rp.next(S);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16(128, kNT, false, false);
+      constexpr uint32_t kIdZ = idesc_bf16(128, kNT, false, false);
+      const uint32_t kIdT = idesc_bf16(128, p.a_rows, false, false);
+      const int ns = (nk + C::kKPS - 1) / C::kKPS;
       RingPos rp;
       bool ok = true;
-      for (int i = 0; i < nk; ++i) {
+      for (int i = 0; i < ns; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
         if constexpr (kW4) {
           if (!mbar_wait(&dq_full[rp.stage], rp.phase, ctl)) { ok = false; break; }
         }
         tc_fence_after();
         if (i == 0) sm_trace(p, kTrFirstData);
-        const uint32_t sw = smem_u32(smem + rp.stage * C::kStageBytes);
-        const uint32_t sa = sw + C::kWBox;
-        const uint32_t sx = sa + C::kABox;
+        if (i < kSmTraceStages) sm_trace(p, kSmTracePoints + kSmTraceStages + i);
+        const int nb = (nk - i * C::kKPS) < C::kKPS ? (nk - i * C::kKPS) : C::kKPS;
+        for (int j = 0; j < nb; ++j) {
+          const uint32_t sblk = smem_u32(smem + rp.stage * C::kStageBytes + j * C::kBlockBytes);
+          const uint32_t sx = sblk + C::kXOff;
+          const uint32_t sa = sblk + C::kAOff;
+          const uint32_t sw = sblk + C::kWOff;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t dw = sdesc_sw128(sw + kk * 32, 16, 1024);
-          const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
-          const uint64_t dx = sdesc_sw128(sx + kk * 32, 16, 1024);
-          const uint32_t acc = (i == 0 && kk == 0) ? 0u : 1u;
-          mma_bf16(tbase, dw, dx, kId, acc);          // Z^T partial: 128 rows of W x tokens
-          mma_bf16(tbase + kNT, da, dx, kId, acc);    // T^T partial: rows of A (r real) x tokens
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t dw = sdesc_sw128(sw + kk * 32, 16, 1024);
+            const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t dx = sdesc_sw128(sx + kk * 32, 16, 1024);
+            const uint32_t acc = (i == 0 && j == 0 && kk == 0) ? 0u : 1u;
+            mma_bf16(tbase, dw, dx, kIdZ, acc);          // Z^T partial: 128 rows of W x tokens
+            mma_bf16(tbase + kNT, dx, da, kIdT, acc);    // T partial: 128-row token window x rows of A
+          }
         }
         mma_commit(&empty[rp.stage]);
         rp.next(S);
@@ -261,11 +290,11 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
     const int et = threadIdx.x - 64;
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int lrow = q * 32 + lane;
-    // this CTA's F rows of B, as fp32 with a padded stride, loaded during the K loop
+    // this CTA's F rows of B (bf16, row stride r + 2), loaded during the K loop
     for (int i = et; i < F * p.r; i += 128) {
       const int fl = i / p.r, c = i - fl * p.r;
       const int n = slice * 128 + f0 + fl;
-      Bs[fl * (p.r + 1) + c] = n < p.d_out ? __bfloat162float(p.B[static_cast<size_t>(n) * p.r + c]) : 0.0f;
+      Bs[fl * (p.r + 2) + c] = n < p.d_out ? p.B[static_cast<size_t>(n) * p.r + c] : __float2bfloat16_rn(0.0f);
     }
     if constexpr (kW4) {
       // Dequantise each stage's W tile: thread lrow owns row lrow (32 bytes of
@@ -277,13 +306,13 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       for (int i = 0; i < nk; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
         if (tr) { const unsigned long long t1 = sm_clock_ns(); t_wait += t1 - t0; t0 = t1; }
-        uint8_t* st = smem + rp.stage * C::kStageBytes;
+        uint8_t* st = smem + rp.stage * C::kStageBytes;     // one K block per stage (kKPS = 1)
         const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + lrow * 32);
         const uint4 c0 = codes[0], c1 = codes[1];
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const __nv_bfloat162 sc2 =
             __bfloat162bfloat162(reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff)[lrow]);
-        uint4* wrow = reinterpret_cast<uint4*>(st + lrow * 128);
+        uint4* wrow = reinterpret_cast<uint4*>(st + C::kWOff + lrow * 128);
 #pragma unroll
         for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
         fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
@@ -293,31 +322,31 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         rp.next(S);
       }
       if (tr) {
-        p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + kTrDqWait] = t_wait;
-        p.trace[static_cast<size_t>(blockIdx.x) * kSmTracePoints + kTrDqWork] = t_work;
+        p.trace[static_cast<size_t>(blockIdx.x) * kSmTraceStride + kTrDqWait] = t_wait;
+        p.trace[static_cast<size_t>(blockIdx.x) * kSmTraceStride + kTrDqWork] = t_work;
       }
     }
     bool got = true;
     if (nk > 0) got = mbar_wait(acc_full, 0, ctl);
     const bool ok = bar_sync_and<1, 128>(got);
-    // only the first r rows of the T partial are real (warp-uniform test)
-    const bool t_rows = q * 32 < p.r;
+    // the T partial's lanes are tokens: only the first kNT are real (a
+    // warp-uniform test); each such thread parks its token's r values
+    // transposed, Tp[c][token], the layout the cluster sum below reads
+    const bool t_rows = q * 32 < kNT;
     float4* drow = reinterpret_cast<float4*>(Dp + lrow * C::kLd);
-    float4* trow = reinterpret_cast<float4*>(Tp + lrow * C::kLd);
     const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
     if (ok && t_rows) {
       if (nk > 0) {
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < kNT; c0 += 16) {
+        for (int c0 = 0; c0 < p.a_rows; c0 += 16) {
           float t[16];
           tmem_ld16f(tl + static_cast<uint32_t>(kNT + c0), t);
 #pragma unroll
-          for (int c = 0; c < 16; c += 4) trow[(c0 + c) / 4] = make_float4(t[c], t[c + 1], t[c + 2], t[c + 3]);
+          for (int c = 0; c < 16; ++c)
+            if (c0 + c < p.r) Tp[(c0 + c) * C::kLd + lrow] = t[c];
         }
       } else {
-#pragma unroll
-        for (int c = 0; c < kNT / 4; ++c) trow[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int c = 0; c < p.r; ++c) Tp[c * C::kLd + lrow] = 0.0f;
       }
     }
     if (ok) {
@@ -388,10 +417,10 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       }
       float z[4] = {zs.x, zs.y, zs.z, zs.w};
       float lora[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      const float* brow = Bs + fl * (p.r + 1);
+      const __nv_bfloat16* brow = Bs + fl * (p.r + 2);
       const float4* tcol = reinterpret_cast<const float4*>(Tf) + m0 / 4;
       for (int c = 0; c < p.r; ++c) {
-        const float b = brow[c];
+        const float b = __bfloat162float(brow[c]);
         const float4 t = tcol[c * (kNT / 4)];
         lora[0] = fmaf(b, t.x, lora[0]);
         lora[1] = fmaf(b, t.y, lora[1]);
@@ -424,10 +453,10 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   }
 }
 
-template <int kNT, bool kW4>
+template <int kNT, bool kW4, int kAR>
 cudaError_t launch_small_m_kernel(const SmallMParams& p, int slices, bool pdl, cudaStream_t st) {
-  using C = SmallMCfg<kNT, kW4>;
-  auto k = small_m_kernel<kNT, kW4>;
+  using C = SmallMCfg<kNT, kW4, kAR>;
+  auto k = small_m_kernel<kNT, kW4, kAR>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -452,10 +481,10 @@ cudaError_t launch_small_m_kernel(const SmallMParams& p, int slices, bool pdl, c
 // Cluster size: the largest power of two (<= 16, <= the K blocks) with which
 // all slices' clusters are resident at once (the device's answer for this
 // kernel, shared memory and cluster shape), so the launch is a single wave.
-template <int kNT, bool kW4>
+template <int kNT, bool kW4, int kAR>
 int small_m_splits_t(int slices, int nkb) {
-  using C = SmallMCfg<kNT, kW4>;
-  auto k = small_m_kernel<kNT, kW4>;
+  using C = SmallMCfg<kNT, kW4, kAR>;
+  auto k = small_m_kernel<kNT, kW4, kAR>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
@@ -485,28 +514,36 @@ int small_m_splits_t(int slices, int nkb) {
   return best;
 }
 
-inline int small_m_splits(int nt, bool w4, int64_t d_in, int64_t d_out) {
+// A-slot rows reserved per K block: 16 (r <= 16) or 64 (r <= 64).
+inline int small_m_ar(int64_t r) { return r <= 16 ? 16 : 64; }
+
+template <bool kW4, int kAR>
+int small_m_splits_ar(int nt, int slices, int nkb) {
+  if (nt == 16) return small_m_splits_t<16, kW4, kAR>(slices, nkb);
+  if (nt == 32) return small_m_splits_t<32, kW4, kAR>(slices, nkb);
+  return small_m_splits_t<64, kW4, kAR>(slices, nkb);
+}
+
+inline int small_m_splits(int nt, bool w4, int64_t r, int64_t d_in, int64_t d_out) {
   const int slices = static_cast<int>((d_out + 127) / 128);
   const int nkb = static_cast<int>((d_in + 63) / 64);
-  if (w4) {
-    if (nt == 16) return small_m_splits_t<16, true>(slices, nkb);
-    if (nt == 32) return small_m_splits_t<32, true>(slices, nkb);
-    return small_m_splits_t<64, true>(slices, nkb);
-  }
-  if (nt == 16) return small_m_splits_t<16, false>(slices, nkb);
-  if (nt == 32) return small_m_splits_t<32, false>(slices, nkb);
-  return small_m_splits_t<64, false>(slices, nkb);
+  const bool a16 = small_m_ar(r) == 16;
+  if (w4) return a16 ? small_m_splits_ar<true, 16>(nt, slices, nkb) : small_m_splits_ar<true, 64>(nt, slices, nkb);
+  return a16 ? small_m_splits_ar<false, 16>(nt, slices, nkb) : small_m_splits_ar<false, 64>(nt, slices, nkb);
+}
+
+template <bool kW4, int kAR>
+cudaError_t launch_small_m_ar(const SmallMParams& p, int nt, int slices, bool pdl, cudaStream_t st) {
+  if (nt == 16) return launch_small_m_kernel<16, kW4, kAR>(p, slices, pdl, st);
+  if (nt == 32) return launch_small_m_kernel<32, kW4, kAR>(p, slices, pdl, st);
+  return launch_small_m_kernel<64, kW4, kAR>(p, slices, pdl, st);
 }
 
 inline cudaError_t launch_small_m(const SmallMParams& p, int nt, bool w4, int slices, bool pdl, cudaStream_t st) {
-  if (w4) {
-    if (nt == 16) return launch_small_m_kernel<16, true>(p, slices, pdl, st);
-    if (nt == 32) return launch_small_m_kernel<32, true>(p, slices, pdl, st);
-    return launch_small_m_kernel<64, true>(p, slices, pdl, st);
-  }
-  if (nt == 16) return launch_small_m_kernel<16, false>(p, slices, pdl, st);
-  if (nt == 32) return launch_small_m_kernel<32, false>(p, slices, pdl, st);
-  return launch_small_m_kernel<64, false>(p, slices, pdl, st);
+  const bool a16 = small_m_ar(p.r) == 16;
+  if (w4) return a16 ? launch_small_m_ar<true, 16>(p, nt, slices, pdl, st) : launch_small_m_ar<true, 64>(p, nt, slices, pdl, st);
+  return a16 ? launch_small_m_ar<false, 16>(p, nt, slices, pdl, st)
+             : launch_small_m_ar<false, 64>(p, nt, slices, pdl, st);
 }
 
 }  // namespace lora

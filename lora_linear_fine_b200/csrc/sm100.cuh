@@ -182,7 +182,15 @@ __device__ __forceinline__ void bar_sync_named() {
 // completed and its memory operations are visible (without the attribute it
 // returns at once).  Every kernel here calls it from every thread after its
 // prologue (barriers, tensor memory) and before its first global access.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Right after the wait it lets the next kernel in the stream be launched
+// (griddepcontrol.launch_dependents): that kernel's CTAs are placed as SMs
+// free up and run their own prologue while this grid finishes; they touch
+// global memory only after their own wait, i.e. after this grid completed.
+// Triggering after the wait keeps at most one grid launched ahead.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tensor core operand reads, TMA stores).
