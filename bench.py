@@ -1039,8 +1039,9 @@ def main():
                     help="skip the other workloads' entries of the default line")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--shape", default=None,
-                    help="M,d_in,d_out,r,act: this shape instead of --config (profiling, with --calls); "
-                         "act 'ce': the output projection + cross-entropy with d_in = hidden, d_out = V")
+                    help="M,d_in,d_out,r,act[,p_drop]: this shape instead of --config (profiling, with --calls); "
+                         "act 'ce': the output projection + cross-entropy with d_in = hidden, d_out = V; "
+                         "p_drop: dropout on the adapter input")
     ap.add_argument("--calls", type=int, default=0,
                     help="run this many untimed forward(+backward) calls, print nothing else, exit (for profilers)")
     ap.add_argument("--fwd-only", action="store_true", help="with --calls: forward calls only")
@@ -1051,6 +1052,8 @@ def main():
         f = args.shape.split(",")
         cfg = dict(M=int(f[0]), d_in=int(f[1]), d_out=int(f[2]), r=int(f[3]), alpha=16.0 if int(f[3]) else 0.0,
                    act=f[4])
+        if len(f) > 5:
+            cfg["dropout"] = float(f[5])
         args.config = "shape " + args.shape
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -333,13 +333,15 @@ lora_status_t lora_linear_fwd_w4_tiled(const lora_linear_desc* desc, const void*
  * T_save holds (X * mask) A^T, without the 1/(1 - p_drop) factor; pass it
  * back to lora_linear_bwd_dropout unchanged.  With r == 0 these calls are the
  * plain ones.  The few-token kernel is not used (dropout is a training-time
- * transform); the masked input is written to the workspace, and the LoRA term
- * of dX is added after the dX GEMM (dx_dropout_kernel).
+ * transform).  No masked copy of X is made: the rank passes that read X for
+ * the adapter (T, dA) zero the dropped elements of each X tile in shared
+ * memory, and the LoRA term of dX is added in the dX GEMM's epilogue (one
+ * projection, r <= 64) or by dx_dropout_kernel after it (SwiGLU, r > 64).
  * ------------------------------------------------------------------------ */
 
 /* Workspace bytes for lora_linear_fwd_dropout (0) / lora_linear_bwd_dropout
- * (1): the layer's workspace plus the masked input(s), M * d_in * 2 bytes per
- * projection.  0 for an invalid desc. */
+ * (1): the layer's workspace for the tiled path (the few-token forward, which
+ * needs none, is not used here).  0 for an invalid desc. */
 size_t lora_linear_workspace_size_dropout(const lora_linear_desc* desc, int for_backward);
 
 lora_status_t lora_linear_fwd_dropout(const lora_linear_desc* desc, const void* X, const void* W, const void* A,

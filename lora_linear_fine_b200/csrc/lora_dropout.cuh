@@ -8,9 +8,11 @@
 //   Z  = X W^T + s' (X_m A^T) B^T
 //   dA = s' U^T X_m,   dB = s' dZ^T (X_m A^T),   U = dZ B
 //   dX = dZ W + m * (s' U A)
-// so the rank passes run unchanged on X_m, and only the LoRA term of dX needs
-// the mask: the dX GEMM then runs without its LoRA K-block and
-// dx_dropout_kernel adds m * (s' U A) afterwards.
+// X_m is never stored: the rank passes that read X for the adapter (T and
+// dA) zero the dropped elements of their X tiles in shared memory.  Only the
+// LoRA term of dX needs the mask outside them: the dX GEMM runs without its
+// LoRA K-block and adds m * (s' U A) in its epilogue (one projection, r <= 64)
+// or dx_dropout_kernel, below, adds it afterwards (SwiGLU, r > 64).
 //
 // Mask layout: [M x d_in/8] bytes, bit j of byte b (least significant first)
 // keeps element 8 b + j.
@@ -22,28 +24,6 @@
 #include "sm100.cuh"
 
 namespace lora {
-
-// X_m = X * m, bf16 [M x d_in].  One thread per 8 elements (16 bytes of X, one
-// mask byte), grid-stride, coalesced.
-__global__ void __launch_bounds__(256) mask_x_kernel(const __nv_bfloat16* __restrict__ X,
-                                                     const uint8_t* __restrict__ mask, long long n8,
-                                                     __nv_bfloat16* __restrict__ Xm) {
-  grid_dep_wait();
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint4 v = reinterpret_cast<const uint4*>(X)[i];
-    const uint32_t b = mask[i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
-      const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
-      o[e] = w[e] & (lo | hi);
-    }
-    reinterpret_cast<uint4*>(Xm)[i] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-}
 
 struct DxDropoutJob {
   const uint8_t* mask;          // [M x d_in/8]

@@ -825,7 +825,7 @@ lora_status_t dequant_w4(const void* Wq, const void* Ws, int64_t d_out, int64_t 
   return check_launch("dequant_w4_kernel");
 }
 
-// Dropout on the adapter branch's input: checks, workspace, the masked inputs.
+// Dropout on the adapter branch's input: checks and workspace.
 lora_status_t check_dropout(const lora_linear_desc* d, const void* X, const void* mask, const void* mask_up,
                             float p_drop) {
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return LORA_ERR_INVALID_ARG;
@@ -841,29 +841,6 @@ size_t dropout_base_bytes(const lora_linear_desc* d, bool backward) {
   if (!backward) return fwd;
   const size_t bwd = make_plan(d, true).total;
   return bwd > fwd ? bwd : fwd;
-}
-
-// The masked copies X * m_j of the adapter inputs, one per projection.
-size_t dropout_xm_bytes(const lora_linear_desc* d) {
-  const size_t np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
-  return np * align_up(static_cast<size_t>(d->M) * static_cast<size_t>(d->d_in) * 2, 256);
-}
-
-lora_status_t mask_inputs(const lora_linear_desc* d, const void* X, const void* mask, const void* mask_up,
-                          uint8_t* dst, const void* Xl[2], const DevInfo& dev, cudaStream_t st) {
-  const int np = d->act == LORA_ACT_SWIGLU ? 2 : 1;
-  const long long n8 = d->M * d->d_in / 8;
-  const size_t stride = align_up(static_cast<size_t>(d->M) * static_cast<size_t>(d->d_in) * 2, 256);
-  for (int j = 0; j < 2; ++j) {
-    if (j >= np) { Xl[j] = Xl[0]; continue; }
-    uint8_t* xm = dst + j * stride;
-    launch_k(mask_x_kernel, dim3(grid_for(n8, 256, dev.sms)), dim3(256), 0, st, false,
-             static_cast<const __nv_bfloat16*>(X), static_cast<const uint8_t*>(j == 0 ? mask : mask_up), n8,
-             reinterpret_cast<__nv_bfloat16*>(xm));
-    LORA_TRY(check_launch("mask_x_kernel"));
-    Xl[j] = xm;
-  }
-  return LORA_OK;
 }
 
 // Rotary tables of the attention-input projections: checks shared by the
@@ -1563,7 +1540,7 @@ lora_status_t lora_linear_bwd_w4(const lora_linear_desc* d, const void* dY, cons
 // ---------------------------------------------------------------------------
 size_t lora_linear_workspace_size_dropout(const lora_linear_desc* desc, int for_backward) {
   if (check_desc(desc) != LORA_OK) return 0;
-  return align_up(dropout_base_bytes(desc, for_backward != 0), 256) + dropout_xm_bytes(desc);
+  return align_up(dropout_base_bytes(desc, for_backward != 0), 256);
 }
 
 lora_status_t lora_linear_fwd_dropout(const lora_linear_desc* d, const void* X, const void* W, const void* A,
@@ -1578,7 +1555,7 @@ lora_status_t lora_linear_fwd_dropout(const lora_linear_desc* d, const void* X, 
   d2.s = d->s / (1.0f - p_drop);
   const size_t base = align_up(dropout_base_bytes(d, false), 256);
   DevInfo dev;
-  LORA_TRY(common_checks(d, workspace, workspace_bytes, base + dropout_xm_bytes(d), &dev));
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, base, &dev));
   if (d->M == 0) return LORA_OK;
   // the T pass reads X and applies the mask to its tiles in shared memory:
   // no masked copy of X in the forward
@@ -1604,7 +1581,7 @@ lora_status_t lora_linear_bwd_dropout(const lora_linear_desc* d, const void* dY,
   d2.s = d->s / (1.0f - p_drop);
   const size_t base = align_up(dropout_base_bytes(d, true), 256);
   DevInfo dev;
-  LORA_TRY(common_checks(d, workspace, workspace_bytes, base + dropout_xm_bytes(d), &dev));
+  LORA_TRY(common_checks(d, workspace, workspace_bytes, base, &dev));
   // the rank passes read X and apply the mask to their tiles in shared
   // memory; the dX GEMM adds the masked LoRA term in its epilogue
   const void* Xl[2] = {X, X};

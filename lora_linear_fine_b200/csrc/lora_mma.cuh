@@ -387,6 +387,27 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       const uint32_t use = it >> 1;
       const int row = mt * C::kTileM + 128 * static_cast<int>(crank) + row_in_tile;
       const bool row_ok = row < p.M;
+      // Dropout: this row's s'U (hi + lo) and its keep bytes for the tile's
+      // 128 columns do not depend on the accumulator; their loads are issued
+      // before the wait for it.
+      constexpr bool kDrop = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
+      float du[kDrop ? kDropMaxRank : 1];
+      uint32_t dkeep[4];
+      if constexpr (kDrop) {
+        const DropEpi& D = p.drop;
+#pragma unroll
+        for (int c = 0; c < kDropMaxRank; ++c) {
+          du[c] = 0.0f;
+          if (c < D.r && row_ok) {
+            const size_t at = static_cast<size_t>(c) * D.ld + row;
+            du[c] = __bfloat162float(D.ut_hi[at]) + __bfloat162float(D.ut_lo[at]);
+          }
+        }
+        const int ldm = p.N / 8;
+        const bool vec = (reinterpret_cast<uintptr_t>(D.mask) % 16) == 0 && ldm % 16 == 0;
+        load_keep_bytes<16>(D.mask + static_cast<size_t>(row_ok ? row : 0) * ldm, (nt * 256 + h * 128) / 8, ldm,
+                            row_ok, vec, dkeep);
+      }
       if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
@@ -596,21 +617,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         }
       } else if constexpr (kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop) {
         // dX = dZ W (the accumulator) + m * (s' U A): this thread's row of
-        // s'U (hi + lo, fp32) in registers, the tile's columns of A read as
-        // warp-wide broadcasts (every lane of a warp reads the same 16
-        // bytes), 16 columns at a time; one bf16 rounding at the end.
+        // s'U (hi + lo, fp32) and keep bytes in registers (loaded above), the
+        // tile's columns of A read as warp-wide broadcasts (every lane of a
+        // warp reads the same 16 bytes), 16 columns at a time; one bf16
+        // rounding at the end.
         const int col0 = nt * 256 + h * 128;
         const DropEpi& D = p.drop;
-        float u[kDropMaxRank];
-#pragma unroll
-        for (int c = 0; c < kDropMaxRank; ++c) {
-          u[c] = 0.0f;
-          if (c < D.r && row_ok) {
-            const size_t at = static_cast<size_t>(c) * D.ld + row;
-            u[c] = __bfloat162float(D.ut_hi[at]) + __bfloat162float(D.ut_lo[at]);
-          }
-        }
-        const size_t mrow = static_cast<size_t>(row) * (p.N / 8);
 #pragma unroll 1
         for (int c16 = 0; c16 < 8; ++c16) {
           uint32_t v[16];
@@ -633,11 +645,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              t[2 * e] = fmaf(u[c], __uint_as_float(w[e] << 16), t[2 * e]);
-              t[2 * e + 1] = fmaf(u[c], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
+              t[2 * e] = fmaf(du[c], __uint_as_float(w[e] << 16), t[2 * e]);
+              t[2 * e + 1] = fmaf(du[c], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
             }
           }
-          const uint32_t mb = D.mask[mrow + cb / 8] | (two ? static_cast<uint32_t>(D.mask[mrow + cb / 8 + 1]) << 8 : 0u);
+          const uint32_t mb = (dkeep[c16 >> 1] >> (16 * (c16 & 1))) & 0xFFFFu;   // keep bytes 2 c16, 2 c16 + 1
           float z[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) z[j] = __uint_as_float(v[j]) + (((mb >> j) & 1u) ? t[j] : 0.0f);

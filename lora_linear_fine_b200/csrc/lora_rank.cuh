@@ -232,41 +232,28 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
     const int row = q * 32 + lane;
     if (masking) {
       // Dropout: zero the dropped elements of each stage's X tiles.  Thread
-      // `row` owns row `row` of every [128 x 64] SWIZZLE_128B box: 16-byte
-      // chunk c (features 8c .. 8c + 7) at position c ^ (row & 7), masked by
-      // byte c of the row's 8 mask bytes for that K block.
+      // `row` owns row `row` of every [128 x 64] SWIZZLE_128B box and its
+      // 8 * KS keep bytes per stage, loaded one stage ahead so that their
+      // latency hides behind the wait for the tiles.
+      constexpr int kMB = 8 * KS;
       const int grow = mt * 128 + row;
       const bool in_rows = grow < p.rows;
       const uint8_t* mrow = p.mask + static_cast<size_t>(in_rows ? grow : 0) * p.mask_ld;
+      const bool vec = (reinterpret_cast<uintptr_t>(p.mask) % kMB) == 0 && p.mask_ld % kMB == 0;
+      uint32_t cur[kMB / 4], nxt[kMB / 4];
+      if (nkb > 0) load_keep_bytes<kMB>(mrow, kb0 * kMB, p.mask_ld, in_rows, vec, cur);
       RingPos rp;
       for (int i = 0; i < nkb; ++i) {
+        if (i + 1 < nkb) load_keep_bytes<kMB>(mrow, (kb0 + i + 1) * kMB, p.mask_ld, in_rows, vec, nxt);
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
-        const int k0 = (kb0 + i) * 64 * KS;
 #pragma unroll
-        for (int kb = 0; kb < KS; ++kb) {
-          uint4* trow = reinterpret_cast<uint4*>(st + kb * 16384 + row * 128);
-          const int byte0 = (k0 + 64 * kb) / 8;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t b = (in_rows && byte0 + c < p.mask_ld) ? mrow[byte0 + c] : 0u;
-            if (b == 0xFFu) continue;
-            uint4& slot = trow[c ^ (row & 7)];
-            const uint4 v = slot;
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
-              const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
-              o[e] = w[e] & (lo | hi);
-            }
-            slot = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        }
+        for (int kb = 0; kb < KS; ++kb) mask_sw128_row(st + kb * 16384 + row * 128, row, cur + 2 * kb);
         fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&masked[rp.stage]);
+#pragma unroll
+        for (int w = 0; w < kMB / 4; ++w) cur[w] = nxt[w];
         rp.next(S);
       }
     }

@@ -249,43 +249,34 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
     }
     if constexpr (kCol && !kRow) {
       if (masking) {
-        // Thread lrow owns token row lrow of both boxes of every stage: 16-byte
-        // chunk c (features 8c .. 8c + 7 of the box) at position c ^ (lrow & 7),
-        // masked by byte c of the row's 8 mask bytes for that box.
-        RingPos rp;
-        bool ok = true;
-        for (int i = 0; i < na && ok; ++i) {
+        // Thread lrow owns token row lrow of both [128 x 64] SWIZZLE_128B boxes
+        // of every stage and the row's 16 keep bytes for the stage's 128
+        // features, loaded one stage ahead so that their latency hides behind
+        // the wait for the tiles.
+        const bool vec = (reinterpret_cast<uintptr_t>(p.mask) % 16) == 0 && p.mask_ld % 16 == 0;
+        auto keep = [&](int i, int j, uint32_t (&m)[4]) {
           const int tok = (ti0 + i) * 128 + lrow;
           const bool in_rows = tok < p.mtok;
           const uint8_t* mrow = p.mask + static_cast<size_t>(in_rows ? tok : 0) * p.mask_ld;
+          load_keep_bytes<16>(mrow, (fj0 + j) * 16, p.mask_ld, in_rows, vec, m);
+        };
+        uint32_t cur[4], nxt[4];
+        keep(0, 0, cur);
+        RingPos rp;
+        bool ok = true;
+        for (int i = 0; i < na && ok; ++i) {
           for (int j = 0; j < nb; ++j) {
+            const bool last_j = j + 1 == nb;
+            if (!last_j || i + 1 < na) keep(last_j ? i + 1 : i, last_j ? 0 : j + 1, nxt);
             if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
             uint8_t* st = smem + rp.stage * C::kStageBytes;
-            const int f0 = (fj0 + j) * 128;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint4* trow = reinterpret_cast<uint4*>(st + h * C::kZBox + lrow * 128);
-              const int byte0 = (f0 + 64 * h) / 8;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint32_t b = (in_rows && byte0 + c < p.mask_ld) ? mrow[byte0 + c] : 0u;
-                if (b == 0xFFu) continue;
-                uint4& slot = trow[c ^ (lrow & 7)];
-                const uint4 v = slot;
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
-                  const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
-                  o[e] = w[e] & (lo | hi);
-                }
-                slot = make_uint4(o[0], o[1], o[2], o[3]);
-              }
-            }
+            for (int h = 0; h < 2; ++h) mask_sw128_row(st + h * C::kZBox + lrow * 128, lrow, cur + 2 * h);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&masked[rp.stage]);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) cur[w] = nxt[w];
             rp.next(S);
           }
         }

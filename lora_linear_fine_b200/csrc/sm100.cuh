@@ -199,6 +199,60 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ----------------------------------------------------------------------------
+// Dropout keep bits: one bit per element, bit j of byte b keeping element
+// 8 b + j of a row of `ld` bytes.
+// ----------------------------------------------------------------------------
+
+// kBytes consecutive keep bytes of one row from byte b0 (a multiple of
+// kBytes), packed four to a word.  One vector load when the row start is
+// kBytes-aligned (`vec`), byte loads otherwise; bytes at or past `ld`, and all
+// bytes of a row that does not exist (!ok), read as 0.  All loads are issued
+// before any value is used, so their latencies overlap.
+template <int kBytes>
+__device__ __forceinline__ void load_keep_bytes(const uint8_t* mrow, int b0, int ld, bool ok, bool vec,
+                                                uint32_t (&m)[kBytes / 4]) {
+  static_assert(kBytes == 8 || kBytes == 16, "8 or 16 keep bytes");
+  if (ok && vec && b0 + kBytes <= ld) {
+    if constexpr (kBytes == 16) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(mrow + b0));
+      m[0] = v.x; m[1] = v.y; m[2] = v.z; m[3] = v.w;
+    } else {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(mrow + b0));
+      m[0] = v.x; m[1] = v.y;
+    }
+    return;
+  }
+  uint32_t b[kBytes];
+#pragma unroll
+  for (int c = 0; c < kBytes; ++c) b[c] = (ok && b0 + c < ld) ? static_cast<uint32_t>(__ldg(mrow + b0 + c)) : 0u;
+#pragma unroll
+  for (int w = 0; w < kBytes / 4; ++w) m[w] = b[4 * w] | (b[4 * w + 1] << 8) | (b[4 * w + 2] << 16) | (b[4 * w + 3] << 24);
+}
+
+// Zero the dropped elements of one 128-byte row of a SWIZZLE_128B bf16 box:
+// 16-byte chunk c (elements 8c .. 8c + 7) sits at position c ^ (row & 7) and
+// takes keep byte c (byte c % 4 of word c / 4 of `m`).
+__device__ __forceinline__ void mask_sw128_row(uint8_t* row_base, int row, const uint32_t* m) {
+  uint4* trow = reinterpret_cast<uint4*>(row_base);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t b = (m[c >> 2] >> (8 * (c & 3))) & 0xFFu;
+    if (b == 0xFFu) continue;
+    uint4& slot = trow[c ^ (row & 7)];
+    const uint4 v = slot;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
+      const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
+      o[e] = w[e] & (lo | hi);
+    }
+    slot = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation MMA
 // ----------------------------------------------------------------------------
 // Allocate `ncols` (power of two >= 32) TMEM columns; the base address is
