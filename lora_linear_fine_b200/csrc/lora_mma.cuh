@@ -387,22 +387,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       const uint32_t use = it >> 1;
       const int row = mt * C::kTileM + 128 * static_cast<int>(crank) + row_in_tile;
       const bool row_ok = row < p.M;
-      // Dropout: this row's s'U (hi + lo) and its keep bytes for the tile's
-      // 128 columns do not depend on the accumulator; their loads are issued
-      // before the wait for it.
+      // Dropout: this row's keep bytes for the tile's 128 columns do not
+      // depend on the accumulator; their load is issued before the wait for it.
       constexpr bool kDrop = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
-      float du[kDrop ? kDropMaxRank : 1];
       uint32_t dkeep[4];
       if constexpr (kDrop) {
         const DropEpi& D = p.drop;
-#pragma unroll
-        for (int c = 0; c < kDropMaxRank; ++c) {
-          du[c] = 0.0f;
-          if (c < D.r && row_ok) {
-            const size_t at = static_cast<size_t>(c) * D.ld + row;
-            du[c] = __bfloat162float(D.ut_hi[at]) + __bfloat162float(D.ut_lo[at]);
-          }
-        }
         const int ldm = p.N / 8;
         const bool vec = (reinterpret_cast<uintptr_t>(D.mask) % 16) == 0 && ldm % 16 == 0;
         load_keep_bytes<16>(D.mask + static_cast<size_t>(row_ok ? row : 0) * ldm, (nt * 256 + h * 128) / 8, ldm,
@@ -616,11 +606,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           }
         }
       } else if constexpr (kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop) {
-        // dX = dZ W (the accumulator) + m * (s' U A): this thread's row of
-        // s'U (hi + lo, fp32) and keep bytes in registers (loaded above), the
-        // tile's columns of A read as warp-wide broadcasts (every lane of a
-        // warp reads the same 16 bytes), 16 columns at a time; one bf16
-        // rounding at the end.
+        // dX = dZ W (the accumulator) + m * (s' U A), 16 columns at a time:
+        // the tile's columns of A are read as warp-wide broadcasts (every lane
+        // of a warp reads the same 16 bytes) and this thread's row of s'U
+        // (hi + lo, fp32) with them, eight ranks per batch of loads so that a
+        // batch costs one memory latency; keep bytes in registers (loaded
+        // above); one bf16 rounding at the end.
         const int col0 = nt * 256 + h * 128;
         const DropEpi& D = p.drop;
 #pragma unroll 1
@@ -636,17 +627,29 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < 16; ++j) t[j] = 0.0f;
           const bool two = cb + 8 < p.N;
+          for (int g = 0; g < D.r; g += 8) {
+            uint4 a0[8], a1[8];
+            float u[8];
 #pragma unroll
-          for (int c = 0; c < kDropMaxRank; ++c) {
-            if (c >= D.r) break;
-            const uint4* ap = reinterpret_cast<const uint4*>(D.A + static_cast<size_t>(c) * p.N + cb);
-            const uint4 a0 = __ldg(ap);
-            const uint4 a1 = two ? __ldg(ap + 1) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            for (int k = 0; k < 8; ++k) {
+              // ranks past r contribute exact zeros (u = 0, A = 0; no load)
+              const bool in = g + k < D.r;
+              const int c = in ? g + k : 0;
+              const uint4* ap = reinterpret_cast<const uint4*>(D.A + static_cast<size_t>(c) * p.N + cb);
+              a0[k] = in ? __ldg(ap) : make_uint4(0u, 0u, 0u, 0u);
+              a1[k] = in && two ? __ldg(ap + 1) : make_uint4(0u, 0u, 0u, 0u);
+              const size_t at = static_cast<size_t>(c) * D.ld + row;
+              const float uh = __bfloat162float(D.ut_hi[at]), ul = __bfloat162float(D.ut_lo[at]);
+              u[k] = in ? uh + ul : 0.0f;
+            }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              t[2 * e] = fmaf(du[c], __uint_as_float(w[e] << 16), t[2 * e]);
-              t[2 * e + 1] = fmaf(du[c], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t w[8] = {a0[k].x, a0[k].y, a0[k].z, a0[k].w, a1[k].x, a1[k].y, a1[k].z, a1[k].w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                t[2 * e] = fmaf(u[k], __uint_as_float(w[e] << 16), t[2 * e]);
+                t[2 * e + 1] = fmaf(u[k], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
+              }
             }
           }
           const uint32_t mb = (dkeep[c16 >> 1] >> (16 * (c16 & 1))) & 0xFFFFu;   // keep bytes 2 c16, 2 c16 + 1

@@ -247,8 +247,7 @@ __global__ void __launch_bounds__(kRankThreads, 1) rank_gemm_kernel(const __grid
         if (i + 1 < nkb) load_keep_bytes<kMB>(mrow, (kb0 + i + 1) * kMB, p.mask_ld, in_rows, vec, nxt);
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
-#pragma unroll
-        for (int kb = 0; kb < KS; ++kb) mask_sw128_row(st + kb * 16384 + row * 128, row, cur + 2 * kb);
+        mask_sw128_rows<KS>(st + row * 128, 16384, row, cur);
         fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&masked[rp.stage]);
@@ -303,12 +302,13 @@ struct RankReduceJob {
   RankOut out;
 };
 
-// Blocks of rpb (<= kReduceRows) result rows (grid-stride over row blocks; blockIdx.y
-// selects the job).  Splits are summed in order into a shared-memory tile with
-// the column fastest (the partials' layout), each thread keeping up to
-// 2 elements x 8 splits of loads in flight; then row-major outputs are written
-// column-fastest and transposed outputs row-fastest, so every global access is
-// coalesced.
+// Blocks of rpb (<= kReduceRows) result rows (grid-stride over row blocks;
+// blockIdx.y selects the job).  Each thread sums float4 pieces of the partial
+// rows over the splits in split order (eight splits of loads in flight), into
+// a shared-memory tile; then row-major outputs are written by warps along a
+// row and transposed outputs by warps along a column, so every global access
+// is coalesced and no index needs a division.  RP is a power of two and r a
+// multiple of 8, so a float4 piece lies wholly inside or wholly past r.
 constexpr int kReduceRows = 32;
 constexpr int kMaxRank = 128;
 
@@ -320,71 +320,90 @@ __global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, R
   const RankOut& o = J.out;
   const int rpb = J.rpb;
   const int nblk = (J.out.rows + rpb - 1) / rpb;
-  const size_t stride = static_cast<size_t>(J.rows_pad) * J.RP;   // between splits
+  const int q4 = J.RP / 4;                    // float4 pieces per partial row
+  const int lgq = __ffs(q4) - 1;
+  const size_t stride4 = static_cast<size_t>(J.rows_pad) * q4;   // between splits, in float4
+  const float4* part4 = reinterpret_cast<const float4*>(J.partial);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kEPT = 2;
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
     const int row0 = blk * rpb;
     const int nrows = J.out.rows - row0 < rpb ? J.out.rows - row0 : rpb;
-    const int E = nrows * r;
+    const int U = nrows * q4;
     __syncthreads();
-    for (int base = 0; base < E; base += 256 * kEPT) {
-      float acc[kEPT];
-      const float* src[kEPT];
+    for (int base = 0; base < U; base += 256 * kEPT) {
+      float4 acc[kEPT];
+      const float4* src[kEPT];
       bool in[kEPT];
+      int rr[kEPT], c0[kEPT];
 #pragma unroll
       for (int e = 0; e < kEPT; ++e) {
-        const int i = base + static_cast<int>(threadIdx.x) + 256 * e;
-        in[e] = i < E;
-        const int rr = in[e] ? i / r : 0, c = in[e] ? i - rr * r : 0;
-        src[e] = J.partial + static_cast<size_t>(row0 + rr) * J.RP + c;
-        acc[e] = 0.0f;
+        const int u = base + static_cast<int>(threadIdx.x) + 256 * e;
+        rr[e] = u >> lgq;
+        c0[e] = 4 * (u & (q4 - 1));
+        in[e] = u < U && c0[e] < r;
+        src[e] = part4 + static_cast<size_t>(row0 + (in[e] ? rr[e] : 0)) * q4 + (c0[e] >> 2);
+        acc[e] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       }
       for (int sp0 = 0; sp0 < J.splits; sp0 += 8) {
-        float v[kEPT][8];
+        float4 v[kEPT][8];
 #pragma unroll
         for (int e = 0; e < kEPT; ++e)
 #pragma unroll
-          for (int u = 0; u < 8; ++u) v[e][u] = (in[e] && sp0 + u < J.splits) ? src[e][(sp0 + u) * stride] : 0.0f;
+          for (int k = 0; k < 8; ++k)
+            v[e][k] = (in[e] && sp0 + k < J.splits) ? __ldcg(src[e] + static_cast<size_t>(sp0 + k) * stride4)
+                                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
         for (int e = 0; e < kEPT; ++e)
 #pragma unroll
-          for (int u = 0; u < 8; ++u) acc[e] += v[e][u];      // split order; + 0 past the last split
+          for (int k = 0; k < 8; ++k) {      // split order; + 0 past the last split
+            acc[e].x += v[e][k].x;
+            acc[e].y += v[e][k].y;
+            acc[e].z += v[e][k].z;
+            acc[e].w += v[e][k].w;
+          }
       }
 #pragma unroll
       for (int e = 0; e < kEPT; ++e) {
-        const int i = base + static_cast<int>(threadIdx.x) + 256 * e;
-        if (in[e]) tile[i / r][i % r] = acc[e];
+        if (!in[e]) continue;
+        float* t = &tile[rr[e]][c0[e]];
+        t[0] = acc[e].x;
+        t[1] = acc[e].y;
+        t[2] = acc[e].z;
+        t[3] = acc[e].w;
       }
     }
     __syncthreads();
-    // row-major outputs: column fastest
+    // row-major outputs: a warp along a row (columns across lanes)
     if ((o.f32 != nullptr && !o.transpose_f32) || o.s16 != nullptr) {
-      for (int i = threadIdx.x; i < nrows * r; i += blockDim.x) {
-        const int rr = i / r, c = i - rr * r;
-        const float v = tile[rr][c];
-        const size_t idx = static_cast<size_t>(row0 + rr) * r + c;
-        if (o.f32 != nullptr && !o.transpose_f32) o.f32[idx] = v;
-        if (o.s16 != nullptr) o.s16[idx] = __float2bfloat16_rn(o.scale * v);
+      for (int rr = warp; rr < nrows; rr += 8) {
+        const size_t rowoff = static_cast<size_t>(row0 + rr) * r;
+        for (int c = lane; c < r; c += 32) {
+          const float v = tile[rr][c];
+          if (o.f32 != nullptr && !o.transpose_f32) o.f32[rowoff + c] = v;
+          if (o.s16 != nullptr) o.s16[rowoff + c] = __float2bfloat16_rn(o.scale * v);
+        }
       }
     }
-    // transposed outputs: row fastest
+    // transposed outputs: a warp along a column (rows across lanes)
     if ((o.f32 != nullptr && o.transpose_f32) || o.hi != nullptr) {
-      for (int i = threadIdx.x; i < nrows * r; i += blockDim.x) {
-        const int c = i / nrows, rr = i - c * nrows;
-        const float v = tile[rr][c];
-        const int row = row0 + rr;
-        if (o.f32 != nullptr && o.transpose_f32) o.f32[static_cast<size_t>(c) * o.rows + row] = v;
-        if (o.hi != nullptr) {
-          const float x = o.scale * v;
-          const size_t k = static_cast<size_t>(c) * o.ld + row;
-          if (o.hilo_f16) {
-            const __half h = __float2half_rn(x);
-            static_cast<__half*>(o.hi)[k] = h;
-            static_cast<__half*>(o.lo)[k] = __float2half_rn(x - __half2float(h));
-          } else {
-            const __nv_bfloat16 h = __float2bfloat16_rn(x);
-            static_cast<__nv_bfloat16*>(o.hi)[k] = h;
-            static_cast<__nv_bfloat16*>(o.lo)[k] = __float2bfloat16_rn(x - __bfloat162float(h));
+      for (int c = warp; c < r; c += 8) {
+        for (int rr = lane; rr < nrows; rr += 32) {
+          const float v = tile[rr][c];
+          const int row = row0 + rr;
+          if (o.f32 != nullptr && o.transpose_f32) o.f32[static_cast<size_t>(c) * o.rows + row] = v;
+          if (o.hi != nullptr) {
+            const float x = o.scale * v;
+            const size_t k = static_cast<size_t>(c) * o.ld + row;
+            if (o.hilo_f16) {
+              const __half h = __float2half_rn(x);
+              static_cast<__half*>(o.hi)[k] = h;
+              static_cast<__half*>(o.lo)[k] = __float2half_rn(x - __half2float(h));
+            } else {
+              const __nv_bfloat16 h = __float2bfloat16_rn(x);
+              static_cast<__nv_bfloat16*>(o.hi)[k] = h;
+              static_cast<__nv_bfloat16*>(o.lo)[k] = __float2bfloat16_rn(x - __bfloat162float(h));
+            }
           }
         }
       }

@@ -270,8 +270,7 @@ __global__ void __launch_bounds__(kRank2dThreads, 1) rank2d_kernel(const __grid_
             if (!last_j || i + 1 < na) keep(last_j ? i + 1 : i, last_j ? 0 : j + 1, nxt);
             if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
             uint8_t* st = smem + rp.stage * C::kStageBytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) mask_sw128_row(st + h * C::kZBox + lrow * 128, lrow, cur + 2 * h);
+            mask_sw128_rows<2>(st + lrow * 128, C::kZBox, lrow, cur);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&masked[rp.stage]);

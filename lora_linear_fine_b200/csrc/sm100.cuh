@@ -229,26 +229,36 @@ __device__ __forceinline__ void load_keep_bytes(const uint8_t* mrow, int b0, int
   for (int w = 0; w < kBytes / 4; ++w) m[w] = b[4 * w] | (b[4 * w + 1] << 8) | (b[4 * w + 2] << 16) | (b[4 * w + 3] << 24);
 }
 
-// Zero the dropped elements of one 128-byte row of a SWIZZLE_128B bf16 box:
-// 16-byte chunk c (elements 8c .. 8c + 7) sits at position c ^ (row & 7) and
-// takes keep byte c (byte c % 4 of word c / 4 of `m`).
-__device__ __forceinline__ void mask_sw128_row(uint8_t* row_base, int row, const uint32_t* m) {
-  uint4* trow = reinterpret_cast<uint4*>(row_base);
+// Zero the dropped elements of one 128-byte row in each of kBoxes
+// SWIZZLE_128B bf16 boxes (box k at row_base + k * box_stride): 16-byte chunk
+// c (elements 8c .. 8c + 7) of box k sits at position c ^ (row & 7) and takes
+// keep byte 8k + c (byte (8k + c) % 4 of word (8k + c) / 4 of `m`).  All
+// chunks are read before any is written, so the row costs one shared-memory
+// latency.
+template <int kBoxes>
+__device__ __forceinline__ void mask_sw128_rows(uint8_t* row_base, int box_stride, int row, const uint32_t* m) {
+  uint4 v[kBoxes][8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint32_t b = (m[c >> 2] >> (8 * (c & 3))) & 0xFFu;
-    if (b == 0xFFu) continue;
-    uint4& slot = trow[c ^ (row & 7)];
-    const uint4 v = slot;
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+  for (int k = 0; k < kBoxes; ++k)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
-      const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
-      o[e] = w[e] & (lo | hi);
+    for (int c = 0; c < 8; ++c) v[k][c] = reinterpret_cast<const uint4*>(row_base + k * box_stride)[c ^ (row & 7)];
+#pragma unroll
+  for (int k = 0; k < kBoxes; ++k) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = 8 * k + c;
+      const uint32_t b = (m[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+      if (b == 0xFFu) continue;
+      const uint32_t w[4] = {v[k][c].x, v[k][c].y, v[k][c].z, v[k][c].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
+        const uint32_t hi = (b >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
+        o[e] = w[e] & (lo | hi);
+      }
+      reinterpret_cast<uint4*>(row_base + k * box_stride)[c ^ (row & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    slot = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
