@@ -120,7 +120,11 @@ struct MmaCfg {
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
   // shared memory (4 KB per warp) so that global stores are row-contiguous.
   static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
-  static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : 0;
+  // The dropout epilogue keeps each column half's 128 columns of A in a
+  // shared-memory slab (kDropMaxRank rows of 256 bytes per half).
+  static constexpr bool kDropEpi = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
+  static constexpr int kDropSlabBytes = kDropMaxRank * 128 * 2;
+  static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : (kDropEpi ? 2 * kDropSlabBytes : 0);
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kEpiStageBytes + 2048;
@@ -387,18 +391,47 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       const uint32_t use = it >> 1;
       const int row = mt * C::kTileM + 128 * static_cast<int>(crank) + row_in_tile;
       const bool row_ok = row < p.M;
-      // Dropout: this row's keep bytes for the tile's 128 columns do not
-      // depend on the accumulator; their load is issued before the wait for it.
-      constexpr bool kDrop = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
+      // Dropout: the tile's 128 columns of A (this warp's column half) go to
+      // the half's shared-memory slab, and this row's s'U (hi + lo) and keep
+      // bytes to registers, before the wait for the accumulator: none of them
+      // depends on it.  The half's four warps first agree (named barrier
+      // 1 + h) that the previous tile's slab is no longer read.
+      constexpr bool kDrop = C::kDropEpi;
       uint32_t dkeep[4];
+      float du[kDrop ? kDropMaxRank : 1];
+      const uint4* slab = reinterpret_cast<const uint4*>(epi_stage + h * C::kDropSlabBytes);
       if constexpr (kDrop) {
         const DropEpi& D = p.drop;
+        if (h == 0) bar_sync_named<1, 128>();
+        else bar_sync_named<2, 128>();
+        uint4* sl = reinterpret_cast<uint4*>(epi_stage + h * C::kDropSlabBytes);
+        const int th = (ew & 3) * 32 + lane;
+        const int col0 = nt * 256 + h * 128;
+        for (int i = th; i < D.r * 16; i += 128) {     // rank c = i / 16, 8 columns from col0 + 8 (i % 16)
+          const int col = col0 + 8 * (i & 15);
+          sl[i] = col < p.N ? __ldg(reinterpret_cast<const uint4*>(D.A + static_cast<size_t>(i >> 4) * p.N + col))
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int c = 0; c < kDropMaxRank; ++c) {
+          du[c] = 0.0f;
+          if (c < D.r && row_ok) {
+            const size_t at = static_cast<size_t>(c) * D.ld + row;
+            du[c] = __bfloat162float(D.ut_hi[at]) + __bfloat162float(D.ut_lo[at]);
+          }
+        }
         const int ldm = p.N / 8;
         const bool vec = (reinterpret_cast<uintptr_t>(D.mask) % 16) == 0 && ldm % 16 == 0;
-        load_keep_bytes<16>(D.mask + static_cast<size_t>(row_ok ? row : 0) * ldm, (nt * 256 + h * 128) / 8, ldm,
-                            row_ok, vec, dkeep);
+        load_keep_bytes<16>(D.mask + static_cast<size_t>(row_ok ? row : 0) * ldm, col0 / 8, ldm, row_ok, vec, dkeep);
       }
-      if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
+      const bool got = wait_bar<kPair>(&acc_full[buf], use & 1u, ctl);
+      if constexpr (kDrop) {
+        // one decision for the half's four warps, which also orders the
+        // slab's stores before its reads
+        if (!(h == 0 ? bar_sync_and<1, 128>(got) : bar_sync_and<2, 128>(got))) break;
+      } else {
+        if (!got) break;
+      }
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
       const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
@@ -607,11 +640,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         }
       } else if constexpr (kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop) {
         // dX = dZ W (the accumulator) + m * (s' U A), 16 columns at a time:
-        // the tile's columns of A are read as warp-wide broadcasts (every lane
-        // of a warp reads the same 16 bytes) and this thread's row of s'U
-        // (hi + lo, fp32) with them, eight ranks per batch of loads so that a
-        // batch costs one memory latency; keep bytes in registers (loaded
-        // above); one bf16 rounding at the end.
+        // the columns of A come from the half's slab (every lane of a warp
+        // reads the same 32 bytes per rank), s'U and the keep bits from
+        // registers (all loaded above), so the loop makes no global load; one
+        // bf16 rounding at the end.
         const int col0 = nt * 256 + h * 128;
         const DropEpi& D = p.drop;
 #pragma unroll 1
@@ -627,28 +659,23 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 #pragma unroll
           for (int j = 0; j < 16; ++j) t[j] = 0.0f;
           const bool two = cb + 8 < p.N;
-          for (int g = 0; g < D.r; g += 8) {
+#pragma unroll
+          for (int g = 0; g < kDropMaxRank; g += 8) {     // eight ranks per batch of shared-memory loads
+            if (g >= D.r) break;
             uint4 a0[8], a1[8];
-            float u[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              // ranks past r contribute exact zeros (u = 0, A = 0; no load)
-              const bool in = g + k < D.r;
-              const int c = in ? g + k : 0;
-              const uint4* ap = reinterpret_cast<const uint4*>(D.A + static_cast<size_t>(c) * p.N + cb);
-              a0[k] = in ? __ldg(ap) : make_uint4(0u, 0u, 0u, 0u);
-              a1[k] = in && two ? __ldg(ap + 1) : make_uint4(0u, 0u, 0u, 0u);
-              const size_t at = static_cast<size_t>(c) * D.ld + row;
-              const float uh = __bfloat162float(D.ut_hi[at]), ul = __bfloat162float(D.ut_lo[at]);
-              u[k] = in ? uh + ul : 0.0f;
+              const bool in = g + k < D.r;                 // slab rows past r are not written: read as 0
+              a0[k] = in ? slab[(g + k) * 16 + 2 * c16] : make_uint4(0u, 0u, 0u, 0u);
+              a1[k] = in ? slab[(g + k) * 16 + 2 * c16 + 1] : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const uint32_t w[8] = {a0[k].x, a0[k].y, a0[k].z, a0[k].w, a1[k].x, a1[k].y, a1[k].z, a1[k].w};
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                t[2 * e] = fmaf(u[k], __uint_as_float(w[e] << 16), t[2 * e]);
-                t[2 * e + 1] = fmaf(u[k], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
+                t[2 * e] = fmaf(du[g + k], __uint_as_float(w[e] << 16), t[2 * e]);
+                t[2 * e + 1] = fmaf(du[g + k], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
               }
             }
           }

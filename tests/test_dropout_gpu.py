@@ -19,6 +19,10 @@ pytestmark = pytest.mark.gpu
     (16, 512, 264, 16, "identity", 0.1),      # few tokens: dropout keeps the tiled path
     (256, 512, 520, 128, "identity", 0.3),    # rank 128
     (300, 640, 264, 72, "silu", 0.5),
+    # every CTA pair runs several dX tiles, so the epilogue's shared-memory
+    # copy of A's columns is refilled between tiles (256 and 128 pair tiles)
+    (4096, 4096, 1024, 64, "identity", 0.1),
+    (2048, 4096, 512, 8, "silu", 0.1),
 ])
 def test_dropout_fwd_bwd(M, d_in, d_out, r, act, p_drop):
     import lora_linear_fine_b200 as L
