@@ -1248,6 +1248,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
   }
 
   // 4. dX = [dZ | sU] [W ; A]
+  const bool drop_in_gemm = masks[0] != nullptr && np == 1 && r > 0 && dXf == nullptr;
   {
     MmaParams p;
     std::memset(&p, 0, sizeof(p));
@@ -1272,19 +1273,13 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     p.M = M;
     p.N = static_cast<int>(d->d_in);
     p.K = static_cast<int>(d->d_out);
-    p.lora_ksteps = masks[0] != nullptr ? 0 : (r + 15) / 16;   // dropout: the masked LoRA term is separate
-    // dropout, one projection, r <= 64: the masked LoRA term m * (s' U A) is
-    // added in the dX GEMM's epilogue; otherwise dx_dropout_kernel adds it
-    // after the GEMM
-    const bool drop_epi = masks[0] != nullptr && np == 1 && r > 0 && r <= kDropMaxRank && dXf == nullptr;
-    if (drop_epi) {
-      p.drop.mask = masks[0];
-      p.drop.ut_hi = static_cast<const __nv_bfloat16*>(at(P.ut_hi[0]));
-      p.drop.ut_lo = static_cast<const __nv_bfloat16*>(at(P.ut_lo[0]));
-      p.drop.A = static_cast<const __nv_bfloat16*>(Ap[0]);
-      p.drop.r = r;
-      p.drop.ld = M8;
-    }
+    // Dropout with one projection: the LoRA K-blocks form s'U A in the
+    // accumulator first, its dropped entries are zeroed in tensor memory, and
+    // the main K-blocks accumulate on top (kMEpiGradDrop).  SwiGLU (two masks
+    // on one accumulator) runs without the LoRA K-blocks and
+    // dx_dropout_kernel adds the masked terms after the GEMM.
+    p.lora_ksteps = (masks[0] != nullptr && !drop_in_gemm) ? 0 : (r + 15) / 16;
+    if (drop_in_gemm) p.drop.mask = masks[0];
     p.out = static_cast<__nv_bfloat16*>(dX);
     p.out_f32 = dXf;
     p.out_acc = dXf_acc;
@@ -1296,7 +1291,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     set_raster(p, pair, 2.0 * np * M * d->d_out, 2.0 * np * d->d_out * d->d_in);
     timing_begin(1, st);
     lora_status_t rs;
-    if (drop_epi) {
+    if (drop_in_gemm) {
       rs = f16 ? launch_mma_any<true, 1, kMEpiGradF16Drop>(pair, p, dev.sms, st)
                : launch_mma_any<true, 1, kMEpiGradDrop>(pair, p, dev.sms, st);
     } else if (dXf != nullptr) {
@@ -1315,7 +1310,7 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     LORA_TRY(rs);
   }
   if (r == 0) return LORA_OK;
-  if (masks[0] != nullptr && !(np == 1 && r <= kDropMaxRank && dXf == nullptr)) {
+  if (masks[0] != nullptr && !drop_in_gemm) {
     // dX += sum_j mask_j * (s' U_j A_j), from the (s' U_j)^T hi/lo of the U pass
     DxDropoutJob jb[2];
     for (int j = 0; j < 2; ++j) {

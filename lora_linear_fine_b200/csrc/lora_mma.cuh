@@ -64,13 +64,10 @@ enum MmaEpi : int {
 };
 
 // Dropout on the adapter input, dX epilogue (kMEpiGradDrop / kMEpiGradF16Drop).
-constexpr int kDropMaxRank = 64;
+// Dropout keep bits of the dX GEMM's outputs (the elements of X): [M x N/8]
+// bytes, bit j of byte b (least significant first) keeping column 8 b + j.
 struct DropEpi {
-  const uint8_t* mask;            // [M x N/8] bits, least significant first
-  const __nv_bfloat16* ut_hi;     // (s' U)^T hi [r x ld]
-  const __nv_bfloat16* ut_lo;     // (s' U)^T lo [r x ld]
-  const __nv_bfloat16* A;         // [r x N]
-  int r, ld;                      // r <= kDropMaxRank
+  const uint8_t* mask;
 };
 
 // Output projection fused with the cross-entropy loss (rows = tokens of this
@@ -120,11 +117,10 @@ struct MmaCfg {
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
   // shared memory (4 KB per warp) so that global stores are row-contiguous.
   static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
-  // The dropout epilogue keeps each column half's 128 columns of A in a
-  // shared-memory slab (kDropMaxRank rows of 256 bytes per half).
+  // Dropout on the adapter input (backward, one projection): the masked
+  // LoRA term is formed in the accumulator before the main K-loop.
   static constexpr bool kDropEpi = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
-  static constexpr int kDropSlabBytes = kDropMaxRank * 128 * 2;
-  static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : (kDropEpi ? 2 * kDropSlabBytes : 0);
+  static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : 0;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kEpiStageBytes + 2048;
@@ -176,7 +172,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   uint64_t* acc_full = bars + 2 * S;      // [2] accumulator buffer b complete
   uint64_t* acc_empty = acc_full + 2;     // [2] accumulator buffer b drained
   uint64_t* mma_done = acc_full + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
+  uint64_t* lora_done = acc_full + 5;     // [2] dropout: the LoRA term of buffer b is in the accumulator
+  uint64_t* masked = acc_full + 7;        // [2] dropout: its dropped entries are zeroed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 9);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -191,6 +189,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     // acc_empty: one arrival per epilogue warp of every CTA of the unit
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 8 * C::kCtas); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&lora_done[b], 1); mbar_init(&masked[b], 8 * C::kCtas); }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -234,68 +233,89 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       // area and 128 rows of N-side operand (64 per CTA of a pair).
       constexpr uint32_t kTxFull = C::kCtas * C::kStageBytes;
       constexpr uint32_t kTxSwigluLora = C::kCtas * C::kABytes + 128 * 64 * 2;
-      for (int t = unit; t < p.num_tiles && ok; t += nunits) {
+      // Block blk of tile t (main K-blocks first, then the LoRA blocks) into
+      // the next ring stage; false if the wait for the stage gave up.
+      auto put = [&](int t, int blk) -> bool {
         int mt, nt;
         mma_tile_coords(t, p, mt, nt);
         const int m0 = mt * C::kTileM + 128 * static_cast<int>(crank);
         const int n0 = nt * C::kOutCols;
-        const int nblocks = C::kKPairs * nkb + nlora;
-        for (int blk = 0; blk < nblocks; ++blk) {
-          if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) { ok = false; break; }
-          uint8_t* sa = smem + rp.stage * C::kStageBytes;
-          uint8_t* sb = sa + C::kABytes;
-          const uint32_t fb = rp.stage;
-          const bool lora_blk = blk >= C::kKPairs * nkb;
-          if (leader)
-            mbar_arrive_expect_tx(&full[rp.stage], (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull);
-          if (!lora_blk) {
-            // main block: projection j, K-block kb
-            const int j = blk / nkb;
-            const int k0 = (blk - j * nkb) * 64;
-            load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
-            if constexpr (!kBwd) {
-              if constexpr (C::kSwigluFwd) {
-                if constexpr (kPair) load(sb, &p.tm_w[crank], fb, k0, n0, pol_keep);
-                else {
-                  load(sb, &p.tm_w[0], fb, k0, n0, pol_keep);
-                  load(sb + C::kBBytes / 2, &p.tm_w[1], fb, k0, n0, pol_keep);
-                }
-              } else {
-                load(sb, &p.tm_w[0], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+        if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) return false;
+        uint8_t* sa = smem + rp.stage * C::kStageBytes;
+        uint8_t* sb = sa + C::kABytes;
+        const uint32_t fb = rp.stage;
+        const bool lora_blk = blk >= C::kKPairs * nkb;
+        if (leader)
+          mbar_arrive_expect_tx(&full[rp.stage], (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull);
+        if (!lora_blk) {
+          // main block: projection j, K-block kb
+          const int j = blk / nkb;
+          const int k0 = (blk - j * nkb) * 64;
+          load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
+          if constexpr (!kBwd) {
+            if constexpr (C::kSwigluFwd) {
+              if constexpr (kPair) load(sb, &p.tm_w[crank], fb, k0, n0, pol_keep);
+              else {
+                load(sb, &p.tm_w[0], fb, k0, n0, pol_keep);
+                load(sb + C::kBBytes / 2, &p.tm_w[1], fb, k0, n0, pol_keep);
               }
-            } else if (p.b_mn) {
-#pragma unroll
-              for (int b = 0; b < C::kBRows / 64; ++b)
-                load(sb + b * 8192, &p.tm_w[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, k0, pol_keep);
             } else {
-              // W^T (K-major copy of W made by the backward): rows = outputs of dX
-              load(sb, &p.tm_w[j], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+              load(sb, &p.tm_w[0], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
             }
+          } else if (p.b_mn) {
+#pragma unroll
+            for (int b = 0; b < C::kBRows / 64; ++b)
+              load(sb + b * 8192, &p.tm_w[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, k0, pol_keep);
           } else {
-            // LoRA block of projection j: s*T_j (s*U_j) rows and B_j (A_j) rows,
-            // K = r columns [kx, kx + 64) of the rank, zero-filled past r
-            const int lb = blk - C::kKPairs * nkb;
-            const int j = lb / lkb;
-            const int kx = (lb - j * lkb) * 64;
-            load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
-            if constexpr (!kBwd) {
-              if constexpr (C::kSwigluFwd) {
-                // N = 128 outputs of projection j: 128 rows (single) or 64 per CTA (pair)
-                load(sb, &p.tm_lb[j], fb, kx, n0 + 64 * static_cast<int>(crank), pol_keep);
-              } else {
-                load(sb, &p.tm_lb[0], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
-              }
-            } else if (p.b_mn) {
-#pragma unroll
-              for (int b = 0; b < C::kBRows / 64; ++b)
-                load(sb + b * 8192, &p.tm_lb[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, kx, pol_keep);
-            } else {
-              load(sb, &p.tm_lb[j], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);   // A^T rows
-            }
+            // W^T (K-major copy of W made by the backward): rows = outputs of dX
+            load(sb, &p.tm_w[j], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
           }
-          ++issued;
-          rp.next(S);
+        } else {
+          // LoRA block of projection j: s*T_j (s*U_j) rows and B_j (A_j) rows,
+          // K = r columns [kx, kx + 64) of the rank, zero-filled past r
+          const int lb = blk - C::kKPairs * nkb;
+          const int j = lb / lkb;
+          const int kx = (lb - j * lkb) * 64;
+          load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
+          if constexpr (!kBwd) {
+            if constexpr (C::kSwigluFwd) {
+              // N = 128 outputs of projection j: 128 rows (single) or 64 per CTA (pair)
+              load(sb, &p.tm_lb[j], fb, kx, n0 + 64 * static_cast<int>(crank), pol_keep);
+            } else {
+              load(sb, &p.tm_lb[0], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+            }
+          } else if (p.b_mn) {
+#pragma unroll
+            for (int b = 0; b < C::kBRows / 64; ++b)
+              load(sb + b * 8192, &p.tm_lb[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, kx, pol_keep);
+          } else {
+            load(sb, &p.tm_lb[j], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);   // A^T rows
+          }
         }
+        ++issued;
+        rp.next(S);
+        return true;
+      };
+      const int nmain = C::kKPairs * nkb;
+      if constexpr (C::kDropEpi) {
+        // Dropout: the tensor core first writes the LoRA term of a tile into
+        // its accumulator, the epilogue warps zero its dropped entries, then
+        // the main K-blocks accumulate on top.  The next tile's LoRA blocks
+        // ride in the middle of this tile's main blocks, so that the masking
+        // of the other accumulator buffer overlaps this tile's K-loop:
+        //   L(t0), main(t0)[0, h), L(t1), main(t0)[h, n), main(t1)[0, h), L(t2), ...
+        const int h = nmain / 2;
+        for (int t = unit; t < p.num_tiles && ok; t += nunits) {
+          if (t == unit)
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(t, nmain + lb);
+          for (int blk = 0; blk < h && ok; ++blk) ok = put(t, blk);
+          if (t + nunits < p.num_tiles)
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(t + nunits, nmain + lb);
+          for (int blk = h; blk < nmain && ok; ++blk) ok = put(t, blk);
+        }
+      } else {
+        for (int t = unit; t < p.num_tiles && ok; t += nunits)
+          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(t, blk);
       }
       if (!ok && leader) {
         RingPos q = rp;
@@ -328,43 +348,79 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         else mma_commit(bar);
       };
       RingPos rp;
-      uint32_t it = 0;
-      for (int t = unit; t < p.num_tiles; t += nunits, ++it) {
-        const uint32_t buf = it & 1u;
-        const uint32_t use = it >> 1;        // how many times this buffer was used before
-        if (!wait_bar<kPair>(&acc_empty[buf], (use & 1u) ^ 1u, ctl)) break;
+      const int nmain = C::kKPairs * nkb;
+      // Block blk of a tile (main K-blocks first, then the LoRA blocks) from
+      // the next ring stage into the accumulator at dacc.  The first MMA of a
+      // tile starts the accumulator: main block 0 normally, LoRA block 0 with
+      // dropout (where the main blocks then accumulate on the masked term).
+      auto take = [&](int blk, uint32_t dacc) -> bool {
+        if (!wait_bar<kPair>(&full[rp.stage], rp.phase, ctl)) return false;
         tc_fence_after();
-        const uint32_t dacc = tbase + buf * 256;
-        const int nblocks = C::kKPairs * nkb + nlora;
-        bool ok = true;
-        for (int blk = 0; blk < nblocks; ++blk) {
-          if (!wait_bar<kPair>(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + rp.stage * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
-          if (blk < C::kKPairs * nkb) {
+        const uint32_t sa = smem_u32(smem + rp.stage * C::kStageBytes);
+        const uint32_t sb = sa + C::kABytes;
+        if (blk < nmain) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
-              mma(dacc, da, db, kIdMain, (blk == 0 && kk == 0) ? 0u : 1u);
-            }
-          } else {
-            const int lb = blk - C::kKPairs * nkb;
-            const int j = lb / lkb;
-            const int steps = p.lora_ksteps - 4 * (lb - j * lkb);     // this block's 16-wide steps
-            const uint32_t dcol = C::kSwigluFwd ? static_cast<uint32_t>(128 * j) : 0u;
-            for (int kk = 0; kk < (steps < 4 ? steps : 4); ++kk) {
-              const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
-              mma(dacc + dcol, da, db, kIdLora, 1u);
-            }
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
+            mma(dacc, da, db, kIdMain, (!C::kDropEpi && blk == 0 && kk == 0) ? 0u : 1u);
           }
-          commit(&empty[rp.stage]);
-          rp.next(S);
+        } else {
+          const int lb = blk - nmain;
+          const int j = lb / lkb;
+          const int steps = p.lora_ksteps - 4 * (lb - j * lkb);     // this block's 16-wide steps
+          const uint32_t dcol = C::kSwigluFwd ? static_cast<uint32_t>(128 * j) : 0u;
+          for (int kk = 0; kk < (steps < 4 ? steps : 4); ++kk) {
+            const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
+            mma(dacc + dcol, da, db, kIdLora, (C::kDropEpi && lb == 0 && kk == 0) ? 0u : 1u);
+          }
         }
-        if (!ok) break;
-        commit(&acc_full[buf]);
+        commit(&empty[rp.stage]);
+        rp.next(S);
+        return true;
+      };
+      uint32_t it = 0;
+      if constexpr (C::kDropEpi) {
+        // Ring order (the producer's): L(t0), main(t0)[0, h), L(t1),
+        // main(t0)[h, n), main(t1)[0, h), L(t2), ...  L(t) goes into t's
+        // buffer once the epilogue has drained it; the main blocks of t wait
+        // until the epilogue warps have zeroed the dropped entries of L(t).
+        const int h = nmain / 2;
+        auto lora_into = [&](uint32_t i) -> bool {      // L of the unit's i-th tile
+          const uint32_t b = i & 1u, u = i >> 1;
+          if (!wait_bar<kPair>(&acc_empty[b], (u & 1u) ^ 1u, ctl)) return false;
+          tc_fence_after();
+          for (int lb = 0; lb < nlora; ++lb)
+            if (!take(nmain + lb, tbase + b * 256)) return false;
+          commit(&lora_done[b]);
+          return true;
+        };
+        bool ok = true;
+        for (int t = unit; t < p.num_tiles && ok; t += nunits, ++it) {
+          const uint32_t buf = it & 1u;
+          const uint32_t use = it >> 1;
+          const uint32_t dacc = tbase + buf * 256;
+          if (t == unit) ok = lora_into(it);
+          if (ok) ok = wait_bar<kPair>(&masked[buf], use & 1u, ctl);
+          tc_fence_after();
+          for (int blk = 0; blk < h && ok; ++blk) ok = take(blk, dacc);
+          if (ok && t + nunits < p.num_tiles) ok = lora_into(it + 1);
+          for (int blk = h; blk < nmain && ok; ++blk) ok = take(blk, dacc);
+          if (ok) commit(&acc_full[buf]);
+        }
+      } else {
+        for (int t = unit; t < p.num_tiles; t += nunits, ++it) {
+          const uint32_t buf = it & 1u;
+          const uint32_t use = it >> 1;        // how many times this buffer was used before
+          if (!wait_bar<kPair>(&acc_empty[buf], (use & 1u) ^ 1u, ctl)) break;
+          tc_fence_after();
+          const uint32_t dacc = tbase + buf * 256;
+          bool ok = true;
+          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = take(blk, dacc);
+          if (!ok) break;
+          commit(&acc_full[buf]);
+        }
       }
       if constexpr (kPair) mma_commit_pair(mma_done, 0x1);
       else mma_commit(mma_done);
@@ -383,6 +439,43 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 #pragma unroll
     for (int b = 0; b < 2; ++b)
       acc_empty_addr[b] = kPair ? mapa_shared(smem_u32(&acc_empty[b]), 0) : smem_u32(&acc_empty[b]);
+    // Dropout: in the accumulator buffer of the unit's i-th tile (tile tt),
+    // keep the LoRA term m * (s'U A) where this thread's row keeps the
+    // element and zero it elsewhere; 16 columns per TMEM load / store.
+    auto mask_pass = [&](int tt, uint32_t i) -> bool {
+      const uint32_t b = i & 1u, u = i >> 1;
+      int mt2, nt2;
+      mma_tile_coords(tt, p, mt2, nt2);
+      const int row2 = mt2 * C::kTileM + 128 * static_cast<int>(crank) + row_in_tile;
+      const bool ok_row = row2 < p.M;
+      const int ldm = p.N / 8;
+      const bool vec = (reinterpret_cast<uintptr_t>(p.drop.mask) % 16) == 0 && ldm % 16 == 0;
+      uint32_t keep[4];
+      load_keep_bytes<16>(p.drop.mask + static_cast<size_t>(ok_row ? row2 : 0) * ldm, (nt2 * 256 + h * 128) / 8, ldm,
+                          ok_row, vec, keep);
+      if (!wait_bar<kPair>(&lora_done[b], u & 1u, ctl)) return false;
+      tc_fence_after();
+      __syncwarp();
+      const uint32_t tl2 = tbase + b * 256 + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
+#pragma unroll 1
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint32_t v[16];
+        tmem_ld16(tl2 + 16 * c16, v);
+        tmem_wait_ld();
+        const uint32_t mb = (keep[c16 >> 1] >> (16 * (c16 & 1))) & 0xFFFFu;   // keep bytes 2 c16, 2 c16 + 1
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = ((mb >> j) & 1u) ? v[j] : 0u;
+        tmem_st16(tl2 + 16 * c16, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&masked[b]), 0));
+        else mbar_arrive(&masked[b]);
+      }
+      return true;
+    };
     uint32_t it = 0;
     for (int t = unit; t < p.num_tiles; t += nunits, ++it) {
       int mt, nt;
@@ -391,47 +484,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       const uint32_t use = it >> 1;
       const int row = mt * C::kTileM + 128 * static_cast<int>(crank) + row_in_tile;
       const bool row_ok = row < p.M;
-      // Dropout: the tile's 128 columns of A (this warp's column half) go to
-      // the half's shared-memory slab, and this row's s'U (hi + lo) and keep
-      // bytes to registers, before the wait for the accumulator: none of them
-      // depends on it.  The half's four warps first agree (named barrier
-      // 1 + h) that the previous tile's slab is no longer read.
-      constexpr bool kDrop = C::kDropEpi;
-      uint32_t dkeep[4];
-      float du[kDrop ? kDropMaxRank : 1];
-      const uint4* slab = reinterpret_cast<const uint4*>(epi_stage + h * C::kDropSlabBytes);
-      if constexpr (kDrop) {
-        const DropEpi& D = p.drop;
-        if (h == 0) bar_sync_named<1, 128>();
-        else bar_sync_named<2, 128>();
-        uint4* sl = reinterpret_cast<uint4*>(epi_stage + h * C::kDropSlabBytes);
-        const int th = (ew & 3) * 32 + lane;
-        const int col0 = nt * 256 + h * 128;
-        for (int i = th; i < D.r * 16; i += 128) {     // rank c = i / 16, 8 columns from col0 + 8 (i % 16)
-          const int col = col0 + 8 * (i & 15);
-          sl[i] = col < p.N ? __ldg(reinterpret_cast<const uint4*>(D.A + static_cast<size_t>(i >> 4) * p.N + col))
-                            : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int c = 0; c < kDropMaxRank; ++c) {
-          du[c] = 0.0f;
-          if (c < D.r && row_ok) {
-            const size_t at = static_cast<size_t>(c) * D.ld + row;
-            du[c] = __bfloat162float(D.ut_hi[at]) + __bfloat162float(D.ut_lo[at]);
-          }
-        }
-        const int ldm = p.N / 8;
-        const bool vec = (reinterpret_cast<uintptr_t>(D.mask) % 16) == 0 && ldm % 16 == 0;
-        load_keep_bytes<16>(D.mask + static_cast<size_t>(row_ok ? row : 0) * ldm, col0 / 8, ldm, row_ok, vec, dkeep);
+      if constexpr (C::kDropEpi) {
+        // Zero the dropped entries of the LoRA term before the main blocks
+        // accumulate on it: the unit's first tile's term before anything
+        // else, the next tile's (in the other buffer) before this tile's
+        // epilogue, which the MMA warp needs next.
+        bool okm = true;
+        if (t == unit) okm = mask_pass(t, it);
+        if (okm && t + nunits < p.num_tiles) okm = mask_pass(t + nunits, it + 1);
+        if (!okm) break;
       }
-      const bool got = wait_bar<kPair>(&acc_full[buf], use & 1u, ctl);
-      if constexpr (kDrop) {
-        // one decision for the half's four warps, which also orders the
-        // slab's stores before its reads
-        if (!(h == 0 ? bar_sync_and<1, 128>(got) : bar_sync_and<2, 128>(got))) break;
-      } else {
-        if (!got) break;
-      }
+      if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
       tc_fence_after();
       __syncwarp();   // tcgen05.ld is .sync.aligned
       const uint32_t tl = tbase + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
@@ -636,62 +699,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
                                            __float_as_uint(o.w)),
                                 pol_out);
             }
-          }
-        }
-      } else if constexpr (kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop) {
-        // dX = dZ W (the accumulator) + m * (s' U A), 16 columns at a time:
-        // the columns of A come from the half's slab (every lane of a warp
-        // reads the same 32 bytes per rank), s'U and the keep bits from
-        // registers (all loaded above), so the loop makes no global load; one
-        // bf16 rounding at the end.
-        const int col0 = nt * 256 + h * 128;
-        const DropEpi& D = p.drop;
-#pragma unroll 1
-        for (int c16 = 0; c16 < 8; ++c16) {
-          uint32_t v[16];
-          __syncwarp();
-          tmem_ld16(tl + h * 128 + 16 * c16, v);
-          tmem_wait_ld();
-          if (c16 == 7) release_acc();
-          const int cb = col0 + 16 * c16;
-          if (!row_ok || cb >= p.N) continue;
-          float t[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) t[j] = 0.0f;
-          const bool two = cb + 8 < p.N;
-#pragma unroll
-          for (int g = 0; g < kDropMaxRank; g += 8) {     // eight ranks per batch of shared-memory loads
-            if (g >= D.r) break;
-            uint4 a0[8], a1[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const bool in = g + k < D.r;                 // slab rows past r are not written: read as 0
-              a0[k] = in ? slab[(g + k) * 16 + 2 * c16] : make_uint4(0u, 0u, 0u, 0u);
-              a1[k] = in ? slab[(g + k) * 16 + 2 * c16 + 1] : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t w[8] = {a0[k].x, a0[k].y, a0[k].z, a0[k].w, a1[k].x, a1[k].y, a1[k].z, a1[k].w};
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                t[2 * e] = fmaf(du[g + k], __uint_as_float(w[e] << 16), t[2 * e]);
-                t[2 * e + 1] = fmaf(du[g + k], __uint_as_float(w[e] & 0xFFFF0000u), t[2 * e + 1]);
-              }
-            }
-          }
-          const uint32_t mb = (dkeep[c16 >> 1] >> (16 * (c16 & 1))) & 0xFFFFu;   // keep bytes 2 c16, 2 c16 + 1
-          float z[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) z[j] = __uint_as_float(v[j]) + (((mb >> j) & 1u) ? t[j] : 0.0f);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            if (q == 1 && !two) break;
-            uint4 pk;
-            pk.x = pack_bf16x2(z[8 * q], z[8 * q + 1]);
-            pk.y = pack_bf16x2(z[8 * q + 2], z[8 * q + 3]);
-            pk.z = pack_bf16x2(z[8 * q + 4], z[8 * q + 5]);
-            pk.w = pack_bf16x2(z[8 * q + 6], z[8 * q + 7]);
-            st_global_v4_hint(p.out + static_cast<size_t>(row) * p.N + cb + 8 * q, pk, pol_out);
           }
         }
       } else if constexpr (kEpi == kMEpiCeFwd) {
