@@ -616,6 +616,17 @@ bool pair_kernel_enabled() {
   return v == 1;
 }
 
+// LORA_LINEAR_FUSED_T=0 turns off the forward GEMM's fused T (one tile per
+// unit), so that the separate T pass runs instead (for comparisons).
+bool fused_t_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("LORA_LINEAR_FUSED_T");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
 lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
   using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
@@ -1007,7 +1018,6 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const int np = P.np, RP = P.RP;
-  (void)RP;
   const int64_t M = d->M, r = d->r;
 
   if (P.small_m) return run_small_m_fwd(d, P.sm_nt, X, W, nullptr, nullptr, A, B, Y, T_save, Z_save, status, st);
@@ -1015,8 +1025,16 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   const void* Wp[2] = {W, W_up};
   const void* Ap[2] = {A, A_up};
   const void* Bp[2] = {B, B_up};
+  const bool pair = pair_kernel_enabled() && M > 128;
+  // One GEMM tile per unit (a single wave, e.g. about a thousand tokens): the
+  // GEMM's second accumulator buffer is free, so T accumulates there during
+  // the main K-loop and the separate T pass (and its split-K reduction) is
+  // skipped.  One identity projection, r <= 64, no dropout, no rotation.
+  const int64_t tiles1 = ceil_div(M, pair ? 256 : 128) * ceil_div(d->d_out, 256);
+  const bool fuse_t = fused_t_enabled() && r > 0 && RP <= 64 && np == 1 && d->act == LORA_ACT_IDENTITY &&
+                      rope == nullptr && fmasks == nullptr && tiles1 <= (pair ? dev.sms / 2 : dev.sms);
   // 1. T_j = X A_j^T (fp32, saved for the backward) and bf16(s T_j) for the LoRA K-block
-  if (r > 0) {
+  if (r > 0 && !fuse_t) {
     for (int j = 0; j < np; ++j) {
       RankOut o = rank_out(static_cast<int>(M), static_cast<int>(r));
       o.f32 = T_save ? T_save + static_cast<size_t>(j) * M * r
@@ -1029,7 +1047,6 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   // 2. Z = [X | sT] [W | B]^T, activation, bf16 Y
   MmaParams p;
   std::memset(&p, 0, sizeof(p));
-  const bool pair = pair_kernel_enabled() && M > 128;
   const int outc = swiglu ? 128 : 256;
   const int brows = swiglu ? (pair ? 64 : 128) : (pair ? 128 : 256);   // N-side rows per CTA box
   bool ok = make_tm(&p.tm_a[0], X, d->d_in, M, d->d_in, 64, 128);
@@ -1057,6 +1074,17 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   if (rope != nullptr) {
     p.rope = *rope;
     rs = launch_mma_any<false, 1, kMEpiRope>(pair, p, dev.sms, st);
+    timing_end(0, st);
+    return rs;
+  }
+  if (fuse_t) {
+    p.am_rows = RP / (pair ? 2 : 1);
+    p.rp = RP;
+    p.r = static_cast<int>(r);
+    p.lora_scale = d->s;
+    p.t_save = T_save;
+    if (!make_tm(&p.tm_am, A, d->d_in, r, d->d_in, 64, p.am_rows)) return LORA_ERR_CUDA;
+    rs = launch_mma_any<false, 1, kMEpiIdentityT>(pair, p, dev.sms, st);
     timing_end(0, st);
     return rs;
   }

@@ -60,7 +60,7 @@ constexpr int kMmaThreads = 320;
 enum MmaEpi : int {
   kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5,
   kMEpiCeFwd = 6, kMEpiCeGrad = 7, kMEpiGradF32 = 8, kMEpiGradF16F32 = 9, kMEpiGradDrop = 10,
-  kMEpiGradF16Drop = 11
+  kMEpiGradF16Drop = 11, kMEpiIdentityT = 12
 };
 
 // Dropout on the adapter input, dX epilogue (kMEpiGradDrop / kMEpiGradF16Drop).
@@ -100,6 +100,14 @@ struct MmaParams {
   int out_acc;            // with out_f32: dX += the product (else dX = the product)
   CeParams ce;            // kMEpiCeFwd / kMEpiCeGrad
   DropEpi drop;           // kMEpiGradDrop / kMEpiGradF16Drop
+  // kMEpiIdentityT (forward, one tile per unit): T = X A^T accumulates in the
+  // second accumulator buffer during the main K-loop
+  CUtensorMap tm_am;      // A [r x K], box 64 x am_rows (this CTA's am_rows rows of the padded rank)
+  int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
+  int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
+  int r;                  // the rank
+  float lora_scale;       // s: the LoRA block's operand is bf16(s T)
+  float* t_save;          // fp32 T [M x r] for the backward (written by the N-tile-0 units), or null
 };
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
@@ -113,7 +121,10 @@ struct MmaCfg {
   static constexpr int kABytes = 128 * 64 * 2;               // 16 KB
   static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
   static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  // kMEpiIdentityT: rows of A (the rank, up to 64 in all) per stage and CTA
+  static constexpr bool kTFused = kEpi == kMEpiIdentityT;
+  static constexpr int kAMBytes = kTFused ? (64 / kCtas) * 64 * 2 : 0;
+  static constexpr int kStageBytes = kABytes + kBBytes + kAMBytes;
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
   // shared memory (4 KB per warp) so that global stores are row-contiguous.
   static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
@@ -174,7 +185,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   uint64_t* mma_done = acc_full + 4;
   uint64_t* lora_done = acc_full + 5;     // [2] dropout: the LoRA term of buffer b is in the accumulator
   uint64_t* masked = acc_full + 7;        // [2] dropout: its dropped entries are zeroed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 9);
+  uint64_t* t_done = acc_full + 9;        // fused T: the main K-loop (and T) is complete
+  uint64_t* t_ready = acc_full + 10;      // fused T: bf16(s T) is in the LoRA stage's A area
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 11);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -184,12 +197,22 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   const int unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;        // scheduling unit (CTA or pair)
   const int nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
   AbortCtl ctl{abort_flag, p.status};
+  if constexpr (C::kTFused) {
+    // The fused T needs one tile per unit (the host's choice); anything else
+    // is refused before any barrier, tensor memory or cluster step.
+    if (p.num_tiles > nunits || p.rp < 16 || p.rp > 64 || p.rp % 16 != 0 || p.am_rows * C::kCtas != p.rp) {
+      if (threadIdx.x == 0 && p.status != nullptr) atomicOr(p.status, kStatusBadArgument);
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     // acc_empty: one arrival per epilogue warp of every CTA of the unit
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 8 * C::kCtas); }
     for (int b = 0; b < 2; ++b) { mbar_init(&lora_done[b], 1); mbar_init(&masked[b], 8 * C::kCtas); }
+    mbar_init(t_done, 1);
+    mbar_init(t_ready, 4 * C::kCtas);
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -245,13 +268,20 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         uint8_t* sb = sa + C::kABytes;
         const uint32_t fb = rp.stage;
         const bool lora_blk = blk >= C::kKPairs * nkb;
-        if (leader)
-          mbar_arrive_expect_tx(&full[rp.stage], (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull);
+        if (leader) {
+          uint32_t tx = (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull;
+          if constexpr (C::kTFused)   // main: X, W and am_rows rows of A; LoRA: B only (the epilogue writes s T)
+            tx = lora_blk ? C::kCtas * C::kBBytes
+                          : C::kCtas * (C::kABytes + C::kBBytes + static_cast<uint32_t>(p.am_rows) * 128u);
+          mbar_arrive_expect_tx(&full[rp.stage], tx);
+        }
         if (!lora_blk) {
           // main block: projection j, K-block kb
           const int j = blk / nkb;
           const int k0 = (blk - j * nkb) * 64;
           load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
+          if constexpr (C::kTFused)
+            load(sb + C::kBBytes, &p.tm_am, fb, k0, p.am_rows * static_cast<int>(crank), pol_keep);
           if constexpr (!kBwd) {
             if constexpr (C::kSwigluFwd) {
               if constexpr (kPair) load(sb, &p.tm_w[crank], fb, k0, n0, pol_keep);
@@ -276,7 +306,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           const int lb = blk - C::kKPairs * nkb;
           const int j = lb / lkb;
           const int kx = (lb - j * lkb) * 64;
-          load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
+          if (!C::kTFused) load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
           if constexpr (!kBwd) {
             if constexpr (C::kSwigluFwd) {
               // N = 128 outputs of projection j: 128 rows (single) or 64 per CTA (pair)
@@ -347,6 +377,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         if constexpr (kPair) mma_commit_pair(bar, kBoth);
         else mma_commit(bar);
       };
+      const uint32_t kIdT = idesc_mma(kM, C::kTFused ? p.rp : 16, false, false, false);
       RingPos rp;
       const int nmain = C::kKPairs * nkb;
       // Block blk of a tile (main K-blocks first, then the LoRA blocks) from
@@ -364,6 +395,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
             const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
             mma(dacc, da, db, kIdMain, (!C::kDropEpi && blk == 0 && kk == 0) ? 0u : 1u);
+            if constexpr (C::kTFused) {   // T += X tile x (rows of A)^T, into the second buffer's columns
+              const uint64_t dam = sdesc_sw128(sb + C::kBBytes + kk * 32, 16, 1024);
+              mma(tbase + 256, da, dam, kIdT, (blk == 0 && kk == 0) ? 0u : 1u);
+            }
           }
         } else {
           const int lb = blk - nmain;
@@ -417,7 +452,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           tc_fence_after();
           const uint32_t dacc = tbase + buf * 256;
           bool ok = true;
-          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = take(blk, dacc);
+          for (int blk = 0; blk < nmain && ok; ++blk) ok = take(blk, dacc);
+          if constexpr (C::kTFused) {
+            // T is complete once these MMAs retire; the epilogue warps turn it
+            // into the LoRA block's operand in shared memory
+            if (ok) commit(t_done);
+            if (ok) ok = wait_bar<kPair>(t_ready, 0u, ctl);
+            tc_fence_after();
+          }
+          for (int blk = nmain; blk < nmain + nlora && ok; ++blk) ok = take(blk, dacc);
           if (!ok) break;
           commit(&acc_full[buf]);
         }
@@ -493,6 +536,55 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         if (t == unit) okm = mask_pass(t, it);
         if (okm && t + nunits < p.num_tiles) okm = mask_pass(t + nunits, it + 1);
         if (!okm) break;
+      }
+      if constexpr (C::kTFused) {
+        // Fused T (one tile per unit): once the main K-loop has retired, the
+        // column-half-0 warps read this row's T from tensor memory, save it in
+        // fp32 (the N-tile-0 unit only; every unit of the row block computes
+        // the same T) and write bf16(s T) as row row_in_tile of the LoRA
+        // block's A operand: the A area of the stage the LoRA block occupies
+        // (the unit's blocks are the main K-blocks, then the LoRA block),
+        // SWIZZLE_128B, 16-byte chunk c at position c ^ (row & 7).
+        if (h == 0) {
+          if (!wait_bar<kPair>(t_done, 0u, ctl)) break;
+          tc_fence_after();
+          __syncwarp();
+          uint4* lrow = reinterpret_cast<uint4*>(smem + static_cast<uint32_t>(C::kKPairs * nkb % S) * C::kStageBytes +
+                                                 row_in_tile * 128);
+          const uint32_t tlT = tbase + 256 + (static_cast<uint32_t>(q * 32) << 16);
+          const bool wr = p.t_save != nullptr && nt == 0 && row_ok;
+          for (int c0 = 0; c0 < p.rp; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(tlT + static_cast<uint32_t>(c0), v);
+            tmem_wait_ld();
+            if (wr) {
+              float* dst = p.t_save + static_cast<size_t>(row) * p.r + c0;
+#pragma unroll
+              for (int c = 0; c < 16; c += 4)
+                if (c0 + c < p.r)
+                  *reinterpret_cast<float4*>(dst + c) = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                                                    __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = p.lora_scale * __uint_as_float(v[8 * hh + e]);
+              uint4 pk;
+              pk.x = pack_bf16x2(f[0], f[1]);
+              pk.y = pack_bf16x2(f[2], f[3]);
+              pk.z = pack_bf16x2(f[4], f[5]);
+              pk.w = pack_bf16x2(f[6], f[7]);
+              lrow[((c0 >> 3) + hh) ^ (row_in_tile & 7)] = pk;
+            }
+          }
+          fence_proxy_async_smem();     // the tensor core reads the operand through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(t_ready), 0));
+            else mbar_arrive(t_ready);
+          }
+        }
       }
       if (!wait_bar<kPair>(&acc_full[buf], use & 1u, ctl)) break;
       tc_fence_after();

@@ -21,6 +21,7 @@ CASES = [
     (260, 512, 264, 64, 16.0, "silu"),
     (136, 256, 392, 8, 16.0, "swiglu"),
     (256, 512, 520, 64, 16.0, "swiglu"),
+    (100, 512, 520, 16, 16.0, "identity"),      # one CTA per tile: T fused into the forward GEMM
     (1, 256, 256, 8, 16.0, "identity"),         # single token
     (17, 264, 1032, 24, 16.0, "identity"),      # r not a power of two
     # ranks above 64: two 64-wide LoRA K-blocks per projection
