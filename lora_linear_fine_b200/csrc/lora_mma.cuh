@@ -256,13 +256,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       // area and 128 rows of N-side operand (64 per CTA of a pair).
       constexpr uint32_t kTxFull = C::kCtas * C::kStageBytes;
       constexpr uint32_t kTxSwigluLora = C::kCtas * C::kABytes + 128 * 64 * 2;
-      // Block blk of tile t (main K-blocks first, then the LoRA blocks) into
-      // the next ring stage; false if the wait for the stage gave up.
-      auto put = [&](int t, int blk) -> bool {
+      // This CTA's first row and the tile's first column of tile t.
+      auto origin = [&](int t, int& m0, int& n0) {
         int mt, nt;
         mma_tile_coords(t, p, mt, nt);
-        const int m0 = mt * C::kTileM + 128 * static_cast<int>(crank);
-        const int n0 = nt * C::kOutCols;
+        m0 = mt * C::kTileM + 128 * static_cast<int>(crank);
+        n0 = nt * C::kOutCols;
+      };
+      // Block blk (main K-blocks first, then the LoRA blocks) of the tile at
+      // (m0, n0) into the next ring stage; false if the wait for the stage
+      // gave up.
+      auto put = [&](int m0, int n0, int blk) -> bool {
         if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) return false;
         uint8_t* sa = smem + rp.stage * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
@@ -335,17 +339,24 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         // of the other accumulator buffer overlaps this tile's K-loop:
         //   L(t0), main(t0)[0, h), L(t1), main(t0)[h, n), main(t1)[0, h), L(t2), ...
         const int h = nmain / 2;
+        int m0, n0, m1 = 0, n1 = 0;
         for (int t = unit; t < p.num_tiles && ok; t += nunits) {
+          origin(t, m0, n0);
           if (t == unit)
-            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(t, nmain + lb);
-          for (int blk = 0; blk < h && ok; ++blk) ok = put(t, blk);
-          if (t + nunits < p.num_tiles)
-            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(t + nunits, nmain + lb);
-          for (int blk = h; blk < nmain && ok; ++blk) ok = put(t, blk);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m0, n0, nmain + lb);
+          for (int blk = 0; blk < h && ok; ++blk) ok = put(m0, n0, blk);
+          if (t + nunits < p.num_tiles) {
+            origin(t + nunits, m1, n1);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m1, n1, nmain + lb);
+          }
+          for (int blk = h; blk < nmain && ok; ++blk) ok = put(m0, n0, blk);
         }
       } else {
-        for (int t = unit; t < p.num_tiles && ok; t += nunits)
-          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(t, blk);
+        int m0, n0;
+        for (int t = unit; t < p.num_tiles && ok; t += nunits) {
+          origin(t, m0, n0);
+          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
+        }
       }
       if (!ok && leader) {
         RingPos q = rp;
