@@ -119,32 +119,39 @@ __device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&out)[16]) {
 template <int kNT, bool kW4, int kAR>
 struct SmallMCfg {
   static constexpr int kKPS = kW4 ? 1 : 2;              // 64-wide K blocks per stage
-  // per K block: [X slot | A slot | W tile | (4-bit) codes | scales]
+  // per K block, bf16: [X slot | A slot | W tile]; 4-bit: [X slot | A slot |
+  // codes | scales], the expanded W tiles living in a short ring of their own
+  // (kWBufs tiles), so that the small code stages can all be in flight
   static constexpr int kXBox = kNT * 64 * 2;            // X tile: kNT rows x 64
   static constexpr int kABox = kAR * 64 * 2;            // A slot: kAR >= a_rows rows x 64
-  static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64 (4-bit weight: expanded here)
+  static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64
   static constexpr int kQBox = kW4 ? 128 * 32 : 0;      // 4-bit weight: packed codes, 128 rows x 32 bytes
   static constexpr int kSBox = kW4 ? 128 * 2 : 0;       // 4-bit weight: the 128 rows' scales of this K block
   static constexpr int kXOff = 0;
   static constexpr int kAOff = kXBox;
-  static constexpr int kWOff = kXBox + kABox;
-  static constexpr int kQOff = kWOff + kWBox;
+  static constexpr int kWOff = kXBox + kABox;           // bf16
+  static constexpr int kQOff = kXBox + kABox;           // 4-bit
   static constexpr int kSOff = kQOff + kQBox;
-  static constexpr int kBlockBytes = (kSOff + kSBox + 1023) / 1024 * 1024;
+  static constexpr int kBlockBytes = kW4 ? (kSOff + kSBox + 1023) / 1024 * 1024 : kWOff + kWBox;
   static constexpr int kStageBytes = kKPS * kBlockBytes;
+  static constexpr int kWBufs = kW4 ? 3 : 0;            // expanded W tiles (4-bit)
+  static constexpr int kWRingBytes = kWBufs * kWBox;
   static constexpr int kLd = kNT + 4;                   // parked row stride (floats): 16-byte rows, conflict-free float4 stores
   static constexpr int kBsBytes = 128 * 66 * 2;         // B rows of this CTA's features, bf16, stride r + 2
   static constexpr int kTailBytes = kBsBytes + 1024 + 1024;   // B rows, barriers, alignment slack
-  static constexpr int kStages0 = (kSmemLimitBytes - kTailBytes) / kStageBytes;
-  static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
+  static constexpr int kStages0 = (kSmemLimitBytes - kTailBytes - kWRingBytes) / kStageBytes;
+  static constexpr int kMaxStages = kW4 ? 16 : 8;
+  static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kWRingBytes + kTailBytes;
   static constexpr uint32_t kTmemCols = 128;            // D_Z: kNT columns, then D_T: kAR columns
   // after the K loop the ring holds: Dp [128][kLd], Tp [128][kLd], Tf [64][kNT]
   static constexpr int kParkBytes = 2 * 128 * kLd * 4 + kNT * 64 * 4;
-  static_assert(kXBox % 1024 == 0 && kABox % 1024 == 0 && kWBox % 1024 == 0, "swizzle atoms");
+  static_assert(kXBox % 1024 == 0 && kABox % 1024 == 0 && kWBox % 1024 == 0 && kBlockBytes % 1024 == 0, "swizzle atoms");
   static_assert(kNT + kAR <= static_cast<int>(kTmemCols), "tensor memory");
-  // the T window (128 rows = 16 KB from the X slot) stays inside its block
-  static_assert(kXBox + kABox + kWBox >= 128 * 128, "T window");
+  // The T product reads a 128-row window (16 KB) from the X slot; only its
+  // first kNT rows are used.  It stays inside this block (bf16) or inside the
+  // ring plus the W tiles behind it (4-bit, from the last stage's X slot).
+  static_assert(kW4 ? kStageBytes + kWRingBytes >= 128 * 128 : kXBox + kABox + kWBox >= 128 * 128, "T window");
   static_assert(kStages >= 3, "ring too shallow");
   static_assert(kParkBytes <= kStages * kStageBytes, "parked partials must fit the ring");
 };
@@ -159,15 +166,17 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kBsBytes);
+  uint8_t* wring = smem + S * C::kStageBytes;         // [kWBufs][16 KB] 4-bit: expanded W tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wring + C::kWRingBytes + C::kBsBytes);
   uint64_t* full = bars;                 // [S]
   uint64_t* empty = bars + S;            // [S]
-  uint64_t* dq_full = bars + 2 * S;      // [S] 4-bit weight: W tile expanded (one arrival per epilogue warp)
-  uint64_t* acc_full = bars + 3 * S;
+  uint64_t* wfull = bars + 2 * S;        // [kWBufs] 4-bit: W tile expanded (one arrival per epilogue warp)
+  uint64_t* wempty = wfull + (kW4 ? C::kWBufs : 0);   // [kWBufs] 4-bit: W tile read by the MMAs
+  uint64_t* acc_full = wempty + (kW4 ? C::kWBufs : 0);
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  __nv_bfloat16* Bs = reinterpret_cast<__nv_bfloat16*>(smem + S * C::kStageBytes);   // [F][r + 2], first in the tail
+  __nv_bfloat16* Bs = reinterpret_cast<__nv_bfloat16*>(wring + C::kWRingBytes);   // [F][r + 2], first in the tail
   float* Dp = reinterpret_cast<float*>(smem);                               // [128][kLd]  Z^T partial
   float* Tp = Dp + 128 * C::kLd;                                            // [128][kLd]  T^T partial
   float* Tf = Tp + 128 * C::kLd;                                            // [64][kNT]   summed T, tokens contiguous
@@ -185,7 +194,8 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
   const int f0 = rank * F;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); mbar_init(&dq_full[i], 4); }
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < (kW4 ? C::kWBufs : 0); ++i) { mbar_init(&wfull[i], 4); mbar_init(&wempty[i], 1); }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -248,12 +258,12 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       constexpr uint32_t kIdZ = idesc_bf16(128, kNT, false, false);
       const uint32_t kIdT = idesc_bf16(128, p.a_rows, false, false);
       const int ns = (nk + C::kKPS - 1) / C::kKPS;
-      RingPos rp;
+      RingPos rp, wp;                   // wp: the 4-bit W tile ring
       bool ok = true;
       for (int i = 0; i < ns; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
         if constexpr (kW4) {
-          if (!mbar_wait(&dq_full[rp.stage], rp.phase, ctl)) { ok = false; break; }
+          if (!mbar_wait(&wfull[wp.stage], wp.phase, ctl)) { ok = false; break; }
         }
         tc_fence_after();
         if (i == 0) sm_trace(p, kTrFirstData);
@@ -263,7 +273,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
           const uint32_t sblk = smem_u32(smem + rp.stage * C::kStageBytes + j * C::kBlockBytes);
           const uint32_t sx = sblk + C::kXOff;
           const uint32_t sa = sblk + C::kAOff;
-          const uint32_t sw = sblk + C::kWOff;
+          const uint32_t sw = kW4 ? smem_u32(wring + wp.stage * C::kWBox) : sblk + C::kWOff;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t dw = sdesc_sw128(sw + kk * 32, 16, 1024);
@@ -276,6 +286,10 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
         }
         mma_commit(&empty[rp.stage]);
         rp.next(S);
+        if constexpr (kW4) {            // one K block per stage: one W tile
+          mma_commit(&wempty[wp.stage]);
+          wp.next(C::kWBufs);
+        }
       }
       if (ok && nk > 0) mma_commit(acc_full);
       // Teardown: every MMA issued here retires before TMEM is freed.
@@ -297,29 +311,32 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       Bs[fl * (p.r + 2) + c] = n < p.d_out ? p.B[static_cast<size_t>(n) * p.r + c] : __float2bfloat16_rn(0.0f);
     }
     if constexpr (kW4) {
-      // Dequantise each stage's W tile: thread lrow owns row lrow (32 bytes of
-      // codes, one scale) and writes its 128-byte row of the SWIZZLE_128B tile,
-      // 16-byte chunk c (features 8c .. 8c + 7) at position c ^ (lrow & 7).
-      RingPos rp;
+      // Dequantise each stage's codes into the next W tile of the W ring:
+      // thread lrow owns row lrow (32 bytes of codes, one scale) and writes
+      // its 128-byte row of the SWIZZLE_128B tile, 16-byte chunk c (features
+      // 8c .. 8c + 7) at position c ^ (lrow & 7).
+      RingPos rp, wp;
       const bool tr = p.trace != nullptr && et == 0;
       unsigned long long t_wait = 0, t_work = 0, t0 = tr ? sm_clock_ns() : 0;
       for (int i = 0; i < nk; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
+        if (!mbar_wait(&wempty[wp.stage], wp.phase ^ 1u, ctl)) break;
         if (tr) { const unsigned long long t1 = sm_clock_ns(); t_wait += t1 - t0; t0 = t1; }
-        uint8_t* st = smem + rp.stage * C::kStageBytes;     // one K block per stage (kKPS = 1)
+        const uint8_t* st = smem + rp.stage * C::kStageBytes;     // one K block per stage (kKPS = 1)
         const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + lrow * 32);
         const uint4 c0 = codes[0], c1 = codes[1];
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const __nv_bfloat162 sc2 =
             __bfloat162bfloat162(reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff)[lrow]);
-        uint4* wrow = reinterpret_cast<uint4*>(st + C::kWOff + lrow * 128);
+        uint4* wrow = reinterpret_cast<uint4*>(wring + wp.stage * C::kWBox + lrow * 128);
 #pragma unroll
         for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
         fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
         __syncwarp();                 // the warp's rows are written; one arrival per warp
-        if (lane == 0) mbar_arrive(&dq_full[rp.stage]);
+        if (lane == 0) mbar_arrive(&wfull[wp.stage]);
         if (tr) { const unsigned long long t1 = sm_clock_ns(); t_work += t1 - t0; t0 = t1; }
         rp.next(S);
+        wp.next(C::kWBufs);
       }
       if (tr) {
         p.trace[static_cast<size_t>(blockIdx.x) * kSmTraceStride + kTrDqWait] = t_wait;
