@@ -651,6 +651,17 @@ def small_m_roofline(lay, ms, peaks):
             "hbm_gbs": round(gbs, 1), "roofline_us": round(max(t_tensor, t_hbm) * 1e6, 2)}
 
 
+def small_m_kernel_name(lay, launches_per_forward):
+    """The kernel(s) one forward of a few-token workload runs: the cluster
+    split-K kernel up to 64 tokens; above, one GEMM launch when T is
+    accumulated inside it (one tile per CTA pair), else the T pass first."""
+    if lay.M <= 64:
+        return "small_m_kernel"
+    if launches_per_forward == 1:
+        return "lora_mma_kernel (forward GEMM, T accumulated in the GEMM)"
+    return "rank_gemm_kernel (T) + lora_mma_kernel (forward GEMM)"
+
+
 def small_m_back_to_back(L, lay, peaks, copies=None, reps=20):
     """Few-token forwards launched back to back over distinct copies of W (as
     the layers of one decode step), no flush between them: each launch streams
@@ -698,8 +709,7 @@ def measure_small_m(L, name, local, flush, seconds=0.3, peaks=None, lay=None):
     r = time_steps(L, lay.fwd, steps, 3, flush, lay.stream, local)
     ms = statistics.median(r["ms"])
     roof = small_m_roofline(lay, ms, peaks)
-    kernel = "small_m_kernel" if lay.M <= 64 else "rank_gemm_kernel (T) + lora_mma_kernel (forward GEMM)"
-    roof["kernel"] = kernel
+    roof["kernel"] = small_m_kernel_name(lay, r["launches"] // steps)
     if lay.M <= 64:
         roof["traffic"] = committed_traffic(name, "small_m_traffic.json", "lora_small_m.cuh")
     F = roof["flop_per_launch"]
@@ -939,7 +949,7 @@ def run_small_m_line(args, cfg, L, world, rank, local, dist, flush, peaks):
     med = statistics.median(r["ms"])
     tot_ms = max_over_ranks(sum(r["ms"]), dist, "cuda")
     roof = small_m_roofline(lay, med, peaks)
-    roof["kernel"] = "small_m_kernel" if lay.M <= 64 else "rank_gemm_kernel (T) + lora_mma_kernel (forward GEMM)"
+    roof["kernel"] = small_m_kernel_name(lay, r["launches"] // max(args.steps, 1))
     if lay.M <= 64:
         roof["traffic"] = committed_traffic(args.config, "small_m_traffic.json", "lora_small_m.cuh")
     F = roof["flop_per_launch"]
