@@ -255,8 +255,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       // LoRA blocks fill both areas; a forward SwiGLU LoRA block fills the A
       // area and 128 rows of N-side operand (64 per CTA of a pair).
       constexpr uint32_t kTxFull = C::kCtas * C::kStageBytes;
-      constexpr int kL2Ahead = 8;                      // K blocks prefetched into L2 past the ring
-      const bool single_wave = p.num_tiles <= nunits;
       constexpr uint32_t kTxSwigluLora = C::kCtas * C::kABytes + 128 * 64 * 2;
       // This CTA's first row and the tile's first column of tile t.
       auto origin = [&](int t, int& m0, int& n0) {
@@ -288,23 +286,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
           if constexpr (C::kTFused)
             load(sb + C::kBBytes, &p.tm_am, fb, k0, p.am_rows * static_cast<int>(crank), pol_keep);
-          if constexpr (!kBwd && !C::kSwigluFwd) {
-            // One wave of tiles: every unit sweeps K in step, so each K block is
-            // a first touch of DRAM just when it is needed.  Prefetch into L2
-            // the blocks kL2Ahead past the ring's reach (and, over the first
-            // kL2Ahead blocks, the ones just past the ring).
-            if (single_wave) {
-              const int kb = blk - j * nkb;
-              auto pf = [&](int kbp) {
-                if (kbp < nkb) {
-                  tma_prefetch_l2_2d(&p.tm_a[j], kbp * 64, m0);
-                  tma_prefetch_l2_2d(&p.tm_w[0], kbp * 64, n0 + C::kBRows * static_cast<int>(crank));
-                }
-              };
-              if (kb < kL2Ahead) pf(kb + S);
-              pf(kb + S + kL2Ahead);
-            }
-          }
           if constexpr (!kBwd) {
             if constexpr (C::kSwigluFwd) {
               if constexpr (kPair) load(sb, &p.tm_w[crank], fb, k0, n0, pol_keep);
