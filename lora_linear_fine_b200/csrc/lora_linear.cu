@@ -110,6 +110,23 @@ bool make_tm(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, u
   return r == CUDA_SUCCESS;
 }
 
+// 3D bf16 view [K blocks][rows][64] of a row-major [rows x 64 nkb] matrix
+// (rows row_elems elements apart), 128-byte swizzle: box 64 x box_rows x
+// box_kb lands in shared memory as box_kb consecutive [box_rows x 64] tiles.
+bool make_tm3(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t nkb, uint64_t row_elems, uint32_t box_rows,
+              uint32_t box_kb) {
+  cuuint64_t dims[3] = {64, rows, nkb};
+  cuuint64_t strides[2] = {row_elems * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_kb};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) LORA_LOG("cuTensorMapEncodeTiled (3D) failed (%d): rows=%llu nkb=%llu box=%ux%u", (int)r,
+                                  (unsigned long long)rows, (unsigned long long)nkb, box_rows, box_kb);
+  return r == CUDA_SUCCESS;
+}
+
 // Tensor map over a plain row-major array without swizzle (the 4-bit weight's
 // codes and scales): inner x outer elements of elem_bytes, rows row_bytes apart.
 bool make_tm_plain(CUtensorMap* tm, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
@@ -700,13 +717,14 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
   SmallMParams q;
   std::memset(&q, 0, sizeof(q));
   const bool w4 = Wq != nullptr || Wt != nullptr;
+  const uint32_t kps = static_cast<uint32_t>(small_m_kps(nt, w4, small_m_ar(r)));
   q.Wt = static_cast<const uint8_t*>(Wt);
   bool ok = Wt != nullptr ? make_tm_plain(&q.tm_ws, Ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->d_out,
-                                          d->d_in / kW4Group, d->d_out * 2, 128, 1)
+                                          d->d_in / kW4Group, d->d_out * 2, 128, kps)
           : w4 ? make_tm_plain(&q.tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, d->d_in / 2, d->d_out, d->d_in / 2, 32,
                                128) &&
                      make_tm_plain(&q.tm_ws, Ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->d_out, d->d_in / kW4Group,
-                                   d->d_out * 2, 128, 1)
+                                   d->d_out * 2, 128, kps)
                : make_tm(&q.tm_w, W, d->d_in, d->d_out, d->d_in, 64, 128);
   if (!ok ||
       !make_tm(&q.tm_a, A, d->d_in, r, d->d_in, 64, static_cast<uint32_t>(align_up(static_cast<size_t>(r), 16))) ||
@@ -724,6 +742,15 @@ lora_status_t run_small_m_fwd(const lora_linear_desc* d, int nt, const void* X, 
   q.s = d->s;
   q.act = d->act;
   q.a_rows = static_cast<int>(align_up(static_cast<size_t>(r), 16));
+  // One TMA load per operand and stage through 3D views when the K blocks
+  // are whole (a 3D view cannot zero-fill a ragged last block); otherwise
+  // one 2D box per K block into the same layout.
+  if (d->d_in % 64 == 0) {
+    const uint64_t nkb = static_cast<uint64_t>(d->d_in / 64);
+    q.load3d = make_tm3(&q.tm_x3, X, M, nkb, d->d_in, static_cast<uint32_t>(nt), kps) &&
+               make_tm3(&q.tm_a3, A, r, nkb, d->d_in, static_cast<uint32_t>(small_m_ar(r)), kps) &&
+               (w4 || make_tm3(&q.tm_w3, W, d->d_out, nkb, d->d_in, 128, kps));
+  }
   const int slices = static_cast<int>(ceil_div(d->d_out, 128));
   {
     // The cluster size depends only on the device and the shape: ask the

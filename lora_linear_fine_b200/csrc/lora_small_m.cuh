@@ -41,10 +41,14 @@ constexpr int kSmMaxCluster = 16;
 
 struct SmallMParams {
   CUtensorMap tm_w;          // W [d_out x d_in], box 64 x 128; 4-bit weight: Wq [d_out x d_in/2] bytes, box 32 x 128
-  CUtensorMap tm_ws;         // 4-bit weight only: scales [d_in/64 x d_out] bf16, box 128 x 1
+  CUtensorMap tm_ws;         // 4-bit weight only: scales [d_in/64 x d_out] bf16, box 128 x kKPS
   const uint8_t* Wt;         // 4-bit weight: the codes in the tiled layout (lora_w4.cuh), or null (tm_w)
   CUtensorMap tm_a;          // A [r x d_in],     box 64 x a_rows (rows >= r zero-filled)
   CUtensorMap tm_x;          // X [M x d_in],     box 64 x kNT (rows >= M zero-filled)
+  // The same operands as 3D views [K blocks][rows][64] (d_in a multiple of
+  // 64): box 64 x rows x kKPS, one TMA load per operand and stage
+  CUtensorMap tm_x3, tm_a3, tm_w3;   // tm_a3: box kAR rows; tm_w3: bf16 weight only
+  int load3d;                // 1: the 3D views are used; 0: one 2D box per K block
   const __nv_bfloat16* B;    // [d_out x r]
   __nv_bfloat16* Y;          // [M x d_out]
   float* T_save;             // [M x r] or null
@@ -116,42 +120,48 @@ __device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&out)[16]) {
   for (int c = 0; c < 16; ++c) out[c] = __uint_as_float(v[c]);
 }
 
+// 64-wide K blocks per pipeline stage.  Each operand of a stage arrives in
+// one TMA operation (a 3D box over consecutive K blocks), and the SM issues
+// TMA operations at a roughly fixed cost each, whatever their size: so the
+// 4-bit kernel, whose per-block tiles are small, takes four blocks a stage
+// when its X and A tiles are small enough, the others two.
+constexpr int small_m_kps(int nt, bool w4, int ar) { return w4 ? ((nt + ar) * 128 <= 4096 ? 4 : 2) : 2; }
+
 template <int kNT, bool kW4, int kAR>
 struct SmallMCfg {
-  static constexpr int kKPS = kW4 ? 1 : 2;              // 64-wide K blocks per stage
-  // per K block, bf16: [X slot | A slot | W tile]; 4-bit: [X slot | A slot |
-  // codes | scales], the expanded W tiles living in a short ring of their own
-  // (kWBufs tiles), so that the small code stages can all be in flight
+  static constexpr int kKPS = small_m_kps(kNT, kW4, kAR);
+  // stage = [X tiles | A tiles | W tiles (bf16) or code tiles + scale rows
+  // (4-bit)], kKPS of each, every tile a SWIZZLE_128B image of its 64-wide K
+  // block; the 4-bit kernel expands its codes into a short ring of W tiles
+  // of its own (kWBufs), so that the small code stages can all be in flight
   static constexpr int kXBox = kNT * 64 * 2;            // X tile: kNT rows x 64
   static constexpr int kABox = kAR * 64 * 2;            // A slot: kAR >= a_rows rows x 64
   static constexpr int kWBox = 128 * 64 * 2;            // W tile: 128 rows x 64
   static constexpr int kQBox = kW4 ? 128 * 32 : 0;      // 4-bit weight: packed codes, 128 rows x 32 bytes
-  static constexpr int kSBox = kW4 ? 128 * 2 : 0;       // 4-bit weight: the 128 rows' scales of this K block
+  static constexpr int kSBox = kW4 ? 128 * 2 : 0;       // 4-bit weight: the 128 rows' scales of one K block
   static constexpr int kXOff = 0;
-  static constexpr int kAOff = kXBox;
-  static constexpr int kWOff = kXBox + kABox;           // bf16
-  static constexpr int kQOff = kXBox + kABox;           // 4-bit
-  static constexpr int kSOff = kQOff + kQBox;
-  static constexpr int kBlockBytes = kW4 ? (kSOff + kSBox + 1023) / 1024 * 1024 : kWOff + kWBox;
-  static constexpr int kStageBytes = kKPS * kBlockBytes;
+  static constexpr int kAOff = kKPS * kXBox;
+  static constexpr int kWOff = kAOff + kKPS * kABox;    // bf16
+  static constexpr int kQOff = kWOff;                   // 4-bit
+  static constexpr int kSOff = kQOff + kKPS * kQBox;    // 4-bit
+  static constexpr int kStageBytes = kW4 ? (kSOff + kKPS * kSBox + 1023) / 1024 * 1024 : kWOff + kKPS * kWBox;
   static constexpr int kWBufs = kW4 ? 3 : 0;            // expanded W tiles (4-bit)
   static constexpr int kWRingBytes = kWBufs * kWBox;
   static constexpr int kLd = kNT + 4;                   // parked row stride (floats): 16-byte rows, conflict-free float4 stores
   static constexpr int kBsBytes = 128 * 66 * 2;         // B rows of this CTA's features, bf16, stride r + 2
   static constexpr int kTailBytes = kBsBytes + 1024 + 1024;   // B rows, barriers, alignment slack
   static constexpr int kStages0 = (kSmemLimitBytes - kTailBytes - kWRingBytes) / kStageBytes;
-  static constexpr int kMaxStages = kW4 ? 16 : 8;
-  static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
+  static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kWRingBytes + kTailBytes;
   static constexpr uint32_t kTmemCols = 128;            // D_Z: kNT columns, then D_T: kAR columns
   // after the K loop the ring holds: Dp [128][kLd], Tp [128][kLd], Tf [64][kNT]
   static constexpr int kParkBytes = 2 * 128 * kLd * 4 + kNT * 64 * 4;
-  static_assert(kXBox % 1024 == 0 && kABox % 1024 == 0 && kWBox % 1024 == 0 && kBlockBytes % 1024 == 0, "swizzle atoms");
+  static_assert(kXBox % 1024 == 0 && kABox % 1024 == 0 && kWBox % 1024 == 0 && kStageBytes % 1024 == 0, "swizzle atoms");
   static_assert(kNT + kAR <= static_cast<int>(kTmemCols), "tensor memory");
-  // The T product reads a 128-row window (16 KB) from the X slot; only its
-  // first kNT rows are used.  It stays inside this block (bf16) or inside the
-  // ring plus the W tiles behind it (4-bit, from the last stage's X slot).
-  static_assert(kW4 ? kStageBytes + kWRingBytes >= 128 * 128 : kXBox + kABox + kWBox >= 128 * 128, "T window");
+  // The T product reads a 128-row window (16 KB) from an X tile; only its
+  // first kNT rows are used.  From the last stage's last X tile it stays
+  // inside the ring plus what follows it (the W tiles or the B rows).
+  static_assert((kKPS - 1) * kXBox + 128 * 128 <= kStageBytes + kWRingBytes + kBsBytes, "T window");
   static_assert(kStages >= 3, "ring too shallow");
   static_assert(kParkBytes <= kStages * kStageBytes, "parked partials must fit the ring");
 };
@@ -219,34 +229,46 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
     if (lane == 0) {
       const uint64_t pol_x = l2_policy_evict_last();     // X and A are re-read by every cluster
       // Every slice's CTA of the same rank reads the same A and X tiles; each
-      // slice starts its K loop at a different block (slice mod nk) so that
-      // those reads spread over the L2 instead of converging on one tile.
-      const int rot = nk > 0 ? slice % nk : 0;
-      RingPos rp;
+      // slice starts its K loop at a different stage (slice mod stages) so
+      // that those reads spread over the L2 instead of converging on one tile.
       const int ns = (nk + C::kKPS - 1) / C::kKPS;      // stages: kKPS K blocks each, the last possibly fewer
+      const int rot = ns > 0 ? slice % ns : 0;
+      RingPos rp;
       for (int i = 0; i < ns; ++i) {
         if (!mbar_wait(&empty[rp.stage], rp.phase ^ 1u, ctl)) break;
         uint8_t* st = smem + rp.stage * C::kStageBytes;
-        const int nb = (nk - i * C::kKPS) < C::kKPS ? (nk - i * C::kKPS) : C::kKPS;
-        constexpr uint32_t kWBytes = kW4 ? C::kQBox + C::kSBox : C::kWBox;
-        mbar_arrive_expect_tx(&full[rp.stage],
-                              static_cast<uint32_t>(nb * (kWBytes + C::kXBox + p.a_rows * 128)));
-        for (int j = 0; j < nb; ++j) {
-          const int kb = kb0 + (i * C::kKPS + j + rot) % nk;
-          const int k0 = kb * 64;
-          uint8_t* blk = st + j * C::kBlockBytes;
-          if constexpr (kW4) {
-            if (p.Wt != nullptr)      // one 4 KB tile of codes
-              bulk_load_1d(blk + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kb) * kW4TileBytes,
-                           kW4TileBytes, &full[rp.stage]);
-            else
-              tma_load_2d(blk + C::kQOff, &p.tm_w, &full[rp.stage], k0 / 2, slice * 128);  // codes: k0 / 2 bytes in
-            tma_load_2d(blk + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kb);    // scales of group kb
-          } else {
-            tma_load_2d(blk + C::kWOff, &p.tm_w, &full[rp.stage], k0, slice * 128);
+        const int si = (i + rot) % ns;
+        const int kbf = kb0 + si * C::kKPS;              // the stage's first K block
+        const int nb = (nk - si * C::kKPS) < C::kKPS ? (nk - si * C::kKPS) : C::kKPS;
+        // bytes: 3D boxes and the scales' box count all kKPS blocks (zero
+        // fill past the tensor included); per-block 2D boxes and code tiles nb
+        // (the 3D A box is kAR rows, zero past r, so that A tile j sits at
+        // kAOff + j * kABox as the 2D boxes of a_rows rows put it)
+        uint32_t tx = p.load3d ? static_cast<uint32_t>(C::kKPS * (C::kXBox + C::kABox))
+                               : static_cast<uint32_t>(nb * (C::kXBox + p.a_rows * 128));
+        if constexpr (kW4) tx += C::kKPS * C::kSBox + nb * C::kQBox;
+        else tx += (p.load3d ? C::kKPS : nb) * C::kWBox;
+        mbar_arrive_expect_tx(&full[rp.stage], tx);
+        if (p.load3d) {
+          tma_load_3d_hint(st + C::kXOff, &p.tm_x3, &full[rp.stage], 0, 0, kbf, pol_x);
+          tma_load_3d_hint(st + C::kAOff, &p.tm_a3, &full[rp.stage], 0, 0, kbf, pol_x);
+          if constexpr (!kW4) tma_load_3d(st + C::kWOff, &p.tm_w3, &full[rp.stage], 0, slice * 128, kbf);
+        } else {
+          for (int j = 0; j < nb; ++j) {
+            const int k0 = (kbf + j) * 64;
+            tma_load_2d_hint(st + C::kXOff + j * C::kXBox, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
+            tma_load_2d_hint(st + C::kAOff + j * C::kABox, &p.tm_a, &full[rp.stage], k0, 0, pol_x);
+            if constexpr (!kW4) tma_load_2d(st + C::kWOff + j * C::kWBox, &p.tm_w, &full[rp.stage], k0, slice * 128);
           }
-          tma_load_2d_hint(blk + C::kAOff, &p.tm_a, &full[rp.stage], k0, 0, pol_x);
-          tma_load_2d_hint(blk + C::kXOff, &p.tm_x, &full[rp.stage], k0, 0, pol_x);
+        }
+        if constexpr (kW4) {
+          if (p.Wt != nullptr)        // the stage's code tiles are contiguous in the tiled layout
+            bulk_load_1d(st + C::kQOff, p.Wt + (static_cast<size_t>(slice) * nkb + kbf) * kW4TileBytes,
+                         static_cast<uint32_t>(nb * kW4TileBytes), &full[rp.stage]);
+          else
+            for (int j = 0; j < nb; ++j)   // codes: (kbf + j) * 32 bytes into each row
+              tma_load_2d(st + C::kQOff + j * C::kQBox, &p.tm_w, &full[rp.stage], (kbf + j) * 32, slice * 128);
+          tma_load_2d(st + C::kSOff, &p.tm_ws, &full[rp.stage], slice * 128, kbf);   // scales of groups kbf ..
         }
         if (i == 0) sm_trace(p, kTrFirstIssue);
         if (i < kSmTraceStages) sm_trace(p, kSmTracePoints + i);
@@ -258,22 +280,25 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       constexpr uint32_t kIdZ = idesc_bf16(128, kNT, false, false);
       const uint32_t kIdT = idesc_bf16(128, p.a_rows, false, false);
       const int ns = (nk + C::kKPS - 1) / C::kKPS;
+      const int rot = ns > 0 ? slice % ns : 0;          // the producer's stage order
       RingPos rp, wp;                   // wp: the 4-bit W tile ring
       bool ok = true;
-      for (int i = 0; i < ns; ++i) {
+      for (int i = 0; i < ns && ok; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) { ok = false; break; }
-        if constexpr (kW4) {
-          if (!mbar_wait(&wfull[wp.stage], wp.phase, ctl)) { ok = false; break; }
-        }
         tc_fence_after();
         if (i == 0) sm_trace(p, kTrFirstData);
         if (i < kSmTraceStages) sm_trace(p, kSmTracePoints + kSmTraceStages + i);
-        const int nb = (nk - i * C::kKPS) < C::kKPS ? (nk - i * C::kKPS) : C::kKPS;
+        const int si = (i + rot) % ns;
+        const int nb = (nk - si * C::kKPS) < C::kKPS ? (nk - si * C::kKPS) : C::kKPS;
+        const uint32_t sst = smem_u32(smem + rp.stage * C::kStageBytes);
         for (int j = 0; j < nb; ++j) {
-          const uint32_t sblk = smem_u32(smem + rp.stage * C::kStageBytes + j * C::kBlockBytes);
-          const uint32_t sx = sblk + C::kXOff;
-          const uint32_t sa = sblk + C::kAOff;
-          const uint32_t sw = kW4 ? smem_u32(wring + wp.stage * C::kWBox) : sblk + C::kWOff;
+          if constexpr (kW4) {
+            if (!mbar_wait(&wfull[wp.stage], wp.phase, ctl)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint32_t sx = sst + C::kXOff + j * C::kXBox;
+          const uint32_t sa = sst + C::kAOff + j * C::kABox;
+          const uint32_t sw = kW4 ? smem_u32(wring + wp.stage * C::kWBox) : sst + C::kWOff + j * C::kWBox;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t dw = sdesc_sw128(sw + kk * 32, 16, 1024);
@@ -283,13 +308,14 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
             mma_bf16(tbase, dw, dx, kIdZ, acc);          // Z^T partial: 128 rows of W x tokens
             mma_bf16(tbase + kNT, dx, da, kIdT, acc);    // T partial: 128-row token window x rows of A
           }
+          if constexpr (kW4) {            // this block's W tile is free once these MMAs retire
+            mma_commit(&wempty[wp.stage]);
+            wp.next(C::kWBufs);
+          }
         }
+        if (!ok) break;
         mma_commit(&empty[rp.stage]);
         rp.next(S);
-        if constexpr (kW4) {            // one K block per stage: one W tile
-          mma_commit(&wempty[wp.stage]);
-          wp.next(C::kWBufs);
-        }
       }
       if (ok && nk > 0) mma_commit(acc_full);
       // Teardown: every MMA issued here retires before TMEM is freed.
@@ -311,32 +337,40 @@ __global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_con
       Bs[fl * (p.r + 2) + c] = n < p.d_out ? p.B[static_cast<size_t>(n) * p.r + c] : __float2bfloat16_rn(0.0f);
     }
     if constexpr (kW4) {
-      // Dequantise each stage's codes into the next W tile of the W ring:
+      // Dequantise each K block's codes into the next W tile of the W ring:
       // thread lrow owns row lrow (32 bytes of codes, one scale) and writes
       // its 128-byte row of the SWIZZLE_128B tile, 16-byte chunk c (features
-      // 8c .. 8c + 7) at position c ^ (lrow & 7).
+      // 8c .. 8c + 7) at position c ^ (lrow & 7).  Stages come in the
+      // producer's order (rotated by slice).
+      const int ns = (nk + C::kKPS - 1) / C::kKPS;
+      const int rot = ns > 0 ? slice % ns : 0;
       RingPos rp, wp;
       const bool tr = p.trace != nullptr && et == 0;
       unsigned long long t_wait = 0, t_work = 0, t0 = tr ? sm_clock_ns() : 0;
-      for (int i = 0; i < nk; ++i) {
+      bool ok_dq = true;
+      for (int i = 0; i < ns && ok_dq; ++i) {
         if (!mbar_wait(&full[rp.stage], rp.phase, ctl)) break;
-        if (!mbar_wait(&wempty[wp.stage], wp.phase ^ 1u, ctl)) break;
-        if (tr) { const unsigned long long t1 = sm_clock_ns(); t_wait += t1 - t0; t0 = t1; }
-        const uint8_t* st = smem + rp.stage * C::kStageBytes;     // one K block per stage (kKPS = 1)
-        const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + lrow * 32);
-        const uint4 c0 = codes[0], c1 = codes[1];
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const __nv_bfloat162 sc2 =
-            __bfloat162bfloat162(reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff)[lrow]);
-        uint4* wrow = reinterpret_cast<uint4*>(wring + wp.stage * C::kWBox + lrow * 128);
+        const int si = (i + rot) % ns;
+        const int nb = (nk - si * C::kKPS) < C::kKPS ? (nk - si * C::kKPS) : C::kKPS;
+        const uint8_t* st = smem + rp.stage * C::kStageBytes;
+        for (int j = 0; j < nb; ++j) {
+          if (!mbar_wait(&wempty[wp.stage], wp.phase ^ 1u, ctl)) { ok_dq = false; break; }
+          if (tr) { const unsigned long long t1 = sm_clock_ns(); t_wait += t1 - t0; t0 = t1; }
+          const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + j * C::kQBox + lrow * 32);
+          const uint4 c0 = codes[0], c1 = codes[1];
+          const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const __nv_bfloat162 sc2 =
+              __bfloat162bfloat162(reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff + j * C::kSBox)[lrow]);
+          uint4* wrow = reinterpret_cast<uint4*>(wring + wp.stage * C::kWBox + lrow * 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
-        fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
-        __syncwarp();                 // the warp's rows are written; one arrival per warp
-        if (lane == 0) mbar_arrive(&wfull[wp.stage]);
-        if (tr) { const unsigned long long t1 = sm_clock_ns(); t_work += t1 - t0; t0 = t1; }
+          for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
+          fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
+          __syncwarp();                 // the warp's rows are written; one arrival per warp
+          if (lane == 0) mbar_arrive(&wfull[wp.stage]);
+          if (tr) { const unsigned long long t1 = sm_clock_ns(); t_work += t1 - t0; t0 = t1; }
+          wp.next(C::kWBufs);
+        }
         rp.next(S);
-        wp.next(C::kWBufs);
       }
       if (tr) {
         p.trace[static_cast<size_t>(blockIdx.x) * kSmTraceStride + kTrDqWait] = t_wait;
