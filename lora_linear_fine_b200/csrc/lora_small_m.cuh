@@ -145,7 +145,11 @@ struct SmallMCfg {
   static constexpr int kQOff = kWOff;                   // 4-bit
   static constexpr int kSOff = kQOff + kKPS * kQBox;    // 4-bit
   static constexpr int kStageBytes = kW4 ? (kSOff + kKPS * kSBox + 1023) / 1024 * 1024 : kWOff + kKPS * kWBox;
-  static constexpr int kWBufs = kW4 ? 3 : 0;            // expanded W tiles (4-bit)
+  // expanded W tiles (4-bit): a tile is free again only when the MMAs of the
+  // block that used it have retired, so the ring must cover that latency
+  // (three tiles measured short at four blocks a stage: the expanding warps
+  // waited as long as they worked)
+  static constexpr int kWBufs = kW4 ? (kKPS == 4 ? 6 : 3) : 0;
   static constexpr int kWRingBytes = kWBufs * kWBox;
   static constexpr int kLd = kNT + 4;                   // parked row stride (floats): 16-byte rows, conflict-free float4 stores
   static constexpr int kBsBytes = 128 * 66 * 2;         // B rows of this CTA's features, bf16, stride r + 2
