@@ -304,8 +304,9 @@ struct RankReduceJob {
 
 // Blocks of rpb (<= kReduceRows) result rows (grid-stride over row blocks;
 // blockIdx.y selects the job).  Each thread sums float4 pieces of the partial
-// rows over the splits in split order (eight splits of loads in flight), into
-// a shared-memory tile; then row-major outputs are written by warps along a
+// rows over the splits in split order (eight splits of loads in flight; with
+// few pieces and many splits, four threads per piece over quarters of the
+// splits), into a shared-memory tile; then row-major outputs are written by warps along a
 // row and transposed outputs by warps along a column, so every global access
 // is coalesced and no index needs a division.  RP is a power of two and r a
 // multiple of 8, so a float4 piece lies wholly inside or wholly past r.
@@ -316,6 +317,7 @@ __global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, R
   grid_dep_wait();
   const RankReduceJob& J = blockIdx.y == 0 ? j0 : j1;
   __shared__ float tile[kReduceRows][kMaxRank + 1];
+  __shared__ float4 quarter[4][64];
   const int r = J.out.r;
   const RankOut& o = J.out;
   const int rpb = J.rpb;
@@ -331,7 +333,50 @@ __global__ void __launch_bounds__(256, 2) reduce_rank_kernel(RankReduceJob j0, R
     const int nrows = J.out.rows - row0 < rpb ? J.out.rows - row0 : rpb;
     const int U = nrows * q4;
     __syncthreads();
-    for (int base = 0; base < U; base += 256 * kEPT) {
+    if (U <= 64 && J.splits > 8) {
+      // Few pieces, many splits (dB: a few rows per block, a split per token
+      // range): four threads per piece, each summing a quarter of the splits
+      // in order, then the four quarter sums added in order.
+      const int g = threadIdx.x >> 6, u = threadIdx.x & 63;
+      const int rr = u >> lgq, c0 = 4 * (u & (q4 - 1));
+      const bool in = u < U && c0 < r;
+      const int per = (J.splits + 3) / 4;
+      const int s0 = g * per, s1 = s0 + per < J.splits ? s0 + per : J.splits;
+      const float4* src = part4 + static_cast<size_t>(row0 + (in ? rr : 0)) * q4 + (c0 >> 2);
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int sp0 = s0; sp0 < s1; sp0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = (in && sp0 + k < s1) ? __ldcg(src + static_cast<size_t>(sp0 + k) * stride4)
+                                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          acc.x += v[k].x;
+          acc.y += v[k].y;
+          acc.z += v[k].z;
+          acc.w += v[k].w;
+        }
+      }
+      quarter[g][u] = acc;
+      __syncthreads();
+      if (g == 0 && in) {
+        float4 a = quarter[0][u];
+#pragma unroll
+        for (int k = 1; k < 4; ++k) {
+          a.x += quarter[k][u].x;
+          a.y += quarter[k][u].y;
+          a.z += quarter[k][u].z;
+          a.w += quarter[k][u].w;
+        }
+        float* t = &tile[rr][c0];
+        t[0] = a.x;
+        t[1] = a.y;
+        t[2] = a.z;
+        t[3] = a.w;
+      }
+    }
+    for (int base = 0; base < (U <= 64 && J.splits > 8 ? 0 : U); base += 256 * kEPT) {
       float4 acc[kEPT];
       const float4* src[kEPT];
       bool in[kEPT];
