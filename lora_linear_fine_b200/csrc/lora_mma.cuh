@@ -256,23 +256,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       // area and 128 rows of N-side operand (64 per CTA of a pair).
       constexpr uint32_t kTxFull = C::kCtas * C::kStageBytes;
       constexpr uint32_t kTxSwigluLora = C::kCtas * C::kABytes + 128 * 64 * 2;
-      // This CTA's first row and the tile's first column of tile t, and the
-      // K block its main loop starts at.  With one tile per unit all units
-      // sweep K at once; starting each tile at a different block, spread
-      // evenly over K, makes every K block a first touch of DRAM for one
-      // tile and an L2 hit for the others sharing its X rows or W rows.
-      const bool single_wave = p.num_tiles <= nunits;
-      auto origin = [&](int t, int& m0, int& n0, int& rot) {
+      // This CTA's first row and the tile's first column of tile t.
+      auto origin = [&](int t, int& m0, int& n0) {
         int mt, nt;
         mma_tile_coords(t, p, mt, nt);
         m0 = mt * C::kTileM + 128 * static_cast<int>(crank);
         n0 = nt * C::kOutCols;
-        rot = single_wave ? static_cast<int>((static_cast<long long>(nt * p.m_tiles + mt) * nkb) / p.num_tiles) : 0;
       };
       // Block blk (main K-blocks first, then the LoRA blocks) of the tile at
       // (m0, n0) into the next ring stage; false if the wait for the stage
       // gave up.
-      auto put = [&](int m0, int n0, int rot, int blk) -> bool {
+      auto put = [&](int m0, int n0, int blk) -> bool {
         if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) return false;
         uint8_t* sa = smem + rp.stage * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
@@ -288,9 +282,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         if (!lora_blk) {
           // main block: projection j, K-block kb
           const int j = blk / nkb;
-          int kb = blk - j * nkb + rot;
-          if (kb >= nkb) kb -= nkb;
-          const int k0 = kb * 64;
+          const int k0 = (blk - j * nkb) * 64;
           load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
           if constexpr (C::kTFused)
             load(sb + C::kBBytes, &p.tm_am, fb, k0, p.am_rows * static_cast<int>(crank), pol_keep);
@@ -347,23 +339,23 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         // of the other accumulator buffer overlaps this tile's K-loop:
         //   L(t0), main(t0)[0, h), L(t1), main(t0)[h, n), main(t1)[0, h), L(t2), ...
         const int h = nmain / 2;
-        int m0, n0, r0, m1 = 0, n1 = 0, r1 = 0;
+        int m0, n0, m1 = 0, n1 = 0;
         for (int t = unit; t < p.num_tiles && ok; t += nunits) {
-          origin(t, m0, n0, r0);
+          origin(t, m0, n0);
           if (t == unit)
-            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m0, n0, r0, nmain + lb);
-          for (int blk = 0; blk < h && ok; ++blk) ok = put(m0, n0, r0, blk);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m0, n0, nmain + lb);
+          for (int blk = 0; blk < h && ok; ++blk) ok = put(m0, n0, blk);
           if (t + nunits < p.num_tiles) {
-            origin(t + nunits, m1, n1, r1);
-            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m1, n1, r1, nmain + lb);
+            origin(t + nunits, m1, n1);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m1, n1, nmain + lb);
           }
-          for (int blk = h; blk < nmain && ok; ++blk) ok = put(m0, n0, r0, blk);
+          for (int blk = h; blk < nmain && ok; ++blk) ok = put(m0, n0, blk);
         }
       } else {
-        int m0, n0, r0;
+        int m0, n0;
         for (int t = unit; t < p.num_tiles && ok; t += nunits) {
-          origin(t, m0, n0, r0);
-          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, r0, blk);
+          origin(t, m0, n0);
+          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
         }
       }
       if (!ok && leader) {
