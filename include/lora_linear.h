@@ -474,11 +474,14 @@ typedef struct lora_ce_desc {
     int64_t V;     /* vocabulary size (rows of W) */
 } lora_ce_desc;
 
-/* Bytes of device workspace lora_linear_ce_fwd (0) or lora_linear_ce_bwd (1)
- * needs: the forward holds 8 bytes per token and 128-entry block of the
- * vocabulary plus 8 bytes per token; the backward holds the gradient of the
- * logits of one chunk of at most 8192 tokens (chunk * V * 2 bytes).  The
- * backward size is never below the forward size.  0 for an invalid desc. */
+/* Bytes of device workspace lora_linear_ce_fwd (0), lora_linear_ce_bwd (1)
+ * or lora_linear_ce_fwd_bwd (2) needs: the forward holds 8 bytes per token
+ * and 128-entry block of the vocabulary plus 8 bytes per token; the backward
+ * holds the gradient of the logits of one chunk of at most 8192 tokens
+ * (chunk * V * 2 bytes); the fused call holds, per chunk, the forward's
+ * partials, the chunk's fp32 logits and their bf16 gradient (chunk * V * 6
+ * bytes, 6.3 GB at 8192 tokens and V = 128256).  The backward size is never
+ * below the forward size.  0 for an invalid desc. */
 size_t lora_linear_ce_workspace_size(const lora_ce_desc* desc, int for_backward);
 
 /* Forward.  H, W (device, read); labels [M] (device, read); loss: device fp32
@@ -497,6 +500,21 @@ lora_status_t lora_linear_ce_fwd(const lora_ce_desc* desc, const void* H, const 
 lora_status_t lora_linear_ce_bwd(const lora_ce_desc* desc, const void* H, const void* W, const int32_t* labels,
                                  const float* lse, const float* dloss, void* dH, void* workspace,
                                  size_t workspace_bytes, void* stream);
+
+/* Forward and backward in one call, for a loss that is the step's final
+ * scalar (its upstream factor *dloss already on the device, e.g. 1.0): the
+ * fine-tuning libraries the pages describe compute this loss's gradient
+ * during the forward pass, chunk by chunk.  Per chunk of at most 8192 tokens
+ * the logit GEMM writes the chunk's fp32 logits to the workspace next to its
+ * (max, sum) partials; the chunk's lse follows, then the logits' gradient
+ * (bf16, the same arithmetic as lora_linear_ce_bwd) and dH = dz W.  The
+ * logits are never recomputed, and never held beyond one chunk.  Writes loss,
+ * lse and dH exactly as lora_linear_ce_fwd followed by lora_linear_ce_bwd
+ * would (the same bits).  workspace >= lora_linear_ce_workspace_size(desc, 2);
+ * other arguments and errors as those two calls. */
+lora_status_t lora_linear_ce_fwd_bwd(const lora_ce_desc* desc, const void* H, const void* W, const int32_t* labels,
+                                     const float* dloss, float* loss, float* lse, void* dH, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

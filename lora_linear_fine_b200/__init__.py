@@ -50,7 +50,7 @@ EXPORTED = ("lora_linear_workspace_size", "lora_linear_workspace_init", "lora_li
             "lora_linear_w4_tiled_bytes", "lora_linear_w4_tile", "lora_linear_fwd_w4_tiled",
             "lora_linear_rmsnorm_fwd", "lora_linear_rmsnorm_bwd", "lora_linear_workspace_size_rope",
             "lora_linear_fwd_rope", "lora_linear_bwd_rope", "lora_linear_ce_workspace_size",
-            "lora_linear_ce_fwd", "lora_linear_ce_bwd")
+            "lora_linear_ce_fwd", "lora_linear_ce_bwd", "lora_linear_ce_fwd_bwd")
 
 
 class LoraLinearDesc(ctypes.Structure):
@@ -148,6 +148,8 @@ def _load():
     lib.lora_linear_ce_fwd.restype = i32
     lib.lora_linear_ce_bwd.argtypes = [cp] + [vp] * 6 + [vp, sz, vp]
     lib.lora_linear_ce_bwd.restype = i32
+    lib.lora_linear_ce_fwd_bwd.argtypes = [cp] + [vp] * 7 + [vp, sz, vp]
+    lib.lora_linear_ce_fwd_bwd.restype = i32
     return lib
 
 
@@ -307,6 +309,11 @@ def lora_linear_ce_fwd(desc, H, W, labels, loss, lse, workspace, workspace_bytes
 def lora_linear_ce_bwd(desc, H, W, labels, lse, dloss, dH, workspace, workspace_bytes, stream) -> int:
     return int(_lib.lora_linear_ce_bwd(ctypes.byref(desc), H, W, labels, lse, dloss, dH, workspace, workspace_bytes,
                                        stream))
+
+
+def lora_linear_ce_fwd_bwd(desc, H, W, labels, dloss, loss, lse, dH, workspace, workspace_bytes, stream) -> int:
+    return int(_lib.lora_linear_ce_fwd_bwd(ctypes.byref(desc), H, W, labels, dloss, loss, lse, dH, workspace,
+                                           workspace_bytes, stream))
 
 
 def linear_cross_entropy(H, W, labels, workspace=None, stream=None):
@@ -496,3 +503,23 @@ def lora_linear_bwd_dropout(desc, dY, X, W, A, B, W_up, A_up, B_up, mask, mask_u
     return int(_lib.lora_linear_bwd_dropout(ctypes.byref(desc), dY, X, W, A, B, W_up, A_up, B_up, mask, mask_up,
                                             float(p_drop), T_save, Z_save, dX, dA, dB, dA_up, dB_up, workspace,
                                             workspace_bytes, stream))
+
+
+def linear_cross_entropy_fwd_bwd(H, W, labels, dloss, workspace=None, stream=None):
+    """(loss, lse, dH) in one call, for a loss that is the step's final scalar
+    (dloss: its upstream factor, a 0-d fp32 device tensor): the same results
+    as linear_cross_entropy followed by linear_cross_entropy_backward, without
+    recomputing the logits."""
+    import torch
+    M, d = H.shape
+    V = W.shape[0]
+    desc = make_ce_desc(M, d, V)
+    ws = (workspace or Workspace(lora_linear_ce_workspace_size(desc, 2), H.device, stream)).ensure(
+        lora_linear_ce_workspace_size(desc, 2), stream)
+    loss = torch.empty((), dtype=torch.float32, device=H.device)
+    lse = torch.empty(M, dtype=torch.float32, device=H.device)
+    dH = torch.empty((M, d), dtype=torch.bfloat16, device=H.device)
+    _check(lora_linear_ce_fwd_bwd(desc, _ptr(H), W.data_ptr(), _ptr(labels), dloss.data_ptr(), loss.data_ptr(),
+                                  _ptr(lse), _ptr(dH), ws.buf.data_ptr(), ws.nbytes, _stream_handle(stream)),
+           "lora_linear_ce_fwd_bwd")
+    return loss, lse, dH

@@ -13,6 +13,9 @@
 //                       accumulation, fixed tree order)
 //   ce_scale_kernel     one CTA: d(loss) / (number of valid tokens), the factor
 //                       of every gradient entry
+//   ce_dz_kernel        the fused forward + backward: the gradient of the loss
+//                       with respect to stored fp32 logits, bf16, with the same
+//                       arithmetic as the kMEpiCeGrad epilogue
 //
 // A token is valid when 0 <= label < V; label < 0 marks a token to ignore.  A
 // label >= V is an argument error: status bit 0x2, and the token is ignored.
@@ -97,6 +100,43 @@ __global__ void __launch_bounds__(kCeMeanThreads) ce_scale_kernel(const int32_t*
   if (bad && status) atomicOr(status, kStatusBadArgument);
   cnt = ce_block_sum(cnt, sh);
   if (threadIdx.x == 0) *scale = cnt > 0.0 ? static_cast<float>(static_cast<double>(*dloss) / cnt) : 0.0f;
+}
+
+// dz[m][v] = (exp(z[m][v] - lse[m]) - [v == label[m]]) * scale, bf16, from
+// the fp32 logits z [M x V] (row-major); 0 for an ignored token.  One thread
+// per 8 consecutive columns (two 16-byte loads, one 16-byte store), grid
+// stride; the expressions are those of the kMEpiCeGrad epilogue, so the
+// result is the one the recomputing backward gives.
+__global__ void __launch_bounds__(256) ce_dz_kernel(const float* __restrict__ z, int M, int V,
+                                                    const int32_t* __restrict__ labels,
+                                                    const float* __restrict__ lse, const float* __restrict__ scale,
+                                                    __nv_bfloat16* __restrict__ dz) {
+  grid_dep_wait();
+  const int per_row = V / 8;
+  const long long n = static_cast<long long>(M) * per_row;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int m = static_cast<int>(i / per_row);
+    const int c0 = static_cast<int>(i - static_cast<long long>(m) * per_row) * 8;
+    const int lab = __ldg(labels + m);
+    const float l = __ldg(lse + m);
+    const float sc = (lab >= 0 && lab < V) ? __ldg(scale) : 0.0f;
+    const float4* src = reinterpret_cast<const float4*>(z + static_cast<size_t>(m) * V + c0);
+    const float4 a = __ldcs(src), b = __ldcs(src + 1);
+    const float zz[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float g[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float pz = __expf(zz[e] - l);
+      g[e] = (pz - (c0 + e == lab ? 1.0f : 0.0f)) * sc;
+    }
+    uint4 pk;
+    pk.x = pack_bf16x2(g[0], g[1]);
+    pk.y = pack_bf16x2(g[2], g[3]);
+    pk.z = pack_bf16x2(g[4], g[5]);
+    pk.w = pack_bf16x2(g[6], g[7]);
+    *reinterpret_cast<uint4*>(dz + static_cast<size_t>(m) * V + c0) = pk;
+  }
 }
 
 }  // namespace lora

@@ -1769,8 +1769,8 @@ constexpr int64_t kCeChunkTokens = 8192;
 
 struct CePlan {
   int n_tiles = 0;        // 256-column vocabulary tiles
-  int64_t chunk = 0;      // tokens per backward chunk
-  size_t part = 0, zlab = 0, loss_tok = 0, scale = 0, dz = 0, total = 0;
+  int64_t chunk = 0;      // tokens per backward (or fused) chunk
+  size_t part = 0, zlab = 0, loss_tok = 0, scale = 0, dz = 0, zf = 0, total = 0;
 };
 
 lora_status_t check_ce_desc(const lora_ce_desc* d) {
@@ -1782,7 +1782,9 @@ lora_status_t check_ce_desc(const lora_ce_desc* d) {
   return LORA_OK;
 }
 
-CePlan ce_plan(const lora_ce_desc* d, bool backward) {
+// mode 0: forward; 1: backward; 2: fused forward + backward (per chunk: the
+// forward's partials, the chunk's fp32 logits and bf16 gradient).
+CePlan ce_plan(const lora_ce_desc* d, int mode) {
   CePlan P;
   const int64_t M = d->M > 0 ? d->M : 1;
   P.n_tiles = static_cast<int>(ceil_div(d->V, 256));
@@ -1792,7 +1794,15 @@ CePlan ce_plan(const lora_ce_desc* d, bool backward) {
     off += align_up(bytes, 256);
     return o;
   };
-  if (!backward) {
+  if (mode == 2) {
+    P.chunk = M < kCeChunkTokens ? M : kCeChunkTokens;
+    P.part = take(static_cast<size_t>(2 * P.n_tiles) * P.chunk * sizeof(float2));
+    P.zlab = take(static_cast<size_t>(P.chunk) * 4);
+    P.loss_tok = take(static_cast<size_t>(M) * 4);
+    P.scale = take(4);
+    P.zf = take(static_cast<size_t>(P.chunk) * d->V * 4);
+    P.dz = take(static_cast<size_t>(P.chunk) * d->V * 2);
+  } else if (mode == 0) {
     P.part = take(static_cast<size_t>(2 * P.n_tiles) * M * sizeof(float2));
     P.zlab = take(static_cast<size_t>(M) * 4);
     P.loss_tok = take(static_cast<size_t>(M) * 4);
@@ -1811,7 +1821,7 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 // or gradient recompute (kMEpiCeGrad).
 template <int kEpi>
 lora_status_t ce_logit_gemm(const void* H, const void* W, int64_t M, int64_t d, int64_t V, const CeParams& ce,
-                            void* dz, uint32_t* status, int sms, cudaStream_t st) {
+                            void* dz, uint32_t* status, int sms, cudaStream_t st, float* zf = nullptr) {
   MmaParams p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = pair_kernel_enabled() && M > 128;
@@ -1822,6 +1832,7 @@ lora_status_t ce_logit_gemm(const void* H, const void* W, int64_t M, int64_t d, 
   p.K = static_cast<int>(d);
   p.lora_ksteps = 0;
   p.out = static_cast<__nv_bfloat16*>(dz);
+  p.out_f32 = zf;
   p.status = status;
   p.ce = ce;
   p.m_tiles = static_cast<int>(ceil_div(M, pair ? 256 : 128));
@@ -1834,15 +1845,41 @@ lora_status_t ce_logit_gemm(const void* H, const void* W, int64_t M, int64_t d, 
   return rs;
 }
 
+// dH [C x d] = dz [C x V] W [V x d]: K = V, W read in place as the MN-major
+// operand.
+lora_status_t ce_dh_gemm(const void* dz, const void* W, int64_t C, int64_t dm, int64_t V, void* dHc, uint32_t* status,
+                         int sms, cudaStream_t st) {
+  MmaParams g;
+  std::memset(&g, 0, sizeof(g));
+  const bool pair = pair_kernel_enabled() && C > 128;
+  if (!make_tm(&g.tm_a[0], dz, V, C, V, 64, 128) || !make_tm(&g.tm_w[0], W, dm, V, dm, 64, 64)) return LORA_ERR_CUDA;
+  g.b_mn = 1;
+  g.M = static_cast<int>(C);
+  g.N = static_cast<int>(dm);
+  g.K = static_cast<int>(V);
+  g.lora_ksteps = 0;
+  g.out = static_cast<__nv_bfloat16*>(dHc);
+  g.status = status;
+  g.m_tiles = static_cast<int>(ceil_div(C, pair ? 256 : 128));
+  g.n_tiles = static_cast<int>(ceil_div(dm, 256));
+  g.num_tiles = g.m_tiles * g.n_tiles;
+  set_raster(g, pair, 2.0 * C * V, 2.0 * V * dm);
+  timing_begin(1, st);
+  const lora_status_t rs = launch_mma_any<true, 1, kMEpiGrad>(pair, g, sms, st);
+  timing_end(1, st);
+  return rs;
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t lora_linear_ce_workspace_size(const lora_ce_desc* desc, int for_backward) {
   if (check_ce_desc(desc) != LORA_OK) return 0;
-  const size_t fwd = ce_plan(desc, false).total;
+  if (for_backward == 2) return ce_plan(desc, 2).total;
+  const size_t fwd = ce_plan(desc, 0).total;
   if (for_backward == 0) return fwd;
-  const size_t bwd = ce_plan(desc, true).total;
+  const size_t bwd = ce_plan(desc, 1).total;
   return bwd > fwd ? bwd : fwd;
 }
 
@@ -1854,7 +1891,7 @@ lora_status_t lora_linear_ce_fwd(const lora_ce_desc* d, const void* H, const voi
   if ((H && !aligned16(H)) || !aligned16(W) || (labels && !aligned4(labels)) || !aligned4(loss) ||
       (lse && !aligned4(lse)))
     return LORA_ERR_ALIGNMENT;
-  const CePlan P = ce_plan(d, false);
+  const CePlan P = ce_plan(d, 0);
   DevInfo dev;
   LORA_TRY(check_arch(&dev));
   if (workspace == nullptr || workspace_bytes < P.total || !aligned16(workspace)) return LORA_ERR_WORKSPACE;
@@ -1894,7 +1931,7 @@ lora_status_t lora_linear_ce_bwd(const lora_ce_desc* d, const void* H, const voi
   if ((H && !aligned16(H)) || !aligned16(W) || (dH && !aligned16(dH)) || (labels && !aligned4(labels)) ||
       (lse && !aligned4(lse)) || !aligned4(dloss))
     return LORA_ERR_ALIGNMENT;
-  const CePlan P = ce_plan(d, true);
+  const CePlan P = ce_plan(d, 1);
   DevInfo dev;
   LORA_TRY(check_arch(&dev));
   if (workspace == nullptr || workspace_bytes < P.total || !aligned16(workspace)) return LORA_ERR_WORKSPACE;
@@ -1919,29 +1956,72 @@ lora_status_t lora_linear_ce_bwd(const lora_ce_desc* d, const void* H, const voi
     ce.lse = lse + m0;
     ce.scale = scale;
     LORA_TRY(ce_logit_gemm<kMEpiCeGrad>(Hc, W, C, dm, V, ce, dz, status, dev.sms, st));
-    // 3. dH = dz W: K = V, W [V x d] read in place as the MN-major operand
-    MmaParams g;
-    std::memset(&g, 0, sizeof(g));
-    const bool pair = pair_kernel_enabled() && C > 128;
-    if (!make_tm(&g.tm_a[0], dz, V, C, V, 64, 128) || !make_tm(&g.tm_w[0], W, dm, V, dm, 64, 64))
-      return LORA_ERR_CUDA;
-    g.b_mn = 1;
-    g.M = static_cast<int>(C);
-    g.N = static_cast<int>(dm);
-    g.K = static_cast<int>(V);
-    g.lora_ksteps = 0;
-    g.out = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(dH) + static_cast<size_t>(m0) * dm * 2);
-    g.status = status;
-    g.m_tiles = static_cast<int>(ceil_div(C, pair ? 256 : 128));
-    g.n_tiles = static_cast<int>(ceil_div(dm, 256));
-    g.num_tiles = g.m_tiles * g.n_tiles;
-    set_raster(g, pair, 2.0 * C * V, 2.0 * V * dm);
-    timing_begin(1, st);
-    const lora_status_t rs = launch_mma_any<true, 1, kMEpiGrad>(pair, g, dev.sms, st);
-    timing_end(1, st);
-    LORA_TRY(rs);
+    // 3. dH = dz W
+    LORA_TRY(ce_dh_gemm(dz, W, C, dm, V, static_cast<uint8_t*>(dH) + static_cast<size_t>(m0) * dm * 2, status,
+                        dev.sms, st));
   }
   return LORA_OK;
+}
+
+lora_status_t lora_linear_ce_fwd_bwd(const lora_ce_desc* d, const void* H, const void* W, const int32_t* labels,
+                                     const float* dloss, float* loss, float* lse, void* dH, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  LORA_TRY(check_ce_desc(d));
+  if (W == nullptr || dloss == nullptr || loss == nullptr ||
+      (d->M > 0 && (H == nullptr || labels == nullptr || lse == nullptr || dH == nullptr)))
+    return LORA_ERR_INVALID_ARG;
+  if ((H && !aligned16(H)) || !aligned16(W) || (dH && !aligned16(dH)) || (labels && !aligned4(labels)) ||
+      (lse && !aligned4(lse)) || !aligned4(dloss) || !aligned4(loss))
+    return LORA_ERR_ALIGNMENT;
+  const CePlan P = ce_plan(d, 2);
+  DevInfo dev;
+  LORA_TRY(check_arch(&dev));
+  if (workspace == nullptr || workspace_bytes < P.total || !aligned16(workspace)) return LORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->M == 0) {   // no token: the mean over no valid token is 0, and there is no dH
+    if (cudaMemsetAsync(loss, 0, sizeof(float), st) != cudaSuccess) return cuda_error("cudaMemsetAsync(loss)");
+    return LORA_OK;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* scale = reinterpret_cast<float*>(ws + P.scale);
+  float* loss_tok = reinterpret_cast<float*>(ws + P.loss_tok);
+  float* zf = reinterpret_cast<float*>(ws + P.zf);
+  void* dz = ws + P.dz;
+  const int64_t M = d->M, dm = d->d, V = d->V;
+  // 1. scale = d(loss) / (number of valid tokens), from the labels alone
+  launch_k(ce_scale_kernel, dim3(1), dim3(kCeMeanThreads), 0, st, false, labels, static_cast<int>(M),
+           static_cast<int>(V), dloss, scale, status);
+  LORA_TRY(check_launch("ce_scale_kernel"));
+  for (int64_t m0 = 0; m0 < M; m0 += P.chunk) {
+    const int C = static_cast<int>((M - m0) < P.chunk ? (M - m0) : P.chunk);
+    const void* Hc = static_cast<const uint8_t*>(H) + static_cast<size_t>(m0) * dm * 2;
+    // 2. the chunk's logits on the tensor cores: (max, sum exp) per
+    //    128-column block and the label's logit, and the fp32 logits themselves
+    CeParams ce{};
+    ce.labels = labels + m0;
+    ce.part = reinterpret_cast<float2*>(ws + P.part);
+    ce.zlab = reinterpret_cast<float*>(ws + P.zlab);
+    LORA_TRY(ce_logit_gemm<kMEpiCeFwdZ>(Hc, W, C, dm, V, ce, nullptr, status, dev.sms, st, zf));
+    // 3. lse and each token's loss
+    launch_k(ce_combine_kernel, dim3(grid_for(C, 256, dev.sms)), dim3(256), 0, st, false,
+             static_cast<const float2*>(ce.part), 2 * P.n_tiles, C, static_cast<int>(V), labels + m0,
+             static_cast<const float*>(ce.zlab), lse + m0, loss_tok + m0, status);
+    LORA_TRY(check_launch("ce_combine_kernel"));
+    // 4. the gradient with respect to the logits, bf16 [C x V]
+    const long long n8 = static_cast<long long>(C) * (V / 8);
+    launch_k(ce_dz_kernel, dim3(grid_for(n8, 256, dev.sms)), dim3(256), 0, st, false,
+             static_cast<const float*>(zf), C, static_cast<int>(V), labels + m0, static_cast<const float*>(lse + m0),
+             static_cast<const float*>(scale), static_cast<__nv_bfloat16*>(dz));
+    LORA_TRY(check_launch("ce_dz_kernel"));
+    // 5. dH = dz W
+    LORA_TRY(ce_dh_gemm(dz, W, C, dm, V, static_cast<uint8_t*>(dH) + static_cast<size_t>(m0) * dm * 2, status,
+                        dev.sms, st));
+  }
+  // 6. the mean over valid tokens
+  launch_k(ce_mean_kernel, dim3(1), dim3(kCeMeanThreads), 0, st, false, static_cast<const float*>(loss_tok), labels,
+           static_cast<int>(M), static_cast<int>(V), loss);
+  return check_launch("ce_mean_kernel");
 }
 
 }  // extern "C"

@@ -60,7 +60,7 @@ constexpr int kMmaThreads = 320;
 enum MmaEpi : int {
   kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5,
   kMEpiCeFwd = 6, kMEpiCeGrad = 7, kMEpiGradF32 = 8, kMEpiGradF16F32 = 9, kMEpiGradDrop = 10,
-  kMEpiGradF16Drop = 11, kMEpiIdentityT = 12
+  kMEpiGradF16Drop = 11, kMEpiIdentityT = 12, kMEpiCeFwdZ = 13
 };
 
 // Dropout on the adapter input, dX epilogue (kMEpiGradDrop / kMEpiGradF16Drop).
@@ -804,10 +804,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             }
           }
         }
-      } else if constexpr (kEpi == kMEpiCeFwd) {
+      } else if constexpr (kEpi == kMEpiCeFwd || kEpi == kMEpiCeFwdZ) {
         // This thread's token row and 128 vocabulary columns [col0, col0 + 128):
         // a running max and sum of exp(z - max) over four 32-column loads
         // (columns past N count as -inf), and z[label] if the label is here.
+        // kMEpiCeFwdZ also stores the fp32 logits, row-major [M x N] at
+        // out_f32 (the fused forward + backward turns them into the gradient).
         const int col0 = nt * 256 + h * 128;
         const int lab = row_ok ? __ldg(p.ce.labels + row) : -1;
         float mx = -INFINITY, se = 0.0f, zl = 0.0f;
@@ -819,6 +821,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           tmem_wait_ld();
           if (c == 3) release_acc();
           const int cb = col0 + 32 * c;
+          if constexpr (kEpi == kMEpiCeFwdZ) {
+            if (row_ok) {
+              float* zr = p.out_f32 + static_cast<size_t>(row) * p.N + cb;
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)      // N is a multiple of 8: a float4 is wholly in or past N
+                if (cb + i < p.N)
+                  st_global_v4_hint(zr + i, make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]), pol_out);
+            }
+          }
           float cm = -INFINITY;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {

@@ -243,6 +243,17 @@ def test_cross_entropy_argument_checks(lib):
     assert fwd(lse=None) == 1
     assert fwd(H=24) == 2
     assert fwd(lab=18) == 2
+    # the fused call: the chunk's fp32 logits and bf16 gradient on top of the forward's partials
+    assert lib.lora_linear_ce_workspace_size(d, 2) >= f + 64 * 1000 * 6
+    both = lambda H=16, dl=16, loss=16, lse=16, dH=16: lib.lora_linear_ce_fwd_bwd(d, H, 16, 16, dl, loss, lse, dH,
+                                                                                 16, 1 << 30, None)
+    assert both(dl=None) == 1
+    assert both(loss=None) == 1
+    assert both(lse=None) == 1
+    assert both(dH=None) == 1
+    assert both(H=None) == 1
+    assert both(dH=24) == 2
+    assert both(dl=18) == 2
     bwd = lambda H=16, lse=16, dl=16, dH=16: lib.lora_linear_ce_bwd(d, H, 16, 16, lse, dl, dH, 16, 1 << 30, None)
     assert bwd(dl=None) == 1
     assert bwd(dH=None) == 1

@@ -152,3 +152,29 @@ def test_ce_llama3_vocabulary_8192_tokens():
            "lse": oracle.compare(lse, lse_ref),
            "dH_rows": oracle.compare(dH[rows], b["dH"])}
     G.assert_all_ok(res)
+
+
+@pytest.mark.parametrize("M,d,V,dloss", [
+    (300, 264, 2048, 1.0),       # CTA pairs, ragged tokens and hidden size
+    (64, 256, 1000, 0.5),        # single CTA, ragged vocabulary tail, upstream factor
+    (8200, 256, 1032, 1.0),      # two chunks (8192 + 8 tokens)
+    (512, 4096, 128256, 1.0),    # Llama-3-8B vocabulary
+])
+def test_ce_fused_forward_backward_matches_separate_calls(M, d, V, dloss):
+    """The fused call's loss, lse and dH equal, bit for bit, those of the
+    forward followed by the backward (same GEMM, same gradient arithmetic),
+    with ignored labels in the batch; and the loss matches the oracle."""
+    import torch
+    import lora_linear_fine_b200 as L
+    H, W, labels = seeded_inputs.draw_ce(M, d, V, seed=3 * M + V)
+    tH, tW, tl = G.dev(H), G.dev(W), _dev_i32(labels)
+    dl = torch.tensor(dloss, dtype=torch.float32, device="cuda")
+    loss1, lse1 = L.linear_cross_entropy(tH, tW, tl)
+    dH1 = L.linear_cross_entropy_backward(tH, tW, tl, lse1, dl)
+    loss2, lse2, dH2 = L.linear_cross_entropy_fwd_bwd(tH, tW, tl, dl)
+    torch.cuda.synchronize()
+    assert (labels < 0).any()
+    assert torch.equal(loss1, loss2) and torch.equal(lse1, lse2) and torch.equal(dH1, dH2)
+    if V <= 32768:
+        ref = CE.linear_ce_forward(G.f64(H), G.f64(W), labels)
+        G.assert_all_ok({"loss": oracle.compare(np.array([float(loss2.item())]), np.array([ref["loss"] * 1.0]))})
