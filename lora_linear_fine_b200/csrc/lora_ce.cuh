@@ -27,29 +27,60 @@ namespace lora {
 
 constexpr int kCeMeanThreads = 1024;
 
+// Merges (max, sum exp(z - max)) partial q into the running (mx, se):
+// rescales the running sum whenever the maximum grows; a partial of a block
+// wholly past V (max -inf) changes nothing.
+__device__ __forceinline__ void ce_merge(float& mx, float& se, float2 q) {
+  if (q.x == -INFINITY) return;
+  if (q.x > mx) {
+    se = se * expf(mx - q.x) + q.y;
+    mx = q.x;
+  } else {
+    se += q.y * expf(q.x - mx);
+  }
+}
+
+constexpr int kCeCombineTokens = 8;                          // tokens per CTA
+constexpr int kCeCombineGroups = 256 / kCeCombineTokens;     // threads per token
+
+// A CTA of 256 threads per 8 tokens: thread (group g, token t) merges the
+// blocks g, g + 32, g + 64, ... of its token in that order; then one thread
+// per token merges the 32 group results in group order (a fixed order, so the
+// result is deterministic) and finishes lse and the token's loss.
 __global__ void __launch_bounds__(256) ce_combine_kernel(const float2* __restrict__ part, int nblk, int M, int V,
                                                          const int32_t* __restrict__ labels,
                                                          const float* __restrict__ zlab, float* __restrict__ lse,
                                                          float* __restrict__ loss_tok, uint32_t* status) {
   grid_dep_wait();
-  for (int m = blockIdx.x * blockDim.x + threadIdx.x; m < M; m += gridDim.x * blockDim.x) {
-    // one pass, rescaling the running sum whenever the maximum grows
+  __shared__ float2 grp[kCeCombineGroups][kCeCombineTokens];
+  const int t = threadIdx.x % kCeCombineTokens, g = threadIdx.x / kCeCombineTokens;
+  for (int m0 = blockIdx.x * kCeCombineTokens; m0 < M; m0 += gridDim.x * kCeCombineTokens) {
+    const int m = m0 + t;
     float mx = -INFINITY, se = 0.0f;
-    for (int b = 0; b < nblk; ++b) {
-      const float2 q = part[static_cast<size_t>(b) * M + m];
-      if (q.x == -INFINITY) continue;        // a block wholly past V
-      if (q.x > mx) {
-        se = se * expf(mx - q.x) + q.y;
-        mx = q.x;
-      } else {
-        se += q.y * expf(q.x - mx);
+    if (m < M) {
+      int b = g;
+      for (; b + 3 * kCeCombineGroups < nblk; b += 4 * kCeCombineGroups) {
+        float2 q[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = part[static_cast<size_t>(b + k * kCeCombineGroups) * M + m];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ce_merge(mx, se, q[k]);
       }
+      for (; b < nblk; b += kCeCombineGroups) ce_merge(mx, se, part[static_cast<size_t>(b) * M + m]);
     }
-    const float l = mx + logf(se);
-    lse[m] = l;
-    const int lab = labels[m];
-    if (lab >= V && status) atomicOr(status, kStatusBadArgument);
-    loss_tok[m] = (lab >= 0 && lab < V) ? l - zlab[m] : 0.0f;
+    grp[g][t] = make_float2(mx, se);
+    __syncthreads();
+    if (g == 0 && m < M) {
+      float tm = -INFINITY, ts = 0.0f;
+#pragma unroll 1
+      for (int k = 0; k < kCeCombineGroups; ++k) ce_merge(tm, ts, grp[k][t]);
+      const float l = tm + logf(ts);
+      lse[m] = l;
+      const int lab = labels[m];
+      if (lab >= V && status) atomicOr(status, kStatusBadArgument);
+      loss_tok[m] = (lab >= 0 && lab < V) ? l - zlab[m] : 0.0f;
+    }
+    __syncthreads();
   }
 }
 

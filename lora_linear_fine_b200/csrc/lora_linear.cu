@@ -1911,7 +1911,7 @@ lora_status_t lora_linear_ce_fwd(const lora_ce_desc* d, const void* H, const voi
   LORA_TRY(ce_logit_gemm<kMEpiCeFwd>(H, W, d->M, d->d, d->V, ce, nullptr, status, dev.sms, st));
   // 2. lse and each token's loss; 3. the mean over valid tokens
   const int M = static_cast<int>(d->M);
-  launch_k(ce_combine_kernel, dim3(grid_for(M, 256, dev.sms)), dim3(256), 0, st, false,
+  launch_k(ce_combine_kernel, dim3(grid_for(M, kCeCombineTokens, dev.sms)), dim3(256), 0, st, false,
            static_cast<const float2*>(ce.part), 2 * P.n_tiles, M, static_cast<int>(d->V), labels,
            static_cast<const float*>(ce.zlab), lse, reinterpret_cast<float*>(ws + P.loss_tok), status);
   LORA_TRY(check_launch("ce_combine_kernel"));
@@ -2004,7 +2004,7 @@ lora_status_t lora_linear_ce_fwd_bwd(const lora_ce_desc* d, const void* H, const
     ce.zlab = reinterpret_cast<float*>(ws + P.zlab);
     LORA_TRY(ce_logit_gemm<kMEpiCeFwdZ>(Hc, W, C, dm, V, ce, nullptr, status, dev.sms, st, zf));
     // 3. lse and each token's loss
-    launch_k(ce_combine_kernel, dim3(grid_for(C, 256, dev.sms)), dim3(256), 0, st, false,
+    launch_k(ce_combine_kernel, dim3(grid_for(C, kCeCombineTokens, dev.sms)), dim3(256), 0, st, false,
              static_cast<const float2*>(ce.part), 2 * P.n_tiles, C, static_cast<int>(V), labels + m0,
              static_cast<const float*>(ce.zlab), lse + m0, loss_tok + m0, status);
     LORA_TRY(check_launch("ce_combine_kernel"));
