@@ -37,9 +37,6 @@ namespace lora {
 
 constexpr int64_t kSmallMMax = 64;
 constexpr int kSmThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-// The 4-bit kernel adds warps 6..7, which only help expand the codes during
-// the K loop (its stream is paced by that expansion).
-constexpr int small_m_threads(bool w4) { return w4 ? kSmThreads + 64 : kSmThreads; }
 constexpr int kSmMaxCluster = 16;
 
 struct SmallMParams {
@@ -178,7 +175,7 @@ struct SmallMCfg {
 // stage's codes into the bf16 W tile (value = bf16(scale * (code - 8)), laid
 // out as the SWIZZLE_128B tile TMA would have written) before the MMA reads it.
 template <int kNT, bool kW4, int kAR>
-__global__ void __launch_bounds__(small_m_threads(kW4), 1) small_m_kernel(const __grid_constant__ SmallMParams p) {
+__global__ void __launch_bounds__(kSmThreads, 1) small_m_kernel(const __grid_constant__ SmallMParams p) {
   using C = SmallMCfg<kNT, kW4, kAR>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -212,10 +209,7 @@ __global__ void __launch_bounds__(small_m_threads(kW4), 1) small_m_kernel(const 
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < (kW4 ? C::kWBufs : 0); ++i) {
-      mbar_init(&wfull[i], (small_m_threads(kW4) - 64) / 32);   // one arrival per expanding warp
-      mbar_init(&wempty[i], 1);
-    }
+    for (int i = 0; i < (kW4 ? C::kWBufs : 0); ++i) { mbar_init(&wfull[i], 4); mbar_init(&wempty[i], 1); }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -341,19 +335,17 @@ __global__ void __launch_bounds__(small_m_threads(kW4), 1) small_m_kernel(const 
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int lrow = q * 32 + lane;
     // this CTA's F rows of B (bf16, row stride r + 2), loaded during the K loop
-    for (int i = et; et < 128 && i < F * p.r; i += 128) {
+    for (int i = et; i < F * p.r; i += 128) {
       const int fl = i / p.r, c = i - fl * p.r;
       const int n = slice * 128 + f0 + fl;
       Bs[fl * (p.r + 2) + c] = n < p.d_out ? p.B[static_cast<size_t>(n) * p.r + c] : __float2bfloat16_rn(0.0f);
     }
     if constexpr (kW4) {
-      // Dequantise each K block's codes into the next W tile of the W ring.
-      // The kET expanding threads (warps 2..7) share the tile's 1024 units
-      // (row, 16-byte chunk c): unit u = (row u / 8, c = u % 8) reads the
-      // row's c-th 4 bytes of codes and writes 8 weights at position
-      // c ^ (row & 7) of the row's 128 bytes (SWIZZLE_128B).  Stages come in
-      // the producer's order (rotated by slice).
-      constexpr int kET = small_m_threads(kW4) - 64;
+      // Dequantise each K block's codes into the next W tile of the W ring:
+      // thread lrow owns row lrow (32 bytes of codes, one scale) and writes
+      // its 128-byte row of the SWIZZLE_128B tile, 16-byte chunk c (features
+      // 8c .. 8c + 7) at position c ^ (lrow & 7).  Stages come in the
+      // producer's order (rotated by slice).
       const int ns = (nk + C::kKPS - 1) / C::kKPS;
       const int rot = ns > 0 ? slice % ns : 0;
       RingPos rp, wp;
@@ -368,20 +360,16 @@ __global__ void __launch_bounds__(small_m_threads(kW4), 1) small_m_kernel(const 
         for (int j = 0; j < nb; ++j) {
           if (!mbar_wait(&wempty[wp.stage], wp.phase ^ 1u, ctl)) { ok_dq = false; break; }
           if (tr) { const unsigned long long t1 = sm_clock_ns(); t_wait += t1 - t0; t0 = t1; }
-          const uint8_t* codes = st + C::kQOff + j * C::kQBox;
-          const __nv_bfloat16* scl = reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff + j * C::kSBox);
-          uint8_t* wt = wring + wp.stage * C::kWBox;
+          const uint4* codes = reinterpret_cast<const uint4*>(st + C::kQOff + j * C::kQBox + lrow * 32);
+          const uint4 c0 = codes[0], c1 = codes[1];
+          const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const __nv_bfloat162 sc2 =
+              __bfloat162bfloat162(reinterpret_cast<const __nv_bfloat16*>(st + C::kSOff + j * C::kSBox)[lrow]);
+          uint4* wrow = reinterpret_cast<uint4*>(wring + wp.stage * C::kWBox + lrow * 128);
 #pragma unroll
-          for (int k = 0; k < (1024 + kET - 1) / kET; ++k) {
-            const int u = et + k * kET;
-            if (u >= 1024) break;
-            const int row = u >> 3, c = u & 7;
-            const uint32_t word = *reinterpret_cast<const uint32_t*>(codes + row * 32 + c * 4);
-            *reinterpret_cast<uint4*>(wt + row * 128 + ((c ^ (row & 7)) << 4)) =
-                w4_word(word, __bfloat162bfloat162(scl[row]));
-          }
+          for (int c = 0; c < 8; ++c) wrow[c ^ (lrow & 7)] = w4_word(words[c], sc2);
           fence_proxy_async_smem();     // the tensor core reads the tile through the async proxy
-          __syncwarp();                 // the warp's units are written; one arrival per warp
+          __syncwarp();                 // the warp's rows are written; one arrival per warp
           if (lane == 0) mbar_arrive(&wfull[wp.stage]);
           if (tr) { const unsigned long long t1 = sm_clock_ns(); t_work += t1 - t0; t0 = t1; }
           wp.next(C::kWBufs);
@@ -393,55 +381,53 @@ __global__ void __launch_bounds__(small_m_threads(kW4), 1) small_m_kernel(const 
         p.trace[static_cast<size_t>(blockIdx.x) * kSmTraceStride + kTrDqWork] = t_work;
       }
     }
-    if (warp < 6) {   // warps 2..5 (the 4-bit kernel's warps 6..7 only expanded codes)
-      bool got = true;
-      if (nk > 0) got = mbar_wait(acc_full, 0, ctl);
-      const bool ok = bar_sync_and<1, 128>(got);
-      // the T partial's lanes are tokens: only the first kNT are real (a
-      // warp-uniform test); each such thread parks its token's r values
-      // transposed, Tp[c][token], the layout the cluster sum below reads
-      const bool t_rows = q * 32 < kNT;
-      float4* drow = reinterpret_cast<float4*>(Dp + lrow * C::kLd);
-      const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
-      if (ok && t_rows) {
-        if (nk > 0) {
-          tc_fence_after();
-          for (int c0 = 0; c0 < p.a_rows; c0 += 16) {
-            float t[16];
-            tmem_ld16f(tl + static_cast<uint32_t>(kNT + c0), t);
-  #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              if (c0 + c < p.r) Tp[(c0 + c) * C::kLd + lrow] = t[c];
-          }
-        } else {
-          for (int c = 0; c < p.r; ++c) Tp[c * C::kLd + lrow] = 0.0f;
+    bool got = true;
+    if (nk > 0) got = mbar_wait(acc_full, 0, ctl);
+    const bool ok = bar_sync_and<1, 128>(got);
+    // the T partial's lanes are tokens: only the first kNT are real (a
+    // warp-uniform test); each such thread parks its token's r values
+    // transposed, Tp[c][token], the layout the cluster sum below reads
+    const bool t_rows = q * 32 < kNT;
+    float4* drow = reinterpret_cast<float4*>(Dp + lrow * C::kLd);
+    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
+    if (ok && t_rows) {
+      if (nk > 0) {
+        tc_fence_after();
+        for (int c0 = 0; c0 < p.a_rows; c0 += 16) {
+          float t[16];
+          tmem_ld16f(tl + static_cast<uint32_t>(kNT + c0), t);
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (c0 + c < p.r) Tp[(c0 + c) * C::kLd + lrow] = t[c];
         }
+      } else {
+        for (int c = 0; c < p.r; ++c) Tp[c * C::kLd + lrow] = 0.0f;
       }
-      if (ok) {
-        // Z partial of feature row lrow
-        if (nk > 0) {
-          tc_fence_after();
-  #pragma unroll
-          for (int c0 = 0; c0 < kNT; c0 += 16) {
-            float v[16];
-            tmem_ld16f(tl + static_cast<uint32_t>(c0), v);
-  #pragma unroll
-            for (int c = 0; c < 16; c += 4) drow[(c0 + c) / 4] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-          }
-        } else {
-  #pragma unroll
-          for (int c = 0; c < kNT / 4; ++c) drow[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        }
-      }
-      if (et == 0) sm_trace(p, kTrPublished);
     }
+    if (ok) {
+      // Z partial of feature row lrow
+      if (nk > 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < kNT; c0 += 16) {
+          float v[16];
+          tmem_ld16f(tl + static_cast<uint32_t>(c0), v);
+#pragma unroll
+          for (int c = 0; c < 16; c += 4) drow[(c0 + c) / 4] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kNT / 4; ++c) drow[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+    }
+    if (et == 0) sm_trace(p, kTrPublished);
   }
   tc_fence_before();
   __syncwarp();   // the cluster barrier is .aligned: each warp arrives converged
   // every CTA of the cluster has parked its partials
   cluster_sync_all();
 
-  if (warp >= 2 && warp < 6 && *abort_flag == 0u) {
+  if (warp >= 2 && *abort_flag == 0u) {
     const int et = threadIdx.x - 64;
     if (et == 0) sm_trace(p, kTrSynced);
     const uint32_t dp_addr = smem_u32(Dp), tp_addr = smem_u32(Tp);
@@ -532,7 +518,7 @@ cudaError_t launch_small_m_kernel(const SmallMParams& p, int slices, bool pdl, c
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(slices * p.splits), 1, 1);
-  cfg.blockDim = dim3(small_m_threads(kW4), 1, 1);
+  cfg.blockDim = dim3(kSmThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -563,7 +549,7 @@ int small_m_splits_t(int slices, int nkb) {
   for (int s = 2; s <= kSmMaxCluster && s <= nkb; s *= 2) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(slices * s), 1, 1);
-    cfg.blockDim = dim3(small_m_threads(kW4), 1, 1);
+    cfg.blockDim = dim3(kSmThreads, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
