@@ -335,8 +335,9 @@ lora_status_t lora_linear_fwd_w4_tiled(const lora_linear_desc* desc, const void*
  * plain ones.  The few-token kernel is not used (dropout is a training-time
  * transform).  No masked copy of X is made: the rank passes that read X for
  * the adapter (T, dA) zero the dropped elements of each X tile in shared
- * memory, and the LoRA term of dX is added in the dX GEMM's epilogue (one
- * projection, r <= 64) or by dx_dropout_kernel after it (SwiGLU, r > 64).
+ * memory.  The masked LoRA term of dX is formed on the tensor cores inside
+ * the dX GEMM (one projection: the term first, its dropped entries zeroed,
+ * dZ W accumulated on top) or added after it (SwiGLU).
  * ------------------------------------------------------------------------ */
 
 /* Workspace bytes for lora_linear_fwd_dropout (0) / lora_linear_bwd_dropout

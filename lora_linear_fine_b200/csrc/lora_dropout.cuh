@@ -10,9 +10,11 @@
 //   dX = dZ W + m * (s' U A)
 // X_m is never stored: the rank passes that read X for the adapter (T and
 // dA) zero the dropped elements of their X tiles in shared memory.  Only the
-// LoRA term of dX needs the mask outside them: the dX GEMM runs without its
-// LoRA K-block and adds m * (s' U A) in its epilogue (one projection, r <= 64)
-// or dx_dropout_kernel, below, adds it afterwards (SwiGLU, r > 64).
+// LoRA term of dX needs the mask outside them.  With one projection the dX
+// GEMM forms s' U A in its accumulator first, zeroes its dropped entries in
+// tensor memory and accumulates dZ W on top (lora_mma.cuh, kMEpiGradDrop);
+// with SwiGLU (two masks on one accumulator) the GEMM runs without its LoRA
+// K-blocks and dx_dropout_kernel, below, adds m * (s' U A) afterwards.
 //
 // Mask layout: [M x d_in/8] bytes, bit j of byte b (least significant first)
 // keeps element 8 b + j.

@@ -1010,9 +1010,9 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
   return v == 0 ? LORA_OK : LORA_ERR_DEVICE_STATUS;
 }
 
-// The forward.  Xl[j] is the input of projection j's adapter branch (X, or
-// the dropout-masked copy of X); allow_small_m = false keeps the tiled path
-// for few tokens.
+// The forward.  Xl[j] is the input of projection j's adapter branch (X; with
+// dropout, fmasks[j] are the keep bits the T pass applies to its X tiles);
+// allow_small_m = false keeps the tiled path for few tokens.
 // Host-side argument checks of a forward (desc, required pointers,
 // alignment): everything that needs neither the device nor the workspace.
 static lora_status_t fwd_check_args(const lora_linear_desc* d, const void* X, const void* W, const void* A,
@@ -1132,8 +1132,10 @@ lora_status_t lora_linear_fwd(const lora_linear_desc* d, const void* X, const vo
 }
 
 // The backward.  Xl[j] is the input of projection j's adapter branch; with
-// dropout masks (masks[0] != null) the dX GEMM runs without its LoRA K-block
-// and dx_dropout_kernel adds the masked LoRA term afterwards.
+// dropout masks (masks[0] != null) the rank passes mask their X tiles, and the
+// dX GEMM forms the masked LoRA term in its accumulator before the main
+// K-blocks (one projection) or runs without its LoRA K-blocks while
+// dx_dropout_kernel adds the masked terms afterwards (SwiGLU).
 static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const void* X, const void* W, const void* A,
                               const void* B, const void* W_up, const void* A_up, const void* B_up,
                               const float* T_save, const float* Z_save, void* dX, float* dA, float* dB,
