@@ -33,8 +33,8 @@ def _ptr(t):
 def _noalloc_call_and_check(M, d_in, d_out, r, act, calls=2):
     """Run the no-alloc forward `calls` times on one seeded problem; after each
     call read its status word (expect 0) and compare Y, T (and Z) with the
-    ordinary workspace forward within the parity tolerance, and Y with the
-    fp64 oracle."""
+    ordinary workspace forward within the parity tolerance, and Y, T (and Z)
+    with the fp64 oracle."""
     import torch
     import lora_linear_fine_b200 as L
     s = 16.0 / r
@@ -58,8 +58,10 @@ def _noalloc_call_and_check(M, d_in, d_out, r, act, calls=2):
         res = {"Y": oracle.compare(G.host_f64(Y), G.host_f64(Y_ref)),
                "T": oracle.compare(G.host_f64(T), G.host_f64(T_ref)),
                "Y_vs_oracle": oracle.compare(G.host_f64(Y), f["Y"])}
+        res["T_vs_oracle"] = oracle.compare(G.host_f64(T).reshape(f["T"].shape), f["T"])
         if Z is not None:
             res["Z"] = oracle.compare(G.host_f64(Z), G.host_f64(Z_ref))
+            res["Z_vs_oracle"] = oracle.compare(G.host_f64(Z).reshape(f["Z"].shape), f["Z"])
         bad = {k: v for k, v in res.items() if not v["ok"]}
         assert not bad, f"call {call}: {bad}"
 
