@@ -427,6 +427,30 @@ class Layer:
     def fwd_gemm_flops(self):    # X W^T + (sT) B^T, per projection
         return self.np * (2.0 * self.M * self.d_in * self.d_out + 2.0 * self.M * self.r * self.d_out)
 
+    def t_in_gemm(self):
+        """Whether the library accumulates T = X A^T inside the forward GEMM
+        (then that launch also does T's 2 M d_in r FLOPs): one identity
+        projection with 0 < r <= 64, no dropout, more than 64 tokens, and
+        either one GEMM tile per CTA pair or at most one 256-row block per
+        pair (the library's own test, with its switches)."""
+        if os.environ.get("LORA_LINEAR_FUSED_T", "1")[:1] == "0":
+            return False
+        if not (0 < self.r <= 64) or self.np != 1 or self.act != "identity" or self.p_drop is not None:
+            return False
+        if self.M <= 64:
+            return False
+        import torch
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        pair = self.M > 128
+        units = sms // 2 if pair else sms
+        m_tiles = -(-self.M // (256 if pair else 128))
+        if m_tiles * -(-self.d_out // 256) <= units:
+            return True
+        return m_tiles <= units and os.environ.get("LORA_LINEAR_SHARED_T", "1")[:1] != "0"
+
+    def fwd_launch_flops(self):  # the forward GEMM launch's work: + T when it is accumulated there
+        return self.fwd_gemm_flops() + (2.0 * self.M * self.d_in * self.r if self.t_in_gemm() else 0.0)
+
     def dx_gemm_flops(self):     # dZ W + (sU) A, per projection
         return self.np * (2.0 * self.M * self.d_in * self.d_out + 2.0 * self.M * self.r * self.d_in)
 
@@ -510,7 +534,7 @@ def measure_layer_workload(L, name, local, flush, seconds=0.5, peaks=None):
            "value": round(tf, 2), "unit": UNIT,
            "roofline": {"bound": "tensor", "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
                         "flop_per_step": F},
-           "forward_gemm": gemm_record(lay.fwd_gemm_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 1, pk),
+           "forward_gemm": gemm_record(lay.fwd_launch_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 1, pk),
            "dx_gemm": gemm_record(lay.dx_gemm_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"], 1, pk),
            "gpu_launches_per_step": r["launches"] // steps, "clocks": r["clocks"]}
     if name == "tiny":
@@ -547,7 +571,7 @@ def measure_mlp(L, local, flush, seconds=0.5, peaks=None):
            "value": round(tf, 2), "unit": UNIT,
            "roofline": {"bound": "tensor", "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
                         "flop_per_step": F},
-           "forward_gemms": gemm_record(gu.fwd_gemm_flops() + dn.fwd_gemm_flops(), r["gemm_fwd_ms"],
+           "forward_gemms": gemm_record(gu.fwd_launch_flops() + dn.fwd_launch_flops(), r["gemm_fwd_ms"],
                                         r["gemm_fwd_n"], 2, pk),
            "dx_gemms": gemm_record(gu.dx_gemm_flops() + dn.dx_gemm_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"],
                                    2, pk),
@@ -1120,12 +1144,14 @@ def main():
     # forward or dX) took longer per launch, each timed by the library's event
     # pair around its launch on this stream; the other is reported beside it.
     pk = peaks["bf16_tflops"]
-    gf = gemm_record(lay.fwd_gemm_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 1, pk)
+    gf = gemm_record(lay.fwd_launch_flops(), r["gemm_fwd_ms"], r["gemm_fwd_n"], 1, pk)
     gb = gemm_record(lay.dx_gemm_flops(), r["gemm_bwd_ms"], r["gemm_bwd_n"], 1, pk)
     traffic = committed_traffic(args.config)
     dom_is_dx = gb is not None and (gf is None or gb["ms_per_launch"] > gf["ms_per_launch"])
     dom, other = (gb, gf) if dom_is_dx else (gf, gb)
-    roof = {"kernel": "lora_mma_kernel (dX GEMM)" if dom_is_dx else "lora_mma_kernel (forward GEMM)",
+    fwd_name = ("lora_mma_kernel (forward GEMM, T accumulated in the GEMM)" if lay.t_in_gemm()
+                else "lora_mma_kernel (forward GEMM)")
+    roof = {"kernel": "lora_mma_kernel (dX GEMM)" if dom_is_dx else fwd_name,
             "bound": "tensor", "achieved": dom["achieved"] if dom else None, "peak": pk, "unit": "TFLOP/s",
             "frac": dom["frac"] if dom else None,
             "peak_kind": f"bf16 burst, {peaks['source']} (sustained {peaks['bf16_tflops_sustained']})",
@@ -1133,8 +1159,7 @@ def main():
             "flop_per_launch": dom["flop_per_step"] if dom else None,
             "ms_per_launch": dom["ms_per_launch"] if dom else None,
             "traffic": (traffic or {}).get("dx" if dom_is_dx else "forward") if isinstance(traffic, dict) else None,
-            "other_gemm": dict(other or {}, kernel="lora_mma_kernel (forward GEMM)" if dom_is_dx
-                               else "lora_mma_kernel (dX GEMM)",
+            "other_gemm": dict(other or {}, kernel=fwd_name if dom_is_dx else "lora_mma_kernel (dX GEMM)",
                                traffic=(traffic or {}).get("forward" if dom_is_dx else "dx")
                                if isinstance(traffic, dict) else None),
             "step_frac": round(value / world / pk, 4)}

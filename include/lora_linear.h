@@ -55,7 +55,10 @@
  * - The workspace holds a 32-bit device status word at offset 0.  Kernels OR
  *   error bits into it (a bounded wait that gave up, a failed device-side
  *   check); they never clear it.  Zero it once with lora_linear_workspace_init
- *   before the first call; read it with lora_linear_device_status.
+ *   before the first call; read it with lora_linear_device_status.  Words 8
+ *   to 27 of the same 256-byte header are flags of the forward GEMM (one
+ *   launch sets them and zeroes them again before it ends);
+ *   lora_linear_workspace_init zeroes them too.
  * - Calls that share a workspace must not overlap in time (issue them on one
  *   stream): they use the same scratch regions.
  */
@@ -136,7 +139,13 @@ lora_status_t lora_linear_device_status(const void* workspace, void* stream, uin
  * its predecessor before touching memory).  With 1..64 tokens, identity or
  * SiLU and r > 0 the forward is one launch of thread-block clusters (one
  * cluster of 1..16 CTAs per 128 output features; the cluster size is the
- * largest the device reports it can keep resident for every slice at once). */
+ * largest the device reports it can keep resident for every slice at once).
+ * With more tokens, identity and 0 < r <= 64, it is one GEMM launch that
+ * also computes T, as long as M <= 256 x (SMs / 2) (18944 on a B200): each
+ * 256-row block's first output tile accumulates T = X A^T beside its main
+ * product and publishes bf16(s T) in the workspace; the block's other tiles
+ * wait for it (bounded, as every wait here) before their adapter K-block.
+ * Otherwise a T pass (with its split-K reduction) runs before the GEMM. */
 lora_status_t lora_linear_fwd(const lora_linear_desc* desc,
                               const void* X, const void* W, const void* A, const void* B,
                               const void* W_up, const void* A_up, const void* B_up,

@@ -32,8 +32,13 @@ using namespace lora;
 constexpr int kAbiVersion = 1;
 constexpr int kTargetCtas = 148;   // SM count of a B200; sets split-K widths
 constexpr int64_t kKMajorMinTokens = 12288;   // dX from a W^T copy at and above this many tokens
-// Workspace header, zero at rest: the status block (word 0 is the status word).
+// Workspace header, zero at rest: the status block (word 0 is the status
+// word; words kTFlagWord0 .. kTFlagWord0 + kTFlagWords are the shared-T
+// forward GEMM's exit count and flag bits, which that kernel sets and
+// zeroes again within one launch).
 constexpr size_t kHeaderBytes = 256;
+constexpr int kTFlagWord0 = 8;
+static_assert((kTFlagWord0 + 1 + kTFlagWords) * 4 <= kHeaderBytes, "header too small for the shared-T flags");
 
 // ---------------------------------------------------------------------------
 // debug logging (LORA_LINEAR_DEBUG=1)
@@ -633,12 +638,21 @@ bool pair_kernel_enabled() {
   return v == 1;
 }
 
-// LORA_LINEAR_FUSED_T=0 turns off the forward GEMM's fused T (one tile per
-// unit), so that the separate T pass runs instead (for comparisons).
+// LORA_LINEAR_FUSED_T=0 turns off the forward GEMM's fused T, so that the
+// separate T pass runs instead (for comparisons); LORA_LINEAR_SHARED_T=0
+// turns off only its multi-tile form (a shared T per row block).
 bool fused_t_enabled() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("LORA_LINEAR_FUSED_T");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+bool shared_t_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("LORA_LINEAR_SHARED_T");
     v = (e && e[0] == '0') ? 0 : 1;
   }
   return v == 1;
@@ -1053,13 +1067,22 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   const void* Ap[2] = {A, A_up};
   const void* Bp[2] = {B, B_up};
   const bool pair = pair_kernel_enabled() && M > 128;
-  // One GEMM tile per unit (a single wave, e.g. about a thousand tokens): the
-  // GEMM's second accumulator buffer is free, so T accumulates there during
-  // the main K-loop and the separate T pass (and its split-K reduction) is
-  // skipped.  One identity projection, r <= 64, no dropout, no rotation.
-  const int64_t tiles1 = ceil_div(M, pair ? 256 : 128) * ceil_div(d->d_out, 256);
-  const bool fuse_t = fused_t_enabled() && r > 0 && RP <= 64 && np == 1 && d->act == LORA_ACT_IDENTITY &&
-                      rope == nullptr && fmasks == nullptr && tiles1 <= (pair ? dev.sms / 2 : dev.sms);
+  // T accumulated inside the forward GEMM (one identity projection, r <= 64,
+  // no dropout, no rotation), so that the separate T pass (and its split-K
+  // reduction) is skipped and X is streamed by the GEMM alone:
+  // - one GEMM tile per unit (a single wave, e.g. about a thousand tokens):
+  //   every tile accumulates T in the free second accumulator buffer;
+  // - at most one row block per unit (up to 256 x 74 tokens): the N-tile-0
+  //   tile of each row block goes first on its unit, accumulates T there and
+  //   publishes bf16(s T); the row block's other tiles load it for their
+  //   LoRA block.
+  const int64_t m_tiles1 = ceil_div(M, pair ? 256 : 128);
+  const int64_t tiles1 = m_tiles1 * ceil_div(d->d_out, 256);
+  const int64_t units1 = pair ? dev.sms / 2 : dev.sms;
+  const bool t_in_gemm = fused_t_enabled() && r > 0 && RP <= 64 && np == 1 && d->act == LORA_ACT_IDENTITY &&
+                         rope == nullptr && fmasks == nullptr;
+  const bool share_t = t_in_gemm && tiles1 > units1 && m_tiles1 <= units1 && shared_t_enabled();
+  const bool fuse_t = t_in_gemm && (tiles1 <= units1 || share_t);
   // 1. T_j = X A_j^T (fp32, saved for the backward) and bf16(s T_j) for the LoRA K-block
   if (r > 0 && !fuse_t) {
     for (int j = 0; j < np; ++j) {
@@ -1110,6 +1133,11 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
     p.r = static_cast<int>(r);
     p.lora_scale = d->s;
     p.t_save = T_save;
+    if (share_t) {
+      p.t_shared = 1;
+      p.st_out = reinterpret_cast<__nv_bfloat16*>(ws + P.s16[0]);
+      p.t_flags = status + kTFlagWord0;
+    }
     if (!make_tm(&p.tm_am, A, d->d_in, r, d->d_in, 64, p.am_rows)) return LORA_ERR_CUDA;
     rs = launch_mma_any<false, 1, kMEpiIdentityT>(pair, p, dev.sms, st);
     timing_end(0, st);

@@ -100,15 +100,27 @@ struct MmaParams {
   int out_acc;            // with out_f32: dX += the product (else dX = the product)
   CeParams ce;            // kMEpiCeFwd / kMEpiCeGrad
   DropEpi drop;           // kMEpiGradDrop / kMEpiGradF16Drop
-  // kMEpiIdentityT (forward, one tile per unit): T = X A^T accumulates in the
-  // second accumulator buffer during the main K-loop
+  // kMEpiIdentityT (forward): T = X A^T accumulates in the second accumulator
+  // buffer during the main K-loop of a T tile.  t_shared = 0: every tile is
+  // a T tile (one tile per unit).  t_shared = 1: the first m_tiles tiles are
+  // the N-tile-0 tiles of each row block, one per unit and each its unit's
+  // first tile; they publish bf16(s T) to st_out, and the row block's other
+  // tiles load it from there (tm_la[0]) for their LoRA block once the
+  // publishing CTA's flag bits are set.
   CUtensorMap tm_am;      // A [r x K], box 64 x am_rows (this CTA's am_rows rows of the padded rank)
   int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
   int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
   int r;                  // the rank
   float lora_scale;       // s: the LoRA block's operand is bf16(s T)
   float* t_save;          // fp32 T [M x r] for the backward (written by the N-tile-0 units), or null
+  int t_shared;
+  __nv_bfloat16* st_out;  // t_shared: bf16(s T) [M x r], row-major
+  uint32_t* t_flags;      // t_shared: [0] exit count, [1..kTFlagWords] flag bits; zero at rest
 };
+
+// Flag words of the shared-T forward: 4 bits (one per writing epilogue warp)
+// per CTA of each T tile; the last CTA to exit zeroes them again.
+constexpr int kTFlagWords = 19;
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
 struct MmaCfg {
@@ -121,10 +133,12 @@ struct MmaCfg {
   static constexpr int kABytes = 128 * 64 * 2;               // 16 KB
   static constexpr int kBRows = 256 / kCtas;                 // N-side rows held per CTA
   static constexpr int kBBytes = kBRows * 64 * 2;            // 32 KB (single) / 16 KB (pair)
-  // kMEpiIdentityT: rows of A (the rank, up to 64 in all) per stage and CTA
+  // kMEpiIdentityT: rows of A (the rank, up to 64 in all) per stage and CTA,
+  // in a ring of their own after the main stages, which keep the plain
+  // kernel's layout
   static constexpr bool kTFused = kEpi == kMEpiIdentityT;
   static constexpr int kAMBytes = kTFused ? (64 / kCtas) * 64 * 2 : 0;
-  static constexpr int kStageBytes = kABytes + kBBytes + kAMBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes;
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
   // shared memory (4 KB per warp) so that global stores are row-contiguous.
   static constexpr bool kStaged = kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
@@ -132,9 +146,11 @@ struct MmaCfg {
   // LoRA term is formed in the accumulator before the main K-loop.
   static constexpr bool kDropEpi = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
   static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : 0;
-  static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / kStageBytes;
+  static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / (kStageBytes + kAMBytes);
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kEpiStageBytes + 2048;
+  static constexpr int kAMOff = kStages * kStageBytes;              // the A-rows ring
+  static constexpr int kRingBytes = kStages * (kStageBytes + kAMBytes);
+  static constexpr int kSmemBytes = kRingBytes + kEpiStageBytes + 2048;
   static constexpr uint32_t kTmemCols = 512;                 // 2 accumulator buffers
   static_assert(kStages >= 3, "ring too shallow");
 };
@@ -144,22 +160,31 @@ struct MmaCfg {
 // inside a group of `group` M tiles) or their M-side operand (group_along_n = 1:
 // M fastest inside a group of `group` N tiles, so the whole M-side operand is
 // swept per group and stays in L2 while the N-side operand streams once).
+// With a shared T (t_shared), tiles 0 .. m_tiles - 1 are the N-tile-0 tiles
+// in row order, and the raster covers the remaining N tiles.
 __device__ __forceinline__ void mma_tile_coords(int t, const MmaParams& p, int& mt, int& nt) {
+  int n_tiles = p.n_tiles, nt0 = 0;
+  if (p.t_shared) {
+    if (t < p.m_tiles) { mt = t; nt = 0; return; }
+    t -= p.m_tiles;
+    n_tiles -= 1;
+    nt0 = 1;
+  }
   if (p.group_along_n) {
     const int per_group = p.group * p.m_tiles;
     const int g = t / per_group;
     const int idx = t - g * per_group;
     mt = idx % p.m_tiles;
-    nt = g * p.group + idx / p.m_tiles;
+    nt = nt0 + g * p.group + idx / p.m_tiles;
   } else {
-    const int per_group = p.group * p.n_tiles;
+    const int per_group = p.group * n_tiles;
     const int g = t / per_group;
     const int first_m = g * p.group;
     const int rem = p.m_tiles - first_m;
     const int gm = rem < p.group ? rem : p.group;
     const int idx = t - g * per_group;
     mt = first_m + idx % gm;
-    nt = idx / gm;
+    nt = nt0 + idx / gm;
   }
 }
 
@@ -176,8 +201,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* epi_stage = smem + S * C::kStageBytes;          // [8 warps][4 KB] (kStaged)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kEpiStageBytes);
+  uint8_t* epi_stage = smem + C::kRingBytes;               // [8 warps][4 KB] (kStaged)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kRingBytes + C::kEpiStageBytes);
   uint64_t* full = bars;                  // [S]
   uint64_t* empty = bars + S;             // [S]
   uint64_t* acc_full = bars + 2 * S;      // [2] accumulator buffer b complete
@@ -198,9 +223,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   const int nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
   AbortCtl ctl{abort_flag, p.status};
   if constexpr (C::kTFused) {
-    // The fused T needs one tile per unit (the host's choice); anything else
-    // is refused before any barrier, tensor memory or cluster step.
-    if (p.num_tiles > nunits || p.rp < 16 || p.rp > 64 || p.rp % 16 != 0 || p.am_rows * C::kCtas != p.rp) {
+    // The fused T needs its T tiles to be their units' first tiles (one tile
+    // per unit, or with a shared T one row block per unit); anything else is
+    // refused before any barrier, tensor memory or cluster step.
+    const bool bad_sched = p.t_shared ? (p.m_tiles > nunits || p.st_out == nullptr || p.t_flags == nullptr ||
+                                         p.m_tiles * C::kCtas * 4 > 32 * kTFlagWords)
+                                      : p.num_tiles > nunits;
+    if (bad_sched || p.rp < 16 || p.rp > 64 || p.rp % 16 != 0 || p.am_rows * C::kCtas != p.rp) {
       if (threadIdx.x == 0 && p.status != nullptr) atomicOr(p.status, kStatusBadArgument);
       return;
     }
@@ -272,20 +301,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         uint8_t* sb = sa + C::kABytes;
         const uint32_t fb = rp.stage;
         const bool lora_blk = blk >= C::kKPairs * nkb;
-        if (leader) {
-          uint32_t tx = (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull;
-          if constexpr (C::kTFused)   // main: X, W and am_rows rows of A; LoRA: B only (the epilogue writes s T)
-            tx = lora_blk ? C::kCtas * C::kBBytes
-                          : C::kCtas * (C::kABytes + C::kBBytes + static_cast<uint32_t>(p.am_rows) * 128u);
-          mbar_arrive_expect_tx(&full[rp.stage], tx);
-        }
+        if (leader) mbar_arrive_expect_tx(&full[rp.stage], (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull);
         if (!lora_blk) {
           // main block: projection j, K-block kb
           const int j = blk / nkb;
           const int k0 = (blk - j * nkb) * 64;
           load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
-          if constexpr (C::kTFused)
-            load(sb + C::kBBytes, &p.tm_am, fb, k0, p.am_rows * static_cast<int>(crank), pol_keep);
           if constexpr (!kBwd) {
             if constexpr (C::kSwigluFwd) {
               if constexpr (kPair) load(sb, &p.tm_w[crank], fb, k0, n0, pol_keep);
@@ -310,7 +331,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           const int lb = blk - C::kKPairs * nkb;
           const int j = lb / lkb;
           const int kx = (lb - j * lkb) * 64;
-          if (!C::kTFused) load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
+          load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
           if constexpr (!kBwd) {
             if constexpr (C::kSwigluFwd) {
               // N = 128 outputs of projection j: 128 rows (single) or 64 per CTA (pair)
@@ -325,6 +346,33 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           } else {
             load(sb, &p.tm_lb[j], fb, kx, n0 + C::kBRows * static_cast<int>(crank), pol_keep);   // A^T rows
           }
+        }
+        ++issued;
+        rp.next(S);
+        return true;
+      };
+      // Fused T, a T tile's block blk (one identity projection): a main block
+      // brings X, W and this CTA's am_rows rows of A (into the A-rows ring);
+      // the LoRA block brings only B, since the epilogue warps write bf16(s T)
+      // into its A area.  Kept apart from put so that the other tiles run the
+      // plain per-block path: the producer's per-block work sets the pace of
+      // the whole pipeline.
+      auto put_t = [&](int m0, int n0, int blk) -> bool {
+        if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) return false;
+        uint8_t* sa = smem + rp.stage * C::kStageBytes;
+        uint8_t* sb = sa + C::kABytes;
+        const uint32_t fb = rp.stage;
+        if (blk < nkb) {
+          if (leader)
+            mbar_arrive_expect_tx(&full[rp.stage],
+                                  C::kCtas * (C::kABytes + C::kBBytes + static_cast<uint32_t>(p.am_rows) * 128u));
+          load(sa, &p.tm_a[0], fb, blk * 64, m0, pol_stream);
+          load(smem + C::kAMOff + rp.stage * C::kAMBytes, &p.tm_am, fb, blk * 64,
+               p.am_rows * static_cast<int>(crank), pol_keep);
+          load(sb, &p.tm_w[0], fb, blk * 64, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
+        } else {
+          if (leader) mbar_arrive_expect_tx(&full[rp.stage], C::kCtas * C::kBBytes);
+          load(sb, &p.tm_lb[0], fb, (blk - nkb) * 64, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
         }
         ++issued;
         rp.next(S);
@@ -355,7 +403,21 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         int m0, n0;
         for (int t = unit; t < p.num_tiles && ok; t += nunits) {
           origin(t, m0, n0);
-          for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
+          if constexpr (C::kTFused) {
+            if (!p.t_shared || t < p.m_tiles) {
+              for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put_t(m0, n0, blk);
+            } else {
+              // the row block's T tile publishes bf16(s T): wait for this
+              // CTA's four flag bits before the LoRA block loads it
+              for (int blk = 0; blk < nmain && ok; ++blk) ok = put(m0, n0, blk);
+              const int bit = ((m0 - 128 * static_cast<int>(crank)) / C::kTileM * C::kCtas + static_cast<int>(crank)) * 4;
+              if (ok) ok = flag_wait_all(p.t_flags + 1 + bit / 32, 0xFu << (bit % 32), ctl);
+              fence_proxy_async_global();
+              for (int blk = nmain; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
+            }
+          } else {
+            for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
+          }
         }
       }
       if (!ok && leader) {
@@ -406,10 +468,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
             const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
             mma(dacc, da, db, kIdMain, (!C::kDropEpi && blk == 0 && kk == 0) ? 0u : 1u);
-            if constexpr (C::kTFused) {   // T += X tile x (rows of A)^T, into the second buffer's columns
-              const uint64_t dam = sdesc_sw128(sb + C::kBBytes + kk * 32, 16, 1024);
-              mma(tbase + 256, da, dam, kIdT, (blk == 0 && kk == 0) ? 0u : 1u);
-            }
           }
         } else {
           const int lb = blk - nmain;
@@ -421,6 +479,25 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             const uint64_t db = bmn ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
             mma(dacc + dcol, da, db, kIdLora, (C::kDropEpi && lb == 0 && kk == 0) ? 0u : 1u);
           }
+        }
+        commit(&empty[rp.stage]);
+        rp.next(S);
+        return true;
+      };
+      // Fused T, a T tile's main block blk: the main product and T += X tile
+      // x (rows of A)^T into the second buffer's columns.
+      auto take_t = [&](int blk, uint32_t dacc) -> bool {
+        if (!wait_bar<kPair>(&full[rp.stage], rp.phase, ctl)) return false;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + rp.stage * C::kStageBytes);
+        const uint32_t sb = sa + C::kABytes;
+        const uint32_t sam = smem_u32(smem + C::kAMOff + rp.stage * C::kAMBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = sdesc_sw128(sa + kk * 32, 16, 1024);
+          const uint32_t acc = (blk == 0 && kk == 0) ? 0u : 1u;
+          mma(dacc, da, sdesc_sw128(sb + kk * 32, 16, 1024), kIdMain, acc);
+          mma(tbase + 256, da, sdesc_sw128(sam + kk * 32, 16, 1024), kIdT, acc);
         }
         commit(&empty[rp.stage]);
         rp.next(S);
@@ -463,13 +540,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           tc_fence_after();
           const uint32_t dacc = tbase + buf * 256;
           bool ok = true;
-          for (int blk = 0; blk < nmain && ok; ++blk) ok = take(blk, dacc);
-          if constexpr (C::kTFused) {
+          if (C::kTFused && (!p.t_shared || t < p.m_tiles)) {
+            for (int blk = 0; blk < nmain && ok; ++blk) ok = take_t(blk, dacc);
             // T is complete once these MMAs retire; the epilogue warps turn it
-            // into the LoRA block's operand in shared memory
+            // into the LoRA block's operand in shared memory.  (A unit has at
+            // most one T tile, its first, so both barriers complete once.)
             if (ok) commit(t_done);
             if (ok) ok = wait_bar<kPair>(t_ready, 0u, ctl);
             tc_fence_after();
+          } else {
+            for (int blk = 0; blk < nmain && ok; ++blk) ok = take(blk, dacc);
           }
           for (int blk = nmain; blk < nmain + nlora && ok; ++blk) ok = take(blk, dacc);
           if (!ok) break;
@@ -549,14 +629,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         if (!okm) break;
       }
       if constexpr (C::kTFused) {
-        // Fused T (one tile per unit): once the main K-loop has retired, the
-        // column-half-0 warps read this row's T from tensor memory, save it in
-        // fp32 (the N-tile-0 unit only; every unit of the row block computes
-        // the same T) and write bf16(s T) as row row_in_tile of the LoRA
-        // block's A operand: the A area of the stage the LoRA block occupies
-        // (the unit's blocks are the main K-blocks, then the LoRA block),
-        // SWIZZLE_128B, 16-byte chunk c at position c ^ (row & 7).
-        if (h == 0) {
+        // Fused T: once a T tile's main K-loop has retired, the column-half-0
+        // warps read this row's T from tensor memory, save it in fp32 (the
+        // N-tile-0 unit only; without a shared T every unit of the row block
+        // computes the same T) and write bf16(s T) as row row_in_tile of the
+        // LoRA block's A operand: the A area of the stage the LoRA block
+        // occupies (the T tile is the unit's first, so its blocks are the
+        // ring's first: the main K-blocks, then the LoRA block),
+        // SWIZZLE_128B, 16-byte chunk c at position c ^ (row & 7).  With a
+        // shared T they also store bf16(s T) to st_out and then set this
+        // warp's flag bit for the row block.
+        if (h == 0 && (!p.t_shared || t < p.m_tiles)) {
           if (!wait_bar<kPair>(t_done, 0u, ctl)) break;
           tc_fence_after();
           __syncwarp();
@@ -564,6 +647,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
                                                  row_in_tile * 128);
           const uint32_t tlT = tbase + 256 + (static_cast<uint32_t>(q * 32) << 16);
           const bool wr = p.t_save != nullptr && nt == 0 && row_ok;
+          const bool pub = p.t_shared && row_ok;
           for (int c0 = 0; c0 < p.rp; c0 += 16) {
             uint32_t v[16];
             tmem_ld16(tlT + static_cast<uint32_t>(c0), v);
@@ -587,13 +671,25 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               pk.z = pack_bf16x2(f[4], f[5]);
               pk.w = pack_bf16x2(f[6], f[7]);
               lrow[((c0 >> 3) + hh) ^ (row_in_tile & 7)] = pk;
+              if (pub && c0 + 8 * hh < p.r)
+                *reinterpret_cast<uint4*>(p.st_out + static_cast<size_t>(row) * p.r + c0 + 8 * hh) = pk;
             }
           }
           fence_proxy_async_smem();     // the tensor core reads the operand through the async proxy
+          if (p.t_shared) {
+            // other CTAs read st_out through TMA (the async proxy)
+            fence_proxy_async_global();
+            __threadfence();
+          }
+          tc_fence_before();            // the T columns are rewritten by this unit's next tile
           __syncwarp();
           if (lane == 0) {
             if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(t_ready), 0));
             else mbar_arrive(t_ready);
+            if (p.t_shared) {
+              const int bit = (mt * C::kCtas + static_cast<int>(crank)) * 4 + q;
+              red_or_release_gpu(p.t_flags + 1 + bit / 32, 1u << (bit % 32));
+            }
           }
         }
       }
@@ -907,6 +1003,17 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
   tc_fence_before();
   __syncthreads();
   if constexpr (kPair) cluster_sync_all();
+  if constexpr (C::kTFused) {
+    // Shared T: the last CTA to get here (every other CTA is done with the
+    // flags) zeroes them for the next launch.
+    if (p.t_shared && threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(p.t_flags, 1u) == gridDim.x - 1) {
+        for (int i = 1; i <= kTFlagWords; ++i) atomicExch(p.t_flags + i, 0u);
+        atomicExch(p.t_flags, 0u);
+      }
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     if constexpr (kPair) tmem_dealloc_pair(tbase, C::kTmemCols);

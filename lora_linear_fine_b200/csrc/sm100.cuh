@@ -219,6 +219,45 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same between generic-proxy global accesses and TMA (async-proxy)
+// accesses of global memory: a CTA that publishes data with plain stores for
+// another CTA's TMA loads fences after its stores, and the reader fences
+// after it has acquired the flag and before it issues the loads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Publication flags in global memory: OR with release semantics at GPU scope
+// (the writer's earlier stores become visible to any thread that acquires
+// the bit), and a load with acquire semantics.
+__device__ __forceinline__ void red_or_release_gpu(uint32_t* addr, uint32_t bits) {
+  asm volatile("red.release.gpu.global.or.b32 [%0], %1;" ::"l"(addr), "r"(bits) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+// Wait until all of `bits` are set in the global word at addr (set by
+// another CTA of the same grid).  Bounded like mbar_wait: gives up after
+// kWaitLimitCycles, sets the status word and the CTA's abort flag, and
+// returns false; returns false at once if the CTA is already aborting.
+__device__ __forceinline__ bool flag_wait_all(const uint32_t* addr, uint32_t bits, const AbortCtl& ctl) {
+  if ((ld_acquire_gpu(addr) & bits) == bits) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(64);
+    if ((ld_acquire_gpu(addr) & bits) == bits) return true;
+    if (*ctl.flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      if (ctl.status) atomicOr(ctl.status, kStatusWaitTimeout);
+      *ctl.flag = 1u;
+      return false;
+    }
+  }
+}
+
 // ----------------------------------------------------------------------------
 // Dropout keep bits: one bit per element, bit j of byte b keeping element
 // 8 b + j of a row of `ld` bytes.

@@ -81,12 +81,13 @@ def test_dropout_fwd_bwd(M, d_in, d_out, r, act, p_drop):
 
 def test_dropout_all_kept_matches_plain_layer():
     """p = 0 with every element kept: the forward is bit-identical to the
-    plain call.  The shape has more GEMM tiles (16 x 5) than CTA pairs, so the
-    plain forward also takes the separate T pass (with one tile per pair it
-    fuses T into the GEMM, a different summation order)."""
+    plain call.  The shape has more 256-row blocks (75) than the 74 CTA pairs
+    of a B200, so the plain forward also takes the separate T pass (with at
+    most one row block per pair it accumulates T inside the GEMM, a different
+    summation order)."""
     import lora_linear_fine_b200 as L
     import torch
-    M, d_in, d_out, r = 4096, 512, 1280, 16
+    M, d_in, d_out, r = 75 * 256, 512, 512, 16
     inp = seeded_inputs.make_inputs(M, d_in, d_out, r, "identity", seed=10)
     t = {k: G.dev(v) for k, v in inp.items()}
     ones = torch.full((M, d_in // 8), 0xFF, dtype=torch.uint8, device="cuda")
