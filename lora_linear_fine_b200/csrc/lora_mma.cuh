@@ -292,20 +292,19 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         m0 = mt * C::kTileM + 128 * static_cast<int>(crank);
         n0 = nt * C::kOutCols;
       };
-      // Block blk (main K-blocks first, then the LoRA blocks) of the tile at
-      // (m0, n0) into the next ring stage; false if the wait for the stage
-      // gave up.
-      auto put = [&](int m0, int n0, int blk) -> bool {
+      // The blocks of the tile at (m0, n0), each into the next ring stage:
+      // the main K-blocks (projection j, columns [k0, k0 + 64) of K), then
+      // the LoRA blocks; false if the wait for the stage gave up.  Main and
+      // LoRA blocks go through separate functions that the tile loops call
+      // in order, so that the per-block path (which sets the pace of the
+      // whole pipeline) carries no branch or division between the two kinds.
+      auto put_main = [&](int m0, int n0, int j, int k0) -> bool {
         if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) return false;
         uint8_t* sa = smem + rp.stage * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
         const uint32_t fb = rp.stage;
-        const bool lora_blk = blk >= C::kKPairs * nkb;
-        if (leader) mbar_arrive_expect_tx(&full[rp.stage], (C::kSwigluFwd && lora_blk) ? kTxSwigluLora : kTxFull);
-        if (!lora_blk) {
-          // main block: projection j, K-block kb
-          const int j = blk / nkb;
-          const int k0 = (blk - j * nkb) * 64;
+        if (leader) mbar_arrive_expect_tx(&full[rp.stage], kTxFull);
+        {
           load(sa, &p.tm_a[j], fb, k0, m0, pol_stream);
           if constexpr (!kBwd) {
             if constexpr (C::kSwigluFwd) {
@@ -325,10 +324,20 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             // W^T (K-major copy of W made by the backward): rows = outputs of dX
             load(sb, &p.tm_w[j], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
           }
-        } else {
-          // LoRA block of projection j: s*T_j (s*U_j) rows and B_j (A_j) rows,
-          // K = r columns [kx, kx + 64) of the rank, zero-filled past r
-          const int lb = blk - C::kKPairs * nkb;
+        }
+        ++issued;
+        rp.next(S);
+        return true;
+      };
+      auto put_lora = [&](int m0, int n0, int lb) -> bool {
+        if (!wait_bar<kPair>(&empty[rp.stage], rp.phase ^ 1u, ctl)) return false;
+        uint8_t* sa = smem + rp.stage * C::kStageBytes;
+        uint8_t* sb = sa + C::kABytes;
+        const uint32_t fb = rp.stage;
+        if (leader) mbar_arrive_expect_tx(&full[rp.stage], C::kSwigluFwd ? kTxSwigluLora : kTxFull);
+        {
+          // LoRA block lb, of projection j: s*T_j (s*U_j) rows and B_j (A_j)
+          // rows, K = r columns [kx, kx + 64) of the rank, zero-filled past r
           const int j = lb / lkb;
           const int kx = (lb - j * lkb) * 64;
           load(sa, &p.tm_la[j], fb, kx, m0, pol_keep);
@@ -391,13 +400,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         for (int t = unit; t < p.num_tiles && ok; t += nunits) {
           origin(t, m0, n0);
           if (t == unit)
-            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m0, n0, nmain + lb);
-          for (int blk = 0; blk < h && ok; ++blk) ok = put(m0, n0, blk);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put_lora(m0, n0, lb);
+          for (int blk = 0; blk < h && ok; ++blk) ok = put_main(m0, n0, 0, blk * 64);
           if (t + nunits < p.num_tiles) {
             origin(t + nunits, m1, n1);
-            for (int lb = 0; lb < nlora && ok; ++lb) ok = put(m1, n1, nmain + lb);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put_lora(m1, n1, lb);
           }
-          for (int blk = h; blk < nmain && ok; ++blk) ok = put(m0, n0, blk);
+          for (int blk = h; blk < nmain && ok; ++blk) ok = put_main(m0, n0, 0, blk * 64);
         }
       } else {
         int m0, n0;
@@ -409,14 +418,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             } else {
               // the row block's T tile publishes bf16(s T): wait for this
               // CTA's four flag bits before the LoRA block loads it
-              for (int blk = 0; blk < nmain && ok; ++blk) ok = put(m0, n0, blk);
+              for (int kb = 0; kb < nkb && ok; ++kb) ok = put_main(m0, n0, 0, kb * 64);
               const int bit = ((m0 - 128 * static_cast<int>(crank)) / C::kTileM * C::kCtas + static_cast<int>(crank)) * 4;
               if (ok) ok = flag_wait_all(p.t_flags + 1 + bit / 32, 0xFu << (bit % 32), ctl);
               fence_proxy_async_global();
-              for (int blk = nmain; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
+              for (int lb = 0; lb < nlora && ok; ++lb) ok = put_lora(m0, n0, lb);
             }
           } else {
-            for (int blk = 0; blk < nmain + nlora && ok; ++blk) ok = put(m0, n0, blk);
+            for (int j = 0; j < C::kKPairs && ok; ++j)
+              for (int kb = 0; kb < nkb && ok; ++kb) ok = put_main(m0, n0, j, kb * 64);
+            for (int lb = 0; lb < nlora && ok; ++lb) ok = put_lora(m0, n0, lb);
           }
         }
       }
