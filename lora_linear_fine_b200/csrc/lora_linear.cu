@@ -659,9 +659,14 @@ bool shared_t_enabled() {
 }
 
 template <bool kPair, bool kBwd, int kNPair, int kEpi>
-lora_status_t launch_mma(const MmaParams& p, int sms, cudaStream_t st) {
+lora_status_t launch_mma(const MmaParams& p0, int sms, cudaStream_t st) {
   using C = MmaCfg<kPair, kBwd, kNPair, kEpi>;
   auto k = lora_mma_kernel<kPair, kBwd, kNPair, kEpi>;
+  MmaParams p = p0;
+  if constexpr (C::kTmaOut) {
+    // the epilogue's TMA stores: bf16 out [M x N], boxes of 64 columns x 32 rows
+    if (p.out == nullptr || !make_tm(&p.tm_out, p.out, p.N, p.M, p.N, 64, 32)) return LORA_ERR_CUDA;
+  }
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return cuda_error("cudaFuncSetAttribute(mma)");
   const int max_units = kPair ? sms / 2 : sms;

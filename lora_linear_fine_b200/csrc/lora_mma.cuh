@@ -108,6 +108,7 @@ struct MmaParams {
   // tiles load it from there (tm_la[0]) for their LoRA block once the
   // publishing CTA's flag bits are set.
   CUtensorMap tm_am;      // A [r x K], box 64 x am_rows (this CTA's am_rows rows of the padded rank)
+  CUtensorMap tm_out;     // bf16 out [M x N], box 64 x 32 (set by the launcher for the TMA-store epilogue)
   int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
   int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
   int r;                  // the rank
@@ -145,7 +146,14 @@ struct MmaCfg {
   // Dropout on the adapter input (backward, one projection): the masked
   // LoRA term is formed in the accumulator before the main K-loop.
   static constexpr bool kDropEpi = kEpi == kMEpiGradDrop || kEpi == kMEpiGradF16Drop;
-  static constexpr int kEpiStageBytes = kStaged ? 8 * 4096 : 0;
+  // The bf16 epilogues without their own output path (identity forward,
+  // dX) stage each warp's rows in shared memory as well and write them with
+  // TMA stores: per-thread 16-byte stores scattered over 32 rows slowed the
+  // loads that feed the tensor core by 1.3-1.8k cycles per tile.
+  static constexpr bool kTmaOut = !(kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiRope || kEpi == kMEpiGradF32 ||
+                                    kEpi == kMEpiGradF16F32 || kEpi == kMEpiCeFwd || kEpi == kMEpiCeFwdZ ||
+                                    kEpi == kMEpiCeGrad);
+  static constexpr int kEpiStageBytes = (kStaged || kTmaOut) ? 8 * 4096 : 0;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / (kStageBytes + kAMBytes);
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kAMOff = kStages * kStageBytes;              // the A-rows ring
@@ -995,19 +1003,53 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         for (int c = 0; c < 4; ++c) tmem_ld32(tl + h * 128 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
         tmem_wait_ld();
         release_acc();
-        if (!row_ok) continue;
         const int col0 = nt * 256 + h * 128;
-        const size_t base = static_cast<size_t>(row) * p.N + col0;
+        if constexpr (C::kTmaOut) {
+          // This warp's 32 rows x 128 columns leave as two 64-column boxes:
+          // packed to bf16 in its 4 KB slot of shared memory (row r at 128 r
+          // bytes, 16-byte chunk j at position j ^ (r & 7): the 128-byte
+          // swizzle the tensor map expects), then one TMA store per box,
+          // clipped at the tensor's last row and column.
+          uint4* stg = reinterpret_cast<uint4*>(epi_stage + ew * 4096);
+          const int row0 = row - lane;
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
-          uint4 pk;
-          pk.x = pack_bf16x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
-          pk.y = pack_bf16x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-          pk.z = pack_bf16x2(__uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
-          pk.w = pack_bf16x2(__uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
-          if (col0 + c < p.N) st_global_v4_hint(p.out + base + c, pk, pol_out);
+          for (int k = 0; k < 2; ++k) {
+            if (lane == 0) bulk_wait_read_all();   // the slot's previous box has been read out
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = 64 * k + 8 * j;
+              uint4 pk;
+              pk.x = pack_bf16x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+              pk.y = pack_bf16x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+              pk.z = pack_bf16x2(__uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+              pk.w = pack_bf16x2(__uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
+              stg[lane * 8 + (j ^ (lane & 7))] = pk;
+            }
+            fence_proxy_async_smem();              // the TMA engine reads the slot through the async proxy
+            __syncwarp();
+            if (lane == 0 && row0 < p.M && col0 + 64 * k < p.N) {
+              tma_store_2d_hint(&p.tm_out, stg, col0 + 64 * k, row0, pol_out);
+              bulk_commit_group();
+            }
+          }
+        } else {
+          if (!row_ok) continue;
+          const size_t base = static_cast<size_t>(row) * p.N + col0;
+#pragma unroll
+          for (int c = 0; c < 128; c += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+            pk.y = pack_bf16x2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+            pk.z = pack_bf16x2(__uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+            pk.w = pack_bf16x2(__uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
+            if (col0 + c < p.N) st_global_v4_hint(p.out + base + c, pk, pol_out);
+          }
         }
       }
+    }
+    if constexpr (C::kTmaOut) {
+      if (lane == 0) bulk_wait_all();   // this warp's stores are complete before the CTA exits
     }
   }
 

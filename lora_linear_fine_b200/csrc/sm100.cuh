@@ -219,6 +219,23 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// TMA tiled store of one box from this CTA's shared memory to global memory,
+// tracked in the thread's bulk async-group (commit, then wait).  Coordinates
+// are non-negative; the tensor map's bounds clip a box that runs past the
+// tensor's last row or column.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* tm, const void* src, int32_t x, int32_t y,
+                                                  uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(tm),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The thread's committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // The same between generic-proxy global accesses and TMA (async-proxy)
 // accesses of global memory: a CTA that publishes data with plain stores for
 // another CTA's TMA loads fences after its stores, and the reader fences
