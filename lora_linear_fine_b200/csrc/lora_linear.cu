@@ -115,6 +115,22 @@ bool make_tm(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, u
   return r == CUDA_SUCCESS;
 }
 
+// fp32 [outer x inner] row-major (rows row_elems elements apart), 128-byte
+// swizzle: the target of the fp32 logits' TMA stores (box 32 x box_outer).
+bool make_tm_f32(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_elems,
+                 uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_elems * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) LORA_LOG("cuTensorMapEncodeTiled (fp32) failed (%d): inner=%llu outer=%llu", (int)r,
+                                  (unsigned long long)inner, (unsigned long long)outer);
+  return r == CUDA_SUCCESS;
+}
+
 // 3D bf16 view [K blocks][rows][64] of a row-major [rows x 64 nkb] matrix
 // (rows row_elems elements apart), 128-byte swizzle: box 64 x box_rows x
 // box_kb lands in shared memory as box_kb consecutive [box_rows x 64] tiles.
@@ -666,6 +682,10 @@ lora_status_t launch_mma(const MmaParams& p0, int sms, cudaStream_t st) {
   if constexpr (C::kTmaOut) {
     // the epilogue's TMA stores: bf16 out [M x N], boxes of 64 columns x 32 rows
     if (p.out == nullptr || !make_tm(&p.tm_out, p.out, p.N, p.M, p.N, 64, 32)) return LORA_ERR_CUDA;
+  }
+  if constexpr (C::kTmaZ) {
+    // the fp32 logits' TMA stores: out_f32 [M x N], boxes of 32 columns x 32 rows
+    if (p.out_f32 == nullptr || !make_tm_f32(&p.tm_out, p.out_f32, p.N, p.M, p.N, 32, 32)) return LORA_ERR_CUDA;
   }
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return cuda_error("cudaFuncSetAttribute(mma)");

@@ -108,7 +108,8 @@ struct MmaParams {
   // tiles load it from there (tm_la[0]) for their LoRA block once the
   // publishing CTA's flag bits are set.
   CUtensorMap tm_am;      // A [r x K], box 64 x am_rows (this CTA's am_rows rows of the padded rank)
-  CUtensorMap tm_out;     // bf16 out [M x N], box 64 x 32 (set by the launcher for the TMA-store epilogue)
+  CUtensorMap tm_out;     // set by the launcher for the TMA-store epilogues: bf16 out [M x N], box 64 x 32;
+                          // kMEpiCeFwdZ: fp32 out_f32 [M x N], box 32 x 32
   int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
   int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
   int r;                  // the rank
@@ -153,7 +154,9 @@ struct MmaCfg {
   static constexpr bool kTmaOut = !(kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiRope || kEpi == kMEpiGradF32 ||
                                     kEpi == kMEpiGradF16F32 || kEpi == kMEpiCeFwd || kEpi == kMEpiCeFwdZ ||
                                     kEpi == kMEpiCeGrad);
-  static constexpr int kEpiStageBytes = (kStaged || kTmaOut) ? 8 * 4096 : 0;
+  // The fp32 logits of kMEpiCeFwdZ leave the same way.
+  static constexpr bool kTmaZ = kEpi == kMEpiCeFwdZ;
+  static constexpr int kEpiStageBytes = (kStaged || kTmaOut || kTmaZ) ? 8 * 4096 : 0;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / (kStageBytes + kAMBytes);
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kAMOff = kStages * kStageBytes;              // the A-rows ring
@@ -937,12 +940,21 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           if (c == 3) release_acc();
           const int cb = col0 + 32 * c;
           if constexpr (kEpi == kMEpiCeFwdZ) {
-            if (row_ok) {
-              float* zr = p.out_f32 + static_cast<size_t>(row) * p.N + cb;
+            // the warp's 32 rows x 32 columns of fp32 logits: into its 4 KB
+            // slot (row r at 128 r bytes, 16-byte chunk j at j ^ (r & 7)),
+            // then one TMA store, clipped at the last row and column
+            uint4* stg = reinterpret_cast<uint4*>(epi_stage + ew * 4096);
+            const int row0 = row - lane;
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
 #pragma unroll
-              for (int i = 0; i < 32; i += 4)      // N is a multiple of 8: a float4 is wholly in or past N
-                if (cb + i < p.N)
-                  st_global_v4_hint(zr + i, make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]), pol_out);
+            for (int j = 0; j < 8; ++j)
+              stg[lane * 8 + (j ^ (lane & 7))] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && row0 < p.M && cb < p.N) {
+              tma_store_2d_hint(&p.tm_out, stg, cb, row0, pol_out);
+              bulk_commit_group();
             }
           }
           float cm = -INFINITY;
@@ -1048,7 +1060,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         }
       }
     }
-    if constexpr (C::kTmaOut) {
+    if constexpr (C::kTmaOut || C::kTmaZ) {
       if (lane == 0) bulk_wait_all();   // this warp's stores are complete before the CTA exits
     }
   }
