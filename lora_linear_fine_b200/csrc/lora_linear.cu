@@ -101,14 +101,15 @@ lora_status_t device_info(DevInfo* out) {
 // 2D bf16 tensor map with 128-byte swizzle: `inner` contiguous elements per
 // row, `outer` rows `row_elems` elements apart; box = box_inner x box_outer.
 bool make_tm(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_elems,
-             uint32_t box_inner, uint32_t box_outer, bool f16 = false) {
+             uint32_t box_inner, uint32_t box_outer, bool f16 = false,
+             CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_elems * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   const CUtensorMapDataType dt = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUresult r = g_encode(tm, dt, 2, const_cast<void*>(ptr), dims, strides, box,
-                              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) LORA_LOG("cuTensorMapEncodeTiled failed (%d): inner=%llu outer=%llu box=%ux%u", (int)r,
                                   (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
@@ -682,6 +683,11 @@ lora_status_t launch_mma(const MmaParams& p0, int sms, cudaStream_t st) {
   if constexpr (C::kTmaOut) {
     // the epilogue's TMA stores: bf16 out [M x N], boxes of 64 columns x 32 rows
     if (p.out == nullptr || !make_tm(&p.tm_out, p.out, p.N, p.M, p.N, 64, 32)) return LORA_ERR_CUDA;
+  }
+  if constexpr (C::kTmaRope) {
+    // the rotated output's TMA stores: bf16 out [M x N], boxes of 32 columns x 32 rows, 64-byte swizzle
+    if (p.out == nullptr || !make_tm(&p.tm_out, p.out, p.N, p.M, p.N, 32, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
+      return LORA_ERR_CUDA;
   }
   if constexpr (C::kTmaZ) {
     // the fp32 logits' TMA stores: out_f32 [M x N], boxes of 32 columns x 32 rows

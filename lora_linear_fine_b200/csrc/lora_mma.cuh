@@ -109,7 +109,8 @@ struct MmaParams {
   // publishing CTA's flag bits are set.
   CUtensorMap tm_am;      // A [r x K], box 64 x am_rows (this CTA's am_rows rows of the padded rank)
   CUtensorMap tm_out;     // set by the launcher for the TMA-store epilogues: bf16 out [M x N], box 64 x 32;
-                          // kMEpiCeFwdZ: fp32 out_f32 [M x N], box 32 x 32
+                          // kMEpiCeFwdZ: fp32 out_f32 [M x N], box 32 x 32;
+                          // kMEpiRope: bf16 out [M x N], box 32 x 32, 64-byte swizzle
   int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
   int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
   int r;                  // the rank
@@ -156,7 +157,9 @@ struct MmaCfg {
                                     kEpi == kMEpiCeGrad);
   // The fp32 logits of kMEpiCeFwdZ leave the same way.
   static constexpr bool kTmaZ = kEpi == kMEpiCeFwdZ;
-  static constexpr int kEpiStageBytes = (kStaged || kTmaOut || kTmaZ) ? 8 * 4096 : 0;
+  // ... and the rotated bf16 output of kMEpiRope, in 32-column boxes.
+  static constexpr bool kTmaRope = kEpi == kMEpiRope;
+  static constexpr int kEpiStageBytes = (kStaged || kTmaOut || kTmaZ || kTmaRope) ? 8 * 4096 : 0;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / (kStageBytes + kAMBytes);
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
   static constexpr int kAMOff = kStages * kStageBytes;              // the A-rows ring
@@ -841,32 +844,49 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         if (row_ok && !turn && p.status) atomicOr(p.status, kStatusBadArgument);   // left unturned
         const size_t trow = static_cast<size_t>(turn ? pr : 0) * half;
         const int col0 = nt * 256 + h * 128;
-        const size_t base = static_cast<size_t>(row) * p.N + col0;
+        // Each 32-column group leaves as one box: packed to bf16 in half
+        // `part` of the warp's 4 KB slot (row r at 64 r bytes, 16-byte chunk
+        // j at position j ^ ((r >> 1) & 3): the 64-byte swizzle of the
+        // tensor map), then one TMA store, clipped at the last row and
+        // column.  Rows past M carry zeros (their inputs were zero-filled)
+        // and are clipped.
+        uint4* stg = reinterpret_cast<uint4*>(epi_stage + ew * 4096);
+        const int row0 = row - lane;
 #pragma unroll
         for (int hv = 0; hv < 2; ++hv) {
           const int c0 = half == 64 ? 32 * hv : 64 * hv;
           uint32_t u[64];
-          __syncwarp();   // lanes past M skipped the stores of the previous pass; tcgen05.ld is .sync.aligned
+          __syncwarp();   // tcgen05.ld is .sync.aligned
           tmem_ld32(tl + h * 128 + c0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
           tmem_ld32(tl + h * 128 + c0 + half, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tmem_wait_ld();
           if (hv == 1) release_acc();
-          if (!row_ok) continue;
           const int toff = c0 % half;
           if (turn) rope_rotate32(u, p.rope.cos + trow + toff, p.rope.sin + trow + toff);
+          if (lane == 0) bulk_wait_read_all();   // both halves of the slot have been read out
+          __syncwarp();
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
-            const int cc = c0 + part * half;
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              const uint32_t* w = &u[32 * part + j];
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t* w = &u[32 * part + 8 * j];
               uint4 pk;
               pk.x = pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1]));
               pk.y = pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3]));
               pk.z = pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5]));
               pk.w = pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7]));
-              if (col0 + cc + j < p.N) st_global_v4_hint(p.out + base + cc + j, pk, pol_out);
+              stg[part * 128 + lane * 4 + (j ^ ((lane >> 1) & 3))] = pk;
             }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.M) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+              const int cc = col0 + c0 + part * half;
+              if (cc < p.N) tma_store_2d_hint(&p.tm_out, stg + part * 128, cc, row0, pol_out);
+            }
+            bulk_commit_group();
           }
         }
       } else if constexpr (kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32) {
@@ -1060,7 +1080,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         }
       }
     }
-    if constexpr (C::kTmaOut || C::kTmaZ) {
+    if constexpr (C::kTmaOut || C::kTmaZ || C::kTmaRope) {
       if (lane == 0) bulk_wait_all();   // this warp's stores are complete before the CTA exits
     }
   }
