@@ -109,7 +109,7 @@ struct MmaParams {
   // publishing CTA's flag bits are set.
   CUtensorMap tm_am;      // A [r x K], box 64 x am_rows (this CTA's am_rows rows of the padded rank)
   CUtensorMap tm_out;     // set by the launcher for the TMA-store epilogues: bf16 out [M x N], box 64 x 32;
-                          // kMEpiCeFwdZ: fp32 out_f32 [M x N], box 32 x 32;
+                          // kMEpiCeFwdZ, kMEpiGradF32, kMEpiGradF16F32: fp32 out_f32 [M x N], box 32 x 32;
                           // kMEpiRope: bf16 out [M x N], box 32 x 32, 64-byte swizzle
   int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
   int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
@@ -155,8 +155,9 @@ struct MmaCfg {
   static constexpr bool kTmaOut = !(kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiRope || kEpi == kMEpiGradF32 ||
                                     kEpi == kMEpiGradF16F32 || kEpi == kMEpiCeFwd || kEpi == kMEpiCeFwdZ ||
                                     kEpi == kMEpiCeGrad);
-  // The fp32 logits of kMEpiCeFwdZ leave the same way.
-  static constexpr bool kTmaZ = kEpi == kMEpiCeFwdZ;
+  // The fp32 logits of kMEpiCeFwdZ and the fp32 dX of kMEpiGradF32 /
+  // kMEpiGradF16F32 (stored, or added at L2 with out_acc) leave the same way.
+  static constexpr bool kTmaZ = kEpi == kMEpiCeFwdZ || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
   // ... and the rotated bf16 output of kMEpiRope, in 32-column boxes.
   static constexpr bool kTmaRope = kEpi == kMEpiRope;
   static constexpr int kEpiStageBytes = (kStaged || kTmaOut || kTmaZ || kTmaRope) ? 8 * 4096 : 0;
@@ -892,9 +893,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       } else if constexpr (kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32) {
         // fp32 dX, written or added to (several projections' input gradients
         // summed in a fixed order, one launch after another).  Each 32-column
-        // chunk of the warp's 32 rows goes through shared memory (4 KB per
-        // warp, 16-byte chunk j of row rr at j ^ (rr & 7)) and out row by
-        // row: 8 lanes cover 128 contiguous bytes of one row.
+        // chunk of the warp's 32 rows goes into its 4 KB slot of shared
+        // memory (16-byte chunk j of row rr at j ^ (rr & 7), the 128-byte
+        // swizzle of the fp32 tensor map) and leaves as one TMA store, or
+        // with out_acc one TMA reduce-add (the addition done at L2, one per
+        // element and launch), clipped at the last row and column.
         const int row0 = row - lane;                 // first row of this warp's 32
         float4* stg = reinterpret_cast<float4*>(epi_stage + ew * 4096);
         const int col0 = nt * 256 + h * 128;
@@ -905,41 +908,20 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
           tmem_ld32(tl + h * 128 + 32 * c, v);
           tmem_wait_ld();
           if (c == 3) release_acc();
+          if (lane == 0) bulk_wait_read_all();       // the slot's previous box has been read out
+          __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             stg[lane * 8 + (j ^ (lane & 7))] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                                            __uint_as_float(v[4 * j + 2]),
                                                            __uint_as_float(v[4 * j + 3]));
+          fence_proxy_async_smem();
           __syncwarp();
-          const int j = lane & 7;
-          const int col = col0 + 32 * c + 4 * j;
-          float4 a[8];
-          if (p.out_acc) {
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int grow = row0 + it * 4 + (lane >> 3);
-              a[it] = (grow < p.M && col < p.N)
-                          ? *reinterpret_cast<const float4*>(p.out_f32 + static_cast<size_t>(grow) * p.N + col)
-                          : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            }
-          }
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rr = it * 4 + (lane >> 3);
-            const int grow = row0 + rr;
-            if (grow < p.M && col < p.N) {
-              float4 o = stg[rr * 8 + (j ^ (rr & 7))];
-              if (p.out_acc) {
-                o.x += a[it].x;
-                o.y += a[it].y;
-                o.z += a[it].z;
-                o.w += a[it].w;
-              }
-              st_global_v4_hint(p.out_f32 + static_cast<size_t>(grow) * p.N + col,
-                                make_uint4(__float_as_uint(o.x), __float_as_uint(o.y), __float_as_uint(o.z),
-                                           __float_as_uint(o.w)),
-                                pol_out);
-            }
+          const int cb = col0 + 32 * c;
+          if (lane == 0 && row0 < p.M && cb < p.N) {
+            if (p.out_acc) tma_reduce_add_2d_hint(&p.tm_out, stg, cb, row0, pol_out);
+            else tma_store_2d_hint(&p.tm_out, stg, cb, row0, pol_out);
+            bulk_commit_group();
           }
         }
       } else if constexpr (kEpi == kMEpiCeFwd || kEpi == kMEpiCeFwdZ) {

@@ -230,6 +230,15 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* tm, const v
       "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
+// The same box added element by element to what global memory holds (the
+// addition is done at L2; fp32 tensor maps).
+__device__ __forceinline__ void tma_reduce_add_2d_hint(const CUtensorMap* tm, const void* src, int32_t x, int32_t y,
+                                                       uint64_t policy) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;"
+      ::"l"(tm), "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // The thread's committed bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
