@@ -689,6 +689,16 @@ lora_status_t launch_mma(const MmaParams& p0, int sms, cudaStream_t st) {
     if (p.out == nullptr || !make_tm(&p.tm_out, p.out, p.N, p.M, p.N, 32, 32, false, CU_TENSOR_MAP_SWIZZLE_64B))
       return LORA_ERR_CUDA;
   }
+  if constexpr (C::kTmaAct) {
+    // the SiLU / SwiGLU forward's TMA stores: bf16 Y (boxes of 64 columns x
+    // 32 rows) and, when saved, fp32 Z (32 x 32; SwiGLU: gate, then up)
+    if (p.out == nullptr || !make_tm(&p.tm_out, p.out, p.N, p.M, p.N, 64, 32)) return LORA_ERR_CUDA;
+    if (p.z_save != nullptr) {
+      for (int j = 0; j < (C::kSwigluFwd ? 2 : 1); ++j)
+        if (!make_tm_f32(&p.tm_z[j], p.z_save + static_cast<size_t>(j) * p.M * p.N, p.N, p.M, p.N, 32, 32))
+          return LORA_ERR_CUDA;
+    }
+  }
   if constexpr (C::kTmaZ) {
     // the fp32 logits' TMA stores: out_f32 [M x N], boxes of 32 columns x 32 rows
     if (p.out_f32 == nullptr || !make_tm_f32(&p.tm_out, p.out_f32, p.N, p.M, p.N, 32, 32)) return LORA_ERR_CUDA;

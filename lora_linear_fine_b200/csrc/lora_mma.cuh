@@ -111,6 +111,7 @@ struct MmaParams {
   CUtensorMap tm_out;     // set by the launcher for the TMA-store epilogues: bf16 out [M x N], box 64 x 32;
                           // kMEpiCeFwdZ, kMEpiGradF32, kMEpiGradF16F32: fp32 out_f32 [M x N], box 32 x 32;
                           // kMEpiRope: bf16 out [M x N], box 32 x 32, 64-byte swizzle
+  CUtensorMap tm_z[2];    // SiLU / SwiGLU forward with z_save: fp32 Z (SwiGLU: gate, up) [M x N], box 32 x 32
   int am_rows;            // rows of A per CTA: RP / (CTAs per unit)
   int rp;                 // the rank padded to a multiple of 16 (the T MMA's N)
   int r;                  // the rank
@@ -160,6 +161,8 @@ struct MmaCfg {
   static constexpr bool kTmaZ = kEpi == kMEpiCeFwdZ || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
   // ... and the rotated bf16 output of kMEpiRope, in 32-column boxes.
   static constexpr bool kTmaRope = kEpi == kMEpiRope;
+  // ... and the SiLU / SwiGLU forward's bf16 Y and fp32 Z.
+  static constexpr bool kTmaAct = kSwigluFwd || (kEpi == kMEpiSilu && !kBwd);
   static constexpr int kEpiStageBytes = (kStaged || kTmaOut || kTmaZ || kTmaRope) ? 8 * 4096 : 0;
   static constexpr int kStages0 = (kSmemLimitBytes - 2048 - kEpiStageBytes) / (kStageBytes + kAMBytes);
   static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
@@ -734,21 +737,24 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
       if constexpr (C::kSwigluFwd || kEpi == kMEpiSilu) {
         // Two halves of this thread's columns (SiLU: 64 + 64 of its 128;
         // SwiGLU: 32 + 32 gate columns with their up columns), so that only 64
-        // accumulator values are live at a time.  Rows go out through shared
-        // memory, 32 rows x 8 uint4 per flush, then row-contiguous: 8 lanes
-        // cover 128 bytes of a row.
+        // accumulator values are live at a time.  Each flush is one box of the
+        // warp's 32 rows x 128 bytes (32 fp32 Z or 64 bf16 Y columns): into
+        // its 4 KB slot of shared memory (16-byte chunk j of row r at
+        // j ^ (r & 7)), then one TMA store at column x, clipped at the last
+        // row and column.
         const int row0 = row - lane;                 // first row of this warp's 32
         uint4* stg = reinterpret_cast<uint4*>(epi_stage + ew * 4096);
-        auto flush = [&](const uint4 (&mine)[8], auto&& store) {
+        auto flush = [&](const uint4 (&mine)[8], const CUtensorMap* tm, int x) {
+          if (lane == 0) bulk_wait_read_all();       // the slot's previous box has been read out
+          __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j) stg[lane * 8 + (j ^ (lane & 7))] = mine[j];
+          fence_proxy_async_smem();
           __syncwarp();
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rr = it * 4 + (lane >> 3), j = lane & 7;
-            if (row0 + rr < p.M) store(row0 + rr, j, stg[rr * 8 + (j ^ (rr & 7))]);
+          if (lane == 0 && row0 < p.M && x < p.N) {
+            tma_store_2d_hint(tm, stg, x, row0, pol_out);
+            bulk_commit_group();
           }
-          __syncwarp();
         };
         const int col0 = C::kSwigluFwd ? nt * 128 + h * 64 : nt * 256 + h * 128;
         uint32_t ylo[16];                            // SwiGLU: packed bf16 Y of the first half
@@ -768,7 +774,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             // fp32 Z, 32 columns per flush: SwiGLU gate then up; SiLU two column runs
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
-              float* zdst = p.z_save + (C::kSwigluFwd ? static_cast<size_t>(part) * p.M * p.N : 0);
               const int zc0 = C::kSwigluFwd ? col0 + 32 * hv : col0 + 64 * hv + 32 * part;
               uint4 mine[8];
 #pragma unroll
@@ -776,10 +781,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
                 const int c = part * 32 + 4 * j;
                 mine[j] = make_uint4(v[c], v[c + 1], v[c + 2], v[c + 3]);
               }
-              flush(mine, [&](int grow, int j, uint4 val) {
-                const int col = zc0 + 4 * j;
-                if (col < p.N) st_global_v4_hint(zdst + static_cast<size_t>(grow) * p.N + col, val, pol_out);
-              });
+              flush(mine, &p.tm_z[C::kSwigluFwd ? part : 0], zc0);
             }
           }
           if constexpr (C::kSwigluFwd) {
@@ -806,10 +808,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
                 mine[j] = make_uint4(ylo[4 * j], ylo[4 * j + 1], ylo[4 * j + 2], ylo[4 * j + 3]);
                 mine[4 + j] = make_uint4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
               }
-              flush(mine, [&](int grow, int j, uint4 val) {
-                const int col = col0 + 8 * j;
-                if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
-              });
+              flush(mine, &p.tm_out, col0);
             }
           } else {
             // bf16 Y = SiLU(z): 64 columns per half, one flush
@@ -827,10 +826,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
               mine[j].z = pack_bf16x2(yv[4], yv[5]);
               mine[j].w = pack_bf16x2(yv[6], yv[7]);
             }
-            flush(mine, [&](int grow, int j, uint4 val) {
-              const int col = col0 + 64 * hv + 8 * j;
-              if (col < p.N) st_global_v4_hint(p.out + static_cast<size_t>(grow) * p.N + col, val, pol_out);
-            });
+            flush(mine, &p.tm_out, col0 + 64 * hv);
           }
         }
       } else if constexpr (kEpi == kMEpiRope) {
@@ -1062,7 +1058,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
         }
       }
     }
-    if constexpr (C::kTmaOut || C::kTmaZ || C::kTmaRope) {
+    if constexpr (C::kTmaOut || C::kTmaZ || C::kTmaRope || C::kTmaAct) {
       if (lane == 0) bulk_wait_all();   // this warp's stores are complete before the CTA exits
     }
   }
