@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(32 * kNormWarps)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const double inv = 1.0 / sqrt(ss / static_cast<double>(d) + eps);
-    if (lane == 0) rstd[row] = static_cast<float>(inv);
+    const float inv32 = static_cast<float>(inv);
+    if (lane == 0) rstd[row] = inv32;
     uint4* yr = reinterpret_cast<uint4*>(Xn + row * d);
     for (int c = lane; c < nv; c += 32) {
       float f[8], w[8];
@@ -93,7 +94,22 @@ __global__ void __launch_bounds__(32 * kNormWarps)
       unpack_bf16x8(__ldg(gv + c), w);
       __align__(16) __nv_bfloat16 o[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = bf16_from_f64((static_cast<double>(f[e]) * inv) * static_cast<double>(w[e]));
+      for (int e = 0; e < 8; ++e) {
+        // The value to round is y = (x * inv) * g in fp64.  In fp32 (inv
+        // rounded to fp32, two products) it is off by at most 3 units in the
+        // last place of fp32 (each of the three roundings adds at most half
+        // an ulp, relative 2^-24, and an ulp is at least 2^-24 of |y|).  So
+        // unless its 16 bits below bf16 precision lie within 16 ulps of
+        // 0x8000 (a bf16 rounding midpoint), the fp32 value rounds to the
+        // same bf16 as y.  Zero, subnormal and non-finite fp32 values and
+        // the near-midpoint ones take the fp64 path.
+        const float y = (f[e] * inv32) * w[e];
+        const uint32_t b = __float_as_uint(y);
+        const uint32_t ex = (b >> 23) & 0xFFu;
+        const int low = static_cast<int>(b & 0xFFFFu) - 0x8000;
+        if (ex != 0u && ex != 0xFFu && (low > 16 || low < -16)) o[e] = __float2bfloat16_rn(y);
+        else o[e] = bf16_from_f64((static_cast<double>(f[e]) * inv) * static_cast<double>(w[e]));
+      }
       yr[c] = *reinterpret_cast<const uint4*>(o);
     }
   }
