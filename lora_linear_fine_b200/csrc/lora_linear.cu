@@ -31,7 +31,6 @@ using namespace lora;
 
 constexpr int kAbiVersion = 1;
 constexpr int kTargetCtas = 148;   // SM count of a B200; sets split-K widths
-constexpr int64_t kKMajorMinTokens = 12288;   // dX from a W^T copy at and above this many tokens
 // Workspace header, zero at rest: the status block (word 0 is the status
 // word; words kTFlagWord0 .. kTFlagWord0 + kTFlagWords are the shared-T
 // forward GEMM's exit count and flag bits, which that kernel sets and
@@ -200,11 +199,11 @@ struct Plan {
   size_t tt_hi[2] = {}, tt_lo[2] = {};       // (s*T)^T hi / lo [r x M8] (bwd, dB)
   size_t ut_hi[2] = {}, ut_lo[2] = {};       // (s*U)^T hi / lo [r x M8] (bwd, dA)
   size_t dz_hi[2] = {}, dz_lo[2] = {};     // activation backward: fp16 dZ operands
-  // dX's N-side operands: K-major copies W^T [d_in x d_out], A^T [d_in x r]
-  // (kmajor), or W read in place MN-major (an fp16 copy with an activation)
-  bool kmajor = false;
+  // dX's N-side operands W and A are read in place, MN-major (with an
+  // activation W as an fp16 copy).  A K-major copy of W paid for itself at
+  // 16384 tokens while the epilogue stored its output per thread; with TMA
+  // stores, reading W in place is faster at every size measured.
   size_t wt[2] = {};
-  size_t at_[2] = {};
   size_t part_t = 0, part_u = 0, part_a = 0, part_b = 0;   // split-K partials
   // backward rank passes on rank2d_kernel: U and dB from one read of dZ
   // (identity, r <= 32), dA over X
@@ -271,11 +270,8 @@ Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = tr
     P.total = off;
     return P;
   }
-  // The W^T copy pays for itself when the dX GEMM is long against one pass
-  // over W: many tokens (measured: M = 16384 gains, M = 8192 does not).
-  P.kmajor = !P.act_f16 && M >= kKMajorMinTokens;
   for (int j = 0; j < P.np; ++j) {
-    if (P.kmajor || P.act_f16) P.wt[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
+    if (P.act_f16) P.wt[j] = take(static_cast<size_t>(d->d_out) * d->d_in * 2);
     if (P.act_f16) {
       P.dz_hi[j] = take(static_cast<size_t>(M) * d->d_out * 2);
       P.dz_lo[j] = take(static_cast<size_t>(M) * d->d_out * 2);
@@ -283,7 +279,6 @@ Plan make_plan(const lora_linear_desc* d, bool backward, bool allow_small_m = tr
   }
   if (r > 0) {
     for (int j = 0; j < P.np; ++j) {
-      if (P.kmajor) P.at_[j] = take(static_cast<size_t>(d->d_in) * r * 2);
       P.bt[j] = take(static_cast<size_t>(r) * d->d_out * 2);
       P.tt_hi[j] = take(static_cast<size_t>(r) * P.M8 * 2);
       P.tt_lo[j] = take(static_cast<size_t>(r) * P.M8 * 2);
@@ -1253,22 +1248,11 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
   auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
 
   // 1. dZ operands.  identity: dZ = dY (bf16, exact).  Otherwise dZ = dY * act'(Z)
-  //    as fp16 hi + lo.  W for the dX product: a K-major copy W^T (kmajor), or
-  //    read in place (an fp16 copy with an activation).
+  //    as fp16 hi + lo.  W for the dX product is read in place (an fp16 copy
+  //    with an activation).
   const void* dZ[2] = {dY, nullptr};
   const void* dZlo[2] = {nullptr, nullptr};
   const void* Wmain[2] = {W, W_up};
-  if (P.kmajor) {
-    const long long tiles = ceil_div(d->d_out, 64) * ceil_div(d->d_in, 64);
-    const int grid = static_cast<int>(tiles < static_cast<long long>(dev.sms) * 8 ? tiles : dev.sms * 8);
-    for (int j = 0; j < np; ++j) {
-      launch_k(transpose_w_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, false,
-               static_cast<const __nv_bfloat16*>(Wp[j]), static_cast<int>(d->d_out), static_cast<int>(d->d_in),
-               static_cast<__nv_bfloat16*>(at(P.wt[j])), status);
-      LORA_TRY(check_launch("transpose_w_kernel"));
-      Wmain[j] = at(P.wt[j]);
-    }
-  }
   if (f16) {
     const long long n = static_cast<long long>(M) * d->d_out;
     const int grid = grid_for(n / 8, 256, dev.sms);
@@ -1299,24 +1283,22 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     }
   }
 
-  // 2. B^T, A^T and (s T)^T hi/lo (from the saved T, or a rank pass recomputing
-  //    T); B^T and (s T)^T in the dZ operand type.
+  // 2. B^T and (s T)^T hi/lo (from the saved T, or a rank pass recomputing
+  //    T), in the dZ operand type.
   if (r > 0) {
     for (int j = 0; j < np; ++j) {
       const float* Tj = T_save ? T_save + static_cast<size_t>(j) * M * r : nullptr;
       // one thread per row and 8-column chunk
-      const long long n = (d->d_out + (P.kmajor ? d->d_in : 0) + (Tj ? M : 0)) * (r / 8);
-      const __nv_bfloat16* Aj = static_cast<const __nv_bfloat16*>(Ap[j]);
-      __nv_bfloat16* Atj = P.kmajor ? static_cast<__nv_bfloat16*>(at(P.at_[j])) : nullptr;
+      const long long n = (d->d_out + (Tj ? M : 0)) * (r / 8);
       if (f16)
         launch_k(bwd_prep_kernel<__half>, dim3(grid_for(n, 256, dev.sms)), dim3(256), 0, st, false,
                  static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
-                 static_cast<__half*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
+                 static_cast<__half*>(at(P.bt[j])), Tj, M, d->s,
                  static_cast<__half*>(at(P.tt_hi[j])), static_cast<__half*>(at(P.tt_lo[j])), M8, status);
       else
         launch_k(bwd_prep_kernel<__nv_bfloat16>, dim3(grid_for(n, 256, dev.sms)), dim3(256), 0, st, false,
                  static_cast<const __nv_bfloat16*>(Bp[j]), static_cast<int>(d->d_out), r,
-                 static_cast<__nv_bfloat16*>(at(P.bt[j])), Aj, static_cast<int>(d->d_in), Atj, Tj, M, d->s,
+                 static_cast<__nv_bfloat16*>(at(P.bt[j])), Tj, M, d->s,
                  static_cast<__nv_bfloat16*>(at(P.tt_hi[j])), static_cast<__nv_bfloat16*>(at(P.tt_lo[j])), M8,
                  status);
       LORA_TRY(check_launch("bwd_prep_kernel"));
@@ -1380,21 +1362,15 @@ static lora_status_t bwd_core(const lora_linear_desc* d, const void* dY, const v
     std::memset(&p, 0, sizeof(p));
     const bool pair = pair_kernel_enabled() && M > 128;
     bool ok = true;
-    const uint32_t brows = pair ? 128 : 256;   // N-side rows per CTA box (K-major)
     for (int j = 0; j < np; ++j) {
       ok = ok && make_tm(&p.tm_a[j], dZ[j], d->d_out, M, d->d_out, 64, 128, f16);
-      if (P.kmajor) {
-        ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_out, d->d_in, d->d_out, 64, brows, f16);
-      } else {
-        ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_in, d->d_out, d->d_in, 64, 64, f16);
-      }
+      ok = ok && make_tm(&p.tm_w[j], Wmain[j], d->d_in, d->d_out, d->d_in, 64, 64, f16);   // MN-major
       if (r > 0) {
         ok = ok && make_tm(&p.tm_la[j], at(P.s16[j]), r, M, r, 64, 128);
-        if (P.kmajor) ok = ok && make_tm(&p.tm_lb[j], at(P.at_[j]), r, d->d_in, r, 64, brows);
-        else ok = ok && make_tm(&p.tm_lb[j], Ap[j], d->d_in, r, d->d_in, 64, 64);
+        ok = ok && make_tm(&p.tm_lb[j], Ap[j], d->d_in, r, d->d_in, 64, 64);
       }
     }
-    p.b_mn = P.kmajor ? 0 : 1;
+    p.b_mn = 1;
     if (!ok) return LORA_ERR_CUDA;
     p.M = M;
     p.N = static_cast<int>(d->d_in);

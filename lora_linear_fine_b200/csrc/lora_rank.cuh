@@ -467,13 +467,11 @@ constexpr float kF16Max = 65504.0f;
 // Backward preparation in one launch, one thread per row of the small
 // operands and 8-column chunk (each thread moves one 16-byte piece of a row;
 // neighbouring threads take neighbouring rows, so the transposed writes are
-// coalesced): B^T ([r x d_out], bf16 or fp16), A^T ([d_in x r], bf16, the
-// K-major N-side operand of the dX LoRA block; skipped when At is null) and
-// the transposed hi/lo split of s*T ([r x ld]) from the forward's fp32 T
-// (skipped when Tsave is null).  r is a multiple of 8.
+// coalesced): B^T ([r x d_out], bf16 or fp16) and the transposed hi/lo split
+// of s*T ([r x ld]) from the forward's fp32 T (skipped when Tsave is null).
+// r is a multiple of 8.
 template <typename T>
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, int r, T* __restrict__ Bt,
-                                const __nv_bfloat16* __restrict__ A, int d_in, __nv_bfloat16* __restrict__ At,
                                 const float* __restrict__ Tsave, int M, float s, T* __restrict__ t_hi,
                                 T* __restrict__ t_lo, int ld, uint32_t* status) {
   grid_dep_wait();
@@ -481,10 +479,9 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, 
   // the transposed stores of neighbouring threads are contiguous.
   const long long nc = r / 8;
   const long long nb = d_out;
-  const long long na = At != nullptr ? d_in : 0;
   const long long nt = Tsave != nullptr ? M : 0;
   bool bad = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < (nb + na + nt) * nc;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < (nb + nt) * nc;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     if (i < nb * nc) {
       const int jd = static_cast<int>(i % nb), c0 = static_cast<int>(i / nb) * 8;
@@ -496,15 +493,8 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ B, int d_out, 
         Bt[static_cast<size_t>(c0 + e) * d_out + jd] = to16<T>(f);
         if (!std::is_same<T, __nv_bfloat16>::value && !(fabsf(f) <= kF16Max)) bad = true;
       }
-    } else if (i < (nb + na) * nc) {
-      const long long k = i - nb * nc;
-      const int di = static_cast<int>(k % na), c0 = static_cast<int>(k / na) * 8;
-      __align__(16) __nv_bfloat16 o[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = A[static_cast<size_t>(c0 + e) * d_in + di];
-      *reinterpret_cast<uint4*>(At + static_cast<size_t>(di) * r + c0) = *reinterpret_cast<const uint4*>(o);
     } else {
-      const long long k = i - (nb + na) * nc;
+      const long long k = i - nb * nc;
       const int m = static_cast<int>(k % nt), c0 = static_cast<int>(k / nt) * 8;
       const float4* tp = reinterpret_cast<const float4*>(Tsave + static_cast<size_t>(m) * r + c0);
       const float4 ta = tp[0], tb = tp[1];
@@ -542,77 +532,6 @@ __global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half
       if (!(fabsf(f) <= kF16Max)) bad = true;
     }
     reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(h);
-  }
-  if (bad && status) atomicOr(status, kStatusF16Range);
-}
-
-// W [rows x cols] bf16 -> Wt [cols x rows] in T (bf16, or fp16: exact for
-// |w| <= 65504, else the status bit), so that the dX product reads W K-major.
-// 64 x 64 tiles through shared memory: each thread loads the same 8 columns of
-// two adjacent rows and packs them pairwise into 32-bit words
-// tile[column][row pair], which makes both the shared-memory writes and the
-// row-contiguous reads conflict-free and every global access 16 bytes.
-// rows and cols are multiples of 8.
-template <typename T>
-__global__ void __launch_bounds__(256) transpose_w_kernel(const __nv_bfloat16* __restrict__ W, int rows, int cols,
-                                                          T* __restrict__ Wt, uint32_t* status) {
-  __shared__ uint32_t tile[64][33];
-  grid_dep_wait();
-  const int tiles_c = (cols + 63) / 64;
-  const long long ntiles = static_cast<long long>((rows + 63) / 64) * tiles_c;
-  bool bad = false;
-  for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
-    const int r0 = static_cast<int>(t / tiles_c) * 64;
-    const int c0 = static_cast<int>(t % tiles_c) * 64;
-    __syncthreads();
-    {
-      const int pr = threadIdx.x & 31;          // row pair
-      const int cv = (threadIdx.x >> 5) * 8;    // 8 columns
-      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
-      const int ra = r0 + 2 * pr;
-      if (c0 + cv < cols) {
-        if (ra < rows) a = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(ra) * cols + c0 + cv);
-        if (ra + 1 < rows) b = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(ra + 1) * cols + c0 + cv);
-      }
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        // columns cv + 2e (low halves) and cv + 2e + 1 (high halves)
-        tile[cv + 2 * e][pr] = (av[e] & 0xffffu) | (bv[e] << 16);
-        tile[cv + 2 * e + 1][pr] = (av[e] >> 16) | (bv[e] & 0xffff0000u);
-      }
-    }
-    __syncthreads();
-    {
-      const int qv = threadIdx.x & 7;           // 8 output elements: input rows r0 + 8 qv ...
-      const int cc0 = threadIdx.x >> 3;         // output rows (input columns) cc0, cc0 + 32
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int cc = cc0 + 32 * h;
-        if (c0 + cc < cols && r0 + 8 * qv < rows) {
-          uint32_t w[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) w[k] = tile[cc][4 * qv + k];
-          uint4 o;
-          if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-            o = make_uint4(w[0], w[1], w[2], w[3]);
-          } else {
-            uint32_t hv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float lo = __uint_as_float(w[k] << 16);
-              const float hi = __uint_as_float(w[k] & 0xffff0000u);
-              if (!(fabsf(lo) <= kF16Max) || !(fabsf(hi) <= kF16Max)) bad = true;
-              const __half2 h2 = __floats2half2_rn(lo, hi);
-              hv[k] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            o = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-          }
-          *reinterpret_cast<uint4*>(Wt + static_cast<size_t>(c0 + cc) * rows + r0 + 8 * qv) = o;
-        }
-      }
-    }
   }
   if (bad && status) atomicOr(status, kStatusF16Range);
 }
