@@ -855,7 +855,13 @@ def run_qkv(args, cfg, L, world, rank, local, dist):
     e2e = job_throughput(F, args.e2e_steps, world, e2e_ms) / 1e12
 
     peaks = read_peaks()
-    f_fwd = sum(2.0 * M * d * n + 2.0 * M * r * n for n in douts)     # the three forward GEMMs per step
+    # the three forward GEMMs per step; each also accumulates T = x_n A^T
+    # (2 M d r) when r <= 64 and M <= 256 x (SMs / 2) (the library's test)
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    t_in = (0 < r <= 64 and -(-M // 256) <= sms // 2 and os.environ.get("LORA_LINEAR_FUSED_T", "1")[:1] != "0"
+            and (os.environ.get("LORA_LINEAR_SHARED_T", "1")[:1] != "0"
+                 or all(-(-M // 256) * -(-n // 256) <= sms // 2 for n in douts)))
+    f_fwd = sum(2.0 * M * d * n + 2.0 * M * r * n + (2.0 * M * d * r if t_in else 0.0) for n in douts)
     f_bwd = sum(2.0 * M * d * n + 2.0 * M * r * d for n in douts)     # the three dX GEMMs per step
     ach_f = f_fwd * args.steps / (gemm_fwd_ms * 1e-3) / 1e12 if gemm_fwd_n else None
     ach_b = f_bwd * args.steps / (gemm_bwd_ms * 1e-3) / 1e12 if gemm_bwd_n else None

@@ -1103,9 +1103,9 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   const void* Ap[2] = {A, A_up};
   const void* Bp[2] = {B, B_up};
   const bool pair = pair_kernel_enabled() && M > 128;
-  // T accumulated inside the forward GEMM (one identity projection, r <= 64,
-  // no dropout, no rotation), so that the separate T pass (and its split-K
-  // reduction) is skipped and X is streamed by the GEMM alone:
+  // T accumulated inside the forward GEMM (one identity projection, rotated
+  // or not, r <= 64, no dropout), so that the separate T pass (and its
+  // split-K reduction) is skipped and X is streamed by the GEMM alone:
   // - one GEMM tile per unit (a single wave, e.g. about a thousand tokens):
   //   every tile accumulates T in the free second accumulator buffer;
   // - at most one row block per unit (up to 256 x 74 tokens): the N-tile-0
@@ -1116,7 +1116,7 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   const int64_t tiles1 = m_tiles1 * ceil_div(d->d_out, 256);
   const int64_t units1 = pair ? dev.sms / 2 : dev.sms;
   const bool t_in_gemm = fused_t_enabled() && r > 0 && RP <= 64 && np == 1 && d->act == LORA_ACT_IDENTITY &&
-                         rope == nullptr && fmasks == nullptr;
+                         fmasks == nullptr;
   const bool share_t = t_in_gemm && tiles1 > units1 && m_tiles1 <= units1 && shared_t_enabled();
   const bool fuse_t = t_in_gemm && (tiles1 <= units1 || share_t);
   // 1. T_j = X A_j^T (fp32, saved for the backward) and bf16(s T_j) for the LoRA K-block
@@ -1157,12 +1157,6 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
   set_raster(p, pair, 2.0 * M * d->d_in, 2.0 * np * d->d_out * d->d_in);
   timing_begin(0, st);
   lora_status_t rs;
-  if (rope != nullptr) {
-    p.rope = *rope;
-    rs = launch_mma_any<false, 1, kMEpiRope>(pair, p, dev.sms, st);
-    timing_end(0, st);
-    return rs;
-  }
   if (fuse_t) {
     p.am_rows = RP / (pair ? 2 : 1);
     p.rp = RP;
@@ -1175,7 +1169,18 @@ static lora_status_t fwd_core(const lora_linear_desc* d, const void* X, const vo
       p.t_flags = status + kTFlagWord0;
     }
     if (!make_tm(&p.tm_am, A, d->d_in, r, d->d_in, 64, p.am_rows)) return LORA_ERR_CUDA;
-    rs = launch_mma_any<false, 1, kMEpiIdentityT>(pair, p, dev.sms, st);
+    if (rope != nullptr) {
+      p.rope = *rope;
+      rs = launch_mma_any<false, 1, kMEpiRopeT>(pair, p, dev.sms, st);
+    } else {
+      rs = launch_mma_any<false, 1, kMEpiIdentityT>(pair, p, dev.sms, st);
+    }
+    timing_end(0, st);
+    return rs;
+  }
+  if (rope != nullptr) {
+    p.rope = *rope;
+    rs = launch_mma_any<false, 1, kMEpiRope>(pair, p, dev.sms, st);
     timing_end(0, st);
     return rs;
   }

@@ -53,14 +53,18 @@ constexpr int kMmaThreads = 320;
 // kMEpiGradF32 / kMEpiGradF16F32: the dX GEMM (bf16 / fp16 operands) writing
 // or adding to an fp32 dX, staged through shared memory so that each global
 // access covers whole sectors of one row.
-// kMEpiGradDrop / kMEpiGradF16Drop: the dX GEMM (bf16 / fp16 operands, no
-// LoRA K-block) of a layer with dropout on the adapter input; the epilogue
-// adds the masked LoRA term m * (s' U A) on the CUDA cores before the one
-// bf16 rounding.
+// kMEpiGradDrop / kMEpiGradF16Drop: the dX GEMM (bf16 / fp16 operands) of a
+// layer with dropout on the adapter input; its LoRA K-blocks go first, the
+// epilogue warps zero the dropped entries of that term in tensor memory, and
+// the main K-blocks accumulate on top before the one bf16 rounding.
+// kMEpiIdentityT / kMEpiRopeT: the forward of one projection (identity, or
+// rotated as kMEpiRope) with T = X A^T accumulated inside the GEMM by the T
+// tiles (MmaParams: tm_am, t_shared).
+// kMEpiCeFwdZ: kMEpiCeFwd that also stores the fp32 logits.
 enum MmaEpi : int {
   kMEpiIdentity = 0, kMEpiSilu = 1, kMEpiSwiglu = 2, kMEpiGrad = 3, kMEpiGradF16 = 4, kMEpiRope = 5,
   kMEpiCeFwd = 6, kMEpiCeGrad = 7, kMEpiGradF32 = 8, kMEpiGradF16F32 = 9, kMEpiGradDrop = 10,
-  kMEpiGradF16Drop = 11, kMEpiIdentityT = 12, kMEpiCeFwdZ = 13
+  kMEpiGradF16Drop = 11, kMEpiIdentityT = 12, kMEpiCeFwdZ = 13, kMEpiRopeT = 14
 };
 
 // Dropout on the adapter input, dX epilogue (kMEpiGradDrop / kMEpiGradF16Drop).
@@ -140,7 +144,7 @@ struct MmaCfg {
   // kMEpiIdentityT: rows of A (the rank, up to 64 in all) per stage and CTA,
   // in a ring of their own after the main stages, which keep the plain
   // kernel's layout
-  static constexpr bool kTFused = kEpi == kMEpiIdentityT;
+  static constexpr bool kTFused = kEpi == kMEpiIdentityT || kEpi == kMEpiRopeT;
   static constexpr int kAMBytes = kTFused ? (64 / kCtas) * 64 * 2 : 0;
   static constexpr int kStageBytes = kABytes + kBBytes;
   // Epilogues that store fp32 Z (SiLU, SwiGLU) stage each warp's rows through
@@ -153,14 +157,15 @@ struct MmaCfg {
   // dX) stage each warp's rows in shared memory as well and write them with
   // TMA stores: per-thread 16-byte stores scattered over 32 rows slowed the
   // loads that feed the tensor core by 1.3-1.8k cycles per tile.
-  static constexpr bool kTmaOut = !(kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiRope || kEpi == kMEpiGradF32 ||
+  static constexpr bool kTmaOut = !(kSwigluFwd || kEpi == kMEpiSilu || kEpi == kMEpiRope || kEpi == kMEpiRopeT ||
+                                    kEpi == kMEpiGradF32 ||
                                     kEpi == kMEpiGradF16F32 || kEpi == kMEpiCeFwd || kEpi == kMEpiCeFwdZ ||
                                     kEpi == kMEpiCeGrad);
   // The fp32 logits of kMEpiCeFwdZ and the fp32 dX of kMEpiGradF32 /
   // kMEpiGradF16F32 (stored, or added at L2 with out_acc) leave the same way.
   static constexpr bool kTmaZ = kEpi == kMEpiCeFwdZ || kEpi == kMEpiGradF32 || kEpi == kMEpiGradF16F32;
   // ... and the rotated bf16 output of kMEpiRope, in 32-column boxes.
-  static constexpr bool kTmaRope = kEpi == kMEpiRope;
+  static constexpr bool kTmaRope = kEpi == kMEpiRope || kEpi == kMEpiRopeT;
   // ... and the SiLU / SwiGLU forward's bf16 Y and fp32 Z.
   static constexpr bool kTmaAct = kSwigluFwd || (kEpi == kMEpiSilu && !kBwd);
   static constexpr int kEpiStageBytes = (kStaged || kTmaOut || kTmaZ || kTmaRope) ? 8 * 4096 : 0;
@@ -829,7 +834,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             flush(mine, &p.tm_out, col0 + 64 * hv);
           }
         }
-      } else if constexpr (kEpi == kMEpiRope) {
+      } else if constexpr (kEpi == kMEpiRope || kEpi == kMEpiRopeT) {
         // Identity plus the rotary embedding.  This thread's 128 columns start
         // at a multiple of 128, so they hold whole heads (half = 64: one head,
         // pairs (c, c + 64); half = 32: two heads, pairs (c, c + 32) in each).
