@@ -10,10 +10,11 @@
 // the angle whose cosine and sine the caller's tables hold for the token's
 // position: (a, b) -> (a c - b s, b c + a s).
 //
-// * rmsnorm_fwd_kernel writes x_n once; the three projections (and their
-//   rank passes) read it.  The sum of squares, rstd and x * rstd * g are
-//   taken in fp64 and rounded to bf16 in one step, so x_n is the correctly
-//   rounded exact norm.
+// * rmsnorm_fwd_kernel writes x_n once; the three projections' forward GEMMs
+//   (which also form T) and the backward's dA passes read it.  The sum of
+//   squares and rstd are taken in fp64, and x * rstd * g is rounded to bf16
+//   from fp32 where that provably gives the same bf16 as the fp64 value (from
+//   fp64 elsewhere), so x_n is the correctly rounded norm.
 // * The rotation of q and k runs in the forward GEMM's epilogue on the fp32
 //   accumulator (rope_rotate32, kMEpiRope in lora_mma.cuh): the pre-rotation
 //   values never leave the chip.
