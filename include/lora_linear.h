@@ -434,6 +434,8 @@ size_t lora_linear_workspace_size_rope(const lora_linear_desc* desc, int for_bac
  * rounding).  desc->act must be LORA_ACT_IDENTITY (LORA_ERR_UNSUPPORTED).
  * X is x_n.  Other arguments as lora_linear_fwd (no SwiGLU twins, no Z_save);
  * T_save holds T = X A^T for the backward.  The few-token kernel is not used.
+ * As with lora_linear_fwd, r <= 64 and M <= 256 x (SMs / 2) make it one GEMM
+ * launch that also computes T; otherwise a T pass runs first.
  * workspace >= lora_linear_workspace_size_rope(desc, 0). */
 lora_status_t lora_linear_fwd_rope(const lora_linear_desc* desc, const lora_rope_desc* rope, const void* X,
                                    const void* W, const void* A, const void* B, void* Y, float* T_save,
