@@ -344,7 +344,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) lora_mma_kernel(const __grid_c
             for (int b = 0; b < C::kBRows / 64; ++b)
               load(sb + b * 8192, &p.tm_w[j], fb, n0 + C::kBRows * static_cast<int>(crank) + 64 * b, k0, pol_keep);
           } else {
-            // W^T (K-major copy of W made by the backward): rows = outputs of dX
+            // a K-major N-side operand (rows = outputs of dX); the library's
+            // backward launches read W in place (b_mn) instead
             load(sb, &p.tm_w[j], fb, k0, n0 + C::kBRows * static_cast<int>(crank), pol_keep);
           }
         }
